@@ -1,0 +1,174 @@
+"""ctypes front of oracle.c (fp64 CPU reference; test infrastructure only).
+
+Inputs are numpy arrays of bf16 bit patterns (uint16), or the 4-bit code (uint8,
+two codes per byte along d_in, low nibble = even index) with bf16 scales per
+64-element block.  Results are fp64 numpy arrays.  Each function is one step of the
+layer's definition (see oracle.c for the formulas and the passages they follow).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c with gcc (IEEE fp64: no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+               "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P, I64, D, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_int
+        lib.oracle_threads.restype = I
+        lib.oracle_set_threads.argtypes = [I]
+        lib.oracle_weight.argtypes = [I, P, P, P, I64, I64, P]
+        lib.oracle_xa.argtypes = [P, P, I64, I64, I64, P]
+        lib.oracle_h.argtypes = [P, I, P, P, P, P, P, D, I64, I64, I64, I64, P, I64, P]
+        lib.oracle_g.argtypes = [P, P, I64, I64, I64, P]
+        lib.oracle_dx.argtypes = [P, I, P, P, P, P, P, D, I64, I64, I64, I64, P, I64, P]
+        lib.oracle_db.argtypes = [P, P, D, I64, I64, I64, P]
+        lib.oracle_da.argtypes = [P, P, D, I64, I64, I64, P]
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a):
+    return np.ascontiguousarray(a, dtype=np.uint16)
+
+
+def threads() -> int:
+    return _load().oracle_threads()
+
+
+def set_threads(n: int) -> None:
+    _load().oracle_set_threads(int(n))
+
+
+def _wargs(W=None, Wq=None, Wscale=None):
+    if W is not None:
+        return 0, _u16(W), None, None
+    return 1, None, np.ascontiguousarray(Wq, dtype=np.uint8), _u16(Wscale)
+
+
+def weight(d_out, d_in, W=None, Wq=None, Wscale=None) -> np.ndarray:
+    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+    out = np.empty((d_out, d_in), dtype=np.float64)
+    _load().oracle_weight(fmt, _p(w), _p(q), _p(sc), d_out, d_in, _p(out))
+    return out
+
+
+def xa(x, A) -> np.ndarray:
+    """Step 1: xa = x . A^T, [M, r]."""
+    x, A = _u16(x), _u16(A)
+    M, d_in = x.shape
+    r = A.shape[0]
+    out = np.empty((M, r), dtype=np.float64)
+    _load().oracle_xa(_p(x), _p(A), M, d_in, r, _p(out))
+    return out
+
+
+def h(x, B, xa_, s, *, W=None, Wq=None, Wscale=None, rows=None) -> np.ndarray:
+    """Step 2: h = x . W^T + s * xa . B^T for all rows, or only ``rows``."""
+    x, B = _u16(x), _u16(B)
+    M, d_in = x.shape
+    d_out, r = B.shape
+    xa_ = np.ascontiguousarray(xa_, dtype=np.float64)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+    rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = M if rr is None else len(rr)
+    out = np.empty((n, d_out), dtype=np.float64)
+    _load().oracle_h(_p(x), fmt, _p(w), _p(q), _p(sc), _p(B), _p(xa_), float(s), M, d_in, d_out, r,
+                     _p(rr), n, _p(out))
+    return out
+
+
+def g(dY, B) -> np.ndarray:
+    """Step 3: g = dY . B, [M, r]."""
+    dY, B = _u16(dY), _u16(B)
+    M, d_out = dY.shape
+    r = B.shape[1]
+    out = np.empty((M, r), dtype=np.float64)
+    _load().oracle_g(_p(dY), _p(B), M, d_out, r, _p(out))
+    return out
+
+
+def dx(dY, A, g_, s, *, W=None, Wq=None, Wscale=None, rows=None) -> np.ndarray:
+    """Step 4: dX = dY . W + s * g . A for all rows, or only ``rows``."""
+    dY, A = _u16(dY), _u16(A)
+    M, d_out = dY.shape
+    r, d_in = A.shape
+    g_ = np.ascontiguousarray(g_, dtype=np.float64)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+    rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = M if rr is None else len(rr)
+    out = np.empty((n, d_in), dtype=np.float64)
+    _load().oracle_dx(_p(dY), fmt, _p(w), _p(q), _p(sc), _p(A), _p(g_), float(s), M, d_in, d_out, r,
+                      _p(rr), n, _p(out))
+    return out
+
+
+def db(dY, xa_, s) -> np.ndarray:
+    """Step 5: dB = s * dY^T . xa, [d_out, r]."""
+    dY = _u16(dY)
+    M, d_out = dY.shape
+    xa_ = np.ascontiguousarray(xa_, dtype=np.float64)
+    r = xa_.shape[1]
+    out = np.empty((d_out, r), dtype=np.float64)
+    _load().oracle_db(_p(dY), _p(xa_), float(s), M, d_out, r, _p(out))
+    return out
+
+
+def da(x, g_, s) -> np.ndarray:
+    """Step 6: dA = s * g^T . x, [r, d_in]."""
+    x = _u16(x)
+    M, d_in = x.shape
+    g_ = np.ascontiguousarray(g_, dtype=np.float64)
+    r = g_.shape[1]
+    out = np.empty((r, d_in), dtype=np.float64)
+    _load().oracle_da(_p(x), _p(g_), float(s), M, d_in, r, _p(out))
+    return out
+
+
+def forward(x, A, B, s, *, W=None, Wq=None, Wscale=None, rows=None):
+    """Steps 1-2.  Returns (h, xa)."""
+    xa_ = xa(x, A)
+    return h(x, B, xa_, s, W=W, Wq=Wq, Wscale=Wscale, rows=rows), xa_
+
+
+def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, rows=None, xa_=None):
+    """Steps 1, 3-6.  Returns dict with dX (all rows or ``rows``), dA, dB, g, xa."""
+    if xa_ is None:
+        xa_ = xa(x, A)
+    g_ = g(dY, B)
+    return {
+        "dX": dx(dY, A, g_, s, W=W, Wq=Wq, Wscale=Wscale, rows=rows),
+        "dA": da(x, g_, s),
+        "dB": db(dY, xa_, s),
+        "g": g_,
+        "xa": xa_,
+    }

@@ -1,0 +1,253 @@
+"""Seeded synthetic inputs for the LoRA linear layer.
+
+This module draws the tensors that both the fp64 oracle and the CUDA path consume.
+It holds none of the layer's arithmetic: it only produces random numbers, rounds them
+to the storage formats (bf16, or the 4-bit blockwise code for a frozen weight) and
+describes the five workloads.
+
+Random numbers come from a counter-based generator so that a tensor's values do not
+depend on the shapes of the other tensors, and so any element can be regenerated
+from (seed, tensor id, flat index):
+
+* 64-bit words: the splitmix64 output function (Steele, Lea and Flood, "Fast
+  splittable pseudorandom number generators", OOPSLA 2014), applied to
+  ``key + (index + 1) * 0x9E3779B97F4A7C15`` where ``key`` mixes the seed with the
+  tensor id.
+* uniforms in (0, 1): the top 53 bits of a word, offset by half an ulp so 0 never
+  occurs.
+* normals: the Box-Muller transform (cosine branch) of the uniforms at counters
+  2*i and 2*i + 1.
+
+Values are drawn in fp64, rounded to fp32, then to bf16 with round-to-nearest-even.
+The arrays handed out are raw bf16 bit patterns (``uint16``) so both sides read
+exactly the same bits.
+
+Value distributions per tensor (the workloads' own recipe):
+x, dY ~ N(0, 1); W ~ N(0, 1/d_in); A ~ U(-1/sqrt(d_in), +1/sqrt(d_in)); B ~ N(0, 0.02^2).
+"""
+from __future__ import annotations
+
+import math
+import os
+from concurrent.futures import ThreadPoolExecutor
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_GOLDEN = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+_TWO_NEG53 = 2.0 ** -53
+_CHUNK = 1 << 22
+
+# Tensor ids of the counter-based streams.  A multi-layer workload offsets them by
+# 16 * layer so every layer has its own streams.
+TID_X, TID_W, TID_A, TID_B, TID_DY = 1, 2, 3, 4, 5
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    """splitmix64 output function on a uint64 array (wrapping arithmetic)."""
+    z = (z ^ (z >> np.uint64(30))) * _M1
+    z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def stream_key(seed: int, tensor_id: int) -> np.uint64:
+    with np.errstate(over="ignore"):
+        t = _mix(np.array([tensor_id], dtype=np.uint64) + _GOLDEN)
+        k = _mix(np.array([seed], dtype=np.uint64) ^ t)
+    return k[0]
+
+
+def _words(key: np.uint64, idx: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        return _mix(key + (idx + np.uint64(1)) * _GOLDEN)
+
+
+def _uniform01(key: np.uint64, idx: np.ndarray) -> np.ndarray:
+    w = _words(key, idx)
+    return ((w >> np.uint64(11)).astype(np.float64) + 0.5) * _TWO_NEG53
+
+
+def _draw_chunk(kind: str, key: np.uint64, lo: int, hi: int, p0: float) -> np.ndarray:
+    i = np.arange(lo, hi, dtype=np.uint64)
+    if kind == "normal":
+        u1 = _uniform01(key, i * np.uint64(2))
+        u2 = _uniform01(key, i * np.uint64(2) + np.uint64(1))
+        return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2) * p0
+    if kind == "uniform":
+        u = _uniform01(key, i)
+        return (2.0 * u - 1.0) * p0
+    raise ValueError(kind)
+
+
+def draw(kind: str, seed: int, tensor_id: int, n: int, p0: float) -> np.ndarray:
+    """n fp64 draws: ``normal`` with std p0, or ``uniform`` on (-p0, p0)."""
+    key = stream_key(seed, tensor_id)
+    if n <= _CHUNK:
+        return _draw_chunk(kind, key, 0, n, p0)
+    out = np.empty(n, dtype=np.float64)
+    bounds = [(lo, min(n, lo + _CHUNK)) for lo in range(0, n, _CHUNK)]
+
+    def work(b):
+        out[b[0]:b[1]] = _draw_chunk(kind, key, b[0], b[1], p0)
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, bounds))
+    return out
+
+
+def f32_to_bf16_bits(a32: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (nearest, ties to even); returns uint16 bit patterns."""
+    u = np.ascontiguousarray(a32, dtype=np.float32).view(np.uint32)
+    bias = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return ((u + bias) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def to_bf16_bits(a64: np.ndarray) -> np.ndarray:
+    return f32_to_bf16_bits(a64.astype(np.float32))
+
+
+Q4_BLOCK = 64
+
+
+def quantise_q4(w32: np.ndarray):
+    """4-bit blockwise code of a frozen weight [d_out, d_in] (fp32 draws).
+
+    Per block of 64 consecutive d_in elements: absmax = max |w| (fp32);
+    q = clamp(round_half_away(7 * w / absmax) + 8, 1, 15) (a block with absmax 0
+    gets q = 8); the stored scale is bf16(absmax) (nearest-even).  Two codes per
+    byte along d_in: the low nibble holds the even index.  Returns (packed uint8
+    [d_out, d_in/2], scale bf16 bits [d_out, d_in/64]).
+    """
+    d_out, d_in = w32.shape
+    assert d_in % Q4_BLOCK == 0
+    out_q = np.empty((d_out, d_in // 2), dtype=np.uint8)
+    out_s = np.empty((d_out, d_in // Q4_BLOCK), dtype=np.uint16)
+    rows = max(1, (1 << 22) // d_in)
+
+    def work(r0):
+        r1 = min(d_out, r0 + rows)
+        wb = w32[r0:r1].reshape(r1 - r0, d_in // Q4_BLOCK, Q4_BLOCK)
+        amax = np.abs(wb).max(axis=2).astype(np.float32)
+        safe = np.where(amax > 0, amax, np.float32(1)).astype(np.float64)
+        t = 7.0 * wb.astype(np.float64) / safe[:, :, None]
+        q = np.sign(t) * np.floor(np.abs(t) + 0.5) + 8.0
+        q = np.clip(q, 1, 15)
+        q = np.where(amax[:, :, None] > 0, q, 8.0).astype(np.uint8).reshape(r1 - r0, d_in)
+        out_q[r0:r1] = (q[:, 0::2] & 0x0F) | (q[:, 1::2] << 4)
+        out_s[r0:r1] = f32_to_bf16_bits(amax)
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, range(0, d_out, rows)))
+    return out_q, out_s
+
+
+def unpack_q4_codes(packed: np.ndarray) -> np.ndarray:
+    """Inverse of the nibble packing only (codes 0..15, no scaling)."""
+    d_out, half = packed.shape
+    q = np.empty((d_out, half * 2), dtype=np.uint8)
+    q[:, 0::2] = packed & 0x0F
+    q[:, 1::2] = packed >> 4
+    return q
+
+
+@dataclass
+class LayerSpec:
+    """One LoRA linear: M tokens, d_in -> d_out, rank r, scale alpha/r."""
+    name: str
+    M: int
+    d_in: int
+    d_out: int
+    r: int
+    alpha: float
+    q4: bool = False
+    seed: int = 0
+    layer: int = 0
+
+    @property
+    def s(self) -> float:
+        return self.alpha / self.r
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic fwd+bwd FLOPs: 4*M*d_in*d_out + 6*M*r*(d_in+d_out)."""
+        return 4.0 * self.M * self.d_in * self.d_out + 6.0 * self.M * self.r * (self.d_in + self.d_out)
+
+    def with_(self, **kw) -> "LayerSpec":
+        d = dict(self.__dict__)
+        d.update(kw)
+        return LayerSpec(**d)
+
+
+@dataclass
+class Workload:
+    name: str
+    layers: list = field(default_factory=list)
+
+
+def workload(idx: int, r: int | None = None) -> Workload:
+    """The five workloads (seed 0x5EED0000 + index).
+
+    0: tiny, M=64, 256->256, r=8, alpha=16.
+    1: attention projection, M=4096 (2 x 2048), 4096->4096, r=8, alpha=32.
+    2: one 7B MLP set, M=8192: gate 4096->11008, up 4096->11008, down 11008->4096, r=16, alpha=32.
+    3: rank sweep, M=16384 (2 x 8192), 4096->4096, r in {8,16,64,128}, alpha=16.
+    4: 4-bit frozen W, up projection 8192->28672, r=16, alpha=32, M=4096.
+    """
+    seed = 0x5EED0000 + idx
+    if idx == 0:
+        return Workload("tiny M64 256x256 r8", [LayerSpec("tiny", 64, 256, 256, 8, 16.0, seed=seed)])
+    if idx == 1:
+        return Workload("attn-proj M4096 4096x4096 r8",
+                        [LayerSpec("q_proj", 4096, 4096, 4096, 8, 32.0, seed=seed)])
+    if idx == 2:
+        return Workload("mlp-set M8192 4096<->11008 r16", [
+            LayerSpec("gate_proj", 8192, 4096, 11008, 16, 32.0, seed=seed, layer=0),
+            LayerSpec("up_proj", 8192, 4096, 11008, 16, 32.0, seed=seed, layer=1),
+            LayerSpec("down_proj", 8192, 11008, 4096, 16, 32.0, seed=seed, layer=2),
+        ])
+    if idx == 3:
+        rr = 8 if r is None else r
+        return Workload(f"rank-sweep M16384 4096x4096 r{rr}",
+                        [LayerSpec(f"proj_r{rr}", 16384, 4096, 4096, rr, 16.0, seed=seed)])
+    if idx == 4:
+        return Workload("q4 up-proj M4096 8192->28672 r16",
+                        [LayerSpec("up_proj_q4", 4096, 8192, 28672, 16, 32.0, q4=True, seed=seed)])
+    raise ValueError(idx)
+
+
+@dataclass
+class LayerInputs:
+    spec: LayerSpec
+    x: np.ndarray            # bf16 bits [M, d_in]
+    A: np.ndarray            # bf16 bits [r, d_in]
+    B: np.ndarray            # bf16 bits [d_out, r]
+    dY: np.ndarray           # bf16 bits [M, d_out]
+    W: np.ndarray | None     # bf16 bits [d_out, d_in] (None for q4)
+    Wq: np.ndarray | None    # uint8 [d_out, d_in/2] (q4 only)
+    Wscale: np.ndarray | None  # bf16 bits [d_out, d_in/64] (q4 only)
+
+
+def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) -> LayerInputs:
+    """Draw every input of one layer from its seeded streams."""
+    seed, off = spec.seed, 16 * spec.layer
+    M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
+    x = to_bf16_bits(draw("normal", seed, TID_X + off, M * di, 1.0)).reshape(M, di)
+    dY = to_bf16_bits(draw("normal", seed, TID_DY + off, M * do, 1.0)).reshape(M, do)
+    bound = 1.0 / math.sqrt(di)
+    A = to_bf16_bits(draw("uniform", seed, TID_A + off, r * di, bound)).reshape(r, di)
+    B = to_bf16_bits(draw("normal", seed, TID_B + off, do * r, 0.02)).reshape(do, r)
+    if zero_A:
+        A = np.zeros_like(A)
+    if zero_B:
+        B = np.zeros_like(B)
+    w32 = draw("normal", seed, TID_W + off, do * di, 1.0 / math.sqrt(di)).astype(np.float32).reshape(do, di)
+    if spec.q4:
+        Wq, Ws = quantise_q4(w32)
+        return LayerInputs(spec, x, A, B, dY, None, Wq, Ws)
+    return LayerInputs(spec, x, A, B, dY, f32_to_bf16_bits(w32), None, None)

@@ -1,0 +1,54 @@
+"""The seeded input generator: published test values, determinism, distributions."""
+import math
+
+import numpy as np
+
+from rank_linear_lora_b200 import inputs
+
+
+def test_splitmix64_published_sequence():
+    """splitmix64 from state 0: the first three outputs of the published generator."""
+    words = inputs._words(np.uint64(0), np.arange(3, dtype=np.uint64))
+    assert [int(w) for w in words] == [0xE220A8397B1DCDAF, 0x6E789E6AA1B965F4, 0x06C45D188009454F]
+
+
+def test_bf16_round_to_nearest_even():
+    vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 3.0e-3, 1.0 + 2.0 ** -8 + 2.0 ** -20],
+                    dtype=np.float32)
+    bits = inputs.f32_to_bf16_bits(vals)
+    # 1+2^-8 is a tie -> even (1.0); 1+3*2^-8 is a tie -> even (1+2^-6); just above a tie rounds up
+    assert list(bits[:4]) == [0x3F80, 0x3F80, 0x3F82, 0xC020]
+    assert bits[5] == 0x3F81
+    back = inputs.bf16_bits_to_f32(bits[4:5])[0]
+    assert abs(back - 3.0e-3) <= 3.0e-3 * 2.0 ** -8
+
+
+def test_streams_are_deterministic_and_shape_independent():
+    a = inputs.LayerSpec("t", 16, 64, 32, 8, 16.0, seed=123)
+    b = a.with_(d_out=48)
+    ia, ib = inputs.make_inputs(a), inputs.make_inputs(b)
+    np.testing.assert_array_equal(ia.x, ib.x)
+    np.testing.assert_array_equal(ia.A, ib.A)
+    ia2 = inputs.make_inputs(a)
+    for k in ("x", "W", "A", "B", "dY"):
+        np.testing.assert_array_equal(getattr(ia, k), getattr(ia2, k))
+    assert not np.array_equal(ia.x[:, :32], ia.dY)
+
+
+def test_chunked_draws_match_single_pass():
+    n = inputs._CHUNK + 12345
+    big = inputs.draw("normal", 7, 1, n, 1.0)
+    head = inputs._draw_chunk("normal", inputs.stream_key(7, 1), 0, 1000, 1.0)
+    tail = inputs._draw_chunk("normal", inputs.stream_key(7, 1), n - 1000, n, 1.0)
+    np.testing.assert_array_equal(big[:1000], head)
+    np.testing.assert_array_equal(big[-1000:], tail)
+
+
+def test_distributions():
+    n = 1 << 20
+    z = inputs.draw("normal", 99, 1, n, 0.02)
+    assert abs(z.mean()) < 4 * 0.02 / math.sqrt(n) * 1.5
+    assert abs(z.std() / 0.02 - 1.0) < 5e-3
+    u = inputs.draw("uniform", 99, 2, n, 0.25)
+    assert u.min() > -0.25 and u.max() < 0.25
+    assert abs(u.std() - 0.25 / math.sqrt(3)) < 1e-3

@@ -1,0 +1,247 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test ties one or more of the oracle's six steps to a hand-worked value, a
+closed form, an invariance of the layer, brute force in pure Python, finite
+differences of the forward, or a library matmul on a case the definition reduces to.
+A dropped term, a wrong sign, a transposed operand or a swapped gradient fails at
+least one of them.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from rank_linear_lora_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf(a):
+    """Exact bf16 bit patterns of small dyadic values (asserts exact representability)."""
+    a = np.asarray(a, dtype=np.float64)
+    bits = inputs.to_bf16_bits(a)
+    assert np.array_equal(inputs.bf16_bits_to_f32(bits).astype(np.float64), a), "not bf16-exact"
+    return bits
+
+
+def f64(bits):
+    return inputs.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def run_all(x, W, A, B, dY, alpha):
+    r = A.shape[0]
+    s = alpha / r
+    h, xa = oracle.forward(x, A, B, s, W=W)
+    bw = oracle.backward(dY, x, A, B, s, W=W)
+    return dict(h=h, xa=xa, **{k: bw[k] for k in ("dX", "dA", "dB", "g")})
+
+
+@pytest.mark.parametrize("name", ["rank1_hand.json", "rank2_hand.json"])
+def test_hand_worked_cases(name):
+    c = json.load(open(os.path.join(GOLDEN, name)))
+    out = run_all(bf(c["x"]), bf(c["W"]), bf(c["A"]), bf(c["B"]), bf(c["dY"]), c["alpha"])
+    for key in ("xa", "g", "h", "dX", "dA", "dB"):
+        np.testing.assert_array_equal(out[key], np.array(c[key], dtype=np.float64), err_msg=key)
+    assert float((f64(bf(c["dY"])) * out["h"]).sum()) == c["L"]
+
+
+def _rand_bits(rng, shape, scale=1.0):
+    return inputs.to_bf16_bits(rng.standard_normal(shape) * scale)
+
+
+def _py_xwT(x, W):
+    """Brute force x.W^T in pure Python, summing k in increasing order."""
+    M, d_in = x.shape
+    d_out = W.shape[0]
+    out = np.zeros((M, d_out))
+    for m in range(M):
+        for n in range(d_out):
+            acc = 0.0
+            for k in range(d_in):
+                acc += float(x[m, k]) * float(W[n, k])
+            out[m, n] = acc
+    return out
+
+
+def _py_dyW(dY, W):
+    """Brute force dY.W in pure Python, summing n in increasing order."""
+    M, d_out = dY.shape
+    d_in = W.shape[1]
+    out = np.zeros((M, d_in))
+    for m in range(M):
+        for k in range(d_in):
+            acc = 0.0
+            for n in range(d_out):
+                acc += float(dY[m, n]) * float(W[n, k])
+            out[m, k] = acc
+    return out
+
+
+def test_zero_B_is_the_frozen_linear():
+    """Delta W = 0: h = x.W^T and dX = dY.W exactly, dA = 0 exactly, dB stays nonzero."""
+    rng = np.random.default_rng(1)
+    M, d_in, d_out, r = 5, 7, 6, 3
+    x, W, A, dY = (_rand_bits(rng, s) for s in [(M, d_in), (d_out, d_in), (r, d_in), (M, d_out)])
+    B = np.zeros((d_out, r), dtype=np.uint16)
+    out = run_all(x, W, A, B, dY, alpha=6.0)
+    np.testing.assert_array_equal(out["h"], _py_xwT(f64(x), f64(W)))
+    np.testing.assert_array_equal(out["dX"], _py_dyW(f64(dY), f64(W)))
+    assert np.all(out["g"] == 0) and np.all(out["dA"] == 0)
+    assert np.abs(out["dB"]).max() > 0
+
+
+def test_zero_A_is_the_frozen_linear():
+    """A = 0: xa = 0, so h = x.W^T, dB = 0 exactly and dX = dY.W exactly; dA stays nonzero."""
+    rng = np.random.default_rng(2)
+    M, d_in, d_out, r = 4, 6, 5, 2
+    x, W, B, dY = (_rand_bits(rng, s) for s in [(M, d_in), (d_out, d_in), (d_out, r), (M, d_out)])
+    A = np.zeros((r, d_in), dtype=np.uint16)
+    out = run_all(x, W, A, B, dY, alpha=4.0)
+    assert np.all(out["xa"] == 0) and np.all(out["dB"] == 0)
+    np.testing.assert_array_equal(out["h"], _py_xwT(f64(x), f64(W)))
+    np.testing.assert_array_equal(out["dX"], _py_dyW(f64(dY), f64(W)))
+    assert np.abs(out["dA"]).max() > 0
+
+
+@pytest.mark.parametrize("shape", [(64, 256, 256, 8), (37, 48, 80, 16), (9, 120, 24, 1)])
+def test_merged_weight_identity(shape):
+    """x.(W + s.B.A)^T = h and dY.(W + s.B.A) = dX with the d_out x d_in update formed
+    explicitly: the merged weight of deployment, and (B.A)^T.dY = A^T.(B^T.dY), the
+    reassociation the backward relies on."""
+    M, d_in, d_out, r = shape
+    rng = np.random.default_rng(3)
+    x, W, A, B, dY = (_rand_bits(rng, s, sc) for s, sc in
+                      [((M, d_in), 1), ((d_out, d_in), d_in ** -0.5), ((r, d_in), d_in ** -0.5),
+                       ((d_out, r), 0.5), ((M, d_out), 1)])
+    alpha = 2.0 * r
+    s = alpha / r
+    out = run_all(x, W, A, B, dY, alpha)
+    merged = f64(W) + s * (f64(B) @ f64(A))
+    h_ref = f64(x) @ merged.T
+    dx_ref = f64(dY) @ merged
+    np.testing.assert_allclose(out["h"], h_ref, rtol=0, atol=1e-12 * np.abs(h_ref).max())
+    np.testing.assert_allclose(out["dX"], dx_ref, rtol=0, atol=1e-12 * np.abs(dx_ref).max())
+
+
+@pytest.mark.parametrize("shape", [(64, 256, 256, 8), (23, 72, 40, 16)])
+def test_matches_library_matmul(shape):
+    """Every output against numpy fp64 matmuls of the same definition."""
+    M, d_in, d_out, r = shape
+    rng = np.random.default_rng(4)
+    x, W, A, B, dY = (_rand_bits(rng, s, sc) for s, sc in
+                      [((M, d_in), 1), ((d_out, d_in), d_in ** -0.5), ((r, d_in), d_in ** -0.5),
+                       ((d_out, r), 0.02), ((M, d_out), 1)])
+    alpha = 16.0
+    s = alpha / r
+    out = run_all(x, W, A, B, dY, alpha)
+    X, Wd, Ad, Bd, dYd = map(f64, (x, W, A, B, dY))
+    ref = {
+        "xa": X @ Ad.T,
+        "h": X @ Wd.T + s * (X @ Ad.T) @ Bd.T,
+        "g": dYd @ Bd,
+        "dX": dYd @ Wd + s * (dYd @ Bd) @ Ad,
+        "dB": s * dYd.T @ (X @ Ad.T),
+        "dA": s * (dYd @ Bd).T @ X,
+    }
+    for key, want in ref.items():
+        np.testing.assert_allclose(out[key], want, rtol=0, atol=1e-12 * np.abs(want).max(), err_msg=key)
+
+
+def _dyadic(rng, shape):
+    """Multiples of 1/8 in [-2, 2]: with eps = 1/16 every perturbed value stays bf16-exact."""
+    return rng.integers(-16, 17, size=shape).astype(np.float64) / 8.0
+
+
+@pytest.mark.parametrize("r", [1, 2])
+def test_central_differences(r):
+    """dX, dA, dB are the derivatives of L = sum(dY * h).  L is affine in every single
+    entry of x, A and B, so the central difference is exact up to rounding."""
+    M, d_in, d_out = 3, 5, 4
+    rng = np.random.default_rng(10 + r)
+    vals = {k: _dyadic(rng, s) for k, s in
+            [("x", (M, d_in)), ("W", (d_out, d_in)), ("A", (r, d_in)), ("B", (d_out, r)), ("dY", (M, d_out))]}
+    alpha = 2.0 * r
+    s = alpha / r
+    eps = 1.0 / 16.0
+
+    def loss(v):
+        h, _ = oracle.forward(bf(v["x"]), bf(v["A"]), bf(v["B"]), s, W=bf(v["W"]))
+        return float((v["dY"] * h).sum())
+
+    grads = oracle.backward(bf(vals["dY"]), bf(vals["x"]), bf(vals["A"]), bf(vals["B"]), s, W=bf(vals["W"]))
+    for name, gname in (("x", "dX"), ("A", "dA"), ("B", "dB")):
+        fd = np.zeros_like(vals[name])
+        for idx in np.ndindex(vals[name].shape):
+            vp = {k: v.copy() for k, v in vals.items()}
+            vm = {k: v.copy() for k, v in vals.items()}
+            vp[name][idx] += eps
+            vm[name][idx] -= eps
+            fd[idx] = (loss(vp) - loss(vm)) / (2 * eps)
+        scale = max(1.0, np.abs(fd).max())
+        np.testing.assert_allclose(grads[gname], fd, rtol=0, atol=1e-10 * scale, err_msg=gname)
+
+
+def test_rescaling_and_alpha():
+    """(A*c, B/c) leaves h and dX unchanged (c a power of two: exact); doubling alpha
+    doubles the low-rank term of h."""
+    rng = np.random.default_rng(5)
+    M, d_in, d_out, r = 6, 16, 12, 4
+    x, W, A, B, dY = (_rand_bits(rng, s, 0.5) for s in
+                      [(M, d_in), (d_out, d_in), (r, d_in), (d_out, r), (M, d_out)])
+    base = run_all(x, W, A, B, dY, 8.0)
+    resc = run_all(x, W, bf(f64(A) * 2.0), bf(f64(B) / 2.0), dY, 8.0)
+    np.testing.assert_array_equal(base["h"], resc["h"])
+    np.testing.assert_array_equal(base["dX"], resc["dX"])
+    h0 = run_all(x, W, A, np.zeros_like(B), dY, 8.0)["h"]
+    h2 = run_all(x, W, A, B, dY, 16.0)["h"]
+    np.testing.assert_allclose(h2 - h0, 2.0 * (base["h"] - h0), rtol=0, atol=1e-12 * np.abs(h2).max())
+
+
+def test_q4_code_pins():
+    """The 4-bit code of a block [a, -a, 0, a/2, ...] is [15, 1, 8, 12, ...] and
+    decodes to [a, -a, 0, 4a/7, ...]; low nibble = even index; a zero block codes 8."""
+    a = 0.75  # bf16-exact, so the stored scale is exactly a
+    w = np.zeros((2, 128), dtype=np.float32)
+    w[0, :4] = [a, -a, 0.0, a / 2]
+    w[0, 4:64] = np.linspace(-a / 2, a / 2, 60, dtype=np.float32)
+    q, sc = inputs.quantise_q4(w)
+    codes = inputs.unpack_q4_codes(q)
+    assert list(codes[0, :4]) == [15, 1, 8, 12]
+    assert q[0, 0] == (15 | (1 << 4)) and q[0, 1] == (8 | (12 << 4))
+    assert np.all(codes[1] == 8) and np.all(codes[0, 64:] == 8)
+    assert inputs.bf16_bits_to_f32(sc)[0, 0] == np.float32(a)
+    assert np.all(sc[1] == 0)
+    wd = oracle.weight(2, 128, Wq=q, Wscale=sc)
+    np.testing.assert_array_equal(wd[0, :4], [a, -a, 0.0, 4 * a / 7])
+    assert np.all(wd[1] == 0) and np.all(wd[0, 64:] == 0)
+
+
+def test_q4_forward_reads_dequantised_columns():
+    """With B = 0 and x = e_k, row h[k] of the q4 oracle is column k of the decoded weight
+    (q - 8) * scale / 7 computed here from the codes and scales by hand."""
+    d_in, d_out, r = 128, 3, 2
+    rng = np.random.default_rng(6)
+    q = rng.integers(0, 256, size=(d_out, d_in // 2), dtype=np.uint8)
+    sc = inputs.to_bf16_bits(rng.uniform(0.1, 1.0, size=(d_out, d_in // 64)))
+    x = inputs.to_bf16_bits(np.eye(d_in))
+    A = np.zeros((r, d_in), dtype=np.uint16)
+    B = np.zeros((d_out, r), dtype=np.uint16)
+    h, _ = oracle.forward(x, A, B, 1.0, Wq=q, Wscale=sc)
+    codes = inputs.unpack_q4_codes(q).astype(np.float64)
+    scale = np.repeat(inputs.bf16_bits_to_f32(sc).astype(np.float64), 64, axis=1)
+    np.testing.assert_array_equal(h.T, (codes - 8.0) * scale / 7.0)
+
+
+def test_row_selection_matches_full():
+    """The sampled-row mode used at full sizes returns exactly the full rows."""
+    rng = np.random.default_rng(7)
+    M, d_in, d_out, r = 20, 24, 16, 8
+    x, W, A, B, dY = (_rand_bits(rng, s) for s in [(M, d_in), (d_out, d_in), (r, d_in), (d_out, r), (M, d_out)])
+    rows = np.array([19, 0, 7])
+    full = run_all(x, W, A, B, dY, 16.0)
+    hs, _ = oracle.forward(x, A, B, 2.0, W=W, rows=rows)
+    dxs = oracle.backward(dY, x, A, B, 2.0, W=W, rows=rows)["dX"]
+    np.testing.assert_array_equal(hs, full["h"][rows])
+    np.testing.assert_array_equal(dxs, full["dX"][rows])
