@@ -1,0 +1,172 @@
+/*
+ * lora_linear.h -- C ABI of the fused LoRA linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (row-major, tokens are rows):
+ *   forward   h  = x.W^T + s.(x.A^T).B^T                     s = alpha / r
+ *   backward  dX = dY.W + s.(dY.B).A
+ *             dB = s.dY^T.(x.A^T)          dA = s.(dY.B)^T.x
+ * with a frozen weight W (no dW).  The forward is the low-rank update of a frozen
+ * weight, h = W x + B (A x), of page "UnSloth加速库集成：编译级优化带来的性能飞跃",
+ * section 为什么标准LoRA会慢？, written for row vectors with the scale s on the update.
+ * The backward is its chain rule; page "ms-swift高效微调组合：LoRA+UnSloth提速实践",
+ * section 1.2 (梯度计算绕过Autograd) prints the two weight gradients in a shortened
+ * form, and page "Unsloth — 微调 2-5x 加速", section 核心要点 (数学化简反向公式) fixes
+ * the association A.(B.dY) that never forms the d_out x d_in update.
+ *
+ * Shapes and layouts (all row-major, contiguous, element strides = the last dim):
+ *   x [M, d_in]   W [d_out, d_in] (torch.nn.Linear.weight)   A [r, d_in] (lora_A)
+ *   B [d_out, r] (lora_B)   h, dY [M, d_out]   dX [M, d_in]   dA [r, d_in]   dB [d_out, r]
+ *   xa_save [M, r] holds bf16(s . x.A^T), written by the forward, read by the backward.
+ * Element types: "bf16" arguments are bfloat16 values passed as their 16-bit patterns
+ * (uint16_t); dA and dB are fp32.  The 4-bit weight of the *_q4 entry points is
+ * Wq [d_out, d_in/2] (uint8, two codes per byte along d_in, low nibble = even index)
+ * with Wscale [d_out, d_in/64] (bf16): w'[n,k] = (q[n,k] - 8) * Wscale[n, k/64] / 7.
+ *
+ * Conventions shared by every entry point:
+ *   - Pointers are device pointers (cudaMalloc or equivalent) on the current device.
+ *     The caller owns every buffer, including the workspace.  The library never
+ *     allocates, frees or synchronises the stream; all work is enqueued on `stream`
+ *     (a cudaStream_t passed as void*; NULL = the legacy default stream) and the
+ *     call returns without waiting.
+ *   - Outputs are overwritten, never accumulated into.  Inputs and outputs must not
+ *     alias.  Calls on distinct streams with distinct workspaces may run concurrently.
+ *   - Validation happens before any launch; on an error status nothing is enqueued.
+ *     Required: non-null required pointers; every pointer 16-byte aligned; M >= 1;
+ *     d_in and d_out multiples of 8 (>= 8); 1 <= r <= 256 with r % 8 == 0; alpha
+ *     finite; for *_q4 also d_in % 64 == 0.
+ *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
+ *     aligned, and must not be used by two calls that may run at the same time.
+ *   - The device must be compute capability 10.0 (B200); otherwise
+ *     LORA_ERR_UNSUPPORTED is returned and nothing runs.
+ *   - Device-side waits are bounded.  A wait that runs out sets an error word in the
+ *     workspace and the kernels return early; lora_linear_check() reports it.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef LORA_LINEAR_H
+#define LORA_LINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LORA_API __attribute__((visibility("default")))
+#else
+#define LORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LORA_OK = 0,
+    LORA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, r or alpha out of range */
+    LORA_ERR_MISALIGNED = 2,   /* a pointer is not 16-byte (workspace: 256-byte) aligned */
+    LORA_ERR_UNSUPPORTED = 3,  /* no sm_100 device, or a shape this build does not cover */
+    LORA_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+    LORA_ERR_CUDA = 5,         /* a CUDA runtime/driver call failed (launch, tensor map) */
+    LORA_ERR_TIMEOUT = 6       /* a device-side bounded wait ran out (see lora_linear_check) */
+} lora_status_t;
+
+typedef enum {
+    LORA_OP_FWD = 0,
+    LORA_OP_BWD = 1,
+    LORA_OP_FWD_Q4 = 2,
+    LORA_OP_BWD_Q4 = 3
+} lora_op_t;
+
+/* Bytes of workspace the given operation needs for these sizes (0 if the sizes are
+ * invalid).  Pure host function; needs no device. */
+LORA_API size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r);
+
+/*
+ * Forward: h = x.W^T + s.(x.A^T).B^T, s = alpha / r
+ * (page "UnSloth加速库集成：编译级优化带来的性能飞跃", section 为什么标准LoRA会慢？, and
+ * the single fused Linear -> LoRA_A -> LoRA_B -> Add pass of page
+ * "ms-swift高效微调组合：LoRA+UnSloth提速实践", section 1.2, 算子融合).
+ *   x, W, A, B : inputs (bf16).            h : output [M, d_out] (bf16).
+ *   xa_save    : optional output [M, r] (bf16) = bf16(s . x.A^T); pass it to
+ *                lora_linear_bwd to skip recomputing x.A^T.  May be NULL.
+ *   workspace  : scratch of lora_linear_workspace_size(LORA_OP_FWD, ...) bytes.
+ */
+LORA_API lora_status_t lora_linear_fwd(const uint16_t *x, const uint16_t *W, const uint16_t *A,
+                              const uint16_t *B, uint16_t *h, uint16_t *xa_save,
+                              int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Backward: dX = dY.W + s.(dY.B).A, dB = s.dY^T.(x.A^T), dA = s.(dY.B)^T.x
+ * (chain rule of the forward above; the gradient pair of page
+ * "ms-swift高效微调组合：LoRA+UnSloth提速实践", section 1.2, 梯度计算绕过Autograd, in
+ * complete form; association A.(B.dY) from page "Unsloth — 微调 2-5x 加速", section
+ * 核心要点).  W is frozen: no dW.
+ *   dY, x, W, A, B : inputs (bf16).
+ *   xa_save        : bf16(s . x.A^T) from lora_linear_fwd, or NULL to recompute it.
+ *   dX             : output [M, d_in] (bf16), or NULL to skip the input gradient.
+ *   dA, dB         : outputs (fp32), overwritten.
+ */
+LORA_API lora_status_t lora_linear_bwd(const uint16_t *dY, const uint16_t *x, const uint16_t *W,
+                              const uint16_t *A, const uint16_t *B, const uint16_t *xa_save,
+                              uint16_t *dX, float *dA, float *dB,
+                              int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Forward with a 4-bit frozen weight, dequantised in shared memory inside the GEMM
+ * and never written back as bf16 (page "Unsloth — 微调 2-5x 加速", section 核心要点:
+ * 4-bit dequantisation fused into the matmul; page
+ * "ms-swift框架下UnSloth与Liger-Kernel优化实战", section UnSloth：让LoRA真正“低秩”起来:
+ * int4 storage restored on the fly).  As lora_linear_fwd with W replaced by
+ * (Wq, Wscale); d_in % 64 == 0.
+ */
+LORA_API lora_status_t lora_linear_fwd_q4(const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale,
+                                 const uint16_t *A, const uint16_t *B, uint16_t *h,
+                                 uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out,
+                                 int r, float alpha, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+/* Backward with the 4-bit frozen weight (same passages); as lora_linear_bwd with W
+ * replaced by (Wq, Wscale). */
+LORA_API lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x, const uint8_t *Wq,
+                                 const uint16_t *Wscale, const uint16_t *A, const uint16_t *B,
+                                 const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
+                                 int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* Waits for `stream`, then reads and clears the device error word kept in
+ * `workspace`.  Returns LORA_OK, LORA_ERR_TIMEOUT (a bounded device wait ran out) or
+ * LORA_ERR_CUDA (the stream reported an error).  Synchronising: for tests and
+ * diagnostics, not for the hot path. */
+LORA_API lora_status_t lora_linear_check(void *workspace, void *stream);
+
+/* Static description of a status code; never NULL. */
+LORA_API const char *lora_status_string(lora_status_t status);
+
+/* ---- measurement hooks (no effect on results) ---------------------------------
+ * Kernel kinds, in the order a forward + backward launches them. */
+typedef enum {
+    LORA_K_XA = 0,       /* forward prologue: bf16(s . x.A^T), split over d_in      */
+    LORA_K_FWD_MAIN = 1, /* forward main GEMM: [x | s.xa].[W | B]^T                 */
+    LORA_K_G = 2,        /* backward prologue: bf16(s . dY.B), split over d_out     */
+    LORA_K_DX_MAIN = 3,  /* backward main GEMM: [dY | s.g].[W ; A]                  */
+    LORA_K_DB = 4,       /* dB = dY^T.(s.xa), split over tokens                     */
+    LORA_K_DA = 5,       /* dA = (s.g)^T.x, split over tokens                       */
+    LORA_K_COUNT = 6
+} lora_kernel_kind_t;
+
+/* Total kernels this library has launched since it was loaded. */
+LORA_API int64_t lora_linear_launch_count(void);
+
+/* When enabled, every launch is bracketed by CUDA events recorded on its stream.
+ * lora_linear_timing_read() waits for the recorded events and returns, per kernel
+ * kind, the summed device time in ms and the number of launches, then clears the
+ * record.  Returns LORA_OK, or LORA_ERR_CUDA if an event failed. */
+LORA_API lora_status_t lora_linear_timing_enable(int enable);
+LORA_API lora_status_t lora_linear_timing_read(double *ms_per_kind, int64_t *launches_per_kind,
+                                      int kinds);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_LINEAR_H */

@@ -1,0 +1,569 @@
+// lora_linear.cu -- host side of the C ABI declared in include/lora_linear.h.
+//
+// Validates arguments, carves the caller's workspace, encodes TMA tensor maps and
+// enqueues the tcgen05 kernels of tc_gemm.cuh on the caller's stream:
+//
+//   forward   k_xa  : s.xa = bf16(s . x.A^T)            split over d_in   (M x r)
+//             k_fwd : h = [x | s.xa] . [W | B]^T        K = d_in + r, one accumulator
+//   backward  k_xa  : (only when no saved s.xa)
+//             k_g   : s.g = bf16(s . dY.B)              split over d_out  (M x r)
+//             k_dx  : dX = [dY | s.g] . [W ; A]         K = d_out + r, W and A MN-major
+//             k_dB  : dB = dY^T . (s.xa)                split over tokens
+//             k_dA  : dA = (s.g)^T . x  (written as [r, d_in])   split over tokens
+//
+// No allocation, no synchronisation, no exceptions across the ABI.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/lora_linear.h"
+#include "tc_gemm.cuh"
+
+using namespace lora;
+
+namespace {
+
+// ------------------------------------------------------------------ kernel configs
+constexpr int MAIN_BN = 256;
+constexpr int MAIN_STAGES = 4;
+constexpr int SKINNY_SMEM_BUDGET = 196 * 1024;
+
+template <int BN>
+constexpr int skinny_stages() {
+    constexpr int stage = BM * BK * 2 + BN * BK * 2;
+    constexpr int s = SKINNY_SMEM_BUDGET / stage;
+    return s > 8 ? 8 : s;
+}
+
+// ------------------------------------------------------------------ device info
+struct DevInfo {
+    bool probed = false;
+    bool supported = false;
+    int sms = 0;
+    uint64_t attr_set = 0;  // bit per kernel instantiation whose smem attribute is set
+};
+std::mutex g_mu;
+DevInfo g_dev[64];
+
+bool device_info(int *dev_out, DevInfo **info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevInfo &d = g_dev[dev];
+    if (!d.probed) {
+        int major = 0, minor = 0, sms = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        d.supported = (major == 10 && minor == 0);
+        d.sms = sms;
+        d.probed = true;
+    }
+    *dev_out = dev;
+    *info = &d;
+    return true;
+}
+
+// ------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major 2D bf16 tensor [rows][cols] (cols contiguous), tile box {box_cols, box_rows},
+// 128-byte swizzle, zero fill outside the tensor.
+bool tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+               uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ timing hooks
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_timing{0};
+struct TimedLaunch {
+    int kind;
+    cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+std::vector<TimedLaunch> g_timed;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// ------------------------------------------------------------------ launch helpers
+template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
+cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
+    using Cfg = GemmCfg<BN, A_MN, B_MN, EPI, STAGES>;
+    auto kern = k_tc_gemm<BN, A_MN, B_MN, EPI, STAGES>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(dev->attr_set & (1ull << attr_bit))) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            dev->attr_set |= 1ull << attr_bit;
+        }
+    }
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    const bool timed = g_timing.load() != 0;
+    if (timed) {
+        std::lock_guard<std::mutex> lk(g_tmu);
+        ea = pool_event();
+        eb = pool_event();
+        if (ea) cudaEventRecord(ea, st);
+    }
+    kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(args);
+    cudaError_t e = cudaGetLastError();
+    g_launches.fetch_add(1);
+    if (timed && ea && eb) {
+        cudaEventRecord(eb, st);
+        std::lock_guard<std::mutex> lk(g_tmu);
+        g_timed.push_back({kind, ea, eb});
+    }
+    return e;
+}
+
+// Attribute bits of the instantiations (one per template combination).
+enum {
+    AB_FWD = 0,
+    AB_DX = 1,
+    AB_XA16 = 2, AB_XA64, AB_XA128, AB_XA256,
+    AB_G64 = 6, AB_G128, AB_G256,
+    AB_T64 = 9, AB_T128, AB_T256,
+};
+
+int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
+int bn_class_mnmajor(int r) { return r <= 64 ? 64 : r <= 128 ? 128 : 256; }
+
+// ------------------------------------------------------------------ workspace plan
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Split {
+    int splits = 1, per = 1;
+};
+
+// Splits of K (in 64-wide blocks) for a skinny kernel with `mt` output tiles: pick
+// the count that minimises (waves of tiles) x (blocks per split) on `sms` SMs.
+Split choose_split(int64_t mt, int64_t kb, int sms) {
+    Split best;
+    int64_t best_cost = INT64_MAX;
+    const int64_t smax = std::min<int64_t>(kb, 64);
+    for (int64_t s = 1; s <= smax; ++s) {
+        const int64_t per = cdiv(kb, s);
+        const int64_t eff = cdiv(kb, per);
+        const int64_t tiles = mt * eff;
+        const int64_t cost = cdiv(tiles, sms) * per;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best.splits = static_cast<int>(eff);
+            best.per = static_cast<int>(per);
+        }
+    }
+    return best;
+}
+
+constexpr int PLAN_SMS = 148;  // sizes the workspace for up to this many SMs' worth of splits
+
+struct Plan {
+    size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0, total = 0;
+    int64_t n_ctr = 0;
+    Split s_xa, s_g, s_db, s_da;
+};
+
+bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, Plan *pl) {
+    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4);
+    const int64_t mt_tok = cdiv(M, BM), mt_in = cdiv(d_in, BM), mt_out = cdiv(d_out, BM);
+    pl->s_xa = choose_split(mt_tok, cdiv(d_in, BK), sms);
+    pl->s_g = choose_split(mt_tok, cdiv(d_out, BK), sms);
+    pl->s_db = choose_split(mt_out, cdiv(M, BK), sms);
+    pl->s_da = choose_split(mt_in, cdiv(M, BK), sms);
+    size_t off = 0;
+    pl->err = off;
+    off += 256;
+    pl->ctr = off;
+    pl->n_ctr = mt_tok * 2 + mt_in + mt_out;
+    off = align256(off + pl->n_ctr * sizeof(int));
+    pl->xa = off;
+    off = align256(off + M * r * 2);
+    pl->part_xa = off;
+    off = align256(off + static_cast<size_t>(pl->s_xa.splits) * mt_tok * BM * r * 4);
+    if (bwd) {
+        pl->g = off;
+        off = align256(off + M * r * 2);
+        pl->part_g = off;
+        off = align256(off + static_cast<size_t>(pl->s_g.splits) * mt_tok * BM * r * 4);
+        pl->part_db = off;
+        off = align256(off + static_cast<size_t>(pl->s_db.splits) * mt_out * BM * r * 4);
+        pl->part_da = off;
+        off = align256(off + static_cast<size_t>(pl->s_da.splits) * mt_in * BM * r * 4);
+    }
+    pl->total = off;
+    return true;
+}
+
+// ------------------------------------------------------------------ validation
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, bool q4) {
+    if (M < 1 || M > (int64_t(1) << 30)) return LORA_ERR_INVALID_ARG;
+    if (d_in < 8 || d_out < 8 || d_in % 8 || d_out % 8) return LORA_ERR_INVALID_ARG;
+    if (d_in > (int64_t(1) << 24) || d_out > (int64_t(1) << 24)) return LORA_ERR_INVALID_ARG;
+    if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
+    if (!std::isfinite(alpha)) return LORA_ERR_INVALID_ARG;
+    if (q4 && d_in % 64) return LORA_ERR_INVALID_ARG;
+    return LORA_OK;
+}
+
+struct Ctx {
+    int dev = 0;
+    DevInfo *info = nullptr;
+    Plan plan;
+    uint8_t *ws = nullptr;
+    cudaStream_t st = nullptr;
+};
+
+lora_status_t prepare(int op, int64_t M, int64_t d_in, int64_t d_out, int r, void *ws, size_t ws_bytes,
+                      void *stream, Ctx *c) {
+    if (!device_info(&c->dev, &c->info)) return LORA_ERR_CUDA;
+    if (!c->info->supported) return LORA_ERR_UNSUPPORTED;
+    make_plan(op, M, d_in, d_out, r, PLAN_SMS, &c->plan);
+    if (!ws) return LORA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) & 255u) return LORA_ERR_MISALIGNED;
+    if (ws_bytes < c->plan.total) return LORA_ERR_WORKSPACE;
+    c->ws = static_cast<uint8_t *>(ws);
+    c->st = static_cast<cudaStream_t>(stream);
+    return LORA_OK;
+}
+
+// ------------------------------------------------------------------ step launchers
+GemmArgs base_args(const Ctx &c) {
+    GemmArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.err = reinterpret_cast<int *>(c.ws + c.plan.err);
+    a.group_m = 1;
+    return a;
+}
+
+// Skinny split-K contraction D[rows, r] (rows = M-dim) over K, with A [*, *] bf16.
+// a_mn / b_mn select the operand majorness; the tensor maps are built by the caller.
+template <bool A_MN, bool B_MN>
+lora_status_t launch_skinny(const Ctx &c, GemmArgs &a, int r, int64_t rows, int64_t kdim, const Split &sp,
+                            float *part, int *ctr, void *out, int out_mode, int64_t out_ld, float scale,
+                            int kind) {
+    const int64_t mt = cdiv(rows, BM);
+    a.m_tiles = static_cast<int>(mt);
+    a.n_tiles = 1;
+    a.kb0 = static_cast<int>(cdiv(kdim, BK));
+    a.kb1 = 0;
+    a.splits = sp.splits;
+    a.kb_per_split = sp.per;
+    a.num_tiles = static_cast<int>(mt * sp.splits);
+    a.rows_valid = static_cast<int>(rows);
+    a.n_valid = r;
+    a.out_mode = out_mode;
+    a.out_scale = scale;
+    a.part = part;
+    a.counters = ctr;
+    a.out = out;
+    a.out_ld = out_ld;
+    const int grid = std::min(a.num_tiles, c.info->sms);
+    cudaError_t e;
+    if (!A_MN && !B_MN) {
+        switch (bn_class_kmajor(r)) {
+            case 16: e = launch_gemm<16, false, false, EPI_SPLITK, skinny_stages<16>()>(a, grid, c.st, c.info, AB_XA16, kind); break;
+            case 64: e = launch_gemm<64, false, false, EPI_SPLITK, skinny_stages<64>()>(a, grid, c.st, c.info, AB_XA64, kind); break;
+            case 128: e = launch_gemm<128, false, false, EPI_SPLITK, skinny_stages<128>()>(a, grid, c.st, c.info, AB_XA128, kind); break;
+            default: e = launch_gemm<256, false, false, EPI_SPLITK, skinny_stages<256>()>(a, grid, c.st, c.info, AB_XA256, kind); break;
+        }
+    } else if (!A_MN && B_MN) {
+        switch (bn_class_mnmajor(r)) {
+            case 64: e = launch_gemm<64, false, true, EPI_SPLITK, skinny_stages<64>()>(a, grid, c.st, c.info, AB_G64, kind); break;
+            case 128: e = launch_gemm<128, false, true, EPI_SPLITK, skinny_stages<128>()>(a, grid, c.st, c.info, AB_G128, kind); break;
+            default: e = launch_gemm<256, false, true, EPI_SPLITK, skinny_stages<256>()>(a, grid, c.st, c.info, AB_G256, kind); break;
+        }
+    } else {
+        switch (bn_class_mnmajor(r)) {
+            case 64: e = launch_gemm<64, true, true, EPI_SPLITK, skinny_stages<64>()>(a, grid, c.st, c.info, AB_T64, kind); break;
+            case 128: e = launch_gemm<128, true, true, EPI_SPLITK, skinny_stages<128>()>(a, grid, c.st, c.info, AB_T128, kind); break;
+            default: e = launch_gemm<256, true, true, EPI_SPLITK, skinny_stages<256>()>(a, grid, c.st, c.info, AB_T256, kind); break;
+        }
+    }
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// s.xa = bf16(s . x.A^T) -> dst [M, r]
+lora_status_t step_xa(const Ctx &c, const uint16_t *x, const uint16_t *A, uint16_t *dst, int64_t M, int64_t d_in,
+                      int r, float s) {
+    GemmArgs a = base_args(c);
+    const int bn = bn_class_kmajor(r);
+    if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB0, A, d_in, r, 64, bn)) return LORA_ERR_CUDA;
+    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr);
+    return launch_skinny<false, false>(c, a, r, M, d_in, c.plan.s_xa, reinterpret_cast<float *>(c.ws + c.plan.part_xa),
+                                       ctr, dst, OUT_BF16_ROWS, 0, s, LORA_K_XA);
+}
+
+// s.g = bf16(s . dY.B) -> ws g [M, r]; B [d_out, r] is read MN-major (r contiguous).
+lora_status_t step_g(const Ctx &c, const uint16_t *dY, const uint16_t *B, int64_t M, int64_t d_out, int r, float s) {
+    GemmArgs a = base_args(c);
+    if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB0, B, r, d_out, 64, 64)) return LORA_ERR_CUDA;
+    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + cdiv(M, BM);
+    return launch_skinny<false, true>(c, a, r, M, d_out, c.plan.s_g, reinterpret_cast<float *>(c.ws + c.plan.part_g),
+                                      ctr, c.ws + c.plan.g, OUT_BF16_ROWS, 0, s, LORA_K_G);
+}
+
+// dB [d_out, r] = dY^T . (s.xa): M-dim = d_out, K = tokens, both operands MN-major.
+lora_status_t step_db(const Ctx &c, const uint16_t *dY, const uint16_t *sxa, float *dB, int64_t M, int64_t d_out,
+                      int r) {
+    GemmArgs a = base_args(c);
+    if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 64)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB0, sxa, r, M, 64, 64)) return LORA_ERR_CUDA;
+    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + 2 * cdiv(M, BM);
+    return launch_skinny<true, true>(c, a, r, d_out, M, c.plan.s_db, reinterpret_cast<float *>(c.ws + c.plan.part_db),
+                                     ctr, dB, OUT_F32_ROWS, 0, 1.0f, LORA_K_DB);
+}
+
+// dA [r, d_in] = (s.g)^T . x: computed as dA^T (M-dim = d_in) and written transposed.
+lora_status_t step_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float *dA, int64_t M, int64_t d_in,
+                      int64_t d_out, int r) {
+    GemmArgs a = base_args(c);
+    if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 64)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB0, sg, r, M, 64, 64)) return LORA_ERR_CUDA;
+    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + 2 * cdiv(M, BM) + cdiv(d_out, BM);
+    return launch_skinny<true, true>(c, a, r, d_in, M, c.plan.s_da, reinterpret_cast<float *>(c.ws + c.plan.part_da),
+                                     ctr, dA, OUT_F32_COLS, d_in, 1.0f, LORA_K_DA);
+}
+
+// Main K-concatenated GEMM: out [M, N] = A0 . B0^T (K0) + A1 . B1^T (K1 = r).
+lora_status_t step_main(const Ctx &c, GemmArgs &a, int64_t M, int64_t N, int64_t K0, int r, bool b_mn, int kind) {
+    a.m_tiles = static_cast<int>(cdiv(M, BM));
+    a.n_tiles = static_cast<int>(cdiv(N, MAIN_BN));
+    a.kb0 = static_cast<int>(cdiv(K0, BK));
+    a.kb1 = static_cast<int>(cdiv(r, BK));
+    a.mma_last1 = static_cast<int>(cdiv(r - (a.kb1 - 1) * BK, 16));
+    a.splits = 1;
+    a.kb_per_split = a.kb0;
+    a.num_tiles = a.m_tiles * a.n_tiles;
+    a.group_m = std::min(a.m_tiles, 16);
+    const int grid = std::min(a.num_tiles, c.info->sms);
+    cudaError_t e;
+    if (b_mn)
+        e = launch_gemm<MAIN_BN, false, true, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_DX, kind);
+    else
+        e = launch_gemm<MAIN_BN, false, false, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_FWD, kind);
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+lora_status_t zero_counters(const Ctx &c) {
+    return cudaMemsetAsync(c.ws + c.plan.ctr, 0, c.plan.n_ctr * sizeof(int), c.st) == cudaSuccess ? LORA_OK
+                                                                                                   : LORA_ERR_CUDA;
+}
+
+#define LORA_TRY(x)                          \
+    do {                                     \
+        lora_status_t _s = (x);              \
+        if (_s != LORA_OK) return _s;        \
+    } while (0)
+
+lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, const uint16_t *B, uint16_t *h,
+                       uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, void *ws,
+                       size_t ws_bytes, void *stream) {
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, false));
+    if (!x || !W || !A || !B || !h) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(h) ||
+        (xa_save && !aligned16(xa_save)))
+        return LORA_ERR_MISALIGNED;
+    Ctx c;
+    LORA_TRY(prepare(LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    const float s = alpha / static_cast<float>(r);
+    uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
+    LORA_TRY(zero_counters(c));
+    LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
+    GemmArgs a = base_args(c);
+    if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB0, W, d_in, d_out, 64, MAIN_BN)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmA1, sxa, r, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB1, B, r, d_out, 64, MAIN_BN)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmC, h, d_out, M, 64, 32)) return LORA_ERR_CUDA;
+    return step_main(c, a, M, d_out, d_in, r, false, LORA_K_FWD_MAIN);
+}
+
+lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
+                       const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB, int64_t M,
+                       int64_t d_in, int64_t d_out, int r, float alpha, void *ws, size_t ws_bytes, void *stream) {
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, false));
+    if (!dY || !x || !W || !A || !B || !dA || !dB) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(dY) || !aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+        !aligned16(dB) || (xa_save && !aligned16(xa_save)) || (dX && !aligned16(dX)))
+        return LORA_ERR_MISALIGNED;
+    Ctx c;
+    LORA_TRY(prepare(LORA_OP_BWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    const float s = alpha / static_cast<float>(r);
+    LORA_TRY(zero_counters(c));
+    const uint16_t *sxa = xa_save;
+    if (!sxa) {
+        uint16_t *tmp = reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
+        LORA_TRY(step_xa(c, x, A, tmp, M, d_in, r, s));
+        sxa = tmp;
+    }
+    LORA_TRY(step_g(c, dY, B, M, d_out, r, s));
+    const uint16_t *sg = reinterpret_cast<const uint16_t *>(c.ws + c.plan.g);
+    if (dX) {
+        GemmArgs a = base_args(c);
+        if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
+        if (!tmap_bf16(&a.tmB0, W, d_in, d_out, 64, 64)) return LORA_ERR_CUDA;  // MN-major: d_in contiguous
+        if (!tmap_bf16(&a.tmA1, sg, r, M, 64, 128)) return LORA_ERR_CUDA;
+        if (!tmap_bf16(&a.tmB1, A, d_in, r, 64, 64)) return LORA_ERR_CUDA;      // MN-major: d_in contiguous
+        if (!tmap_bf16(&a.tmC, dX, d_in, M, 64, 32)) return LORA_ERR_CUDA;
+        LORA_TRY(step_main(c, a, M, d_in, d_out, r, true, LORA_K_DX_MAIN));
+    }
+    LORA_TRY(step_db(c, dY, sxa, dB, M, d_out, r));
+    LORA_TRY(step_da(c, x, sg, dA, M, d_in, d_out, r));
+    return LORA_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r) {
+    if (op < LORA_OP_FWD || op > LORA_OP_BWD_Q4) return 0;
+    if (check_shapes(M, d_in, d_out, r, 1.0f, op >= LORA_OP_FWD_Q4) != LORA_OK) return 0;
+    Plan pl;
+    make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
+    return pl.total;
+}
+
+lora_status_t lora_linear_fwd(const uint16_t *x, const uint16_t *W, const uint16_t *A, const uint16_t *B, uint16_t *h,
+                              uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    return fwd_impl(x, W, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
+}
+
+lora_status_t lora_linear_bwd(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
+                              const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
+                              int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, void *workspace,
+                              size_t workspace_bytes, void *stream) {
+    return bwd_impl(dY, x, W, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                    stream);
+}
+
+lora_status_t lora_linear_fwd_q4(const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
+                                 const uint16_t *B, uint16_t *h, uint16_t *xa_save, int64_t M, int64_t d_in,
+                                 int64_t d_out, int r, float alpha, void *workspace, size_t workspace_bytes,
+                                 void *stream) {
+    (void)x; (void)Wq; (void)Wscale; (void)A; (void)B; (void)h; (void)xa_save; (void)M; (void)d_in;
+    (void)d_out; (void)r; (void)alpha; (void)workspace; (void)workspace_bytes; (void)stream;
+    return LORA_ERR_UNSUPPORTED;
+}
+
+lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale,
+                                 const uint16_t *A, const uint16_t *B, const uint16_t *xa_save, uint16_t *dX,
+                                 float *dA, float *dB, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    (void)dY; (void)x; (void)Wq; (void)Wscale; (void)A; (void)B; (void)xa_save; (void)dX; (void)dA; (void)dB;
+    (void)M; (void)d_in; (void)d_out; (void)r; (void)alpha; (void)workspace; (void)workspace_bytes; (void)stream;
+    return LORA_ERR_UNSUPPORTED;
+}
+
+lora_status_t lora_linear_check(void *workspace, void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LORA_ERR_CUDA;
+    if (!workspace) return LORA_OK;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LORA_ERR_CUDA;
+    if (word != 0) {
+        cudaMemset(workspace, 0, sizeof(int));
+        return LORA_ERR_TIMEOUT;
+    }
+    return LORA_OK;
+}
+
+const char *lora_status_string(lora_status_t status) {
+    switch (status) {
+        case LORA_OK: return "ok";
+        case LORA_ERR_INVALID_ARG: return "invalid argument (null pointer, shape, r or alpha)";
+        case LORA_ERR_MISALIGNED: return "misaligned pointer (16 B; workspace 256 B)";
+        case LORA_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device / covered shape)";
+        case LORA_ERR_WORKSPACE: return "workspace missing or too small";
+        case LORA_ERR_CUDA: return "CUDA error";
+        case LORA_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int64_t lora_linear_launch_count(void) { return g_launches.load(); }
+
+lora_status_t lora_linear_timing_enable(int enable) {
+    g_timing.store(enable ? 1 : 0);
+    return LORA_OK;
+}
+
+lora_status_t lora_linear_timing_read(double *ms_per_kind, int64_t *launches_per_kind, int kinds) {
+    std::vector<TimedLaunch> rec;
+    {
+        std::lock_guard<std::mutex> lk(g_tmu);
+        rec.swap(g_timed);
+    }
+    for (int k = 0; k < kinds; ++k) {
+        if (ms_per_kind) ms_per_kind[k] = 0.0;
+        if (launches_per_kind) launches_per_kind[k] = 0;
+    }
+    lora_status_t st = LORA_OK;
+    for (const TimedLaunch &t : rec) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(t.b) != cudaSuccess || cudaEventElapsedTime(&ms, t.a, t.b) != cudaSuccess)
+            st = LORA_ERR_CUDA;
+        else if (t.kind >= 0 && t.kind < kinds) {
+            if (ms_per_kind) ms_per_kind[t.kind] += ms;
+            if (launches_per_kind) launches_per_kind[t.kind] += 1;
+        }
+    }
+    std::lock_guard<std::mutex> lk(g_tmu);
+    for (const TimedLaunch &t : rec) {
+        g_event_pool.push_back(t.a);
+        g_event_pool.push_back(t.b);
+    }
+    return st;
+}
+
+}  // extern "C"

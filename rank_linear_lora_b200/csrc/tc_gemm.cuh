@@ -1,0 +1,444 @@
+// tc_gemm.cuh -- the tcgen05 contraction engine behind every step of the layer.
+//
+// One persistent, warp-specialised kernel template computes a 128 x BN output tile
+//     D = sum over K-segments  A_seg . B_seg^T
+// with bf16 operands staged by TMA into 128-byte-swizzled shared memory and fp32
+// accumulators in tensor memory:
+//   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2..5  epilogue: tcgen05.ld of their 32-lane TMEM quarter
+// Two accumulators alternate in TMEM so the epilogue of one tile overlaps the
+// K loop of the next.
+//
+// K-segments: segment 0 is the frozen-weight contraction (K = d_in or d_out);
+// segment 1, when present, is the rank-r side product appended to the same K loop
+// (K = r), so the low-rank term is added by the tensor cores inside the same
+// accumulator instead of by a separate pass.  Operands may be K-major (the K index
+// contiguous in memory) or MN-major (the M/N index contiguous), so W is read in
+// place for both x.W^T and dY.W.
+//
+// Epilogues:
+//   EPI_STORE  bf16 tile -> 128B-swizzled smem staging -> TMA store (h, dX).
+//   EPI_SPLITK fp32 partial of one K-split -> workspace; the last split to finish
+//              a tile (per-tile arrival counter) sums all splits in a fixed order
+//              and writes the result: bf16 rows (s.xa, s.g), fp32 rows (dB) or
+//              fp32 columns (dA, written transposed).  Deterministic.
+//
+// Every wait is bounded (globaltimer); on expiry the kernel records an error code,
+// drains its outstanding copies and MMAs, frees TMEM and returns.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace lora {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int NUM_THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
+
+enum EpiMode { EPI_STORE = 0, EPI_SPLITK = 1 };
+enum OutMode { OUT_BF16_ROWS = 0, OUT_F32_ROWS = 1, OUT_F32_COLS = 2 };
+
+// Error codes written to the workspace error word (first writer wins).
+enum DevErr {
+    DERR_NONE = 0,
+    DERR_WAIT_EMPTY = 0x101,
+    DERR_WAIT_FULL = 0x102,
+    DERR_WAIT_TMEM_EMPTY = 0x103,
+    DERR_WAIT_TMEM_FULL = 0x104,
+    DERR_WAIT_DRAIN = 0x105,
+};
+
+struct GemmArgs {
+    CUtensorMap tmA0, tmB0;  // segment 0
+    CUtensorMap tmA1, tmB1;  // segment 1 (rank-r tail), used when kb1 > 0
+    CUtensorMap tmC;         // EPI_STORE output (bf16, box 64 x 32, 128B swizzle)
+    int m_tiles, n_tiles;
+    int kb0, kb1;            // 64-wide K blocks per segment
+    int mma_last1;           // K=16 MMAs in the last block of segment 1 (1..4)
+    int splits;              // EPI_SPLITK: K splits of segment 0
+    int kb_per_split;
+    int num_tiles;           // m_tiles * n_tiles * splits
+    int group_m;             // EPI_STORE rasterisation: M tiles per group
+    int rows_valid;          // EPI_SPLITK: valid output rows
+    int n_valid;             // EPI_SPLITK: valid output columns (r)
+    int out_mode;            // OutMode
+    float out_scale;
+    float *part;             // EPI_SPLITK partials [splits][m_tiles*BM][n_valid]
+    int *counters;           // EPI_SPLITK per-tile arrival counters (zero on entry)
+    void *out;               // EPI_SPLITK output
+    int64_t out_ld;          // OUT_F32_COLS: row stride of the transposed output
+    int *err;                // device error word
+};
+
+template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
+struct GemmCfg {
+    static constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+    static constexpr int B_BYTES = BN * BK * 2;   // BN rows (or BN/64 chunks) x 128 B
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int EPI_BYTES = (EPI == EPI_STORE) ? 4 * 2 * 32 * 128 : 0;
+    static constexpr int TMEM_COLS = (2 * BN < 32) ? 32 : 2 * BN;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M=128 is 16..256 step 16");
+    static_assert(!B_MN || BN % 64 == 0, "MN-major B uses 64-wide swizzle chunks");
+    static_assert(B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
+    static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM alloc is a power of 2");
+};
+
+// Bounded mbarrier wait.  Returns false (and raises the abort flag and the error
+// word) if the barrier does not reach `parity` within WAIT_LIMIT_NS, or if another
+// role already aborted.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                             int *err, int code) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                atomicCAS(err, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+struct TileCoord {
+    int m, n, split;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const GemmArgs &p, int t, int epi) {
+    TileCoord c;
+    if (epi == EPI_SPLITK) {
+        c.split = t % p.splits;
+        int mn = t / p.splits;
+        c.m = mn % p.m_tiles;
+        c.n = mn / p.m_tiles;
+    } else {
+        // Grouped rasterisation: group_m M-tiles share each B (weight) tile in L2.
+        int group = p.group_m * p.n_tiles;
+        int g = t / group, idx = t % group;
+        int m0 = g * p.group_m;
+        int gm = min(p.group_m, p.m_tiles - m0);
+        c.m = m0 + idx % gm;
+        c.n = idx / gm;
+        c.split = 0;
+    }
+    return c;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
+__global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constant__ GemmArgs p) {
+    using Cfg = GemmCfg<BN, A_MN, B_MN, EPI, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
+    uint8_t *sEpi = smem + STAGES * Cfg::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + Cfg::EPI_BYTES);
+    uint64_t *full_bar = bars;                    // [STAGES]
+    uint64_t *empty_bar = bars + STAGES;          // [STAGES]
+    uint64_t *tfull_bar = bars + 2 * STAGES;      // [2]
+    uint64_t *tempty_bar = bars + 2 * STAGES + 2; // [2]
+    uint64_t *drain_bar = bars + 2 * STAGES + 4;  // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *last_flag = reinterpret_cast<volatile int *>(tmem_slot + 2);
+    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 3);  // [2]
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull_bar[b]), 1);
+            mbar_init(smem_u32(&tempty_bar[b]), 4);
+        }
+        mbar_init(smem_u32(drain_bar), 1);
+        *abort_flag = 0;
+        *last_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&p.tmA0);
+            tma_prefetch_desc(&p.tmB0);
+            if (p.kb1 > 0) {
+                tma_prefetch_desc(&p.tmA1);
+                tma_prefetch_desc(&p.tmB1);
+            }
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued?, parity of last issue
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+                const TileCoord c = decode_tile(p, t, EPI);
+                int kb_lo = 0, kb_hi = p.kb0 + p.kb1;
+                if (EPI == EPI_SPLITK) {
+                    kb_lo = c.split * p.kb_per_split;
+                    kb_hi = min(p.kb0, kb_lo + p.kb_per_split);
+                }
+                for (int kb = kb_lo; kb < kb_hi; ++kb) {
+                    if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
+                                      DERR_WAIT_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                    issued_mask |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    const bool seg1 = kb >= p.kb0;
+                    const CUtensorMap *ta = seg1 ? &p.tmA1 : &p.tmA0;
+                    const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
+                    const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
+                    const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
+                    if (A_MN) {
+                        tma_load_2d(a_dst, ta, fb, c.m * BM, k0);
+                        tma_load_2d(a_dst + 64 * 128, ta, fb, c.m * BM + 64, k0);
+                    } else {
+                        tma_load_2d(a_dst, ta, fb, k0, c.m * BM);
+                    }
+                    if (B_MN) {
+#pragma unroll
+                        for (int i = 0; i < BN / 64; ++i)
+                            tma_load_2d(b_dst + i * 64 * 128, tb, fb, c.n * BN + 64 * i, k0);
+                    } else {
+                        tma_load_2d(b_dst, tb, fb, k0, c.n * BN);
+                    }
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // Drain: every issued copy must have landed before the CTA exits.
+            for (int s = 0; s < STAGES; ++s)
+                if (issued_mask & (1u << s)) {
+                    volatile int never = 0;
+                    wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
+                                 DERR_WAIT_DRAIN);
+                }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+            // K step of 16 elements inside a stage: +32 B along a K-major row,
+            // +16 rows (2 swizzle atoms) for an MN-major tile.
+            constexpr uint32_t a_kstep = A_MN ? 2048u : 32u;
+            constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
+            constexpr uint32_t a_lbo = A_MN ? 64u * 128u : 16u;
+            constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
+                const TileCoord c = decode_tile(p, t, EPI);
+                int nkb = p.kb0 + p.kb1;
+                if (EPI == EPI_SPLITK) {
+                    const int lo = c.split * p.kb_per_split;
+                    nkb = min(p.kb0, lo + p.kb_per_split) - lo;
+                }
+                const int buf = it & 1;
+                const uint32_t aphase = (it >> 1) & 1;
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
+                                  DERR_WAIT_TMEM_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int i = 0; i < nkb; ++i) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err,
+                                      DERR_WAIT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const bool last_tail = (EPI == EPI_STORE) && p.kb1 > 0 && i == nkb - 1;
+                    const int nmma = last_tail ? p.mma_last1 : BK / 16;
+                    const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        const uint64_t ad = sdesc_sw128(a_base + kk * a_kstep, a_lbo, 1024);
+                        const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(smem_u32(&tfull_bar[buf]));
+            }
+            // Drain: all MMAs issued by this thread complete before TMEM is freed.
+            tc_commit(smem_u32(drain_bar));
+            volatile int never = 0;
+            wait_bounded(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;                 // TMEM lane quarter of this warp
+        const int row_local = q * 32 + lane;    // accumulator row of this thread
+        const int epi_tid = threadIdx.x - 64;   // 0..127
+        int it = 0;
+        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
+            const TileCoord c = decode_tile(p, t, EPI);
+            const int buf = it & 1;
+            const uint32_t aphase = (it >> 1) & 1;
+            // One thread waits; the outcome is broadcast so all four warps take the
+            // same path (the split-K fixup below uses named barriers).
+            if (epi_tid == 0)
+                epi_ok[it & 1] = wait_bounded(smem_u32(&tfull_bar[buf]), aphase, abort_flag, p.err,
+                                              DERR_WAIT_TMEM_FULL) ? 1 : 0;
+            named_bar_sync(1, 128);
+            if (!epi_ok[it & 1]) break;
+            tc_fence_after();
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                                   static_cast<uint32_t>(buf * BN);
+            if constexpr (EPI == EPI_STORE) {
+                uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
+#pragma unroll 1
+                for (int ch = 0; ch < BN / 64; ++ch) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(t_row + ch * 64, v0);
+                    tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
+                    tc_wait_ld();
+                    if (ch == BN / 64 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
+                    }
+                    uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                    // The TMA store that used this buffer two chunks ago must have read it.
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    uint32_t packed[32];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 lo2 = __floats2bfloat162_rn(__uint_as_float(v0[2 * j]),
+                                                                   __uint_as_float(v0[2 * j + 1]));
+                        __nv_bfloat162 hi2 = __floats2bfloat162_rn(__uint_as_float(v1[2 * j]),
+                                                                   __uint_as_float(v1[2 * j + 1]));
+                        packed[j] = *reinterpret_cast<uint32_t *>(&lo2);
+                        packed[16 + j] = *reinterpret_cast<uint32_t *>(&hi2);
+                    }
+                    // Row `lane` of a 32 x 64 bf16 box, 128-byte swizzle: 16-byte chunk cc
+                    // lands at chunk (cc ^ (row % 8)).
+                    uint8_t *row_ptr = sbuf + lane * 128;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        uint4 w = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2],
+                                             packed[4 * cc + 3]);
+                        *reinterpret_cast<uint4 *>(row_ptr + ((cc ^ (lane & 7)) * 16)) = w;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&p.tmC, smem_u32(sbuf), c.n * BN + ch * 64, c.m * BM + q * 32);
+                        bulk_commit_group();
+                    }
+                }
+            } else {
+                // fp32 partial of this K split -> workspace.
+                const int64_t rows_total = static_cast<int64_t>(p.m_tiles) * BM;
+                const int64_t grow = static_cast<int64_t>(c.m) * BM + row_local;
+                float *my_part = p.part + ((static_cast<int64_t>(c.split) * rows_total + grow) * p.n_valid);
+                for (int c0 = 0; c0 < p.n_valid; c0 += 8) {
+                    uint32_t v[8];
+                    tmem_ld_32x32b_x8(t_row + c0, v);
+                    tc_wait_ld();
+                    float4 *dst = reinterpret_cast<float4 *>(my_part + c0);
+                    dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
+                                         __uint_as_float(v[3]));
+                    dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
+                                         __uint_as_float(v[7]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
+                __threadfence();
+                named_bar_sync(1, 128);
+                const int ctr = c.n * p.m_tiles + c.m;
+                if (epi_tid == 0) *last_flag = (atomicAdd(&p.counters[ctr], 1) == p.splits - 1) ? 1 : 0;
+                named_bar_sync(1, 128);
+                const bool last = *last_flag != 0;
+                named_bar_sync(1, 128);  // everyone has read last_flag before it is reused
+                if (last) {
+                    __threadfence();
+                    if (grow < p.rows_valid) {
+                        for (int c0 = 0; c0 < p.n_valid; c0 += 4) {
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                            for (int s = 0; s < p.splits; ++s) {
+                                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
+                                    p.part + ((static_cast<int64_t>(s) * rows_total + grow) * p.n_valid + c0)));
+                                acc.x += v.x;
+                                acc.y += v.y;
+                                acc.z += v.z;
+                                acc.w += v.w;
+                            }
+                            acc.x *= p.out_scale;
+                            acc.y *= p.out_scale;
+                            acc.z *= p.out_scale;
+                            acc.w *= p.out_scale;
+                            if (p.out_mode == OUT_BF16_ROWS) {
+                                __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
+                                __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
+                                uint2 w = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+                                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + grow * p.n_valid + c0) = w;
+                            } else if (p.out_mode == OUT_F32_ROWS) {
+                                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + grow * p.n_valid + c0) = acc;
+                            } else {
+                                float *o = static_cast<float *>(p.out);
+                                o[(c0 + 0) * p.out_ld + grow] = acc.x;
+                                o[(c0 + 1) * p.out_ld + grow] = acc.y;
+                                o[(c0 + 2) * p.out_ld + grow] = acc.z;
+                                o[(c0 + 3) * p.out_ld + grow] = acc.w;
+                            }
+                        }
+                    }
+                    if (epi_tid == 0) p.counters[ctr] = 0;  // ready for the next call
+                }
+            }
+        }
+        if constexpr (EPI == EPI_STORE) {
+            if (lane == 0) bulk_wait_group<0>();
+        }
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+    }
+}
+
+}  // namespace lora

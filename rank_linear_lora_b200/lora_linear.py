@@ -1,0 +1,206 @@
+"""Python binding of liblora_linear.so (argument marshalling only).
+
+Every function has the name of its C entry point (include/lora_linear.h), takes
+torch tensors that already live on the GPU, passes their pointers, sizes and the
+current CUDA stream through ctypes, and raises LoraError on a non-OK status.  All
+arithmetic runs in the library's CUDA kernels; there is no fallback: if the shared
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_linear.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lora_linear.h")
+
+LORA_OK = 0
+STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_MISALIGNED", 3: "LORA_ERR_UNSUPPORTED",
+          4: "LORA_ERR_WORKSPACE", 5: "LORA_ERR_CUDA", 6: "LORA_ERR_TIMEOUT"}
+OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4 = 0, 1, 2, 3
+KERNEL_KINDS = ["xa", "fwd_main", "g", "dx_main", "dB", "dA"]
+
+
+class LoraError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({lora_status_string(status)})")
+
+
+_lib = None
+
+
+def load_library():
+    """Load the in-tree CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run rank_linear_lora_b200/build.py)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I, F, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.lora_linear_workspace_size.argtypes = [I, I64, I64, I64, I]
+    lib.lora_linear_workspace_size.restype = SZ
+    lib.lora_linear_fwd.argtypes = [P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_fwd_q4.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_bwd_q4.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    for f in ("lora_linear_fwd", "lora_linear_bwd", "lora_linear_fwd_q4", "lora_linear_bwd_q4"):
+        getattr(lib, f).restype = I
+    lib.lora_linear_check.argtypes = [P, P]
+    lib.lora_linear_check.restype = I
+    lib.lora_status_string.argtypes = [I]
+    lib.lora_status_string.restype = ctypes.c_char_p
+    lib.lora_linear_launch_count.restype = I64
+    lib.lora_linear_timing_enable.argtypes = [I]
+    lib.lora_linear_timing_enable.restype = I
+    lib.lora_linear_timing_read.argtypes = [P, P, I]
+    lib.lora_linear_timing_read.restype = I
+    _lib = lib
+    return lib
+
+
+def declared_functions() -> list[str]:
+    """Names of the functions include/lora_linear.h declares."""
+    text = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^LORA_API\s+[a-z_0-9 ]+?\*?\s*(lora_[a-z_0-9]+)\s*\(", text, re.M)))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != LORA_OK:
+        raise LoraError(status, where)
+
+
+def _bf16(t, name, shape):
+    if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected a contiguous CUDA bfloat16 tensor of shape {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def _f32(t, name, shape):
+    if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected a contiguous CUDA float32 tensor of shape {tuple(shape)}")
+
+
+def lora_status_string(status: int) -> str:
+    return load_library().lora_status_string(int(status)).decode()
+
+
+def lora_linear_workspace_size(op: int, M: int, d_in: int, d_out: int, r: int) -> int:
+    return int(load_library().lora_linear_workspace_size(op, M, d_in, d_out, r))
+
+
+def workspace(op: int, M: int, d_in: int, d_out: int, r: int, device=None) -> torch.Tensor:
+    """A zeroed uint8 workspace of the size the library asks for (torch allocates)."""
+    n = lora_linear_workspace_size(op, M, d_in, d_out, r)
+    if n == 0:
+        raise ValueError("invalid sizes for the workspace")
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def lora_linear_fwd(x, W, A, B, h, xa_save, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = W.shape[0]
+    for t, n, s in ((x, "x", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
+                    (h, "h", (M, d_out))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    st = load_library().lora_linear_fwd(_ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(h), _ptr(xa_save), M, d_in, d_out,
+                                        r, float(alpha), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lora_linear_fwd")
+
+
+def lora_linear_bwd(dY, x, W, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = W.shape[0]
+    for t, n, s in ((dY, "dY", (M, d_out)), (x, "x", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)),
+                    (B, "B", (d_out, r))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    if dX is not None:
+        _bf16(dX, "dX", (M, d_in))
+    _f32(dA, "dA", (r, d_in))
+    _f32(dB, "dB", (d_out, r))
+    st = load_library().lora_linear_bwd(_ptr(dY), _ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(xa_save), _ptr(dX),
+                                        _ptr(dA), _ptr(dB), M, d_in, d_out, r, float(alpha), _ptr(ws), ws.numel(),
+                                        _stream(stream))
+    _check(st, "lora_linear_bwd")
+
+
+def _q4(Wq, Wscale, d_out, d_in):
+    if Wq.dtype != torch.uint8 or not Wq.is_cuda or not Wq.is_contiguous() or tuple(Wq.shape) != (d_out, d_in // 2):
+        raise ValueError(f"Wq: expected a contiguous CUDA uint8 tensor of shape {(d_out, d_in // 2)}")
+    _bf16(Wscale, "Wscale", (d_out, d_in // 64))
+
+
+def lora_linear_fwd_q4(x, Wq, Wscale, A, B, h, xa_save, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = Wq.shape[0]
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (h, "h", (M, d_out))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    st = load_library().lora_linear_fwd_q4(_ptr(x), _ptr(Wq), _ptr(Wscale), _ptr(A), _ptr(B), _ptr(h),
+                                           _ptr(xa_save), M, d_in, d_out, r, float(alpha), _ptr(ws), ws.numel(),
+                                           _stream(stream))
+    _check(st, "lora_linear_fwd_q4")
+
+
+def lora_linear_bwd_q4(dY, x, Wq, Wscale, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = Wq.shape[0]
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((dY, "dY", (M, d_out)), (x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    if dX is not None:
+        _bf16(dX, "dX", (M, d_in))
+    _f32(dA, "dA", (r, d_in))
+    _f32(dB, "dB", (d_out, r))
+    st = load_library().lora_linear_bwd_q4(_ptr(dY), _ptr(x), _ptr(Wq), _ptr(Wscale), _ptr(A), _ptr(B),
+                                           _ptr(xa_save), _ptr(dX), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
+                                           float(alpha), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lora_linear_bwd_q4")
+
+
+def lora_linear_check(ws, stream=None):
+    _check(load_library().lora_linear_check(_ptr(ws), _stream(stream)), "lora_linear_check")
+
+
+def lora_linear_launch_count() -> int:
+    return int(load_library().lora_linear_launch_count())
+
+
+def lora_linear_timing_enable(on: bool):
+    _check(load_library().lora_linear_timing_enable(1 if on else 0), "lora_linear_timing_enable")
+
+
+def lora_linear_timing_read():
+    """{kind: (total_ms, launches)} for every kernel kind since the last read."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    _check(load_library().lora_linear_timing_read(ms, cnt, n), "lora_linear_timing_read")
+    return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}

@@ -1,0 +1,120 @@
+"""Shared helpers of the GPU tests: move generator output to the device, run the
+library through its C ABI, ask the oracle for the same quantities, compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from rank_linear_lora_b200 import inputs
+from rank_linear_lora_b200 import lora_linear as L
+
+# Tolerances of the contract: ||gpu - ref||_inf <= rel * ||ref||_inf + abs.
+TOL_HX = (1e-2, 1e-3)   # h, dX
+TOL_AB = (2e-2, 0.0)    # dA, dB
+# Tighter diagnostic on the rms error (bf16 output rounding is ~2^-9 relative), so a
+# dropped piece of the low-rank term cannot hide under the max-norm bound.
+RMS_HX = 4e-3
+RMS_AB = 1e-2
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev_u8(a: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+class DeviceLayer:
+    """Device copies of one layer's inputs plus output buffers and workspaces."""
+
+    def __init__(self, inp: inputs.LayerInputs):
+        sp = inp.spec
+        self.spec, self.inp = sp, inp
+        self.x, self.A, self.B, self.dY = (dev_bf16(a) for a in (inp.x, inp.A, inp.B, inp.dY))
+        self.q4 = sp.q4
+        if sp.q4:
+            self.Wq, self.Wscale = dev_u8(inp.Wq), dev_bf16(inp.Wscale)
+            self.W = None
+        else:
+            self.W = dev_bf16(inp.W)
+        M, di, do, r = sp.M, sp.d_in, sp.d_out, sp.r
+        self.h = torch.empty(M, do, dtype=torch.bfloat16, device="cuda")
+        self.xa = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
+        self.dX = torch.empty(M, di, dtype=torch.bfloat16, device="cuda")
+        self.dA = torch.empty(r, di, dtype=torch.float32, device="cuda")
+        self.dB = torch.empty(do, r, dtype=torch.float32, device="cuda")
+        fop, bop = (L.OP_FWD_Q4, L.OP_BWD_Q4) if sp.q4 else (L.OP_FWD, L.OP_BWD)
+        self.ws_f = L.workspace(fop, M, di, do, r)
+        self.ws_b = L.workspace(bop, M, di, do, r)
+
+    def forward(self, save_xa=True):
+        xa = self.xa if save_xa else None
+        if self.q4:
+            L.lora_linear_fwd_q4(self.x, self.Wq, self.Wscale, self.A, self.B, self.h, xa, self.spec.alpha, self.ws_f)
+        else:
+            L.lora_linear_fwd(self.x, self.W, self.A, self.B, self.h, xa, self.spec.alpha, self.ws_f)
+
+    def backward(self, use_xa=True, want_dx=True):
+        xa = self.xa if use_xa else None
+        dX = self.dX if want_dx else None
+        if self.q4:
+            L.lora_linear_bwd_q4(self.dY, self.x, self.Wq, self.Wscale, self.A, self.B, xa, dX, self.dA, self.dB,
+                                 self.spec.alpha, self.ws_b)
+        else:
+            L.lora_linear_bwd(self.dY, self.x, self.W, self.A, self.B, xa, dX, self.dA, self.dB, self.spec.alpha,
+                              self.ws_b)
+
+    def check(self):
+        L.lora_linear_check(self.ws_f)
+        L.lora_linear_check(self.ws_b)
+
+    def results(self, rows=None):
+        torch.cuda.synchronize()
+        sel = (lambda t: t) if rows is None else (lambda t: t[torch.as_tensor(rows, device=t.device)])
+        return {"h": host_f64(sel(self.h)), "dX": host_f64(sel(self.dX)), "xa": host_f64(self.xa),
+                "dA": host_f64(self.dA), "dB": host_f64(self.dB)}
+
+
+def oracle_ref(inp: inputs.LayerInputs, rows=None) -> dict:
+    sp = inp.spec
+    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W=inp.W)
+    h, xa = oracle.forward(inp.x, inp.A, inp.B, sp.s, rows=rows, **wkw)
+    bw = oracle.backward(inp.dY, inp.x, inp.A, inp.B, sp.s, rows=rows, xa_=xa, **wkw)
+    return {"h": h, "xa": xa, "dX": bw["dX"], "dA": bw["dA"], "dB": bw["dB"], "g": bw["g"]}
+
+
+def assert_close(name: str, got: np.ndarray, ref: np.ndarray, tol, rms_tol=None):
+    rel, ab = tol
+    assert got.shape == ref.shape, (name, got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    err = np.abs(got - ref)
+    bound = rel * np.abs(ref).max() + ab
+    assert err.max() <= bound, (f"{name}: max|err| {err.max():.4e} > {bound:.4e} "
+                                f"at {np.unravel_index(err.argmax(), err.shape)}")
+    if rms_tol is not None and np.abs(ref).max() > 0:
+        rms = np.sqrt((err ** 2).mean()) / np.sqrt((ref ** 2).mean())
+        assert rms <= rms_tol, f"{name}: rms rel err {rms:.3e} > {rms_tol:.1e}"
+
+
+def compare_all(got: dict, ref: dict, s: float, check_xa=True):
+    assert_close("h", got["h"], ref["h"], TOL_HX, RMS_HX)
+    assert_close("dX", got["dX"], ref["dX"], TOL_HX, RMS_HX)
+    assert_close("dA", got["dA"], ref["dA"], TOL_AB, RMS_AB)
+    assert_close("dB", got["dB"], ref["dB"], TOL_AB, RMS_AB)
+    if check_xa:
+        # xa_save holds bf16(s . x.A^T): one bf16 rounding of the exact product.
+        assert_close("xa_save", got["xa"], s * ref["xa"], (2 ** -8, 1e-6), RMS_HX)
+
+
+def sample_rows(M: int, n_random: int = 24, seed: int = 0) -> np.ndarray:
+    """Rows that cover the first and last tile, tile edges and a random spread."""
+    fixed = {0, 1, 63, 64, 127, 128, M // 2, M - 129, M - 128, M - 2, M - 1}
+    rng = np.random.default_rng(seed)
+    rnd = set(rng.integers(0, M, size=n_random).tolist())
+    return np.array(sorted(v for v in fixed | rnd if 0 <= v < M), dtype=np.int64)

@@ -1,0 +1,68 @@
+"""The C ABI on the CPU: the library loads, exports every declared symbol, sizes
+workspaces, and rejects bad arguments before touching a device."""
+import ctypes
+
+import pytest
+
+from rank_linear_lora_b200 import build as B
+from rank_linear_lora_b200 import lora_linear as L
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = L.declared_functions()
+    expected = {"lora_linear_workspace_size", "lora_linear_fwd", "lora_linear_bwd", "lora_linear_fwd_q4",
+                "lora_linear_bwd_q4", "lora_linear_check", "lora_status_string", "lora_linear_launch_count",
+                "lora_linear_timing_enable", "lora_linear_timing_read"}
+    assert expected <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        s = L.lora_status_string(code)
+        assert isinstance(s, str) and s
+    assert L.lora_status_string(99) == "unknown status"
+
+
+def test_workspace_sizes(lib):
+    for op in (L.OP_FWD, L.OP_BWD, L.OP_FWD_Q4, L.OP_BWD_Q4):
+        assert L.lora_linear_workspace_size(op, 4096, 8192, 28672, 16) > 0
+    assert L.lora_linear_workspace_size(L.OP_BWD, 4096, 4096, 4096, 8) > L.lora_linear_workspace_size(
+        L.OP_FWD, 4096, 4096, 4096, 8)
+    # invalid sizes -> 0
+    assert L.lora_linear_workspace_size(L.OP_FWD, 0, 256, 256, 8) == 0
+    assert L.lora_linear_workspace_size(L.OP_FWD, 64, 250, 256, 8) == 0
+    assert L.lora_linear_workspace_size(L.OP_FWD, 64, 256, 256, 12) == 0
+    assert L.lora_linear_workspace_size(L.OP_FWD, 64, 256, 256, 264) == 0
+    assert L.lora_linear_workspace_size(L.OP_FWD_Q4, 64, 96, 256, 8) == 0
+    assert L.lora_linear_workspace_size(7, 64, 256, 256, 8) == 0
+
+
+def _fwd(lib, x=0x1000, W=0x2000, A=0x3000, B_=0x4000, h=0x5000, xa=None, M=64, di=256, do=256, r=8,
+         alpha=16.0, ws=0x10000, nws=1 << 30):
+    P = ctypes.c_void_p
+    return lib.lora_linear_fwd(P(x), P(W), P(A), P(B_), P(h), P(xa), M, di, do, r, alpha, P(ws), nws, None)
+
+
+def test_validation_before_any_device_work(lib):
+    """Every case below fails validation, so no pointer is ever dereferenced."""
+    assert _fwd(lib, x=None) == 1
+    assert _fwd(lib, h=None) == 1
+    assert _fwd(lib, M=0) == 1
+    assert _fwd(lib, di=250) == 1
+    assert _fwd(lib, r=0) == 1
+    assert _fwd(lib, r=12) == 1
+    assert _fwd(lib, alpha=float("nan")) == 1
+    assert _fwd(lib, x=0x1008) == 2
+    assert _fwd(lib, xa=0x6004) == 2
+    P = ctypes.c_void_p
+    st = lib.lora_linear_bwd(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), None, None, None, P(0x7000),
+                             64, 256, 256, 8, 16.0, P(0x10000), 1 << 30, None)
+    assert st == 1  # dA is required

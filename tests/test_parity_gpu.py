@@ -1,0 +1,189 @@
+"""GPU path against the fp64 oracle, element by element, through the C ABI.
+
+Small and ragged shapes compare every output element; the full-size workloads
+compare every element of dA and dB and sampled token rows of h and dX (rows the
+oracle computes one by one), in the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+from lora_cases import (DeviceLayer, assert_close, compare_all, oracle_ref, sample_rows, TOL_AB, TOL_HX, RMS_AB,
+                        RMS_HX)
+from rank_linear_lora_b200 import inputs
+from rank_linear_lora_b200 import lora_linear as L
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_full(spec, **mk):
+    inp = inputs.make_inputs(spec, **mk)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.backward()
+    dl.check()
+    return inp, dl
+
+
+def test_config0_tiny_full():
+    spec = inputs.workload(0).layers[0]
+    inp, dl = _run_full(spec)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+RAGGED = [
+    # (M, d_in, d_out, r): token tails, K tails (d % 64 != 0), N tails, rank tails (r % 16 != 0)
+    (200, 328, 200, 8),
+    (129, 64, 72, 16),
+    (1, 8, 8, 8),
+    (300, 520, 264, 24),
+    (77, 256, 512, 64),
+    (160, 192, 128, 128),
+    (130, 136, 520, 256),
+    (513, 1032, 776, 40),
+]
+
+
+@pytest.mark.parametrize("shape", RAGGED, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_ragged_full(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("ragged", M, di, do, r, alpha=2.0 * r, seed=0xBEEF + M)
+    inp, dl = _run_full(spec)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+def test_lora_dominant():
+    """B drawn 50x larger than the workloads' init so the rank-r term dominates h and dX:
+    any dropped or mis-indexed piece of the K tail shows up far outside tolerance."""
+    spec = inputs.LayerSpec("dominant", 192, 320, 448, 24, alpha=48.0, seed=77)
+    inp = inputs.make_inputs(spec)
+    inp.B = inputs.to_bf16_bits(inputs.bf16_bits_to_f32(inp.B).astype(np.float64) * 50.0)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.backward()
+    dl.check()
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+def test_zero_B_gives_zero_dA_exactly():
+    spec = inputs.workload(0).layers[0].with_(M=200)
+    inp, dl = _run_full(spec, zero_B=True)
+    got = dl.results()
+    assert np.all(got["dA"] == 0.0)
+    compare_all(got, oracle_ref(inp), spec.s)
+
+
+def test_zero_A_gives_zero_dB_exactly():
+    spec = inputs.workload(0).layers[0].with_(M=136)
+    inp, dl = _run_full(spec, zero_A=True)
+    got = dl.results()
+    assert np.all(got["dB"] == 0.0) and np.all(got["xa"] == 0.0)
+    compare_all(got, oracle_ref(inp), spec.s)
+
+
+def test_recompute_xa_and_skip_dx():
+    """Backward without the saved s.xa recomputes it (same dB); dX = NULL skips dX only."""
+    spec = inputs.LayerSpec("opt", 264, 384, 320, 16, alpha=32.0, seed=5)
+    inp = inputs.make_inputs(spec)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.backward(use_xa=True)
+    torch.cuda.synchronize()
+    dA1, dB1, dX1 = dl.dA.clone(), dl.dB.clone(), dl.dX.clone()
+    dl.dA.fill_(float("nan"))
+    dl.dB.fill_(float("nan"))
+    dl.dX.fill_(7.0)
+    dl.backward(use_xa=False, want_dx=False)
+    dl.check()
+    assert torch.equal(dl.dA, dA1) and torch.equal(dl.dB, dB1)
+    assert torch.all(dl.dX == 7.0)
+    ref = oracle_ref(inp)
+    assert_close("dX", dX1.double().cpu().numpy(), ref["dX"], TOL_HX, RMS_HX)
+
+
+def test_deterministic():
+    spec = inputs.LayerSpec("det", 384, 512, 384, 8, alpha=16.0, seed=9)
+    dl = DeviceLayer(inputs.make_inputs(spec))
+    outs = []
+    for _ in range(2):
+        dl.forward()
+        dl.backward()
+        torch.cuda.synchronize()
+        outs.append([t.clone() for t in (dl.h, dl.xa, dl.dX, dl.dA, dl.dB)])
+    dl.check()
+    for a, b in zip(*outs):
+        assert torch.equal(a.view(torch.uint8) if a.dtype == torch.bfloat16 else a,
+                           b.view(torch.uint8) if b.dtype == torch.bfloat16 else b)
+
+
+def test_outputs_stay_in_bounds():
+    """Guard bands after every output: the kernels write exactly the declared extents."""
+    spec = inputs.LayerSpec("guard", 200, 328, 200, 8, alpha=16.0, seed=11)
+    inp = inputs.make_inputs(spec)
+    dl = DeviceLayer(inp)
+    M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
+    pad = 4096
+    hb = torch.full((M * do + pad,), 3.0, dtype=torch.bfloat16, device="cuda")
+    xb = torch.full((M * r + pad,), 3.0, dtype=torch.bfloat16, device="cuda")
+    dxb = torch.full((M * di + pad,), 3.0, dtype=torch.bfloat16, device="cuda")
+    dab = torch.full((r * di + pad,), 3.0, dtype=torch.float32, device="cuda")
+    dbb = torch.full((do * r + pad,), 3.0, dtype=torch.float32, device="cuda")
+    dl.h, dl.xa, dl.dX = hb[:M * do].view(M, do), xb[:M * r].view(M, r), dxb[:M * di].view(M, di)
+    dl.dA, dl.dB = dab[:r * di].view(r, di), dbb[:do * r].view(do, r)
+    dl.forward()
+    dl.backward()
+    dl.check()
+    for buf, n in ((hb, M * do), (xb, M * r), (dxb, M * di), (dab, r * di), (dbb, do * r)):
+        assert torch.all(buf[n:] == 3.0)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+def test_status_codes_on_device():
+    spec = inputs.workload(0).layers[0]
+    dl = DeviceLayer(inputs.make_inputs(spec))
+    small = dl.ws_f[: dl.ws_f.numel() // 2]
+    with pytest.raises(L.LoraError) as e:
+        L.lora_linear_fwd(dl.x, dl.W, dl.A, dl.B, dl.h, dl.xa, spec.alpha, small)
+    assert e.value.status == 4
+    with pytest.raises(L.LoraError) as e:
+        L.lora_linear_fwd(dl.x, dl.W, dl.A, dl.B, dl.h, dl.xa, spec.alpha, dl.ws_f[16:])
+    assert e.value.status == 2
+    with pytest.raises(L.LoraError) as e:
+        L.lora_linear_fwd(dl.x, dl.W, dl.A, dl.B, dl.h, dl.xa, float("inf"), dl.ws_f)
+    assert e.value.status == 1
+    dl.check()
+
+
+def test_timing_hooks_count_launches():
+    spec = inputs.workload(0).layers[0]
+    dl = DeviceLayer(inputs.make_inputs(spec))
+    L.lora_linear_timing_read()
+    n0 = L.lora_linear_launch_count()
+    L.lora_linear_timing_enable(True)
+    try:
+        dl.forward()
+        dl.backward()
+        rec = L.lora_linear_timing_read()
+    finally:
+        L.lora_linear_timing_enable(False)
+    assert L.lora_linear_launch_count() - n0 == 6
+    assert all(rec[k][1] == 1 and rec[k][0] > 0 for k in L.KERNEL_KINDS)
+
+
+# ------------------------------------------------------------------ full sizes
+FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0)]
+
+
+@pytest.mark.parametrize("cfg", FULL, ids=lambda c: f"cfg{c[0]}_r{c[1]}_layer{c[2]}")
+def test_full_size_sampled(cfg):
+    idx, r, layer = cfg
+    spec = inputs.workload(idx, r=r).layers[layer]
+    inp = inputs.make_inputs(spec)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.backward()
+    dl.check()
+    rows = sample_rows(spec.M, seed=idx * 10 + layer)
+    got = dl.results(rows=rows)
+    ref = oracle_ref(inp, rows=rows)
+    compare_all(got, ref, spec.s)
