@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the fused LoRA linear layer (forward + backward) on B200.
+
+One step = lora_linear_fwd + lora_linear_bwd of one layer over one batch of
+synthetic tokens (every row of the hot path: s.xa, the forward main GEMM, s.g,
+the dX GEMM, dB, dA).  Default workload: the attention-projection layer,
+M = 4096 tokens (2 x 2048), d_in = d_out = 4096, r = 8, alpha = 32.
+
+Timing: W untimed warm-up steps; then, behind a GPU sleep that lets the host
+enqueue all K steps ahead, K back-to-back steps bracketed by CUDA events on the
+launch stream (barrier + synchronize on both sides; max over ranks).  Steps rotate
+over three independent input sets (3 x 160 MiB > the 126 MB L2), so no step finds
+its operands left in L2 by the previous one.
+
+Multi-GPU (torchrun): data parallel over tokens, weak scaling (each rank its own
+M tokens); after the backward the packed [dA | dB] fp32 gradient is summed over
+ranks with one NCCL all-reduce inside the timed region.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (a bounded
+token sample per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused LoRA fwd+bwd TFLOP/s & tokens/s per layer; % of BF16 tensor roofline"
+UNIT = "TFLOP/s"
+N_SETS = 3
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--config", type=int, default=1, help="workload index (1: attention projection)")
+    p.add_argument("--rank-r", type=int, default=None, help="rank for the rank-sweep workload")
+    p.add_argument("--layer", type=int, default=0, help="layer of a multi-layer workload")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+def algorithmic_bytes(spec) -> float:
+    """One read of every operand and one write of every output per fwd + bwd call."""
+    M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
+    w = do * di // 2 + do * (di // 64) * 2 if spec.q4 else do * di * 2
+    fwd = M * di * 2 + w + r * di * 2 + do * r * 2 + M * do * 2 + M * r * 2
+    bwd = M * do * 2 + M * di * 2 + w + r * di * 2 + do * r * 2 + M * r * 2 + M * di * 2 + r * di * 4 + do * r * 4
+    return float(fwd + bwd)
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("ptx.cuh", "tc_gemm.cuh", "lora_linear.cu"):
+        with open(os.path.join(ROOT, "rank_linear_lora_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kind: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    d = json.load(open(path))
+    if d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    e = d.get("kernels", {}).get(kind)
+    if not e or e.get("workload") != workload:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """NVML clocks and throttle reasons sampled in a thread while the timed region runs."""
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period, self.samples, self._stop = index, period_s, [], threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # pragma: no cover - no NVML
+            self.max_mhz = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"], "samples": 0}
+        nv = self.nv
+        names = {
+            "gpu_idle": getattr(nv, "nvmlClocksEventReasonGpuIdle", 0x1),
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        mhz = sorted(s[0] for s in self.samples)
+        seen = sorted({n for _, r in self.samples for n, bit in names.items() if r & bit and n != "gpu_idle"})
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": seen,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------- reference arm
+def run_reference(args, spec, workload_name, rank, world):
+    import numpy as np
+
+    import oracle
+    from rank_linear_lora_b200 import inputs
+
+    if rank != 0:
+        return None
+    inp = inputs.make_inputs(spec)
+    per_token = spec.flops / spec.M
+    # calibrate, then size the per-step token sample so the whole run takes ~2 minutes
+    t0 = time.perf_counter()
+    _oracle_step(oracle, inp, spec, 0, 8)
+    rate = 8 * per_token / max(1e-6, time.perf_counter() - t0)
+    budget = min(20.0, 120.0 / max(1, args.steps + args.warmup))
+    tokens = int(max(8, min(spec.M, budget * rate / per_token)))
+    for i in range(args.warmup):
+        _oracle_step(oracle, inp, spec, i * tokens, tokens)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        _oracle_step(oracle, inp, spec, (args.warmup + i) * tokens, tokens)
+    dt = time.perf_counter() - t0
+    flops = args.steps * tokens * per_token
+    value = flops / dt / 1e12
+    sample = f"{tokens} of the {spec.M} tokens per step (full d_in, d_out, r), fp64"
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_name, "M": spec.M, "d_in": spec.d_in,
+                                         "d_out": spec.d_out, "r": spec.r, "alpha": spec.alpha,
+                                         "parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "tokens_per_s": args.steps * tokens / dt,
+    }
+
+
+def _oracle_step(oracle, inp, spec, start, tokens):
+    M = spec.M
+    rows = [(start + i) % M for i in range(tokens)]
+    x, dY = inp.x[rows], inp.dY[rows]
+    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if spec.q4 else dict(W=inp.W)
+    h, xa = oracle.forward(x, inp.A, inp.B, spec.s, **wkw)
+    oracle.backward(dY, x, inp.A, inp.B, spec.s, xa_=xa, **wkw)
+
+
+def cpu_baseline(spec, seconds=12.0):
+    """The oracle as it stands on this host's cores over a bounded token sample."""
+    import oracle
+    from rank_linear_lora_b200 import inputs
+
+    inp = inputs.make_inputs(spec)
+    per_token = spec.flops / spec.M
+    t0 = time.perf_counter()
+    _oracle_step(oracle, inp, spec, 0, 8)
+    rate = 8 * per_token / max(1e-6, time.perf_counter() - t0)
+    tokens = int(max(8, min(spec.M, seconds * rate / per_token)))
+    t0 = time.perf_counter()
+    _oracle_step(oracle, inp, spec, 0, tokens)
+    dt = time.perf_counter() - t0
+    return {"value": tokens * per_token / dt / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"fwd+bwd of {tokens} of the {spec.M} tokens (full d_in={spec.d_in}, d_out={spec.d_out}, "
+                      f"r={spec.r}) in fp64, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------- our arm
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from rank_linear_lora_b200 import inputs
+
+    wl = inputs.workload(args.config, r=args.rank_r)
+    spec = wl.layers[args.layer]
+    workload_name = f"{wl.name} / {spec.name}"
+
+    if args.impl == "reference":
+        out = run_reference(args, spec, workload_name, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from rank_linear_lora_b200 import lora_linear as L
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    peaks = load_peaks()
+    M, di, do, r, alpha = spec.M, spec.d_in, spec.d_out, spec.r, spec.alpha
+
+    def d16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    # Input sets: set k uses the generator's streams of seed + 1000 * k, shifted by rank.
+    sets = []
+    host_inputs = None
+    for k in range(N_SETS):
+        sp = spec.with_(seed=spec.seed + 1000 * k + 7919 * rank)
+        inp = inputs.make_inputs(sp)
+        if k == 0:
+            host_inputs = inp
+        s = {"x": d16(inp.x), "A": d16(inp.A), "B": d16(inp.B), "dY": d16(inp.dY)}
+        if spec.q4:
+            s["Wq"] = torch.from_numpy(inp.Wq).to(dev)
+            s["Wscale"] = d16(inp.Wscale)
+        else:
+            s["W"] = d16(inp.W)
+        s["h"] = torch.empty(M, do, dtype=torch.bfloat16, device=dev)
+        s["xa"] = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+        s["dX"] = torch.empty(M, di, dtype=torch.bfloat16, device=dev)
+        s["grad"] = torch.empty(r * di + do * r, dtype=torch.float32, device=dev)  # packed [dA | dB]
+        s["dA"] = s["grad"][: r * di].view(r, di)
+        s["dB"] = s["grad"][r * di:].view(do, r)
+        fop, bop = (L.OP_FWD_Q4, L.OP_BWD_Q4) if spec.q4 else (L.OP_FWD, L.OP_BWD)
+        s["wsf"] = L.workspace(fop, M, di, do, r, device=dev)
+        s["wsb"] = L.workspace(bop, M, di, do, r, device=dev)
+        sets.append(s)
+
+    def step(s):
+        if spec.q4:
+            L.lora_linear_fwd_q4(s["x"], s["Wq"], s["Wscale"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
+            L.lora_linear_bwd_q4(s["dY"], s["x"], s["Wq"], s["Wscale"], s["A"], s["B"], s["xa"], s["dX"], s["dA"],
+                                 s["dB"], alpha, s["wsb"])
+        else:
+            L.lora_linear_fwd(s["x"], s["W"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
+            L.lora_linear_bwd(s["dY"], s["x"], s["W"], s["A"], s["B"], s["xa"], s["dX"], s["dA"], s["dB"], alpha,
+                              s["wsb"])
+        if world > 1:
+            dist.all_reduce(s["grad"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for i in range(args.warmup):
+        step(sets[i % N_SETS])
+    torch.cuda.synchronize()
+    for s in sets:
+        L.lora_linear_check(s["wsf"])
+        L.lora_linear_check(s["wsb"])
+
+    stream = torch.cuda.current_stream()
+    host_ms = [0.0]
+
+    def timed_region(n_steps, timing_hooks=False):
+        barrier()
+        torch.cuda.synchronize()
+        if timing_hooks:
+            L.lora_linear_timing_read()
+            L.lora_linear_timing_enable(True)
+        torch.cuda._sleep(int(5e6 + 2e5 * n_steps))  # let the host enqueue every step ahead
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        n0 = L.lora_linear_launch_count()
+        th = time.perf_counter()
+        e0.record(stream)
+        for i in range(n_steps):
+            step(sets[i % N_SETS])
+        e1.record(stream)
+        host_ms[0] = (time.perf_counter() - th) * 1e3
+        n1 = L.lora_linear_launch_count()
+        torch.cuda.synchronize()
+        barrier()
+        rec = None
+        if timing_hooks:
+            L.lora_linear_timing_enable(False)
+            rec = L.lora_linear_timing_read()
+        return e0.elapsed_time(e1), n1 - n0, rec
+
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    with sampler:
+        ms, launches, _ = timed_region(args.steps)
+    clocks = sampler.summary()
+    host_enqueue_ms = host_ms[0]
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_max = float(t.item())
+
+    # Per-kernel device times (separate pass, event pairs around every launch).
+    _, _, rec = timed_region(min(args.steps, 100), timing_hooks=True)
+    for s in sets:
+        L.lora_linear_check(s["wsf"])
+        L.lora_linear_check(s["wsb"])
+
+    flops_step = spec.flops
+    total_flops = flops_step * args.steps * world
+    value = total_flops / (ms_max * 1e-3) / 1e12
+    ms_per_step = ms_max / args.steps
+    tokens_per_s = M * world * args.steps / (ms_max * 1e-3)
+
+    # roofline of the dominant kernel
+    kern_flops = {"fwd_main": 2.0 * M * do * (di + r), "dx_main": 2.0 * M * di * (do + r)}
+    dom = max(("fwd_main", "dx_main"), key=lambda k: rec[k][0])
+    dom_ms = rec[dom][0] / max(1, rec[dom][1])
+    achieved = kern_flops[dom] / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_src": f"{peaks['src']} bf16 burst (MEASURED_PEAKS.json)",
+                "traffic": stored_traffic(dom, workload_name)}
+    t_roof = max(flops_step / (peak * 1e12), algorithmic_bytes(spec) / (peaks["hbm_gbs"] * 1e9))
+    step_roof = {"t_roof_us": t_roof * 1e6, "t_meas_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
+                 "definition": "max(FLOP / bf16 peak, algorithmic bytes / HBM peak) over the measured step time"}
+    kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs from pinned
+    # memory, fwd + bwd, D2H of the step's outputs (W stays resident: frozen model state).
+    e2e = None
+    if not args.no_e2e:
+        s = sets[0]
+        names_in = ["x", "dY", "A", "B"]
+        names_out = ["h", "dX", "dA", "dB"]
+        hin = {k: torch.empty_like(s[k], device="cpu").pin_memory() for k in names_in}
+        for k in names_in:
+            hin[k].copy_(s[k])
+        hout = {k: torch.empty_like(s[k], device="cpu").pin_memory() for k in names_out}
+        n_e2e = max(5, min(args.steps, 50))
+
+        def e2e_step():
+            for k in names_in:
+                s[k].copy_(hin[k], non_blocking=True)
+            step(s)
+            for k in names_out:
+                hout[k].copy_(s[k], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(2e6))
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item())
+        e2e = {"value": flops_step * n_e2e * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(sum(hin[k].numel() * hin[k].element_size() for k in names_in)),
+               "d2h_bytes_per_step": int(sum(hout[k].numel() * hout[k].element_size() for k in names_out)),
+               "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e,
+               "note": "pinned host buffers; frozen W resident on the device"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_name, "M": M, "d_in": di, "d_out": do, "r": r, "alpha": alpha,
+                       "q4": spec.q4, "tokens_per_step": M * world,
+                       "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
+                       "parallelism": f"dp{world}"},
+            "tokens_per_s": tokens_per_s,
+            "roofline": roofline,
+            "roofline_step": step_roof,
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "host_enqueue_ms": host_enqueue_ms,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
