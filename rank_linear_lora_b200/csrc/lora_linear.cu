@@ -127,6 +127,10 @@ cudaEvent_t pool_event() {
     return e;
 }
 
+// Optional device trace buffer: kind k writes its CTAs' records at k * trace_stride words.
+std::atomic<unsigned long long *> g_trace{nullptr};
+std::atomic<size_t> g_trace_stride{0};
+
 // ------------------------------------------------------------------ launch helpers
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
 cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
@@ -148,7 +152,15 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
         eb = pool_event();
         if (ea) cudaEventRecord(ea, st);
     }
-    kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(args);
+    unsigned long long *tr = g_trace.load();
+    const size_t stride = g_trace_stride.load();
+    if (tr && static_cast<size_t>(grid) * TRACE_WORDS <= stride) {
+        GemmArgs a2 = args;
+        a2.trace = tr + static_cast<size_t>(kind) * stride;
+        kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(a2);
+    } else {
+        kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(args);
+    }
     cudaError_t e = cudaGetLastError();
     g_launches.fetch_add(1);
     if (timed && ea && eb) {
@@ -179,24 +191,19 @@ struct Split {
     int splits = 1, per = 1;
 };
 
-// Splits of K (in 64-wide blocks) for a skinny kernel with `mt` output tiles: pick
-// the count that minimises (waves of tiles) x (blocks per split) on `sms` SMs.
+// Splits of K (in 64-wide blocks) for a skinny kernel with `mt` output tiles.  Each
+// CTA should stream one long contiguous K range (the per-tile epilogue and split-K
+// fixup cost about as much as a few blocks of loads), so the split count is the
+// largest that still gives every SM at most one tile, keeping >= 4 blocks per split.
 Split choose_split(int64_t mt, int64_t kb, int sms) {
-    Split best;
-    int64_t best_cost = INT64_MAX;
-    const int64_t smax = std::min<int64_t>(kb, 64);
-    for (int64_t s = 1; s <= smax; ++s) {
-        const int64_t per = cdiv(kb, s);
-        const int64_t eff = cdiv(kb, per);
-        const int64_t tiles = mt * eff;
-        const int64_t cost = cdiv(tiles, sms) * per;
-        if (cost < best_cost) {
-            best_cost = cost;
-            best.splits = static_cast<int>(eff);
-            best.per = static_cast<int>(per);
-        }
-    }
-    return best;
+    Split sp;
+    int64_t s = std::max<int64_t>(1, sms / std::max<int64_t>(1, mt));
+    s = std::min<int64_t>(s, std::max<int64_t>(1, kb / 4));
+    s = std::min<int64_t>(s, 64);
+    const int64_t per = cdiv(kb, s);
+    sp.per = static_cast<int>(per);
+    sp.splits = static_cast<int>(cdiv(kb, per));
+    return sp;
 }
 
 constexpr int PLAN_SMS = 148;  // sizes the workspace for up to this many SMs' worth of splits
@@ -532,6 +539,18 @@ const char *lora_status_string(lora_status_t status) {
 }
 
 int64_t lora_linear_launch_count(void) { return g_launches.load(); }
+
+lora_status_t lora_linear_trace_enable(void *device_buffer, size_t bytes) {
+    if (!device_buffer || bytes < LORA_K_COUNT * 8) {
+        g_trace.store(nullptr);
+        g_trace_stride.store(0);
+        return LORA_OK;
+    }
+    if (reinterpret_cast<uintptr_t>(device_buffer) & 7u) return LORA_ERR_MISALIGNED;
+    g_trace_stride.store(bytes / 8 / LORA_K_COUNT);
+    g_trace.store(static_cast<unsigned long long *>(device_buffer));
+    return LORA_OK;
+}
 
 lora_status_t lora_linear_timing_enable(int enable) {
     g_timing.store(enable ? 1 : 0);

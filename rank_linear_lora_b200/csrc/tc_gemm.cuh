@@ -72,6 +72,14 @@ struct GemmArgs {
     void *out;               // EPI_SPLITK output
     int64_t out_ld;          // OUT_F32_COLS: row stride of the transposed output
     int *err;                // device error word
+    unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
+};
+
+// Trace record of one CTA (globaltimer ns unless noted).
+enum TraceField {
+    TR_ENTRY = 0, TR_SETUP = 1, TR_PROD_END = 2, TR_MMA_END = 3, TR_EPI_END = 4, TR_EXIT = 5,
+    TR_SMID = 6, TR_TILES = 7, TR_TILE_DONE0 = 8,  // epilogue completion of the first 8 tiles
+    TRACE_WORDS = 16
 };
 
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
@@ -154,6 +162,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
+    unsigned long long *trace = p.trace ? p.trace + static_cast<size_t>(blockIdx.x) * TRACE_WORDS : nullptr;
+    if (trace && threadIdx.x == 0) {
+        uint32_t smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        trace[TR_ENTRY] = globaltimer_ns();
+        trace[TR_SMID] = smid;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -177,6 +192,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    if (trace && threadIdx.x == 0) trace[TR_SETUP] = globaltimer_ns();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -240,6 +256,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                     wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
                                  DERR_WAIT_DRAIN);
                 }
+            if (trace) trace[TR_PROD_END] = globaltimer_ns();
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
@@ -300,6 +317,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             tc_commit(smem_u32(drain_bar));
             volatile int never = 0;
             wait_bounded(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
+            if (trace) {
+                trace[TR_MMA_END] = globaltimer_ns();
+                trace[TR_TILES] = static_cast<unsigned long long>(it);
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -392,15 +413,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 if (last) {
                     __threadfence();
                     if (grow < p.rows_valid) {
+                        const float *prow = p.part + grow * p.n_valid;
+                        const int64_t split_stride = rows_total * p.n_valid;
                         for (int c0 = 0; c0 < p.n_valid; c0 += 4) {
                             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                            for (int s = 0; s < p.splits; ++s) {
-                                const float4 v = __ldcg(reinterpret_cast<const float4 *>(
-                                    p.part + ((static_cast<int64_t>(s) * rows_total + grow) * p.n_valid + c0)));
-                                acc.x += v.x;
-                                acc.y += v.y;
-                                acc.z += v.z;
-                                acc.w += v.w;
+                            // Eight splits' loads in flight at a time, summed in split order.
+                            for (int s0 = 0; s0 < p.splits; s0 += 8) {
+                                float4 v[8];
+#pragma unroll
+                                for (int u = 0; u < 8; ++u)
+                                    v[u] = (s0 + u < p.splits)
+                                               ? __ldcg(reinterpret_cast<const float4 *>(
+                                                     prow + (s0 + u) * split_stride + c0))
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                                for (int u = 0; u < 8; ++u) {
+                                    if (s0 + u < p.splits) {
+                                        acc.x += v[u].x;
+                                        acc.y += v[u].y;
+                                        acc.z += v[u].z;
+                                        acc.w += v[u].w;
+                                    }
+                                }
                             }
                             acc.x *= p.out_scale;
                             acc.y *= p.out_scale;
@@ -425,7 +459,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                     if (epi_tid == 0) p.counters[ctr] = 0;  // ready for the next call
                 }
             }
+            if (trace && epi_tid == 0 && it < 8) trace[TR_TILE_DONE0 + it] = globaltimer_ns();
         }
+        if (trace && epi_tid == 0) trace[TR_EPI_END] = globaltimer_ns();
         if constexpr (EPI == EPI_STORE) {
             if (lane == 0) bulk_wait_group<0>();
         }
@@ -439,6 +475,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
+    if (trace && threadIdx.x == 0) trace[TR_EXIT] = globaltimer_ns();
 }
 
 }  // namespace lora

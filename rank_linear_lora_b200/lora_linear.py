@@ -60,6 +60,8 @@ def load_library():
     lib.lora_linear_timing_enable.restype = I
     lib.lora_linear_timing_read.argtypes = [P, P, I]
     lib.lora_linear_timing_read.restype = I
+    lib.lora_linear_trace_enable.argtypes = [P, SZ]
+    lib.lora_linear_trace_enable.restype = I
     _lib = lib
     return lib
 
@@ -204,3 +206,16 @@ def lora_linear_timing_read():
     cnt = (ctypes.c_int64 * n)()
     _check(load_library().lora_linear_timing_read(ms, cnt, n), "lora_linear_timing_read")
     return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
+
+
+TRACE_WORDS = 16
+TRACE_FIELDS = ["entry", "setup", "prod_end", "mma_end", "epi_end", "exit", "smid", "tiles"]
+
+
+def lora_linear_trace_enable(buf):
+    """Trace into a CUDA int64 tensor (None switches tracing off)."""
+    if buf is None:
+        _check(load_library().lora_linear_trace_enable(None, 0), "lora_linear_trace_enable")
+    else:
+        _check(load_library().lora_linear_trace_enable(_ptr(buf), buf.numel() * buf.element_size()),
+               "lora_linear_trace_enable")
