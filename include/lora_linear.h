@@ -35,7 +35,13 @@
  *     d_in and d_out multiples of 8 (>= 8); 1 <= r <= 256 with r % 8 == 0; alpha
  *     finite; for *_q4 also d_in % 64 == 0.
  *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
- *     aligned, and must not be used by two calls that may run at the same time.
+ *     aligned, be zero-filled before its first use, and must not be used by two calls
+ *     that may run at the same time.  Every call that completes leaves the workspace's
+ *     arrival counters at zero again, so a workspace is zeroed once, not per call
+ *     (after LORA_ERR_TIMEOUT the caller zero-fills it again).
+ *   - Consecutive kernels are launched with programmatic dependent launch: each waits
+ *     for its predecessor in the stream before touching global memory, so stream
+ *     order is preserved; only launch latency and set-up overlap.
  *   - The device must be compute capability 10.0 (B200); otherwise
  *     LORA_ERR_UNSUPPORTED is returned and nothing runs.
  *   - Device-side waits are bounded.  A wait that runs out sets an error word in the

@@ -19,6 +19,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -131,6 +132,16 @@ cudaEvent_t pool_event() {
 std::atomic<unsigned long long *> g_trace{nullptr};
 std::atomic<size_t> g_trace_stride{0};
 
+// Programmatic dependent launch between consecutive kernels (LORA_LINEAR_PDL=0 turns
+// it off, for measurement).
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char *v = std::getenv("LORA_LINEAR_PDL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
+
 // ------------------------------------------------------------------ launch helpers
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
 cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
@@ -152,16 +163,23 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
         eb = pool_event();
         if (ea) cudaEventRecord(ea, st);
     }
+    GemmArgs a2 = args;
     unsigned long long *tr = g_trace.load();
     const size_t stride = g_trace_stride.load();
-    if (tr && static_cast<size_t>(grid) * TRACE_WORDS <= stride) {
-        GemmArgs a2 = args;
-        a2.trace = tr + static_cast<size_t>(kind) * stride;
-        kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(a2);
-    } else {
-        kern<<<grid, NUM_THREADS, Cfg::SMEM_BYTES, st>>>(args);
-    }
-    cudaError_t e = cudaGetLastError();
+    if (tr && static_cast<size_t>(grid) * TRACE_WORDS <= stride) a2.trace = tr + static_cast<size_t>(kind) * stride;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a2);
+    if (e == cudaSuccess) e = cudaGetLastError();
     g_launches.fetch_add(1);
     if (timed && ea && eb) {
         cudaEventRecord(eb, st);
@@ -206,11 +224,37 @@ Split choose_split(int64_t mt, int64_t kb, int sms) {
     return sp;
 }
 
-constexpr int PLAN_SMS = 148;  // sizes the workspace for up to this many SMs' worth of splits
+constexpr int PLAN_SMS = 148;  // SMs a launch uses at most (sizes splits and the workspace)
+
+// Main-GEMM schedule: whole tiles in waves over G CTAs; a partial last wave of R
+// tiles is cut into `pieces` K ranges so every CTA gets work (stream-K on the tail).
+struct MainSched {
+    int tiles = 0, dp_tiles = 0, dp_waves = 0, sk_tiles = 0, sk_pieces = 0;
+};
+
+MainSched main_sched(int64_t M, int64_t N, int64_t K0, int r, int G) {
+    MainSched s;
+    const int64_t T = cdiv(M, BM) * cdiv(N, MAIN_BN);
+    const int64_t kbt = cdiv(K0, BK) + cdiv(r, BK);
+    s.tiles = static_cast<int>(T);
+    const int64_t W = T / G, R = T % G;
+    int64_t pieces = (R > 0) ? std::min<int64_t>({G / R, 4, kbt / 8}) : 0;
+    if (W >= 1 && R > 0 && pieces >= 2) {
+        s.dp_tiles = static_cast<int>(W * G);
+        s.dp_waves = static_cast<int>(W);
+        s.sk_tiles = static_cast<int>(R);
+        s.sk_pieces = static_cast<int>(pieces);
+    } else {
+        s.dp_tiles = static_cast<int>(T);
+        s.dp_waves = static_cast<int>(cdiv(T, G));
+    }
+    return s;
+}
 
 struct Plan {
-    size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0, total = 0;
-    int64_t n_ctr = 0;
+    size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0;
+    size_t part_sk = 0, total = 0;
+    int64_t n_ctr = 0, sk_slots = 0;
     Split s_xa, s_g, s_db, s_da;
 };
 
@@ -221,12 +265,18 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     pl->s_g = choose_split(mt_tok, cdiv(d_out, BK), sms);
     pl->s_db = choose_split(mt_out, cdiv(M, BK), sms);
     pl->s_da = choose_split(mt_in, cdiv(M, BK), sms);
+    // Stream-K slots of the main GEMM: pieces x split tiles <= CTAs <= min(tiles, PLAN_SMS)
+    // whatever the device's SM count, so reserve one 128 x 256 fp32 slot per CTA.
+    const int64_t main_tiles = bwd ? cdiv(M, BM) * cdiv(d_in, MAIN_BN) : cdiv(M, BM) * cdiv(d_out, MAIN_BN);
+    pl->sk_slots = std::min<int64_t>(main_tiles, PLAN_SMS);
     size_t off = 0;
     pl->err = off;
     off += 256;
     pl->ctr = off;
-    pl->n_ctr = mt_tok * 2 + mt_in + mt_out;
+    pl->n_ctr = mt_tok * 2 + mt_in + mt_out + PLAN_SMS;  // skinny tiles, then stream-K tiles
     off = align256(off + pl->n_ctr * sizeof(int));
+    pl->part_sk = off;
+    off = align256(off + static_cast<size_t>(pl->sk_slots) * BM * MAIN_BN * 4);
     pl->xa = off;
     off = align256(off + M * r * 2);
     pl->part_xa = off;
@@ -390,18 +440,22 @@ lora_status_t step_main(const Ctx &c, GemmArgs &a, int64_t M, int64_t N, int64_t
     a.kb_per_split = a.kb0;
     a.num_tiles = a.m_tiles * a.n_tiles;
     a.group_m = std::min(a.m_tiles, 16);
-    const int grid = std::min(a.num_tiles, c.info->sms);
+    const int G = std::min(c.info->sms, PLAN_SMS);
+    const MainSched ms = main_sched(M, N, K0, r, G);
+    if (static_cast<int64_t>(ms.sk_tiles) * ms.sk_pieces > c.plan.sk_slots) return LORA_ERR_WORKSPACE;
+    a.dp_tiles = ms.dp_tiles;
+    a.dp_waves = ms.dp_waves;
+    a.sk_tiles = ms.sk_tiles;
+    a.sk_pieces = ms.sk_pieces;
+    a.sk_part = reinterpret_cast<float *>(c.ws + c.plan.part_sk);
+    a.counters = reinterpret_cast<int *>(c.ws + c.plan.ctr) + (c.plan.n_ctr - PLAN_SMS);
+    const int grid = ms.sk_pieces > 1 ? G : std::min(a.num_tiles, G);
     cudaError_t e;
     if (b_mn)
         e = launch_gemm<MAIN_BN, false, true, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_DX, kind);
     else
         e = launch_gemm<MAIN_BN, false, false, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_FWD, kind);
     return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
-}
-
-lora_status_t zero_counters(const Ctx &c) {
-    return cudaMemsetAsync(c.ws + c.plan.ctr, 0, c.plan.n_ctr * sizeof(int), c.st) == cudaSuccess ? LORA_OK
-                                                                                                   : LORA_ERR_CUDA;
 }
 
 #define LORA_TRY(x)                          \
@@ -422,7 +476,6 @@ lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, 
     LORA_TRY(prepare(LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
-    LORA_TRY(zero_counters(c));
     LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
     GemmArgs a = base_args(c);
     if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
@@ -444,7 +497,6 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W,
     Ctx c;
     LORA_TRY(prepare(LORA_OP_BWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
-    LORA_TRY(zero_counters(c));
     const uint16_t *sxa = xa_save;
     if (!sxa) {
         uint16_t *tmp = reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);

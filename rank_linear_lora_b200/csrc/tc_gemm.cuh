@@ -1,13 +1,13 @@
 // tc_gemm.cuh -- the tcgen05 contraction engine behind every step of the layer.
 //
-// One persistent, warp-specialised kernel template computes a 128 x BN output tile
+// One persistent, warp-specialised kernel template computes 128 x BN output tiles
 //     D = sum over K-segments  A_seg . B_seg^T
 // with bf16 operands staged by TMA into 128-byte-swizzled shared memory and fp32
 // accumulators in tensor memory:
 //   warp 0      TMA producer (one elected lane), STAGES-deep smem ring
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 2..5  epilogue: tcgen05.ld of their 32-lane TMEM quarter
-// Two accumulators alternate in TMEM so the epilogue of one tile overlaps the
+// Two accumulators alternate in TMEM so the epilogue of one work item overlaps the
 // K loop of the next.
 //
 // K-segments: segment 0 is the frozen-weight contraction (K = d_in or d_out);
@@ -17,12 +17,21 @@
 // contiguous in memory) or MN-major (the M/N index contiguous), so W is read in
 // place for both x.W^T and dY.W.
 //
-// Epilogues:
-//   EPI_STORE  bf16 tile -> 128B-swizzled smem staging -> TMA store (h, dX).
-//   EPI_SPLITK fp32 partial of one K-split -> workspace; the last split to finish
-//              a tile (per-tile arrival counter) sums all splits in a fixed order
-//              and writes the result: bf16 rows (s.xa, s.g), fp32 rows (dB) or
-//              fp32 columns (dA, written transposed).  Deterministic.
+// Work items and epilogues:
+//   EPI_STORE  (h, dX) whole tiles in grouped raster order, `dp_waves` per CTA; when
+//              the tile count leaves a partial last wave, those `sk_tiles` tiles are
+//              cut into `sk_pieces` K ranges taken by one CTA each ("stream-K" on the
+//              last wave).  A piece writes its fp32 partial to the workspace; the last
+//              piece to finish a tile sums all pieces in piece order (deterministic)
+//              and stores the bf16 tile.  Stores go through 128B-swizzled smem
+//              staging and TMA.
+//   EPI_SPLITK (s.xa, s.g, dB, dA) skinny outputs, K split over CTAs; the last split
+//              to finish a tile sums the fp32 partials in split order and writes bf16
+//              rows, fp32 rows or fp32 columns (dA, written transposed).
+//
+// Launch: programmatic dependent launch is honoured -- set-up (barrier init, TMEM
+// allocation, descriptor prefetch) runs before griddepcontrol.wait; every global
+// memory access comes after it.
 //
 // Every wait is bounded (globaltimer); on expiry the kernel records an error code,
 // drains its outstanding copies and MMAs, frees TMEM and returns.
@@ -59,18 +68,26 @@ struct GemmArgs {
     int m_tiles, n_tiles;
     int kb0, kb1;            // 64-wide K blocks per segment
     int mma_last1;           // K=16 MMAs in the last block of segment 1 (1..4)
-    int splits;              // EPI_SPLITK: K splits of segment 0
+    // EPI_SPLITK
+    int splits;              // K splits of segment 0
     int kb_per_split;
     int num_tiles;           // m_tiles * n_tiles * splits
-    int group_m;             // EPI_STORE rasterisation: M tiles per group
-    int rows_valid;          // EPI_SPLITK: valid output rows
-    int n_valid;             // EPI_SPLITK: valid output columns (r)
+    int rows_valid;          // valid output rows
+    int n_valid;             // valid output columns (r)
     int out_mode;            // OutMode
     float out_scale;
-    float *part;             // EPI_SPLITK partials [splits][m_tiles*BM][n_valid]
-    int *counters;           // EPI_SPLITK per-tile arrival counters (zero on entry)
-    void *out;               // EPI_SPLITK output
+    float *part;             // partials [splits][m_tiles*BM][n_valid]
+    void *out;
     int64_t out_ld;          // OUT_F32_COLS: row stride of the transposed output
+    // EPI_STORE
+    int group_m;             // rasterisation: M tiles per group
+    int dp_tiles;            // tiles done whole (raster order 0 .. dp_tiles-1)
+    int dp_waves;            // whole tiles per CTA (at most)
+    int sk_tiles;            // last-wave tiles split along K (raster dp_tiles ..)
+    int sk_pieces;           // K pieces per split tile (0: none)
+    float *sk_part;          // [sk_tiles][sk_pieces][BN/32][BM][32] fp32
+    // shared
+    int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
 };
@@ -78,7 +95,7 @@ struct GemmArgs {
 // Trace record of one CTA (globaltimer ns unless noted).
 enum TraceField {
     TR_ENTRY = 0, TR_SETUP = 1, TR_PROD_END = 2, TR_MMA_END = 3, TR_EPI_END = 4, TR_EXIT = 5,
-    TR_SMID = 6, TR_TILES = 7, TR_TILE_DONE0 = 8,  // epilogue completion of the first 8 tiles
+    TR_SMID = 6, TR_TILES = 7, TR_TILE_DONE0 = 8,  // epilogue completion of the first 8 items
     TRACE_WORDS = 16
 };
 
@@ -95,6 +112,7 @@ struct GemmCfg {
     static_assert(!B_MN || BN % 64 == 0, "MN-major B uses 64-wide swizzle chunks");
     static_assert(B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM alloc is a power of 2");
+    static_assert(EPI != EPI_STORE || BN % 64 == 0, "store epilogue works in 64-column chunks");
 };
 
 // Bounded mbarrier wait.  Returns false (and raises the abort flag and the error
@@ -117,28 +135,82 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     }
 }
 
-struct TileCoord {
-    int m, n, split;
+// One unit of work of a CTA: output tile (m, n), K blocks [kb_lo, kb_hi) of the
+// concatenated segments, and how its result is finished.
+struct WorkItem {
+    int m, n;
+    int kb_lo, kb_hi;
+    int piece;   // split index (EPI_SPLITK) or stream-K piece (EPI_STORE)
+    int sk;      // EPI_STORE: stream-K tile slot, or -1 for a whole tile
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const GemmArgs &p, int t, int epi) {
-    TileCoord c;
-    if (epi == EPI_SPLITK) {
-        c.split = t % p.splits;
-        int mn = t / p.splits;
-        c.m = mn % p.m_tiles;
-        c.n = mn / p.m_tiles;
-    } else {
-        // Grouped rasterisation: group_m M-tiles share each B (weight) tile in L2.
-        int group = p.group_m * p.n_tiles;
-        int g = t / group, idx = t % group;
-        int m0 = g * p.group_m;
-        int gm = min(p.group_m, p.m_tiles - m0);
-        c.m = m0 + idx % gm;
-        c.n = idx / gm;
-        c.split = 0;
+__device__ __forceinline__ void raster(const GemmArgs &p, int t, int &m, int &n) {
+    // Grouped rasterisation: group_m M-tiles share each B (weight) tile in L2.
+    const int group = p.group_m * p.n_tiles;
+    const int g = t / group, idx = t % group;
+    const int m0 = g * p.group_m;
+    const int gm = min(p.group_m, p.m_tiles - m0);
+    m = m0 + idx % gm;
+    n = idx / gm;
+}
+
+// Item i (0, 1, ...) of this CTA; false when the CTA has no more work.
+template <int EPI>
+__device__ __forceinline__ bool get_item(const GemmArgs &p, int i, WorkItem &w) {
+    const int G = gridDim.x, c = blockIdx.x;
+    if (EPI == EPI_SPLITK) {
+        const int t = c + i * G;
+        if (t >= p.num_tiles) return false;
+        w.piece = t % p.splits;
+        const int mn = t / p.splits;
+        w.m = mn % p.m_tiles;
+        w.n = mn / p.m_tiles;
+        w.kb_lo = w.piece * p.kb_per_split;
+        w.kb_hi = min(p.kb0, w.kb_lo + p.kb_per_split);
+        w.sk = -1;
+        return true;
     }
-    return c;
+    const int kbt = p.kb0 + p.kb1;
+    if (i < p.dp_waves) {
+        const int t = c + i * G;
+        if (t >= p.dp_tiles) return false;
+        raster(p, t, w.m, w.n);
+        w.kb_lo = 0;
+        w.kb_hi = kbt;
+        w.piece = 0;
+        w.sk = -1;
+        return true;
+    }
+    if (i == p.dp_waves && p.sk_pieces > 1 && c < p.sk_tiles * p.sk_pieces) {
+        w.sk = c % p.sk_tiles;
+        w.piece = c / p.sk_tiles;
+        raster(p, p.dp_tiles + w.sk, w.m, w.n);
+        w.kb_lo = (w.piece * kbt) / p.sk_pieces;
+        w.kb_hi = ((w.piece + 1) * kbt) / p.sk_pieces;
+        return true;
+    }
+    return false;
+}
+
+// Pack 64 fp32 columns of one accumulator row to bf16 and write them into row `lane`
+// of a 32 x 64 staging box with the 128-byte swizzle TMA expects (16-byte chunk cc of
+// row r lands at chunk cc ^ (r % 8)).
+__device__ __forceinline__ void stage_row64(uint8_t *sbuf, int lane, const uint32_t (&v0)[32],
+                                            const uint32_t (&v1)[32]) {
+    uint32_t packed[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        __nv_bfloat162 lo2 = __floats2bfloat162_rn(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1]));
+        __nv_bfloat162 hi2 = __floats2bfloat162_rn(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1]));
+        packed[j] = *reinterpret_cast<uint32_t *>(&lo2);
+        packed[16 + j] = *reinterpret_cast<uint32_t *>(&hi2);
+    }
+    uint8_t *row_ptr = sbuf + lane * 128;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint4 w = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
+        *reinterpret_cast<uint4 *>(row_ptr + ((cc ^ (lane & 7)) * 16)) = w;
+    }
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
@@ -184,6 +256,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         *last_flag = 0;
         fence_mbar_init();
     }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&p.tmA0);
+        tma_prefetch_desc(&p.tmB0);
+        if (p.kb1 > 0) {
+            tma_prefetch_desc(&p.tmA1);
+            tma_prefetch_desc(&p.tmB1);
+        }
+        if (EPI == EPI_STORE) tma_prefetch_desc(&p.tmC);
+    }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_slot), Cfg::TMEM_COLS);
         tmem_relinquish();
@@ -192,29 +273,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // Everything above touched no global memory; from here on we may read what the
+    // previous kernel in the stream wrote and overwrite what it read.
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     if (trace && threadIdx.x == 0) trace[TR_SETUP] = globaltimer_ns();
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch_desc(&p.tmA0);
-            tma_prefetch_desc(&p.tmB0);
-            if (p.kb1 > 0) {
-                tma_prefetch_desc(&p.tmA1);
-                tma_prefetch_desc(&p.tmB1);
-            }
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued?, parity of last issue
             bool ok = true;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-                const TileCoord c = decode_tile(p, t, EPI);
-                int kb_lo = 0, kb_hi = p.kb0 + p.kb1;
-                if (EPI == EPI_SPLITK) {
-                    kb_lo = c.split * p.kb_per_split;
-                    kb_hi = min(p.kb0, kb_lo + p.kb_per_split);
-                }
-                for (int kb = kb_lo; kb < kb_hi; ++kb) {
+            WorkItem w;
+            for (int i = 0; ok && get_item<EPI>(p, i, w); ++i) {
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
                                       DERR_WAIT_EMPTY)) {
                         ok = false;
@@ -231,17 +305,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                     const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     if (A_MN) {
-                        tma_load_2d(a_dst, ta, fb, c.m * BM, k0);
-                        tma_load_2d(a_dst + 64 * 128, ta, fb, c.m * BM + 64, k0);
+                        tma_load_2d(a_dst, ta, fb, w.m * BM, k0);
+                        tma_load_2d(a_dst + 64 * 128, ta, fb, w.m * BM + 64, k0);
                     } else {
-                        tma_load_2d(a_dst, ta, fb, k0, c.m * BM);
+                        tma_load_2d(a_dst, ta, fb, k0, w.m * BM);
                     }
                     if (B_MN) {
 #pragma unroll
-                        for (int i = 0; i < BN / 64; ++i)
-                            tma_load_2d(b_dst + i * 64 * 128, tb, fb, c.n * BN + 64 * i, k0);
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(b_dst + j * 64 * 128, tb, fb, w.n * BN + 64 * j, k0);
                     } else {
-                        tma_load_2d(b_dst, tb, fb, k0, c.n * BN);
+                        tma_load_2d(b_dst, tb, fb, k0, w.n * BN);
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -268,17 +342,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
             constexpr uint32_t a_lbo = A_MN ? 64u * 128u : 16u;
             constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
+            const int kb_last = p.kb0 + p.kb1 - 1;
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
-                const TileCoord c = decode_tile(p, t, EPI);
-                int nkb = p.kb0 + p.kb1;
-                if (EPI == EPI_SPLITK) {
-                    const int lo = c.split * p.kb_per_split;
-                    nkb = min(p.kb0, lo + p.kb_per_split) - lo;
-                }
+            WorkItem w;
+            for (; ok && get_item<EPI>(p, it, w); ++it) {
                 const int buf = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
                 if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
@@ -288,21 +358,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-                for (int i = 0; i < nkb; ++i) {
-                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err,
-                                      DERR_WAIT_FULL)) {
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const bool last_tail = (EPI == EPI_STORE) && p.kb1 > 0 && i == nkb - 1;
-                    const int nmma = last_tail ? p.mma_last1 : BK / 16;
+                    const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
                     const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
                     for (int kk = 0; kk < nmma; ++kk) {
                         const uint64_t ad = sdesc_sw128(a_base + kk * a_kstep, a_lbo, 1024);
                         const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
-                        tc_mma_bf16(d_tmem, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&empty_bar[stage]));
                     if (++stage == STAGES) {
@@ -328,12 +396,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         const int row_local = q * 32 + lane;    // accumulator row of this thread
         const int epi_tid = threadIdx.x - 64;   // 0..127
         int it = 0;
-        for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
-            const TileCoord c = decode_tile(p, t, EPI);
+        WorkItem w;
+        for (; get_item<EPI>(p, it, w); ++it) {
             const int buf = it & 1;
             const uint32_t aphase = (it >> 1) & 1;
             // One thread waits; the outcome is broadcast so all four warps take the
-            // same path (the split-K fixup below uses named barriers).
+            // same path (the fixups below use named barriers).
             if (epi_tid == 0)
                 epi_ok[it & 1] = wait_bounded(smem_u32(&tfull_bar[buf]), aphase, abort_flag, p.err,
                                               DERR_WAIT_TMEM_FULL) ? 1 : 0;
@@ -344,52 +412,108 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                                    static_cast<uint32_t>(buf * BN);
             if constexpr (EPI == EPI_STORE) {
                 uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
+                if (w.sk < 0) {
+                    // Whole tile: TMEM -> bf16 -> swizzled smem -> TMA store, 64 columns at a time.
 #pragma unroll 1
-                for (int ch = 0; ch < BN / 64; ++ch) {
-                    uint32_t v0[32], v1[32];
-                    tmem_ld_32x32b_x32(t_row + ch * 64, v0);
-                    tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
-                    tc_wait_ld();
-                    if (ch == BN / 64 - 1) {
-                        tc_fence_before();
+                    for (int ch = 0; ch < BN / 64; ++ch) {
+                        uint32_t v0[32], v1[32];
+                        tmem_ld_32x32b_x32(t_row + ch * 64, v0);
+                        tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
+                        tc_wait_ld();
+                        if (ch == BN / 64 - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
+                        }
+                        uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                        // The TMA store that used this buffer two chunks ago must have read it.
+                        if (lane == 0) bulk_wait_group_read<1>();
                         __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
+                        stage_row64(sbuf, lane, v0, v1);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&p.tmC, smem_u32(sbuf), w.n * BN + ch * 64, w.m * BM + q * 32);
+                            bulk_commit_group();
+                        }
                     }
-                    uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
-                    // The TMA store that used this buffer two chunks ago must have read it.
-                    if (lane == 0) bulk_wait_group_read<1>();
-                    __syncwarp();
-                    uint32_t packed[32];
+                } else {
+                    // Stream-K piece: fp32 partial -> workspace slot [chunk][row][32].
+                    const int64_t slot = static_cast<int64_t>(w.sk) * p.sk_pieces;
+                    float *mine = p.sk_part + (slot + w.piece) * (static_cast<int64_t>(BN) * BM);
+#pragma unroll 1
+                    for (int ch = 0; ch < BN / 32; ++ch) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(t_row + ch * 32, v);
+                        tc_wait_ld();
+                        float4 *dst = reinterpret_cast<float4 *>(mine + (static_cast<int64_t>(ch) * BM + row_local) * 32);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        __nv_bfloat162 lo2 = __floats2bfloat162_rn(__uint_as_float(v0[2 * j]),
-                                                                   __uint_as_float(v0[2 * j + 1]));
-                        __nv_bfloat162 hi2 = __floats2bfloat162_rn(__uint_as_float(v1[2 * j]),
-                                                                   __uint_as_float(v1[2 * j + 1]));
-                        packed[j] = *reinterpret_cast<uint32_t *>(&lo2);
-                        packed[16 + j] = *reinterpret_cast<uint32_t *>(&hi2);
+                        for (int j = 0; j < 8; ++j)
+                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
                     }
-                    // Row `lane` of a 32 x 64 bf16 box, 128-byte swizzle: 16-byte chunk cc
-                    // lands at chunk (cc ^ (row % 8)).
-                    uint8_t *row_ptr = sbuf + lane * 128;
-#pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        uint4 w = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2],
-                                             packed[4 * cc + 3]);
-                        *reinterpret_cast<uint4 *>(row_ptr + ((cc ^ (lane & 7)) * 16)) = w;
-                    }
-                    fence_proxy_async_smem();
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&p.tmC, smem_u32(sbuf), c.n * BN + ch * 64, c.m * BM + q * 32);
-                        bulk_commit_group();
+                    if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
+                    __threadfence();
+                    named_bar_sync(1, 128);
+                    if (epi_tid == 0)
+                        *last_flag = (atomicAdd(&p.counters[w.sk], 1) == p.sk_pieces - 1) ? 1 : 0;
+                    named_bar_sync(1, 128);
+                    const bool last = *last_flag != 0;
+                    named_bar_sync(1, 128);
+                    if (last) {
+                        // Sum every piece of the tile in piece order, then store as a whole tile.
+                        __threadfence();
+                        const float *base = p.sk_part + slot * (static_cast<int64_t>(BN) * BM);
+#pragma unroll 1
+                        for (int ch = 0; ch < BN / 64; ++ch) {
+                            uint32_t v0[32], v1[32];
+#pragma unroll
+                            for (int half = 0; half < 2; ++half) {
+                                float acc[32];
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+                                for (int pc = 0; pc < p.sk_pieces; ++pc) {
+                                    const float4 *src = reinterpret_cast<const float4 *>(
+                                        base + pc * (static_cast<int64_t>(BN) * BM) +
+                                        (static_cast<int64_t>(2 * ch + half) * BM + row_local) * 32);
+                                    float4 t4[8];
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j) t4[j] = __ldcg(src + j);
+#pragma unroll
+                                    for (int j = 0; j < 8; ++j) {
+                                        acc[4 * j] += t4[j].x;
+                                        acc[4 * j + 1] += t4[j].y;
+                                        acc[4 * j + 2] += t4[j].z;
+                                        acc[4 * j + 3] += t4[j].w;
+                                    }
+                                }
+#pragma unroll
+                                for (int j = 0; j < 32; ++j) {
+                                    if (half == 0) v0[j] = __float_as_uint(acc[j]);
+                                    else v1[j] = __float_as_uint(acc[j]);
+                                }
+                            }
+                            uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                            if (lane == 0) bulk_wait_group_read<1>();
+                            __syncwarp();
+                            stage_row64(sbuf, lane, v0, v1);
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) {
+                                tma_store_2d(&p.tmC, smem_u32(sbuf), w.n * BN + ch * 64, w.m * BM + q * 32);
+                                bulk_commit_group();
+                            }
+                        }
+                        if (epi_tid == 0) p.counters[w.sk] = 0;  // ready for the next call
                     }
                 }
             } else {
                 // fp32 partial of this K split -> workspace.
                 const int64_t rows_total = static_cast<int64_t>(p.m_tiles) * BM;
-                const int64_t grow = static_cast<int64_t>(c.m) * BM + row_local;
-                float *my_part = p.part + ((static_cast<int64_t>(c.split) * rows_total + grow) * p.n_valid);
+                const int64_t grow = static_cast<int64_t>(w.m) * BM + row_local;
+                float *my_part = p.part + ((static_cast<int64_t>(w.piece) * rows_total + grow) * p.n_valid);
                 for (int c0 = 0; c0 < p.n_valid; c0 += 8) {
                     uint32_t v[8];
                     tmem_ld_32x32b_x8(t_row + c0, v);
@@ -405,7 +529,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
                 __threadfence();
                 named_bar_sync(1, 128);
-                const int ctr = c.n * p.m_tiles + c.m;
+                const int ctr = w.n * p.m_tiles + w.m;
                 if (epi_tid == 0) *last_flag = (atomicAdd(&p.counters[ctr], 1) == p.splits - 1) ? 1 : 0;
                 named_bar_sync(1, 128);
                 const bool last = *last_flag != 0;
@@ -443,8 +567,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                             if (p.out_mode == OUT_BF16_ROWS) {
                                 __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
                                 __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
-                                uint2 w = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
-                                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + grow * p.n_valid + c0) = w;
+                                uint2 u2 = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
+                                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + grow * p.n_valid + c0) = u2;
                             } else if (p.out_mode == OUT_F32_ROWS) {
                                 *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + grow * p.n_valid + c0) = acc;
                             } else {

@@ -170,6 +170,25 @@ def test_timing_hooks_count_launches():
     assert all(rec[k][1] == 1 and rec[k][0] > 0 for k in L.KERNEL_KINDS)
 
 
+# Shapes whose main-GEMM tile count leaves a partial last wave on 148 SMs, so the
+# last-wave tiles are cut into K pieces (stream-K) and summed by the last piece.
+STREAMK = [
+    (2560, 1024, 2048, 8),    # forward: 160 tiles -> 12 tiles x 2 pieces
+    (2560, 2048, 1024, 16),   # dX: 160 tiles -> 12 tiles x 2 pieces
+    (1920, 2048, 2560, 24),   # forward: 150 tiles -> 2 tiles x 4 pieces, rank tail in the last piece
+]
+
+
+@pytest.mark.parametrize("shape", STREAMK, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_streamk_tail_wave(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("streamk", M, di, do, r, alpha=2.0 * r, seed=0x51 + M + di)
+    inp, dl = _run_full(spec)
+    rows = sample_rows(M, n_random=40, seed=M)
+    # whole output rows of every sampled token, plus full dA/dB
+    compare_all(dl.results(rows=rows), oracle_ref(inp, rows=rows), spec.s)
+
+
 # ------------------------------------------------------------------ full sizes
 FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0)]
 
