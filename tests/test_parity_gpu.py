@@ -184,9 +184,7 @@ def test_streamk_tail_wave(shape):
     M, di, do, r = shape
     spec = inputs.LayerSpec("streamk", M, di, do, r, alpha=2.0 * r, seed=0x51 + M + di)
     inp, dl = _run_full(spec)
-    rows = sample_rows(M, n_random=40, seed=M)
-    # whole output rows of every sampled token, plus full dA/dB
-    compare_all(dl.results(rows=rows), oracle_ref(inp, rows=rows), spec.s)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
 
 
 # ------------------------------------------------------------------ full sizes
