@@ -226,24 +226,24 @@ Split choose_split(int64_t mt, int64_t kb, int sms) {
 
 constexpr int PLAN_SMS = 148;  // SMs a launch uses at most (sizes splits and the workspace)
 
-// Main-GEMM schedule: whole tiles in waves over G CTAs; a partial last wave of R
-// tiles is cut into `pieces` K ranges so every CTA gets work (stream-K on the tail).
+// Main-GEMM schedule: whole 128 x 256 tiles in waves over G CTAs; a partial last
+// wave of R tiles is cut along N into 2 or 4 narrower tiles (one per CTA) when they
+// fit in one wave, so the last wave lasts a half or a quarter tile.
 struct MainSched {
-    int tiles = 0, dp_tiles = 0, dp_waves = 0, sk_tiles = 0, sk_pieces = 0;
+    int tiles = 0, dp_tiles = 0, dp_waves = 0, tail_tiles = 0, tail_split = 1;
 };
 
-MainSched main_sched(int64_t M, int64_t N, int64_t K0, int r, int G) {
+MainSched main_sched(int64_t M, int64_t N, int G) {
     MainSched s;
     const int64_t T = cdiv(M, BM) * cdiv(N, MAIN_BN);
-    const int64_t kbt = cdiv(K0, BK) + cdiv(r, BK);
     s.tiles = static_cast<int>(T);
     const int64_t W = T / G, R = T % G;
-    int64_t pieces = (R > 0) ? std::min<int64_t>({G / R, 4, kbt / 8}) : 0;
-    if (W >= 1 && R > 0 && pieces >= 2) {
+    const int split = (R > 0 && 4 * R <= G) ? 4 : (R > 0 && 2 * R <= G) ? 2 : 1;
+    if (W >= 1 && split > 1) {
         s.dp_tiles = static_cast<int>(W * G);
         s.dp_waves = static_cast<int>(W);
-        s.sk_tiles = static_cast<int>(R);
-        s.sk_pieces = static_cast<int>(pieces);
+        s.tail_tiles = static_cast<int>(R);
+        s.tail_split = split;
     } else {
         s.dp_tiles = static_cast<int>(T);
         s.dp_waves = static_cast<int>(cdiv(T, G));
@@ -253,8 +253,8 @@ MainSched main_sched(int64_t M, int64_t N, int64_t K0, int r, int G) {
 
 struct Plan {
     size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0;
-    size_t part_sk = 0, total = 0;
-    int64_t n_ctr = 0, sk_slots = 0;
+    size_t total = 0;
+    int64_t n_ctr = 0;
     Split s_xa, s_g, s_db, s_da;
 };
 
@@ -265,18 +265,12 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     pl->s_g = choose_split(mt_tok, cdiv(d_out, BK), sms);
     pl->s_db = choose_split(mt_out, cdiv(M, BK), sms);
     pl->s_da = choose_split(mt_in, cdiv(M, BK), sms);
-    // Stream-K slots of the main GEMM: pieces x split tiles <= CTAs <= min(tiles, PLAN_SMS)
-    // whatever the device's SM count, so reserve one 128 x 256 fp32 slot per CTA.
-    const int64_t main_tiles = bwd ? cdiv(M, BM) * cdiv(d_in, MAIN_BN) : cdiv(M, BM) * cdiv(d_out, MAIN_BN);
-    pl->sk_slots = std::min<int64_t>(main_tiles, PLAN_SMS);
     size_t off = 0;
     pl->err = off;
     off += 256;
     pl->ctr = off;
-    pl->n_ctr = mt_tok * 2 + mt_in + mt_out + PLAN_SMS;  // skinny tiles, then stream-K tiles
+    pl->n_ctr = mt_tok * 2 + mt_in + mt_out;
     off = align256(off + pl->n_ctr * sizeof(int));
-    pl->part_sk = off;
-    off = align256(off + static_cast<size_t>(pl->sk_slots) * BM * MAIN_BN * 4);
     pl->xa = off;
     off = align256(off + M * r * 2);
     pl->part_xa = off;
@@ -441,15 +435,12 @@ lora_status_t step_main(const Ctx &c, GemmArgs &a, int64_t M, int64_t N, int64_t
     a.num_tiles = a.m_tiles * a.n_tiles;
     a.group_m = std::min(a.m_tiles, 16);
     const int G = std::min(c.info->sms, PLAN_SMS);
-    const MainSched ms = main_sched(M, N, K0, r, G);
-    if (static_cast<int64_t>(ms.sk_tiles) * ms.sk_pieces > c.plan.sk_slots) return LORA_ERR_WORKSPACE;
+    const MainSched ms = main_sched(M, N, G);
     a.dp_tiles = ms.dp_tiles;
     a.dp_waves = ms.dp_waves;
-    a.sk_tiles = ms.sk_tiles;
-    a.sk_pieces = ms.sk_pieces;
-    a.sk_part = reinterpret_cast<float *>(c.ws + c.plan.part_sk);
-    a.counters = reinterpret_cast<int *>(c.ws + c.plan.ctr) + (c.plan.n_ctr - PLAN_SMS);
-    const int grid = ms.sk_pieces > 1 ? G : std::min(a.num_tiles, G);
+    a.tail_tiles = ms.tail_tiles;
+    a.tail_split = ms.tail_split;
+    const int grid = ms.tail_split > 1 ? G : std::min(a.num_tiles, G);
     cudaError_t e;
     if (b_mn)
         e = launch_gemm<MAIN_BN, false, true, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_DX, kind);
@@ -483,6 +474,14 @@ lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, 
     if (!tmap_bf16(&a.tmA1, sxa, r, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmB1, B, r, d_out, 64, MAIN_BN)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmC, h, d_out, M, 64, 32)) return LORA_ERR_CUDA;
+    {
+        const MainSched ms = main_sched(M, d_out, std::min(c.info->sms, PLAN_SMS));
+        if (ms.tail_split > 1) {
+            const uint32_t rows = MAIN_BN / ms.tail_split;
+            if (!tmap_bf16(&a.tmB0n, W, d_in, d_out, 64, rows)) return LORA_ERR_CUDA;
+            if (!tmap_bf16(&a.tmB1n, B, r, d_out, 64, rows)) return LORA_ERR_CUDA;
+        }
+    }
     return step_main(c, a, M, d_out, d_in, r, false, LORA_K_FWD_MAIN);
 }
 

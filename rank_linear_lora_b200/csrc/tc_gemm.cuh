@@ -19,12 +19,11 @@
 //
 // Work items and epilogues:
 //   EPI_STORE  (h, dX) whole tiles in grouped raster order, `dp_waves` per CTA; when
-//              the tile count leaves a partial last wave, those `sk_tiles` tiles are
-//              cut into `sk_pieces` K ranges taken by one CTA each ("stream-K" on the
-//              last wave).  A piece writes its fp32 partial to the workspace; the last
-//              piece to finish a tile sums all pieces in piece order (deterministic)
-//              and stores the bf16 tile.  Stores go through 128B-swizzled smem
-//              staging and TMA.
+//              the tile count leaves a partial last wave of `tail_tiles` tiles, each of
+//              them is cut along N into `tail_split` narrower tiles (128 x 128 or
+//              128 x 64, full K) taken by one CTA each, so the last wave is shorter and
+//              every output element is still produced by one accumulator.  Stores go
+//              through 128B-swizzled smem staging and TMA.
 //   EPI_SPLITK (s.xa, s.g, dB, dA) skinny outputs, K split over CTAs; the last split
 //              to finish a tile sums the fp32 partials in split order and writes bf16
 //              rows, fp32 rows or fp32 columns (dA, written transposed).
@@ -65,6 +64,7 @@ struct GemmArgs {
     CUtensorMap tmA0, tmB0;  // segment 0
     CUtensorMap tmA1, tmB1;  // segment 1 (rank-r tail), used when kb1 > 0
     CUtensorMap tmC;         // EPI_STORE output (bf16, box 64 x 32, 128B swizzle)
+    CUtensorMap tmB0n, tmB1n;  // K-major B with box rows BN / tail_split (narrow tail tiles)
     int m_tiles, n_tiles;
     int kb0, kb1;            // 64-wide K blocks per segment
     int mma_last1;           // K=16 MMAs in the last block of segment 1 (1..4)
@@ -83,10 +83,9 @@ struct GemmArgs {
     int group_m;             // rasterisation: M tiles per group
     int dp_tiles;            // tiles done whole (raster order 0 .. dp_tiles-1)
     int dp_waves;            // whole tiles per CTA (at most)
-    int sk_tiles;            // last-wave tiles split along K (raster dp_tiles ..)
-    int sk_pieces;           // K pieces per split tile (0: none)
-    float *sk_part;          // [sk_tiles][sk_pieces][BN/32][BM][32] fp32
-    // shared
+    int tail_tiles;          // last-wave tiles cut along N (raster dp_tiles ..)
+    int tail_split;          // 1 (none), 2 or 4 narrow tiles per tail tile
+    // EPI_SPLITK
     int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
@@ -140,8 +139,9 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 struct WorkItem {
     int m, n;
     int kb_lo, kb_hi;
-    int piece;   // split index (EPI_SPLITK) or stream-K piece (EPI_STORE)
-    int sk;      // EPI_STORE: stream-K tile slot, or -1 for a whole tile
+    int piece;   // EPI_SPLITK: split index
+    int col0;    // EPI_STORE: first output column
+    int nsplit;  // EPI_STORE: 1 for a whole tile, else tail_split (width BN / nsplit)
 };
 
 __device__ __forceinline__ void raster(const GemmArgs &p, int t, int &m, int &n) {
@@ -155,7 +155,7 @@ __device__ __forceinline__ void raster(const GemmArgs &p, int t, int &m, int &n)
 }
 
 // Item i (0, 1, ...) of this CTA; false when the CTA has no more work.
-template <int EPI>
+template <int BN, int EPI>
 __device__ __forceinline__ bool get_item(const GemmArgs &p, int i, WorkItem &w) {
     const int G = gridDim.x, c = blockIdx.x;
     if (EPI == EPI_SPLITK) {
@@ -167,26 +167,26 @@ __device__ __forceinline__ bool get_item(const GemmArgs &p, int i, WorkItem &w) 
         w.n = mn / p.m_tiles;
         w.kb_lo = w.piece * p.kb_per_split;
         w.kb_hi = min(p.kb0, w.kb_lo + p.kb_per_split);
-        w.sk = -1;
+        w.col0 = 0;
+        w.nsplit = 1;
         return true;
     }
-    const int kbt = p.kb0 + p.kb1;
+    w.kb_lo = 0;
+    w.kb_hi = p.kb0 + p.kb1;
+    w.piece = 0;
     if (i < p.dp_waves) {
         const int t = c + i * G;
         if (t >= p.dp_tiles) return false;
         raster(p, t, w.m, w.n);
-        w.kb_lo = 0;
-        w.kb_hi = kbt;
-        w.piece = 0;
-        w.sk = -1;
+        w.nsplit = 1;
+        w.col0 = w.n * BN;
         return true;
     }
-    if (i == p.dp_waves && p.sk_pieces > 1 && c < p.sk_tiles * p.sk_pieces) {
-        w.sk = c % p.sk_tiles;
-        w.piece = c / p.sk_tiles;
-        raster(p, p.dp_tiles + w.sk, w.m, w.n);
-        w.kb_lo = (w.piece * kbt) / p.sk_pieces;
-        w.kb_hi = ((w.piece + 1) * kbt) / p.sk_pieces;
+    if (i == p.dp_waves && p.tail_split > 1 && c < p.tail_tiles * p.tail_split) {
+        const int tt = c / p.tail_split, h = c % p.tail_split;
+        raster(p, p.dp_tiles + tt, w.m, w.n);
+        w.nsplit = p.tail_split;
+        w.col0 = w.n * BN + h * (BN / p.tail_split);
         return true;
     }
     return false;
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued?, parity of last issue
             bool ok = true;
             WorkItem w;
-            for (int i = 0; ok && get_item<EPI>(p, i, w); ++i) {
+            for (int i = 0; ok && get_item<BN, EPI>(p, i, w); ++i) {
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
                                       DERR_WAIT_EMPTY)) {
@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                         break;
                     }
                     const uint32_t fb = smem_u32(&full_bar[stage]);
-                    mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                    const int bn = BN / w.nsplit;  // columns of B this item loads
+                    mbar_arrive_expect_tx(fb, Cfg::A_BYTES + bn * BK * 2);
                     issued_mask |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     const bool seg1 = kb >= p.kb0;
@@ -311,11 +312,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                         tma_load_2d(a_dst, ta, fb, k0, w.m * BM);
                     }
                     if (B_MN) {
-#pragma unroll
-                        for (int j = 0; j < BN / 64; ++j)
-                            tma_load_2d(b_dst + j * 64 * 128, tb, fb, w.n * BN + 64 * j, k0);
+                        for (int j = 0; j < bn / 64; ++j)
+                            tma_load_2d(b_dst + j * 64 * 128, tb, fb, w.col0 + 64 * j, k0);
+                    } else if (w.nsplit == 1) {
+                        tma_load_2d(b_dst, tb, fb, k0, w.col0);
                     } else {
-                        tma_load_2d(b_dst, tb, fb, k0, w.n * BN);
+                        tma_load_2d(b_dst, seg1 ? &p.tmB1n : &p.tmB0n, fb, k0, w.col0);
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -335,7 +337,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(BM, BN, A_MN, B_MN);
+            constexpr uint32_t idesc_full = idesc_bf16(BM, BN, A_MN, B_MN);
+            constexpr uint32_t idesc_half = idesc_bf16(BM, BN >= 128 ? BN / 2 : BN, A_MN, B_MN);
+            constexpr uint32_t idesc_quarter = idesc_bf16(BM, BN >= 256 ? BN / 4 : BN, A_MN, B_MN);
             // K step of 16 elements inside a stage: +32 B along a K-major row,
             // +16 rows (2 swizzle atoms) for an MN-major tile.
             constexpr uint32_t a_kstep = A_MN ? 2048u : 32u;
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             int it = 0;
             bool ok = true;
             WorkItem w;
-            for (; ok && get_item<EPI>(p, it, w); ++it) {
+            for (; ok && get_item<BN, EPI>(p, it, w); ++it) {
                 const int buf = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
                 if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
@@ -358,6 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t idesc = w.nsplit == 1 ? idesc_full : (w.nsplit == 2 ? idesc_half : idesc_quarter);
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         const int epi_tid = threadIdx.x - 64;   // 0..127
         int it = 0;
         WorkItem w;
-        for (; get_item<EPI>(p, it, w); ++it) {
+        for (; get_item<BN, EPI>(p, it, w); ++it) {
             const int buf = it & 1;
             const uint32_t aphase = (it >> 1) & 1;
             // One thread waits; the outcome is broadcast so all four warps take the
@@ -411,102 +416,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
             if constexpr (EPI == EPI_STORE) {
+                // TMEM -> bf16 -> swizzled smem -> TMA store, 64 columns at a time.
                 uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
-                if (w.sk < 0) {
-                    // Whole tile: TMEM -> bf16 -> swizzled smem -> TMA store, 64 columns at a time.
+                const int nch = (BN / 64) / w.nsplit;
 #pragma unroll 1
-                    for (int ch = 0; ch < BN / 64; ++ch) {
-                        uint32_t v0[32], v1[32];
-                        tmem_ld_32x32b_x32(t_row + ch * 64, v0);
-                        tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
-                        tc_wait_ld();
-                        if (ch == BN / 64 - 1) {
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
-                        }
-                        uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
-                        // The TMA store that used this buffer two chunks ago must have read it.
-                        if (lane == 0) bulk_wait_group_read<1>();
+                for (int ch = 0; ch < nch; ++ch) {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(t_row + ch * 64, v0);
+                    tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
+                    tc_wait_ld();
+                    if (ch == nch - 1) {
+                        tc_fence_before();
                         __syncwarp();
-                        stage_row64(sbuf, lane, v0, v1);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&p.tmC, smem_u32(sbuf), w.n * BN + ch * 64, w.m * BM + q * 32);
-                            bulk_commit_group();
-                        }
+                        if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
                     }
-                } else {
-                    // Stream-K piece: fp32 partial -> workspace slot [chunk][row][32].
-                    const int64_t slot = static_cast<int64_t>(w.sk) * p.sk_pieces;
-                    float *mine = p.sk_part + (slot + w.piece) * (static_cast<int64_t>(BN) * BM);
-#pragma unroll 1
-                    for (int ch = 0; ch < BN / 32; ++ch) {
-                        uint32_t v[32];
-                        tmem_ld_32x32b_x32(t_row + ch * 32, v);
-                        tc_wait_ld();
-                        float4 *dst = reinterpret_cast<float4 *>(mine + (static_cast<int64_t>(ch) * BM + row_local) * 32);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-                    }
-                    tc_fence_before();
+                    uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                    // The TMA store that used this buffer two chunks ago must have read it.
+                    if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
-                    __threadfence();
-                    named_bar_sync(1, 128);
-                    if (epi_tid == 0)
-                        *last_flag = (atomicAdd(&p.counters[w.sk], 1) == p.sk_pieces - 1) ? 1 : 0;
-                    named_bar_sync(1, 128);
-                    const bool last = *last_flag != 0;
-                    named_bar_sync(1, 128);
-                    if (last) {
-                        // Sum every piece of the tile in piece order, then store as a whole tile.
-                        __threadfence();
-                        const float *base = p.sk_part + slot * (static_cast<int64_t>(BN) * BM);
-#pragma unroll 1
-                        for (int ch = 0; ch < BN / 64; ++ch) {
-                            uint32_t v0[32], v1[32];
-#pragma unroll
-                            for (int half = 0; half < 2; ++half) {
-                                float acc[32];
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) acc[j] = 0.f;
-                                for (int pc = 0; pc < p.sk_pieces; ++pc) {
-                                    const float4 *src = reinterpret_cast<const float4 *>(
-                                        base + pc * (static_cast<int64_t>(BN) * BM) +
-                                        (static_cast<int64_t>(2 * ch + half) * BM + row_local) * 32);
-                                    float4 t4[8];
-#pragma unroll
-                                    for (int j = 0; j < 8; ++j) t4[j] = __ldcg(src + j);
-#pragma unroll
-                                    for (int j = 0; j < 8; ++j) {
-                                        acc[4 * j] += t4[j].x;
-                                        acc[4 * j + 1] += t4[j].y;
-                                        acc[4 * j + 2] += t4[j].z;
-                                        acc[4 * j + 3] += t4[j].w;
-                                    }
-                                }
-#pragma unroll
-                                for (int j = 0; j < 32; ++j) {
-                                    if (half == 0) v0[j] = __float_as_uint(acc[j]);
-                                    else v1[j] = __float_as_uint(acc[j]);
-                                }
-                            }
-                            uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
-                            if (lane == 0) bulk_wait_group_read<1>();
-                            __syncwarp();
-                            stage_row64(sbuf, lane, v0, v1);
-                            fence_proxy_async_smem();
-                            __syncwarp();
-                            if (lane == 0) {
-                                tma_store_2d(&p.tmC, smem_u32(sbuf), w.n * BN + ch * 64, w.m * BM + q * 32);
-                                bulk_commit_group();
-                            }
-                        }
-                        if (epi_tid == 0) p.counters[w.sk] = 0;  // ready for the next call
+                    stage_row64(sbuf, lane, v0, v1);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&p.tmC, smem_u32(sbuf), w.col0 + ch * 64, w.m * BM + q * 32);
+                        bulk_commit_group();
                     }
                 }
             } else {

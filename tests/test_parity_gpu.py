@@ -171,16 +171,18 @@ def test_timing_hooks_count_launches():
 
 
 # Shapes whose main-GEMM tile count leaves a partial last wave on 148 SMs, so the
-# last-wave tiles are cut into K pieces (stream-K) and summed by the last piece.
-STREAMK = [
-    (2560, 1024, 2048, 8),    # forward: 160 tiles -> 12 tiles x 2 pieces
-    (2560, 2048, 1024, 16),   # dX: 160 tiles -> 12 tiles x 2 pieces
-    (1920, 2048, 2560, 24),   # forward: 150 tiles -> 2 tiles x 4 pieces, rank tail in the last piece
+# last-wave 128 x 256 tiles are cut along N into 128 x 128 or 128 x 64 tiles.
+TAIL_WAVE = [
+    (2560, 1024, 2048, 8),    # forward: 160 tiles -> 12 tail tiles x 4 (K-major B, narrow maps)
+    (2560, 2048, 1024, 16),   # dX: 160 tiles -> 12 tail tiles x 4 (MN-major B)
+    (2304, 512, 2816, 16),    # forward: 198 tiles -> 50 tail tiles x 2
+    (2304, 2816, 512, 8),     # dX: 198 tiles -> 50 tail tiles x 2
+    (1920, 2048, 2560, 24),   # forward: 150 tiles -> 2 tail tiles x 4, rank tail r % 16 != 0
 ]
 
 
-@pytest.mark.parametrize("shape", STREAMK, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
-def test_streamk_tail_wave(shape):
+@pytest.mark.parametrize("shape", TAIL_WAVE, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_tail_wave_split(shape):
     M, di, do, r = shape
     spec = inputs.LayerSpec("streamk", M, di, do, r, alpha=2.0 * r, seed=0x51 + M + di)
     inp, dl = _run_full(spec)
