@@ -26,6 +26,7 @@
 
 #include "../../include/lora_linear.h"
 #include "tc_gemm.cuh"
+#include "tc_gemm2.cuh"
 
 using namespace lora;
 
@@ -135,11 +136,15 @@ std::atomic<size_t> g_trace_stride{0};
 // Programmatic dependent launch between consecutive kernels (LORA_LINEAR_PDL=0 turns
 // it off, for measurement).
 bool pdl_enabled() {
-    static const bool on = [] {
-        const char *v = std::getenv("LORA_LINEAR_PDL");
-        return !(v && v[0] == '0');
-    }();
-    return on;
+    const char *v = std::getenv("LORA_LINEAR_PDL");
+    return !(v && v[0] == '0');
+}
+
+// Main GEMMs on CTA pairs (tcgen05 cta_group::2); LORA_LINEAR_PAIR=0 selects the
+// single-SM kernel instead, for measurement.
+bool pair_enabled() {
+    const char *v = std::getenv("LORA_LINEAR_PAIR");
+    return !(v && v[0] == '0');
 }
 
 // ------------------------------------------------------------------ launch helpers
@@ -189,6 +194,101 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
     return e;
 }
 
+constexpr int PAIR_STAGES = 6;
+
+template <bool B_MN>
+cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
+    using Cfg = PairCfg<B_MN, PAIR_STAGES>;
+    auto kern = k_tc_gemm_pair<B_MN, PAIR_STAGES>;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(dev->attr_set & (1ull << attr_bit))) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            dev->attr_set |= 1ull << attr_bit;
+        }
+    }
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    const bool timed = g_timing.load() != 0;
+    if (timed) {
+        std::lock_guard<std::mutex> lk(g_tmu);
+        ea = pool_event();
+        eb = pool_event();
+        if (ea) cudaEventRecord(ea, st);
+    }
+    GemmArgs a2 = args;
+    unsigned long long *tr = g_trace.load();
+    const size_t stride = g_trace_stride.load();
+    if (tr && static_cast<size_t>(grid) * TRACE_WORDS <= stride) a2.trace = tr + static_cast<size_t>(kind) * stride;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a2);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    g_launches.fetch_add(1);
+    if (timed && ea && eb) {
+        cudaEventRecord(eb, st);
+        std::lock_guard<std::mutex> lk(g_tmu);
+        g_timed.push_back({kind, ea, eb});
+    }
+    return e;
+}
+
+// Clusters of two CTAs of the pair kernel that can be resident at once (0 if none).
+int pair_clusters(DevInfo *dev, bool b_mn) {
+    static int cached[64][2] = {};
+    static bool probed[64][2] = {};
+    int d = 0;
+    cudaGetDevice(&d);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (d < 0 || d >= 64) return 0;
+    if (!probed[d][b_mn]) {
+        probed[d][b_mn] = true;
+        int n = 0;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3(2 * (dev->sms / 2));
+        cfg.blockDim = dim3(NUM_THREADS);
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e;
+        if (b_mn) {
+            cfg.dynamicSmemBytes = PairCfg<true, PAIR_STAGES>::SMEM_BYTES;
+            cudaFuncSetAttribute(k_tc_gemm_pair<true, PAIR_STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PairCfg<true, PAIR_STAGES>::SMEM_BYTES);
+            e = cudaOccupancyMaxActiveClusters(&n, k_tc_gemm_pair<true, PAIR_STAGES>, &cfg);
+        } else {
+            cfg.dynamicSmemBytes = PairCfg<false, PAIR_STAGES>::SMEM_BYTES;
+            cudaFuncSetAttribute(k_tc_gemm_pair<false, PAIR_STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 PairCfg<false, PAIR_STAGES>::SMEM_BYTES);
+            e = cudaOccupancyMaxActiveClusters(&n, k_tc_gemm_pair<false, PAIR_STAGES>, &cfg);
+        }
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            n = 0;
+        }
+        cached[d][b_mn] = n;
+    }
+    return cached[d][b_mn];
+}
+
 // Attribute bits of the instantiations (one per template combination).
 enum {
     AB_FWD = 0,
@@ -196,6 +296,7 @@ enum {
     AB_XA16 = 2, AB_XA64, AB_XA128, AB_XA256,
     AB_G64 = 6, AB_G128, AB_G256,
     AB_T64 = 9, AB_T128, AB_T256,
+    AB_PAIR_K = 12, AB_PAIR_MN = 13,
 };
 
 int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
@@ -424,14 +525,57 @@ lora_status_t step_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float
 }
 
 // Main K-concatenated GEMM: out [M, N] = A0 . B0^T (K0) + A1 . B1^T (K1 = r).
-lora_status_t step_main(const Ctx &c, GemmArgs &a, int64_t M, int64_t N, int64_t K0, int r, bool b_mn, int kind) {
-    a.m_tiles = static_cast<int>(cdiv(M, BM));
-    a.n_tiles = static_cast<int>(cdiv(N, MAIN_BN));
+//   A0 [M, K0], A1 [M, r]: K-major bf16.
+//   B0, B1: K-major [N, K] (forward: W, B) or MN-major [K, N] (dX: W, A).
+struct MainOperands {
+    const void *A0, *B0, *A1, *B1;
+    void *C;
+};
+
+lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t N, int64_t K0, int r, bool b_mn,
+                        int kind) {
+    GemmArgs a = base_args(c);
     a.kb0 = static_cast<int>(cdiv(K0, BK));
     a.kb1 = static_cast<int>(cdiv(r, BK));
     a.mma_last1 = static_cast<int>(cdiv(r - (a.kb1 - 1) * BK, 16));
     a.splits = 1;
     a.kb_per_split = a.kb0;
+    if (!tmap_bf16(&a.tmA0, o.A0, K0, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmA1, o.A1, r, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmC, o.C, N, M, 64, 32)) return LORA_ERR_CUDA;
+    const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn), PLAN_SMS / 2) : 0;
+    if (pair_C > 0) {
+        // CTA pairs: 256 x 256 tiles, each CTA stages 128 rows of B.
+        const int64_t T = cdiv(M, PAIR_BM) * cdiv(N, PAIR_BN);
+        a.m_tiles = static_cast<int>(cdiv(M, PAIR_BM));
+        a.n_tiles = static_cast<int>(cdiv(N, PAIR_BN));
+        a.num_tiles = static_cast<int>(T);
+        a.group_m = std::min(a.m_tiles, 8);
+        const int64_t W = T / pair_C, R = T % pair_C;
+        const bool split = W >= 1 && R > 0 && 2 * R <= pair_C;
+        a.dp_tiles = static_cast<int>(split ? W * pair_C : T);
+        a.dp_waves = static_cast<int>(split ? W : cdiv(T, pair_C));
+        a.tail_tiles = static_cast<int>(split ? R : 0);
+        a.tail_split = split ? 2 : 1;
+        if (b_mn) {
+            if (!tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
+            if (!tmap_bf16(&a.tmB1, o.B1, N, r, 64, 64)) return LORA_ERR_CUDA;
+        } else {
+            if (!tmap_bf16(&a.tmB0, o.B0, K0, N, 64, CTA_BN)) return LORA_ERR_CUDA;
+            if (!tmap_bf16(&a.tmB1, o.B1, r, N, 64, CTA_BN)) return LORA_ERR_CUDA;
+            if (split) {
+                if (!tmap_bf16(&a.tmB0n, o.B0, K0, N, 64, CTA_BN / 2)) return LORA_ERR_CUDA;
+                if (!tmap_bf16(&a.tmB1n, o.B1, r, N, 64, CTA_BN / 2)) return LORA_ERR_CUDA;
+            }
+        }
+        const int clusters = split ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
+        cudaError_t e = b_mn ? launch_pair<true>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
+                             : launch_pair<false>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
+        return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    }
+    // Single-SM kernel: 128 x 256 tiles.
+    a.m_tiles = static_cast<int>(cdiv(M, BM));
+    a.n_tiles = static_cast<int>(cdiv(N, MAIN_BN));
     a.num_tiles = a.m_tiles * a.n_tiles;
     a.group_m = std::min(a.m_tiles, 16);
     const int G = std::min(c.info->sms, PLAN_SMS);
@@ -440,6 +584,18 @@ lora_status_t step_main(const Ctx &c, GemmArgs &a, int64_t M, int64_t N, int64_t
     a.dp_waves = ms.dp_waves;
     a.tail_tiles = ms.tail_tiles;
     a.tail_split = ms.tail_split;
+    if (b_mn) {
+        if (!tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
+        if (!tmap_bf16(&a.tmB1, o.B1, N, r, 64, 64)) return LORA_ERR_CUDA;
+    } else {
+        if (!tmap_bf16(&a.tmB0, o.B0, K0, N, 64, MAIN_BN)) return LORA_ERR_CUDA;
+        if (!tmap_bf16(&a.tmB1, o.B1, r, N, 64, MAIN_BN)) return LORA_ERR_CUDA;
+        if (ms.tail_split > 1) {
+            const uint32_t rows = MAIN_BN / ms.tail_split;
+            if (!tmap_bf16(&a.tmB0n, o.B0, K0, N, 64, rows)) return LORA_ERR_CUDA;
+            if (!tmap_bf16(&a.tmB1n, o.B1, r, N, 64, rows)) return LORA_ERR_CUDA;
+        }
+    }
     const int grid = ms.tail_split > 1 ? G : std::min(a.num_tiles, G);
     cudaError_t e;
     if (b_mn)
@@ -468,21 +624,8 @@ lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, 
     const float s = alpha / static_cast<float>(r);
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
-    GemmArgs a = base_args(c);
-    if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmB0, W, d_in, d_out, 64, MAIN_BN)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmA1, sxa, r, M, 64, 128)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmB1, B, r, d_out, 64, MAIN_BN)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmC, h, d_out, M, 64, 32)) return LORA_ERR_CUDA;
-    {
-        const MainSched ms = main_sched(M, d_out, std::min(c.info->sms, PLAN_SMS));
-        if (ms.tail_split > 1) {
-            const uint32_t rows = MAIN_BN / ms.tail_split;
-            if (!tmap_bf16(&a.tmB0n, W, d_in, d_out, 64, rows)) return LORA_ERR_CUDA;
-            if (!tmap_bf16(&a.tmB1n, B, r, d_out, 64, rows)) return LORA_ERR_CUDA;
-        }
-    }
-    return step_main(c, a, M, d_out, d_in, r, false, LORA_K_FWD_MAIN);
+    const MainOperands o{x, W, sxa, B, h};
+    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN);
 }
 
 lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
@@ -505,13 +648,9 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W,
     LORA_TRY(step_g(c, dY, B, M, d_out, r, s));
     const uint16_t *sg = reinterpret_cast<const uint16_t *>(c.ws + c.plan.g);
     if (dX) {
-        GemmArgs a = base_args(c);
-        if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
-        if (!tmap_bf16(&a.tmB0, W, d_in, d_out, 64, 64)) return LORA_ERR_CUDA;  // MN-major: d_in contiguous
-        if (!tmap_bf16(&a.tmA1, sg, r, M, 64, 128)) return LORA_ERR_CUDA;
-        if (!tmap_bf16(&a.tmB1, A, d_in, r, 64, 64)) return LORA_ERR_CUDA;      // MN-major: d_in contiguous
-        if (!tmap_bf16(&a.tmC, dX, d_in, M, 64, 32)) return LORA_ERR_CUDA;
-        LORA_TRY(step_main(c, a, M, d_in, d_out, r, true, LORA_K_DX_MAIN));
+        // W [d_out, d_in] and A [r, d_in] are read MN-major (d_in contiguous).
+        const MainOperands o{dY, W, sg, A, dX};
+        LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN));
     }
     LORA_TRY(step_db(c, dY, sxa, dB, M, d_out, r));
     LORA_TRY(step_da(c, x, sg, dA, M, d_in, d_out, r));

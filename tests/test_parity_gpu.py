@@ -189,6 +189,24 @@ def test_tail_wave_split(shape):
     compare_all(dl.results(), oracle_ref(inp), spec.s)
 
 
+@pytest.mark.parametrize("shape", [TAIL_WAVE[0], TAIL_WAVE[1], TAIL_WAVE[2]], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_single_sm_main_gemm(shape, monkeypatch):
+    """The single-SM main-GEMM kernel (chosen when CTA pairs are unavailable) on the
+    same tail-wave shapes, including its 2-way and 4-way N splits."""
+    monkeypatch.setenv("LORA_LINEAR_PAIR", "0")
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("single", M, di, do, r, alpha=2.0 * r, seed=0x77 + M + di)
+    inp, dl = _run_full(spec)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+def test_without_programmatic_launch(monkeypatch):
+    monkeypatch.setenv("LORA_LINEAR_PDL", "0")
+    spec = inputs.LayerSpec("nopdl", 520, 640, 768, 16, alpha=32.0, seed=0x99)
+    inp, dl = _run_full(spec)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
 # ------------------------------------------------------------------ full sizes
 FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0)]
 
