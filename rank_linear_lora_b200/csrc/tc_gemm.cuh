@@ -89,13 +89,18 @@ struct GemmArgs {
     int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
+    int l2_prefetch;         // main GEMMs: K blocks ahead to prefetch into L2 (0: off)
 };
 
 // Trace record of one CTA (globaltimer ns unless noted).
 enum TraceField {
     TR_ENTRY = 0, TR_SETUP = 1, TR_PROD_END = 2, TR_MMA_END = 3, TR_EPI_END = 4, TR_EXIT = 5,
     TR_SMID = 6, TR_TILES = 7, TR_TILE_DONE0 = 8,  // epilogue completion of the first 8 items
-    TRACE_WORDS = 16
+    TR_WAIT_EMPTY = 16,  // total ns the producer waited for free stages
+    TR_WAIT_FULL = 17,   // total ns the MMA issuer waited for loaded stages
+    TR_WAIT_TEMPTY = 18, // total ns the MMA issuer waited for a drained accumulator
+    TR_KBLOCKS = 19,     // K blocks consumed by the MMA issuer
+    TRACE_WORDS = 24
 };
 
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>

@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             uint32_t phase = 0;
             uint32_t issued_mask = 0, issued_phase = 0;
             bool ok = true;
+            uint64_t wait_empty_ns = 0;
             WorkItem w;
             for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
                 const int bn_cta = (PAIR_BN / w.nsplit) / 2;  // B rows this CTA stages
@@ -148,10 +149,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
                 const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    const uint64_t tw = trace ? globaltimer_ns() : 0;
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
                                       DERR_WAIT_EMPTY)) {
                         ok = false;
                         break;
+                    }
+                    if (trace) wait_empty_ns += globaltimer_ns() - tw;
+                    if (p.l2_prefetch > 0) {
+                        const int kp = kb + p.l2_prefetch;
+                        if (kp < p.kb0) {
+                            tma_prefetch_l2_2d(&p.tmA0, kp * BK, a_row);
+                            if (B_MN) {
+                                for (int j = 0; j < bn_cta / 64; ++j)
+                                    tma_prefetch_l2_2d(&p.tmB0, b_row + 64 * j, kp * BK);
+                            } else {
+                                tma_prefetch_l2_2d(w.nsplit == 1 ? &p.tmB0 : &p.tmB0n, kp * BK, b_row);
+                            }
+                        }
                     }
                     const uint32_t fb_local = smem_u32(&full_bar[stage]);
                     const uint32_t fb_leader = mapa_shared(fb_local, 0);
@@ -189,7 +204,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
                                      DERR_WAIT_DRAIN);
                     }
-            if (trace) trace[TR_PROD_END] = globaltimer_ns();
+            if (trace) {
+                trace[TR_PROD_END] = globaltimer_ns();
+                trace[TR_WAIT_EMPTY] = wait_empty_ns;
+            }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (leader)
@@ -203,22 +221,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
+            uint64_t wait_full_ns = 0, wait_tempty_ns = 0, kblocks = 0;
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
+                const uint64_t tt = trace ? globaltimer_ns() : 0;
                 if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
                                   DERR_WAIT_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
+                if (trace) wait_tempty_ns += globaltimer_ns() - tt;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PAIR_BN);
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : idesc_half;
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    const uint64_t tf = trace ? globaltimer_ns() : 0;
                     if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
+                    }
+                    if (trace) {
+                        wait_full_ns += globaltimer_ns() - tf;
+                        ++kblocks;
                     }
                     tc_fence_after();
                     const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
@@ -244,6 +270,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             if (trace) {
                 trace[TR_MMA_END] = globaltimer_ns();
                 trace[TR_TILES] = static_cast<unsigned long long>(it);
+                trace[TR_WAIT_FULL] = wait_full_ns;
+                trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
+                trace[TR_KBLOCKS] = kblocks;
             }
         }
     } else {
