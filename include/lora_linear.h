@@ -177,7 +177,8 @@ LORA_API lora_status_t lora_linear_timing_read(double *ms_per_kind, int64_t *lau
  * the end of the TMA producer, of the MMA issuer and of the epilogue, at exit; the SM
  * id; the tile count; the epilogue completion time of the CTA's first 8 tiles; then
  * (main GEMMs) the total ns the producer waited for free stages, the MMA issuer for
- * loaded stages and for a drained accumulator, and the K blocks it consumed.
+ * loaded stages and for a drained accumulator, and the K blocks it consumed; then the
+ * SM cycle counter after set-up and at exit (with the two ns stamps: the SM clock).
  * Launches whose grid does not fit their share of the buffer are not traced.  Pass
  * NULL to switch tracing off.  Returns LORA_OK or LORA_ERR_MISALIGNED (8 bytes). */
 LORA_API lora_status_t lora_linear_trace_enable(void *device_buffer, size_t bytes);

@@ -100,6 +100,8 @@ enum TraceField {
     TR_WAIT_FULL = 17,   // total ns the MMA issuer waited for loaded stages
     TR_WAIT_TEMPTY = 18, // total ns the MMA issuer waited for a drained accumulator
     TR_KBLOCKS = 19,     // K blocks consumed by the MMA issuer
+    TR_CLK_SETUP = 20,   // SM cycle counter after set-up
+    TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
     TRACE_WORDS = 24
 };
 
@@ -282,7 +284,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     // previous kernel in the stream wrote and overwrite what it read.
     grid_dep_wait();
     grid_dep_launch_dependents();
-    if (trace && threadIdx.x == 0) trace[TR_SETUP] = globaltimer_ns();
+    if (trace && threadIdx.x == 0) {
+        trace[TR_SETUP] = globaltimer_ns();
+        trace[TR_CLK_SETUP] = clock64();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -537,7 +542,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
-    if (trace && threadIdx.x == 0) trace[TR_EXIT] = globaltimer_ns();
+    if (trace && threadIdx.x == 0) {
+        trace[TR_EXIT] = globaltimer_ns();
+        trace[TR_CLK_EXIT] = clock64();
+    }
 }
 
 }  // namespace lora

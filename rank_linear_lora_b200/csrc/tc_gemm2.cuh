@@ -132,7 +132,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
     const uint32_t tmem_base = *tmem_slot;
     grid_dep_wait();
     grid_dep_launch_dependents();
-    if (trace && threadIdx.x == 0) trace[TR_SETUP] = globaltimer_ns();
+    if (trace && threadIdx.x == 0) {
+        trace[TR_SETUP] = globaltimer_ns();
+        trace[TR_CLK_SETUP] = clock64();
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer (both CTAs)
@@ -334,7 +337,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
         tc_fence_after();
         tmem_dealloc_pair(tmem_base, Cfg::TMEM_COLS);
     }
-    if (trace && threadIdx.x == 0) trace[TR_EXIT] = globaltimer_ns();
+    if (trace && threadIdx.x == 0) {
+        trace[TR_EXIT] = globaltimer_ns();
+        trace[TR_CLK_EXIT] = clock64();
+    }
 }
 
 }  // namespace lora
