@@ -546,6 +546,8 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     {
         const char *v = std::getenv("LORA_LINEAR_L2_PREFETCH");
         a.l2_prefetch = v ? std::atoi(v) : 0;
+        const char *vv = std::getenv("LORA_LINEAR_VARIANT");
+        a.variant = vv ? std::atoi(vv) : 0;
     }
     const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn), PLAN_SMS / 2) : 0;
     if (pair_C > 0) {

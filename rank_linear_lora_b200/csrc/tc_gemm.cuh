@@ -90,6 +90,7 @@ struct GemmArgs {
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
     int l2_prefetch;         // main GEMMs: K blocks ahead to prefetch into L2 (0: off)
+    int variant;             // measurement switches of the pair kernel (0: default)
 };
 
 // Trace record of one CTA (globaltimer ns unless noted).
@@ -102,6 +103,7 @@ enum TraceField {
     TR_KBLOCKS = 19,     // K blocks consumed by the MMA issuer
     TR_CLK_SETUP = 20,   // SM cycle counter after set-up
     TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
+    TR_MMA_ISSUE = 22,   // total ns the MMA issuer spent issuing MMAs and commits
     TRACE_WORDS = 24
 };
 

@@ -224,7 +224,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            uint64_t wait_full_ns = 0, wait_tempty_ns = 0, kblocks = 0;
+            uint64_t wait_full_ns = 0, wait_tempty_ns = 0, kblocks = 0, issue_ns = 0;
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
@@ -245,11 +245,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         ok = false;
                         break;
                     }
+                    const uint64_t ti = trace ? globaltimer_ns() : 0;
                     if (trace) {
-                        wait_full_ns += globaltimer_ns() - tf;
+                        wait_full_ns += ti - tf;
                         ++kblocks;
                     }
-                    tc_fence_after();
+                    if (!(p.variant & 1)) tc_fence_after();
                     const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
                     const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
                     }
                     tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+                    if (trace) issue_ns += globaltimer_ns() - ti;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -276,6 +278,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 trace[TR_WAIT_FULL] = wait_full_ns;
                 trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
                 trace[TR_KBLOCKS] = kblocks;
+                trace[TR_MMA_ISSUE] = issue_ns;
             }
         }
     } else {
