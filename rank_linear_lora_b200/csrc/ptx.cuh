@@ -98,19 +98,6 @@ __device__ __forceinline__ void grid_dep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// ---------------------------------------------------------------- warp helpers
-// True in exactly one lane of the (converged) warp.
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred = 0;
-    asm volatile(
-        "{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\t"
-        "elect.sync rx|px, %1;\n\t"
-        "@px mov.s32 %0, 1;\n\t}\n"
-        : "+r"(pred)
-        : "r"(0xffffffffu));
-    return pred != 0;
-}
-
 // ---------------------------------------------------------------- named barriers
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

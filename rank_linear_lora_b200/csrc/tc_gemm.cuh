@@ -145,16 +145,6 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 
 // One unit of work of a CTA: output tile (m, n), K blocks [kb_lo, kb_hi) of the
 // concatenated segments, and how its result is finished.
-// wait_bounded on lane 0, result broadcast: the whole warp takes the same path and
-// stays converged (role loops run on all 32 lanes so the operands of tcgen05/TMA
-// instructions are warp-uniform values).
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort_flag, int *err,
-                                          int code) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bounded(bar, parity, abort_flag, err, code) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 struct WorkItem {
     int m, n;
     int kb_lo, kb_hi;
@@ -302,29 +292,31 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     }
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer (whole warp, lane 0 issues)
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued?, parity of last issue
-        bool ok = true;
-        WorkItem w;
-        for (int i = 0; ok && get_item<BN, EPI>(p, i, w); ++i) {
-            const int bn = BN / w.nsplit;  // columns of B this item loads
-            const uint32_t tx = static_cast<uint32_t>(Cfg::A_BYTES + bn * BK * 2);
-            for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                if (!wait_warp(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, DERR_WAIT_EMPTY)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t fb = smem_u32(&full_bar[stage]);
-                const bool seg1 = kb >= p.kb0;
-                const CUtensorMap *ta = seg1 ? &p.tmA1 : &p.tmA0;
-                const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
-                const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
-                const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
-                const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, tx);
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_phase = 0;  // per stage: issued?, parity of last issue
+            bool ok = true;
+            WorkItem w;
+            for (int i = 0; ok && get_item<BN, EPI>(p, i, w); ++i) {
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
+                                      DERR_WAIT_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const int bn = BN / w.nsplit;  // columns of B this item loads
+                    mbar_arrive_expect_tx(fb, Cfg::A_BYTES + bn * BK * 2);
+                    issued_mask |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    const bool seg1 = kb >= p.kb0;
+                    const CUtensorMap *ta = seg1 ? &p.tmA1 : &p.tmA0;
+                    const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
+                    const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
+                    const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     if (A_MN) {
                         tma_load_2d(a_dst, ta, fb, w.m * BM, k0);
                         tma_load_2d(a_dst + 64 * 128, ta, fb, w.m * BM + 64, k0);
@@ -339,85 +331,81 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                     } else {
                         tma_load_2d(b_dst, seg1 ? &p.tmB1n : &p.tmB0n, fb, k0, w.col0);
                     }
-                }
-                __syncwarp();
-                issued_mask |= 1u << stage;
-                issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
+            // Drain: every issued copy must have landed before the CTA exits.
+            for (int s = 0; s < STAGES; ++s)
+                if (issued_mask & (1u << s)) {
+                    volatile int never = 0;
+                    wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
+                                 DERR_WAIT_DRAIN);
+                }
+            if (trace) trace[TR_PROD_END] = globaltimer_ns();
         }
-        // Drain: every issued copy must have landed before the CTA exits.
-        for (int s = 0; s < STAGES; ++s)
-            if (issued_mask & (1u << s)) {
-                volatile int never = 0;
-                wait_warp(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err, DERR_WAIT_DRAIN);
-            }
-        if (trace && lane == 0) trace[TR_PROD_END] = globaltimer_ns();
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (whole warp, lane 0 issues)
-        constexpr uint32_t idesc_full = idesc_bf16(BM, BN, A_MN, B_MN);
-        constexpr uint32_t idesc_half = idesc_bf16(BM, BN >= 128 ? BN / 2 : BN, A_MN, B_MN);
-        constexpr uint32_t idesc_quarter = idesc_bf16(BM, BN >= 256 ? BN / 4 : BN, A_MN, B_MN);
-        // K step of 16 elements inside a stage: +32 B along a K-major row,
-        // +16 rows (2 swizzle atoms) for an MN-major tile.
-        constexpr uint32_t a_kstep = A_MN ? 2048u : 32u;
-        constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
-        constexpr uint32_t a_lbo = A_MN ? 64u * 128u : 16u;
-        constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
-        const int kb_last = p.kb0 + p.kb1 - 1;
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        bool ok = true;
-        WorkItem w;
-        for (; ok && get_item<BN, EPI>(p, it, w); ++it) {
-            const int buf = it & 1;
-            const uint32_t aphase = (it >> 1) & 1;
-            if (!wait_warp(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err, DERR_WAIT_TMEM_EMPTY)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
-            const uint32_t idesc = w.nsplit == 1 ? idesc_full : (w.nsplit == 2 ? idesc_half : idesc_quarter);
-            for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                if (!wait_warp(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_full = idesc_bf16(BM, BN, A_MN, B_MN);
+            constexpr uint32_t idesc_half = idesc_bf16(BM, BN >= 128 ? BN / 2 : BN, A_MN, B_MN);
+            constexpr uint32_t idesc_quarter = idesc_bf16(BM, BN >= 256 ? BN / 4 : BN, A_MN, B_MN);
+            // K step of 16 elements inside a stage: +32 B along a K-major row,
+            // +16 rows (2 swizzle atoms) for an MN-major tile.
+            constexpr uint32_t a_kstep = A_MN ? 2048u : 32u;
+            constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
+            constexpr uint32_t a_lbo = A_MN ? 64u * 128u : 16u;
+            constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
+            const int kb_last = p.kb0 + p.kb1 - 1;
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            bool ok = true;
+            WorkItem w;
+            for (; ok && get_item<BN, EPI>(p, it, w); ++it) {
+                const int buf = it & 1;
+                const uint32_t aphase = (it >> 1) & 1;
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
+                                  DERR_WAIT_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
-                const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
-                const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
-                if (lane == 0) {
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t idesc = w.nsplit == 1 ? idesc_full : (w.nsplit == 2 ? idesc_half : idesc_quarter);
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
+                    const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
                     for (int kk = 0; kk < nmma; ++kk) {
                         const uint64_t ad = sdesc_sw128(a_base + kk * a_kstep, a_lbo, 1024);
                         const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
                         tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&empty_bar[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
-                __syncwarp();
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                if (!ok) break;
+                tc_commit(smem_u32(&tfull_bar[buf]));
             }
-            if (!ok) break;
-            if (lane == 0) tc_commit(smem_u32(&tfull_bar[buf]));
-            __syncwarp();
-        }
-        // Drain: all MMAs issued by lane 0 complete before TMEM is freed.
-        if (lane == 0) tc_commit(smem_u32(drain_bar));
-        __syncwarp();
-        volatile int never = 0;
-        wait_warp(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
-        if (trace && lane == 0) {
-            trace[TR_MMA_END] = globaltimer_ns();
-            trace[TR_TILES] = static_cast<unsigned long long>(it);
+            // Drain: all MMAs issued by this thread complete before TMEM is freed.
+            tc_commit(smem_u32(drain_bar));
+            volatile int never = 0;
+            wait_bounded(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
+            if (trace) {
+                trace[TR_MMA_END] = globaltimer_ns();
+                trace[TR_TILES] = static_cast<unsigned long long>(it);
+            }
         }
     } else {
         // ------------------------------------------------------------ epilogue

@@ -138,32 +138,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
     }
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer (both CTAs; whole warp, lane 0 issues)
-        int stage = 0;
-        uint32_t phase = 0;
-        uint32_t issued_mask = 0, issued_phase = 0;
-        bool ok = true;
-        uint64_t wait_empty_ns = 0;
-        WorkItem w;
-        for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
-            const int bn_cta = (PAIR_BN / w.nsplit) / 2;  // B rows this CTA stages
-            const int a_row = w.m * PAIR_BM + static_cast<int>(rank) * 128;
-            const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
-            const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
-            for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                const uint64_t tw = trace ? globaltimer_ns() : 0;
-                if (!wait_warp(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err, DERR_WAIT_EMPTY)) {
-                    ok = false;
-                    break;
-                }
-                if (trace) wait_empty_ns += globaltimer_ns() - tw;
-                const uint32_t fb_local = smem_u32(&full_bar[stage]);
-                const uint32_t fb_leader = mapa_shared(fb_local, 0);
-                const bool seg1 = kb >= p.kb0;
-                const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
-                const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
-                const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
-                if (lane == 0) {
+        // ------------------------------------------------------------ TMA producer (both CTAs)
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued_mask = 0, issued_phase = 0;
+            bool ok = true;
+            uint64_t wait_empty_ns = 0;
+            WorkItem w;
+            for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
+                const int bn_cta = (PAIR_BN / w.nsplit) / 2;  // B rows this CTA stages
+                const int a_row = w.m * PAIR_BM + static_cast<int>(rank) * 128;
+                const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
+                const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    const uint64_t tw = trace ? globaltimer_ns() : 0;
+                    if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
+                                      DERR_WAIT_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    if (trace) wait_empty_ns += globaltimer_ns() - tw;
                     if (p.l2_prefetch > 0) {
                         const int kp = kb + p.l2_prefetch;
                         if (kp < p.kb0) {
@@ -176,7 +171,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                             }
                         }
                     }
-                    if (leader) mbar_arrive_expect_tx(fb_local, tx);
+                    const uint32_t fb_local = smem_u32(&full_bar[stage]);
+                    const uint32_t fb_leader = mapa_shared(fb_local, 0);
+                    if (leader) {
+                        mbar_arrive_expect_tx(fb_local, tx);
+                        issued_mask |= 1u << stage;
+                        issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    }
+                    const bool seg1 = kb >= p.kb0;
+                    const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
+                    const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
+                    const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     tma_load_2d_pair(a_dst, seg1 ? &p.tmA1 : &p.tmA0, fb_leader, k0, a_row);
                     if (B_MN) {
                         const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
@@ -187,32 +192,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                                                               : (seg1 ? &p.tmB1n : &p.tmB0n);
                         tma_load_2d_pair(b_dst, tb, fb_leader, k0, b_row);
                     }
-                }
-                __syncwarp();
-                if (leader) {
-                    issued_mask |= 1u << stage;
-                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                }
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1u;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
                 }
             }
-        }
-        // Drain (leader): every copy of the pair has landed before either CTA leaves
-        // (the teardown cluster barrier orders the partner's exit after this).
-        for (int s = 0; s < STAGES; ++s)
-            if (issued_mask & (1u << s)) {
-                volatile int never = 0;
-                wait_warp(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err, DERR_WAIT_DRAIN);
+            // Drain (leader): every copy of the pair has landed before either CTA leaves
+            // (the teardown cluster barrier orders the partner's exit after this).
+            if (leader)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued_mask & (1u << s)) {
+                        volatile int never = 0;
+                        wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
+                                     DERR_WAIT_DRAIN);
+                    }
+            if (trace) {
+                trace[TR_PROD_END] = globaltimer_ns();
+                trace[TR_WAIT_EMPTY] = wait_empty_ns;
             }
-        if (trace && lane == 0) {
-            trace[TR_PROD_END] = globaltimer_ns();
-            trace[TR_WAIT_EMPTY] = wait_empty_ns;
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer (leader; whole warp, lane 0 issues)
-        if (leader) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && leader) {
             constexpr uint32_t idesc_full = idesc_bf16(PAIR_BM, PAIR_BN, false, B_MN);
             constexpr uint32_t idesc_half = idesc_bf16(PAIR_BM, PAIR_BN / 2, false, B_MN);
             constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
@@ -228,7 +230,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 const int buf = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
                 const uint64_t tt = trace ? globaltimer_ns() : 0;
-                if (!wait_warp(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err, DERR_WAIT_TMEM_EMPTY)) {
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
+                                  DERR_WAIT_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
@@ -238,7 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : idesc_half;
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     const uint64_t tf = trace ? globaltimer_ns() : 0;
-                    if (!wait_warp(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
@@ -251,15 +254,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                     const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
                     const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
-                    if (lane == 0) {
-                        for (int kk = 0; kk < nmma; ++kk) {
-                            const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
-                            const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
-                            tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
-                        }
-                        tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+                    for (int kk = 0; kk < nmma; ++kk) {
+                        const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
+                        const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
+                        tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
                     }
-                    __syncwarp();
+                    tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
                     if (trace) issue_ns += globaltimer_ns() - ti;
                     if (++stage == STAGES) {
                         stage = 0;
@@ -267,14 +267,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                     }
                 }
                 if (!ok) break;
-                if (lane == 0) tc_commit_pair_mc(smem_u32(&tfull_bar[buf]), 0x3);
-                __syncwarp();
+                tc_commit_pair_mc(smem_u32(&tfull_bar[buf]), 0x3);
             }
-            if (lane == 0) tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
-            __syncwarp();
+            tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
             volatile int never = 0;
-            wait_warp(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
-            if (trace && lane == 0) {
+            wait_bounded(smem_u32(drain_bar), 0, &never, p.err, DERR_WAIT_DRAIN);
+            if (trace) {
                 trace[TR_MMA_END] = globaltimer_ns();
                 trace[TR_TILES] = static_cast<unsigned long long>(it);
                 trace[TR_WAIT_FULL] = wait_full_ns;
