@@ -104,7 +104,12 @@ enum TraceField {
     TR_CLK_SETUP = 20,   // SM cycle counter after set-up
     TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
     TR_MMA_ISSUE = 22,   // total ns the MMA issuer spent issuing MMAs and commits
-    TRACE_WORDS = 24
+    TR_CYC_WAIT = 23,    // MMA issuer cycles: waiting + fence before the first MMA of a block
+    TR_CYC_MMA0 = 24,    // cycles spent in the first MMA instruction of each block
+    TR_CYC_MMAR = 25,    // cycles spent in the remaining MMA instructions
+    TR_CYC_COMMIT = 26,  // cycles spent in the stage commit
+    TR_CYC_LOOP = 27,    // cycles from the commit to the next block's wait
+    TRACE_WORDS = 32
 };
 
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>

@@ -225,6 +225,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             int it = 0;
             bool ok = true;
             uint64_t wait_full_ns = 0, wait_tempty_ns = 0, kblocks = 0, issue_ns = 0;
+            long long cyc_wait = 0, cyc_mma0 = 0, cyc_mmar = 0, cyc_commit = 0, cyc_loop = 0;
+            long long c_prev = clock64();
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
@@ -240,27 +242,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PAIR_BN);
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : idesc_half;
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                    const uint64_t tf = trace ? globaltimer_ns() : 0;
+                    const long long c0 = clock64();
+                    if (trace) cyc_loop += c0 - c_prev;
                     if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
-                    const uint64_t ti = trace ? globaltimer_ns() : 0;
-                    if (trace) {
-                        wait_full_ns += ti - tf;
-                        ++kblocks;
-                    }
+                    if (trace) ++kblocks;
                     if (!(p.variant & 1)) tc_fence_after();
                     const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
                     const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
+                    const long long c1 = clock64();
+                    long long c2 = c1;
                     for (int kk = 0; kk < nmma; ++kk) {
                         const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
                         const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
                         tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
+                        if (kk == 0) c2 = clock64();
                     }
+                    const long long c3 = clock64();
                     tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
-                    if (trace) issue_ns += globaltimer_ns() - ti;
+                    const long long c4 = clock64();
+                    if (trace) {
+                        cyc_wait += c1 - c0;
+                        cyc_mma0 += c2 - c1;
+                        cyc_mmar += c3 - c2;
+                        cyc_commit += c4 - c3;
+                    }
+                    c_prev = c4;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -279,6 +289,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
                 trace[TR_KBLOCKS] = kblocks;
                 trace[TR_MMA_ISSUE] = issue_ns;
+                trace[TR_CYC_WAIT] = cyc_wait;
+                trace[TR_CYC_MMA0] = cyc_mma0;
+                trace[TR_CYC_MMAR] = cyc_mmar;
+                trace[TR_CYC_COMMIT] = cyc_commit;
+                trace[TR_CYC_LOOP] = cyc_loop;
             }
         }
     } else {

@@ -208,7 +208,7 @@ def lora_linear_timing_read():
     return {k: (ms[i], int(cnt[i])) for i, k in enumerate(KERNEL_KINDS)}
 
 
-TRACE_WORDS = 24
+TRACE_WORDS = 32
 TRACE_FIELDS = ["entry", "setup", "prod_end", "mma_end", "epi_end", "exit", "smid", "tiles"]
 
 
