@@ -241,28 +241,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PAIR_BN);
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : idesc_half;
-                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                for (int kb = w.kb_lo; kb < w.kb_hi;) {
+                    // Blocks consumed per barrier round: 2 when allowed (fewer waits and
+                    // loop trips per MMA), else 1.
+                    const int nblk = ((p.variant & 2) && kb + 1 < w.kb_hi) ? 2 : 1;
                     const long long c0 = clock64();
                     if (trace) cyc_loop += c0 - c_prev;
                     if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
-                    if (trace) ++kblocks;
+                    const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
+                    const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
+                    if (nblk == 2 &&
+                        !wait_bounded(smem_u32(&full_bar[stage2]), phase2, abort_flag, p.err, DERR_WAIT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    if (trace) kblocks += nblk;
                     if (!(p.variant & 1)) tc_fence_after();
-                    const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
-                    const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
-                    const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
                     const long long c1 = clock64();
                     long long c2 = c1;
-                    for (int kk = 0; kk < nmma; ++kk) {
-                        const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
-                        const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
-                        tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
-                        if (kk == 0) c2 = clock64();
+                    for (int b = 0; b < nblk; ++b) {
+                        const int st = b == 0 ? stage : stage2;
+                        const int kbb = kb + b;
+                        const uint32_t a_base = smem_u32(sA + st * Cfg::A_BYTES);
+                        const uint32_t b_base = smem_u32(sB + st * Cfg::B_BYTES);
+                        const bool full4 = !(p.kb1 > 0 && kbb == kb_last);
+                        if ((p.variant & 4) && full4) {
+                            const uint64_t ad0 = sdesc_sw128(a_base, 16u, 1024);
+                            const uint64_t bd0 = sdesc_sw128(b_base, b_lbo, 1024);
+                            const uint32_t acc0 = (kbb > w.kb_lo) ? 1u : 0u;
+                            tc_mma_bf16_pair(d_tmem, ad0, bd0, idesc, acc0);
+                            if (b == 0) c2 = clock64();
+                            tc_mma_bf16_pair(d_tmem, ad0 + (32u >> 4), bd0 + (b_kstep >> 4), idesc, 1u);
+                            tc_mma_bf16_pair(d_tmem, ad0 + (64u >> 4), bd0 + ((2 * b_kstep) >> 4), idesc, 1u);
+                            tc_mma_bf16_pair(d_tmem, ad0 + (96u >> 4), bd0 + ((3 * b_kstep) >> 4), idesc, 1u);
+                        } else {
+                            const int nmma = full4 ? BK / 16 : p.mma_last1;
+                            for (int kk = 0; kk < nmma; ++kk) {
+                                const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
+                                const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
+                                tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kbb > w.kb_lo || kk > 0) ? 1u : 0u);
+                                if (b == 0 && kk == 0) c2 = clock64();
+                            }
+                        }
                     }
                     const long long c3 = clock64();
                     tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+                    if (nblk == 2) tc_commit_pair_mc(smem_u32(&empty_bar[stage2]), 0x3);
                     const long long c4 = clock64();
                     if (trace) {
                         cyc_wait += c1 - c0;
@@ -271,9 +298,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         cyc_commit += c4 - c3;
                     }
                     c_prev = c4;
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
+                    kb += nblk;
+                    for (int b = 0; b < nblk; ++b) {
+                        if (++stage == STAGES) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
                     }
                 }
                 if (!ok) break;
