@@ -10,8 +10,10 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblora_linear.so")
 SOURCES = [os.path.join(CSRC, "lora_linear.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("ptx.cuh", "tc_gemm.cuh")] + [
-    os.path.join(ROOT, "include", "lora_linear.h")]
+def deps() -> list:
+    """Every source the library is built from (all of csrc/ and the public header)."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))) + [
+        os.path.join(ROOT, "include", "lora_linear.h"), os.path.abspath(__file__)]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -32,7 +34,7 @@ def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    return any(os.path.getmtime(p) > t for p in DEPS if os.path.exists(p))
+    return any(os.path.getmtime(p) > t for p in deps() if os.path.exists(p))
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
