@@ -175,13 +175,11 @@ LORA_API lora_status_t lora_linear_timing_read(double *ms_per_kind, int64_t *lau
  * kernel kind k writes, for each of its CTAs c, 32 uint64 words at word offset
  * k * (bytes / 8 / LORA_K_COUNT) + 32 * c: globaltimer ns at entry, after set-up, at
  * the end of the TMA producer, of the MMA issuer and of the epilogue, at exit; the SM
- * id; the tile count; the epilogue completion time of the CTA's first 8 tiles; then
- * (main GEMMs) the total ns the producer waited for free stages, the MMA issuer for
- * loaded stages and for a drained accumulator, and the K blocks it consumed; then the
- * SM cycle counter after set-up and at exit (with the two ns stamps: the SM clock);
- * the MMA issuer's ns in its issue sections; and its cycles spent waiting (plus the
- * fence) before a block's first MMA, in the first MMA instruction, in the remaining
- * MMA instructions, in the stage commit, and between a commit and the next wait.
+ * id; the tile count; the epilogue completion time of the CTA's first 8 tiles
+ * (words 8-15); for the main GEMMs the total ns the producer waited for free stages
+ * (16), the ns the MMA issuer waited for a drained accumulator (18) and the K blocks
+ * it consumed (19); the SM cycle counter after set-up (20) and at exit (21), which
+ * with the two ns stamps give the SM clock.
  * Launches whose grid does not fit their share of the buffer are not traced.  Pass
  * NULL to switch tracing off.  Returns LORA_OK or LORA_ERR_MISALIGNED (8 bytes). */
 LORA_API lora_status_t lora_linear_trace_enable(void *device_buffer, size_t bytes);

@@ -543,12 +543,6 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     if (!tmap_bf16(&a.tmA0, o.A0, K0, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmA1, o.A1, r, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmC, o.C, N, M, 64, 32)) return LORA_ERR_CUDA;
-    {
-        const char *v = std::getenv("LORA_LINEAR_L2_PREFETCH");
-        a.l2_prefetch = v ? std::atoi(v) : 0;
-        const char *vv = std::getenv("LORA_LINEAR_VARIANT");
-        a.variant = vv ? std::atoi(vv) : 0;
-    }
     const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn), PLAN_SMS / 2) : 0;
     if (pair_C > 0) {
         // CTA pairs: 256 x 256 tiles, each CTA stages 128 rows of B.

@@ -89,8 +89,6 @@ struct GemmArgs {
     int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
-    int l2_prefetch;         // main GEMMs: K blocks ahead to prefetch into L2 (0: off)
-    int variant;             // measurement switches of the pair kernel (0: default)
 };
 
 // Trace record of one CTA (globaltimer ns unless noted).
@@ -98,17 +96,10 @@ enum TraceField {
     TR_ENTRY = 0, TR_SETUP = 1, TR_PROD_END = 2, TR_MMA_END = 3, TR_EPI_END = 4, TR_EXIT = 5,
     TR_SMID = 6, TR_TILES = 7, TR_TILE_DONE0 = 8,  // epilogue completion of the first 8 items
     TR_WAIT_EMPTY = 16,  // total ns the producer waited for free stages
-    TR_WAIT_FULL = 17,   // total ns the MMA issuer waited for loaded stages
     TR_WAIT_TEMPTY = 18, // total ns the MMA issuer waited for a drained accumulator
     TR_KBLOCKS = 19,     // K blocks consumed by the MMA issuer
     TR_CLK_SETUP = 20,   // SM cycle counter after set-up
     TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
-    TR_MMA_ISSUE = 22,   // total ns the MMA issuer spent issuing MMAs and commits
-    TR_CYC_WAIT = 23,    // MMA issuer cycles: waiting + fence before the first MMA of a block
-    TR_CYC_MMA0 = 24,    // cycles spent in the first MMA instruction of each block
-    TR_CYC_MMAR = 25,    // cycles spent in the remaining MMA instructions
-    TR_CYC_COMMIT = 26,  // cycles spent in the stage commit
-    TR_CYC_LOOP = 27,    // cycles from the commit to the next block's wait
     TRACE_WORDS = 32
 };
 
@@ -357,12 +348,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
             constexpr uint32_t idesc_full = idesc_bf16(BM, BN, A_MN, B_MN);
             constexpr uint32_t idesc_half = idesc_bf16(BM, BN >= 128 ? BN / 2 : BN, A_MN, B_MN);
             constexpr uint32_t idesc_quarter = idesc_bf16(BM, BN >= 256 ? BN / 4 : BN, A_MN, B_MN);
-            // K step of 16 elements inside a stage: +32 B along a K-major row,
-            // +16 rows (2 swizzle atoms) for an MN-major tile.
-            constexpr uint32_t a_kstep = A_MN ? 2048u : 32u;
-            constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
+            // Descriptor fields advance in 16-byte units: K step of 16 elements is +32 B
+            // along a K-major row, +16 rows (2 swizzle atoms) in an MN-major tile.
+            constexpr uint64_t a_kstep = (A_MN ? 2048u : 32u) >> 4;
+            constexpr uint64_t b_kstep = (B_MN ? 2048u : 32u) >> 4;
             constexpr uint32_t a_lbo = A_MN ? 64u * 128u : 16u;
             constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
+            const uint64_t ad_base = sdesc_sw128(smem_u32(sA), a_lbo, 1024);
+            const uint64_t bd_base = sdesc_sw128(smem_u32(sB), b_lbo, 1024);
             const int kb_last = p.kb0 + p.kb1 - 1;
             int stage = 0;
             uint32_t phase = 0;
@@ -380,25 +373,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : (w.nsplit == 2 ? idesc_half : idesc_quarter);
+                // Lean K loop: one try_wait on the fast path, constant-offset descriptors,
+                // unrolled MMAs; the issue rate must keep pace with the tensor pipe.
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_try_wait(fb, phase) &&
+                        !wait_bounded(fb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nmma = (p.kb1 > 0 && kb == kb_last) ? p.mma_last1 : BK / 16;
-                    const uint32_t a_base = smem_u32(sA + stage * Cfg::A_BYTES);
-                    const uint32_t b_base = smem_u32(sB + stage * Cfg::B_BYTES);
-                    for (int kk = 0; kk < nmma; ++kk) {
-                        const uint64_t ad = sdesc_sw128(a_base + kk * a_kstep, a_lbo, 1024);
-                        const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
-                        tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > w.kb_lo || kk > 0) ? 1u : 0u);
+                    const uint64_t ad = ad_base + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
+                    const uint64_t bd = bd_base + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
+                    const uint32_t acc0 = kb > w.kb_lo ? 1u : 0u;
+                    if (kb != kb_last || p.kb1 == 0) {
+                        tc_mma_bf16(d_tmem, ad, bd, idesc, acc0);
+                        tc_mma_bf16(d_tmem, ad + a_kstep, bd + b_kstep, idesc, 1u);
+                        tc_mma_bf16(d_tmem, ad + 2 * a_kstep, bd + 2 * b_kstep, idesc, 1u);
+                        tc_mma_bf16(d_tmem, ad + 3 * a_kstep, bd + 3 * b_kstep, idesc, 1u);
+                    } else {
+                        // last block of the rank-r segment: only ceil(r_tail / 16) MMAs
+                        for (int kk = 0; kk < p.mma_last1; ++kk)
+                            tc_mma_bf16(d_tmem, ad + kk * a_kstep, bd + kk * b_kstep, idesc, (acc0 | kk) ? 1u : 0u);
                     }
                     tc_commit(smem_u32(&empty_bar[stage]));
-                    if (++stage == STAGES) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    stage = stage + 1 == STAGES ? 0 : stage + 1;
+                    phase = stage == 0 ? phase ^ 1u : phase;
                 }
                 if (!ok) break;
                 tc_commit(smem_u32(&tfull_bar[buf]));

@@ -159,18 +159,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         break;
                     }
                     if (trace) wait_empty_ns += globaltimer_ns() - tw;
-                    if (p.l2_prefetch > 0) {
-                        const int kp = kb + p.l2_prefetch;
-                        if (kp < p.kb0) {
-                            tma_prefetch_l2_2d(&p.tmA0, kp * BK, a_row);
-                            if (B_MN) {
-                                for (int j = 0; j < bn_cta / 64; ++j)
-                                    tma_prefetch_l2_2d(&p.tmB0, b_row + 64 * j, kp * BK);
-                            } else {
-                                tma_prefetch_l2_2d(w.nsplit == 1 ? &p.tmB0 : &p.tmB0n, kp * BK, b_row);
-                            }
-                        }
-                    }
                     const uint32_t fb_local = smem_u32(&full_bar[stage]);
                     const uint32_t fb_leader = mapa_shared(fb_local, 0);
                     if (leader) {
@@ -217,23 +205,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
         if (lane == 0 && leader) {
             constexpr uint32_t idesc_full = idesc_bf16(PAIR_BM, PAIR_BN, false, B_MN);
             constexpr uint32_t idesc_half = idesc_bf16(PAIR_BM, PAIR_BN / 2, false, B_MN);
-            constexpr uint32_t b_kstep = B_MN ? 2048u : 32u;
+            // Descriptor fields advance in 16-byte units: K step of 16 elements is +32 B
+            // along a K-major row, +16 rows (2 swizzle atoms) in an MN-major tile.
+            constexpr uint64_t a_kstep = 32u >> 4;
+            constexpr uint64_t b_kstep = (B_MN ? 2048u : 32u) >> 4;
             constexpr uint32_t b_lbo = B_MN ? 64u * 128u : 16u;
+            const uint64_t ad_base = sdesc_sw128(smem_u32(sA), 16u, 1024);
+            const uint64_t bd_base = sdesc_sw128(smem_u32(sB), b_lbo, 1024);
             const int kb_last = p.kb0 + p.kb1 - 1;
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
             bool ok = true;
-            uint64_t wait_full_ns = 0, wait_tempty_ns = 0, kblocks = 0, issue_ns = 0;
-            long long cyc_wait = 0, cyc_mma0 = 0, cyc_mmar = 0, cyc_commit = 0, cyc_loop = 0;
-            long long c_prev = clock64();
+            uint64_t wait_tempty_ns = 0, kblocks = 0;
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
                 const uint32_t aphase = (it >> 1) & 1;
                 const uint64_t tt = trace ? globaltimer_ns() : 0;
-                if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err,
-                                  DERR_WAIT_TMEM_EMPTY)) {
+                if (!wait_bounded(smem_u32(&tempty_bar[buf]), aphase ^ 1u, abort_flag, p.err, DERR_WAIT_TMEM_EMPTY)) {
                     ok = false;
                     break;
                 }
@@ -241,72 +231,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * PAIR_BN);
                 const uint32_t idesc = w.nsplit == 1 ? idesc_full : idesc_half;
-                for (int kb = w.kb_lo; kb < w.kb_hi;) {
-                    // Blocks consumed per barrier round: 2 when allowed (fewer waits and
-                    // loop trips per MMA), else 1.
-                    const int nblk = ((p.variant & 2) && kb + 1 < w.kb_hi) ? 2 : 1;
-                    const long long c0 = clock64();
-                    if (trace) cyc_loop += c0 - c_prev;
-                    if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                // Lean K loop: one try_wait on the fast path, constant-offset descriptors,
+                // unrolled MMAs; the issue rate must keep pace with the tensor pipe.
+                for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    if (!mbar_try_wait(fb, phase) &&
+                        !wait_bounded(fb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
-                    const int stage2 = stage + 1 == STAGES ? 0 : stage + 1;
-                    const uint32_t phase2 = stage + 1 == STAGES ? phase ^ 1u : phase;
-                    if (nblk == 2 &&
-                        !wait_bounded(smem_u32(&full_bar[stage2]), phase2, abort_flag, p.err, DERR_WAIT_FULL)) {
-                        ok = false;
-                        break;
+                    tc_fence_after();
+                    const uint64_t ad = ad_base + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
+                    const uint64_t bd = bd_base + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
+                    const uint32_t acc0 = kb > w.kb_lo ? 1u : 0u;
+                    if (kb != kb_last || p.kb1 == 0) {
+                        tc_mma_bf16_pair(d_tmem, ad, bd, idesc, acc0);
+                        tc_mma_bf16_pair(d_tmem, ad + a_kstep, bd + b_kstep, idesc, 1u);
+                        tc_mma_bf16_pair(d_tmem, ad + 2 * a_kstep, bd + 2 * b_kstep, idesc, 1u);
+                        tc_mma_bf16_pair(d_tmem, ad + 3 * a_kstep, bd + 3 * b_kstep, idesc, 1u);
+                    } else {
+                        // last block of the rank-r segment: only ceil(r_tail / 16) MMAs
+                        for (int kk = 0; kk < p.mma_last1; ++kk)
+                            tc_mma_bf16_pair(d_tmem, ad + kk * a_kstep, bd + kk * b_kstep, idesc,
+                                             (acc0 | kk) ? 1u : 0u);
                     }
-                    if (trace) kblocks += nblk;
-                    if (!(p.variant & 1)) tc_fence_after();
-                    const long long c1 = clock64();
-                    long long c2 = c1;
-                    for (int b = 0; b < nblk; ++b) {
-                        const int st = b == 0 ? stage : stage2;
-                        const int kbb = kb + b;
-                        const uint32_t a_base = smem_u32(sA + st * Cfg::A_BYTES);
-                        const uint32_t b_base = smem_u32(sB + st * Cfg::B_BYTES);
-                        const bool full4 = !(p.kb1 > 0 && kbb == kb_last);
-                        if ((p.variant & 4) && full4) {
-                            const uint64_t ad0 = sdesc_sw128(a_base, 16u, 1024);
-                            const uint64_t bd0 = sdesc_sw128(b_base, b_lbo, 1024);
-                            const uint32_t acc0 = (kbb > w.kb_lo) ? 1u : 0u;
-                            tc_mma_bf16_pair(d_tmem, ad0, bd0, idesc, acc0);
-                            if (b == 0) c2 = clock64();
-                            tc_mma_bf16_pair(d_tmem, ad0 + (32u >> 4), bd0 + (b_kstep >> 4), idesc, 1u);
-                            tc_mma_bf16_pair(d_tmem, ad0 + (64u >> 4), bd0 + ((2 * b_kstep) >> 4), idesc, 1u);
-                            tc_mma_bf16_pair(d_tmem, ad0 + (96u >> 4), bd0 + ((3 * b_kstep) >> 4), idesc, 1u);
-                        } else {
-                            const int nmma = full4 ? BK / 16 : p.mma_last1;
-                            for (int kk = 0; kk < nmma; ++kk) {
-                                const uint64_t ad = sdesc_sw128(a_base + kk * 32u, 16u, 1024);
-                                const uint64_t bd = sdesc_sw128(b_base + kk * b_kstep, b_lbo, 1024);
-                                tc_mma_bf16_pair(d_tmem, ad, bd, idesc, (kbb > w.kb_lo || kk > 0) ? 1u : 0u);
-                                if (b == 0 && kk == 0) c2 = clock64();
-                            }
-                        }
-                    }
-                    const long long c3 = clock64();
                     tc_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
-                    if (nblk == 2) tc_commit_pair_mc(smem_u32(&empty_bar[stage2]), 0x3);
-                    const long long c4 = clock64();
-                    if (trace) {
-                        cyc_wait += c1 - c0;
-                        cyc_mma0 += c2 - c1;
-                        cyc_mmar += c3 - c2;
-                        cyc_commit += c4 - c3;
-                    }
-                    c_prev = c4;
-                    kb += nblk;
-                    for (int b = 0; b < nblk; ++b) {
-                        if (++stage == STAGES) {
-                            stage = 0;
-                            phase ^= 1u;
-                        }
-                    }
+                    stage = stage + 1 == STAGES ? 0 : stage + 1;
+                    phase = stage == 0 ? phase ^ 1u : phase;
                 }
                 if (!ok) break;
+                kblocks += static_cast<uint64_t>(w.kb_hi - w.kb_lo);
                 tc_commit_pair_mc(smem_u32(&tfull_bar[buf]), 0x3);
             }
             tc_commit_pair_mc(smem_u32(drain_bar), 0x1);
@@ -315,15 +269,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             if (trace) {
                 trace[TR_MMA_END] = globaltimer_ns();
                 trace[TR_TILES] = static_cast<unsigned long long>(it);
-                trace[TR_WAIT_FULL] = wait_full_ns;
                 trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
                 trace[TR_KBLOCKS] = kblocks;
-                trace[TR_MMA_ISSUE] = issue_ns;
-                trace[TR_CYC_WAIT] = cyc_wait;
-                trace[TR_CYC_MMA0] = cyc_mma0;
-                trace[TR_CYC_MMAR] = cyc_mmar;
-                trace[TR_CYC_COMMIT] = cyc_commit;
-                trace[TR_CYC_LOOP] = cyc_loop;
             }
         }
     } else {
