@@ -3,7 +3,7 @@
 
 One step = lora_linear_fwd + lora_linear_bwd of one layer over one batch of
 synthetic tokens (every row of the hot path: s.xa, the forward main GEMM, s.g,
-the dX GEMM, dB, dA).  Default workload: the attention-projection layer,
+the dX GEMM, and dB with dA).  Default workload: the attention-projection layer,
 M = 4096 tokens (2 x 2048), d_in = d_out = 4096, r = 8, alpha = 32.
 
 Timing: W untimed warm-up steps; then, behind a GPU sleep that lets the host

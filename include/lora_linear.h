@@ -155,9 +155,9 @@ typedef enum {
     LORA_K_FWD_MAIN = 1, /* forward main GEMM: [x | s.xa].[W | B]^T                 */
     LORA_K_G = 2,        /* backward prologue: bf16(s . dY.B), split over d_out     */
     LORA_K_DX_MAIN = 3,  /* backward main GEMM: [dY | s.g].[W ; A]                  */
-    LORA_K_DB = 4,       /* dB = dY^T.(s.xa), split over tokens                     */
-    LORA_K_DA = 5,       /* dA = (s.g)^T.x, split over tokens                       */
-    LORA_K_COUNT = 6
+    LORA_K_DADB = 4,     /* dB = dY^T.(s.xa) and dA = (s.g)^T.x in one launch, each
+                            split over tokens; runs beside the dX GEMM's last wave  */
+    LORA_K_COUNT = 5
 } lora_kernel_kind_t;
 
 /* Total kernels this library has launched since it was loaded. */

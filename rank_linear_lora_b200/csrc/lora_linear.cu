@@ -8,8 +8,8 @@
 //   backward  k_xa  : (only when no saved s.xa)
 //             k_g   : s.g = bf16(s . dY.B)              split over d_out  (M x r)
 //             k_dx  : dX = [dY | s.g] . [W ; A]         K = d_out + r, W and A MN-major
-//             k_dB  : dB = dY^T . (s.xa)                split over tokens
-//             k_dA  : dA = (s.g)^T . x  (written as [r, d_in])   split over tokens
+//             k_dadb: dB = dY^T . (s.xa) and dA = (s.g)^T . x (written as [r, d_in]),
+//                     one launch, split over tokens, overlapping the dX GEMM's last wave
 //
 // No allocation, no synchronisation, no exceptions across the ABI.
 #include <cuda.h>
@@ -433,29 +433,34 @@ GemmArgs base_args(const Ctx &c) {
     return a;
 }
 
-// Skinny split-K contraction D[rows, r] (rows = M-dim) over K, with A [*, *] bf16.
-// a_mn / b_mn select the operand majorness; the tensor maps are built by the caller.
+// One skinny split-K problem: D [rows, r] over K = kdim, split as `sp`.
+SkinnyJob make_job(int r, int64_t rows, int64_t kdim, const Split &sp, float *part, int *ctr, void *out,
+                   int out_mode, int64_t out_ld, float scale) {
+    SkinnyJob j;
+    std::memset(&j, 0, sizeof(j));
+    j.m_tiles = static_cast<int>(cdiv(rows, BM));
+    j.kb0 = static_cast<int>(cdiv(kdim, BK));
+    j.splits = sp.splits;
+    j.kb_per_split = sp.per;
+    j.num_tiles = j.m_tiles * sp.splits;
+    j.rows_valid = static_cast<int>(rows);
+    j.n_valid = r;
+    j.out_mode = out_mode;
+    j.out_scale = scale;
+    j.part = part;
+    j.counters = ctr;
+    j.out = out;
+    j.out_ld = out_ld;
+    return j;
+}
+
+// Launch the skinny split-K kernel over a.job[0 .. a.n_jobs) (tensor maps already set)
+// on at most `grid_cap` CTAs.  a_mn / b_mn select the operand majorness.
 template <bool A_MN, bool B_MN>
-lora_status_t launch_skinny(const Ctx &c, GemmArgs &a, int r, int64_t rows, int64_t kdim, const Split &sp,
-                            float *part, int *ctr, void *out, int out_mode, int64_t out_ld, float scale,
-                            int kind) {
-    const int64_t mt = cdiv(rows, BM);
-    a.m_tiles = static_cast<int>(mt);
-    a.n_tiles = 1;
-    a.kb0 = static_cast<int>(cdiv(kdim, BK));
+lora_status_t launch_skinny(const Ctx &c, GemmArgs &a, int r, int grid_cap, int kind) {
     a.kb1 = 0;
-    a.splits = sp.splits;
-    a.kb_per_split = sp.per;
-    a.num_tiles = static_cast<int>(mt * sp.splits);
-    a.rows_valid = static_cast<int>(rows);
-    a.n_valid = r;
-    a.out_mode = out_mode;
-    a.out_scale = scale;
-    a.part = part;
-    a.counters = ctr;
-    a.out = out;
-    a.out_ld = out_ld;
-    const int grid = std::min(a.num_tiles, c.info->sms);
+    a.num_tiles = a.job[0].num_tiles + (a.n_jobs > 1 ? a.job[1].num_tiles : 0);
+    const int grid = std::max(1, std::min({a.num_tiles, c.info->sms, grid_cap}));
     cudaError_t e;
     if (!A_MN && !B_MN) {
         switch (bn_class_kmajor(r)) {
@@ -480,6 +485,10 @@ lora_status_t launch_skinny(const Ctx &c, GemmArgs &a, int r, int64_t rows, int6
     return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
+int *counters_at(const Ctx &c, int64_t offset_tiles) {
+    return reinterpret_cast<int *>(c.ws + c.plan.ctr) + offset_tiles;
+}
+
 // s.xa = bf16(s . x.A^T) -> dst [M, r]
 lora_status_t step_xa(const Ctx &c, const uint16_t *x, const uint16_t *A, uint16_t *dst, int64_t M, int64_t d_in,
                       int r, float s) {
@@ -487,9 +496,10 @@ lora_status_t step_xa(const Ctx &c, const uint16_t *x, const uint16_t *A, uint16
     const int bn = bn_class_kmajor(r);
     if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmB0, A, d_in, r, 64, bn)) return LORA_ERR_CUDA;
-    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr);
-    return launch_skinny<false, false>(c, a, r, M, d_in, c.plan.s_xa, reinterpret_cast<float *>(c.ws + c.plan.part_xa),
-                                       ctr, dst, OUT_BF16_ROWS, 0, s, LORA_K_XA);
+    a.n_jobs = 1;
+    a.job[0] = make_job(r, M, d_in, c.plan.s_xa, reinterpret_cast<float *>(c.ws + c.plan.part_xa), counters_at(c, 0),
+                        dst, OUT_BF16_ROWS, 0, s);
+    return launch_skinny<false, false>(c, a, r, PLAN_SMS, LORA_K_XA);
 }
 
 // s.g = bf16(s . dY.B) -> ws g [M, r]; B [d_out, r] is read MN-major (r contiguous).
@@ -497,31 +507,32 @@ lora_status_t step_g(const Ctx &c, const uint16_t *dY, const uint16_t *B, int64_
     GemmArgs a = base_args(c);
     if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmB0, B, r, d_out, 64, 64)) return LORA_ERR_CUDA;
-    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + cdiv(M, BM);
-    return launch_skinny<false, true>(c, a, r, M, d_out, c.plan.s_g, reinterpret_cast<float *>(c.ws + c.plan.part_g),
-                                      ctr, c.ws + c.plan.g, OUT_BF16_ROWS, 0, s, LORA_K_G);
+    a.n_jobs = 1;
+    a.job[0] = make_job(r, M, d_out, c.plan.s_g, reinterpret_cast<float *>(c.ws + c.plan.part_g),
+                        counters_at(c, cdiv(M, BM)), c.ws + c.plan.g, OUT_BF16_ROWS, 0, s);
+    return launch_skinny<false, true>(c, a, r, PLAN_SMS, LORA_K_G);
 }
 
-// dB [d_out, r] = dY^T . (s.xa): M-dim = d_out, K = tokens, both operands MN-major.
-lora_status_t step_db(const Ctx &c, const uint16_t *dY, const uint16_t *sxa, float *dB, int64_t M, int64_t d_out,
-                      int r) {
+// The two weight gradients in one launch, both split over tokens with MN-major operands:
+//   job 0: dB [d_out, r] = dY^T . (s.xa)
+//   job 1: dA [r, d_in]  = (s.g)^T . x, computed as its transpose (M-dim = d_in), stored transposed.
+// `defer`: launched right after the dX GEMM, whose outputs it does not read, so it may
+// run on the SMs that GEMM's last wave leaves idle (`grid_cap` CTAs).
+lora_status_t step_dadb(const Ctx &c, const uint16_t *dY, const uint16_t *x, const uint16_t *sxa,
+                        const uint16_t *sg, float *dA, float *dB, int64_t M, int64_t d_in, int64_t d_out, int r,
+                        bool defer, int grid_cap) {
     GemmArgs a = base_args(c);
+    a.defer_dep_wait = defer ? 1 : 0;
     if (!tmap_bf16(&a.tmA0, dY, d_out, M, 64, 64)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmB0, sxa, r, M, 64, 64)) return LORA_ERR_CUDA;
-    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + 2 * cdiv(M, BM);
-    return launch_skinny<true, true>(c, a, r, d_out, M, c.plan.s_db, reinterpret_cast<float *>(c.ws + c.plan.part_db),
-                                     ctr, dB, OUT_F32_ROWS, 0, 1.0f, LORA_K_DB);
-}
-
-// dA [r, d_in] = (s.g)^T . x: computed as dA^T (M-dim = d_in) and written transposed.
-lora_status_t step_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float *dA, int64_t M, int64_t d_in,
-                      int64_t d_out, int r) {
-    GemmArgs a = base_args(c);
-    if (!tmap_bf16(&a.tmA0, x, d_in, M, 64, 64)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmB0, sg, r, M, 64, 64)) return LORA_ERR_CUDA;
-    int *ctr = reinterpret_cast<int *>(c.ws + c.plan.ctr) + 2 * cdiv(M, BM) + cdiv(d_out, BM);
-    return launch_skinny<true, true>(c, a, r, d_in, M, c.plan.s_da, reinterpret_cast<float *>(c.ws + c.plan.part_da),
-                                     ctr, dA, OUT_F32_COLS, d_in, 1.0f, LORA_K_DA);
+    if (!tmap_bf16(&a.tmA1, x, d_in, M, 64, 64)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmB1, sg, r, M, 64, 64)) return LORA_ERR_CUDA;
+    a.n_jobs = 2;
+    a.job[0] = make_job(r, d_out, M, c.plan.s_db, reinterpret_cast<float *>(c.ws + c.plan.part_db),
+                        counters_at(c, 2 * cdiv(M, BM)), dB, OUT_F32_ROWS, 0, 1.0f);
+    a.job[1] = make_job(r, d_in, M, c.plan.s_da, reinterpret_cast<float *>(c.ws + c.plan.part_da),
+                        counters_at(c, 2 * cdiv(M, BM) + cdiv(d_out, BM)), dA, OUT_F32_COLS, d_in, 1.0f);
+    return launch_skinny<true, true>(c, a, r, grid_cap, LORA_K_DADB);
 }
 
 // Main K-concatenated GEMM: out [M, N] = A0 . B0^T (K0) + A1 . B1^T (K1 = r).
@@ -532,14 +543,13 @@ struct MainOperands {
     void *C;
 };
 
+// `idle_sms` (optional) receives how many SMs the last wave leaves without work.
 lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t N, int64_t K0, int r, bool b_mn,
-                        int kind) {
+                        int kind, bool allow_tail_split, int *idle_sms = nullptr) {
     GemmArgs a = base_args(c);
     a.kb0 = static_cast<int>(cdiv(K0, BK));
     a.kb1 = static_cast<int>(cdiv(r, BK));
     a.mma_last1 = static_cast<int>(cdiv(r - (a.kb1 - 1) * BK, 16));
-    a.splits = 1;
-    a.kb_per_split = a.kb0;
     if (!tmap_bf16(&a.tmA0, o.A0, K0, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmA1, o.A1, r, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmC, o.C, N, M, 64, 32)) return LORA_ERR_CUDA;
@@ -552,7 +562,7 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         a.num_tiles = static_cast<int>(T);
         a.group_m = std::min(a.m_tiles, 8);
         const int64_t W = T / pair_C, R = T % pair_C;
-        const bool split = W >= 1 && R > 0 && 2 * R <= pair_C;
+        const bool split = allow_tail_split && W >= 1 && R > 0 && 2 * R <= pair_C;
         a.dp_tiles = static_cast<int>(split ? W * pair_C : T);
         a.dp_waves = static_cast<int>(split ? W : cdiv(T, pair_C));
         a.tail_tiles = static_cast<int>(split ? R : 0);
@@ -569,6 +579,7 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
             }
         }
         const int clusters = split ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
+        if (idle_sms) *idle_sms = (!split && R > 0 && W >= 1) ? c.info->sms - static_cast<int>(2 * R) : 0;
         cudaError_t e = b_mn ? launch_pair<true>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
                              : launch_pair<false>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
         return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
@@ -579,7 +590,13 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     a.num_tiles = a.m_tiles * a.n_tiles;
     a.group_m = std::min(a.m_tiles, 16);
     const int G = std::min(c.info->sms, PLAN_SMS);
-    const MainSched ms = main_sched(M, N, G);
+    MainSched ms = main_sched(M, N, G);
+    if (!allow_tail_split && ms.tail_split > 1) {
+        ms.dp_tiles = ms.tiles;
+        ms.dp_waves = static_cast<int>(cdiv(ms.tiles, G));
+        ms.tail_tiles = 0;
+        ms.tail_split = 1;
+    }
     a.dp_tiles = ms.dp_tiles;
     a.dp_waves = ms.dp_waves;
     a.tail_tiles = ms.tail_tiles;
@@ -597,6 +614,10 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         }
     }
     const int grid = ms.tail_split > 1 ? G : std::min(a.num_tiles, G);
+    if (idle_sms) {
+        const int rem = ms.tiles % G;
+        *idle_sms = (ms.tail_split == 1 && rem > 0 && ms.tiles >= G) ? c.info->sms - rem : 0;
+    }
     cudaError_t e;
     if (b_mn)
         e = launch_gemm<MAIN_BN, false, true, EPI_STORE, MAIN_STAGES>(a, grid, c.st, c.info, AB_DX, kind);
@@ -625,7 +646,7 @@ lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, 
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
     const MainOperands o{x, W, sxa, B, h};
-    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN);
+    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, true);
 }
 
 lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
@@ -647,13 +668,19 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W,
     }
     LORA_TRY(step_g(c, dY, B, M, d_out, r, s));
     const uint16_t *sg = reinterpret_cast<const uint16_t *>(c.ws + c.plan.g);
+    // dB and dA read nothing the dX GEMM writes: launched after it (programmatic
+    // dependent launch), they start on the SMs its last wave leaves idle and wait for
+    // it only before they exit.  The dX tail is then left whole (no narrow tiles) so
+    // those SMs free up early.
+    const bool overlap = dX != nullptr && pdl_enabled();
+    int idle = 0;
     if (dX) {
         // W [d_out, d_in] and A [r, d_in] are read MN-major (d_in contiguous).
         const MainOperands o{dY, W, sg, A, dX};
-        LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN));
+        LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
     }
-    LORA_TRY(step_db(c, dY, sxa, dB, M, d_out, r));
-    LORA_TRY(step_da(c, x, sg, dA, M, d_in, d_out, r));
+    const int cap = (overlap && idle >= 16) ? idle : PLAN_SMS;
+    LORA_TRY(step_dadb(c, dY, x, sxa, sg, dA, dB, M, d_in, d_out, r, overlap && idle >= 16, cap));
     return LORA_OK;
 }
 

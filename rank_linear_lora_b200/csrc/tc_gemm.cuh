@@ -60,6 +60,23 @@ enum DevErr {
     DERR_WAIT_DRAIN = 0x105,
 };
 
+// One skinny split-K problem: output [rows_valid, n_valid] over K = kb0 * 64.
+struct SkinnyJob {
+    int m_tiles;             // 128-row output tiles
+    int kb0;                 // 64-wide K blocks
+    int splits;              // K splits (each a CTA tile)
+    int kb_per_split;
+    int num_tiles;           // m_tiles * splits
+    int rows_valid;          // valid output rows
+    int n_valid;             // valid output columns (r)
+    int out_mode;            // OutMode
+    float out_scale;
+    float *part;             // fp32 partials [splits][m_tiles*BM][n_valid]
+    int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
+    void *out;
+    int64_t out_ld;          // OUT_F32_COLS: row stride of the transposed output
+};
+
 struct GemmArgs {
     CUtensorMap tmA0, tmB0;  // segment 0
     CUtensorMap tmA1, tmB1;  // segment 1 (rank-r tail), used when kb1 > 0
@@ -68,27 +85,23 @@ struct GemmArgs {
     int m_tiles, n_tiles;
     int kb0, kb1;            // 64-wide K blocks per segment
     int mma_last1;           // K=16 MMAs in the last block of segment 1 (1..4)
-    // EPI_SPLITK
-    int splits;              // K splits of segment 0
-    int kb_per_split;
-    int num_tiles;           // m_tiles * n_tiles * splits
-    int rows_valid;          // valid output rows
-    int n_valid;             // valid output columns (r)
-    int out_mode;            // OutMode
-    float out_scale;
-    float *part;             // partials [splits][m_tiles*BM][n_valid]
-    void *out;
-    int64_t out_ld;          // OUT_F32_COLS: row stride of the transposed output
+    int num_tiles;
+    // EPI_SPLITK: one or two independent skinny problems in one launch; job 0 reads
+    // tmA0/tmB0, job 1 tmA1/tmB1.  Tiles of job 0 come first.
+    int n_jobs;
+    SkinnyJob job[2];
     // EPI_STORE
     int group_m;             // rasterisation: M tiles per group
     int dp_tiles;            // tiles done whole (raster order 0 .. dp_tiles-1)
     int dp_waves;            // whole tiles per CTA (at most)
     int tail_tiles;          // last-wave tiles cut along N (raster dp_tiles ..)
     int tail_split;          // 1 (none), 2 or 4 narrow tiles per tail tile
-    // EPI_SPLITK
-    int *counters;           // per-tile arrival counters (zero on entry, zero on exit)
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
+    // 1: this kernel reads nothing its stream predecessor writes, so it starts its work
+    // without waiting and waits for the predecessor only before it exits; its own
+    // completion then still implies the predecessor's (stream order is kept).
+    int defer_dep_wait;
 };
 
 // Trace record of one CTA (globaltimer ns unless noted).
@@ -144,6 +157,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
 struct WorkItem {
     int m, n;
     int kb_lo, kb_hi;
+    int job;     // EPI_SPLITK: which problem
     int piece;   // EPI_SPLITK: split index
     int col0;    // EPI_STORE: first output column
     int nsplit;  // EPI_STORE: 1 for a whole tile, else tail_split (width BN / nsplit)
@@ -164,18 +178,25 @@ template <int BN, int EPI>
 __device__ __forceinline__ bool get_item(const GemmArgs &p, int i, WorkItem &w) {
     const int G = gridDim.x, c = blockIdx.x;
     if (EPI == EPI_SPLITK) {
-        const int t = c + i * G;
-        if (t >= p.num_tiles) return false;
-        w.piece = t % p.splits;
-        const int mn = t / p.splits;
-        w.m = mn % p.m_tiles;
-        w.n = mn / p.m_tiles;
-        w.kb_lo = w.piece * p.kb_per_split;
-        w.kb_hi = min(p.kb0, w.kb_lo + p.kb_per_split);
+        int t = c + i * G;
+        w.job = 0;
+        if (t >= p.job[0].num_tiles) {
+            t -= p.job[0].num_tiles;
+            w.job = 1;
+            if (p.n_jobs < 2 || t >= p.job[1].num_tiles) return false;
+        }
+        const SkinnyJob &J = p.job[w.job];
+        w.piece = t % J.splits;
+        const int mt = t / J.splits;
+        w.m = mt % J.m_tiles;
+        w.n = 0;
+        w.kb_lo = w.piece * J.kb_per_split;
+        w.kb_hi = min(J.kb0, w.kb_lo + J.kb_per_split);
         w.col0 = 0;
         w.nsplit = 1;
         return true;
     }
+    w.job = 0;
     w.kb_lo = 0;
     w.kb_hi = p.kb0 + p.kb1;
     w.piece = 0;
@@ -264,7 +285,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&p.tmA0);
         tma_prefetch_desc(&p.tmB0);
-        if (p.kb1 > 0) {
+        if (p.kb1 > 0 || p.n_jobs > 1) {
             tma_prefetch_desc(&p.tmA1);
             tma_prefetch_desc(&p.tmB1);
         }
@@ -279,8 +300,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     // Everything above touched no global memory; from here on we may read what the
-    // previous kernel in the stream wrote and overwrite what it read.
-    grid_dep_wait();
+    // previous kernel in the stream wrote and overwrite what it read (unless this kernel
+    // is independent of it, see defer_dep_wait).
+    if (!p.defer_dep_wait) grid_dep_wait();
     grid_dep_launch_dependents();
     if (trace && threadIdx.x == 0) {
         trace[TR_SETUP] = globaltimer_ns();
@@ -307,10 +329,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                     mbar_arrive_expect_tx(fb, Cfg::A_BYTES + bn * BK * 2);
                     issued_mask |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
-                    const bool seg1 = kb >= p.kb0;
+                    // Second map pair: the rank-r K segment (EPI_STORE) or job 1 (EPI_SPLITK).
+                    const bool seg1 = (EPI == EPI_SPLITK) ? (w.job == 1) : (kb >= p.kb0);
                     const CUtensorMap *ta = seg1 ? &p.tmA1 : &p.tmA0;
                     const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
-                    const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
+                    const int k0 = ((EPI == EPI_STORE && seg1) ? kb - p.kb0 : kb) * BK;
                     const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     if (A_MN) {
@@ -461,10 +484,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 }
             } else {
                 // fp32 partial of this K split -> workspace.
-                const int64_t rows_total = static_cast<int64_t>(p.m_tiles) * BM;
+                const SkinnyJob &J = p.job[w.job];
+                const int64_t rows_total = static_cast<int64_t>(J.m_tiles) * BM;
                 const int64_t grow = static_cast<int64_t>(w.m) * BM + row_local;
-                float *my_part = p.part + ((static_cast<int64_t>(w.piece) * rows_total + grow) * p.n_valid);
-                for (int c0 = 0; c0 < p.n_valid; c0 += 8) {
+                float *my_part = J.part + ((static_cast<int64_t>(w.piece) * rows_total + grow) * J.n_valid);
+                for (int c0 = 0; c0 < J.n_valid; c0 += 8) {
                     uint32_t v[8];
                     tmem_ld_32x32b_x8(t_row + c0, v);
                     tc_wait_ld();
@@ -479,30 +503,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                 if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[buf]));
                 __threadfence();
                 named_bar_sync(1, 128);
-                const int ctr = w.n * p.m_tiles + w.m;
-                if (epi_tid == 0) *last_flag = (atomicAdd(&p.counters[ctr], 1) == p.splits - 1) ? 1 : 0;
+                const int ctr = w.m;
+                if (epi_tid == 0) *last_flag = (atomicAdd(&J.counters[ctr], 1) == J.splits - 1) ? 1 : 0;
                 named_bar_sync(1, 128);
                 const bool last = *last_flag != 0;
                 named_bar_sync(1, 128);  // everyone has read last_flag before it is reused
                 if (last) {
                     __threadfence();
-                    if (grow < p.rows_valid) {
-                        const float *prow = p.part + grow * p.n_valid;
-                        const int64_t split_stride = rows_total * p.n_valid;
-                        for (int c0 = 0; c0 < p.n_valid; c0 += 4) {
+                    if (grow < J.rows_valid) {
+                        const float *prow = J.part + grow * J.n_valid;
+                        const int64_t split_stride = rows_total * J.n_valid;
+                        for (int c0 = 0; c0 < J.n_valid; c0 += 4) {
                             float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
                             // Eight splits' loads in flight at a time, summed in split order.
-                            for (int s0 = 0; s0 < p.splits; s0 += 8) {
+                            for (int s0 = 0; s0 < J.splits; s0 += 8) {
                                 float4 v[8];
 #pragma unroll
                                 for (int u = 0; u < 8; ++u)
-                                    v[u] = (s0 + u < p.splits)
+                                    v[u] = (s0 + u < J.splits)
                                                ? __ldcg(reinterpret_cast<const float4 *>(
                                                      prow + (s0 + u) * split_stride + c0))
                                                : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                                 for (int u = 0; u < 8; ++u) {
-                                    if (s0 + u < p.splits) {
+                                    if (s0 + u < J.splits) {
                                         acc.x += v[u].x;
                                         acc.y += v[u].y;
                                         acc.z += v[u].z;
@@ -510,27 +534,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
                                     }
                                 }
                             }
-                            acc.x *= p.out_scale;
-                            acc.y *= p.out_scale;
-                            acc.z *= p.out_scale;
-                            acc.w *= p.out_scale;
-                            if (p.out_mode == OUT_BF16_ROWS) {
+                            acc.x *= J.out_scale;
+                            acc.y *= J.out_scale;
+                            acc.z *= J.out_scale;
+                            acc.w *= J.out_scale;
+                            if (J.out_mode == OUT_BF16_ROWS) {
                                 __nv_bfloat162 a = __floats2bfloat162_rn(acc.x, acc.y);
                                 __nv_bfloat162 b = __floats2bfloat162_rn(acc.z, acc.w);
                                 uint2 u2 = make_uint2(*reinterpret_cast<uint32_t *>(&a), *reinterpret_cast<uint32_t *>(&b));
-                                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(p.out) + grow * p.n_valid + c0) = u2;
-                            } else if (p.out_mode == OUT_F32_ROWS) {
-                                *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + grow * p.n_valid + c0) = acc;
+                                *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(J.out) + grow * J.n_valid + c0) = u2;
+                            } else if (J.out_mode == OUT_F32_ROWS) {
+                                *reinterpret_cast<float4 *>(static_cast<float *>(J.out) + grow * J.n_valid + c0) = acc;
                             } else {
-                                float *o = static_cast<float *>(p.out);
-                                o[(c0 + 0) * p.out_ld + grow] = acc.x;
-                                o[(c0 + 1) * p.out_ld + grow] = acc.y;
-                                o[(c0 + 2) * p.out_ld + grow] = acc.z;
-                                o[(c0 + 3) * p.out_ld + grow] = acc.w;
+                                float *o = static_cast<float *>(J.out);
+                                o[(c0 + 0) * J.out_ld + grow] = acc.x;
+                                o[(c0 + 1) * J.out_ld + grow] = acc.y;
+                                o[(c0 + 2) * J.out_ld + grow] = acc.z;
+                                o[(c0 + 3) * J.out_ld + grow] = acc.w;
                             }
                         }
                     }
-                    if (epi_tid == 0) p.counters[ctr] = 0;  // ready for the next call
+                    if (epi_tid == 0) J.counters[ctr] = 0;  // ready for the next call
                 }
             }
             if (trace && epi_tid == 0 && it < 8) trace[TR_TILE_DONE0 + it] = globaltimer_ns();
@@ -549,6 +573,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm(const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
     }
+    if (p.defer_dep_wait) grid_dep_wait();
     if (trace && threadIdx.x == 0) {
         trace[TR_EXIT] = globaltimer_ns();
         trace[TR_CLK_EXIT] = clock64();

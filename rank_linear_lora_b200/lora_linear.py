@@ -22,7 +22,7 @@ LORA_OK = 0
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_MISALIGNED", 3: "LORA_ERR_UNSUPPORTED",
           4: "LORA_ERR_WORKSPACE", 5: "LORA_ERR_CUDA", 6: "LORA_ERR_TIMEOUT"}
 OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4 = 0, 1, 2, 3
-KERNEL_KINDS = ["xa", "fwd_main", "g", "dx_main", "dB", "dA"]
+KERNEL_KINDS = ["xa", "fwd_main", "g", "dx_main", "dadb"]
 
 
 class LoraError(RuntimeError):
