@@ -139,6 +139,31 @@ LORA_API lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x,
                                  int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Forward without a workspace, for callers that cannot allocate device memory: a
+ * plugin inside a host framework that owns every device allocation and passes in
+ * only the op's tensors, or a service that fixes its device-memory budget at start-up
+ * and forbids allocation afterwards (cudaMalloc may synchronise the device and
+ * fragments the heap).  The pages have no counterpart; this is an interface
+ * convenience.  Same arguments and results as lora_linear_fwd, minus the workspace.
+ *   - Scratch: a fixed 4 MiB array in device memory, held by every GPU that loads this
+ *     library until the process exits.  Problems whose forward workspace
+ *     (lora_linear_workspace_size(LORA_OP_FWD, ...)) exceeds 4 MiB are rejected with
+ *     LORA_ERR_WORKSPACE before anything is enqueued (every r <= 16 workload of
+ *     M <= 8192 fits; rank 128 at M = 16384 does not).
+ *   - Allocates nothing: no cudaMalloc/cudaFree; it enqueues a memset that clears the
+ *     part of the scratch the call uses, then the forward kernels.
+ *   - The first call on a device, with that device current, looks up the scratch's
+ *     device address (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - All calls share the one scratch: calls that can overlap on the GPU (different
+ *     streams, or host threads without ordering) race and give wrong results.
+ */
+LORA_API lora_status_t lora_linear_fwd_noalloc(const uint16_t *x, const uint16_t *W, const uint16_t *A,
+                                               const uint16_t *B, uint16_t *h, uint16_t *xa_save,
+                                               int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                                               void *stream);
+
 /* Waits for `stream`, then reads and clears the device error word kept in
  * `workspace`.  Returns LORA_OK, LORA_ERR_TIMEOUT (a bounded device wait ran out) or
  * LORA_ERR_CUDA (the stream reported an error).  Synchronising: for tests and

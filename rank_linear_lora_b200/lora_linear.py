@@ -219,3 +219,25 @@ def lora_linear_trace_enable(buf):
     else:
         _check(load_library().lora_linear_trace_enable(_ptr(buf), buf.numel() * buf.element_size()),
                "lora_linear_trace_enable")
+
+
+def lora_linear_fwd_noalloc(x, W, A, B, h, xa_save, alpha, stream=None):
+    """Forward without a workspace, for callers that cannot allocate device memory
+    (the library's fixed 4 MiB device scratch is used instead; see the header for the
+    size limit and for why concurrent calls must not overlap)."""
+    lib = load_library()
+    fn = lib.lora_linear_fwd_noalloc
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, P, P, I64, I64, I64, I, F, P]
+    fn.restype = I
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = W.shape[0]
+    for t, n, s in ((x, "x", (M, d_in)), (W, "W", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)),
+                    (h, "h", (M, d_out))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    st = fn(_ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(h), _ptr(xa_save), M, d_in, d_out, r, float(alpha),
+            _stream(stream))
+    _check(st, "lora_linear_fwd_noalloc")
