@@ -70,10 +70,15 @@ def algorithmic_bytes(spec) -> float:
 
 
 def kernel_source_hash() -> str:
+    """Hash of every CUDA source of the library (a stored ncu traffic figure is only
+    reported while the kernels it was measured on are unchanged)."""
     h = hashlib.sha256()
-    for f in ("ptx.cuh", "tc_gemm.cuh", "lora_linear.cu"):
-        with open(os.path.join(ROOT, "rank_linear_lora_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "rank_linear_lora_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode())
+                h.update(fh.read())
     return h.hexdigest()[:16]
 
 
