@@ -43,7 +43,8 @@
  *     for its predecessor in the stream before touching global memory, so stream
  *     order is preserved; only launch latency and set-up overlap.
  *   - The device must be compute capability 10.0 (B200); otherwise
- *     LORA_ERR_UNSUPPORTED is returned and nothing runs.
+ *     LORA_ERR_UNSUPPORTED is returned and nothing runs.  The *_q4 entry points also
+ *     need two-SM clusters (CTA pairs); without them they return LORA_ERR_UNSUPPORTED.
  *   - Device-side waits are bounded.  A wait that runs out sets an error word in the
  *     workspace and the kernels return early; lora_linear_check() reports it.
  *   - No C++ exception crosses this interface.

@@ -107,6 +107,22 @@ bool tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, u
     return r == CUDA_SUCCESS;
 }
 
+// Row-major 2D uint8 tensor [rows][cols_bytes], box {box_bytes, box_rows}, no swizzle
+// (the packed 4-bit codes, read by threads rather than by the tensor cores).
+bool tmap_u8(CUtensorMap *m, const void *base, uint64_t cols_bytes, uint64_t rows, uint32_t box_bytes,
+             uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols_bytes, rows};
+    cuuint64_t strides[1] = {cols_bytes};
+    cuuint32_t box[2] = {box_bytes, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ timing hooks
 std::atomic<int64_t> g_launches{0};
 std::atomic<int> g_timing{0};
@@ -195,11 +211,13 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
 }
 
 constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGES_Q4 = 5;
 
-template <bool B_MN>
+template <bool B_MN, bool Q4>
 cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
-    using Cfg = PairCfg<B_MN, PAIR_STAGES>;
-    auto kern = k_tc_gemm_pair<B_MN, PAIR_STAGES>;
+    constexpr int S = Q4 ? PAIR_STAGES_Q4 : PAIR_STAGES;
+    using Cfg = PairCfg<B_MN, Q4, S>;
+    auto kern = k_tc_gemm_pair<B_MN, Q4, S>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!(dev->attr_set & (1ull << attr_bit))) {
@@ -223,7 +241,7 @@ cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.blockDim = dim3(Cfg::THREADS);
     cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -246,47 +264,50 @@ cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
     return e;
 }
 
+template <bool B_MN, bool Q4>
+int probe_pair_clusters(const DevInfo *dev) {
+    constexpr int S = Q4 ? PAIR_STAGES_Q4 : PAIR_STAGES;
+    using Cfg = PairCfg<B_MN, Q4, S>;
+    auto kern = k_tc_gemm_pair<B_MN, Q4, S>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2 * (dev->sms / 2));
+    cfg.blockDim = dim3(Cfg::THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        n = 0;
+    }
+    return n;
+}
+
 // Clusters of two CTAs of the pair kernel that can be resident at once (0 if none).
-int pair_clusters(DevInfo *dev, bool b_mn) {
-    static int cached[64][2] = {};
-    static bool probed[64][2] = {};
+int pair_clusters(DevInfo *dev, bool b_mn, bool q4) {
+    static int cached[64][4] = {};
+    static bool probed[64][4] = {};
     int d = 0;
     cudaGetDevice(&d);
     std::lock_guard<std::mutex> lk(g_mu);
     if (d < 0 || d >= 64) return 0;
-    if (!probed[d][b_mn]) {
-        probed[d][b_mn] = true;
-        int n = 0;
-        cudaLaunchConfig_t cfg;
-        std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3(2 * (dev->sms / 2));
-        cfg.blockDim = dim3(NUM_THREADS);
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaError_t e;
-        if (b_mn) {
-            cfg.dynamicSmemBytes = PairCfg<true, PAIR_STAGES>::SMEM_BYTES;
-            cudaFuncSetAttribute(k_tc_gemm_pair<true, PAIR_STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 PairCfg<true, PAIR_STAGES>::SMEM_BYTES);
-            e = cudaOccupancyMaxActiveClusters(&n, k_tc_gemm_pair<true, PAIR_STAGES>, &cfg);
-        } else {
-            cfg.dynamicSmemBytes = PairCfg<false, PAIR_STAGES>::SMEM_BYTES;
-            cudaFuncSetAttribute(k_tc_gemm_pair<false, PAIR_STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 PairCfg<false, PAIR_STAGES>::SMEM_BYTES);
-            e = cudaOccupancyMaxActiveClusters(&n, k_tc_gemm_pair<false, PAIR_STAGES>, &cfg);
-        }
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            n = 0;
-        }
-        cached[d][b_mn] = n;
+    const int v = (b_mn ? 1 : 0) + (q4 ? 2 : 0);
+    if (!probed[d][v]) {
+        probed[d][v] = true;
+        cached[d][v] = b_mn ? (q4 ? probe_pair_clusters<true, true>(dev) : probe_pair_clusters<true, false>(dev))
+                            : (q4 ? probe_pair_clusters<false, true>(dev) : probe_pair_clusters<false, false>(dev));
     }
-    return cached[d][b_mn];
+    return cached[d][v];
 }
 
 // Attribute bits of the instantiations (one per template combination).
@@ -296,7 +317,7 @@ enum {
     AB_XA16 = 2, AB_XA64, AB_XA128, AB_XA256,
     AB_G64 = 6, AB_G128, AB_G256,
     AB_T64 = 9, AB_T128, AB_T256,
-    AB_PAIR_K = 12, AB_PAIR_MN = 13,
+    AB_PAIR_K = 12, AB_PAIR_MN = 13, AB_PAIR_K_Q4 = 14, AB_PAIR_MN_Q4 = 15,
 };
 
 int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
@@ -541,6 +562,9 @@ lora_status_t step_dadb(const Ctx &c, const uint16_t *dY, const uint16_t *x, con
 struct MainOperands {
     const void *A0, *B0, *A1, *B1;
     void *C;
+    const uint8_t *Wq = nullptr;       // 4-bit frozen weight (B0 is then unused)
+    const uint16_t *Wscale = nullptr;  // its bf16 scales [d_out, d_in / 64]
+    int64_t q_rows = 0, q_cols = 0;    // W shape [d_out, d_in]
 };
 
 // `idle_sms` (optional) receives how many SMs the last wave leaves without work.
@@ -553,7 +577,19 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     if (!tmap_bf16(&a.tmA0, o.A0, K0, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmA1, o.A1, r, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmC, o.C, N, M, 64, 32)) return LORA_ERR_CUDA;
-    const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn), PLAN_SMS / 2) : 0;
+    const bool q4 = o.Wq != nullptr;
+    const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn, q4), PLAN_SMS / 2) : 0;
+    if (q4 && pair_C == 0) return LORA_ERR_UNSUPPORTED;  // the 4-bit path runs on CTA pairs only
+    if (q4) {
+        a.wscale = o.Wscale;
+        a.scale_ld = static_cast<int>(o.q_cols / 64);
+        a.scale_rows = static_cast<int>(o.q_rows);
+        // packed codes [d_out][d_in / 2] bytes; box: this CTA's B half per K block
+        if (b_mn ? !tmap_u8(&a.tmQ, o.Wq, o.q_cols / 2, o.q_rows, CTA_BN / 2, BK)
+                 : !tmap_u8(&a.tmQ, o.Wq, o.q_cols / 2, o.q_rows, BK / 2, CTA_BN))
+            return LORA_ERR_CUDA;
+        allow_tail_split = false;
+    }
     if (pair_C > 0) {
         // CTA pairs: 256 x 256 tiles, each CTA stages 128 rows of B.
         const int64_t T = cdiv(M, PAIR_BM) * cdiv(N, PAIR_BN);
@@ -568,10 +604,10 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         a.tail_tiles = static_cast<int>(split ? R : 0);
         a.tail_split = split ? 2 : 1;
         if (b_mn) {
-            if (!tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
+            if (!q4 && !tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
             if (!tmap_bf16(&a.tmB1, o.B1, N, r, 64, 64)) return LORA_ERR_CUDA;
         } else {
-            if (!tmap_bf16(&a.tmB0, o.B0, K0, N, 64, CTA_BN)) return LORA_ERR_CUDA;
+            if (!q4 && !tmap_bf16(&a.tmB0, o.B0, K0, N, 64, CTA_BN)) return LORA_ERR_CUDA;
             if (!tmap_bf16(&a.tmB1, o.B1, r, N, 64, CTA_BN)) return LORA_ERR_CUDA;
             if (split) {
                 if (!tmap_bf16(&a.tmB0n, o.B0, K0, N, 64, CTA_BN / 2)) return LORA_ERR_CUDA;
@@ -580,8 +616,13 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         }
         const int clusters = split ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
         if (idle_sms) *idle_sms = (!split && R > 0 && W >= 1) ? c.info->sms - static_cast<int>(2 * R) : 0;
-        cudaError_t e = b_mn ? launch_pair<true>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
-                             : launch_pair<false>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
+        cudaError_t e;
+        if (q4)
+            e = b_mn ? launch_pair<true, true>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_Q4, kind)
+                     : launch_pair<false, true>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_Q4, kind);
+        else
+            e = b_mn ? launch_pair<true, false>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
+                     : launch_pair<false, false>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
         return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
     }
     // Single-SM kernel: 128 x 256 tiles.
@@ -632,33 +673,56 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         if (_s != LORA_OK) return _s;        \
     } while (0)
 
-lora_status_t fwd_impl(const uint16_t *x, const uint16_t *W, const uint16_t *A, const uint16_t *B, uint16_t *h,
+// The frozen weight: bf16 W [d_out, d_in], or 4-bit codes Wq [d_out, d_in / 2] with bf16
+// scales Wscale [d_out, d_in / 64] (dequantised in shared memory inside the GEMMs).
+struct Weight {
+    const uint16_t *W = nullptr;
+    const uint8_t *Wq = nullptr;
+    const uint16_t *Wscale = nullptr;
+    bool q4() const { return Wq != nullptr; }
+    bool present() const { return q4() ? (Wq && Wscale) : W != nullptr; }
+    bool aligned() const { return q4() ? (aligned16(Wq) && aligned16(Wscale)) : aligned16(W); }
+};
+
+MainOperands main_operands(const Weight &wt, const void *A0, const void *A1, const void *B1, void *C,
+                           int64_t d_out, int64_t d_in) {
+    MainOperands o{A0, wt.W, A1, B1, C};
+    if (wt.q4()) {
+        o.Wq = wt.Wq;
+        o.Wscale = wt.Wscale;
+        o.q_rows = d_out;
+        o.q_cols = d_in;
+    }
+    return o;
+}
+
+lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, const uint16_t *B, uint16_t *h,
                        uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, void *ws,
                        size_t ws_bytes, void *stream) {
-    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, false));
-    if (!x || !W || !A || !B || !h) return LORA_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(h) ||
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.q4()));
+    if (!x || !wt.present() || !A || !B || !h) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(h) ||
         (xa_save && !aligned16(xa_save)))
         return LORA_ERR_MISALIGNED;
     Ctx c;
-    LORA_TRY(prepare(LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    LORA_TRY(prepare(wt.q4() ? LORA_OP_FWD_Q4 : LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
-    const MainOperands o{x, W, sxa, B, h};
+    const MainOperands o = main_operands(wt, x, sxa, B, h, d_out, d_in);
     return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, true);
 }
 
-lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
+lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, const uint16_t *A,
                        const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB, int64_t M,
                        int64_t d_in, int64_t d_out, int r, float alpha, void *ws, size_t ws_bytes, void *stream) {
-    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, false));
-    if (!dY || !x || !W || !A || !B || !dA || !dB) return LORA_ERR_INVALID_ARG;
-    if (!aligned16(dY) || !aligned16(x) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.q4()));
+    if (!dY || !x || !wt.present() || !A || !B || !dA || !dB) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(dY) || !aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
         !aligned16(dB) || (xa_save && !aligned16(xa_save)) || (dX && !aligned16(dX)))
         return LORA_ERR_MISALIGNED;
     Ctx c;
-    LORA_TRY(prepare(LORA_OP_BWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    LORA_TRY(prepare(wt.q4() ? LORA_OP_BWD_Q4 : LORA_OP_BWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     const uint16_t *sxa = xa_save;
     if (!sxa) {
@@ -675,8 +739,8 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const uint16_t *W,
     const bool overlap = dX != nullptr && pdl_enabled();
     int idle = 0;
     if (dX) {
-        // W [d_out, d_in] and A [r, d_in] are read MN-major (d_in contiguous).
-        const MainOperands o{dY, W, sg, A, dX};
+        // W [d_out, d_in] (or its codes) and A [r, d_in] are read MN-major (d_in contiguous).
+        const MainOperands o = main_operands(wt, dY, sg, A, dX, d_out, d_in);
         LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
     }
     const int cap = (overlap && idle >= 16) ? idle : PLAN_SMS;
@@ -700,14 +764,18 @@ size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out
 lora_status_t lora_linear_fwd(const uint16_t *x, const uint16_t *W, const uint16_t *A, const uint16_t *B, uint16_t *h,
                               uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                               void *workspace, size_t workspace_bytes, void *stream) {
-    return fwd_impl(x, W, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
+    Weight wt;
+    wt.W = W;
+    return fwd_impl(x, wt, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
 }
 
 lora_status_t lora_linear_bwd(const uint16_t *dY, const uint16_t *x, const uint16_t *W, const uint16_t *A,
                               const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
                               int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, void *workspace,
                               size_t workspace_bytes, void *stream) {
-    return bwd_impl(dY, x, W, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+    Weight wt;
+    wt.W = W;
+    return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
                     stream);
 }
 
@@ -715,18 +783,23 @@ lora_status_t lora_linear_fwd_q4(const uint16_t *x, const uint8_t *Wq, const uin
                                  const uint16_t *B, uint16_t *h, uint16_t *xa_save, int64_t M, int64_t d_in,
                                  int64_t d_out, int r, float alpha, void *workspace, size_t workspace_bytes,
                                  void *stream) {
-    (void)x; (void)Wq; (void)Wscale; (void)A; (void)B; (void)h; (void)xa_save; (void)M; (void)d_in;
-    (void)d_out; (void)r; (void)alpha; (void)workspace; (void)workspace_bytes; (void)stream;
-    return LORA_ERR_UNSUPPORTED;
+    Weight wt;
+    wt.Wq = Wq;
+    wt.Wscale = Wscale;
+    if (!Wq || !Wscale) return LORA_ERR_INVALID_ARG;
+    return fwd_impl(x, wt, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
 }
 
 lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale,
                                  const uint16_t *A, const uint16_t *B, const uint16_t *xa_save, uint16_t *dX,
                                  float *dA, float *dB, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                                  void *workspace, size_t workspace_bytes, void *stream) {
-    (void)dY; (void)x; (void)Wq; (void)Wscale; (void)A; (void)B; (void)xa_save; (void)dX; (void)dA; (void)dB;
-    (void)M; (void)d_in; (void)d_out; (void)r; (void)alpha; (void)workspace; (void)workspace_bytes; (void)stream;
-    return LORA_ERR_UNSUPPORTED;
+    Weight wt;
+    wt.Wq = Wq;
+    wt.Wscale = Wscale;
+    if (!Wq || !Wscale) return LORA_ERR_INVALID_ARG;
+    return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                    stream);
 }
 
 lora_status_t lora_linear_check(void *workspace, void *stream) {

@@ -82,6 +82,7 @@ struct GemmArgs {
     CUtensorMap tmA1, tmB1;  // segment 1 (rank-r tail), used when kb1 > 0
     CUtensorMap tmC;         // EPI_STORE output (bf16, box 64 x 32, 128B swizzle)
     CUtensorMap tmB0n, tmB1n;  // K-major B with box rows BN / tail_split (narrow tail tiles)
+    CUtensorMap tmQ;           // 4-bit frozen weight: packed codes (uint8), no swizzle
     int m_tiles, n_tiles;
     int kb0, kb1;            // 64-wide K blocks per segment
     int mma_last1;           // K=16 MMAs in the last block of segment 1 (1..4)
@@ -96,6 +97,10 @@ struct GemmArgs {
     int dp_waves;            // whole tiles per CTA (at most)
     int tail_tiles;          // last-wave tiles cut along N (raster dp_tiles ..)
     int tail_split;          // 1 (none), 2 or 4 narrow tiles per tail tile
+    // 4-bit frozen weight: bf16 scales [scale_rows][scale_ld], one per 64 codes along d_in
+    const uint16_t *wscale;
+    int scale_ld;
+    int scale_rows;
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
     // 1: this kernel reads nothing its stream predecessor writes, so it starts its work

@@ -33,16 +33,36 @@ constexpr int PAIR_BM = 256;      // output rows per pair tile (128 per CTA)
 constexpr int PAIR_BN = 256;      // output columns per pair tile
 constexpr int CTA_BN = PAIR_BN / 2;  // B rows (N) staged per CTA
 
-template <bool B_MN, int STAGES>
+template <bool B_MN, bool Q4, int STAGES>
 struct PairCfg {
     static constexpr int A_BYTES = 128 * BK * 2;      // 16 KB: this CTA's 128 rows of A
     static constexpr int B_BYTES = CTA_BN * BK * 2;   // 16 KB: this CTA's 128 rows of B
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int Q_BYTES = Q4 ? CTA_BN * BK / 2 : 0;  // 4 KB of packed 4-bit codes
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + Q_BYTES;
     static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
     static constexpr int TMEM_COLS = 2 * PAIR_BN;     // two 256-column accumulators
-    static constexpr int BAR_BYTES = 256;
+    static constexpr int BAR_BYTES = 512;
+    static constexpr int THREADS = Q4 ? NUM_THREADS + 128 : NUM_THREADS;  // + dequant warpgroup
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
 };
+
+// Decode one 32-bit word of 4-bit codes (8 consecutive elements, element i in bits
+// 4i..4i+3: low nibble of each byte = even index) into 8 bf16 values
+// w' = (q - 8) * s7, computed in fp32 (q - 8 exact) and rounded once to bf16.
+__device__ __forceinline__ uint4 q4_decode8(uint32_t word, float s7) {
+    uint32_t out[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t q0 = (word >> (8 * j)) & 0xFu;
+        const uint32_t q1 = (word >> (8 * j + 4)) & 0xFu;
+        // 2^23 + q as a float, minus 2^23 + 8: exactly q - 8.
+        const float f0 = (__uint_as_float(0x4B000000u | q0) - 8388616.0f) * s7;
+        const float f1 = (__uint_as_float(0x4B000000u | q1) - 8388616.0f) * s7;
+        __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
+        out[j] = *reinterpret_cast<uint32_t *>(&b);
+    }
+    return make_uint4(out[0], out[1], out[2], out[3]);
+}
 
 // Item i of this cluster: pair tile (m, n), its first output column and width split.
 __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, int n_clusters, int i, WorkItem &w) {
@@ -67,23 +87,28 @@ __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, in
     return false;
 }
 
-template <bool B_MN, int STAGES>
-__global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_constant__ GemmArgs p) {
-    using Cfg = PairCfg<B_MN, STAGES>;
+template <bool B_MN, bool Q4, int STAGES>
+__global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
+    k_tc_gemm_pair(const __grid_constant__ GemmArgs p) {
+    using Cfg = PairCfg<B_MN, Q4, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
+    uint8_t *sQ = smem + STAGES * (Cfg::A_BYTES + Cfg::B_BYTES);  // packed codes (Q4)
     uint8_t *sEpi = smem + STAGES * Cfg::STAGE_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + Cfg::EPI_BYTES);
-    uint64_t *full_bar = bars;                    // [STAGES] (leader's counts the pair's bytes)
+    uint64_t *full_bar = bars;                    // [STAGES] (leader's counts the pair's A (and B) bytes)
     uint64_t *empty_bar = bars + STAGES;          // [STAGES]
     uint64_t *tfull_bar = bars + 2 * STAGES;      // [2]
     uint64_t *tempty_bar = bars + 2 * STAGES + 2; // [2] (leader's: 8 epilogue warps of the pair)
     uint64_t *drain_bar = bars + 2 * STAGES + 4;  // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+    uint64_t *pfull_bar = bars + 2 * STAGES + 5;  // [STAGES] Q4: this CTA's packed codes (or bf16 tail B) landed
+    uint64_t *bready_bar = bars + 3 * STAGES + 5; // [STAGES] Q4, leader: both CTAs' bf16 B tiles written
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 5);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 3);  // [2]
+    volatile int *dq_ok = reinterpret_cast<volatile int *>(tmem_slot + 5);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -109,10 +134,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
             mbar_init(smem_u32(&tempty_bar[b]), 8);
         }
         mbar_init(smem_u32(drain_bar), 1);
+        if (Q4)
+            for (int s = 0; s < STAGES; ++s) {
+                mbar_init(smem_u32(&pfull_bar[s]), 1);
+                mbar_init(smem_u32(&bready_bar[s]), 2);
+            }
         *abort_flag = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
+        if (Q4) tma_prefetch_desc(&p.tmQ);
         tma_prefetch_desc(&p.tmA0);
         tma_prefetch_desc(&p.tmB0);
         if (p.kb1 > 0) {
@@ -142,7 +173,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued_mask = 0, issued_phase = 0;
+            uint32_t issued_mask = 0, issued_phase = 0;    // leader's full barriers
+            uint32_t qissued_mask = 0, qissued_phase = 0;  // Q4: this CTA's packed-code barriers
             bool ok = true;
             uint64_t wait_empty_ns = 0;
             WorkItem w;
@@ -150,7 +182,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 const int bn_cta = (PAIR_BN / w.nsplit) / 2;  // B rows this CTA stages
                 const int a_row = w.m * PAIR_BM + static_cast<int>(rank) * 128;
                 const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
-                const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
+                // Q4: B reaches this CTA's smem as packed codes (main K segment) or bf16 (rank-r
+                // tail), completing on its own barrier; the leader's full barrier counts A only.
+                const uint32_t tx = Q4 ? 2u * static_cast<uint32_t>(Cfg::A_BYTES)
+                                       : 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     const uint64_t tw = trace ? globaltimer_ns() : 0;
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
@@ -171,7 +206,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                     const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     tma_load_2d_pair(a_dst, seg1 ? &p.tmA1 : &p.tmA0, fb_leader, k0, a_row);
-                    if (B_MN) {
+                    if (Q4) {
+                        const uint32_t pb = smem_u32(&pfull_bar[stage]);
+                        qissued_mask |= 1u << stage;
+                        qissued_phase = (qissued_phase & ~(1u << stage)) | (phase << stage);
+                        if (!seg1) {
+                            mbar_arrive_expect_tx(pb, static_cast<uint32_t>(Cfg::Q_BYTES));
+                            const uint32_t q_dst = smem_u32(sQ + stage * Cfg::Q_BYTES);
+                            if (B_MN)  // K rows k0.., bytes of d_in columns b_row..b_row+127
+                                tma_load_2d(q_dst, &p.tmQ, pb, b_row / 2, k0);
+                            else       // N rows b_row.., bytes of K columns k0..k0+63
+                                tma_load_2d(q_dst, &p.tmQ, pb, k0 / 2, b_row);
+                        } else {
+                            mbar_arrive_expect_tx(pb, static_cast<uint32_t>(bn_cta * BK * 2));
+                            if (B_MN) {
+                                for (int j = 0; j < bn_cta / 64; ++j)
+                                    tma_load_2d(b_dst + j * 64 * 128, &p.tmB1, pb, b_row + 64 * j, k0);
+                            } else {
+                                tma_load_2d(b_dst, &p.tmB1, pb, k0, b_row);
+                            }
+                        }
+                    } else if (B_MN) {
                         const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
                         for (int j = 0; j < bn_cta / 64; ++j)
                             tma_load_2d_pair(b_dst + j * 64 * 128, tb, fb_leader, b_row + 64 * j, k0);
@@ -193,6 +248,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                     if (issued_mask & (1u << s)) {
                         volatile int never = 0;
                         wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
+                                     DERR_WAIT_DRAIN);
+                    }
+            if (Q4)
+                for (int s = 0; s < STAGES; ++s)
+                    if (qissued_mask & (1u << s)) {
+                        volatile int never = 0;
+                        wait_bounded(smem_u32(&pfull_bar[s]), (qissued_phase >> s) & 1u, &never, p.err,
                                      DERR_WAIT_DRAIN);
                     }
             if (trace) {
@@ -240,6 +302,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                         ok = false;
                         break;
                     }
+                    if (Q4) {
+                        const uint32_t rb = smem_u32(&bready_bar[stage]);
+                        if (!mbar_try_wait(rb, phase) &&
+                            !wait_bounded(rb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                            ok = false;
+                            break;
+                        }
+                    }
                     tc_fence_after();
                     const uint64_t ad = ad_base + static_cast<uint64_t>((stage * Cfg::A_BYTES) >> 4);
                     const uint64_t bd = bd_base + static_cast<uint64_t>((stage * Cfg::B_BYTES) >> 4);
@@ -271,6 +341,90 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) k_tc_gemm_pair(const __grid_co
                 trace[TR_TILES] = static_cast<unsigned long long>(it);
                 trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
                 trace[TR_KBLOCKS] = kblocks;
+            }
+        }
+    } else if (Q4 && warp >= 6) {
+        // ------------------------------------------------------------ dequant warpgroup (both CTAs, Q4)
+        // Each K block of the weight segment: wait for this CTA's packed codes, decode
+        // them to bf16 into the swizzled B tile the MMA reads, make the generic-proxy
+        // stores visible to the tensor core, then report to the leader's B-ready barrier.
+        // Rank-r tail blocks arrive as bf16 already and are only reported.
+        const int dq = threadIdx.x - 192;  // 0..127
+        const uint32_t bready_leader0 = mapa_shared(smem_u32(&bready_bar[0]), 0);
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        WorkItem w;
+        bool ok = true;
+        for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
+            const int bn_cta = (PAIR_BN / w.nsplit) / 2;
+            const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
+            for (int kb = w.kb_lo; kb < w.kb_hi; ++kb, ++it) {
+                const bool seg1 = kb >= p.kb0;
+                const int k0 = kb * BK;
+                // this thread's row (K-major: weight row n) or K row and 64-column chunk (MN-major)
+                int srow, scol;
+                if (B_MN) {
+                    srow = k0 + (dq & 63);
+                    scol = (b_row + 64 * (dq >> 6)) / 64;
+                } else {
+                    srow = b_row + dq;
+                    scol = kb;
+                }
+                float s7 = 0.f;
+                if (!seg1 && srow < p.scale_rows && scol < p.scale_ld &&
+                    (B_MN ? (dq >> 6) < bn_cta / 64 : dq < bn_cta)) {
+                    const uint16_t sb = __ldg(p.wscale + static_cast<int64_t>(srow) * p.scale_ld + scol);
+                    s7 = __uint_as_float(static_cast<uint32_t>(sb) << 16) / 7.0f;
+                }
+                if (dq == 0)
+                    dq_ok[it & 1] = wait_bounded(smem_u32(&pfull_bar[stage]), phase, abort_flag, p.err,
+                                                 DERR_WAIT_FULL) ? 1 : 0;
+                named_bar_sync(2, 128);
+                if (!dq_ok[it & 1]) {
+                    ok = false;
+                    break;
+                }
+                if (!seg1) {
+                    const uint8_t *qsrc = sQ + stage * Cfg::Q_BYTES;
+                    uint8_t *bdst = sB + stage * Cfg::B_BYTES;
+                    if (B_MN) {
+                        const int k = dq & 63, j = dq >> 6;
+                        if (j < bn_cta / 64) {
+                            const uint4 *src = reinterpret_cast<const uint4 *>(qsrc + k * (bn_cta / 2) + j * 32);
+                            uint8_t *row = bdst + j * 64 * 128 + (k >> 3) * 1024 + (k & 7) * 128;
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const uint4 v = src[h2];
+                                const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) {
+                                    const int c = h2 * 4 + e;
+                                    *reinterpret_cast<uint4 *>(row + ((c ^ (k & 7)) * 16)) = q4_decode8(wds[e], s7);
+                                }
+                            }
+                        }
+                    } else if (dq < bn_cta) {
+                        const int n = dq;
+                        const uint4 *src = reinterpret_cast<const uint4 *>(qsrc + n * 32);
+                        uint8_t *row = bdst + (n >> 3) * 1024 + (n & 7) * 128;
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const uint4 v = src[h2];
+                            const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = h2 * 4 + e;
+                                *reinterpret_cast<uint4 *>(row + ((c ^ (n & 7)) * 16)) = q4_decode8(wds[e], s7);
+                            }
+                        }
+                    }
+                    fence_proxy_async_smem();
+                }
+                named_bar_sync(2, 128);
+                if (dq == 0) mbar_arrive_cluster(bready_leader0 + static_cast<uint32_t>(stage * 8));
+                stage = stage + 1 == STAGES ? 0 : stage + 1;
+                phase = stage == 0 ? phase ^ 1u : phase;
             }
         }
     } else {

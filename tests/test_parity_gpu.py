@@ -207,8 +207,38 @@ def test_without_programmatic_launch(monkeypatch):
     compare_all(dl.results(), oracle_ref(inp), spec.s)
 
 
+# 4-bit frozen weight: codes dequantised in shared memory inside both main GEMMs.
+Q4_SHAPES = [
+    (200, 320, 200, 16),     # ragged M and d_out (out-of-range rows and K rows of the codes)
+    (520, 512, 768, 24),     # rank tail r % 16 != 0
+    (129, 1024, 1536, 8),
+]
+
+
+@pytest.mark.parametrize("shape", Q4_SHAPES, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_q4_full(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("q4", M, di, do, r, alpha=2.0 * r, q4=True, seed=0x44 + M)
+    inp, dl = _run_full(spec)
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+def test_q4_lora_dominant():
+    """Large B so the rank-r tail (bf16, not dequantised) dominates: the tail blocks pass
+    through the dequant stage untouched."""
+    spec = inputs.LayerSpec("q4dom", 264, 384, 320, 16, alpha=32.0, q4=True, seed=0x45)
+    inp = inputs.make_inputs(spec)
+    inp.B = inputs.to_bf16_bits(inputs.bf16_bits_to_f32(inp.B).astype(np.float64) * 50.0)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.backward()
+    dl.check()
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
 # ------------------------------------------------------------------ full sizes
-FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0)]
+FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0),
+        (4, None, 0)]
 
 
 @pytest.mark.parametrize("cfg", FULL, ids=lambda c: f"cfg{c[0]}_r{c[1]}_layer{c[2]}")
