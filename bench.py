@@ -360,13 +360,18 @@ def main():
     dom = max(("fwd_main", "dx_main"), key=lambda k: rec[k][0])
     dom_ms = rec[dom][0] / max(1, rec[dom][1])
     achieved = kern_flops[dom] / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
+    # A kernel timed inside a long, power-capped run is held to the sustained GEMM peak,
+    # one timed in a short burst (no power capping seen) to the burst peak.
+    sustained = ms_max > 250.0 or "sw_power_cap" in (clocks.get("reasons") or [])
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak_kind = "sustained" if sustained else "burst"
     roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_src": f"{peaks['src']} bf16 burst (MEASURED_PEAKS.json)",
+                "frac": achieved / peak,
+                "peak_src": f"{peaks['src']} bf16 {peak_kind} (MEASURED_PEAKS.json; timed region {ms_max:.0f} ms)",
                 "traffic": stored_traffic(dom, workload_name)}
     t_roof = max(flops_step / (peak * 1e12), algorithmic_bytes(spec) / (peaks["hbm_gbs"] * 1e9))
     step_roof = {"t_roof_us": t_roof * 1e6, "t_meas_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
-                 "definition": "max(FLOP / bf16 peak, algorithmic bytes / HBM peak) over the measured step time"}
+                 "definition": f"max(FLOP / bf16 {peak_kind} peak, algorithmic bytes / HBM peak) over the measured step time"}
     kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
 
     # end to end through the C ABI with host buffers: H2D of the step's inputs from pinned

@@ -118,6 +118,11 @@ enum TraceField {
     TR_KBLOCKS = 19,     // K blocks consumed by the MMA issuer
     TR_CLK_SETUP = 20,   // SM cycle counter after set-up
     TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
+    // CTA-pair kernel, SM cycles: the MMA issuer's waits for A tiles (full) and, 4-bit
+    // weight, for decoded B tiles (B-ready); the first dequant warp's waits for packed
+    // codes, its decode time, its waits for a free B tile and its store + publish time.
+    TR_MMA_WAIT_A = 22, TR_MMA_WAIT_B = 23, TR_DQ_WAIT = 24, TR_DQ_DECODE = 25, TR_DQ_PUBLISH = 26,
+    TR_DQ_SLOT = 27, TR_DQ_ISSUE = 28,
     TRACE_WORDS = 32
 };
 
@@ -146,6 +151,27 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                atomicCAS(err, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait until a monotonic shared-memory counter reaches `target` (acquire);
+// false on timeout or abort, as wait_bounded.  Polls with a short sleep so that a
+// waiting thread takes little shared-memory bandwidth from the tensor core.
+__device__ __forceinline__ bool wait_count_bounded(uint32_t addr, uint32_t target, volatile int *abort_flag,
+                                                   int *err, int code) {
+    if (ld_acquire_shared(addr) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(32);
+        if (ld_acquire_shared(addr) >= target) return true;
         if ((i & 31u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
@@ -241,6 +267,23 @@ __device__ __forceinline__ void stage_row64(uint8_t *sbuf, int lane, const uint3
     for (int cc = 0; cc < 8; ++cc) {
         uint4 w = make_uint4(packed[4 * cc], packed[4 * cc + 1], packed[4 * cc + 2], packed[4 * cc + 3]);
         *reinterpret_cast<uint4 *>(row_ptr + ((cc ^ (lane & 7)) * 16)) = w;
+    }
+}
+
+// Half of stage_row64: 32 fp32 columns (half 0: columns 0..31, half 1: 32..63) of one
+// accumulator row into their four swizzled 16-byte chunks; for kernels short of registers.
+__device__ __forceinline__ void stage_row32(uint8_t *sbuf, int lane, int half, const uint32_t (&v)[32]) {
+    uint8_t *row_ptr = sbuf + lane * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+            w[e] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        const int cc = half * 4 + q;
+        *reinterpret_cast<uint4 *>(row_ptr + ((cc ^ (lane & 7)) * 16)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 

@@ -13,6 +13,11 @@
 //   warps 2..5  epilogue in both CTAs: each drains its own 128 accumulator rows from
 //               TMEM, reports to the leader's accumulator-empty barrier, and stores
 //               bf16 through 128B-swizzled smem staging with TMA
+//   warps 6..   (4-bit frozen weight only) dequant warps in both CTAs: fetch packed
+//               codes by TMA, decode them to bf16 straight into the B tile of the
+//               weight K segment and report to the leader's B-ready barrier; the
+//               producer then loads only A for those blocks (and A + B for the rank-r
+//               tail blocks, as in the bf16 case)
 //
 // Schedule: whole pair tiles in grouped raster order, `dp_waves` per cluster; a
 // partial last wave of `tail_tiles` tiles is cut along N into two 256 x 128 tiles,
@@ -32,36 +37,55 @@ namespace lora {
 constexpr int PAIR_BM = 256;      // output rows per pair tile (128 per CTA)
 constexpr int PAIR_BN = 256;      // output columns per pair tile
 constexpr int CTA_BN = PAIR_BN / 2;  // B rows (N) staged per CTA
+constexpr int DQ_WARPS = 16;         // 4-bit weight: dequant warps per CTA
+constexpr int DQ_GROUPS = 4;         // groups of dequant warps that take K blocks in turn
+constexpr int DQ_QDEPTH = 2;         // packed-code slots per dequant warp (own K blocks in flight)
+constexpr int DQ_QSLOT = 32 * 32;    // one slot: 32 rows x 32 bytes (64 codes) of the packed weight
 
 template <bool B_MN, bool Q4, int STAGES>
 struct PairCfg {
     static constexpr int A_BYTES = 128 * BK * 2;      // 16 KB: this CTA's 128 rows of A
     static constexpr int B_BYTES = CTA_BN * BK * 2;   // 16 KB: this CTA's 128 rows of B
-    static constexpr int Q_BYTES = Q4 ? CTA_BN * BK / 2 : 0;  // 4 KB of packed 4-bit codes
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + Q_BYTES;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int Q_BYTES = Q4 ? DQ_WARPS * DQ_QDEPTH * DQ_QSLOT : 0;  // per-warp packed-code rings
     static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
     static constexpr int TMEM_COLS = 2 * PAIR_BN;     // two 256-column accumulators
-    static constexpr int BAR_BYTES = 512;
-    static constexpr int THREADS = Q4 ? NUM_THREADS + 128 : NUM_THREADS;  // + dequant warpgroup
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES;
+    static constexpr int BAR_BYTES = Q4 ? 1024 : 512;
+    static constexpr int THREADS = Q4 ? NUM_THREADS + 32 * DQ_WARPS : NUM_THREADS;  // + dequant warps
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + Q_BYTES + EPI_BYTES + BAR_BYTES;
+    static_assert(STAGES <= 32, "per-stage phase bits are kept in one 32-bit mask");
 };
 
+// Two codes, each given as the fp32 bit pattern of 2^23 + q, to the bf16 pair
+// ((q_even - 8) * s7, (q_odd - 8) * s7), even element in the low half.  The packed
+// fp32 add is exact (it leaves q - 8), the packed multiply rounds once in fp32 and the
+// conversion rounds once more to bf16.
+__device__ __forceinline__ uint32_t q4_pair(uint32_t f_even, uint32_t f_odd, uint64_t s7x2) {
+    constexpr uint64_t kMinus2p23p8x2 = 0xCB000008CB000008ull;  // -(2^23 + 8) in both fp32 halves
+    uint32_t out;
+    asm("{\n\t.reg .b64 v;\n\t.reg .b32 e, o;\n\t"
+        "mov.b64 v, {%1, %2};\n\t"
+        "add.rn.f32x2 v, v, %3;\n\t"
+        "mul.rn.f32x2 v, v, %4;\n\t"
+        "mov.b64 {e, o}, v;\n\t"
+        "cvt.rn.bf16x2.f32 %0, o, e;\n\t}"
+        : "=r"(out)
+        : "r"(f_even), "r"(f_odd), "l"(kMinus2p23p8x2), "l"(s7x2));
+    return out;
+}
+
 // Decode one 32-bit word of 4-bit codes (8 consecutive elements, element i in bits
-// 4i..4i+3: low nibble of each byte = even index) into 8 bf16 values
-// w' = (q - 8) * s7, computed in fp32 (q - 8 exact) and rounded once to bf16.
-__device__ __forceinline__ uint4 q4_decode8(uint32_t word, float s7) {
-    uint32_t out[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const uint32_t q0 = (word >> (8 * j)) & 0xFu;
-        const uint32_t q1 = (word >> (8 * j + 4)) & 0xFu;
-        // 2^23 + q as a float, minus 2^23 + 8: exactly q - 8.
-        const float f0 = (__uint_as_float(0x4B000000u | q0) - 8388616.0f) * s7;
-        const float f1 = (__uint_as_float(0x4B000000u | q1) - 8388616.0f) * s7;
-        __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
-        out[j] = *reinterpret_cast<uint32_t *>(&b);
-    }
-    return make_uint4(out[0], out[1], out[2], out[3]);
+// 4i..4i+3: low nibble of each byte = even index) into 8 bf16 values (q - 8) * s7.
+// A byte permute places each nibble under the exponent of 2^23.
+__device__ __forceinline__ uint4 q4_decode8(uint32_t word, uint64_t s7x2) {
+    const uint32_t lo = word & 0x0F0F0F0Fu, hi = (word >> 4) & 0x0F0F0F0Fu;
+    constexpr uint32_t kExp = 0x4B000000u;  // 2^23
+    uint4 r;
+    r.x = q4_pair(__byte_perm(lo, kExp, 0x7540), __byte_perm(hi, kExp, 0x7540), s7x2);
+    r.y = q4_pair(__byte_perm(lo, kExp, 0x7541), __byte_perm(hi, kExp, 0x7541), s7x2);
+    r.z = q4_pair(__byte_perm(lo, kExp, 0x7542), __byte_perm(hi, kExp, 0x7542), s7x2);
+    r.w = q4_pair(__byte_perm(lo, kExp, 0x7543), __byte_perm(hi, kExp, 0x7543), s7x2);
+    return r;
 }
 
 // Item i of this cluster: pair tile (m, n), its first output column and width split.
@@ -95,20 +119,24 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
-    uint8_t *sQ = smem + STAGES * (Cfg::A_BYTES + Cfg::B_BYTES);  // packed codes (Q4)
-    uint8_t *sEpi = smem + STAGES * Cfg::STAGE_BYTES;
+    uint8_t *sQ = smem + STAGES * Cfg::STAGE_BYTES;  // Q4: packed-code rings of the dequant warps
+    uint8_t *sEpi = sQ + Cfg::Q_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + Cfg::EPI_BYTES);
     uint64_t *full_bar = bars;                    // [STAGES] (leader's counts the pair's A (and B) bytes)
     uint64_t *empty_bar = bars + STAGES;          // [STAGES]
     uint64_t *tfull_bar = bars + 2 * STAGES;      // [2]
     uint64_t *tempty_bar = bars + 2 * STAGES + 2; // [2] (leader's: 8 epilogue warps of the pair)
     uint64_t *drain_bar = bars + 2 * STAGES + 4;  // [1]
-    uint64_t *pfull_bar = bars + 2 * STAGES + 5;  // [STAGES] Q4: this CTA's packed codes (or bf16 tail B) landed
-    uint64_t *bready_bar = bars + 3 * STAGES + 5; // [STAGES] Q4, leader: both CTAs' bf16 B tiles written
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 4 * STAGES + 5);
+    uint64_t *bready_bar = bars + 2 * STAGES + 5; // [STAGES] Q4, leader: both CTAs' decoded B tiles written
+    uint64_t *qfull_bar = bars + 3 * STAGES + 5;  // [DQ_WARPS][DQ_QDEPTH] Q4: a warp's packed codes landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qfull_bar + (Q4 ? DQ_WARPS * DQ_QDEPTH : 0));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 3);  // [2]
-    volatile int *dq_ok = reinterpret_cast<volatile int *>(tmem_slot + 5);   // [2]
+    // Q4: K blocks (in the CTA's sequence) whose stage the producer has seen released by
+    // the MMA, i.e. whose B tile the dequant warps may write.  A monotonic count: the
+    // dequant groups run ahead of the MMA by different amounts, so a parity wait on the
+    // stage's empty barrier could match a later phase than the one meant.
+    uint32_t *bfree = tmem_slot + 5;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -134,12 +162,12 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             mbar_init(smem_u32(&tempty_bar[b]), 8);
         }
         mbar_init(smem_u32(drain_bar), 1);
-        if (Q4)
-            for (int s = 0; s < STAGES; ++s) {
-                mbar_init(smem_u32(&pfull_bar[s]), 1);
-                mbar_init(smem_u32(&bready_bar[s]), 2);
-            }
+        if (Q4) {
+            for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * (DQ_WARPS / DQ_GROUPS));
+            for (int q = 0; q < DQ_WARPS * DQ_QDEPTH; ++q) mbar_init(smem_u32(&qfull_bar[q]), 1);
+        }
         *abort_flag = 0;
+        *bfree = 0;
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
@@ -173,20 +201,21 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued_mask = 0, issued_phase = 0;    // leader's full barriers
-            uint32_t qissued_mask = 0, qissued_phase = 0;  // Q4: this CTA's packed-code barriers
+            uint32_t issued_mask = 0, issued_phase = 0;  // leader's full barriers
             bool ok = true;
             uint64_t wait_empty_ns = 0;
+            uint32_t flat = 0;  // K blocks of the CTA's sequence handled so far
             WorkItem w;
             for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
                 const int bn_cta = (PAIR_BN / w.nsplit) / 2;  // B rows this CTA stages
                 const int a_row = w.m * PAIR_BM + static_cast<int>(rank) * 128;
                 const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
-                // Q4: B reaches this CTA's smem as packed codes (main K segment) or bf16 (rank-r
-                // tail), completing on its own barrier; the leader's full barrier counts A only.
-                const uint32_t tx = Q4 ? 2u * static_cast<uint32_t>(Cfg::A_BYTES)
-                                       : 2u * static_cast<uint32_t>(Cfg::A_BYTES + bn_cta * BK * 2);
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
+                    // Q4: the weight segment's B tiles are written by the dequant warps, so the
+                    // leader's full barrier then counts A only; rank-r tail B tiles come by TMA.
+                    const bool seg1 = kb >= p.kb0;
+                    const bool b_tma = !Q4 || seg1;
+                    const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + (b_tma ? bn_cta * BK * 2 : 0));
                     const uint64_t tw = trace ? globaltimer_ns() : 0;
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
                                       DERR_WAIT_EMPTY)) {
@@ -194,6 +223,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                         break;
                     }
                     if (trace) wait_empty_ns += globaltimer_ns() - tw;
+                    if (Q4) st_release_shared(smem_u32(bfree), ++flat);
                     const uint32_t fb_local = smem_u32(&full_bar[stage]);
                     const uint32_t fb_leader = mapa_shared(fb_local, 0);
                     if (leader) {
@@ -201,31 +231,11 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                         issued_mask |= 1u << stage;
                         issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     }
-                    const bool seg1 = kb >= p.kb0;
                     const int k0 = (seg1 ? kb - p.kb0 : kb) * BK;
                     const uint32_t a_dst = smem_u32(sA + stage * Cfg::A_BYTES);
                     const uint32_t b_dst = smem_u32(sB + stage * Cfg::B_BYTES);
                     tma_load_2d_pair(a_dst, seg1 ? &p.tmA1 : &p.tmA0, fb_leader, k0, a_row);
-                    if (Q4) {
-                        const uint32_t pb = smem_u32(&pfull_bar[stage]);
-                        qissued_mask |= 1u << stage;
-                        qissued_phase = (qissued_phase & ~(1u << stage)) | (phase << stage);
-                        if (!seg1) {
-                            mbar_arrive_expect_tx(pb, static_cast<uint32_t>(Cfg::Q_BYTES));
-                            const uint32_t q_dst = smem_u32(sQ + stage * Cfg::Q_BYTES);
-                            if (B_MN)  // K rows k0.., bytes of d_in columns b_row..b_row+127
-                                tma_load_2d(q_dst, &p.tmQ, pb, b_row / 2, k0);
-                            else       // N rows b_row.., bytes of K columns k0..k0+63
-                                tma_load_2d(q_dst, &p.tmQ, pb, k0 / 2, b_row);
-                        } else {
-                            mbar_arrive_expect_tx(pb, static_cast<uint32_t>(bn_cta * BK * 2));
-                            if (B_MN) {
-                                for (int j = 0; j < bn_cta / 64; ++j)
-                                    tma_load_2d(b_dst + j * 64 * 128, &p.tmB1, pb, b_row + 64 * j, k0);
-                            } else {
-                                tma_load_2d(b_dst, &p.tmB1, pb, k0, b_row);
-                            }
-                        }
+                    if (!b_tma) {
                     } else if (B_MN) {
                         const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
                         for (int j = 0; j < bn_cta / 64; ++j)
@@ -248,13 +258,6 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                     if (issued_mask & (1u << s)) {
                         volatile int never = 0;
                         wait_bounded(smem_u32(&full_bar[s]), (issued_phase >> s) & 1u, &never, p.err,
-                                     DERR_WAIT_DRAIN);
-                    }
-            if (Q4)
-                for (int s = 0; s < STAGES; ++s)
-                    if (qissued_mask & (1u << s)) {
-                        volatile int never = 0;
-                        wait_bounded(smem_u32(&pfull_bar[s]), (qissued_phase >> s) & 1u, &never, p.err,
                                      DERR_WAIT_DRAIN);
                     }
             if (trace) {
@@ -280,6 +283,8 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             int it = 0;
             bool ok = true;
             uint64_t wait_tempty_ns = 0, kblocks = 0;
+            long long wait_a_cyc = 0, wait_b_cyc = 0;
+            uint32_t bready_phase = 0;  // Q4: bit s = parity of the next B-ready completion of stage s
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
@@ -297,17 +302,27 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 // unrolled MMAs; the issue rate must keep pace with the tensor pipe.
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
                     const uint32_t fb = smem_u32(&full_bar[stage]);
-                    if (!mbar_try_wait(fb, phase) &&
-                        !wait_bounded(fb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
-                        ok = false;
-                        break;
-                    }
-                    if (Q4) {
-                        const uint32_t rb = smem_u32(&bready_bar[stage]);
-                        if (!mbar_try_wait(rb, phase) &&
-                            !wait_bounded(rb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
+                    if (!mbar_try_wait(fb, phase)) {
+                        const long long c0 = trace ? clock64() : 0;
+                        if (!wait_bounded(fb, phase, abort_flag, p.err, DERR_WAIT_FULL)) {
                             ok = false;
                             break;
+                        }
+                        if (trace) wait_a_cyc += clock64() - c0;
+                    }
+                    if (Q4 && kb < p.kb0) {
+                        // B-ready completes only for weight K blocks (rank-r tail blocks come
+                        // by TMA), so its phase per stage is tracked apart from the ring's.
+                        const uint32_t rb = smem_u32(&bready_bar[stage]);
+                        const uint32_t bp = (bready_phase >> stage) & 1u;
+                        bready_phase ^= 1u << stage;
+                        if (!mbar_try_wait(rb, bp)) {
+                            const long long c0 = trace ? clock64() : 0;
+                            if (!wait_bounded(rb, bp, abort_flag, p.err, DERR_WAIT_FULL)) {
+                                ok = false;
+                                break;
+                            }
+                            if (trace) wait_b_cyc += clock64() - c0;
                         }
                     }
                     tc_fence_after();
@@ -341,91 +356,161 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 trace[TR_TILES] = static_cast<unsigned long long>(it);
                 trace[TR_WAIT_TEMPTY] = wait_tempty_ns;
                 trace[TR_KBLOCKS] = kblocks;
+                trace[TR_MMA_WAIT_A] = static_cast<unsigned long long>(wait_a_cyc);
+                trace[TR_MMA_WAIT_B] = static_cast<unsigned long long>(wait_b_cyc);
             }
         }
     } else if (Q4 && warp >= 6) {
-        // ------------------------------------------------------------ dequant warpgroup (both CTAs, Q4)
-        // Each K block of the weight segment: wait for this CTA's packed codes, decode
-        // them to bf16 into the swizzled B tile the MMA reads, make the generic-proxy
-        // stores visible to the tensor core, then report to the leader's B-ready barrier.
-        // Rank-r tail blocks arrive as bf16 already and are only reported.
-        const int dq = threadIdx.x - 192;  // 0..127
+        // ------------------------------------------------------------ dequant warps (both CTAs, Q4)
+        // The weight segment's B tiles are decoded here from 4-bit codes.  Warps form
+        // DQ_GROUPS groups of GW; group g takes the weight K blocks g, g + DQ_GROUPS, ... of
+        // the CTA's sequence (the rank-r tail blocks come by TMA and are not touched).  One
+        // thread owns one 32-byte run of codes (64 elements): K-major, weight row rn of the
+        // tile; MN-major, K row rn of 64-column chunk jc.  Each warp fetches its own 32 runs
+        // by TMA into a private DQ_QDEPTH-slot ring, DQ_QDEPTH own blocks ahead, so code
+        // loads never wait for a stage.  Per block: wait for the codes, wait until the MMA
+        // has released the stage's B tile, decode straight into the 128B-swizzled layout
+        // the MMA reads, fence to the async proxy, and arrive (one arrival per warp) on the
+        // leader's B-ready barrier.  One block takes a warp ~2 us end to end (measured;
+        // decode, stores and the cluster-scope release arrival dominate), so DQ_GROUPS
+        // blocks are in flight at once.
+        constexpr int GW = DQ_WARPS / DQ_GROUPS;  // warps per group
+        static_assert(GW * 32 == 128, "one thread per 32-byte run of a 128-run B tile");
+        const int dw = warp - 6;                  // dequant warp 0 .. DQ_WARPS-1
+        const int grp = dw / GW, wg = dw % GW;
+        const int t = wg * 32 + lane;             // run 0..127
+        const int rn = B_MN ? (t & 63) : t;
+        const int jc = B_MN ? (t >> 6) : 0;
+        uint8_t *qring = sQ + dw * (DQ_QDEPTH * DQ_QSLOT);
+        uint64_t *qbar = qfull_bar + dw * DQ_QDEPTH;
         const uint32_t bready_leader0 = mapa_shared(smem_u32(&bready_bar[0]), 0);
-        int stage = 0;
-        uint32_t phase = 0;
-        int it = 0;
-        WorkItem w;
-        bool ok = true;
-        for (int i = 0; ok && get_pair_item(p, cluster, n_clusters, i, w); ++i) {
-            const int bn_cta = (PAIR_BN / w.nsplit) / 2;
-            const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
-            for (int kb = w.kb_lo; kb < w.kb_hi; ++kb, ++it) {
-                const bool seg1 = kb >= p.kb0;
-                const int k0 = kb * BK;
-                // this thread's row (K-major: weight row n) or K row and 64-column chunk (MN-major)
-                int srow, scol;
-                if (B_MN) {
-                    srow = k0 + (dq & 63);
-                    scol = (b_row + 64 * (dq >> 6)) / 64;
-                } else {
-                    srow = b_row + dq;
-                    scol = kb;
-                }
-                float s7 = 0.f;
-                if (!seg1 && srow < p.scale_rows && scol < p.scale_ld &&
-                    (B_MN ? (dq >> 6) < bn_cta / 64 : dq < bn_cta)) {
-                    const uint16_t sb = __ldg(p.wscale + static_cast<int64_t>(srow) * p.scale_ld + scol);
-                    s7 = __uint_as_float(static_cast<uint32_t>(sb) << 16) / 7.0f;
-                }
-                if (dq == 0)
-                    dq_ok[it & 1] = wait_bounded(smem_u32(&pfull_bar[stage]), phase, abort_flag, p.err,
-                                                 DERR_WAIT_FULL) ? 1 : 0;
-                named_bar_sync(2, 128);
-                if (!dq_ok[it & 1]) {
-                    ok = false;
-                    break;
-                }
-                if (!seg1) {
-                    const uint8_t *qsrc = sQ + stage * Cfg::Q_BYTES;
-                    uint8_t *bdst = sB + stage * Cfg::B_BYTES;
-                    if (B_MN) {
-                        const int k = dq & 63, j = dq >> 6;
-                        if (j < bn_cta / 64) {
-                            const uint4 *src = reinterpret_cast<const uint4 *>(qsrc + k * (bn_cta / 2) + j * 32);
-                            uint8_t *row = bdst + j * 64 * 128 + (k >> 3) * 1024 + (k & 7) * 128;
-#pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                const uint4 v = src[h2];
-                                const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) {
-                                    const int c = h2 * 4 + e;
-                                    *reinterpret_cast<uint4 *>(row + ((c ^ (k & 7)) * 16)) = q4_decode8(wds[e], s7);
-                                }
-                            }
-                        }
-                    } else if (dq < bn_cta) {
-                        const int n = dq;
-                        const uint4 *src = reinterpret_cast<const uint4 *>(qsrc + n * 32);
-                        uint8_t *row = bdst + (n >> 3) * 1024 + (n & 7) * 128;
-#pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const uint4 v = src[h2];
-                            const uint32_t wds[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                const int c = h2 * 4 + e;
-                                *reinterpret_cast<uint4 *>(row + ((c ^ (n & 7)) * 16)) = q4_decode8(wds[e], s7);
-                            }
-                        }
-                    }
-                    fence_proxy_async_smem();
-                }
-                named_bar_sync(2, 128);
-                if (dq == 0) mbar_arrive_cluster(bready_leader0 + static_cast<uint32_t>(stage * 8));
-                stage = stage + 1 == STAGES ? 0 : stage + 1;
-                phase = stage == 0 ? phase ^ 1u : phase;
+        const int kb_all = p.kb0 + p.kb1;
+        // Own block j is weight K block kb of work item `item`, with flat weight index
+        // grp + j * DQ_GROUPS.  Cursors step from one own block to the next without
+        // divisions; the item's geometry is recomputed only when a cursor enters a new item.
+        struct Cursor {
+            int j, item, kb, b_row;
+            bool valid;
+        };
+        auto enter_item = [&](Cursor &c) {
+            WorkItem wi;
+            c.valid = get_pair_item(p, cluster, n_clusters, c.item, wi);
+            c.b_row = c.valid ? wi.col0 + static_cast<int>(rank) * ((PAIR_BN / wi.nsplit) / 2) : 0;
+        };
+        auto seek = [&](Cursor &c, int j) {
+            const int wit = grp + j * DQ_GROUPS;
+            c.j = j;
+            c.item = wit / p.kb0;
+            c.kb = wit - c.item * p.kb0;
+            enter_item(c);
+        };
+        auto step = [&](Cursor &c) {
+            ++c.j;
+            c.kb += DQ_GROUPS;
+            if (c.kb >= p.kb0) {
+                const int adv = c.kb / p.kb0;
+                c.kb -= adv * p.kb0;
+                c.item += adv;
+                enter_item(c);
             }
+        };
+        // Lane 0: TMA of this warp's 32 runs of own block c.j into slot c.j % DQ_QDEPTH.
+        auto issue = [&](const Cursor &c) {
+            const uint32_t bar = smem_u32(&qbar[c.j % DQ_QDEPTH]);
+            const uint32_t dst = smem_u32(qring + (c.j % DQ_QDEPTH) * DQ_QSLOT);
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(DQ_QSLOT));
+            if (B_MN)  // K rows kb*64 + 32*(wg&1) .., bytes of d_in columns b_row + 64*(wg>>1) ..
+                tma_load_2d(dst, &p.tmQ, bar, c.b_row / 2 + 32 * (wg >> 1), c.kb * BK + 32 * (wg & 1));
+            else       // weight rows b_row + 32*wg .., bytes of K columns kb*64 ..
+                tma_load_2d(dst, &p.tmQ, bar, c.kb * (BK / 2), c.b_row + 32 * wg);
+        };
+        // Raw bf16 bits of this thread's group scale for own block c.j (0 outside the weight).
+        auto scale_bits = [&](const Cursor &c) -> uint32_t {
+            if (!c.valid) return 0u;
+            const int srow = B_MN ? c.kb * BK + rn : c.b_row + rn;
+            const int scol = B_MN ? (c.b_row + 64 * jc) / 64 : c.kb;
+            if (srow >= p.scale_rows || scol >= p.scale_ld) return 0u;
+            return static_cast<uint32_t>(__ldg(p.wscale + static_cast<int64_t>(srow) * p.scale_ld + scol));
+        };
+        const bool tr_dq = trace != nullptr && dw == 0 && lane == 0;
+        long long dq_wait = 0, dq_decode = 0, dq_slot = 0, dq_publish = 0, dq_issue = 0;
+        Cursor cur, ahead;  // own block being decoded; the next one whose codes to fetch
+        seek(cur, 0);
+        seek(ahead, 0);
+        int issued = 0;  // own blocks whose codes were requested
+        while (issued < DQ_QDEPTH && ahead.valid) {
+            if (lane == 0) issue(ahead);
+            ++issued;
+            step(ahead);
+        }
+        uint32_t sc = scale_bits(cur);  // fetched one own block ahead (at the end of the previous one)
+        while (cur.valid) {
+            const int j = cur.j;
+            const int flat = cur.item * kb_all + cur.kb;
+            const int stage = flat % STAGES;
+            const int slot = j % DQ_QDEPTH;
+            const long long c0 = tr_dq ? clock64() : 0;
+            if (!__all_sync(0xffffffffu, wait_bounded(smem_u32(&qbar[slot]), static_cast<uint32_t>(j / DQ_QDEPTH) & 1u,
+                                                      abort_flag, p.err, DERR_WAIT_FULL)))
+                break;
+            const long long c1 = tr_dq ? clock64() : 0;
+            const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * DQ_QSLOT + (t & 31) * 32);
+            const uint4 v0 = src[0], v1 = src[1];
+            const float s7 = __uint_as_float(sc << 16) / 7.0f;
+            const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
+            const long long c2 = tr_dq ? clock64() : 0;
+            // The stage's B tile is free once the producer has seen the MMA release it.
+            // Lane 0 polls; the warp barrier passes its acquire on to the other lanes.
+            bool granted = true;
+            if (lane == 0)
+                granted = wait_count_bounded(smem_u32(bfree), static_cast<uint32_t>(flat) + 1u, abort_flag, p.err,
+                                             DERR_WAIT_EMPTY);
+            __syncwarp();
+            if (!__shfl_sync(0xffffffffu, granted, 0)) break;
+            const long long c3 = tr_dq ? clock64() : 0;
+            uint8_t *row = sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
+            const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = q4_decode8(wds[c], s7x2);
+            // Orders the B-tile stores (and this slot's code reads, whose values are used
+            // above) before the tensor core's reads and the slot's next TMA write.
+            fence_proxy_async_smem();
+            __syncwarp();
+            long long c4 = 0;
+            if (lane == 0) {
+                mbar_arrive_cluster(bready_leader0 + static_cast<uint32_t>(stage * 8));
+                if (tr_dq) c4 = clock64();
+            }
+            if (ahead.valid) {  // the slot just read is free: fetch own block j + DQ_QDEPTH
+                if (lane == 0) issue(ahead);
+                ++issued;
+                step(ahead);
+            }
+            step(cur);
+            sc = scale_bits(cur);
+            if (tr_dq) {
+                const long long c5 = clock64();
+                dq_wait += c1 - c0;
+                dq_decode += c2 - c1;
+                dq_slot += c3 - c2;
+                dq_publish += c4 - c3;
+                dq_issue += c5 - c4;
+            }
+        }
+        const int j = cur.j;
+        // Copies still in flight (only after a failed wait): let them land before exit.
+        if (lane == 0)
+            for (int jj = j; jj < issued; ++jj) {
+                volatile int never = 0;
+                wait_bounded(smem_u32(&qbar[jj % DQ_QDEPTH]), static_cast<uint32_t>(jj / DQ_QDEPTH) & 1u, &never,
+                             p.err, DERR_WAIT_DRAIN);
+            }
+        if (tr_dq) {
+            trace[TR_DQ_WAIT] = static_cast<unsigned long long>(dq_wait);
+            trace[TR_DQ_DECODE] = static_cast<unsigned long long>(dq_decode);
+            trace[TR_DQ_SLOT] = static_cast<unsigned long long>(dq_slot);
+            trace[TR_DQ_PUBLISH] = static_cast<unsigned long long>(dq_publish);
+            trace[TR_DQ_ISSUE] = static_cast<unsigned long long>(dq_issue);
         }
     } else {
         // ------------------------------------------------------------ epilogue (both CTAs)
@@ -451,19 +536,37 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             const int out_row = w.m * PAIR_BM + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
             for (int ch = 0; ch < nch; ++ch) {
-                uint32_t v0[32], v1[32];
-                tmem_ld_32x32b_x32(t_row + ch * 64, v0);
-                tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
-                tc_wait_ld();
-                if (ch == nch - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
-                }
                 uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-                stage_row64(sbuf, lane, v0, v1);
+                if (Q4) {
+                    // 32 columns at a time: the dequant warps leave fewer registers per thread
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(t_row + ch * 64 + 32 * half, v);
+                        tc_wait_ld();
+                        if (half == 1 && ch == nch - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+                        }
+                        stage_row32(sbuf, lane, half, v);
+                    }
+                } else {
+                    uint32_t v0[32], v1[32];
+                    tmem_ld_32x32b_x32(t_row + ch * 64, v0);
+                    tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
+                    tc_wait_ld();
+                    if (ch == nch - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+                    }
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    stage_row64(sbuf, lane, v0, v1);
+                }
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {

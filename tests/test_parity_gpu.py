@@ -212,6 +212,11 @@ Q4_SHAPES = [
     (200, 320, 200, 16),     # ragged M and d_out (out-of-range rows and K rows of the codes)
     (520, 512, 768, 24),     # rank tail r % 16 != 0
     (129, 1024, 1536, 8),
+    # more 256 x 256 tiles than CTA pairs, so CTAs take several work items; K blocks per
+    # item (11 and 17, incl. the rank-r block) are not a multiple of the stage count, so
+    # the rank-r block falls on a different stage in each item
+    (1100, 640, 4000, 16),   # forward: 5 x 16 tiles
+    (1100, 4096, 1000, 16),  # dX: 5 x 16 tiles, K = d_out ragged
 ]
 
 
