@@ -244,6 +244,7 @@ def main():
     import torch.distributed as dist
 
     from rank_linear_lora_b200 import lora_linear as L
+    from rank_linear_lora_b200.dp import PackedGrads
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -274,9 +275,8 @@ def main():
         s["h"] = torch.empty(M, do, dtype=torch.bfloat16, device=dev)
         s["xa"] = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
         s["dX"] = torch.empty(M, di, dtype=torch.bfloat16, device=dev)
-        s["grad"] = torch.empty(r * di + do * r, dtype=torch.float32, device=dev)  # packed [dA | dB]
-        s["dA"] = s["grad"][: r * di].view(r, di)
-        s["dB"] = s["grad"][r * di:].view(do, r)
+        s["grad"] = PackedGrads(r, di, do, device=dev)  # fp32 [dA | dB], the one all-reduced buffer
+        s["dA"], s["dB"] = s["grad"].dA, s["grad"].dB
         fop, bop = (L.OP_FWD_Q4, L.OP_BWD_Q4) if spec.q4 else (L.OP_FWD, L.OP_BWD)
         s["wsf"] = L.workspace(fop, M, di, do, r, device=dev)
         s["wsb"] = L.workspace(bop, M, di, do, r, device=dev)
@@ -292,7 +292,7 @@ def main():
             L.lora_linear_bwd(s["dY"], s["x"], s["W"], s["A"], s["B"], s["xa"], s["dX"], s["dA"], s["dB"], alpha,
                               s["wsb"])
         if world > 1:
-            dist.all_reduce(s["grad"])
+            s["grad"].all_reduce()
 
     def barrier():
         if world > 1:

@@ -17,4 +17,6 @@ from .oracle import (  # noqa: F401
     da,
     forward,
     backward,
+    h_projections,
+    dx_projections,
 )

@@ -172,3 +172,61 @@ def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, rows=None, xa_=Non
         "g": g_,
         "xa": xa_,
     }
+
+
+# ------------------------------------------------------------------ projections
+# Properties of steps 2 and 4 that hold at any size: a projection of h (or dX) on a
+# vector follows from the definition by associativity, and costs O(M d) instead of
+# O(M d_in d_out).  Checking every row projection and every column projection of a
+# GPU result touches every element of it.  The weight is dequantised (oracle_weight,
+# the same rule as steps 2 and 4) a block of rows at a time, never as a whole.
+
+def _f64(bits) -> np.ndarray:
+    """bf16 bit patterns -> fp64 (exact)."""
+    return (_u16(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, rows=2048):
+    """(n0, fp64 rows n0 .. n0+k) of the dequantised weight, block by block."""
+    for n0 in range(0, d_out, rows):
+        n1 = min(d_out, n0 + rows)
+        if W is not None:
+            yield n0, weight(n1 - n0, d_in, W=_u16(W)[n0:n1])
+        else:
+            yield n0, weight(n1 - n0, d_in, Wq=np.ascontiguousarray(Wq)[n0:n1], Wscale=_u16(Wscale)[n0:n1])
+
+
+def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, xa_=None, block_rows=2048):
+    """Step 2 projected: (h . v [M], u^T . h [d_out]) for v [d_out], u [M], with
+    h . v = x . (W^T v) + s * xa . (B^T v) and u^T . h = W (x^T u) + s * B (xa^T u)."""
+    M, d_in = np.shape(x)
+    d_out = np.shape(B)[0]
+    xa_ = xa(x, A) if xa_ is None else xa_
+    xf, Bf = _f64(x), _f64(B)
+    wt_v = np.zeros(d_in)
+    xt_u = xf.T @ u
+    col = np.empty(d_out)
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, rows=block_rows):
+        wt_v += Wb.T @ v[n0:n0 + len(Wb)]
+        col[n0:n0 + len(Wb)] = Wb @ xt_u
+    row = xf @ wt_v + s * (xa_ @ (Bf.T @ v))
+    col += s * (Bf @ (xa_.T @ u))
+    return row, col
+
+
+def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, g_=None, block_rows=2048):
+    """Step 4 projected: (dX . v [M], u^T . dX [d_in]) for v [d_in], u [M], with
+    dX . v = dY . (W v) + s * g . (A v) and u^T . dX = (dY^T u)^T W + s * (g^T u)^T A."""
+    M, d_out = np.shape(dY)
+    d_in = np.shape(A)[1]
+    g_ = g(dY, B) if g_ is None else g_
+    dYf, Af = _f64(dY), _f64(A)
+    w_v = np.empty(d_out)
+    dyt_u = dYf.T @ u
+    col = np.zeros(d_in)
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, rows=block_rows):
+        w_v[n0:n0 + len(Wb)] = Wb @ v
+        col += dyt_u[n0:n0 + len(Wb)] @ Wb
+    row = dYf @ w_v + s * (g_ @ (Af @ v))
+    col += s * ((g_.T @ u) @ Af)
+    return row, col

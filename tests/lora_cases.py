@@ -118,3 +118,41 @@ def sample_rows(M: int, n_random: int = 24, seed: int = 0) -> np.ndarray:
     rng = np.random.default_rng(seed)
     rnd = set(rng.integers(0, M, size=n_random).tolist())
     return np.array(sorted(v for v in fixed | rnd if 0 <= v < M), dtype=np.int64)
+
+
+def check_projections(dl: "DeviceLayer", inp: inputs.LayerInputs, ref: dict, seed: int = 0):
+    """Every element of h and dX at sizes the oracle cannot produce whole: each row and
+    each column of the GPU result, projected on a random +-1 vector (fp64, on the
+    device), against the oracle's projection of the definition.  Per element the GPU
+    result carries rounding error of at most ~2^-8 of the element scale (bf16 output,
+    bf16 s.xa / s.g, fp32 accumulation; the 4-bit weight's bf16 rounding included), with
+    independent signs, so a projection over N terms is allowed 8 sigma of that random
+    walk, sigma = sqrt(N) * 2^-8 / sqrt(3) * rms(reference), rms taken from the oracle's
+    exact rows `ref`.  A wrong tile, row, column or term moves its projections by far
+    more.  Returns the largest residual / allowance (for reporting)."""
+    sp = inp.spec
+    rng = np.random.default_rng(0xC0DE + seed)
+    M, di, do = sp.M, sp.d_in, sp.d_out
+    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W=inp.W)
+    u = rng.choice([-1.0, 1.0], M)
+    v_h = rng.choice([-1.0, 1.0], do)
+    v_x = rng.choice([-1.0, 1.0], di)
+    worst = 0.0
+    for name, out, v, proj in (("h", dl.h, v_h, oracle.h_projections), ("dX", dl.dX, v_x, oracle.dx_projections)):
+        if name == "h":
+            row_ref, col_ref = proj(inp.x, inp.A, inp.B, sp.s, v, u, **wkw)
+        else:
+            row_ref, col_ref = proj(inp.dY, inp.A, inp.B, sp.s, v, u, **wkw)
+        od = out.double()
+        row = (od @ torch.from_numpy(v).to(od.device)).cpu().numpy()
+        col = (torch.from_numpy(u).to(od.device) @ od).cpu().numpy()
+        del od
+        rms = float(np.sqrt(np.mean(ref[name] ** 2)))
+        for what, got, want, n in (("row", row, row_ref, out.shape[1]), ("column", col, col_ref, out.shape[0])):
+            allow = 8.0 * np.sqrt(n) * 2.0 ** -8 / np.sqrt(3.0) * rms
+            resid = np.abs(got - want)
+            i = int(np.argmax(resid))
+            assert resid[i] <= allow, (f"{name} {what} projection {i}: got {got[i]:.6g}, oracle {want[i]:.6g}, "
+                                       f"|diff| {resid[i]:.3g} > {allow:.3g}")
+            worst = max(worst, float(resid[i] / allow))
+    return worst

@@ -245,3 +245,25 @@ def test_row_selection_matches_full():
     dxs = oracle.backward(dY, x, A, B, 2.0, W=W, rows=rows)["dX"]
     np.testing.assert_array_equal(hs, full["h"][rows])
     np.testing.assert_array_equal(dxs, full["dX"][rows])
+
+
+@pytest.mark.parametrize("q4", [False, True], ids=["bf16", "q4"])
+def test_projections_match_full_outputs(q4):
+    """The row/column projections used to cover every element at full sizes equal the
+    projections of the oracle's full h and dX (associativity, fp64 rounding only), also
+    when the weight is taken in several row blocks."""
+    spec = inputs.LayerSpec("proj", 37, 128, 80, 8, alpha=16.0, q4=q4, seed=0x9E)
+    inp = inputs.make_inputs(spec)
+    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if q4 else dict(W=inp.W)
+    h_full, xa_ = oracle.forward(inp.x, inp.A, inp.B, spec.s, **wkw)
+    bwd = oracle.backward(inp.dY, inp.x, inp.A, inp.B, spec.s, **wkw)
+    rng = np.random.default_rng(3)
+    v_h, u = rng.choice([-1.0, 1.0], 80), rng.choice([-1.0, 1.0], 37)
+    v_x = rng.choice([-1.0, 1.0], 128)
+    for blk in (2048, 24):
+        row, col = oracle.h_projections(inp.x, inp.A, inp.B, spec.s, v_h, u, block_rows=blk, **wkw)
+        np.testing.assert_allclose(row, h_full @ v_h, rtol=0, atol=1e-12 * np.abs(h_full).sum(1).max())
+        np.testing.assert_allclose(col, u @ h_full, rtol=0, atol=1e-12 * np.abs(h_full).sum(0).max())
+        row, col = oracle.dx_projections(inp.dY, inp.A, inp.B, spec.s, v_x, u, block_rows=blk, **wkw)
+        np.testing.assert_allclose(row, bwd["dX"] @ v_x, rtol=0, atol=1e-12 * np.abs(bwd["dX"]).sum(1).max())
+        np.testing.assert_allclose(col, u @ bwd["dX"], rtol=0, atol=1e-12 * np.abs(bwd["dX"]).sum(0).max())

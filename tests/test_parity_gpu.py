@@ -2,14 +2,15 @@
 
 Small and ragged shapes compare every output element; the full-size workloads
 compare every element of dA and dB and sampled token rows of h and dX (rows the
-oracle computes one by one), in the same launch configuration the benchmark times.
+oracle computes one by one), in the same launch configuration the benchmark times,
+and cover every other element of h and dX through all row and column projections.
 """
 import numpy as np
 import pytest
 import torch
 
-from lora_cases import (DeviceLayer, assert_close, compare_all, oracle_ref, sample_rows, TOL_AB, TOL_HX, RMS_AB,
-                        RMS_HX)
+from lora_cases import (DeviceLayer, assert_close, check_projections, compare_all, oracle_ref, sample_rows, TOL_AB,
+                        TOL_HX, RMS_AB, RMS_HX)
 from rank_linear_lora_b200 import inputs
 from rank_linear_lora_b200 import lora_linear as L
 
@@ -259,3 +260,34 @@ def test_full_size_sampled(cfg):
     got = dl.results(rows=rows)
     ref = oracle_ref(inp, rows=rows)
     compare_all(got, ref, spec.s)
+    # every other element of h and dX: all row and column projections
+    worst = check_projections(dl, inp, ref, seed=idx * 10 + layer)
+    print(f"projection residual / allowance: {worst:.3f}")
+
+
+def test_data_parallel_shards_sum_to_full_batch():
+    """Data parallel over tokens on one GPU: the layer run on two token shards, each
+    backward writing into its own packed [dA | dB] buffer, sums (what the all-reduce
+    does across ranks) to the whole batch's dA and dB; every shard's buffer is bitwise
+    what the backward writes into separately allocated dA and dB."""
+    from rank_linear_lora_b200.dp import PackedGrads, token_shard
+    spec = inputs.LayerSpec("dp", 645, 512, 320, 16, alpha=32.0, seed=0xDB)
+    inp = inputs.make_inputs(spec)
+    total = PackedGrads(spec.r, spec.d_in, spec.d_out, device="cuda").zero_()
+    for rank in range(2):
+        start, count = token_shard(spec.M, 2, rank)
+        sp = spec.with_(M=count)
+        shard = inputs.LayerInputs(sp, inp.x[start:start + count], inp.A, inp.B, inp.dY[start:start + count], inp.W,
+                                   None, None)
+        dl = DeviceLayer(shard)
+        dl.forward()
+        dl.backward()
+        packed = PackedGrads(spec.r, spec.d_in, spec.d_out, device="cuda")
+        L.lora_linear_bwd(dl.dY, dl.x, dl.W, dl.A, dl.B, dl.xa, dl.dX, packed.dA, packed.dB, spec.alpha, dl.ws_b)
+        dl.check()
+        torch.cuda.synchronize()
+        assert torch.equal(packed.dA, dl.dA) and torch.equal(packed.dB, dl.dB)
+        total.buf += packed.buf
+    ref = oracle_ref(inp)
+    assert_close("dA", total.dA.cpu().numpy().astype(np.float64), ref["dA"], TOL_AB, RMS_AB)
+    assert_close("dB", total.dB.cpu().numpy().astype(np.float64), ref["dB"], TOL_AB, RMS_AB)
