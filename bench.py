@@ -48,6 +48,9 @@ def parse():
     p.add_argument("--layer", type=int, default=0, help="layer of a multi-layer workload")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--shape", type=str, default=None,
+                   help="M,d_in,d_out: resize the layer (same r, alpha, weight format), e.g. a case small "
+                        "enough for a full profiler capture; the line then names the resized workload")
     return p.parse_args()
 
 
@@ -232,6 +235,10 @@ def main():
     wl = inputs.workload(args.config, r=args.rank_r)
     spec = wl.layers[args.layer]
     workload_name = f"{wl.name} / {spec.name}"
+    if args.shape:
+        M_, di_, do_ = (int(v) for v in args.shape.split(","))
+        spec = spec.with_(M=M_, d_in=di_, d_out=do_)
+        workload_name += f" resized to M{M_} {di_}->{do_}"
 
     if args.impl == "reference":
         out = run_reference(args, spec, workload_name, rank, world)

@@ -584,9 +584,9 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         a.wscale = o.Wscale;
         a.scale_ld = static_cast<int>(o.q_cols / 64);
         a.scale_rows = static_cast<int>(o.q_rows);
-        // packed codes [d_out][d_in / 2] bytes; each dequant warp fetches 32 rows x 32
-        // bytes (64 codes per row) at a time
-        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols / 2, o.q_rows, 32, 32))
+        // packed codes [d_out][d_in / 2] bytes; each dequant warp fetches DQ_QROWS rows
+        // x 32 bytes (64 codes per row) at a time
+        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols / 2, o.q_rows, 32, DQ_QROWS))
             return LORA_ERR_CUDA;
         allow_tail_split = false;
     }

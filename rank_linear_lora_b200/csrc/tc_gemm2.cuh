@@ -13,11 +13,11 @@
 //   warps 2..5  epilogue in both CTAs: each drains its own 128 accumulator rows from
 //               TMEM, reports to the leader's accumulator-empty barrier, and stores
 //               bf16 through 128B-swizzled smem staging with TMA
-//   warps 6..   (4-bit frozen weight only) dequant warps in both CTAs: fetch packed
-//               codes by TMA, decode them to bf16 straight into the B tile of the
-//               weight K segment and report to the leader's B-ready barrier; the
-//               producer then loads only A for those blocks (and A + B for the rank-r
-//               tail blocks, as in the bf16 case)
+//   warps 6..   (4-bit frozen weight only) dequant warps in both CTAs, none on warp
+//               1's scheduler: fetch packed codes by TMA, decode them to bf16 straight
+//               into the B tile of the weight K segment and report to the leader's
+//               B-ready barrier; the producer then loads only A for those blocks (and
+//               A + B for the rank-r tail blocks, as in the bf16 case)
 //
 // Schedule: whole pair tiles in grouped raster order, `dp_waves` per cluster; a
 // partial last wave of `tail_tiles` tiles is cut along N into two 256 x 128 tiles,
@@ -37,10 +37,31 @@ namespace lora {
 constexpr int PAIR_BM = 256;      // output rows per pair tile (128 per CTA)
 constexpr int PAIR_BN = 256;      // output columns per pair tile
 constexpr int CTA_BN = PAIR_BN / 2;  // B rows (N) staged per CTA
-constexpr int DQ_WARPS = 16;         // 4-bit weight: dequant warps per CTA
-constexpr int DQ_GROUPS = 4;         // groups of dequant warps that take K blocks in turn
-constexpr int DQ_QDEPTH = 2;         // packed-code slots per dequant warp (own K blocks in flight)
-constexpr int DQ_QSLOT = 32 * 32;    // one slot: 32 rows x 32 bytes (64 codes) of the packed weight
+constexpr int DQ_WARPS = 12;         // 4-bit weight: dequant warps per CTA (3 idle warps besides)
+constexpr int DQ_RUNS = 2;           // 32-byte runs of codes (64 elements each) per thread per K block
+constexpr int DQ_GROUP_WARPS = 4 / DQ_RUNS;               // warps decoding one 128-run B tile
+constexpr int DQ_GROUPS = DQ_WARPS / DQ_GROUP_WARPS;       // groups that take K blocks in turn
+constexpr int DQ_QDEPTH = 1;         // packed-code slots per dequant warp (own K blocks in flight)
+constexpr int DQ_QROWS = 32 * DQ_RUNS;                     // runs fetched per warp and K block
+constexpr int DQ_QSLOT = DQ_QROWS * 32;                    // one slot: DQ_QROWS runs x 32 bytes
+
+// A warp's scheduler (SM sub-partition) is its id mod 4.  The single-thread MMA issuer
+// (warp 1) must issue each tcgen05.mma as soon as the tensor core takes the previous one
+// (its queue is about one MMA deep), so no dequant warp shares its sub-partition: warp
+// ids >= 6 that are 1 mod 4 stay idle and the dequant warps take the others in order
+// (measured on the 4-bit up projection: the main GEMMs 1.93 -> 1.72 ms).
+__host__ __device__ constexpr bool dq_idle_warp(int w) { return w >= 6 && w % 4 == 1; }
+// Warp ids from 6 on that host n dequant warps; dequant index of (non-idle) warp w.
+__host__ __device__ constexpr int dq_warp_span(int n) {
+    int w = 6, got = 0;
+    while (got < n) got += dq_idle_warp(w++) ? 0 : 1;
+    return w - 6;
+}
+__host__ __device__ constexpr int dq_index(int w) {
+    int i = 0;
+    for (int v = 6; v < w; ++v) i += dq_idle_warp(v) ? 0 : 1;
+    return i;
+}
 
 template <bool B_MN, bool Q4, int STAGES>
 struct PairCfg {
@@ -51,7 +72,7 @@ struct PairCfg {
     static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
     static constexpr int TMEM_COLS = 2 * PAIR_BN;     // two 256-column accumulators
     static constexpr int BAR_BYTES = Q4 ? 1024 : 512;
-    static constexpr int THREADS = Q4 ? NUM_THREADS + 32 * DQ_WARPS : NUM_THREADS;  // + dequant warps
+    static constexpr int THREADS = Q4 ? NUM_THREADS + 32 * dq_warp_span(DQ_WARPS) : NUM_THREADS;  // + dequant warps
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + Q_BYTES + EPI_BYTES + BAR_BYTES;
     static_assert(STAGES <= 32, "per-stage phase bits are kept in one 32-bit mask");
 };
@@ -163,7 +184,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
         }
         mbar_init(smem_u32(drain_bar), 1);
         if (Q4) {
-            for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * (DQ_WARPS / DQ_GROUPS));
+            for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * DQ_GROUP_WARPS);
             for (int q = 0; q < DQ_WARPS * DQ_QDEPTH; ++q) mbar_init(smem_u32(&qfull_bar[q]), 1);
         }
         *abort_flag = 0;
@@ -360,27 +381,27 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 trace[TR_MMA_WAIT_B] = static_cast<unsigned long long>(wait_b_cyc);
             }
         }
+    } else if (Q4 && warp >= 6 && dq_idle_warp(warp)) {
+        // idle: keeps the MMA issuer's sub-partition free of decode work
     } else if (Q4 && warp >= 6) {
         // ------------------------------------------------------------ dequant warps (both CTAs, Q4)
         // The weight segment's B tiles are decoded here from 4-bit codes.  Warps form
-        // DQ_GROUPS groups of GW; group g takes the weight K blocks g, g + DQ_GROUPS, ... of
-        // the CTA's sequence (the rank-r tail blocks come by TMA and are not touched).  One
-        // thread owns one 32-byte run of codes (64 elements): K-major, weight row rn of the
-        // tile; MN-major, K row rn of 64-column chunk jc.  Each warp fetches its own 32 runs
-        // by TMA into a private DQ_QDEPTH-slot ring, DQ_QDEPTH own blocks ahead, so code
-        // loads never wait for a stage.  Per block: wait for the codes, wait until the MMA
-        // has released the stage's B tile, decode straight into the 128B-swizzled layout
-        // the MMA reads, fence to the async proxy, and arrive (one arrival per warp) on the
-        // leader's B-ready barrier.  One block takes a warp ~2 us end to end (measured;
-        // decode, stores and the cluster-scope release arrival dominate), so DQ_GROUPS
-        // blocks are in flight at once.
-        constexpr int GW = DQ_WARPS / DQ_GROUPS;  // warps per group
-        static_assert(GW * 32 == 128, "one thread per 32-byte run of a 128-run B tile");
-        const int dw = warp - 6;                  // dequant warp 0 .. DQ_WARPS-1
-        const int grp = dw / GW, wg = dw % GW;
-        const int t = wg * 32 + lane;             // run 0..127
-        const int rn = B_MN ? (t & 63) : t;
-        const int jc = B_MN ? (t >> 6) : 0;
+        // DQ_GROUPS groups of DQ_GROUP_WARPS; group g takes the weight K blocks g,
+        // g + DQ_GROUPS, ... of the CTA's sequence (the rank-r tail blocks come by TMA and
+        // are not touched).  A thread owns DQ_RUNS 32-byte runs of codes (64 elements
+        // each): K-major, weight row rn of the tile; MN-major, K row rn of 64-column chunk
+        // jc.  Each warp fetches its own DQ_QROWS runs by TMA into a private DQ_QDEPTH-slot
+        // ring, DQ_QDEPTH own blocks ahead, so code loads never wait for a stage.  Per
+        // block: wait for the codes, wait until the MMA has released the stage's B tile,
+        // decode straight into the 128B-swizzled layout the MMA reads, fence to the async
+        // proxy, and arrive (one arrival per warp) on the leader's B-ready barrier.  The
+        // per-block cost outside the decode (waits, scale fetch, addressing, the
+        // cluster-scope release) is paid once per DQ_RUNS runs, and one block takes a
+        // group microseconds end to end, so DQ_GROUPS blocks are in flight at once.
+        static_assert(DQ_RUNS == 1 || DQ_RUNS == 2, "a warp's runs stay inside one 64-run chunk");
+        const int dw = dq_index(warp);                       // dequant warp 0 .. DQ_WARPS-1
+        const int grp = dw / DQ_GROUP_WARPS, wg = dw % DQ_GROUP_WARPS;
+        const int r0 = wg * DQ_QROWS;                  // the warp's first run; lane owns r0 + lane + 32 i
         uint8_t *qring = sQ + dw * (DQ_QDEPTH * DQ_QSLOT);
         uint64_t *qbar = qfull_bar + dw * DQ_QDEPTH;
         const uint32_t bready_leader0 = mapa_shared(smem_u32(&bready_bar[0]), 0);
@@ -414,18 +435,21 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 enter_item(c);
             }
         };
-        // Lane 0: TMA of this warp's 32 runs of own block c.j into slot c.j % DQ_QDEPTH.
+        // Lane 0: TMA of this warp's DQ_QROWS runs of own block c.j into slot c.j % DQ_QDEPTH.
         auto issue = [&](const Cursor &c) {
             const uint32_t bar = smem_u32(&qbar[c.j % DQ_QDEPTH]);
             const uint32_t dst = smem_u32(qring + (c.j % DQ_QDEPTH) * DQ_QSLOT);
             mbar_arrive_expect_tx(bar, static_cast<uint32_t>(DQ_QSLOT));
-            if (B_MN)  // K rows kb*64 + 32*(wg&1) .., bytes of d_in columns b_row + 64*(wg>>1) ..
-                tma_load_2d(dst, &p.tmQ, bar, c.b_row / 2 + 32 * (wg >> 1), c.kb * BK + 32 * (wg & 1));
-            else       // weight rows b_row + 32*wg .., bytes of K columns kb*64 ..
-                tma_load_2d(dst, &p.tmQ, bar, c.kb * (BK / 2), c.b_row + 32 * wg);
+            if (B_MN)  // K rows kb*64 + (r0 % 64) .., bytes of d_in columns b_row + 64*(r0 / 64) ..
+                tma_load_2d(dst, &p.tmQ, bar, c.b_row / 2 + 32 * (r0 >> 6), c.kb * BK + (r0 & 63));
+            else       // weight rows b_row + r0 .., bytes of K columns kb*64 ..
+                tma_load_2d(dst, &p.tmQ, bar, c.kb * (BK / 2), c.b_row + r0);
         };
-        // Raw bf16 bits of this thread's group scale for own block c.j (0 outside the weight).
-        auto scale_bits = [&](const Cursor &c) -> uint32_t {
+        // Raw bf16 bits of the group scale of this thread's run i in own block c.j (0
+        // outside the weight).  K-major: weight row rn; MN-major: K row rn, chunk jc.
+        auto scale_bits = [&](const Cursor &c, int i) -> uint32_t {
+            const int run = r0 + lane + 32 * i;
+            const int rn = B_MN ? (run & 63) : run, jc = B_MN ? (run >> 6) : 0;
             if (!c.valid) return 0u;
             const int srow = B_MN ? c.kb * BK + rn : c.b_row + rn;
             const int scol = B_MN ? (c.b_row + 64 * jc) / 64 : c.kb;
@@ -443,7 +467,9 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             ++issued;
             step(ahead);
         }
-        uint32_t sc = scale_bits(cur);  // fetched one own block ahead (at the end of the previous one)
+        uint32_t sc[DQ_RUNS];  // fetched one own block ahead (at the end of the previous one)
+#pragma unroll
+        for (int i = 0; i < DQ_RUNS; ++i) sc[i] = scale_bits(cur, i);
         while (cur.valid) {
             const int j = cur.j;
             const int flat = cur.item * kb_all + cur.kb;
@@ -454,10 +480,6 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                                                       abort_flag, p.err, DERR_WAIT_FULL)))
                 break;
             const long long c1 = tr_dq ? clock64() : 0;
-            const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * DQ_QSLOT + (t & 31) * 32);
-            const uint4 v0 = src[0], v1 = src[1];
-            const float s7 = __uint_as_float(sc << 16) / 7.0f;
-            const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
             const long long c2 = tr_dq ? clock64() : 0;
             // The stage's B tile is free once the producer has seen the MMA release it.
             // Lane 0 polls; the warp barrier passes its acquire on to the other lanes.
@@ -468,10 +490,21 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             __syncwarp();
             if (!__shfl_sync(0xffffffffu, granted, 0)) break;
             const long long c3 = tr_dq ? clock64() : 0;
-            uint8_t *row = sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
-            const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = q4_decode8(wds[c], s7x2);
+            for (int i = 0; i < DQ_RUNS; ++i) {
+                const int run = r0 + lane + 32 * i;
+                const int rn = B_MN ? (run & 63) : run, jc = B_MN ? (run >> 6) : 0;
+                const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * DQ_QSLOT + (lane + 32 * i) * 32);
+                const uint4 v0 = src[0], v1 = src[1];
+                const float s7 = __uint_as_float(sc[i] << 16) / 7.0f;
+                const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
+                uint8_t *row =
+                    sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
+                const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = q4_decode8(wds[c], s7x2);
+            }
             // Orders the B-tile stores (and this slot's code reads, whose values are used
             // above) before the tensor core's reads and the slot's next TMA write.
             fence_proxy_async_smem();
@@ -487,7 +520,8 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 step(ahead);
             }
             step(cur);
-            sc = scale_bits(cur);
+#pragma unroll
+            for (int i = 0; i < DQ_RUNS; ++i) sc[i] = scale_bits(cur, i);
             if (tr_dq) {
                 const long long c5 = clock64();
                 dq_wait += c1 - c0;
