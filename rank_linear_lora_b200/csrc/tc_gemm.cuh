@@ -140,6 +140,7 @@ struct GemmCfg {
     static_assert(B_BYTES % 1024 == 0, "stage tiles must stay 1024-byte aligned");
     static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM alloc is a power of 2");
     static_assert(EPI != EPI_STORE || BN % 64 == 0, "store epilogue works in 64-column chunks");
+    static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
 };
 
 // Bounded mbarrier wait.  Returns false (and raises the abort flag and the error

@@ -75,6 +75,7 @@ struct PairCfg {
     static constexpr int THREADS = Q4 ? NUM_THREADS + 32 * dq_warp_span(DQ_WARPS) : NUM_THREADS;  // + dequant warps
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + Q_BYTES + EPI_BYTES + BAR_BYTES;
     static_assert(STAGES <= 32, "per-stage phase bits are kept in one 32-bit mask");
+    static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
 };
 
 // Two codes, each given as the fp32 bit pattern of 2^23 + q, to the bf16 pair
