@@ -93,10 +93,8 @@ def stored_traffic(kind: str, workload: str):
     d = json.load(open(path))
     if d.get("kernel_source_hash") != kernel_source_hash():
         return None
-    e = d.get("kernels", {}).get(kind)
-    if not e or e.get("workload") != workload:
-        return None
-    return e.get("dram_bytes_per_launch")
+    e = d.get("workloads", {}).get(workload, {}).get("kernels", {}).get(kind)
+    return e.get("dram_bytes_per_launch") if e else None
 
 
 class ClockSampler:
