@@ -379,48 +379,79 @@ def main():
                  "definition": f"max(FLOP / bf16 {peak_kind} peak, algorithmic bytes / HBM peak) over the measured step time"}
     kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
 
-    # end to end through the C ABI with host buffers: H2D of the step's inputs from pinned
-    # memory, fwd + bwd, D2H of the step's outputs (W stays resident: frozen model state).
+    # end to end through the C ABI with host buffers: every step copies its inputs in from
+    # pinned host memory and its outputs back out (W stays resident: frozen model state).
+    # Steps are pipelined the way a training loop overlaps its data movement: copies in
+    # on one stream, fwd + bwd on the launch stream, copies out on a third, over two
+    # device buffer sets; events order each step's copy-in -> compute -> copy-out and
+    # keep a set from being overwritten before its previous step is done with it.
     e2e = None
     if not args.no_e2e:
-        s = sets[0]
+        pair = sets[:2]
         names_in = ["x", "dY", "A", "B"]
         names_out = ["h", "dX", "dA", "dB"]
-        hin = {k: torch.empty_like(s[k], device="cpu").pin_memory() for k in names_in}
+        hin = {k: torch.empty_like(pair[0][k], device="cpu").pin_memory() for k in names_in}
         for k in names_in:
-            hin[k].copy_(s[k])
-        hout = {k: torch.empty_like(s[k], device="cpu").pin_memory() for k in names_out}
+            hin[k].copy_(pair[0][k])
+        hout = {k: torch.empty_like(pair[0][k], device="cpu").pin_memory() for k in names_out}
         n_e2e = max(5, min(args.steps, 50))
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
 
-        def e2e_step():
-            for k in names_in:
-                s[k].copy_(hin[k], non_blocking=True)
-            step(s)
-            for k in names_out:
-                hout[k].copy_(s[k], non_blocking=True)
+        def e2e_run(n):
+            computed = [None, None]   # per set: its last step's fwd + bwd finished
+            copied_out = [None, None]  # per set: its last step's outputs copied out
+            for i in range(n):
+                j = i % 2
+                st = pair[j]
+                if computed[j] is not None:
+                    s_in.wait_event(computed[j])
+                with torch.cuda.stream(s_in):
+                    for k in names_in:
+                        st[k].copy_(hin[k], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(s_in)
+                stream.wait_event(ev_in)
+                if copied_out[j] is not None:
+                    stream.wait_event(copied_out[j])
+                with torch.cuda.stream(stream):
+                    step(st)
+                ev_c = torch.cuda.Event()
+                ev_c.record(stream)
+                computed[j] = ev_c
+                s_out.wait_event(ev_c)
+                with torch.cuda.stream(s_out):
+                    for k in names_out:
+                        hout[k].copy_(st[k], non_blocking=True)
+                ev_o = torch.cuda.Event()
+                ev_o.record(s_out)
+                copied_out[j] = ev_o
 
-        for _ in range(2):
-            e2e_step()
+        e2e_run(2)
         barrier()
         torch.cuda.synchronize()
-        torch.cuda._sleep(int(2e6))
+        with torch.cuda.stream(s_in):
+            torch.cuda._sleep(int(2e6))
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        e2e_run(n_e2e)
+        s_out.wait_stream(stream)
+        e1.record(s_out)
         torch.cuda.synchronize()
         barrier()
         te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e_ms = float(te.item())
+        for st in pair:
+            L.lora_linear_check(st["wsf"])
+            L.lora_linear_check(st["wsb"])
         e2e = {"value": flops_step * n_e2e * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": int(sum(hin[k].numel() * hin[k].element_size() for k in names_in)),
                "d2h_bytes_per_step": int(sum(hout[k].numel() * hout[k].element_size() for k in names_out)),
                "ms_per_step": e2e_ms / n_e2e, "steps": n_e2e,
-               "note": "pinned host buffers; frozen W resident on the device"}
+               "note": "pinned host buffers; frozen W resident on the device; copies in, fwd+bwd and copies "
+                       "out pipelined over two device buffer sets on three streams"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
