@@ -174,6 +174,19 @@ LORA_API lora_status_t lora_linear_check(void *workspace, void *stream);
 /* Static description of a status code; never NULL. */
 LORA_API const char *lora_status_string(lora_status_t status);
 
+/* Failure-path self-test (no counterpart in the pages: it tests this library's
+ * bounded waits).  Enqueues on `stream` a one-warp kernel that waits, through the same
+ * bounded-wait routine the layer's kernels use, on a barrier nothing arrives on; after
+ * `limit_us` microseconds (1 .. 2000000) the wait gives up and records its code in the
+ * error word of `workspace` (any workspace from lora_linear_workspace_size, 256-byte
+ * aligned), exactly as a stalled pipeline stage would, and the kernel returns: the GPU
+ * is neither hung nor faulted.  A following lora_linear_check(workspace, stream)
+ * then returns LORA_ERR_TIMEOUT and clears the word.  Returns LORA_OK once enqueued,
+ * LORA_ERR_WORKSPACE / LORA_ERR_MISALIGNED / LORA_ERR_INVALID_ARG for bad arguments,
+ * LORA_ERR_UNSUPPORTED off sm_100, LORA_ERR_CUDA if the launch fails. */
+LORA_API lora_status_t lora_linear_selftest_timeout(void *workspace, size_t ws_bytes, uint32_t limit_us,
+                                                    void *stream);
+
 /* ---- measurement hooks (no effect on results) ---------------------------------
  * Kernel kinds, in the order a forward + backward launches them. */
 typedef enum {

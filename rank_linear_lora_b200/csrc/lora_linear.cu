@@ -815,6 +815,34 @@ lora_status_t lora_linear_check(void *workspace, void *stream) {
     return LORA_OK;
 }
 
+// Failure-path self-test: one warp waits, through the kernels' own bounded wait, on an
+// mbarrier that nothing ever arrives on; the wait runs out after `limit_ns` and records
+// its code in the error word, as a stalled pipeline stage in the layer's kernels would.
+__global__ void k_wait_selftest(int *err, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ volatile int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) wait_bounded(smem_u32(&bar), 0, &abort_flag, err, DERR_WAIT_FULL, limit_ns);
+}
+
+lora_status_t lora_linear_selftest_timeout(void *workspace, size_t ws_bytes, uint32_t limit_us, void *stream) {
+    if (!workspace || ws_bytes < sizeof(int)) return LORA_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return LORA_ERR_MISALIGNED;
+    if (limit_us == 0 || limit_us > 2000000u) return LORA_ERR_INVALID_ARG;
+    int dev = 0;
+    DevInfo *info = nullptr;
+    if (!device_info(&dev, &info)) return LORA_ERR_CUDA;
+    if (!info->supported) return LORA_ERR_UNSUPPORTED;
+    k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<int *>(workspace),
+                                                                     uint64_t(limit_us) * 1000u);
+    return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
 const char *lora_status_string(lora_status_t status) {
     switch (status) {
         case LORA_OK: return "ok";

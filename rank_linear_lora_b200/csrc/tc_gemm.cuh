@@ -144,17 +144,17 @@ struct GemmCfg {
 };
 
 // Bounded mbarrier wait.  Returns false (and raises the abort flag and the error
-// word) if the barrier does not reach `parity` within WAIT_LIMIT_NS, or if another
-// role already aborted.
+// word) if the barrier does not reach `parity` within `limit_ns` (WAIT_LIMIT_NS unless
+// a self-test shortens it), or if another role already aborted.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                             int *err, int code) {
+                                             int *err, int code, uint64_t limit_ns = WAIT_LIMIT_NS) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 31u) == 0) {
             if (*abort_flag) return false;
-            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicCAS(err, 0, code);
                 return false;

@@ -191,6 +191,17 @@ def lora_linear_check(ws, stream=None):
     _check(load_library().lora_linear_check(_ptr(ws), _stream(stream)), "lora_linear_check")
 
 
+def lora_linear_selftest_timeout(ws, limit_us: int = 1000, stream=None):
+    """Enqueue the failure-path self-test on the workspace's error word (a bounded wait
+    that runs out after limit_us); lora_linear_check then raises LORA_ERR_TIMEOUT."""
+    lib = load_library()
+    fn = lib.lora_linear_selftest_timeout
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us), _stream(stream)),
+           "lora_linear_selftest_timeout")
+
+
 def lora_linear_launch_count() -> int:
     return int(load_library().lora_linear_launch_count())
 

@@ -66,3 +66,16 @@ def test_validation_before_any_device_work(lib):
     st = lib.lora_linear_bwd(P(0x1000), P(0x2000), P(0x3000), P(0x4000), P(0x5000), None, None, None, P(0x7000),
                              64, 256, 256, 8, 16.0, P(0x10000), 1 << 30, None)
     assert st == 1  # dA is required
+
+
+def test_selftest_timeout_argument_checks(lib):
+    """The failure-path self-test rejects bad arguments on the host, before any launch."""
+    fn = lib.lora_linear_selftest_timeout
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    P = ctypes.c_void_p
+    assert fn(None, 1024, 1000, None) == 4           # LORA_ERR_WORKSPACE
+    assert fn(P(0x1000), 2, 1000, None) == 4         # smaller than the error word
+    assert fn(P(0x1004), 1024, 1000, None) == 2      # LORA_ERR_MISALIGNED
+    assert fn(P(0x1000), 1024, 0, None) == 1         # LORA_ERR_INVALID_ARG
+    assert fn(P(0x1000), 1024, 2000001, None) == 1

@@ -291,3 +291,21 @@ def test_data_parallel_shards_sum_to_full_batch():
     ref = oracle_ref(inp)
     assert_close("dA", total.dA.cpu().numpy().astype(np.float64), ref["dA"], TOL_AB, RMS_AB)
     assert_close("dB", total.dB.cpu().numpy().astype(np.float64), ref["dB"], TOL_AB, RMS_AB)
+
+
+def test_bounded_wait_timeout_is_reported_and_recoverable():
+    """A device wait that can never complete (nothing arrives on its barrier) runs out,
+    records LORA_ERR_TIMEOUT in the workspace error word, and returns: the check reports
+    it once, clears it, and the same workspace and context then run a layer correctly."""
+    spec = inputs.LayerSpec("after-timeout", 200, 256, 192, 8, alpha=16.0, seed=0x7E)
+    inp = inputs.make_inputs(spec)
+    dl = DeviceLayer(inp)
+    L.lora_linear_selftest_timeout(dl.ws_f, 2000)  # 2 ms
+    with pytest.raises(L.LoraError) as e:
+        L.lora_linear_check(dl.ws_f)
+    assert e.value.status == 6  # LORA_ERR_TIMEOUT
+    L.lora_linear_check(dl.ws_f)  # cleared
+    dl.forward()
+    dl.backward()
+    dl.check()
+    compare_all(dl.results(), oracle_ref(inp), spec.s)
