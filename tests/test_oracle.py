@@ -267,3 +267,28 @@ def test_projections_match_full_outputs(q4):
         row, col = oracle.dx_projections(inp.dY, inp.A, inp.B, spec.s, v_x, u, block_rows=blk, **wkw)
         np.testing.assert_allclose(row, bwd["dX"] @ v_x, rtol=0, atol=1e-12 * np.abs(bwd["dX"]).sum(1).max())
         np.testing.assert_allclose(col, u @ bwd["dX"], rtol=0, atol=1e-12 * np.abs(bwd["dX"]).sum(0).max())
+
+
+def test_matches_library_matmul_at_attention_projection_size():
+    """The oracle at the attention-projection size (M=4096, 4096x4096, r=8, its seeded
+    inputs) against numpy fp64: every element of xa, g, dA, dB, and 16 token rows of h
+    and dX (the oracle's row mode, which the full-size GPU tests use)."""
+    spec = inputs.workload(1).layers[0]
+    inp = inputs.make_inputs(spec)
+    s = spec.s
+    rows = np.array([0, 1, 127, 128, 255, 1000, 2047, 2048, 2049, 3000, 3967, 3968, 4000, 4094, 4095, 511])
+    h_rows, xa_ = oracle.forward(inp.x, inp.A, inp.B, s, W=inp.W, rows=rows)
+    bwd = oracle.backward(inp.dY, inp.x, inp.A, inp.B, s, W=inp.W, rows=rows, xa_=xa_)
+    X, Wd, Ad, Bd, dYd = map(f64, (inp.x, inp.W, inp.A, inp.B, inp.dY))
+    xa_ref = X @ Ad.T
+    g_ref = dYd @ Bd
+    ref = {
+        "xa": (xa_, xa_ref),
+        "g": (bwd["g"], g_ref),
+        "dB": (bwd["dB"], s * dYd.T @ xa_ref),
+        "dA": (bwd["dA"], s * g_ref.T @ X),
+        "h": (h_rows, X[rows] @ Wd.T + s * xa_ref[rows] @ Bd.T),
+        "dX": (bwd["dX"], dYd[rows] @ Wd + s * g_ref[rows] @ Ad),
+    }
+    for key, (got, want) in ref.items():
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-12 * np.abs(want).max(), err_msg=key)
