@@ -379,6 +379,43 @@ def main():
                  "definition": f"max(FLOP / bf16 {peak_kind} peak, algorithmic bytes / HBM peak) over the measured step time"}
     kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
 
+    # The deploy-time merge W' = W + s.B.A of the same layer (HBM-bound: one read of the
+    # weight, one write of W'), timed per launch with CUDA events on the launch stream,
+    # median of 20.  Before each launch L2 is flushed by reading 256 MB (clean lines: a
+    # write would leave ~126 MB of dirty lines for the merge to write back).
+    merge = None
+    if rank == 0:
+        s0 = sets[0]
+        w_out = torch.empty(do, di, dtype=torch.bfloat16, device=dev)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+
+        def merge_once():
+            if spec.q4:
+                L.lora_linear_merge_q4(s0["Wq"], s0["Wscale"], s0["A"], s0["B"], w_out, alpha)
+            else:
+                L.lora_linear_merge(s0["W"], s0["A"], s0["B"], w_out, alpha)
+
+        for _ in range(3):
+            merge_once()
+        times = []
+        for _ in range(20):
+            flush.sum()
+            m0 = torch.cuda.Event(enable_timing=True)
+            m1 = torch.cuda.Event(enable_timing=True)
+            m0.record(stream)
+            merge_once()
+            m1.record(stream)
+            torch.cuda.synchronize()
+            times.append(m0.elapsed_time(m1))
+        del flush
+        t_merge = sorted(times)[len(times) // 2]
+        w_bytes = (do * di // 2 + do * (di // 64) * 2) if spec.q4 else do * di * 2
+        m_bytes = w_bytes + r * di * 2 + do * r * 2 + do * di * 2
+        ach = m_bytes / (t_merge * 1e-3) / 1e9
+        merge = {"us": t_merge * 1e3, "bytes": m_bytes, "achieved_gbs": ach, "peak_gbs": peaks["hbm_gbs"],
+                 "frac": ach / peaks["hbm_gbs"], "bound": "hbm",
+                 "what": "W' = W + s.B.A (4-bit W decoded)" if spec.q4 else "W' = W + s.B.A"}
+
     # end to end through the C ABI with host buffers: every step copies its inputs in from
     # pinned host memory and its outputs back out (W stays resident: frozen model state).
     # Steps are pipelined the way a training loop overlaps its data movement: copies in
@@ -474,6 +511,7 @@ def main():
             "clocks": clocks,
             "e2e": e2e,
             "gpu_launches": int(launches),
+            "merge": merge,
             "host_enqueue_ms": host_enqueue_ms,
         }
         print(json.dumps(out), flush=True)

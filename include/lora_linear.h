@@ -174,6 +174,38 @@ LORA_API lora_status_t lora_linear_check(void *workspace, void *stream);
 /* Static description of a status code; never NULL. */
 LORA_API const char *lora_status_string(lora_status_t status);
 
+/*
+ * Merge the adapter into the frozen weight for deployment:
+ *     W_out = W + s * B . A,   s = alpha / r
+ * (page "ms-swift框架下UnSloth与Liger-Kernel优化实战", section 设计权衡与最佳实践, item 4:
+ * the model is exported in the standard format, adapter merged, before inference).
+ *   W, W_out  bf16 [d_out, d_in] row-major, 16-byte aligned; W_out may equal W (in place)
+ *             but must not otherwise overlap it.
+ *   A [r, d_in], B [d_out, r]  bf16 row-major (A 16-byte aligned).
+ * Per element: w + s * sum_j B[n, j] * A[j, k] in fp32 (the bf16 products are exact,
+ * summed in j order), rounded once to bf16.  For r <= 64 a persistent TMA-fed kernel
+ * streams the tiles (bounded waits; see lora_linear_merge_check); larger r uses one CTA
+ * per tile.  Requires 8 <= d_in <= 2^24 with
+ * d_in % 8 == 0, 1 <= d_out <= 2^24, 1 <= r <= 256, r % 8 == 0, finite alpha; otherwise
+ * LORA_ERR_INVALID_ARG / LORA_ERR_MISALIGNED before any launch.  Stream-ordered,
+ * allocates nothing, needs no workspace.
+ */
+LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uint16_t *A, const uint16_t *B, uint16_t *W_out,
+                                         int64_t d_in, int64_t d_out, int r, float alpha, void *stream);
+
+/* The same from the 4-bit weight (codes Wq [d_out, d_in/2], bf16 scales [d_out,
+ * d_in/64], layout as lora_linear_fwd_q4; d_in % 64 == 0):
+ *     W_out = (q - 8) * scale / 7 + s * B . A
+ * with the decoded weight formed in fp32 as in the 4-bit GEMMs, rounded once to bf16. */
+LORA_API lora_status_t lora_linear_merge_q4(const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
+                                            const uint16_t *B, uint16_t *W_out, int64_t d_in, int64_t d_out, int r,
+                                            float alpha, void *stream);
+
+/* Waits for `stream`, then reads and clears the merge kernels' device error word
+ * (their pipeline waits are bounded like the layer's).  LORA_OK, LORA_ERR_TIMEOUT, or
+ * LORA_ERR_CUDA.  Synchronising: for tests and diagnostics. */
+LORA_API lora_status_t lora_linear_merge_check(void *stream);
+
 /* Failure-path self-test (no counterpart in the pages: it tests this library's
  * bounded waits).  Enqueues on `stream` a one-warp kernel that waits, through the same
  * bounded-wait routine the layer's kernels use, on a barrier nothing arrives on; after

@@ -19,4 +19,5 @@ from .oracle import (  # noqa: F401
     backward,
     h_projections,
     dx_projections,
+    merged_weight,
 )

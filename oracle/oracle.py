@@ -230,3 +230,11 @@ def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, g_=None, 
     row = dYf @ w_v + s * (g_ @ (Af @ v))
     col += s * ((g_.T @ u) @ Af)
     return row, col
+
+
+def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None) -> np.ndarray:
+    """The merged weight of step 2, W + s * B . A, in fp64 [d_out, d_in]: the weight for
+    which h = x . (W + s B A)^T (the adapter folded in for deployment).  The 4-bit weight
+    is decoded by the same rule as steps 2 and 4."""
+    d_out, d_in = np.shape(B)[0], np.shape(A)[1]
+    return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale) + s * (_f64(B) @ _f64(A))

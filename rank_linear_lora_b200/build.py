@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "liblora_linear.so")
-SOURCES = [os.path.join(CSRC, "lora_linear.cu"), os.path.join(CSRC, "noalloc.cu")]
+SOURCES = [os.path.join(CSRC, "lora_linear.cu"), os.path.join(CSRC, "noalloc.cu"), os.path.join(CSRC, "merge.cu")]
 def deps() -> list:
     """Every source the library is built from (all of csrc/ and the public header)."""
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cu", ".cuh", ".h"))) + [

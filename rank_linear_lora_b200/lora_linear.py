@@ -191,6 +191,42 @@ def lora_linear_check(ws, stream=None):
     _check(load_library().lora_linear_check(_ptr(ws), _stream(stream)), "lora_linear_check")
 
 
+def lora_linear_merge(W, A, B, W_out, alpha, stream=None):
+    """W_out = W + (alpha / r) * B . A in bf16 (W_out may be W: in place)."""
+    d_out, d_in = W.shape
+    r = A.shape[0]
+    for t, n, s in ((W, "W", (d_out, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (W_out, "W_out", (d_out, d_in))):
+        _bf16(t, n, s)
+    fn = load_library().lora_linear_merge
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, I64, I64, I, F, P]
+    fn.restype = I
+    _check(fn(_ptr(W), _ptr(A), _ptr(B), _ptr(W_out), d_in, d_out, r, float(alpha), _stream(stream)),
+           "lora_linear_merge")
+
+
+def lora_linear_merge_q4(Wq, Wscale, A, B, W_out, alpha, stream=None):
+    """W_out = decode(Wq, Wscale) + (alpha / r) * B . A in bf16."""
+    d_out = Wq.shape[0]
+    r, d_in = A.shape
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((A, "A", (r, d_in)), (B, "B", (d_out, r)), (W_out, "W_out", (d_out, d_in))):
+        _bf16(t, n, s)
+    fn = load_library().lora_linear_merge_q4
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, P, I64, I64, I, F, P]
+    fn.restype = I
+    _check(fn(_ptr(Wq), _ptr(Wscale), _ptr(A), _ptr(B), _ptr(W_out), d_in, d_out, r, float(alpha), _stream(stream)),
+           "lora_linear_merge_q4")
+
+
+def lora_linear_merge_check(stream=None):
+    fn = load_library().lora_linear_merge_check
+    fn.argtypes = [ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(_stream(stream)), "lora_linear_merge_check")
+
+
 def lora_linear_selftest_timeout(ws, limit_us: int = 1000, stream=None):
     """Enqueue the failure-path self-test on the workspace's error word (a bounded wait
     that runs out after limit_us); lora_linear_check then raises LORA_ERR_TIMEOUT."""

@@ -292,3 +292,15 @@ def test_matches_library_matmul_at_attention_projection_size():
     }
     for key, (got, want) in ref.items():
         np.testing.assert_allclose(got, want, rtol=0, atol=1e-12 * np.abs(want).max(), err_msg=key)
+
+
+@pytest.mark.parametrize("q4", [False, True], ids=["bf16", "q4"])
+def test_merged_weight_reproduces_the_forward(q4):
+    """The merged weight the deploy-time merge is checked against gives the oracle's own
+    forward: x . merged^T = h (steps 1-2), for the bf16 and the 4-bit weight."""
+    spec = inputs.LayerSpec("merge", 29, 128, 72, 16, alpha=24.0, q4=q4, seed=0x3E)
+    inp = inputs.make_inputs(spec)
+    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if q4 else dict(W=inp.W)
+    merged = oracle.merged_weight(inp.A, inp.B, spec.s, **wkw)
+    h, _ = oracle.forward(inp.x, inp.A, inp.B, spec.s, **wkw)
+    np.testing.assert_allclose(f64(inp.x) @ merged.T, h, rtol=0, atol=1e-12 * np.abs(h).max())
