@@ -379,6 +379,74 @@ def main():
                  "definition": f"max(FLOP / bf16 {peak_kind} peak, algorithmic bytes / HBM peak) over the measured step time"}
     kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
 
+    # Forward and backward separately: events around each call over 50 steps (the event
+    # between them breaks the programmatic-launch overlap of the two, so the parts sum to
+    # a little more than the step).
+    fb = None
+    if world == 1:
+        def fwd_call(st):
+            if spec.q4:
+                L.lora_linear_fwd_q4(st["x"], st["Wq"], st["Wscale"], st["A"], st["B"], st["h"], st["xa"], alpha,
+                                     st["wsf"])
+            else:
+                L.lora_linear_fwd(st["x"], st["W"], st["A"], st["B"], st["h"], st["xa"], alpha, st["wsf"])
+
+        def bwd_call(st):
+            if spec.q4:
+                L.lora_linear_bwd_q4(st["dY"], st["x"], st["Wq"], st["Wscale"], st["A"], st["B"], st["xa"], st["dX"],
+                                     st["dA"], st["dB"], alpha, st["wsb"])
+            else:
+                L.lora_linear_bwd(st["dY"], st["x"], st["W"], st["A"], st["B"], st["xa"], st["dX"], st["dA"],
+                                  st["dB"], alpha, st["wsb"])
+
+        n_fb = 50
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_fb)]
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(5e6 + 2e5 * n_fb))
+        for i in range(n_fb):
+            st = sets[i % N_SETS]
+            evs[i][0].record(stream)
+            fwd_call(st)
+            evs[i][1].record(stream)
+            bwd_call(st)
+            evs[i][2].record(stream)
+        torch.cuda.synchronize()
+        f_ms = sorted(e[0].elapsed_time(e[1]) for e in evs)[n_fb // 2]
+        b_ms = sorted(e[1].elapsed_time(e[2]) for e in evs)[n_fb // 2]
+        fb = {"fwd_us": f_ms * 1e3, "bwd_us": b_ms * 1e3, "note": "medians over 50 steps"}
+
+    # Context, not the reference arm: the unfused composition of the same layer in PyTorch
+    # with autograd (x@W.T + s*(x@A.T)@B.T, cuBLAS bf16), same inputs, same GPU.
+    context = None
+    if world == 1 and not spec.q4:
+        st = sets[0]
+        xg = st["x"].detach().clone().requires_grad_(True)
+        Ag = st["A"].detach().clone().requires_grad_(True)
+        Bg = st["B"].detach().clone().requires_grad_(True)
+        sc = spec.s
+
+        def torch_step():
+            xg.grad = Ag.grad = Bg.grad = None
+            hh = xg @ st["W"].t() + sc * ((xg @ Ag.t()) @ Bg.t())
+            hh.backward(st["dY"])
+
+        for _ in range(3):
+            torch_step()
+        n_t = 20
+        torch.cuda.synchronize()
+        torch.cuda._sleep(int(2e7))
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(n_t):
+            torch_step()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        t_ms = c0.elapsed_time(c1) / n_t
+        context = {"what": "unfused PyTorch composition with autograd (x@W.T + s*(x@A.T)@B.T), bf16, same inputs",
+                   "ms_per_step": t_ms, "tflops": spec.flops / (t_ms * 1e-3) / 1e12}
+        del xg, Ag, Bg
+
     # The deploy-time merge W' = W + s.B.A of the same layer (HBM-bound: one read of the
     # weight, one write of W'), timed per launch with CUDA events on the launch stream,
     # median of 20.  Before each launch L2 is flushed by reading 256 MB (clean lines: a
@@ -512,6 +580,8 @@ def main():
             "e2e": e2e,
             "gpu_launches": int(launches),
             "merge": merge,
+            "fwd_bwd": fb,
+            "context_torch_unfused": context,
             "host_enqueue_ms": host_enqueue_ms,
         }
         print(json.dumps(out), flush=True)
