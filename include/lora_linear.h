@@ -48,6 +48,10 @@
  *   - Device-side waits are bounded.  A wait that runs out sets an error word in the
  *     workspace and the kernels return early; lora_linear_check() reports it.
  *   - No C++ exception crosses this interface.
+ *   - Two environment variables, read at each call, exist for measurement and tests:
+ *     LORA_LINEAR_PAIR=0 runs the main GEMMs on single SMs instead of CTA pairs (the
+ *     4-bit entry points then return LORA_ERR_UNSUPPORTED); LORA_LINEAR_PDL=0 launches
+ *     without programmatic dependent launch.  Results are the same either way.
  */
 #ifndef LORA_LINEAR_H
 #define LORA_LINEAR_H
