@@ -51,7 +51,7 @@
  *   - Two environment variables, read at each call, exist for measurement and tests:
  *     LORA_LINEAR_PAIR=0 runs the main GEMMs on single SMs instead of CTA pairs (the
  *     4-bit entry points then return LORA_ERR_UNSUPPORTED); LORA_LINEAR_PDL=0 launches
- *     without programmatic dependent launch.  Results are the same either way.
+ *     without programmatic dependent launch.  Either way the results meet the same bounds.
  */
 #ifndef LORA_LINEAR_H
 #define LORA_LINEAR_H
