@@ -743,8 +743,13 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
         const MainOperands o = main_operands(wt, dY, sg, A, dX, d_out, d_in);
         LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
     }
-    const int cap = (overlap && idle >= 16) ? idle : PLAN_SMS;
-    LORA_TRY(step_dadb(c, dY, x, sxa, sg, dA, dB, M, d_in, d_out, r, overlap && idle >= 16, cap));
+    // Grid: the idle SMs when they can take all the dB / dA split tiles within about
+    // four each (they then finish close to the dX GEMM); otherwise every SM, the rest of
+    // the CTAs starting as the dX CTAs exit (at M = 16384 only 24 SMs are idle, and 256
+    // tiles on 24 CTAs took 255 us where the full grid takes 72 us).
+    const int64_t dadb_tiles = cdiv(d_out, BM) * c.plan.s_db.splits + cdiv(d_in, BM) * c.plan.s_da.splits;
+    const bool few = overlap && idle >= 16 && dadb_tiles <= 4 * static_cast<int64_t>(idle);
+    LORA_TRY(step_dadb(c, dY, x, sxa, sg, dA, dB, M, d_in, d_out, r, overlap, few ? idle : PLAN_SMS));
     return LORA_OK;
 }
 
