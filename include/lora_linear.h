@@ -256,9 +256,9 @@ LORA_API lora_status_t lora_linear_timing_read(double *ms_per_kind, int64_t *lau
  * it consumed (19); the SM cycle counter after set-up (20) and at exit (21), which
  * with the two ns stamps give the SM clock.  The CTA-pair main GEMMs add, in SM
  * cycles: the MMA issuer's waits for A tiles (22) and for decoded B tiles (23, 4-bit
- * weight), and the first dequant warp's waits for packed codes (24), its decode time
- * (25), store + publish time (26), waits for a free B tile (27) and code-fetch issue
- * time (28).
+ * weight), and the first dequant warp's waits for packed codes (24), its code reads
+ * and scale preparation (25), decode + stores + publish (26), waits for a free B tile
+ * (27) and code-fetch issue (28), summed over its K blocks.
  * Launches whose grid does not fit their share of the buffer are not traced.  Pass
  * NULL to switch tracing off.  Returns LORA_OK or LORA_ERR_MISALIGNED (8 bytes). */
 LORA_API lora_status_t lora_linear_trace_enable(void *device_buffer, size_t bytes);

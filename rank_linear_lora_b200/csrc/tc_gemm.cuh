@@ -120,7 +120,8 @@ enum TraceField {
     TR_CLK_EXIT = 21,    // SM cycle counter at exit (with TR_SETUP/TR_EXIT gives the SM clock)
     // CTA-pair kernel, SM cycles: the MMA issuer's waits for A tiles (full) and, 4-bit
     // weight, for decoded B tiles (B-ready); the first dequant warp's waits for packed
-    // codes, its decode time, its waits for a free B tile and its store + publish time.
+    // codes, its code reads and scale preparation (DECODE), decode + stores + publish
+    // (PUBLISH), waits for a free B tile (SLOT) and code-fetch issue (ISSUE).
     TR_MMA_WAIT_A = 22, TR_MMA_WAIT_B = 23, TR_DQ_WAIT = 24, TR_DQ_DECODE = 25, TR_DQ_PUBLISH = 26,
     TR_DQ_SLOT = 27, TR_DQ_ISSUE = 28,
     TRACE_WORDS = 32
