@@ -73,15 +73,20 @@ def algorithmic_bytes(spec) -> float:
 
 
 def kernel_source_hash() -> str:
-    """Hash of every CUDA source of the library (a stored ncu traffic figure is only
-    reported while the kernels it was measured on are unchanged)."""
+    """Hash of the code of every CUDA source of the library, comments and blank space
+    removed (a stored ncu traffic figure is only reported while the kernels and launches
+    it was measured on are unchanged; editing a comment does not change them)."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_linear_lora_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode())
-                h.update(fh.read())
+            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+                text = fh.read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", "", text)
+            h.update(f.encode())
+            h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
