@@ -80,7 +80,7 @@ def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_linear_lora_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh")):
+        if f.endswith((".cu", ".cuh", ".h")):
             with open(os.path.join(csrc, f), encoding="utf-8") as fh:
                 text = fh.read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)

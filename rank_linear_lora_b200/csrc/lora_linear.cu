@@ -27,6 +27,7 @@
 #include "../../include/lora_linear.h"
 #include "tc_gemm.cuh"
 #include "tc_gemm2.cuh"
+#include "tmap.h"
 
 using namespace lora;
 
@@ -74,53 +75,20 @@ bool device_info(int *dev_out, DevInfo **info) {
 }
 
 // ------------------------------------------------------------------ tensor maps
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
 // Row-major 2D bf16 tensor [rows][cols] (cols contiguous), tile box {box_cols, box_rows},
-// 128-byte swizzle, zero fill outside the tensor.
+// 128-byte swizzle (the tensor cores' operand layout), zero fill outside the tensor.
 bool tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
                uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return lora_host::tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, cols, rows, box_cols, box_rows,
+                              CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 // Row-major 2D uint8 tensor [rows][cols_bytes], box {box_bytes, box_rows}, no swizzle
 // (the packed 4-bit codes, read by threads rather than by the tensor cores).
 bool tmap_u8(CUtensorMap *m, const void *base, uint64_t cols_bytes, uint64_t rows, uint32_t box_bytes,
              uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols_bytes, rows};
-    cuuint64_t strides[1] = {cols_bytes};
-    cuuint32_t box[2] = {box_bytes, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return lora_host::tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, cols_bytes, rows, box_bytes, box_rows,
+                              CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // ------------------------------------------------------------------ timing hooks

@@ -25,6 +25,7 @@
 
 #include "../../include/lora_linear.h"
 #include "tc_gemm.cuh"  // bounded mbarrier waits, TMA and mbarrier wrappers
+#include "tmap.h"
 
 namespace {
 
@@ -324,36 +325,11 @@ lora_status_t merge_checks(const void *w0, const void *A, const void *B, const v
 }
 
 // ------------------------------------------------------------------ host
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
 // Row-major 2D tensor [rows][cols] of `esize`-byte elements, box {box_cols, box_rows},
 // no swizzle (threads read the tiles), zero fill outside.
 bool tmap_plain(CUtensorMap *m, CUtensorMapDataType type, int esize, const void *base, uint64_t cols, uint64_t rows,
                 uint32_t box_cols, uint32_t box_rows) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(esize)};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return lora_host::tmap_2d(m, type, esize, base, cols, rows, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 std::mutex g_err_mu;
