@@ -105,18 +105,31 @@ def stored_traffic(kind: str, workload: str):
 class ClockSampler:
     """NVML clocks and throttle reasons sampled in a thread while the timed region runs."""
 
-    def __init__(self, index: int, period_s: float = 0.01):
-        self.index, self.period, self.samples, self._stop = index, period_s, [], threading.Event()
+    def __init__(self, dev, period_s: float = 0.01):
+        self.period, self.samples, self._stop = period_s, [], threading.Event()
         self.ok = False
         try:
             import pynvml
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.h = self._handle(pynvml, dev)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception:  # pragma: no cover - no NVML
             self.max_mhz = None
+
+    @staticmethod
+    def _handle(nv, dev):
+        """The NVML device of torch device ``dev``, matched by PCI address (NVML numbers
+        every GPU of the machine and ignores CUDA_VISIBLE_DEVICES)."""
+        import torch
+        p = torch.cuda.get_device_properties(dev)
+        for i in range(nv.nvmlDeviceGetCount()):
+            h = nv.nvmlDeviceGetHandleByIndex(i)
+            pci = nv.nvmlDeviceGetPciInfo(h)
+            if (pci.domain, pci.bus, pci.device) == (p.pci_domain_id, p.pci_bus_id, p.pci_device_id):
+                return h
+        raise RuntimeError("no NVML device at the PCI address of %s" % dev)
 
     def _run(self):
         nv = self.nv
@@ -343,7 +356,7 @@ def main():
             rec = L.lora_linear_timing_read()
         return e0.elapsed_time(e1), n1 - n0, rec
 
-    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local)
+    sampler = ClockSampler(dev)
     with sampler:
         ms, launches, _ = timed_region(args.steps)
     clocks = sampler.summary()
