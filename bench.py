@@ -64,11 +64,14 @@ def load_peaks():
 
 
 def algorithmic_bytes(spec) -> float:
-    """One read of every operand and one write of every output per fwd + bwd call."""
+    """One read of every operand and one write of every output per fwd + bwd call.  For
+    projections stacked on one x only the diagonal blocks of B and dB count (rb = r/proj
+    columns per row); A, xa and dA hold every projection's ranks."""
     M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
+    rb = r // spec.proj
     w = do * di // 2 + do * (di // 64) * 2 if spec.q4 else do * di * 2
-    fwd = M * di * 2 + w + r * di * 2 + do * r * 2 + M * do * 2 + M * r * 2
-    bwd = M * do * 2 + M * di * 2 + w + r * di * 2 + do * r * 2 + M * r * 2 + M * di * 2 + r * di * 4 + do * r * 4
+    fwd = M * di * 2 + w + r * di * 2 + do * rb * 2 + M * do * 2 + M * r * 2
+    bwd = M * do * 2 + M * di * 2 + w + r * di * 2 + do * rb * 2 + M * r * 2 + M * di * 2 + r * di * 4 + do * rb * 4
     return float(fwd + bwd)
 
 
@@ -203,6 +206,7 @@ def run_reference(args, spec, workload_name, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": workload_name, "M": spec.M, "d_in": spec.d_in,
                                          "d_out": spec.d_out, "r": spec.r, "alpha": spec.alpha,
+                                         "projections": spec.proj,
                                          "parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
                          "sample": sample},
@@ -379,7 +383,8 @@ def main():
     tokens_per_s = M * world * args.steps / (ms_max * 1e-3)
 
     # roofline of the dominant kernel
-    kern_flops = {"fwd_main": 2.0 * M * do * (di + r), "dx_main": 2.0 * M * di * (do + r)}
+    # (stacked projections: each output column of the forward uses its own r/proj ranks)
+    kern_flops = {"fwd_main": 2.0 * M * do * (di + r // spec.proj), "dx_main": 2.0 * M * di * (do + r)}
     dom = max(("fwd_main", "dx_main"), key=lambda k: rec[k][0])
     dom_ms = rec[dom][0] / max(1, rec[dom][1])
     achieved = kern_flops[dom] / (dom_ms * 1e-3) / 1e12
@@ -586,7 +591,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": workload_name, "M": M, "d_in": di, "d_out": do, "r": r, "alpha": alpha,
-                       "q4": spec.q4, "tokens_per_step": M * world,
+                       "q4": spec.q4, "projections": spec.proj, "tokens_per_step": M * world,
                        "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
                        "parallelism": f"dp{world}"},
             "tokens_per_s": tokens_per_s,

@@ -158,7 +158,13 @@ def unpack_q4_codes(packed: np.ndarray) -> np.ndarray:
 
 @dataclass
 class LayerSpec:
-    """One LoRA linear: M tokens, d_in -> d_out, rank r, scale alpha/r."""
+    """One LoRA linear: M tokens, d_in -> d_out, rank r, scale alpha/r.
+
+    ``proj`` > 1 describes that many projections of one x stacked into one layer
+    (equal sizes d_out/proj and r/proj each, scale alpha/r = (alpha/proj)/(r/proj)):
+    W and A stacked by rows, B block-diagonal [d_out, r] with projection p's rank
+    columns p*r/proj.. used only by its own rows.
+    """
     name: str
     M: int
     d_in: int
@@ -168,6 +174,7 @@ class LayerSpec:
     q4: bool = False
     seed: int = 0
     layer: int = 0
+    proj: int = 1
 
     @property
     def s(self) -> float:
@@ -175,8 +182,10 @@ class LayerSpec:
 
     @property
     def flops(self) -> float:
-        """Algorithmic fwd+bwd FLOPs: 4*M*d_in*d_out + 6*M*r*(d_in+d_out)."""
-        return 4.0 * self.M * self.d_in * self.d_out + 6.0 * self.M * self.r * (self.d_in + self.d_out)
+        """Algorithmic fwd+bwd FLOPs: 4*M*d_in*d_out + 6*M*r*(d_in+d_out) per projection,
+        summed over the ``proj`` projections (the zero blocks of a stacked B are no work)."""
+        rp = self.r // self.proj
+        return 4.0 * self.M * self.d_in * self.d_out + 6.0 * self.M * rp * (self.proj * self.d_in + self.d_out)
 
     def with_(self, **kw) -> "LayerSpec":
         d = dict(self.__dict__)
@@ -195,7 +204,8 @@ def workload(idx: int, r: int | None = None) -> Workload:
 
     0: tiny, M=64, 256->256, r=8, alpha=16.
     1: attention projection, M=4096 (2 x 2048), 4096->4096, r=8, alpha=32.
-    2: one 7B MLP set, M=8192: gate 4096->11008, up 4096->11008, down 11008->4096, r=16, alpha=32.
+    2: one 7B MLP set, M=8192: gate 4096->11008, up 4096->11008, down 11008->4096, r=16, alpha=32;
+       layer 3 is gate and up on one x stacked into one layer (4096->22016, 2 x r16).
     3: rank sweep, M=16384 (2 x 8192), 4096->4096, r in {8,16,64,128}, alpha=16.
     4: 4-bit frozen W, up projection 8192->28672, r=16, alpha=32, M=4096.
     """
@@ -210,6 +220,7 @@ def workload(idx: int, r: int | None = None) -> Workload:
             LayerSpec("gate_proj", 8192, 4096, 11008, 16, 32.0, seed=seed, layer=0),
             LayerSpec("up_proj", 8192, 4096, 11008, 16, 32.0, seed=seed, layer=1),
             LayerSpec("down_proj", 8192, 11008, 4096, 16, 32.0, seed=seed, layer=2),
+            LayerSpec("gate_up_proj", 8192, 4096, 22016, 32, 64.0, seed=seed, layer=3, proj=2),
         ])
     if idx == 3:
         rr = 8 if r is None else r
@@ -242,6 +253,10 @@ def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) 
     bound = 1.0 / math.sqrt(di)
     A = to_bf16_bits(draw("uniform", seed, TID_A + off, r * di, bound)).reshape(r, di)
     B = to_bf16_bits(draw("normal", seed, TID_B + off, do * r, 0.02)).reshape(do, r)
+    if spec.proj > 1:  # stacked projections: keep only the diagonal blocks of B
+        P = spec.proj
+        own = (np.arange(do)[:, None] // (do // P)) == (np.arange(r)[None, :] // (r // P))
+        B = np.where(own, B, np.uint16(0)).astype(np.uint16)
     if zero_A:
         A = np.zeros_like(A)
     if zero_B:

@@ -81,6 +81,16 @@ class DeviceLayer:
                 "dA": host_f64(self.dA), "dB": host_f64(self.dB)}
 
 
+def shared_input_projections(M, d_in, d_outs, r, alpha, q4, seed) -> list:
+    """Inputs of several projections of one x: each its own W, A, B and dY (streams
+    offset by the projection's index), all with the first projection's x."""
+    layers = [inputs.make_inputs(inputs.LayerSpec(f"p{p}", M, d_in, d, r, alpha, q4=q4, seed=seed, layer=p))
+              for p, d in enumerate(d_outs)]
+    for inp in layers[1:]:
+        inp.x = layers[0].x
+    return layers
+
+
 def oracle_ref(inp: inputs.LayerInputs, rows=None) -> dict:
     sp = inp.spec
     wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W=inp.W)

@@ -243,8 +243,8 @@ def test_q4_lora_dominant():
 
 
 # ------------------------------------------------------------------ full sizes
-FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (3, 8, 0), (3, 16, 0), (3, 64, 0), (3, 128, 0),
-        (4, None, 0)]
+FULL = [(1, None, 0), (2, None, 0), (2, None, 1), (2, None, 2), (2, None, 3), (3, 8, 0), (3, 16, 0), (3, 64, 0),
+        (3, 128, 0), (4, None, 0)]
 
 
 @pytest.mark.parametrize("cfg", FULL, ids=lambda c: f"cfg{c[0]}_r{c[1]}_layer{c[2]}")
