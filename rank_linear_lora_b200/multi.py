@@ -20,8 +20,9 @@ dY = [dY_0 | dY_1 | ...] gives g = dY B = [dY_0 B_0 | ...] and
 * the diagonal blocks of dB are the dB_p.  The off-diagonal blocks are gradients of
   entries held at zero; they are computed but never read.
 
-The call passes r_call = P r and alpha_call = P alpha.  Both products are exact in
-fp32 (checked here), so the library's s = alpha_call / r_call equals alpha / r bit for bit.
+The call passes r_call = P r and alpha_call = P alpha.  Both products are exact in fp32
+(checked here for alpha as the library receives it, rounded to fp32), so the library's
+s = alpha_call / r_call is bit for bit the s of a single projection's call.
 
 What the stacking saves: the forward prologue reads x once for all P projections, one
 main GEMM runs with N = sum d_p, the backward reads x once for dA, and dX needs no
@@ -43,8 +44,11 @@ from .dp import PackedGrads
 
 
 def _exact_f32_product(a: float, n: int) -> bool:
-    a32 = np.float32(a)
-    return float(a32) == a and float(np.float32(a32 * np.float32(n))) == float(a32) * n
+    """n times alpha as the library receives it (rounded to fp32) is exact in fp32."""
+    with np.errstate(over="ignore"):
+        a32 = np.float32(a)
+        prod = np.float32(a32 * np.float32(n))
+    return bool(np.isfinite(prod)) and float(prod) == float(a32) * n
 
 
 class SharedInputProjections:
@@ -66,8 +70,8 @@ class SharedInputProjections:
             raise ValueError(f"every projection width must be a multiple of 8 (16-byte rows), got {d_outs}")
         if r < 1 or r % 8 or P * r > 256:
             raise ValueError(f"r={r} with {P} projections: need r % 8 == 0 and P*r <= 256")
-        if not (np.isfinite(alpha) and _exact_f32_product(alpha, P)):
-            raise ValueError(f"alpha={alpha!r}: alpha and {P}*alpha must both be exact in fp32")
+        if not _exact_f32_product(alpha, P):
+            raise ValueError(f"alpha={alpha!r}: {P}*alpha must be exact in fp32")
         self.d_in, self.d_outs, self.r, self.alpha, self.q4 = d_in, d_outs, r, float(alpha), q4
         self.P = P
         self.offsets = np.concatenate([[0], np.cumsum(d_outs)]).astype(int).tolist()

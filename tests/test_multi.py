@@ -106,10 +106,20 @@ def test_views_alias_the_stacked_storage():
     (dict(d_outs=(16,) * 3, r=96, alpha=16.0), "P\\*r <= 256"),
     (dict(d_outs=(16, 16, 16), r=8, alpha=1.0 / 3.0), "exact in fp32"),
     (dict(d_outs=(), r=8, alpha=16.0), "at least one"),
+    (dict(d_outs=(16, 16), r=8, alpha=3e38), "exact in fp32"),          # 2*alpha overflows fp32
+    (dict(d_outs=(16, 16), r=8, alpha=float("nan")), "exact in fp32"),
 ])
 def test_rejects_stacks_the_layer_cannot_take(kw, msg):
     with pytest.raises(ValueError, match=msg):
         SharedInputProjections(64, kw["d_outs"], kw["r"], kw["alpha"])
+
+
+def test_alpha_rounded_to_fp32_as_the_single_call_does():
+    """alpha = 0.1 is not an fp32 value; the library takes it as fp32(0.1), and so does
+    the stack: 2 * fp32(0.1) / 16 is fp32(0.1) / 8 exactly."""
+    st = SharedInputProjections(64, (16, 16), 8, 0.1)
+    a32 = np.float32(0.1)
+    assert np.float32(st.alpha_call) / np.float32(st.r_call) == a32 / np.float32(8)
 
 
 def test_stacked_workload_spec():
