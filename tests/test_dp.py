@@ -86,3 +86,53 @@ def test_allreduce_of_shards_equals_full_batch(tmp_path, M):
         np.testing.assert_allclose(got, ref, rtol=0, atol=4e-7 * np.abs(ref).max())
     # every rank holds the same sum
     assert np.array_equal(np.load(tmp_path / "rank0.npy"), np.load(tmp_path / "rank1.npy"))
+
+
+def _stack(M, d_in, d_outs, r, alpha, seed):
+    """Projections of one x (per-projection seeded inputs) and their stacked layout."""
+    from lora_cases import shared_input_projections
+    from rank_linear_lora_b200.multi import SharedInputProjections
+
+    layers = shared_input_projections(M, d_in, d_outs, r, alpha, False, seed)
+    st = SharedInputProjections(d_in, d_outs, r, alpha)
+    t16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)  # noqa: E731
+    for p, inp in enumerate(layers):
+        st.load(p, W=t16(inp.W), A=t16(inp.A), B=t16(inp.B))
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)  # noqa: E731
+    return layers, st, bits(st.W), bits(st.A), bits(st.B)
+
+
+def _stack_worker(rank, world, port, case, result_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        M, d_in, d_outs, r, alpha, seed = case
+        layers, st, W, A, B = _stack(*case)
+        dY = np.concatenate([inp.dY for inp in layers], axis=1)
+        start, count = token_shard(M, world, rank)
+        bwd = oracle.backward(dY[start:start + count], layers[0].x[start:start + count], A, B,
+                              st.alpha_call / st.r_call, W=W)
+        st.grads.dA.copy_(torch.from_numpy(bwd["dA"]).float())
+        st.grads.dB.copy_(torch.from_numpy(bwd["dB"]).float())
+        st.grads.all_reduce()  # one collective for every projection of the stack
+        np.save(os.path.join(result_dir, f"rank{rank}.npy"), st.grads.buf.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+def test_stacked_projections_reduce_in_one_allreduce(tmp_path):
+    """Projections of one x stacked into one layer: each rank's backward of its token
+    shard fills the stack's packed buffer, one all-reduce sums it, and every
+    projection's dA, dB view then holds that projection's whole-batch gradient."""
+    world, case = 2, (41, 64, (24, 16), 8, 16.0, 0xDA)
+    mp.spawn(_stack_worker, args=(world, _free_port(), case, str(tmp_path)), nprocs=world, join=True)
+    layers, st, *_ = _stack(*case)
+    for rank in range(world):
+        st.grads.buf.copy_(torch.from_numpy(np.load(tmp_path / f"rank{rank}.npy")))
+        for p, (dA_p, dB_p) in enumerate(st.split_grads()):
+            inp = layers[p]
+            full = oracle.backward(inp.dY, inp.x, inp.A, inp.B, inp.spec.s, W=inp.W)
+            for got, ref in ((dA_p, full["dA"]), (dB_p, full["dB"])):
+                np.testing.assert_allclose(got.numpy().astype(np.float64), ref, rtol=0,
+                                           atol=4e-7 * np.abs(ref).max())
