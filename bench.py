@@ -75,21 +75,25 @@ def algorithmic_bytes(spec) -> float:
     return float(fwd + bwd)
 
 
+# The sources the layer's kernels and their launches are built from: lora_linear.cu and
+# every header it includes (the merge and the workspace-free forward are other files).
+LAYER_SOURCES = ("lora_linear.cu", "tc_gemm.cuh", "tc_gemm2.cuh", "ptx.cuh", "tmap.h")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the code of every CUDA source of the library, comments and blank space
-    removed (a stored ncu traffic figure is only reported while the kernels and launches
-    it was measured on are unchanged; editing a comment does not change them)."""
+    """Hash of the code of the layer's CUDA sources, comments and blank space removed (a
+    stored ncu traffic figure is only reported while the kernels and launches it was
+    measured on are unchanged; editing a comment does not change them)."""
     import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rank_linear_lora_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
-                text = fh.read()
-            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-            text = re.sub(r"//[^\n]*", "", text)
-            h.update(f.encode())
-            h.update(" ".join(text.split()).encode())
+    for f in sorted(LAYER_SOURCES):
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(f.encode())
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

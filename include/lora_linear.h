@@ -183,9 +183,9 @@ LORA_API const char *lora_status_string(lora_status_t status);
  *     W_out = W + s * B . A,   s = alpha / r
  * (page "ms-swift框架下UnSloth与Liger-Kernel优化实战", section 设计权衡与最佳实践, item 4:
  * the model is exported in the standard format, adapter merged, before inference).
- *   W, W_out  bf16 [d_out, d_in] row-major, 16-byte aligned; W_out may equal W (in place)
- *             but must not otherwise overlap it.
- *   A [r, d_in], B [d_out, r]  bf16 row-major (A 16-byte aligned).
+ *   W, W_out  bf16 [d_out, d_in] row-major; W_out may equal W (in place) but must not
+ *             otherwise overlap it.
+ *   A [r, d_in], B [d_out, r]  bf16 row-major.  Every pointer 16-byte aligned.
  * Per element: w + s * sum_j B[n, j] * A[j, k] in fp32 (the bf16 products are exact,
  * summed in j order), rounded once to bf16.  For r <= 64 a persistent TMA-fed kernel
  * streams the tiles (bounded waits; see lora_linear_merge_check); larger r uses one CTA
@@ -198,7 +198,8 @@ LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uint16_t *A, c
                                          int64_t d_in, int64_t d_out, int r, float alpha, void *stream);
 
 /* The same from the 4-bit weight (codes Wq [d_out, d_in/2], bf16 scales [d_out,
- * d_in/64], layout as lora_linear_fwd_q4; d_in % 64 == 0):
+ * d_in/64], layout as lora_linear_fwd_q4; d_in % 64 == 0; Wscale non-null and 16-byte
+ * aligned like the other pointers):
  *     W_out = (q - 8) * scale / 7 + s * B . A
  * with the decoded weight formed in fp32 as in the 4-bit GEMMs, rounded once to bf16. */
 LORA_API lora_status_t lora_linear_merge_q4(const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,

@@ -312,15 +312,18 @@ __global__ void __launch_bounds__(THREADS_TMA, 2) k_merge_ring(const __grid_cons
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-lora_status_t merge_checks(const void *w0, const void *A, const void *B, const void *Wout, int64_t d_in,
-                           int64_t d_out, int r, float alpha, bool q4) {
-    if (!w0 || !A || !B || !Wout) return LORA_ERR_INVALID_ARG;
+// Every pointer 16-byte aligned, as for the layer: the ring kernel reads W (or the codes),
+// A and B by TMA and the other kernel reads W and A in 16-byte vectors.
+lora_status_t merge_checks(const void *w0, const void *scale, const void *A, const void *B, const void *Wout,
+                           int64_t d_in, int64_t d_out, int r, float alpha, bool q4) {
+    if (!w0 || !A || !B || !Wout || (q4 && !scale)) return LORA_ERR_INVALID_ARG;
     if (d_in < 8 || d_out < 1 || d_in % 8 || (q4 && d_in % 64)) return LORA_ERR_INVALID_ARG;
     if (d_in > (int64_t(1) << 24) || d_out > (int64_t(1) << 24)) return LORA_ERR_INVALID_ARG;
     if (((d_out + MT - 1) / MT) * ((d_in + NT - 1) / NT) > 0x7FFFFFFF) return LORA_ERR_INVALID_ARG;
     if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
     if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) return LORA_ERR_INVALID_ARG;
-    if (!aligned16(w0) || !aligned16(A) || !aligned16(Wout)) return LORA_ERR_MISALIGNED;
+    if (!aligned16(w0) || !aligned16(A) || !aligned16(B) || !aligned16(Wout) || (q4 && !aligned16(scale)))
+        return LORA_ERR_MISALIGNED;
     return LORA_OK;
 }
 
@@ -402,7 +405,7 @@ lora_status_t merge_launch(bool q4, const uint16_t *W, const uint8_t *Wq, const 
 extern "C" LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uint16_t *A, const uint16_t *B,
                                                     uint16_t *W_out, int64_t d_in, int64_t d_out, int r, float alpha,
                                                     void *stream) {
-    const lora_status_t st = merge_checks(W, A, B, W_out, d_in, d_out, r, alpha, false);
+    const lora_status_t st = merge_checks(W, nullptr, A, B, W_out, d_in, d_out, r, alpha, false);
     if (st != LORA_OK) return st;
     return merge_launch(false, W, nullptr, nullptr, A, B, W_out, d_in, d_out, r, alpha, stream);
 }
@@ -410,9 +413,8 @@ extern "C" LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uin
 extern "C" LORA_API lora_status_t lora_linear_merge_q4(const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
                                                        const uint16_t *B, uint16_t *W_out, int64_t d_in, int64_t d_out,
                                                        int r, float alpha, void *stream) {
-    lora_status_t st = merge_checks(Wq, A, B, W_out, d_in, d_out, r, alpha, true);
+    const lora_status_t st = merge_checks(Wq, Wscale, A, B, W_out, d_in, d_out, r, alpha, true);
     if (st != LORA_OK) return st;
-    if (!Wscale) return LORA_ERR_INVALID_ARG;
     return merge_launch(true, nullptr, Wq, Wscale, A, B, W_out, d_in, d_out, r, alpha, stream);
 }
 

@@ -79,3 +79,31 @@ def test_selftest_timeout_argument_checks(lib):
     assert fn(P(0x1004), 1024, 1000, None) == 2      # LORA_ERR_MISALIGNED
     assert fn(P(0x1000), 1024, 0, None) == 1         # LORA_ERR_INVALID_ARG
     assert fn(P(0x1000), 1024, 2000001, None) == 1
+
+
+def test_merge_argument_checks(lib):
+    """The deploy-time merge validates before touching a device: null or misaligned
+    pointers (every one, B and the 4-bit scales included), shapes, r and alpha."""
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    mg = lib.lora_linear_merge
+    mg.argtypes = [P, P, P, P, I64, I64, I, F, P]
+    mg.restype = I
+    mq = lib.lora_linear_merge_q4
+    mq.argtypes = [P, P, P, P, P, I64, I64, I, F, P]
+    mq.restype = I
+
+    def m(W=0x1000, A=0x2000, B_=0x3000, out=0x4000, di=256, do=64, r=8, alpha=16.0):
+        return mg(P(W), P(A), P(B_), P(out), di, do, r, alpha, None)
+
+    def q(Wq=0x1000, sc=0x5000, A=0x2000, B_=0x3000, out=0x4000, di=256, do=64, r=8, alpha=16.0):
+        return mq(P(Wq), P(sc), P(A), P(B_), P(out), di, do, r, alpha, None)
+
+    for bad in (dict(W=None), dict(A=None), dict(B_=None), dict(out=None), dict(di=4), dict(di=260),
+                dict(do=0), dict(di=(1 << 24) + 8), dict(r=0), dict(r=12), dict(r=264),
+                dict(alpha=float("nan")), dict(alpha=float("inf"))):
+        assert m(**bad) == 1, bad                     # LORA_ERR_INVALID_ARG
+    for bad in (dict(W=0x1008), dict(A=0x2004), dict(B_=0x3002), dict(out=0x4008)):
+        assert m(**bad) == 2, bad                     # LORA_ERR_MISALIGNED
+    assert q(sc=None) == 1                            # the scales are required
+    assert q(di=96) == 1                              # 4-bit weight: d_in % 64 == 0
+    assert q(sc=0x5002) == 2 and q(Wq=0x1008) == 2
