@@ -30,10 +30,15 @@
  *     call returns without waiting.
  *   - Outputs are overwritten, never accumulated into.  Inputs and outputs must not
  *     alias.  Calls on distinct streams with distinct workspaces may run concurrently.
- *   - Validation happens before any launch; on an error status nothing is enqueued.
- *     Required: non-null required pointers; every pointer 16-byte aligned; M >= 1;
- *     d_in and d_out multiples of 8 (>= 8); 1 <= r <= 256 with r % 8 == 0; alpha
- *     finite; for *_q4 also d_in % 64 == 0.
+ *   - Validation happens before any launch; on a validation error (INVALID_ARG,
+ *     MISALIGNED, WORKSPACE, UNSUPPORTED) nothing is enqueued.  LORA_ERR_CUDA from a
+ *     launch may leave the call's earlier kernels enqueued; their outputs are then
+ *     undefined.
+ *     Required: non-null required pointers; every pointer 16-byte aligned;
+ *     1 <= M <= 2^30; d_in and d_out multiples of 8 in 8 .. 2^24, with
+ *     ceil(M/128) * ceil(max(d_in, d_out)/128) <= 2^31 - 1 (32-bit tile counts: only
+ *     an output of more than 2^45 elements reaches it); 1 <= r <= 256 with r % 8 == 0; alpha finite;
+ *     for *_q4 also d_in % 64 == 0.
  *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
  *     aligned, be zero-filled before its first use, and must not be used by two calls
  *     that may run at the same time.  Every call that completes leaves the workspace's

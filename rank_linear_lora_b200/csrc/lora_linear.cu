@@ -386,6 +386,9 @@ lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float 
     if (M < 1 || M > (int64_t(1) << 30)) return LORA_ERR_INVALID_ARG;
     if (d_in < 8 || d_out < 8 || d_in % 8 || d_out % 8) return LORA_ERR_INVALID_ARG;
     if (d_in > (int64_t(1) << 24) || d_out > (int64_t(1) << 24)) return LORA_ERR_INVALID_ARG;
+    // Tile counts are 32-bit: bound the 128 x 128 tiles of the larger output (past this
+    // bound the larger output alone holds more than 2^45 elements).
+    if (((M + 127) / 128) * ((std::max(d_in, d_out) + 127) / 128) > INT32_MAX) return LORA_ERR_INVALID_ARG;
     if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
     if (!std::isfinite(alpha)) return LORA_ERR_INVALID_ARG;
     if (q4 && d_in % 64) return LORA_ERR_INVALID_ARG;

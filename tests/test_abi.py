@@ -60,6 +60,12 @@ def test_validation_before_any_device_work(lib):
     assert _fwd(lib, r=0) == 1
     assert _fwd(lib, r=12) == 1
     assert _fwd(lib, alpha=float("nan")) == 1
+    assert _fwd(lib, M=(1 << 30) + 1) == 1
+    assert _fwd(lib, di=(1 << 24) + 8) == 1
+    assert _fwd(lib, M=1 << 30, di=1 << 24) == 1   # 2^22 x 2^17 tiles: past 32-bit counts
+    # the bound itself: 2^23 x 255 tiles pass, 2^23 x 256 = 2^31 do not
+    assert L.lora_linear_workspace_size(L.OP_FWD, 1 << 30, 32640, 32640, 8) > 0
+    assert L.lora_linear_workspace_size(L.OP_FWD, 1 << 30, 32768, 64, 8) == 0
     assert _fwd(lib, x=0x1008) == 2
     assert _fwd(lib, xa=0x6004) == 2
     P = ctypes.c_void_p
