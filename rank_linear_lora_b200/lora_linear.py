@@ -79,7 +79,24 @@ def _ptr(t):
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
+    elif stream.device_index != torch.cuda.current_device():
+        raise ValueError(f"stream is on cuda:{stream.device_index}, the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _on_current_device(t, name):
+    """The library works on the current device: every tensor must live there."""
+    if not t.is_cuda or t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name}: on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
+
+
+def _ws(ws):
+    """(pointer, bytes) of a workspace tensor: contiguous, on the current device."""
+    if ws is None or not ws.is_contiguous():
+        raise ValueError("workspace: expected a contiguous CUDA tensor")
+    _on_current_device(ws, "workspace")
+    return _ptr(ws), ws.numel() * ws.element_size()
 
 
 def _check(status: int, where: str):
@@ -91,11 +108,13 @@ def _bf16(t, name, shape):
     if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected a contiguous CUDA bfloat16 tensor of shape {tuple(shape)}, "
                          f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+    _on_current_device(t, name)
 
 
 def _f32(t, name, shape):
     if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous() or tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name}: expected a contiguous CUDA float32 tensor of shape {tuple(shape)}")
+    _on_current_device(t, name)
 
 
 def lora_status_string(status: int) -> str:
@@ -124,7 +143,7 @@ def lora_linear_fwd(x, W, A, B, h, xa_save, alpha, ws, stream=None):
     if xa_save is not None:
         _bf16(xa_save, "xa_save", (M, r))
     st = load_library().lora_linear_fwd(_ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(h), _ptr(xa_save), M, d_in, d_out,
-                                        r, float(alpha), _ptr(ws), ws.numel(), _stream(stream))
+                                        r, float(alpha), *_ws(ws), _stream(stream))
     _check(st, "lora_linear_fwd")
 
 
@@ -142,7 +161,7 @@ def lora_linear_bwd(dY, x, W, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None)
     _f32(dA, "dA", (r, d_in))
     _f32(dB, "dB", (d_out, r))
     st = load_library().lora_linear_bwd(_ptr(dY), _ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(xa_save), _ptr(dX),
-                                        _ptr(dA), _ptr(dB), M, d_in, d_out, r, float(alpha), _ptr(ws), ws.numel(),
+                                        _ptr(dA), _ptr(dB), M, d_in, d_out, r, float(alpha), *_ws(ws),
                                         _stream(stream))
     _check(st, "lora_linear_bwd")
 
@@ -150,6 +169,7 @@ def lora_linear_bwd(dY, x, W, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None)
 def _q4(Wq, Wscale, d_out, d_in):
     if Wq.dtype != torch.uint8 or not Wq.is_cuda or not Wq.is_contiguous() or tuple(Wq.shape) != (d_out, d_in // 2):
         raise ValueError(f"Wq: expected a contiguous CUDA uint8 tensor of shape {(d_out, d_in // 2)}")
+    _on_current_device(Wq, "Wq")
     _bf16(Wscale, "Wscale", (d_out, d_in // 64))
 
 
@@ -163,7 +183,7 @@ def lora_linear_fwd_q4(x, Wq, Wscale, A, B, h, xa_save, alpha, ws, stream=None):
     if xa_save is not None:
         _bf16(xa_save, "xa_save", (M, r))
     st = load_library().lora_linear_fwd_q4(_ptr(x), _ptr(Wq), _ptr(Wscale), _ptr(A), _ptr(B), _ptr(h),
-                                           _ptr(xa_save), M, d_in, d_out, r, float(alpha), _ptr(ws), ws.numel(),
+                                           _ptr(xa_save), M, d_in, d_out, r, float(alpha), *_ws(ws),
                                            _stream(stream))
     _check(st, "lora_linear_fwd_q4")
 
@@ -183,12 +203,13 @@ def lora_linear_bwd_q4(dY, x, Wq, Wscale, A, B, xa_save, dX, dA, dB, alpha, ws, 
     _f32(dB, "dB", (d_out, r))
     st = load_library().lora_linear_bwd_q4(_ptr(dY), _ptr(x), _ptr(Wq), _ptr(Wscale), _ptr(A), _ptr(B),
                                            _ptr(xa_save), _ptr(dX), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
-                                           float(alpha), _ptr(ws), ws.numel(), _stream(stream))
+                                           float(alpha), *_ws(ws), _stream(stream))
     _check(st, "lora_linear_bwd_q4")
 
 
 def lora_linear_check(ws, stream=None):
-    _check(load_library().lora_linear_check(_ptr(ws), _stream(stream)), "lora_linear_check")
+    ptr = None if ws is None else _ws(ws)[0]  # no workspace: only wait for the stream
+    _check(load_library().lora_linear_check(ptr, _stream(stream)), "lora_linear_check")
 
 
 def lora_linear_merge(W, A, B, W_out, alpha, stream=None):
@@ -234,7 +255,7 @@ def lora_linear_selftest_timeout(ws, limit_us: int = 1000, stream=None):
     fn = lib.lora_linear_selftest_timeout
     fn.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_void_p]
     fn.restype = ctypes.c_int
-    _check(fn(_ptr(ws), ws.numel() * ws.element_size(), int(limit_us), _stream(stream)),
+    _check(fn(*_ws(ws), int(limit_us), _stream(stream)),
            "lora_linear_selftest_timeout")
 
 
