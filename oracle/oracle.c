@@ -5,9 +5,9 @@
  * this file; it is used by the tests, by the package's smoke check and by the
  * benchmark's CPU-baseline leg.  It shares no code with the CUDA library.
  *
- * Every input arrives exactly as the GPU receives it (bf16 bit patterns, or the
- * 4-bit blockwise code plus bf16 scales for a frozen weight) and is widened to
- * fp64 without rounding.  Every sum runs in fp64, in increasing index order, with
+ * Every input arrives exactly as the GPU receives it (bf16 bit patterns; for a frozen
+ * weight also the 4-bit blockwise code plus bf16 scales, or 8-bit e4m3 codes plus a
+ * bf16 scale per row) and is widened to fp64 without rounding.  Every sum runs in fp64, in increasing index order, with
  * no blocking or reordering beyond what the definition states.
  *
  * Notation (row-major, tokens are rows):
@@ -58,12 +58,29 @@ void oracle_set_threads(int n) {
 }
 
 /*
+ * FP8 E4M3 value of an 8-bit code, as the OCP 8-bit floating point specification
+ * defines the format: sign bit, 4 exponent bits with bias 7, 3 mantissa bits; exponent
+ * field 0 is subnormal, m/8 * 2^-6; otherwise (1 + m/8) * 2^(e - 7); no infinities,
+ * and S.1111.111 is NaN (so the largest value is 1.75 * 2^8 = 448).
+ */
+static double e4m3_to_f64(uint8_t c) {
+    const int e = (c >> 3) & 0xF, m = c & 0x7;
+    const double sign = (c & 0x80) ? -1.0 : 1.0;
+    if (e == 0xF && m == 0x7) return NAN;
+    if (e == 0) return sign * ldexp((double)m, -9);
+    return sign * ldexp(1.0 + m / 8.0, e - 7);
+}
+
+/*
  * Frozen weight W[n, k] as fp64.  wfmt 0: bf16 [d_out, d_in].  wfmt 1: 4-bit code,
  * w'[n, k] = (q[n, k] - 8) * scale[n, k / 64] / 7 with the stored bf16 scale; two
  * codes per byte along d_in, low nibble = even k (page "Unsloth — 微调 2-5x 加速",
  * section 核心要点: 4-bit weights dequantised inside the matmul; page
  * "ms-swift框架下UnSloth与Liger-Kernel优化实战", section UnSloth：让LoRA真正“低秩”起来:
- * int4 storage restored on the fly).
+ * int4 storage restored on the fly).  wfmt 2: 8-bit FP8 E4M3 codes [d_out, d_in], one
+ * per byte, with a bf16 scale per row: w'[n, k] = e4m3(q[n, k]) * scale[n] (page
+ * "ms-swift高效微调组合：LoRA+UnSloth提速实践", section 3.2: weights stored in FP8,
+ * computed in BF16).
  */
 typedef struct {
     int wfmt;
@@ -77,6 +94,12 @@ static void w_row(const wsrc_t *W, int64_t n, double *row) {
     if (W->wfmt == 0) {
         const uint16_t *p = W->w + n * W->d_in;
         for (int64_t k = 0; k < W->d_in; ++k) row[k] = bf16_to_f64(p[k]);
+        return;
+    }
+    if (W->wfmt == 2) {
+        const uint8_t *p = W->q + n * W->d_in;
+        const double sc = bf16_to_f64(W->scale[n]);
+        for (int64_t k = 0; k < W->d_in; ++k) row[k] = e4m3_to_f64(p[k]) * sc;
         return;
     }
     const uint8_t *p = W->q + n * (W->d_in / 2);

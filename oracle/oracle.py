@@ -1,9 +1,11 @@
 """ctypes front of oracle.c (fp64 CPU reference; test infrastructure only).
 
-Inputs are numpy arrays of bf16 bit patterns (uint16), or the 4-bit code (uint8,
-two codes per byte along d_in, low nibble = even index) with bf16 scales per
-64-element block.  Results are fp64 numpy arrays.  Each function is one step of the
-layer's definition (see oracle.c for the formulas and the passages they follow).
+Inputs are numpy arrays of bf16 bit patterns (uint16).  A frozen weight is W (bf16),
+or the 4-bit code Wq (uint8, two codes per byte along d_in, low nibble = even index)
+with bf16 scales Wscale per 64-element block, or FP8 E4M3 codes W8 (uint8, one per
+element) with a bf16 scale W8scale per row.  Results are fp64 numpy arrays.  Each
+function is one step of the layer's definition (see oracle.c for the formulas and the
+passages they follow).
 """
 from __future__ import annotations
 
@@ -69,14 +71,16 @@ def set_threads(n: int) -> None:
     _load().oracle_set_threads(int(n))
 
 
-def _wargs(W=None, Wq=None, Wscale=None):
+def _wargs(W=None, Wq=None, Wscale=None, W8=None, W8scale=None):
     if W is not None:
         return 0, _u16(W), None, None
+    if W8 is not None:
+        return 2, None, np.ascontiguousarray(W8, dtype=np.uint8), _u16(W8scale)
     return 1, None, np.ascontiguousarray(Wq, dtype=np.uint8), _u16(Wscale)
 
 
-def weight(d_out, d_in, W=None, Wq=None, Wscale=None) -> np.ndarray:
-    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+def weight(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None) -> np.ndarray:
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
     out = np.empty((d_out, d_in), dtype=np.float64)
     _load().oracle_weight(fmt, _p(w), _p(q), _p(sc), d_out, d_in, _p(out))
     return out
@@ -92,13 +96,13 @@ def xa(x, A) -> np.ndarray:
     return out
 
 
-def h(x, B, xa_, s, *, W=None, Wq=None, Wscale=None, rows=None) -> np.ndarray:
+def h(x, B, xa_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None) -> np.ndarray:
     """Step 2: h = x . W^T + s * xa . B^T for all rows, or only ``rows``."""
     x, B = _u16(x), _u16(B)
     M, d_in = x.shape
     d_out, r = B.shape
     xa_ = np.ascontiguousarray(xa_, dtype=np.float64)
-    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
     rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = M if rr is None else len(rr)
     out = np.empty((n, d_out), dtype=np.float64)
@@ -117,13 +121,13 @@ def g(dY, B) -> np.ndarray:
     return out
 
 
-def dx(dY, A, g_, s, *, W=None, Wq=None, Wscale=None, rows=None) -> np.ndarray:
+def dx(dY, A, g_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None) -> np.ndarray:
     """Step 4: dX = dY . W + s * g . A for all rows, or only ``rows``."""
     dY, A = _u16(dY), _u16(A)
     M, d_out = dY.shape
     r, d_in = A.shape
     g_ = np.ascontiguousarray(g_, dtype=np.float64)
-    fmt, w, q, sc = _wargs(W, Wq, Wscale)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
     rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = M if rr is None else len(rr)
     out = np.empty((n, d_in), dtype=np.float64)
@@ -154,19 +158,19 @@ def da(x, g_, s) -> np.ndarray:
     return out
 
 
-def forward(x, A, B, s, *, W=None, Wq=None, Wscale=None, rows=None):
+def forward(x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None):
     """Steps 1-2.  Returns (h, xa)."""
     xa_ = xa(x, A)
-    return h(x, B, xa_, s, W=W, Wq=Wq, Wscale=Wscale, rows=rows), xa_
+    return h(x, B, xa_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, rows=rows), xa_
 
 
-def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, rows=None, xa_=None):
+def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None, xa_=None):
     """Steps 1, 3-6.  Returns dict with dX (all rows or ``rows``), dA, dB, g, xa."""
     if xa_ is None:
         xa_ = xa(x, A)
     g_ = g(dY, B)
     return {
-        "dX": dx(dY, A, g_, s, W=W, Wq=Wq, Wscale=Wscale, rows=rows),
+        "dX": dx(dY, A, g_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, rows=rows),
         "dA": da(x, g_, s),
         "dB": db(dY, xa_, s),
         "g": g_,
@@ -186,17 +190,20 @@ def _f64(bits) -> np.ndarray:
     return (_u16(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, rows=2048):
+def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=2048):
     """(n0, fp64 rows n0 .. n0+k) of the dequantised weight, block by block."""
     for n0 in range(0, d_out, rows):
         n1 = min(d_out, n0 + rows)
         if W is not None:
             yield n0, weight(n1 - n0, d_in, W=_u16(W)[n0:n1])
+        elif W8 is not None:
+            yield n0, weight(n1 - n0, d_in, W8=np.ascontiguousarray(W8)[n0:n1], W8scale=_u16(W8scale)[n0:n1])
         else:
             yield n0, weight(n1 - n0, d_in, Wq=np.ascontiguousarray(Wq)[n0:n1], Wscale=_u16(Wscale)[n0:n1])
 
 
-def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, xa_=None, block_rows=2048):
+def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, xa_=None,
+                  block_rows=2048):
     """Step 2 projected: (h . v [M], u^T . h [d_out]) for v [d_out], u [M], with
     h . v = x . (W^T v) + s * xa . (B^T v) and u^T . h = W (x^T u) + s * B (xa^T u)."""
     M, d_in = np.shape(x)
@@ -206,7 +213,7 @@ def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, xa_=None, b
     wt_v = np.zeros(d_in)
     xt_u = xf.T @ u
     col = np.empty(d_out)
-    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, rows=block_rows):
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows):
         wt_v += Wb.T @ v[n0:n0 + len(Wb)]
         col[n0:n0 + len(Wb)] = Wb @ xt_u
     row = xf @ wt_v + s * (xa_ @ (Bf.T @ v))
@@ -214,7 +221,8 @@ def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, xa_=None, b
     return row, col
 
 
-def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, g_=None, block_rows=2048):
+def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, g_=None,
+                   block_rows=2048):
     """Step 4 projected: (dX . v [M], u^T . dX [d_in]) for v [d_in], u [M], with
     dX . v = dY . (W v) + s * g . (A v) and u^T . dX = (dY^T u)^T W + s * (g^T u)^T A."""
     M, d_out = np.shape(dY)
@@ -224,7 +232,7 @@ def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, g_=None, 
     w_v = np.empty(d_out)
     dyt_u = dYf.T @ u
     col = np.zeros(d_in)
-    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, rows=block_rows):
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows):
         w_v[n0:n0 + len(Wb)] = Wb @ v
         col += dyt_u[n0:n0 + len(Wb)] @ Wb
     row = dYf @ w_v + s * (g_ @ (Af @ v))
@@ -232,9 +240,9 @@ def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, g_=None, 
     return row, col
 
 
-def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None) -> np.ndarray:
+def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None) -> np.ndarray:
     """The merged weight of step 2, W + s * B . A, in fp64 [d_out, d_in]: the weight for
     which h = x . (W + s B A)^T (the adapter folded in for deployment).  The 4-bit weight
     is decoded by the same rule as steps 2 and 4."""
     d_out, d_in = np.shape(B)[0], np.shape(A)[1]
-    return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale) + s * (_f64(B) @ _f64(A))
+    return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale) + s * (_f64(B) @ _f64(A))

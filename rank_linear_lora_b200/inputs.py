@@ -156,6 +156,67 @@ def unpack_q4_codes(packed: np.ndarray) -> np.ndarray:
     return q
 
 
+E4M3_MAX = 448.0
+
+
+def e4m3_encode(v: np.ndarray) -> np.ndarray:
+    """FP8 E4M3 codes (OCP 8-bit floating point specification: sign, 4 exponent bits
+    with bias 7, 3 mantissa bits, no infinities) of finite values |v| <= 448, rounded
+    to the nearest representable value, ties to even.
+
+    In the binade [2^e, 2^(e+1)), e = -6 .. 8, representable values are 2^(e-3) apart;
+    below 2^-6 (the subnormals) they are 2^-9 apart, the spacing of the lowest binade.
+    So a value is k * 2^(e-3) for an integer k, with k in 8..15 for a normal value
+    (exponent field e + 7, mantissa k - 8) and k in 0..7 for a subnormal one
+    (exponent field 0, mantissa k).  The sign of -0.0 is kept.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    if not np.all(a <= E4M3_MAX):
+        raise ValueError("e4m3_encode: values must be finite with |v| <= 448")
+    _, E = np.frexp(a)                      # a = f * 2^E, f in [0.5, 1)
+    e = np.clip(E - 1, -6, 8)               # binade exponent; subnormals share -6
+    k = np.rint(np.ldexp(a, 3 - e))         # spacing multiples, ties to even (exact scaling)
+    carry = k >= 16                         # rounded up into the next binade
+    e = np.where(carry, e + 1, e)
+    k = np.where(carry, 8, k).astype(np.int64)
+    normal = k >= 8
+    code = np.where(normal, ((e + 7) << 3) | (k - 8), k)
+    return (code | (np.signbit(v).astype(np.int64) << 7)).astype(np.uint8)
+
+
+def quantise_fp8(w32: np.ndarray):
+    """FP8 E4M3 code of a frozen weight [d_out, d_in] (fp32 draws), one scale per row.
+
+    absmax = max |w| over the row (fp32); the stored scale is bf16(absmax / 448)
+    (fp32 quotient, then nearest-even); each code is e4m3_encode of w / scale (the
+    stored scale, quotient in fp64), clamped to +-448 since the rounded scale may sit
+    just below absmax / 448.  A row with absmax 0 gets scale 0 and codes 0.  Returns
+    (codes uint8 [d_out, d_in], scale bf16 bits [d_out]).
+    """
+    d_out, d_in = w32.shape
+    out_q = np.empty((d_out, d_in), dtype=np.uint8)
+    out_s = np.empty(d_out, dtype=np.uint16)
+    rows = max(1, (1 << 22) // d_in)
+
+    def work(r0):
+        r1 = min(d_out, r0 + rows)
+        wb = w32[r0:r1]
+        amax = np.abs(wb).max(axis=1).astype(np.float32)
+        sbits = f32_to_bf16_bits((amax / np.float32(E4M3_MAX)).astype(np.float32))
+        sc = bf16_bits_to_f32(sbits).astype(np.float64)
+        safe = np.where(sc > 0, sc, 1.0)
+        t = np.clip(wb.astype(np.float64) / safe[:, None], -E4M3_MAX, E4M3_MAX)
+        q = e4m3_encode(t)
+        q[sc == 0] = 0
+        out_q[r0:r1] = q
+        out_s[r0:r1] = sbits
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, range(0, d_out, rows)))
+    return out_q, out_s
+
+
 @dataclass
 class LayerSpec:
     """One LoRA linear: M tokens, d_in -> d_out, rank r, scale alpha/r.
@@ -175,6 +236,7 @@ class LayerSpec:
     seed: int = 0
     layer: int = 0
     proj: int = 1
+    fp8: bool = False
 
     @property
     def s(self) -> float:
@@ -242,6 +304,8 @@ class LayerInputs:
     W: np.ndarray | None     # bf16 bits [d_out, d_in] (None for q4)
     Wq: np.ndarray | None    # uint8 [d_out, d_in/2] (q4 only)
     Wscale: np.ndarray | None  # bf16 bits [d_out, d_in/64] (q4 only)
+    W8: np.ndarray | None = None       # uint8 E4M3 codes [d_out, d_in] (fp8 only)
+    W8scale: np.ndarray | None = None  # bf16 bits [d_out] (fp8 only)
 
 
 def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) -> LayerInputs:
@@ -265,4 +329,7 @@ def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) 
     if spec.q4:
         Wq, Ws = quantise_q4(w32)
         return LayerInputs(spec, x, A, B, dY, None, Wq, Ws)
+    if spec.fp8:
+        W8, W8s = quantise_fp8(w32)
+        return LayerInputs(spec, x, A, B, dY, None, None, None, W8, W8s)
     return LayerInputs(spec, x, A, B, dY, f32_to_bf16_bits(w32), None, None)

@@ -93,7 +93,12 @@ def shared_input_projections(M, d_in, d_outs, r, alpha, q4, seed) -> list:
 
 def oracle_ref(inp: inputs.LayerInputs, rows=None) -> dict:
     sp = inp.spec
-    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W=inp.W)
+    if sp.q4:
+        wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale)
+    elif sp.fp8:
+        wkw = dict(W8=inp.W8, W8scale=inp.W8scale)
+    else:
+        wkw = dict(W=inp.W)
     h, xa = oracle.forward(inp.x, inp.A, inp.B, sp.s, rows=rows, **wkw)
     bw = oracle.backward(inp.dY, inp.x, inp.A, inp.B, sp.s, rows=rows, xa_=xa, **wkw)
     return {"h": h, "xa": xa, "dX": bw["dX"], "dA": bw["dA"], "dB": bw["dB"], "g": bw["g"]}

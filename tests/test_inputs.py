@@ -2,6 +2,7 @@
 import math
 
 import numpy as np
+import pytest
 
 from rank_linear_lora_b200 import inputs
 
@@ -52,3 +53,26 @@ def test_distributions():
     u = inputs.draw("uniform", 99, 2, n, 0.25)
     assert u.min() > -0.25 and u.max() < 0.25
     assert abs(u.std() - 0.25 / math.sqrt(3)) < 1e-3
+
+
+def test_e4m3_encoder_matches_library_cast():
+    """The FP8 E4M3 encoder rounds like torch's float32 -> float8_e4m3fn cast (nearest,
+    ties to even, subnormals included) over every binade and both signs."""
+    import torch
+    rng = np.random.default_rng(11)
+    mag = rng.choice([1e-4, 3e-3, 0.05, 1.0, 20.0, 200.0], size=100_000)
+    v = np.clip(rng.standard_normal(100_000) * mag, -448, 448).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(inputs.e4m3_encode(v), ref)
+
+
+def test_e4m3_encoder_exact_values_and_ties():
+    """Every representable value encodes to its own code; midpoints go to the even
+    mantissa (1.0625 -> 1.0, 1.1875 -> 1.25); the top value is 448."""
+    import torch
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(inputs.e4m3_encode(vals), codes)
+    assert list(inputs.e4m3_encode(np.array([1.0625, 1.1875, -1.0625, 448.0]))) == [0x38, 0x3A, 0xB8, 0x7E]
+    with pytest.raises(ValueError):
+        inputs.e4m3_encode(np.array([449.0]))

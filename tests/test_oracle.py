@@ -234,6 +234,96 @@ def test_q4_forward_reads_dequantised_columns():
     np.testing.assert_array_equal(h.T, (codes - 8.0) * scale / 7.0)
 
 
+def _e4m3_library_values() -> np.ndarray:
+    """All 256 FP8 E4M3 codes decoded by torch's float8_e4m3fn (a library routine)."""
+    import torch
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_fp8_decode_matches_library_for_every_code():
+    """The oracle's E4M3 decode of all 256 codes (scale 1) equals the library's, NaN
+    codes and the sign of zero included."""
+    codes = np.arange(256, dtype=np.uint8).reshape(1, 256)
+    got = oracle.weight(1, 256, W8=codes, W8scale=bf([1.0]))[0]
+    ref = _e4m3_library_values()
+    np.testing.assert_array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+    np.testing.assert_array_equal(np.signbit(got[ok]), np.signbit(ref[ok]))
+
+
+def test_fp8_hand_values():
+    """Codes decoded by hand from the E4M3 layout (sign | 4-bit exponent, bias 7 |
+    3-bit mantissa): 0x01 is the smallest subnormal 2^-9, 0x08 the smallest normal
+    2^-6, 0x38 = 0.0111.000 is 1, 0x3C = 1 + 4/8, 0x7E = 0.1111.110 is 1.75 * 2^8 = 448
+    (0x7F is NaN, not a number above it); the row scale multiplies every code."""
+    table = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x30: 0.5, 0x38: 1.0,
+             0x3C: 1.5, 0x7E: 448.0, 0xFE: -448.0, 0xB8: -1.0}
+    codes = np.array([list(table)], dtype=np.uint8)
+    got = oracle.weight(1, len(table), W8=codes, W8scale=bf([1.0]))[0]
+    np.testing.assert_array_equal(got, list(table.values()))
+    got = oracle.weight(2, len(table), W8=np.repeat(codes, 2, axis=0), W8scale=bf([0.375, -2.0]))
+    np.testing.assert_array_equal(got, np.outer([0.375, -2.0], list(table.values())))
+    assert np.isnan(oracle.weight(1, 2, W8=np.array([[0x7F, 0xFF]], np.uint8), W8scale=bf([1.0]))).all()
+
+
+def test_fp8_quantiser_pins():
+    """Row absmax 28 gives the bf16-exact scale 28/448 = 1/16, so w/scale is exact:
+    [28, -28, 14, 0] code to [0x7E, 0xFE, 0x76, 0x00] and decode back exactly; the
+    midpoints 1.0625/16 and 1.1875/16 round to the even mantissa (1/16, 1.25/16); a zero
+    row gets scale 0.  A row whose rounded scale sits below absmax/448 saturates at 448."""
+    w = np.zeros((3, 8), dtype=np.float32)
+    w[0, :6] = [28.0, -28.0, 14.0, 0.0, 1.0625 / 16, 1.1875 / 16]
+    w[2, :2] = [3.0, -3.0]  # bf16(3/448) < 3/448: w / scale > 448, clamped
+    q, sc = inputs.quantise_fp8(w)
+    assert list(q[0, :6]) == [0x7E, 0xFE, 0x76, 0x00, 0x38, 0x3A]
+    assert inputs.bf16_bits_to_f32(sc)[0] == np.float32(1 / 16)
+    assert sc[1] == 0 and not q[1].any()
+    assert list(q[2, :2]) == [0x7E, 0xFE]
+    wd = oracle.weight(3, 8, W8=q, W8scale=sc)
+    np.testing.assert_array_equal(wd[0, :6], [28.0, -28.0, 14.0, 0.0, 1 / 16, 1.25 / 16])
+    assert abs(wd[2, 0] - 3.0) <= 3.0 * 2.0 ** -8  # within the bf16 rounding of the scale
+
+
+def test_fp8_forward_reads_decoded_columns():
+    """With B = 0 and x = e_k, row h[k] of the fp8 oracle is column k of the decoded
+    weight, decoded here through the library table times each row's scale."""
+    d_in, d_out, r = 64, 5, 2
+    rng = np.random.default_rng(16)
+    q = rng.integers(0, 256, size=(d_out, d_in), dtype=np.uint8)
+    q[(q & 0x7F) == 0x7F] = 0x3F  # no NaN codes
+    sc = inputs.to_bf16_bits(rng.uniform(0.01, 1.0, size=d_out))
+    x = inputs.to_bf16_bits(np.eye(d_in))
+    A = np.zeros((r, d_in), dtype=np.uint16)
+    B = np.zeros((d_out, r), dtype=np.uint16)
+    h, _ = oracle.forward(x, A, B, 1.0, W8=q, W8scale=sc)
+    want = _e4m3_library_values()[q] * inputs.bf16_bits_to_f32(sc).astype(np.float64)[:, None]
+    np.testing.assert_array_equal(h.T, want)
+
+
+def test_fp8_matches_library_matmul():
+    """Every output with an FP8 weight against numpy fp64 matmuls of the same definition,
+    the weight decoded through the library table."""
+    M, d_in, d_out, r = 19, 96, 40, 8
+    rng = np.random.default_rng(17)
+    w32 = (rng.standard_normal((d_out, d_in)) / np.sqrt(d_in)).astype(np.float32)
+    q, sc = inputs.quantise_fp8(w32)
+    x, A, B, dY = (_rand_bits(rng, s_, c) for s_, c in
+                   [((M, d_in), 1), ((r, d_in), d_in ** -0.5), ((d_out, r), 0.02), ((M, d_out), 1)])
+    s = 2.0
+    h, xa = oracle.forward(x, A, B, s, W8=q, W8scale=sc)
+    bw = oracle.backward(dY, x, A, B, s, W8=q, W8scale=sc)
+    Wd = _e4m3_library_values()[q] * inputs.bf16_bits_to_f32(sc).astype(np.float64)[:, None]
+    X, Ad, Bd, dYd = map(f64, (x, A, B, dY))
+    ref = {"h": X @ Wd.T + s * (X @ Ad.T) @ Bd.T, "dX": dYd @ Wd + s * (dYd @ Bd) @ Ad,
+           "dA": s * (dYd @ Bd).T @ X, "dB": s * dYd.T @ (X @ Ad.T)}
+    got = {"h": h, "dX": bw["dX"], "dA": bw["dA"], "dB": bw["dB"]}
+    for key, want in ref.items():
+        np.testing.assert_allclose(got[key], want, rtol=0, atol=1e-12 * np.abs(want).max(), err_msg=key)
+    # the quantised weight is close to the draws it codes (3 mantissa bits: 2^-4 relative)
+    np.testing.assert_allclose(Wd, w32, rtol=0, atol=2.0 ** -4 * np.abs(w32).max())
+
+
 def test_row_selection_matches_full():
     """The sampled-row mode used at full sizes returns exactly the full rows."""
     rng = np.random.default_rng(7)
