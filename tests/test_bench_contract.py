@@ -24,3 +24,20 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("tiny")
+
+
+def test_stacked_layer_counts_the_work_of_its_projections():
+    """The gate+up layer stacked on one x is measured by the work of the two
+    projections: FLOPs are twice gate's, and the bytes are gate's twice less one read
+    of the shared x (forward and backward) and with one dX written instead of two; the
+    zero blocks of the stacked B and dB count nothing."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from rank_linear_lora_b200 import inputs
+
+    gate, stacked = inputs.workload(2).layers[0], inputs.workload(2).layers[3]
+    assert stacked.flops == 2 * gate.flops
+    M, di = gate.M, gate.d_in
+    x_bytes = M * di * 2
+    # forward reads x once; backward reads x once and writes one dX
+    assert bench.algorithmic_bytes(stacked) == 2 * bench.algorithmic_bytes(gate) - 3 * x_bytes
