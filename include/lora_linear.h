@@ -175,9 +175,9 @@ LORA_API lora_status_t lora_linear_fwd_noalloc(const uint16_t *x, const uint16_t
                                                void *stream);
 
 /* Waits for `stream`, then reads and clears the device error word kept in
- * `workspace`.  Returns LORA_OK, LORA_ERR_TIMEOUT (a bounded device wait ran out) or
- * LORA_ERR_CUDA (the stream reported an error).  Synchronising: for tests and
- * diagnostics, not for the hot path. */
+ * `workspace` (NULL: only waits).  Returns LORA_OK, LORA_ERR_TIMEOUT (a bounded device
+ * wait ran out) or LORA_ERR_CUDA (the stream reported an error).  Synchronising: for
+ * tests and diagnostics, not for the hot path. */
 LORA_API lora_status_t lora_linear_check(void *workspace, void *stream);
 
 /* Static description of a status code; never NULL. */
