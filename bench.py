@@ -12,9 +12,11 @@ launch stream (barrier + synchronize on both sides; max over ranks).  Steps rota
 over three independent input sets (3 x 160 MiB > the 126 MB L2), so no step finds
 its operands left in L2 by the previous one.
 
-Multi-GPU (torchrun): data parallel over tokens, weak scaling (each rank its own
-M tokens); after the backward the packed [dA | dB] fp32 gradient is summed over
-ranks with one NCCL all-reduce inside the timed region.
+Multi-GPU: data parallel over tokens, weak scaling (each rank its own M tokens);
+after the backward the packed [dA | dB] fp32 gradient is summed over ranks with one
+NCCL all-reduce inside the timed region.  `--gpus N` with N > 1 and no launcher
+around it starts N ranks itself (torch.distributed.run on this node, one per GPU);
+under an outside launcher (RANK / WORLD_SIZE set) it runs as one of its ranks.
 
 --impl reference times the fp64 CPU oracle on the host cores instead (a bounded
 token sample per step).
@@ -48,6 +50,12 @@ def parse():
     p.add_argument("--layer", type=int, default=0, help="layer of a multi-layer workload")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
+                   help="process-group backend of a multi-rank run (gloo only with --dry-run)")
+    p.add_argument("--dry-run", action="store_true",
+                   help="no GPU: each rank computes its token shard's dA, dB with the oracle on the host, sums "
+                        "them over ranks with one all-reduce of the packed buffer and prints the JSON line; "
+                        "checks the multi-rank launch and reduction plumbing on a CPU-only machine")
     p.add_argument("--shape", type=str, default=None,
                    help="M,d_in,d_out: resize the layer (same r, alpha, weight format), e.g. a case small "
                         "enough for a full profiler capture; the line then names the resized workload")
@@ -112,7 +120,7 @@ def stored_traffic(kind: str, workload: str):
 class ClockSampler:
     """NVML clocks and throttle reasons sampled in a thread while the timed region runs."""
 
-    def __init__(self, dev, period_s: float = 0.01):
+    def __init__(self, dev, period_s: float = 0.0005):
         self.period, self.samples, self._stop = period_s, [], threading.Event()
         self.ok = False
         try:
@@ -178,6 +186,102 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def config_dict(spec, workload_name: str, world: int) -> dict:
+    """The workload as both arms name it (identical keys and values)."""
+    return {"workload": workload_name, "M": spec.M, "d_in": spec.d_in, "d_out": spec.d_out, "r": spec.r,
+            "alpha": spec.alpha, "q4": spec.q4, "projections": spec.proj, "tokens_per_step": spec.M * world,
+            "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
+            "parallelism": f"dp{world}"}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as so:
+        so.bind(("127.0.0.1", 0))
+        return so.getsockname()[1]
+
+
+def launch_ranks(args) -> int:
+    """Run this script as `args.gpus` ranks on this node (torch.distributed.run), one per
+    GPU, rendezvous on 127.0.0.1; rank 0 prints the JSON line.  The launcher is bounded
+    by a timeout well above the process group's own, after which its process group is
+    killed."""
+    import signal
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr=127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__)] + sys.argv[1:]
+    proc = subprocess.Popen(cmd, start_new_session=True)
+    try:
+        return proc.wait(timeout=1800)
+    except subprocess.TimeoutExpired:
+        os.killpg(proc.pid, signal.SIGKILL)
+        proc.wait()
+        print(f"bench.py: the {args.gpus} ranks did not finish within 1800 s", file=sys.stderr)
+        return 1
+
+
+def run_dry(args, spec, workload_name, rank, world):
+    """CPU-only multi-rank run: the plumbing of the data-parallel step without a GPU."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import oracle
+    from rank_linear_lora_b200 import inputs
+    from rank_linear_lora_b200.dp import PackedGrads, token_shard
+
+    if world > 1:
+        dist.init_process_group(args.backend, timeout=timedelta(seconds=60))
+        assert dist.get_world_size() == world
+    tokens = min(spec.M, 64 * max(1, world))
+    small = spec.with_(M=tokens, d_in=min(spec.d_in, 256), d_out=min(spec.d_out, 256))
+    inp = inputs.make_inputs(small)
+    start, count = token_shard(small.M, world, rank)
+    grads = PackedGrads(small.r, small.d_in, small.d_out, device="cpu")
+    t0 = time.perf_counter()
+    if count > 0:
+        xa_ = oracle.xa(inp.x[start:start + count], inp.A)
+        g_ = oracle.g(inp.dY[start:start + count], inp.B)
+        grads.dA.copy_(torch.from_numpy(oracle.da(inp.x[start:start + count], g_, small.s)))
+        grads.dB.copy_(torch.from_numpy(oracle.db(inp.dY[start:start + count], xa_, small.s)))
+    else:
+        grads.zero_()
+    if world > 1:
+        grads.all_reduce()
+    dt = time.perf_counter() - t0
+    ok = None
+    if rank == 0:
+        xa_ = oracle.xa(inp.x, inp.A)
+        g_ = oracle.g(inp.dY, inp.B)
+        full_dA, full_dB = oracle.da(inp.x, g_, small.s), oracle.db(inp.dY, xa_, small.s)
+        ok = bool(np.allclose(grads.dA.double().numpy(), full_dA, rtol=0, atol=1e-5 * np.abs(full_dA).max())
+                  and np.allclose(grads.dB.double().numpy(), full_dB, rtol=0, atol=1e-5 * np.abs(full_dB).max()))
+        out = {"metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world, "world_size": world,
+               "steps": 1, "warmup": 0, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+               "vs_baseline": None, "dtype": "f64", "data": "synthetic", "dry_run": True,
+               "backend": args.backend if world > 1 else None,
+               "config": config_dict(small, workload_name + f" (dry run: M{small.M} {small.d_in}->{small.d_out})",
+                                     world),
+               "reduced_grads_match_whole_batch": ok}
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0 if ok in (None, True) else 1
+
+
 # ---------------------------------------------------------------------- reference arm
 def run_reference(args, spec, workload_name, rank, world):
     import numpy as np
@@ -208,12 +312,10 @@ def run_reference(args, spec, workload_name, rank, world):
         "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_name, "M": spec.M, "d_in": spec.d_in,
-                                         "d_out": spec.d_out, "r": spec.r, "alpha": spec.alpha,
-                                         "projections": spec.proj,
-                                         "parallelism": "host cores (OpenMP)"},
+        "data": "synthetic", "config": config_dict(spec, workload_name, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model(),
+                         "where": "host cores of rank 0 (OpenMP), the other ranks idle"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "tokens_per_s": args.steps * tokens / dt,
     }
@@ -243,16 +345,45 @@ def cpu_baseline(spec, seconds=12.0):
     _oracle_step(oracle, inp, spec, 0, tokens)
     dt = time.perf_counter() - t0
     return {"value": tokens * per_token / dt / 1e12, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "cpu_model": cpu_model(),
             "sample": f"fwd+bwd of {tokens} of the {spec.M} tokens (full d_in={spec.d_in}, d_out={spec.d_out}, "
-                      f"r={spec.r}) in fp64, {dt:.1f} s"}
+                      f"r={spec.r}) in fp64, {dt:.1f} s",
+            "single_thread_tiny": single_thread_tiny()}
+
+
+def single_thread_tiny():
+    """The oracle on one host thread, whole tiny workload (M=64, 256x256, r=8)."""
+    import oracle
+    from rank_linear_lora_b200 import inputs
+
+    spec = inputs.workload(0).layers[0]
+    inp = inputs.make_inputs(spec)
+    n0 = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        _oracle_step(oracle, inp, spec, 0, spec.M)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 3 or time.perf_counter() - t0 < 0.5:
+            _oracle_step(oracle, inp, spec, 0, spec.M)
+            reps += 1
+        dt = (time.perf_counter() - t0) / reps
+    finally:
+        oracle.set_threads(n0)
+    return {"workload": "tiny M64 256x256 r8, whole", "threads": 1, "s_per_step": dt,
+            "gflops": spec.flops / dt / 1e9}
 
 
 # ---------------------------------------------------------------------- our arm
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_ranks(args)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and not (args.gpus == 1 and world > 1):
+        print(f"bench.py: --gpus {args.gpus} but the launcher started {world} ranks", file=sys.stderr)
+        return 2
 
     from rank_linear_lora_b200 import inputs
 
@@ -264,6 +395,8 @@ def main():
         spec = spec.with_(M=M_, d_in=di_, d_out=do_)
         workload_name += f" resized to M{M_} {di_}->{do_}"
 
+    if args.dry_run:
+        return run_dry(args, spec, workload_name, rank, world)
     if args.impl == "reference":
         out = run_reference(args, spec, workload_name, rank, world)
         if out is not None:
@@ -282,6 +415,7 @@ def main():
     if world > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        assert dist.get_world_size() == world
 
     peaks = load_peaks()
     M, di, do, r, alpha = spec.M, spec.d_in, spec.d_out, spec.r, spec.alpha
@@ -594,10 +728,8 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_name, "M": M, "d_in": di, "d_out": do, "r": r, "alpha": alpha,
-                       "q4": spec.q4, "projections": spec.proj, "tokens_per_step": M * world,
-                       "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
-                       "parallelism": f"dp{world}"},
+            "config": config_dict(spec, workload_name, world),
+            "world_size": dist.get_world_size() if world > 1 else 1,
             "tokens_per_s": tokens_per_s,
             "roofline": roofline,
             "roofline_step": step_roof,

@@ -155,17 +155,25 @@ LORA_API lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x,
  * only the op's tensors, or a service that fixes its device-memory budget at start-up
  * and forbids allocation afterwards (cudaMalloc may synchronise the device and
  * fragments the heap).  The pages have no counterpart; this is an interface
- * convenience.  Same arguments and results as lora_linear_fwd, minus the workspace.
+ * convenience.  Same arguments and results as lora_linear_fwd, minus the workspace;
+ * it runs the same kernels, so h and xa_save are bit for bit those of
+ * lora_linear_fwd.
  *   - Scratch: a fixed 4 MiB array in device memory, held by every GPU that loads this
  *     library until the process exits.  Problems whose forward workspace
  *     (lora_linear_workspace_size(LORA_OP_FWD, ...)) exceeds 4 MiB are rejected with
  *     LORA_ERR_WORKSPACE before anything is enqueued (every r <= 16 workload of
  *     M <= 8192 fits; rank 128 at M = 16384 does not).
  *   - Allocates nothing: no cudaMalloc/cudaFree; it enqueues a memset that clears the
- *     part of the scratch the call uses, then the forward kernels.
- *   - The first call on a device, with that device current, looks up the scratch's
- *     device address (cudaGetSymbolAddress); make that first call before any stream
- *     capture.
+ *     part of the scratch the call uses (all but the error word), then the forward
+ *     kernels.
+ *   - The first call in a CUDA context (with that context current; the runtime's
+ *     primary context of the current device when none is) looks up the scratch's
+ *     device address in it (cudaGetSymbolAddress) and enqueues a clear of its error
+ *     word; make that first call before any stream capture.  Each context has its own
+ *     copy of the scratch.
+ *   - Errors: a bounded device wait that runs out records its code in the scratch's
+ *     error word, which later calls leave in place; lora_linear_noalloc_check reports
+ *     it (LORA_ERR_TIMEOUT) and clears it.  lora_linear_check cannot see it.
  *   - All calls share the one scratch: calls that can overlap on the GPU (different
  *     streams, or host threads without ordering) race and give wrong results.
  */
@@ -173,6 +181,19 @@ LORA_API lora_status_t lora_linear_fwd_noalloc(const uint16_t *x, const uint16_t
                                                const uint16_t *B, uint16_t *h, uint16_t *xa_save,
                                                int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                                                void *stream);
+
+/* Companion of lora_linear_fwd_noalloc (no counterpart in the pages): waits for
+ * `stream`, then reads and clears the error word of the workspace-free forward's
+ * scratch in the current context.  LORA_OK, LORA_ERR_TIMEOUT (a bounded device wait of
+ * an earlier call ran out; that call's h is undefined) or LORA_ERR_CUDA.
+ * Synchronising: for tests and diagnostics, not for the hot path. */
+LORA_API lora_status_t lora_linear_noalloc_check(void *stream);
+
+/* Failure-path self-test of the workspace-free forward (no counterpart in the pages):
+ * as lora_linear_selftest_timeout, on the error word of that forward's scratch in the
+ * current context, so that lora_linear_noalloc_check then reports LORA_ERR_TIMEOUT.
+ * limit_us in 1 .. 2000000. */
+LORA_API lora_status_t lora_linear_noalloc_selftest_timeout(uint32_t limit_us, void *stream);
 
 /* Waits for `stream`, then reads and clears the device error word kept in
  * `workspace` (NULL: only waits).  Returns LORA_OK, LORA_ERR_TIMEOUT (a bounded device

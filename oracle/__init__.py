@@ -20,4 +20,6 @@ from .oracle import (  # noqa: F401
     h_projections,
     dx_projections,
     merged_weight,
+    h_dense,
+    dx_dense,
 )

@@ -246,3 +246,25 @@ def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=Non
     is decoded by the same rule as steps 2 and 4."""
     d_out, d_in = np.shape(B)[0], np.shape(A)[1]
     return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale) + s * (_f64(B) @ _f64(A))
+
+
+# ------------------------------------------------------------------ whole tensors at full size
+# Steps 2 and 4 for a block of token rows, with numpy's fp64 matrix product (a library
+# primitive) as the summation step in place of oracle.c's loops.  The inputs are the
+# same exact fp64 widenings and the weight is dequantised by oracle.c's own rule
+# (weight()); only the order of the fp64 additions differs from oracle.c, which puts
+# the two within ~1e-13 of each other (pinned in the CPU tests).  This is what lets
+# the tests compare every element of h and dX of the full-size workloads (up to 2e12
+# multiply-adds per output) in seconds rather than the minutes oracle.c's plain loops
+# take on the host cores.
+
+def h_dense(x, B, xa_, s, Wf) -> np.ndarray:
+    """Step 2 for the given token rows: h = x . Wf^T + s * xa . B^T, with Wf the fp64
+    weight [d_out, d_in] from weight() and xa_ the fp64 step-1 rows of the same tokens."""
+    return _f64(x) @ np.asarray(Wf, dtype=np.float64).T + s * (np.asarray(xa_, dtype=np.float64) @ _f64(B).T)
+
+
+def dx_dense(dY, A, g_, s, Wf) -> np.ndarray:
+    """Step 4 for the given token rows: dX = dY . Wf + s * g . A, with Wf the fp64 weight
+    [d_out, d_in] from weight() and g_ the fp64 step-3 rows of the same tokens."""
+    return _f64(dY) @ np.asarray(Wf, dtype=np.float64) + s * (np.asarray(g_, dtype=np.float64) @ _f64(A))

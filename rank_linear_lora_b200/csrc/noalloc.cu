@@ -9,6 +9,12 @@
 // heap).  This file gives them lora_linear_fwd_noalloc, which takes the same inputs
 // and outputs but no workspace: its scratch is a fixed 4 MiB array in device global
 // memory that every GPU loading this library holds until the process exits.
+//
+// The scratch starts, like every workspace of this library, with the device error
+// word (bytes 0..255); the kernels' arrival counters and partial sums follow.  Each
+// call clears only what follows the error word, so a bounded wait that ran out in one
+// call stays recorded until lora_linear_noalloc_check reads and clears it.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -18,26 +24,64 @@
 namespace {
 
 constexpr size_t kNoallocScratchBytes = size_t(4) << 20;
+constexpr size_t kErrBytes = 256;  // the error word's slot at the start of every workspace
 
 // The scratch itself.  In host code this name is only a host-side stand-in for the
-// symbol; the device address comes from cudaGetSymbolAddress (once per device).
+// symbol; the device address comes from cudaGetSymbolAddress, once per context.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
-std::mutex g_noalloc_mu;
-void *g_noalloc_addr[64] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
 
-// Device address of the scratch on the current device, looked up on the first call
-// made with that device current.
-lora_status_t scratch_address(void **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+// The driver's cuCtxGetCurrent, looked up through the runtime (no link to libcuda).
+CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
         void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    return fn;
+}
+
+// Scratch addresses already looked up, keyed by CUDA context: the address of a
+// __device__ array belongs to the context the module was loaded in, so a caller that
+// switches between contexts of one device gets each context's own copy.
+struct Entry {
+    CUcontext ctx;
+    void *addr;
+};
+constexpr int kMaxEntries = 64;
+std::mutex g_noalloc_mu;
+Entry g_entries[kMaxEntries];
+int g_n_entries = 0;
+
+// Device address of the scratch in the current context, looked up (and its error word
+// cleared, on `stream`) on the first call made with that context current.
+lora_status_t scratch_address(cudaStream_t stream, void **out) {
+    CtxGetCurrentFn get = ctx_get_current();
+    if (!get) return LORA_ERR_CUDA;
+    CUcontext ctx = nullptr;
+    if (get(&ctx) != CUDA_SUCCESS) return LORA_ERR_CUDA;
+    void *p = nullptr;
+    if (!ctx) {
+        // No context current on this thread yet: the runtime call makes the current
+        // device's primary context current (and resolves the address in it).
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return LORA_ERR_CUDA;
-        g_noalloc_addr[dev] = p;
+        if (get(&ctx) != CUDA_SUCCESS || !ctx) return LORA_ERR_CUDA;
     }
-    *out = g_noalloc_addr[dev];
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    for (int i = 0; i < g_n_entries; ++i)
+        if (g_entries[i].ctx == ctx) {
+            *out = g_entries[i].addr;
+            return LORA_OK;
+        }
+    if (!p && (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)) return LORA_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, kErrBytes, stream) != cudaSuccess) return LORA_ERR_CUDA;
+    if (g_n_entries < kMaxEntries) g_entries[g_n_entries++] = {ctx, p};
+    *out = p;
     return LORA_OK;
 }
 
@@ -50,11 +94,28 @@ extern "C" LORA_API lora_status_t lora_linear_fwd_noalloc(const uint16_t *x, con
     const size_t need = lora_linear_workspace_size(LORA_OP_FWD, M, d_in, d_out, r);
     if (need == 0) return LORA_ERR_INVALID_ARG;
     if (need > kNoallocScratchBytes) return LORA_ERR_WORKSPACE;  // problem too large for the fixed scratch
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     void *scratch = nullptr;
-    lora_status_t st = scratch_address(&scratch);
-    if (st != LORA_OK) return st;
-    // The scratch keeps whatever the previous call left; the counters and the error
-    // word must start at zero, so clear the part this call uses.
-    if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess) return LORA_ERR_CUDA;
+    lora_status_t s = scratch_address(st, &scratch);
+    if (s != LORA_OK) return s;
+    // The scratch keeps whatever the previous call left; the arrival counters must start
+    // at zero, so clear the part this call uses, all but the error word.
+    if (need > kErrBytes &&
+        cudaMemsetAsync(static_cast<unsigned char *>(scratch) + kErrBytes, 0, need - kErrBytes, st) != cudaSuccess)
+        return LORA_ERR_CUDA;
     return lora_linear_fwd(x, W, A, B, h, xa_save, M, d_in, d_out, r, alpha, scratch, kNoallocScratchBytes, stream);
+}
+
+extern "C" LORA_API lora_status_t lora_linear_noalloc_check(void *stream) {
+    void *scratch = nullptr;
+    lora_status_t s = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
+    if (s != LORA_OK) return s;
+    return lora_linear_check(scratch, stream);
+}
+
+extern "C" LORA_API lora_status_t lora_linear_noalloc_selftest_timeout(uint32_t limit_us, void *stream) {
+    void *scratch = nullptr;
+    lora_status_t s = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
+    if (s != LORA_OK) return s;
+    return lora_linear_selftest_timeout(scratch, kNoallocScratchBytes, limit_us, stream);
 }

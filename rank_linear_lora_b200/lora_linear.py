@@ -309,3 +309,20 @@ def lora_linear_fwd_noalloc(x, W, A, B, h, xa_save, alpha, stream=None):
     st = fn(_ptr(x), _ptr(W), _ptr(A), _ptr(B), _ptr(h), _ptr(xa_save), M, d_in, d_out, r, float(alpha),
             _stream(stream))
     _check(st, "lora_linear_fwd_noalloc")
+
+
+def lora_linear_noalloc_check(stream=None):
+    """Wait for the stream, then read and clear the workspace-free forward's device error
+    word (raises LoraError LORA_ERR_TIMEOUT if a bounded wait of an earlier call ran out)."""
+    fn = load_library().lora_linear_noalloc_check
+    fn.argtypes = [ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(_stream(stream)), "lora_linear_noalloc_check")
+
+
+def lora_linear_noalloc_selftest_timeout(limit_us: int = 1000, stream=None):
+    """Enqueue the failure-path self-test on the workspace-free forward's error word."""
+    fn = load_library().lora_linear_noalloc_selftest_timeout
+    fn.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(int(limit_us), _stream(stream)), "lora_linear_noalloc_selftest_timeout")

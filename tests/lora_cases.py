@@ -2,6 +2,8 @@
 library through its C ABI, ask the oracle for the same quantities, compare."""
 from __future__ import annotations
 
+import time
+
 import numpy as np
 import torch
 
@@ -171,3 +173,86 @@ def check_projections(dl: "DeviceLayer", inp: inputs.LayerInputs, ref: dict, see
                                        f"|diff| {resid[i]:.3g} > {allow:.3g}")
             worst = max(worst, float(resid[i] / allow))
     return worst
+
+
+class ErrorTally:
+    """Running max-norm and rms statistics of (got - ref) over blocks of one tensor, so
+    that a tensor too large to hold twice in fp64 is still held to the contract's bound
+    on every element: ||got - ref||_inf <= rel * ||ref||_inf + abs, over the whole tensor."""
+
+    def __init__(self, name: str):
+        self.name = name
+        self.max_err = 0.0
+        self.max_ref = 0.0
+        self.where = None
+        self.sq_err = 0.0
+        self.sq_ref = 0.0
+        self.n = 0
+
+    def add(self, got: np.ndarray, ref: np.ndarray, row0: int = 0):
+        assert got.shape == ref.shape, (self.name, got.shape, ref.shape)
+        assert np.all(np.isfinite(got)), f"{self.name}: non-finite values in rows {row0}.."
+        err = np.abs(got - ref)
+        i = np.unravel_index(int(err.argmax()), err.shape)
+        if err[i] > self.max_err:
+            self.max_err = float(err[i])
+            self.where = (row0 + int(i[0]),) + tuple(int(v) for v in i[1:])
+        self.max_ref = max(self.max_ref, float(np.abs(ref).max()))
+        self.sq_err += float((err ** 2).sum())
+        self.sq_ref += float((ref ** 2).sum())
+        self.n += err.size
+
+    def check(self, tol, rms_tol=None):
+        rel, ab = tol
+        bound = rel * self.max_ref + ab
+        assert self.max_err <= bound, (f"{self.name}: max|err| {self.max_err:.4e} > {bound:.4e} at {self.where} "
+                                       f"({self.n} elements compared)")
+        if rms_tol is not None and self.sq_ref > 0:
+            rms = np.sqrt(self.sq_err / self.sq_ref)
+            assert rms <= rms_tol, f"{self.name}: rms rel err {rms:.3e} > {rms_tol:.1e}"
+        return self.max_err / bound
+
+
+def compare_every_element(dl: "DeviceLayer", inp: inputs.LayerInputs, block_rows: int = 1024) -> dict:
+    """Every element of h, dX, s.xa, dA and dB of a layer already run on the GPU against
+    the oracle's whole tensors: steps 1, 3, 5 and 6 from oracle.c, steps 2 and 4 for
+    every token row from the oracle's dense steps (numpy's fp64 product as the summation
+    primitive), a block of rows at a time.  Returns the worst error / bound per output
+    and the oracle's wall time."""
+    sp = inp.spec
+    if sp.q4:
+        wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale)
+    elif getattr(sp, "fp8", False):
+        wkw = dict(W8=inp.W8, W8scale=inp.W8scale)
+    else:
+        wkw = dict(W=inp.W)
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+    t_oracle = 0.0
+    t0 = time.perf_counter()
+    Wf = oracle.weight(sp.d_out, sp.d_in, **wkw)
+    xa_ = oracle.xa(inp.x, inp.A)
+    g_ = oracle.g(inp.dY, inp.B)
+    dA = oracle.da(inp.x, g_, sp.s)
+    dB = oracle.db(inp.dY, xa_, sp.s)
+    t_oracle += time.perf_counter() - t0
+    tally = {k: ErrorTally(k) for k in ("h", "dX", "xa_save", "dA", "dB")}
+    for r0 in range(0, sp.M, block_rows):
+        r1 = min(sp.M, r0 + block_rows)
+        t0 = time.perf_counter()
+        h_ref = oracle.h_dense(inp.x[r0:r1], inp.B, xa_[r0:r1], sp.s, Wf)
+        dx_ref = oracle.dx_dense(inp.dY[r0:r1], inp.A, g_[r0:r1], sp.s, Wf)
+        t_oracle += time.perf_counter() - t0
+        tally["h"].add(host_f64(dl.h[r0:r1]), h_ref, r0)
+        tally["dX"].add(host_f64(dl.dX[r0:r1]), dx_ref, r0)
+    tally["xa_save"].add(host_f64(dl.xa), sp.s * xa_)
+    tally["dA"].add(host_f64(dl.dA), dA)
+    tally["dB"].add(host_f64(dl.dB), dB)
+    worst = {
+        "h": tally["h"].check(TOL_HX, RMS_HX),
+        "dX": tally["dX"].check(TOL_HX, RMS_HX),
+        "xa_save": tally["xa_save"].check((2 ** -8, 1e-6), RMS_HX),
+        "dA": tally["dA"].check(TOL_AB, RMS_AB),
+        "dB": tally["dB"].check(TOL_AB, RMS_AB),
+    }
+    return {"worst": worst, "oracle_s": t_oracle, "elements": sum(t.n for t in tally.values())}

@@ -24,6 +24,13 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["cores"] >= 1 and d["cpu_baseline"]["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"].startswith("tiny")
+    # the same config keys as the GPU arm's line, so the two lines name one workload
+    sys.path.insert(0, ROOT)
+    import bench
+    from rank_linear_lora_b200 import inputs
+    spec = inputs.workload(0).layers[0]
+    assert d["config"] == bench.config_dict(spec, d["config"]["workload"], 1)
+    assert d["cpu_baseline"]["cpu_model"]
 
 
 def test_stacked_layer_counts_the_work_of_its_projections():
@@ -41,3 +48,24 @@ def test_stacked_layer_counts_the_work_of_its_projections():
     x_bytes = M * di * 2
     # forward reads x once; backward reads x once and writes one dX
     assert bench.algorithmic_bytes(stacked) == 2 * bench.algorithmic_bytes(gate) - 3 * x_bytes
+
+
+def test_gpus_2_spawns_two_ranks_and_prints_one_line():
+    """`bench.py --gpus 2` with no launcher around it starts two ranks itself; over a gloo
+    data plane (--dry-run: no GPU, the oracle on the host) they all-reduce the packed
+    [dA | dB] of their token shards, and rank 0 alone prints one JSON line whose reduced
+    gradients equal the whole batch's, with n_gpus 2 from the communicator."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run", "--backend",
+                        "gloo", "--config", "0"], capture_output=True, text=True, timeout=300, env=env)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    out = json.loads(lines[0])
+    assert out["n_gpus"] == 2 and out["world_size"] == 2 and out["dry_run"] is True
+    assert out["reduced_grads_match_whole_batch"] is True
+    assert out["config"]["parallelism"] == "dp2"

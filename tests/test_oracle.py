@@ -394,3 +394,32 @@ def test_merged_weight_reproduces_the_forward(q4):
     merged = oracle.merged_weight(inp.A, inp.B, spec.s, **wkw)
     h, _ = oracle.forward(inp.x, inp.A, inp.B, spec.s, **wkw)
     np.testing.assert_allclose(f64(inp.x) @ merged.T, h, rtol=0, atol=1e-12 * np.abs(h).max())
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "q4", "fp8"])
+def test_dense_steps_match_the_loops(fmt):
+    """The dense steps 2 and 4 (numpy's fp64 product as the summation primitive, used for
+    whole tensors at full size) equal oracle.c's loops up to fp64 summation order, for
+    every weight format, whole and a block of rows at a time."""
+    spec = inputs.LayerSpec("dense", 70, 192, 136, 16, alpha=32.0, q4=(fmt == "q4"), seed=0xD5)
+    inp = inputs.make_inputs(spec)
+    if fmt == "q4":
+        wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale)
+    elif fmt == "fp8":
+        W8, W8scale = inputs.quantise_fp8(inputs.bf16_bits_to_f32(inp.W))
+        wkw = dict(W8=W8, W8scale=W8scale)
+    else:
+        wkw = dict(W=inp.W)
+    h, xa_ = oracle.forward(inp.x, inp.A, inp.B, spec.s, **wkw)
+    bwd = oracle.backward(inp.dY, inp.x, inp.A, inp.B, spec.s, xa_=xa_, **wkw)
+    Wf = oracle.weight(spec.d_out, spec.d_in, **wkw)
+    hd = oracle.h_dense(inp.x, inp.B, xa_, spec.s, Wf)
+    dd = oracle.dx_dense(inp.dY, inp.A, bwd["g"], spec.s, Wf)
+    np.testing.assert_allclose(hd, h, rtol=0, atol=1e-13 * np.abs(h).max())
+    np.testing.assert_allclose(dd, bwd["dX"], rtol=0, atol=1e-13 * np.abs(bwd["dX"]).max())
+    # a block of rows (BLAS may take another kernel, e.g. for one row: same sums, other order)
+    for r0, r1 in ((0, 32), (32, 33), (33, 70)):
+        np.testing.assert_allclose(oracle.h_dense(inp.x[r0:r1], inp.B, xa_[r0:r1], spec.s, Wf), h[r0:r1],
+                                   rtol=0, atol=1e-13 * np.abs(h).max())
+        np.testing.assert_allclose(oracle.dx_dense(inp.dY[r0:r1], inp.A, bwd["g"][r0:r1], spec.s, Wf),
+                                   bwd["dX"][r0:r1], rtol=0, atol=1e-13 * np.abs(bwd["dX"]).max())
