@@ -159,6 +159,10 @@ class ClockSampler:
 
     def __enter__(self):
         if self.ok:
+            # The sampling thread needs the interpreter lock every half millisecond; the
+            # default switch interval (5 ms) would leave it one sample per timed region.
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
             self.t = threading.Thread(target=self._run, daemon=True)
             self.t.start()
         return self
@@ -167,6 +171,7 @@ class ClockSampler:
         if self.ok:
             self._stop.set()
             self.t.join()
+            sys.setswitchinterval(self._switch)
 
     def summary(self):
         if not self.ok or not self.samples:

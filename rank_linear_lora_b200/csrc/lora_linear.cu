@@ -3,13 +3,17 @@
 // Validates arguments, carves the caller's workspace, encodes TMA tensor maps and
 // enqueues the tcgen05 kernels of tc_gemm.cuh on the caller's stream:
 //
-//   forward   k_xa  : s.xa = bf16(s . x.A^T)            split over d_in   (M x r)
-//             k_fwd : h = [x | s.xa] . [W | B]^T        K = d_in + r, one accumulator
-//   backward  k_xa  : (only when no saved s.xa)
-//             k_g   : s.g = bf16(s . dY.B)              split over d_out  (M x r)
-//             k_dx  : dX = [dY | s.g] . [W ; A]         K = d_out + r, W and A MN-major
-//             k_dadb: dB = dY^T . (s.xa) and dA = (s.g)^T . x (written as [r, d_in]),
-//                     one launch, split over tokens, overlapping the dX GEMM's last wave
+//   forward   xa  : s.xa = bf16(s . x.A^T)                      reduction over d_in
+//             fwd : h = [x | s.xa] . [W | B]^T                  K = d_in + r, one accumulator
+//   backward  xa  : (only when no saved s.xa)
+//             g   : s.g = bf16(s . dY.B), and dB's partials     one pass over dY
+//             dx  : dX = [dY | s.g] . [W ; A]                   K = d_out + r, W and A MN-major
+//             dadb: dA = (s.g)^T . x (written as [r, d_in]), and dB summed from its
+//                   partials, overlapping the dX GEMM's last wave
+//
+// For r <= 64 the rank-r products run on the cluster-reduction side kernels of
+// side.cuh; wider ranks use the split-K kernels of tc_gemm.cuh (s.xa, s.g, then dB and
+// dA in one launch, each split over its reduction dimension with a fixed-order fix-up).
 //
 // No allocation, no synchronisation, no exceptions across the ABI.
 #include <cuda.h>
@@ -25,6 +29,7 @@
 #include <vector>
 
 #include "../../include/lora_linear.h"
+#include "side.cuh"
 #include "tc_gemm.cuh"
 #include "tc_gemm2.cuh"
 #include "tmap.h"
@@ -131,6 +136,14 @@ bool pair_enabled() {
     return !(v && v[0] == '0');
 }
 
+// Rank-r products (r <= 64) on the cluster-reduction side kernels; LORA_LINEAR_SIDE=0
+// selects the split-K kernels instead, for measurement.  Read when a plan is made
+// (the workspace size follows it).
+bool side_enabled() {
+    const char *v = std::getenv("LORA_LINEAR_SIDE");
+    return !(v && v[0] == '0');
+}
+
 // ------------------------------------------------------------------ launch helpers
 template <int BN, bool A_MN, bool B_MN, int EPI, int STAGES>
 cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
@@ -232,6 +245,86 @@ cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
     return e;
 }
 
+// Side kernels: clusters of C CTAs (1, 2 or 4), programmatic dependent launch.  The
+// grid is `clusters` clusters, capped at the clusters the device keeps resident at once
+// (the rounds are then spread over fewer clusters; results do not depend on the grid).
+template <int MODE, int STAGES>
+cudaError_t launch_side(const SideArgs &args, int clusters, int C, cudaStream_t st, DevInfo *dev, int attr_bit,
+                        int kind) {
+    using Cfg = SideCfg<MODE, STAGES>;
+    auto kern = k_side<MODE, STAGES>;
+    static int resident[64][4] = {};  // [device][log2 C]: clusters resident at once (0: not probed)
+    int d = 0;
+    cudaGetDevice(&d);
+    const int lc = C >= 4 ? 2 : C >= 2 ? 1 : 0;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (!(dev->attr_set & (1ull << attr_bit))) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            dev->attr_set |= 1ull << attr_bit;
+        }
+        if (d >= 0 && d < 64 && resident[d][lc] == 0) {
+            cudaLaunchConfig_t oc;
+            std::memset(&oc, 0, sizeof(oc));
+            oc.gridDim = dim3(static_cast<unsigned>(C * std::max(1, dev->sms / C)));
+            oc.blockDim = dim3(SIDE_THREADS);
+            oc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+            cudaLaunchAttribute ca[1];
+            ca[0].id = cudaLaunchAttributeClusterDimension;
+            ca[0].val.clusterDim.x = C;
+            ca[0].val.clusterDim.y = 1;
+            ca[0].val.clusterDim.z = 1;
+            oc.attrs = ca;
+            oc.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &oc) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = -1;  // unknown: no cap
+            }
+            resident[d][lc] = n;
+        }
+        if (d >= 0 && d < 64 && resident[d][lc] > 0) clusters = std::min(clusters, resident[d][lc]);
+    }
+    const int grid = clusters * C;
+    cudaEvent_t ea = nullptr, eb = nullptr;
+    const bool timed = g_timing.load() != 0;
+    if (timed) {
+        std::lock_guard<std::mutex> lk(g_tmu);
+        ea = pool_event();
+        eb = pool_event();
+        if (ea) cudaEventRecord(ea, st);
+    }
+    SideArgs a2 = args;
+    unsigned long long *tr = g_trace.load();
+    const size_t stride = g_trace_stride.load();
+    if (tr && static_cast<size_t>(grid) * TRACE_WORDS <= stride) a2.trace = tr + static_cast<size_t>(kind) * stride;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(SIDE_THREADS);
+    cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a2);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    g_launches.fetch_add(1);
+    if (timed && ea && eb) {
+        cudaEventRecord(eb, st);
+        std::lock_guard<std::mutex> lk(g_tmu);
+        g_timed.push_back({kind, ea, eb});
+    }
+    return e;
+}
+
 template <bool B_MN, bool Q4>
 int probe_pair_clusters(const DevInfo *dev) {
     constexpr int S = Q4 ? PAIR_STAGES_Q4 : PAIR_STAGES;
@@ -286,6 +379,7 @@ enum {
     AB_G64 = 6, AB_G128, AB_G256,
     AB_T64 = 9, AB_T128, AB_T256,
     AB_PAIR_K = 12, AB_PAIR_MN = 13, AB_PAIR_K_Q4 = 14, AB_PAIR_MN_Q4 = 15,
+    AB_SIDE_XA = 16, AB_SIDE_GDB = 17, AB_SIDE_DA = 18,
 };
 
 int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
@@ -341,39 +435,141 @@ MainSched main_sched(int64_t M, int64_t N, int G) {
     return s;
 }
 
+// Side-kernel plan (r <= 64): a cluster of C CTAs takes `group` 128-row output blocks
+// per round and splits the n_red reduction blocks among its CTAs.
+struct SidePlan {
+    int C = 1, clusters = 0, group = 1, rounds = 0, per_cta = 0, n_out = 0, n_red = 0;
+};
+
+constexpr int SIDE_XA_STAGES = 8;
+constexpr int SIDE_GDB_STAGES = 3;
+constexpr int SIDE_DA_STAGES = 4;
+
+// Cluster sizes of the side kernels.  A cluster's CTAs (one per SM: each holds ~225 KB
+// of shared memory) must fit in one GPC together; clusters of 8 did not all fit at once
+// on B200 and ran in two waves, clusters of 4 did.  dA, which starts on the SMs the dX
+// GEMM's CTA pairs leave as they finish, takes pairs.
+constexpr int SIDE_MAX_C = 4;
+constexpr int SIDE_MAX_C_DA = 2;
+
+// One output block per round; C the largest power of two <= max_c that keeps one round
+// of every output block within `sms` CTAs and gives each CTA some reduction work.
+SidePlan side_plan(int64_t n_out, int64_t n_red, int sms, int max_c) {
+    SidePlan sp;
+    int C = 1;
+    while (C < max_c && n_out * 2 * C <= sms && 2 * C <= n_red) C *= 2;
+    sp.C = C;
+    sp.n_out = static_cast<int>(n_out);
+    sp.n_red = static_cast<int>(n_red);
+    sp.group = 1;
+    sp.rounds = static_cast<int>(n_out);
+    sp.clusters = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(n_out, sms / C)));
+    sp.per_cta = static_cast<int>(cdiv(n_red, C));
+    return sp;
+}
+
+// Streaming cost model of the plans below: HBM bandwidth shared by the CTAs that
+// stream, up to what one SM's copy engine sustains on its own (both measured on B200).
+constexpr double SIDE_HBM_GBS = 6100.0;
+constexpr double SIDE_SM_GBS = 55.0;
+
+double side_stream_us(double bytes_per_cta, int ctas) {
+    const double bw = std::min(SIDE_HBM_GBS / std::max(1, ctas), SIDE_SM_GBS);
+    return bytes_per_cta / (bw * 1e3);
+}
+
+// s.g and dB in one pass over dY: `group` token blocks per round (their g accumulators
+// stay in tensor memory while the round's CTAs sweep d_out), C CTAs split d_out.  Each
+// round leaves one fp32 dB partial [d_out, r]; the choice weighs the streaming time of
+// the busiest CTA against writing those partials.
+SidePlan side_plan_gdb(int64_t M, int64_t d_out, int r, int sms) {
+    const int64_t n_out = cdiv(M, BM), n_red = cdiv(d_out, 128);
+    SidePlan best;
+    double best_cost = 1e300;
+    for (int a = 1; a <= 6; ++a) {
+        if (static_cast<int64_t>(a) * 128 * r * 4 > SIDE_RED_BYTES) break;  // the round's partials fit
+        for (int C = 1; C <= SIDE_MAX_C && C <= n_red; C *= 2) {
+            const int64_t need = cdiv(n_out, a);
+            const int64_t clusters = std::min<int64_t>(need, sms / C);
+            if (clusters < 1) continue;
+            const int64_t rounds_max = cdiv(need, clusters);
+            const int64_t per_cta = cdiv(n_red, C);
+            const double us = side_stream_us(double(rounds_max * a * per_cta) * 32768.0, static_cast<int>(clusters * C)) +
+                              double(need) * double(d_out) * r * 4.0 / (SIDE_HBM_GBS * 1e3);
+            if (us < best_cost * 0.999) {
+                best_cost = us;
+                best.C = C;
+                best.group = a;
+                best.n_out = static_cast<int>(n_out);
+                best.n_red = static_cast<int>(n_red);
+                best.rounds = static_cast<int>(need);
+                best.clusters = static_cast<int>(clusters);
+                best.per_cta = static_cast<int>(per_cta);
+            }
+        }
+    }
+    return best;
+}
+
+// The one-pass backward (s.g with dB's partials, then dA) writes one fp32 dB partial per
+// round of `group` token blocks: r / (64 * group) of the dY stream's bytes, with group
+// at most 64 / r (the landing area).  It is taken up to r = 32 (at most a quarter of the
+// stream); wider ranks run the backward's side products on the split-K kernels.
+constexpr int SIDE_MAX_R_BWD = 32;
+
 struct Plan {
     size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0;
     size_t total = 0;
     int64_t n_ctr = 0;
     Split s_xa, s_g, s_db, s_da;
+    bool side = false;          // s.xa on the side kernels (r <= 64)
+    bool side_bwd = false;      // s.g + dB and dA on the side kernels (r <= 32)
+    SidePlan sx, sg, sd;        // s.xa, s.g + dB partials, dA + dB
 };
 
 bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, Plan *pl) {
     const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4);
     const int64_t mt_tok = cdiv(M, BM), mt_in = cdiv(d_in, BM), mt_out = cdiv(d_out, BM);
+    size_t off = 0;
+    pl->err = off;
+    off += 256;
+    pl->side = r <= SIDE_MAX_R && side_enabled();
+    pl->side_bwd = bwd && r <= SIDE_MAX_R_BWD && side_enabled();
+    // split-K counters and partials (every s.xa when not on the side kernels; the
+    // backward's s.g, dB and dA when not on the side kernels)
+    const bool sk_xa = !pl->side, sk_bwd = bwd && !pl->side_bwd;
     pl->s_xa = choose_split(mt_tok, cdiv(d_in, BK), sms);
     pl->s_g = choose_split(mt_tok, cdiv(d_out, BK), sms);
     pl->s_db = choose_split(mt_out, cdiv(M, BK), sms);
     pl->s_da = choose_split(mt_in, cdiv(M, BK), sms);
-    size_t off = 0;
-    pl->err = off;
-    off += 256;
+    if (pl->side) pl->sx = side_plan(mt_tok, cdiv(d_in, BK), sms, SIDE_MAX_C);
+    if (pl->side_bwd) {
+        pl->sg = side_plan_gdb(M, d_out, r, sms);
+        pl->sd = side_plan(mt_in, mt_tok, sms, SIDE_MAX_C_DA);
+    }
     pl->ctr = off;
-    pl->n_ctr = mt_tok * 2 + mt_in + mt_out;
+    pl->n_ctr = (sk_xa || sk_bwd) ? mt_tok * 2 + mt_in + mt_out : 0;
     off = align256(off + pl->n_ctr * sizeof(int));
     pl->xa = off;
     off = align256(off + M * r * 2);
-    pl->part_xa = off;
-    off = align256(off + static_cast<size_t>(pl->s_xa.splits) * mt_tok * BM * r * 4);
+    if (sk_xa) {
+        pl->part_xa = off;
+        off = align256(off + static_cast<size_t>(pl->s_xa.splits) * mt_tok * BM * r * 4);
+    }
     if (bwd) {
         pl->g = off;
         off = align256(off + M * r * 2);
-        pl->part_g = off;
-        off = align256(off + static_cast<size_t>(pl->s_g.splits) * mt_tok * BM * r * 4);
-        pl->part_db = off;
-        off = align256(off + static_cast<size_t>(pl->s_db.splits) * mt_out * BM * r * 4);
-        pl->part_da = off;
-        off = align256(off + static_cast<size_t>(pl->s_da.splits) * mt_in * BM * r * 4);
+        if (pl->side_bwd) {
+            pl->part_db = off;
+            off = align256(off + static_cast<size_t>(pl->sg.rounds) * d_out * r * 4);
+        } else {
+            pl->part_g = off;
+            off = align256(off + static_cast<size_t>(pl->s_g.splits) * mt_tok * BM * r * 4);
+            pl->part_db = off;
+            off = align256(off + static_cast<size_t>(pl->s_db.splits) * mt_out * BM * r * 4);
+            pl->part_da = off;
+            off = align256(off + static_cast<size_t>(pl->s_da.splits) * mt_in * BM * r * 4);
+        }
     }
     pl->total = off;
     return true;
@@ -525,6 +721,84 @@ lora_status_t step_dadb(const Ctx &c, const uint16_t *dY, const uint16_t *x, con
     a.job[1] = make_job(r, d_in, M, c.plan.s_da, reinterpret_cast<float *>(c.ws + c.plan.part_da),
                         counters_at(c, 2 * cdiv(M, BM) + cdiv(d_out, BM)), dA, OUT_F32_COLS, d_in, 1.0f);
     return launch_skinny<true, true>(c, a, r, grid_cap, LORA_K_DADB);
+}
+
+// ------------------------------------------------------------------ side kernels (r <= 64)
+SideArgs side_args(const Ctx &c) {
+    SideArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.err = reinterpret_cast<int *>(c.ws + c.plan.err);
+    a.group = 1;
+    return a;
+}
+
+void side_fill(SideArgs &a, const SidePlan &sp, int r) {
+    a.r = r;
+    a.n_out = sp.n_out;
+    a.n_red = sp.n_red;
+    a.per_cta = sp.per_cta;
+    a.group = sp.group;
+    a.n_rounds = sp.rounds;
+}
+
+// s.xa = bf16(s . x.A^T) -> dst [M, r]
+lora_status_t side_xa(const Ctx &c, const uint16_t *x, const uint16_t *A, uint16_t *dst, int64_t M, int64_t d_in,
+                      int r, float s) {
+    const SidePlan &sp = c.plan.sx;
+    SideArgs a = side_args(c);
+    side_fill(a, sp, r);
+    a.nr = (r + 15) / 16 * 16;
+    if (!tmap_bf16(&a.tmX, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmS0, A, d_in, r, 64, a.nr)) return LORA_ERR_CUDA;
+    a.rows_valid = static_cast<int>(M);
+    a.scale = s;
+    a.out_bf16 = dst;
+    const cudaError_t e =
+        launch_side<SIDE_XA, SIDE_XA_STAGES>(a, sp.clusters, sp.C, c.st, c.info, AB_SIDE_XA, LORA_K_XA);
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// One pass over dY: s.g = bf16(s . dY.B) -> ws g [M, r], and dB's partials over each
+// round's tokens -> ws [rounds][d_out][r].  B [d_out, r] and s.xa [M, r] are read MN-major.
+lora_status_t side_gdb(const Ctx &c, const uint16_t *dY, const uint16_t *B, const uint16_t *sxa, int64_t M,
+                       int64_t d_out, int r, float s) {
+    const SidePlan &sp = c.plan.sg;
+    SideArgs a = side_args(c);
+    side_fill(a, sp, r);
+    if (!tmap_bf16(&a.tmX, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmS0, B, r, d_out, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmS1, sxa, r, M, 64, 128)) return LORA_ERR_CUDA;
+    a.rows_valid = static_cast<int>(M);
+    a.scale = s;
+    a.out_bf16 = reinterpret_cast<uint16_t *>(c.ws + c.plan.g);
+    a.db_part = reinterpret_cast<float *>(c.ws + c.plan.part_db);
+    a.d_out = static_cast<int>(d_out);
+    const cudaError_t e =
+        launch_side<SIDE_GDB, SIDE_GDB_STAGES>(a, sp.clusters, sp.C, c.st, c.info, AB_SIDE_GDB, LORA_K_G);
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+// dA [r, d_in] = ((s.g)^T . x), and dB [d_out, r] = the sum of the partials.  `defer`:
+// launched right after the dX GEMM, whose outputs it does not read, so it starts on the
+// SMs that GEMM's last wave leaves idle; `grid_cap` bounds its CTAs.
+lora_status_t side_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float *dA, float *dB, int64_t M,
+                      int64_t d_in, int64_t d_out, int r, bool defer, int grid_cap) {
+    const SidePlan &sp = c.plan.sd;
+    SideArgs a = side_args(c);
+    side_fill(a, sp, r);
+    a.defer_dep_wait = defer ? 1 : 0;
+    if (!tmap_bf16(&a.tmX, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_bf16(&a.tmS0, sg, r, M, 64, 128)) return LORA_ERR_CUDA;
+    a.rows_valid = static_cast<int>(d_in);
+    a.out_f32 = dA;
+    a.db_part = reinterpret_cast<float *>(c.ws + c.plan.part_db);
+    a.d_out = static_cast<int>(d_out);
+    a.dB = dB;
+    a.db_rounds = c.plan.sg.rounds;
+    const int clusters = std::max(1, std::min(sp.clusters, grid_cap / sp.C));
+    const cudaError_t e =
+        launch_side<SIDE_DA, SIDE_DA_STAGES>(a, clusters, sp.C, c.st, c.info, AB_SIDE_DA, LORA_K_DADB);
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
 // Main K-concatenated GEMM: out [M, N] = A0 . B0^T (K0) + A1 . B1^T (K1 = r).
@@ -679,7 +953,7 @@ lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, c
     LORA_TRY(prepare(wt.q4() ? LORA_OP_FWD_Q4 : LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
-    LORA_TRY(step_xa(c, x, A, sxa, M, d_in, r, s));
+    LORA_TRY(c.plan.side ? side_xa(c, x, A, sxa, M, d_in, r, s) : step_xa(c, x, A, sxa, M, d_in, r, s));
     const MainOperands o = main_operands(wt, x, sxa, B, h, d_out, d_in);
     return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, true);
 }
@@ -698,12 +972,15 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
     const uint16_t *sxa = xa_save;
     if (!sxa) {
         uint16_t *tmp = reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
-        LORA_TRY(step_xa(c, x, A, tmp, M, d_in, r, s));
+        LORA_TRY(c.plan.side ? side_xa(c, x, A, tmp, M, d_in, r, s) : step_xa(c, x, A, tmp, M, d_in, r, s));
         sxa = tmp;
     }
-    LORA_TRY(step_g(c, dY, B, M, d_out, r, s));
+    if (c.plan.side_bwd)
+        LORA_TRY(side_gdb(c, dY, B, sxa, M, d_out, r, s));
+    else
+        LORA_TRY(step_g(c, dY, B, M, d_out, r, s));
     const uint16_t *sg = reinterpret_cast<const uint16_t *>(c.ws + c.plan.g);
-    // dB and dA read nothing the dX GEMM writes: launched after it (programmatic
+    // dA (and dB) read nothing the dX GEMM writes: launched after it (programmatic
     // dependent launch), they start on the SMs its last wave leaves idle and wait for
     // it only before they exit.  The dX tail is then left whole (no narrow tiles) so
     // those SMs free up early.
@@ -713,6 +990,13 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
         // W [d_out, d_in] (or its codes) and A [r, d_in] are read MN-major (d_in contiguous).
         const MainOperands o = main_operands(wt, dY, sg, A, dX, d_out, d_in);
         LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
+    }
+    if (c.plan.side_bwd) {
+        // On the idle SMs alone when there are enough of them to be worth a cluster grid;
+        // otherwise every SM, the rest of the CTAs starting as the dX CTAs exit.
+        const int cap = (overlap && idle >= 32) ? idle : PLAN_SMS;
+        LORA_TRY(side_da(c, x, sg, dA, dB, M, d_in, d_out, r, overlap, cap));
+        return LORA_OK;
     }
     // Grid: the idle SMs when they can take all the dB / dA split tiles within about
     // four each (they then finish close to the dX GEMM); otherwise every SM, the rest of

@@ -312,3 +312,36 @@ def test_bounded_wait_timeout_is_reported_and_recoverable():
     dl.backward()
     dl.check()
     compare_all(dl.results(), oracle_ref(inp), spec.s)
+
+
+# Rank-r side kernels (r <= 64): clusters of 1 to 8 CTAs reduce over distributed shared
+# memory; these shapes reach several rounds per cluster (more 128-row output blocks
+# than CTAs), s.g + dB rounds of 1 to 5 token blocks, clusters in which some CTAs hold
+# no share of the reduction, and every rank width the MMA pads (r % 16 != 0, r = 64).
+SIDE = [
+    (40000, 64, 64, 8),       # s.xa: 313 token blocks on 148 CTAs (3 rounds); dA on an 8-CTA cluster
+    (40000, 192, 1000, 16),   # s.g + dB: 5 token blocks per round, 2-CTA clusters
+    (2048, 2048, 2048, 32),
+    (1024, 512, 3000, 48),    # ragged d_out (partial last column block), r = 48
+    (4500, 4160, 1800, 56),   # ragged M, d_in, d_out
+    (384, 320, 8, 64),        # d_out = 8: one column block; d_in = 320: CTAs with no reduction share
+]
+
+
+@pytest.mark.parametrize("shape", SIDE, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_side_kernels_every_element(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("side", M, di, do, r, alpha=2.0 * r, seed=0x51DE + M + do)
+    inp, dl = _run_full(spec)
+    compare_every_element(dl, inp)
+
+
+@pytest.mark.parametrize("shape", [(200, 328, 200, 8), (1024, 512, 3000, 48), (2048, 2048, 2048, 32)],
+                         ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_split_k_side_products_for_narrow_ranks(shape, monkeypatch):
+    """The split-K kernels (used above r = 64) on ranks the side kernels take by default."""
+    monkeypatch.setenv("LORA_LINEAR_SIDE", "0")
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("splitk", M, di, do, r, alpha=2.0 * r, seed=0x5B1 + M)
+    inp, dl = _run_full(spec)
+    compare_every_element(dl, inp)
