@@ -48,6 +48,8 @@ def parse():
     p.add_argument("--config", type=int, default=1, help="workload index (1: attention projection)")
     p.add_argument("--rank-r", type=int, default=None, help="rank for the rank-sweep workload")
     p.add_argument("--layer", type=int, default=0, help="layer of a multi-layer workload")
+    p.add_argument("--fp8", action="store_true",
+                   help="store the workload's frozen weight as FP8 (E4M3 codes, one bf16 scale per row)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
@@ -77,7 +79,7 @@ def algorithmic_bytes(spec) -> float:
     columns per row); A, xa and dA hold every projection's ranks."""
     M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
     rb = r // spec.proj
-    w = do * di // 2 + do * (di // 64) * 2 if spec.q4 else do * di * 2
+    w = do * di // 2 + do * (di // 64) * 2 if spec.q4 else do * di + do * 2 if spec.fp8 else do * di * 2
     fwd = M * di * 2 + w + r * di * 2 + do * rb * 2 + M * do * 2 + M * r * 2
     bwd = M * do * 2 + M * di * 2 + w + r * di * 2 + do * rb * 2 + M * r * 2 + M * di * 2 + r * di * 4 + do * rb * 4
     return float(fwd + bwd)
@@ -194,7 +196,8 @@ class ClockSampler:
 def config_dict(spec, workload_name: str, world: int) -> dict:
     """The workload as both arms name it (identical keys and values)."""
     return {"workload": workload_name, "M": spec.M, "d_in": spec.d_in, "d_out": spec.d_out, "r": spec.r,
-            "alpha": spec.alpha, "q4": spec.q4, "projections": spec.proj, "tokens_per_step": spec.M * world,
+            "alpha": spec.alpha, "q4": spec.q4, "fp8": spec.fp8, "projections": spec.proj,
+            "tokens_per_step": spec.M * world,
             "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
             "parallelism": f"dp{world}"}
 
@@ -330,7 +333,8 @@ def _oracle_step(oracle, inp, spec, start, tokens):
     M = spec.M
     rows = [(start + i) % M for i in range(tokens)]
     x, dY = inp.x[rows], inp.dY[rows]
-    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if spec.q4 else dict(W=inp.W)
+    wkw = (dict(Wq=inp.Wq, Wscale=inp.Wscale) if spec.q4 else dict(W8=inp.W8, W8scale=inp.W8scale) if spec.fp8
+           else dict(W=inp.W))
     h, xa = oracle.forward(x, inp.A, inp.B, spec.s, **wkw)
     oracle.backward(dY, x, inp.A, inp.B, spec.s, xa_=xa, **wkw)
 
@@ -395,6 +399,9 @@ def main():
     wl = inputs.workload(args.config, r=args.rank_r)
     spec = wl.layers[args.layer]
     workload_name = f"{wl.name} / {spec.name}"
+    if args.fp8:
+        spec = spec.with_(q4=False, fp8=True)
+        workload_name += " with the FP8 weight"
     if args.shape:
         M_, di_, do_ = (int(v) for v in args.shape.split(","))
         spec = spec.with_(M=M_, d_in=di_, d_out=do_)
@@ -440,6 +447,9 @@ def main():
         if spec.q4:
             s["Wq"] = torch.from_numpy(inp.Wq).to(dev)
             s["Wscale"] = d16(inp.Wscale)
+        elif spec.fp8:
+            s["W8"] = torch.from_numpy(inp.W8).to(dev)
+            s["W8scale"] = d16(inp.W8scale)
         else:
             s["W"] = d16(inp.W)
         s["h"] = torch.empty(M, do, dtype=torch.bfloat16, device=dev)
@@ -447,7 +457,8 @@ def main():
         s["dX"] = torch.empty(M, di, dtype=torch.bfloat16, device=dev)
         s["grad"] = PackedGrads(r, di, do, device=dev)  # fp32 [dA | dB], the one all-reduced buffer
         s["dA"], s["dB"] = s["grad"].dA, s["grad"].dB
-        fop, bop = (L.OP_FWD_Q4, L.OP_BWD_Q4) if spec.q4 else (L.OP_FWD, L.OP_BWD)
+        fop, bop = ((L.OP_FWD_Q4, L.OP_BWD_Q4) if spec.q4 else (L.OP_FWD_FP8, L.OP_BWD_FP8) if spec.fp8
+                    else (L.OP_FWD, L.OP_BWD))
         s["wsf"] = L.workspace(fop, M, di, do, r, device=dev)
         s["wsb"] = L.workspace(bop, M, di, do, r, device=dev)
         sets.append(s)
@@ -457,6 +468,10 @@ def main():
             L.lora_linear_fwd_q4(s["x"], s["Wq"], s["Wscale"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
             L.lora_linear_bwd_q4(s["dY"], s["x"], s["Wq"], s["Wscale"], s["A"], s["B"], s["xa"], s["dX"], s["dA"],
                                  s["dB"], alpha, s["wsb"])
+        elif spec.fp8:
+            L.lora_linear_fwd_fp8(s["x"], s["W8"], s["W8scale"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
+            L.lora_linear_bwd_fp8(s["dY"], s["x"], s["W8"], s["W8scale"], s["A"], s["B"], s["xa"], s["dX"],
+                                  s["dA"], s["dB"], alpha, s["wsb"])
         else:
             L.lora_linear_fwd(s["x"], s["W"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
             L.lora_linear_bwd(s["dY"], s["x"], s["W"], s["A"], s["B"], s["xa"], s["dX"], s["dA"], s["dB"], alpha,
@@ -554,6 +569,9 @@ def main():
             if spec.q4:
                 L.lora_linear_fwd_q4(st["x"], st["Wq"], st["Wscale"], st["A"], st["B"], st["h"], st["xa"], alpha,
                                      st["wsf"])
+            elif spec.fp8:
+                L.lora_linear_fwd_fp8(st["x"], st["W8"], st["W8scale"], st["A"], st["B"], st["h"], st["xa"], alpha,
+                                      st["wsf"])
             else:
                 L.lora_linear_fwd(st["x"], st["W"], st["A"], st["B"], st["h"], st["xa"], alpha, st["wsf"])
 
@@ -561,6 +579,9 @@ def main():
             if spec.q4:
                 L.lora_linear_bwd_q4(st["dY"], st["x"], st["Wq"], st["Wscale"], st["A"], st["B"], st["xa"], st["dX"],
                                      st["dA"], st["dB"], alpha, st["wsb"])
+            elif spec.fp8:
+                L.lora_linear_bwd_fp8(st["dY"], st["x"], st["W8"], st["W8scale"], st["A"], st["B"], st["xa"],
+                                      st["dX"], st["dA"], st["dB"], alpha, st["wsb"])
             else:
                 L.lora_linear_bwd(st["dY"], st["x"], st["W"], st["A"], st["B"], st["xa"], st["dX"], st["dA"],
                                   st["dB"], alpha, st["wsb"])
@@ -584,7 +605,7 @@ def main():
     # Context, not the reference arm: the unfused composition of the same layer in PyTorch
     # with autograd (x@W.T + s*(x@A.T)@B.T, cuBLAS bf16), same inputs, same GPU.
     context = None
-    if world == 1 and not spec.q4:
+    if world == 1 and not spec.q4 and not spec.fp8:
         st = sets[0]
         xg = st["x"].detach().clone().requires_grad_(True)
         Ag = st["A"].detach().clone().requires_grad_(True)
@@ -618,7 +639,7 @@ def main():
     # median of 20.  Before each launch L2 is flushed by reading 256 MB (clean lines: a
     # write would leave ~126 MB of dirty lines for the merge to write back).
     merge = None
-    if rank == 0:
+    if rank == 0 and not spec.fp8:
         s0 = sets[0]
         w_out = torch.empty(do, di, dtype=torch.bfloat16, device=dev)
         flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)

@@ -38,7 +38,7 @@
  *     1 <= M <= 2^30; d_in and d_out multiples of 8 in 8 .. 2^24, with
  *     ceil(M/128) * ceil(max(d_in, d_out)/128) <= 2^31 - 1 (32-bit tile counts: only
  *     an output of more than 2^45 elements reaches it); 1 <= r <= 256 with r % 8 == 0; alpha finite;
- *     for *_q4 also d_in % 64 == 0.
+ *     for *_q4 also d_in % 64 == 0; for *_fp8 d_in % 16 == 0.
  *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
  *     aligned, be zero-filled before its first use, and must not be used by two calls
  *     that may run at the same time.  Every call that completes leaves the workspace's
@@ -48,8 +48,9 @@
  *     for its predecessor in the stream before touching global memory, so stream
  *     order is preserved; only launch latency and set-up overlap.
  *   - The device must be compute capability 10.0 (B200); otherwise
- *     LORA_ERR_UNSUPPORTED is returned and nothing runs.  The *_q4 entry points also
- *     need two-SM clusters (CTA pairs); without them they return LORA_ERR_UNSUPPORTED.
+ *     LORA_ERR_UNSUPPORTED is returned and nothing runs.  The *_q4 and *_fp8 entry
+ *     points also need two-SM clusters (CTA pairs); without them they return
+ *     LORA_ERR_UNSUPPORTED.
  *   - Device-side waits are bounded.  A wait that runs out sets an error word in the
  *     workspace and the kernels return early; lora_linear_check() reports it.
  *   - No C++ exception crosses this interface.
@@ -88,7 +89,9 @@ typedef enum {
     LORA_OP_FWD = 0,
     LORA_OP_BWD = 1,
     LORA_OP_FWD_Q4 = 2,
-    LORA_OP_BWD_Q4 = 3
+    LORA_OP_BWD_Q4 = 3,
+    LORA_OP_FWD_FP8 = 4,
+    LORA_OP_BWD_FP8 = 5
 } lora_op_t;
 
 /* Bytes of workspace the given operation needs for these sizes (0 if the sizes are
@@ -148,6 +151,31 @@ LORA_API lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x,
                                  const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
                                  int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Forward with an FP8 frozen weight: the weight is stored as E4M3 codes with one bf16
+ * scale per output row and the layer computes in bf16 (page
+ * "ms-swift高效微调组合：LoRA+UnSloth提速实践", section 3.2: FP8 storage of the
+ * weights with BF16 computation).  The codes are decoded in shared memory inside the
+ * GEMMs and never written back as bf16; each decoded weight is e4m3(q) * scale, formed
+ * exactly in fp32 and rounded once to bf16 for the tensor cores.
+ *   W8 [d_out, d_in] uint8, one E4M3 code per weight (sign, 4-bit exponent of bias 7,
+ *   3-bit mantissa; 0x7F / 0xFF are NaN);  W8scale [d_out] bf16.
+ * As lora_linear_fwd with W replaced by (W8, W8scale); d_in % 16 == 0; the workspace is
+ * lora_linear_workspace_size(LORA_OP_FWD_FP8, ...). */
+LORA_API lora_status_t lora_linear_fwd_fp8(const uint16_t *x, const uint8_t *W8, const uint16_t *W8scale,
+                                           const uint16_t *A, const uint16_t *B, uint16_t *h,
+                                           uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out,
+                                           int r, float alpha, void *workspace, size_t workspace_bytes,
+                                           void *stream);
+
+/* Backward with the FP8 frozen weight (same passage and layout); as lora_linear_bwd
+ * with W replaced by (W8, W8scale); workspace of LORA_OP_BWD_FP8. */
+LORA_API lora_status_t lora_linear_bwd_fp8(const uint16_t *dY, const uint16_t *x, const uint8_t *W8,
+                                           const uint16_t *W8scale, const uint16_t *A, const uint16_t *B,
+                                           const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
+                                           int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                                           void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Forward without a workspace, for callers that cannot allocate device memory: a

@@ -193,12 +193,18 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
 
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_STAGES_Q4 = 5;
+constexpr int PAIR_STAGES_FP8 = 4;  // the FP8 code rings take twice the 4-bit ones' shared memory
 
-template <bool B_MN, bool Q4>
+template <int WF>
+constexpr int pair_stages() {
+    return WF == WF_Q4 ? PAIR_STAGES_Q4 : WF == WF_FP8 ? PAIR_STAGES_FP8 : PAIR_STAGES;
+}
+
+template <bool B_MN, int WF>
 cudaError_t launch_pair(const GemmArgs &args, int grid, cudaStream_t st, DevInfo *dev, int attr_bit, int kind) {
-    constexpr int S = Q4 ? PAIR_STAGES_Q4 : PAIR_STAGES;
-    using Cfg = PairCfg<B_MN, Q4, S>;
-    auto kern = k_tc_gemm_pair<B_MN, Q4, S>;
+    constexpr int S = pair_stages<WF>();
+    using Cfg = PairCfg<B_MN, WF, S>;
+    auto kern = k_tc_gemm_pair<B_MN, WF, S>;
     {
         std::lock_guard<std::mutex> lk(g_mu);
         if (!(dev->attr_set & (1ull << attr_bit))) {
@@ -325,11 +331,11 @@ cudaError_t launch_side(const SideArgs &args, int clusters, int C, cudaStream_t 
     return e;
 }
 
-template <bool B_MN, bool Q4>
+template <bool B_MN, int WF>
 int probe_pair_clusters(const DevInfo *dev) {
-    constexpr int S = Q4 ? PAIR_STAGES_Q4 : PAIR_STAGES;
-    using Cfg = PairCfg<B_MN, Q4, S>;
-    auto kern = k_tc_gemm_pair<B_MN, Q4, S>;
+    constexpr int S = pair_stages<WF>();
+    using Cfg = PairCfg<B_MN, WF, S>;
+    auto kern = k_tc_gemm_pair<B_MN, WF, S>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM_BYTES) != cudaSuccess) {
         cudaGetLastError();
         return 0;
@@ -355,18 +361,24 @@ int probe_pair_clusters(const DevInfo *dev) {
 }
 
 // Clusters of two CTAs of the pair kernel that can be resident at once (0 if none).
-int pair_clusters(DevInfo *dev, bool b_mn, bool q4) {
-    static int cached[64][4] = {};
-    static bool probed[64][4] = {};
+int pair_clusters(DevInfo *dev, bool b_mn, int wf) {
+    static int cached[64][6] = {};
+    static bool probed[64][6] = {};
     int d = 0;
     cudaGetDevice(&d);
     std::lock_guard<std::mutex> lk(g_mu);
     if (d < 0 || d >= 64) return 0;
-    const int v = (b_mn ? 1 : 0) + (q4 ? 2 : 0);
+    const int v = (b_mn ? 1 : 0) + 2 * wf;
     if (!probed[d][v]) {
         probed[d][v] = true;
-        cached[d][v] = b_mn ? (q4 ? probe_pair_clusters<true, true>(dev) : probe_pair_clusters<true, false>(dev))
-                            : (q4 ? probe_pair_clusters<false, true>(dev) : probe_pair_clusters<false, false>(dev));
+        switch (v) {
+            case 0: cached[d][v] = probe_pair_clusters<false, WF_BF16>(dev); break;
+            case 1: cached[d][v] = probe_pair_clusters<true, WF_BF16>(dev); break;
+            case 2: cached[d][v] = probe_pair_clusters<false, WF_Q4>(dev); break;
+            case 3: cached[d][v] = probe_pair_clusters<true, WF_Q4>(dev); break;
+            case 4: cached[d][v] = probe_pair_clusters<false, WF_FP8>(dev); break;
+            default: cached[d][v] = probe_pair_clusters<true, WF_FP8>(dev); break;
+        }
     }
     return cached[d][v];
 }
@@ -380,6 +392,7 @@ enum {
     AB_T64 = 9, AB_T128, AB_T256,
     AB_PAIR_K = 12, AB_PAIR_MN = 13, AB_PAIR_K_Q4 = 14, AB_PAIR_MN_Q4 = 15,
     AB_SIDE_XA = 16, AB_SIDE_GDB = 17, AB_SIDE_DA = 18,
+    AB_PAIR_K_FP8 = 19, AB_PAIR_MN_FP8 = 20,
 };
 
 int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
@@ -528,7 +541,7 @@ struct Plan {
 };
 
 bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, Plan *pl) {
-    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4);
+    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8);
     const int64_t mt_tok = cdiv(M, BM), mt_in = cdiv(d_in, BM), mt_out = cdiv(d_out, BM);
     size_t off = 0;
     pl->err = off;
@@ -578,7 +591,8 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
 // ------------------------------------------------------------------ validation
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, bool q4) {
+// wf: the frozen weight's format (WF_BF16, WF_Q4, WF_FP8).
+lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, int wf) {
     if (M < 1 || M > (int64_t(1) << 30)) return LORA_ERR_INVALID_ARG;
     if (d_in < 8 || d_out < 8 || d_in % 8 || d_out % 8) return LORA_ERR_INVALID_ARG;
     if (d_in > (int64_t(1) << 24) || d_out > (int64_t(1) << 24)) return LORA_ERR_INVALID_ARG;
@@ -587,7 +601,8 @@ lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float 
     if (((M + 127) / 128) * ((std::max(d_in, d_out) + 127) / 128) > INT32_MAX) return LORA_ERR_INVALID_ARG;
     if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
     if (!std::isfinite(alpha)) return LORA_ERR_INVALID_ARG;
-    if (q4 && d_in % 64) return LORA_ERR_INVALID_ARG;
+    if (wf == WF_Q4 && d_in % 64) return LORA_ERR_INVALID_ARG;   // one scale per 64 codes
+    if (wf == WF_FP8 && d_in % 16) return LORA_ERR_INVALID_ARG;  // code rows of whole 16-byte units
     return LORA_OK;
 }
 
@@ -807,9 +822,10 @@ lora_status_t side_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float
 struct MainOperands {
     const void *A0, *B0, *A1, *B1;
     void *C;
-    const uint8_t *Wq = nullptr;       // 4-bit frozen weight (B0 is then unused)
-    const uint16_t *Wscale = nullptr;  // its bf16 scales [d_out, d_in / 64]
+    const uint8_t *Wq = nullptr;       // 4-bit or FP8 frozen weight's codes (B0 is then unused)
+    const uint16_t *Wscale = nullptr;  // its bf16 scales: [d_out, d_in / 64] (4-bit) or [d_out] (FP8)
     int64_t q_rows = 0, q_cols = 0;    // W shape [d_out, d_in]
+    int wf = WF_BF16;
 };
 
 // `idle_sms` (optional) receives how many SMs the last wave leaves without work.
@@ -822,17 +838,17 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     if (!tmap_bf16(&a.tmA0, o.A0, K0, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmA1, o.A1, r, M, 64, 128)) return LORA_ERR_CUDA;
     if (!tmap_bf16(&a.tmC, o.C, N, M, 64, 32)) return LORA_ERR_CUDA;
-    const bool q4 = o.Wq != nullptr;
-    const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn, q4), PLAN_SMS / 2) : 0;
-    if (q4 && pair_C == 0) return LORA_ERR_UNSUPPORTED;  // the 4-bit path runs on CTA pairs only
+    const bool q4 = o.wf != WF_BF16;  // codes decoded in shared memory (4-bit or FP8)
+    const int pair_C = pair_enabled() ? std::min(pair_clusters(c.info, b_mn, o.wf), PLAN_SMS / 2) : 0;
+    if (q4 && pair_C == 0) return LORA_ERR_UNSUPPORTED;  // decoded weights run on CTA pairs only
     if (q4) {
         a.wscale = o.Wscale;
-        a.scale_ld = static_cast<int>(o.q_cols / 64);
+        a.scale_ld = o.wf == WF_Q4 ? static_cast<int>(o.q_cols / 64) : 1;
         a.scale_rows = static_cast<int>(o.q_rows);
-        // packed codes [d_out][d_in / 2] bytes; each dequant warp fetches DQ_QROWS rows
-        // x 32 bytes (64 codes per row) at a time
-        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols / 2, o.q_rows, 32, DQ_QROWS))
-            return LORA_ERR_CUDA;
+        // codes [d_out][d_in / 2] (4-bit) or [d_out][d_in] (FP8) bytes; each dequant warp
+        // fetches DQ_QROWS rows x the bytes of 64 codes at a time
+        const int rb = dq_run_bytes(o.wf);
+        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols * rb / 64, o.q_rows, rb, DQ_QROWS)) return LORA_ERR_CUDA;
         allow_tail_split = false;
     }
     if (pair_C > 0) {
@@ -862,12 +878,15 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         const int clusters = split ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
         if (idle_sms) *idle_sms = (!split && R > 0 && W >= 1) ? c.info->sms - static_cast<int>(2 * R) : 0;
         cudaError_t e;
-        if (q4)
-            e = b_mn ? launch_pair<true, true>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_Q4, kind)
-                     : launch_pair<false, true>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_Q4, kind);
+        if (o.wf == WF_Q4)
+            e = b_mn ? launch_pair<true, WF_Q4>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_Q4, kind)
+                     : launch_pair<false, WF_Q4>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_Q4, kind);
+        else if (o.wf == WF_FP8)
+            e = b_mn ? launch_pair<true, WF_FP8>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_FP8, kind)
+                     : launch_pair<false, WF_FP8>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_FP8, kind);
         else
-            e = b_mn ? launch_pair<true, false>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
-                     : launch_pair<false, false>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
+            e = b_mn ? launch_pair<true, WF_BF16>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
+                     : launch_pair<false, WF_BF16>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
         return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
     }
     // Single-SM kernel: 128 x 256 tiles.
@@ -922,19 +941,23 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
 // scales Wscale [d_out, d_in / 64] (dequantised in shared memory inside the GEMMs).
 struct Weight {
     const uint16_t *W = nullptr;
-    const uint8_t *Wq = nullptr;
+    const uint8_t *Wq = nullptr;       // 4-bit or FP8 codes
     const uint16_t *Wscale = nullptr;
-    bool q4() const { return Wq != nullptr; }
-    bool present() const { return q4() ? (Wq && Wscale) : W != nullptr; }
-    bool aligned() const { return q4() ? (aligned16(Wq) && aligned16(Wscale)) : aligned16(W); }
+    int wf = WF_BF16;
+    bool coded() const { return wf != WF_BF16; }
+    bool present() const { return coded() ? (Wq && Wscale) : W != nullptr; }
+    bool aligned() const { return coded() ? (aligned16(Wq) && aligned16(Wscale)) : aligned16(W); }
+    int op_fwd() const { return wf == WF_Q4 ? LORA_OP_FWD_Q4 : wf == WF_FP8 ? LORA_OP_FWD_FP8 : LORA_OP_FWD; }
+    int op_bwd() const { return wf == WF_Q4 ? LORA_OP_BWD_Q4 : wf == WF_FP8 ? LORA_OP_BWD_FP8 : LORA_OP_BWD; }
 };
 
 MainOperands main_operands(const Weight &wt, const void *A0, const void *A1, const void *B1, void *C,
                            int64_t d_out, int64_t d_in) {
     MainOperands o{A0, wt.W, A1, B1, C};
-    if (wt.q4()) {
+    if (wt.coded()) {
         o.Wq = wt.Wq;
         o.Wscale = wt.Wscale;
+        o.wf = wt.wf;
         o.q_rows = d_out;
         o.q_cols = d_in;
     }
@@ -944,13 +967,13 @@ MainOperands main_operands(const Weight &wt, const void *A0, const void *A1, con
 lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, const uint16_t *B, uint16_t *h,
                        uint16_t *xa_save, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha, void *ws,
                        size_t ws_bytes, void *stream) {
-    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.q4()));
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.wf));
     if (!x || !wt.present() || !A || !B || !h) return LORA_ERR_INVALID_ARG;
     if (!aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(h) ||
         (xa_save && !aligned16(xa_save)))
         return LORA_ERR_MISALIGNED;
     Ctx c;
-    LORA_TRY(prepare(wt.q4() ? LORA_OP_FWD_Q4 : LORA_OP_FWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    LORA_TRY(prepare(wt.op_fwd(), M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(c.plan.side ? side_xa(c, x, A, sxa, M, d_in, r, s) : step_xa(c, x, A, sxa, M, d_in, r, s));
@@ -961,13 +984,13 @@ lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, c
 lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, const uint16_t *A,
                        const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB, int64_t M,
                        int64_t d_in, int64_t d_out, int r, float alpha, void *ws, size_t ws_bytes, void *stream) {
-    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.q4()));
+    LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.wf));
     if (!dY || !x || !wt.present() || !A || !B || !dA || !dB) return LORA_ERR_INVALID_ARG;
     if (!aligned16(dY) || !aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
         !aligned16(dB) || (xa_save && !aligned16(xa_save)) || (dX && !aligned16(dX)))
         return LORA_ERR_MISALIGNED;
     Ctx c;
-    LORA_TRY(prepare(wt.q4() ? LORA_OP_BWD_Q4 : LORA_OP_BWD, M, d_in, d_out, r, ws, ws_bytes, stream, &c));
+    LORA_TRY(prepare(wt.op_bwd(), M, d_in, d_out, r, ws, ws_bytes, stream, &c));
     const float s = alpha / static_cast<float>(r);
     const uint16_t *sxa = xa_save;
     if (!sxa) {
@@ -1014,8 +1037,9 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
 extern "C" {
 
 size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r) {
-    if (op < LORA_OP_FWD || op > LORA_OP_BWD_Q4) return 0;
-    if (check_shapes(M, d_in, d_out, r, 1.0f, op >= LORA_OP_FWD_Q4) != LORA_OK) return 0;
+    if (op < LORA_OP_FWD || op > LORA_OP_BWD_FP8) return 0;
+    const int wf = op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
+    if (check_shapes(M, d_in, d_out, r, 1.0f, wf) != LORA_OK) return 0;
     Plan pl;
     make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
     return pl.total;
@@ -1046,6 +1070,7 @@ lora_status_t lora_linear_fwd_q4(const uint16_t *x, const uint8_t *Wq, const uin
     Weight wt;
     wt.Wq = Wq;
     wt.Wscale = Wscale;
+    wt.wf = WF_Q4;
     if (!Wq || !Wscale) return LORA_ERR_INVALID_ARG;
     return fwd_impl(x, wt, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
 }
@@ -1057,7 +1082,33 @@ lora_status_t lora_linear_bwd_q4(const uint16_t *dY, const uint16_t *x, const ui
     Weight wt;
     wt.Wq = Wq;
     wt.Wscale = Wscale;
+    wt.wf = WF_Q4;
     if (!Wq || !Wscale) return LORA_ERR_INVALID_ARG;
+    return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                    stream);
+}
+
+lora_status_t lora_linear_fwd_fp8(const uint16_t *x, const uint8_t *W8, const uint16_t *W8scale, const uint16_t *A,
+                                  const uint16_t *B, uint16_t *h, uint16_t *xa_save, int64_t M, int64_t d_in,
+                                  int64_t d_out, int r, float alpha, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    Weight wt;
+    wt.Wq = W8;
+    wt.Wscale = W8scale;
+    wt.wf = WF_FP8;
+    if (!W8 || !W8scale) return LORA_ERR_INVALID_ARG;
+    return fwd_impl(x, wt, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
+}
+
+lora_status_t lora_linear_bwd_fp8(const uint16_t *dY, const uint16_t *x, const uint8_t *W8, const uint16_t *W8scale,
+                                  const uint16_t *A, const uint16_t *B, const uint16_t *xa_save, uint16_t *dX,
+                                  float *dA, float *dB, int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    Weight wt;
+    wt.Wq = W8;
+    wt.Wscale = W8scale;
+    wt.wf = WF_FP8;
+    if (!W8 || !W8scale) return LORA_ERR_INVALID_ARG;
     return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
                     stream);
 }

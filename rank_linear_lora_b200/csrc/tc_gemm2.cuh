@@ -13,11 +13,11 @@
 //   warps 2..5  epilogue in both CTAs: each drains its own 128 accumulator rows from
 //               TMEM, reports to the leader's accumulator-empty barrier, and stores
 //               bf16 through 128B-swizzled smem staging with TMA
-//   warps 6..   (4-bit frozen weight only) dequant warps in both CTAs, none on warp
-//               1's scheduler: fetch packed codes by TMA, decode them to bf16 straight
-//               into the B tile of the weight K segment and report to the leader's
-//               B-ready barrier; the producer then loads only A for those blocks (and
-//               A + B for the rank-r tail blocks, as in the bf16 case)
+//   warps 6..   (4-bit or FP8 frozen weight) dequant warps in both CTAs, none on warp
+//               1's scheduler: fetch the weight's codes by TMA, decode them to bf16
+//               straight into the B tile of the weight K segment and report to the
+//               leader's B-ready barrier; the producer then loads only A for those
+//               blocks (and A + B for the rank-r tail blocks, as in the bf16 case)
 //
 // Schedule: whole pair tiles in grouped raster order, `dp_waves` per cluster; a
 // partial last wave of `tail_tiles` tiles is cut along N into two 256 x 128 tiles,
@@ -43,7 +43,13 @@ constexpr int DQ_GROUP_WARPS = 4 / DQ_RUNS;               // warps decoding one 
 constexpr int DQ_GROUPS = DQ_WARPS / DQ_GROUP_WARPS;       // groups that take K blocks in turn
 constexpr int DQ_QDEPTH = 1;         // packed-code slots per dequant warp (own K blocks in flight)
 constexpr int DQ_QROWS = 32 * DQ_RUNS;                     // runs fetched per warp and K block
-constexpr int DQ_QSLOT = DQ_QROWS * 32;                    // one slot: DQ_QROWS runs x 32 bytes
+
+// Frozen-weight formats of the pair GEMM.
+enum WeightFmt { WF_BF16 = 0, WF_Q4 = 1, WF_FP8 = 2 };
+// Bytes of codes per run of 64 weights: two 4-bit codes per byte, or one E4M3 code per byte.
+__host__ __device__ constexpr int dq_run_bytes(int wf) { return wf == WF_FP8 ? 64 : 32; }
+// One packed-code slot of a dequant warp: DQ_QROWS runs.
+__host__ __device__ constexpr int dq_qslot(int wf) { return DQ_QROWS * dq_run_bytes(wf); }
 
 // A warp's scheduler (SM sub-partition) is its id mod 4.  The single-thread MMA issuer
 // (warp 1) must issue each tcgen05.mma as soon as the tensor core takes the previous one
@@ -63,16 +69,17 @@ __host__ __device__ constexpr int dq_index(int w) {
     return i;
 }
 
-template <bool B_MN, bool Q4, int STAGES>
+template <bool B_MN, int WF, int STAGES>
 struct PairCfg {
+    static constexpr bool DQ = WF != WF_BF16;         // the weight's B tiles are decoded in shared memory
     static constexpr int A_BYTES = 128 * BK * 2;      // 16 KB: this CTA's 128 rows of A
     static constexpr int B_BYTES = CTA_BN * BK * 2;   // 16 KB: this CTA's 128 rows of B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int Q_BYTES = Q4 ? DQ_WARPS * DQ_QDEPTH * DQ_QSLOT : 0;  // per-warp packed-code rings
+    static constexpr int Q_BYTES = DQ ? DQ_WARPS * DQ_QDEPTH * dq_qslot(WF) : 0;  // per-warp packed-code rings
     static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
     static constexpr int TMEM_COLS = 2 * PAIR_BN;     // two 256-column accumulators
-    static constexpr int BAR_BYTES = Q4 ? 1024 : 512;
-    static constexpr int THREADS = Q4 ? NUM_THREADS + 32 * dq_warp_span(DQ_WARPS) : NUM_THREADS;  // + dequant warps
+    static constexpr int BAR_BYTES = DQ ? 1024 : 512;
+    static constexpr int THREADS = DQ ? NUM_THREADS + 32 * dq_warp_span(DQ_WARPS) : NUM_THREADS;  // + dequant warps
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + Q_BYTES + EPI_BYTES + BAR_BYTES;
     static_assert(STAGES <= 32, "per-stage phase bits are kept in one 32-bit mask");
     static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
@@ -110,6 +117,34 @@ __device__ __forceinline__ uint4 q4_decode8(uint32_t word, uint64_t s7x2) {
     return r;
 }
 
+// Eight E4M3 codes (two 32-bit words, element i in byte i) to eight bf16 values
+// e4m3(q) * scale: each code pair converts exactly to f16x2, each half widens exactly to
+// fp32, the fp32 product with the bf16 scale is exact (4 + 8 significant bits), and the
+// conversion to bf16x2 is the one rounding.
+__device__ __forceinline__ uint32_t fp8_pair(uint32_t two_codes, float sc) {
+    uint32_t out;
+    asm("{\n\t.reg .b16 c;\n\t.reg .b32 h;\n\t.reg .b16 hl, hh;\n\t.reg .f32 fl, fh;\n\t"
+        "cvt.u16.u32 c, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, c;\n\t"
+        "mov.b32 {hl, hh}, h;\n\t"
+        "cvt.f32.f16 fl, hl;\n\t"
+        "cvt.f32.f16 fh, hh;\n\t"
+        "mul.rn.f32 fl, fl, %2;\n\t"
+        "mul.rn.f32 fh, fh, %2;\n\t"
+        "cvt.rn.bf16x2.f32 %0, fh, fl;\n\t}"
+        : "=r"(out)
+        : "r"(two_codes), "f"(sc));
+    return out;
+}
+__device__ __forceinline__ uint4 fp8_decode8(uint32_t w0, uint32_t w1, float sc) {
+    uint4 r;
+    r.x = fp8_pair(w0 & 0xFFFFu, sc);
+    r.y = fp8_pair(w0 >> 16, sc);
+    r.z = fp8_pair(w1 & 0xFFFFu, sc);
+    r.w = fp8_pair(w1 >> 16, sc);
+    return r;
+}
+
 // Item i of this cluster: pair tile (m, n), its first output column and width split.
 __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, int n_clusters, int i, WorkItem &w) {
     w.kb_lo = 0;
@@ -133,15 +168,17 @@ __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, in
     return false;
 }
 
-template <bool B_MN, bool Q4, int STAGES>
-__global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
+template <bool B_MN, int WF, int STAGES>
+__global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
     k_tc_gemm_pair(const __grid_constant__ GemmArgs p) {
-    using Cfg = PairCfg<B_MN, Q4, STAGES>;
+    using Cfg = PairCfg<B_MN, WF, STAGES>;
+    constexpr bool DQ = Cfg::DQ;  // the weight's B tiles are decoded (4-bit or FP8 codes)
+    constexpr int QSLOT = dq_qslot(WF);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = smem + STAGES * Cfg::A_BYTES;
-    uint8_t *sQ = smem + STAGES * Cfg::STAGE_BYTES;  // Q4: packed-code rings of the dequant warps
+    uint8_t *sQ = smem + STAGES * Cfg::STAGE_BYTES;  // decoded weight: packed-code rings of the dequant warps
     uint8_t *sEpi = sQ + Cfg::Q_BYTES;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sEpi + Cfg::EPI_BYTES);
     uint64_t *full_bar = bars;                    // [STAGES] (leader's counts the pair's A (and B) bytes)
@@ -149,12 +186,12 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
     uint64_t *tfull_bar = bars + 2 * STAGES;      // [2]
     uint64_t *tempty_bar = bars + 2 * STAGES + 2; // [2] (leader's: 8 epilogue warps of the pair)
     uint64_t *drain_bar = bars + 2 * STAGES + 4;  // [1]
-    uint64_t *bready_bar = bars + 2 * STAGES + 5; // [STAGES] Q4, leader: both CTAs' decoded B tiles written
+    uint64_t *bready_bar = bars + 2 * STAGES + 5; // [STAGES] DQ, leader: both CTAs' decoded B tiles written
     uint64_t *qfull_bar = bars + 3 * STAGES + 5;  // [DQ_WARPS][DQ_QDEPTH] Q4: a warp's packed codes landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qfull_bar + (Q4 ? DQ_WARPS * DQ_QDEPTH : 0));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(qfull_bar + (DQ ? DQ_WARPS * DQ_QDEPTH : 0));
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 3);  // [2]
-    // Q4: K blocks (in the CTA's sequence) whose stage the producer has seen released by
+    // decoded weight: K blocks (in the CTA's sequence) whose stage the producer has seen released by
     // the MMA, i.e. whose B tile the dequant warps may write.  A monotonic count: the
     // dequant groups run ahead of the MMA by different amounts, so a parity wait on the
     // stage's empty barrier could match a later phase than the one meant.
@@ -184,7 +221,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             mbar_init(smem_u32(&tempty_bar[b]), 8);
         }
         mbar_init(smem_u32(drain_bar), 1);
-        if (Q4) {
+        if (DQ) {
             for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * DQ_GROUP_WARPS);
             for (int q = 0; q < DQ_WARPS * DQ_QDEPTH; ++q) mbar_init(smem_u32(&qfull_bar[q]), 1);
         }
@@ -193,7 +230,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        if (Q4) tma_prefetch_desc(&p.tmQ);
+        if (DQ) tma_prefetch_desc(&p.tmQ);
         tma_prefetch_desc(&p.tmA0);
         tma_prefetch_desc(&p.tmB0);
         if (p.kb1 > 0) {
@@ -233,10 +270,10 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 const int a_row = w.m * PAIR_BM + static_cast<int>(rank) * 128;
                 const int b_row = w.col0 + static_cast<int>(rank) * bn_cta;
                 for (int kb = w.kb_lo; kb < w.kb_hi; ++kb) {
-                    // Q4: the weight segment's B tiles are written by the dequant warps, so the
+                    // decoded weight: the weight segment's B tiles are written by the dequant warps, so the
                     // leader's full barrier then counts A only; rank-r tail B tiles come by TMA.
                     const bool seg1 = kb >= p.kb0;
-                    const bool b_tma = !Q4 || seg1;
+                    const bool b_tma = !DQ || seg1;
                     const uint32_t tx = 2u * static_cast<uint32_t>(Cfg::A_BYTES + (b_tma ? bn_cta * BK * 2 : 0));
                     const uint64_t tw = trace ? globaltimer_ns() : 0;
                     if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1u, abort_flag, p.err,
@@ -245,7 +282,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                         break;
                     }
                     if (trace) wait_empty_ns += globaltimer_ns() - tw;
-                    if (Q4) st_release_shared(smem_u32(bfree), ++flat);
+                    if (DQ) st_release_shared(smem_u32(bfree), ++flat);
                     const uint32_t fb_local = smem_u32(&full_bar[stage]);
                     const uint32_t fb_leader = mapa_shared(fb_local, 0);
                     if (leader) {
@@ -306,7 +343,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             bool ok = true;
             uint64_t wait_tempty_ns = 0, kblocks = 0;
             long long wait_a_cyc = 0, wait_b_cyc = 0;
-            uint32_t bready_phase = 0;  // Q4: bit s = parity of the next B-ready completion of stage s
+            uint32_t bready_phase = 0;  // decoded weight: bit s = parity of the next B-ready completion of stage s
             WorkItem w;
             for (; ok && get_pair_item(p, cluster, n_clusters, it, w); ++it) {
                 const int buf = it & 1;
@@ -332,7 +369,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                         }
                         if (trace) wait_a_cyc += clock64() - c0;
                     }
-                    if (Q4 && kb < p.kb0) {
+                    if (DQ && kb < p.kb0) {
                         // B-ready completes only for weight K blocks (rank-r tail blocks come
                         // by TMA), so its phase per stage is tracked apart from the ring's.
                         const uint32_t rb = smem_u32(&bready_bar[stage]);
@@ -382,10 +419,10 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
                 trace[TR_MMA_WAIT_B] = static_cast<unsigned long long>(wait_b_cyc);
             }
         }
-    } else if (Q4 && warp >= 6 && dq_idle_warp(warp)) {
+    } else if (DQ && warp >= 6 && dq_idle_warp(warp)) {
         // idle: keeps the MMA issuer's sub-partition free of decode work
-    } else if (Q4 && warp >= 6) {
-        // ------------------------------------------------------------ dequant warps (both CTAs, Q4)
+    } else if (DQ && warp >= 6) {
+        // ------------------------------------------------------------ dequant warps (both CTAs, 4-bit or FP8 weight)
         // The weight segment's B tiles are decoded here from 4-bit codes.  Warps form
         // DQ_GROUPS groups of DQ_GROUP_WARPS; group g takes the weight K blocks g,
         // g + DQ_GROUPS, ... of the CTA's sequence (the rank-r tail blocks come by TMA and
@@ -403,7 +440,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
         const int dw = dq_index(warp);                       // dequant warp 0 .. DQ_WARPS-1
         const int grp = dw / DQ_GROUP_WARPS, wg = dw % DQ_GROUP_WARPS;
         const int r0 = wg * DQ_QROWS;                  // the warp's first run; lane owns r0 + lane + 32 i
-        uint8_t *qring = sQ + dw * (DQ_QDEPTH * DQ_QSLOT);
+        uint8_t *qring = sQ + dw * (DQ_QDEPTH * QSLOT);
         uint64_t *qbar = qfull_bar + dw * DQ_QDEPTH;
         const uint32_t bready_leader0 = mapa_shared(smem_u32(&bready_bar[0]), 0);
         const int kb_all = p.kb0 + p.kb1;
@@ -439,12 +476,13 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
         // Lane 0: TMA of this warp's DQ_QROWS runs of own block c.j into slot c.j % DQ_QDEPTH.
         auto issue = [&](const Cursor &c) {
             const uint32_t bar = smem_u32(&qbar[c.j % DQ_QDEPTH]);
-            const uint32_t dst = smem_u32(qring + (c.j % DQ_QDEPTH) * DQ_QSLOT);
-            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(DQ_QSLOT));
+            const uint32_t dst = smem_u32(qring + (c.j % DQ_QDEPTH) * QSLOT);
+            mbar_arrive_expect_tx(bar, static_cast<uint32_t>(QSLOT));
+            constexpr int RB = dq_run_bytes(WF);  // bytes of codes per 64 weights
             if (B_MN)  // K rows kb*64 + (r0 % 64) .., bytes of d_in columns b_row + 64*(r0 / 64) ..
-                tma_load_2d(dst, &p.tmQ, bar, c.b_row / 2 + 32 * (r0 >> 6), c.kb * BK + (r0 & 63));
+                tma_load_2d(dst, &p.tmQ, bar, (c.b_row + 64 * (r0 >> 6)) * RB / 64, c.kb * BK + (r0 & 63));
             else       // weight rows b_row + r0 .., bytes of K columns kb*64 ..
-                tma_load_2d(dst, &p.tmQ, bar, c.kb * (BK / 2), c.b_row + r0);
+                tma_load_2d(dst, &p.tmQ, bar, c.kb * RB, c.b_row + r0);
         };
         // Raw bf16 bits of the group scale of this thread's run i in own block c.j (0
         // outside the weight).  K-major: weight row rn; MN-major: K row rn, chunk jc.
@@ -453,7 +491,8 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             const int rn = B_MN ? (run & 63) : run, jc = B_MN ? (run >> 6) : 0;
             if (!c.valid) return 0u;
             const int srow = B_MN ? c.kb * BK + rn : c.b_row + rn;
-            const int scol = B_MN ? (c.b_row + 64 * jc) / 64 : c.kb;
+            // 4-bit: one scale per 64 weights of a row; FP8: one per row
+            const int scol = WF == WF_FP8 ? 0 : B_MN ? (c.b_row + 64 * jc) / 64 : c.kb;
             if (srow >= p.scale_rows || scol >= p.scale_ld) return 0u;
             return static_cast<uint32_t>(__ldg(p.wscale + static_cast<int64_t>(srow) * p.scale_ld + scol));
         };
@@ -495,16 +534,28 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
             for (int i = 0; i < DQ_RUNS; ++i) {
                 const int run = r0 + lane + 32 * i;
                 const int rn = B_MN ? (run & 63) : run, jc = B_MN ? (run >> 6) : 0;
-                const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * DQ_QSLOT + (lane + 32 * i) * 32);
-                const uint4 v0 = src[0], v1 = src[1];
-                const float s7 = __uint_as_float(sc[i] << 16) / 7.0f;
-                const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
+                const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * QSLOT +
+                                                                   (lane + 32 * i) * dq_run_bytes(WF));
                 uint8_t *row =
                     sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
-                const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                if constexpr (WF == WF_FP8) {
+                    // 64 codes: 16-byte chunk c of the bf16 row holds codes 8c .. 8c+7
+                    const float sc_f = __uint_as_float(sc[i] << 16);
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = q4_decode8(wds[c], s7x2);
+                    for (int h = 0; h < 4; ++h) {
+                        const uint4 v = src[h];
+                        *reinterpret_cast<uint4 *>(row + (((2 * h) ^ (rn & 7)) * 16)) = fp8_decode8(v.x, v.y, sc_f);
+                        *reinterpret_cast<uint4 *>(row + (((2 * h + 1) ^ (rn & 7)) * 16)) = fp8_decode8(v.z, v.w, sc_f);
+                    }
+                } else {
+                    const uint4 v0 = src[0], v1 = src[1];
+                    const float s7 = __uint_as_float(sc[i] << 16) / 7.0f;
+                    const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
+                    const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = q4_decode8(wds[c], s7x2);
+                }
             }
             // Orders the B-tile stores (and this slot's code reads, whose values are used
             // above) before the tensor core's reads and the slot's next TMA write.
@@ -572,7 +623,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, Q4, STAGES>::THREADS, 1)
 #pragma unroll 1
             for (int ch = 0; ch < nch; ++ch) {
                 uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
-                if (Q4) {
+                if (DQ) {
                     // 32 columns at a time: the dequant warps leave fewer registers per thread
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();

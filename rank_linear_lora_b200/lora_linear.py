@@ -21,7 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lora_linear.h")
 LORA_OK = 0
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_MISALIGNED", 3: "LORA_ERR_UNSUPPORTED",
           4: "LORA_ERR_WORKSPACE", 5: "LORA_ERR_CUDA", 6: "LORA_ERR_TIMEOUT"}
-OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4 = 0, 1, 2, 3
+OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4, OP_FWD_FP8, OP_BWD_FP8 = 0, 1, 2, 3, 4, 5
 KERNEL_KINDS = ["xa", "fwd_main", "g", "dx_main", "dadb"]
 
 
@@ -49,7 +49,10 @@ def load_library():
     lib.lora_linear_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     lib.lora_linear_fwd_q4.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     lib.lora_linear_bwd_q4.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
-    for f in ("lora_linear_fwd", "lora_linear_bwd", "lora_linear_fwd_q4", "lora_linear_bwd_q4"):
+    lib.lora_linear_fwd_fp8.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_bwd_fp8.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    for f in ("lora_linear_fwd", "lora_linear_bwd", "lora_linear_fwd_q4", "lora_linear_bwd_q4", "lora_linear_fwd_fp8",
+              "lora_linear_bwd_fp8"):
         getattr(lib, f).restype = I
     lib.lora_linear_check.argtypes = [P, P]
     lib.lora_linear_check.restype = I
@@ -205,6 +208,47 @@ def lora_linear_bwd_q4(dY, x, Wq, Wscale, A, B, xa_save, dX, dA, dB, alpha, ws, 
                                            _ptr(xa_save), _ptr(dX), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
                                            float(alpha), *_ws(ws), _stream(stream))
     _check(st, "lora_linear_bwd_q4")
+
+
+def _fp8(W8, W8scale, d_out, d_in):
+    if W8.dtype != torch.uint8 or not W8.is_cuda or not W8.is_contiguous() or tuple(W8.shape) != (d_out, d_in):
+        raise ValueError(f"W8: expected a contiguous CUDA uint8 tensor of shape {(d_out, d_in)} (E4M3 codes)")
+    _on_current_device(W8, "W8")
+    _bf16(W8scale, "W8scale", (d_out,))
+
+
+def lora_linear_fwd_fp8(x, W8, W8scale, A, B, h, xa_save, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = W8.shape[0]
+    _fp8(W8, W8scale, d_out, d_in)
+    for t, n, s in ((x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (h, "h", (M, d_out))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    st = load_library().lora_linear_fwd_fp8(_ptr(x), _ptr(W8), _ptr(W8scale), _ptr(A), _ptr(B), _ptr(h),
+                                            _ptr(xa_save), M, d_in, d_out, r, float(alpha), *_ws(ws),
+                                            _stream(stream))
+    _check(st, "lora_linear_fwd_fp8")
+
+
+def lora_linear_bwd_fp8(dY, x, W8, W8scale, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = W8.shape[0]
+    _fp8(W8, W8scale, d_out, d_in)
+    for t, n, s in ((dY, "dY", (M, d_out)), (x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    if dX is not None:
+        _bf16(dX, "dX", (M, d_in))
+    _f32(dA, "dA", (r, d_in))
+    _f32(dB, "dB", (d_out, r))
+    st = load_library().lora_linear_bwd_fp8(_ptr(dY), _ptr(x), _ptr(W8), _ptr(W8scale), _ptr(A), _ptr(B),
+                                            _ptr(xa_save), _ptr(dX), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
+                                            float(alpha), *_ws(ws), _stream(stream))
+    _check(st, "lora_linear_bwd_fp8")
 
 
 def lora_linear_check(ws, stream=None):

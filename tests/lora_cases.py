@@ -40,9 +40,12 @@ class DeviceLayer:
         self.spec, self.inp = sp, inp
         self.x, self.A, self.B, self.dY = (dev_bf16(a) for a in (inp.x, inp.A, inp.B, inp.dY))
         self.q4 = sp.q4
+        self.fp8 = getattr(sp, "fp8", False)
+        self.W = None
         if sp.q4:
             self.Wq, self.Wscale = dev_u8(inp.Wq), dev_bf16(inp.Wscale)
-            self.W = None
+        elif self.fp8:
+            self.W8, self.W8scale = dev_u8(inp.W8), dev_bf16(inp.W8scale)
         else:
             self.W = dev_bf16(inp.W)
         M, di, do, r = sp.M, sp.d_in, sp.d_out, sp.r
@@ -51,7 +54,8 @@ class DeviceLayer:
         self.dX = torch.empty(M, di, dtype=torch.bfloat16, device="cuda")
         self.dA = torch.empty(r, di, dtype=torch.float32, device="cuda")
         self.dB = torch.empty(do, r, dtype=torch.float32, device="cuda")
-        fop, bop = (L.OP_FWD_Q4, L.OP_BWD_Q4) if sp.q4 else (L.OP_FWD, L.OP_BWD)
+        fop, bop = ((L.OP_FWD_Q4, L.OP_BWD_Q4) if sp.q4 else (L.OP_FWD_FP8, L.OP_BWD_FP8) if self.fp8
+                    else (L.OP_FWD, L.OP_BWD))
         self.ws_f = L.workspace(fop, M, di, do, r)
         self.ws_b = L.workspace(bop, M, di, do, r)
 
@@ -59,6 +63,9 @@ class DeviceLayer:
         xa = self.xa if save_xa else None
         if self.q4:
             L.lora_linear_fwd_q4(self.x, self.Wq, self.Wscale, self.A, self.B, self.h, xa, self.spec.alpha, self.ws_f)
+        elif self.fp8:
+            L.lora_linear_fwd_fp8(self.x, self.W8, self.W8scale, self.A, self.B, self.h, xa, self.spec.alpha,
+                                  self.ws_f)
         else:
             L.lora_linear_fwd(self.x, self.W, self.A, self.B, self.h, xa, self.spec.alpha, self.ws_f)
 
@@ -68,6 +75,9 @@ class DeviceLayer:
         if self.q4:
             L.lora_linear_bwd_q4(self.dY, self.x, self.Wq, self.Wscale, self.A, self.B, xa, dX, self.dA, self.dB,
                                  self.spec.alpha, self.ws_b)
+        elif self.fp8:
+            L.lora_linear_bwd_fp8(self.dY, self.x, self.W8, self.W8scale, self.A, self.B, xa, dX, self.dA, self.dB,
+                                  self.spec.alpha, self.ws_b)
         else:
             L.lora_linear_bwd(self.dY, self.x, self.W, self.A, self.B, xa, dX, self.dA, self.dB, self.spec.alpha,
                               self.ws_b)
@@ -150,7 +160,8 @@ def check_projections(dl: "DeviceLayer", inp: inputs.LayerInputs, ref: dict, see
     sp = inp.spec
     rng = np.random.default_rng(0xC0DE + seed)
     M, di, do = sp.M, sp.d_in, sp.d_out
-    wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W=inp.W)
+    wkw = (dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W8=inp.W8, W8scale=inp.W8scale)
+           if getattr(sp, "fp8", False) else dict(W=inp.W))
     u = rng.choice([-1.0, 1.0], M)
     v_h = rng.choice([-1.0, 1.0], do)
     v_x = rng.choice([-1.0, 1.0], di)
@@ -210,7 +221,7 @@ class ErrorTally:
         if rms_tol is not None and self.sq_ref > 0:
             rms = np.sqrt(self.sq_err / self.sq_ref)
             assert rms <= rms_tol, f"{self.name}: rms rel err {rms:.3e} > {rms_tol:.1e}"
-        return self.max_err / bound
+        return self.max_err / bound if bound > 0 else 0.0  # a zero bound (exactly-zero reference) passed exactly
 
 
 def compare_every_element(dl: "DeviceLayer", inp: inputs.LayerInputs, block_rows: int = 1024) -> dict:

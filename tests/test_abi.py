@@ -113,3 +113,29 @@ def test_merge_argument_checks(lib):
     assert q(sc=None) == 1                            # the scales are required
     assert q(di=96) == 1                              # 4-bit weight: d_in % 64 == 0
     assert q(sc=0x5002) == 2 and q(Wq=0x1008) == 2
+
+
+def test_fp8_validation_before_any_device_work(lib):
+    """The FP8 entry points: workspace sizes for their ops, and argument checks (codes
+    and scales required, 16-byte aligned, d_in % 16 == 0) before any launch."""
+    assert {"lora_linear_fwd_fp8", "lora_linear_bwd_fp8"} <= set(L.declared_functions())
+    for op in (L.OP_FWD_FP8, L.OP_BWD_FP8):
+        assert L.lora_linear_workspace_size(op, 4096, 4096, 4096, 8) == L.lora_linear_workspace_size(
+            op - 4, 4096, 4096, 4096, 8)  # the workspace does not depend on the weight's format
+    assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1040, 256, 8) > 0      # d_in % 16 == 0 suffices
+    assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1032, 256, 8) == 0     # d_in % 16 != 0
+    assert L.lora_linear_workspace_size(6, 64, 256, 256, 8) == 0
+    P = ctypes.c_void_p
+    fn = lib.lora_linear_fwd_fp8
+
+    def fwd(W8=0x2000, Ws=0x2800, di=256, x=0x1000):
+        return fn(P(x), P(W8), P(Ws), P(0x3000), P(0x4000), P(0x5000), None, 64, di, 256, 8, 16.0, P(0x10000),
+                  1 << 30, None)
+    assert fwd(W8=None) == 1
+    assert fwd(Ws=None) == 1
+    assert fwd(di=264) == 1        # not a multiple of 16
+    assert fwd(W8=0x2004) == 2
+    assert fwd(Ws=0x2808) == 2
+    st = lib.lora_linear_bwd_fp8(P(0x1000), P(0x1000), P(0x2000), P(0x2800), P(0x3000), P(0x4000), None, None,
+                                 None, P(0x7000), 64, 256, 256, 8, 16.0, P(0x10000), 1 << 30, None)
+    assert st == 1  # dA is required

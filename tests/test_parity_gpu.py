@@ -345,3 +345,40 @@ def test_split_k_side_products_for_narrow_ranks(shape, monkeypatch):
     spec = inputs.LayerSpec("splitk", M, di, do, r, alpha=2.0 * r, seed=0x5B1 + M)
     inp, dl = _run_full(spec)
     compare_every_element(dl, inp)
+
+
+# FP8 (E4M3) frozen weight with one bf16 scale per row, decoded in shared memory inside
+# both main GEMMs: every element against the oracle's weight format 2.
+FP8_SHAPES = [
+    (200, 320, 200, 16),     # ragged M and d_out
+    (520, 512, 768, 24),     # rank tail r % 16 != 0
+    (129, 1040, 1536, 8),    # d_in % 64 != 0 (a partial last K block of codes)
+    (1100, 640, 4000, 16),   # forward: 5 x 16 tiles, several work items per CTA pair
+    (1100, 4096, 1000, 16),  # dX: 5 x 16 tiles, K = d_out ragged
+]
+
+
+@pytest.mark.parametrize("shape", FP8_SHAPES, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_fp8_every_element(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("fp8", M, di, do, r, alpha=2.0 * r, fp8=True, seed=0xF8 + M)
+    inp, dl = _run_full(spec)
+    compare_every_element(dl, inp)
+
+
+def test_fp8_code_order_dominant_weight():
+    """B = 0, so h and dX are the decoded weight's products alone: any swapped code
+    pair, wrong scale row or chunk order shows far outside the bound."""
+    spec = inputs.LayerSpec("fp8w", 256, 192, 320, 8, alpha=16.0, fp8=True, seed=0xF9)
+    inp, dl = _run_full(spec, zero_B=True)
+    compare_every_element(dl, inp)
+
+
+@pytest.mark.parametrize("idx", [1, 4], ids=["attn_proj", "up_proj"])
+def test_fp8_full_size_every_element(idx):
+    """The attention projection and the up projection's sizes with the FP8 weight."""
+    spec = inputs.workload(idx).layers[0].with_(q4=False, fp8=True)
+    inp, dl = _run_full(spec)
+    res = compare_every_element(dl, inp)
+    print(f"{spec.name} fp8: {res['elements']} elements, oracle {res['oracle_s']:.1f} s; worst error / bound "
+          + ", ".join(f"{k} {v:.3f}" for k, v in res["worst"].items()))
