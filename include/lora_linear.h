@@ -94,6 +94,46 @@ typedef enum {
     LORA_OP_BWD_FP8 = 5
 } lora_op_t;
 
+/*
+ * Plans.  How a layer of a given shape splits its work: which kernels compute the
+ * rank-r side products, how their CTAs are grouped, and how the main GEMMs end their
+ * last wave.  The library chooses a plan per shape from fixed rules and a streaming
+ * cost model; lora_linear_set_plan overrides any part of it for one shape, which is
+ * how a tuner that times candidate plans on the device installs its choice (page
+ * "UnSloth加速库集成：编译级优化带来的性能飞跃", section 技术三: probe the kernel
+ * configuration per GPU, sequence length and rank, and cache the result).  Every
+ * plan computes the same function; results differ only in the order of fp32 sums.
+ * A field of 0 means "the library's choice".
+ */
+typedef struct {
+    int32_t side_fwd;   /* s.xa: 1 the cluster-reduction side kernel (r <= 64), 2 the split-K kernel */
+    int32_t side_bwd;   /* s.g with dB, then dA: 1 the side kernels (one pass over dY; r <= 32),
+                           2 the split-K kernels (s.g, then dB and dA in one launch) */
+    int32_t xa_cluster; /* side s.xa: CTAs per cluster, 1, 2 or 4 (they split d_in) */
+    int32_t g_cluster;  /* side s.g + dB: CTAs per cluster, 1, 2 or 4 (they split d_out) */
+    int32_t g_group;    /* side s.g + dB: 128-token blocks per round, 1..6, with g_group * r <= 64 */
+    int32_t da_cluster; /* side dA: CTAs per cluster, 1 or 2 (they split the tokens) */
+    int32_t fwd_tail;   /* forward main GEMM: 1 a partial last wave is cut along N, 2 it is not */
+    int32_t dx_overlap; /* backward: 1 dA (and dB) start beside the dX GEMM's last wave, whose tiles
+                           stay whole; 2 they follow the dX GEMM, whose last wave is cut along N */
+    int32_t splitk[4];  /* split-K kernels: K splits (1 .. 64) of s.xa, s.g, dB and dA */
+} lora_plan_t;
+
+/* Install `plan` for every operation on layers of exactly this shape (M, d_in, d_out,
+ * r), replacing any earlier one; NULL removes it.  Fields out of range, or a side kernel
+ * asked for a rank it does not take, give LORA_ERR_INVALID_ARG / LORA_ERR_UNSUPPORTED
+ * and change nothing.  The workspace size follows the plan: call
+ * lora_linear_workspace_size again after changing it.  Host-only and thread-safe (at
+ * most 256 shapes hold a plan); takes effect for calls made after it returns. */
+LORA_API lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r, const lora_plan_t *plan);
+
+/* The plan `op` uses for this shape: the override's fields and the library's choice for
+ * the rest, filled in for the kernels the plan runs (fields of kernels it does not run,
+ * e.g. the split-K splits when the side kernels take the products, are 0).  Host-only;
+ * LORA_ERR_INVALID_ARG for invalid sizes or op. */
+LORA_API lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r,
+                                            lora_plan_t *plan);
+
 /* Bytes of workspace the given operation needs for these sizes (0 if the sizes are
  * invalid).  Pure host function; needs no device. */
 LORA_API size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r);

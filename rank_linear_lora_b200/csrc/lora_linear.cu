@@ -467,10 +467,11 @@ constexpr int SIDE_MAX_C_DA = 2;
 
 // One output block per round; C the largest power of two <= max_c that keeps one round
 // of every output block within `sms` CTAs and gives each CTA some reduction work.
-SidePlan side_plan(int64_t n_out, int64_t n_red, int sms, int max_c) {
+SidePlan side_plan(int64_t n_out, int64_t n_red, int sms, int max_c, int force_c = 0) {
     SidePlan sp;
     int C = 1;
     while (C < max_c && n_out * 2 * C <= sms && 2 * C <= n_red) C *= 2;
+    if (force_c > 0) C = force_c;
     sp.C = C;
     sp.n_out = static_cast<int>(n_out);
     sp.n_red = static_cast<int>(n_red);
@@ -495,13 +496,15 @@ double side_stream_us(double bytes_per_cta, int ctas) {
 // stay in tensor memory while the round's CTAs sweep d_out), C CTAs split d_out.  Each
 // round leaves one fp32 dB partial [d_out, r]; the choice weighs the streaming time of
 // the busiest CTA against writing those partials.
-SidePlan side_plan_gdb(int64_t M, int64_t d_out, int r, int sms) {
+SidePlan side_plan_gdb(int64_t M, int64_t d_out, int r, int sms, int force_c = 0, int force_a = 0) {
     const int64_t n_out = cdiv(M, BM), n_red = cdiv(d_out, 128);
     SidePlan best;
     double best_cost = 1e300;
     for (int a = 1; a <= 6; ++a) {
         if (static_cast<int64_t>(a) * 128 * r * 4 > SIDE_RED_BYTES) break;  // the round's partials fit
-        for (int C = 1; C <= SIDE_MAX_C && C <= n_red; C *= 2) {
+        if (force_a > 0 && a != force_a) continue;
+        for (int C = 1; C <= SIDE_MAX_C; C *= 2) {
+            if (force_c > 0 ? C != force_c : C > n_red) continue;
             const int64_t need = cdiv(n_out, a);
             const int64_t clusters = std::min<int64_t>(need, sms / C);
             if (clusters < 1) continue;
@@ -538,27 +541,63 @@ struct Plan {
     bool side = false;          // s.xa on the side kernels (r <= 64)
     bool side_bwd = false;      // s.g + dB and dA on the side kernels (r <= 32)
     SidePlan sx, sg, sd;        // s.xa, s.g + dB partials, dA + dB
+    bool fwd_tail = true;       // forward main GEMM: cut a partial last wave along N
+    bool dx_overlap = true;     // dA (and dB) beside the dX GEMM's last wave
 };
+
+// ------------------------------------------------------------------ plan overrides
+struct PlanOverride {
+    int64_t M, d_in, d_out;
+    int r;
+    lora_plan_t p;
+};
+std::mutex g_plan_mu;
+std::vector<PlanOverride> g_overrides;
+constexpr size_t MAX_OVERRIDES = 256;
+
+bool find_override(int64_t M, int64_t d_in, int64_t d_out, int r, lora_plan_t *out) {
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    for (const PlanOverride &o : g_overrides)
+        if (o.M == M && o.d_in == d_in && o.d_out == d_out && o.r == r) {
+            *out = o.p;
+            return true;
+        }
+    return false;
+}
+
+// Split of kb K blocks into `splits` (as even as whole blocks allow).
+Split forced_split(int64_t kb, int splits) {
+    Split sp;
+    const int64_t per = cdiv(kb, std::min<int64_t>(splits, kb));
+    sp.per = static_cast<int>(per);
+    sp.splits = static_cast<int>(cdiv(kb, per));
+    return sp;
+}
 
 bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, Plan *pl) {
     const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8);
     const int64_t mt_tok = cdiv(M, BM), mt_in = cdiv(d_in, BM), mt_out = cdiv(d_out, BM);
+    lora_plan_t ov;
+    std::memset(&ov, 0, sizeof(ov));
+    find_override(M, d_in, d_out, r, &ov);  // all zero (the library's choice) without one
     size_t off = 0;
     pl->err = off;
     off += 256;
-    pl->side = r <= SIDE_MAX_R && side_enabled();
-    pl->side_bwd = bwd && r <= SIDE_MAX_R_BWD && side_enabled();
+    pl->side = ov.side_fwd ? ov.side_fwd == 1 : (r <= SIDE_MAX_R && side_enabled());
+    pl->side_bwd = bwd && (ov.side_bwd ? ov.side_bwd == 1 : (r <= SIDE_MAX_R_BWD && side_enabled()));
+    pl->fwd_tail = ov.fwd_tail != 2;
+    pl->dx_overlap = ov.dx_overlap != 2;
     // split-K counters and partials (every s.xa when not on the side kernels; the
     // backward's s.g, dB and dA when not on the side kernels)
     const bool sk_xa = !pl->side, sk_bwd = bwd && !pl->side_bwd;
-    pl->s_xa = choose_split(mt_tok, cdiv(d_in, BK), sms);
-    pl->s_g = choose_split(mt_tok, cdiv(d_out, BK), sms);
-    pl->s_db = choose_split(mt_out, cdiv(M, BK), sms);
-    pl->s_da = choose_split(mt_in, cdiv(M, BK), sms);
-    if (pl->side) pl->sx = side_plan(mt_tok, cdiv(d_in, BK), sms, SIDE_MAX_C);
+    pl->s_xa = ov.splitk[0] ? forced_split(cdiv(d_in, BK), ov.splitk[0]) : choose_split(mt_tok, cdiv(d_in, BK), sms);
+    pl->s_g = ov.splitk[1] ? forced_split(cdiv(d_out, BK), ov.splitk[1]) : choose_split(mt_tok, cdiv(d_out, BK), sms);
+    pl->s_db = ov.splitk[2] ? forced_split(cdiv(M, BK), ov.splitk[2]) : choose_split(mt_out, cdiv(M, BK), sms);
+    pl->s_da = ov.splitk[3] ? forced_split(cdiv(M, BK), ov.splitk[3]) : choose_split(mt_in, cdiv(M, BK), sms);
+    if (pl->side) pl->sx = side_plan(mt_tok, cdiv(d_in, BK), sms, SIDE_MAX_C, ov.xa_cluster);
     if (pl->side_bwd) {
-        pl->sg = side_plan_gdb(M, d_out, r, sms);
-        pl->sd = side_plan(mt_in, mt_tok, sms, SIDE_MAX_C_DA);
+        pl->sg = side_plan_gdb(M, d_out, r, sms, ov.g_cluster, ov.g_group);
+        pl->sd = side_plan(mt_in, mt_tok, sms, SIDE_MAX_C_DA, ov.da_cluster);
     }
     pl->ctr = off;
     pl->n_ctr = (sk_xa || sk_bwd) ? mt_tok * 2 + mt_in + mt_out : 0;
@@ -978,7 +1017,7 @@ lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, c
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(c.plan.side ? side_xa(c, x, A, sxa, M, d_in, r, s) : step_xa(c, x, A, sxa, M, d_in, r, s));
     const MainOperands o = main_operands(wt, x, sxa, B, h, d_out, d_in);
-    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, true);
+    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, c.plan.fwd_tail);
 }
 
 lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, const uint16_t *A,
@@ -1007,7 +1046,7 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
     // dependent launch), they start on the SMs its last wave leaves idle and wait for
     // it only before they exit.  The dX tail is then left whole (no narrow tiles) so
     // those SMs free up early.
-    const bool overlap = dX != nullptr && pdl_enabled();
+    const bool overlap = dX != nullptr && pdl_enabled() && c.plan.dx_overlap;
     int idle = 0;
     if (dX) {
         // W [d_out, d_in] (or its codes) and A [r, d_in] are read MN-major (d_in contiguous).
@@ -1111,6 +1150,65 @@ lora_status_t lora_linear_bwd_fp8(const uint16_t *dY, const uint16_t *x, const u
     if (!W8 || !W8scale) return LORA_ERR_INVALID_ARG;
     return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
                     stream);
+}
+
+lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r, const lora_plan_t *plan) {
+    if (check_shapes(M, d_in, d_out, r, 1.0f, WF_BF16) != LORA_OK) return LORA_ERR_INVALID_ARG;
+    if (plan) {
+        const lora_plan_t &q = *plan;
+        auto in = [](int32_t v, std::initializer_list<int32_t> ok) {
+            for (int32_t o : ok)
+                if (v == o) return true;
+            return false;
+        };
+        if (!in(q.side_fwd, {0, 1, 2}) || !in(q.side_bwd, {0, 1, 2}) || !in(q.xa_cluster, {0, 1, 2, 4}) ||
+            !in(q.g_cluster, {0, 1, 2, 4}) || q.g_group < 0 || q.g_group > 6 || !in(q.da_cluster, {0, 1, 2}) ||
+            !in(q.fwd_tail, {0, 1, 2}) || !in(q.dx_overlap, {0, 1, 2}))
+            return LORA_ERR_INVALID_ARG;
+        for (int i = 0; i < 4; ++i)
+            if (q.splitk[i] < 0 || q.splitk[i] > 64) return LORA_ERR_INVALID_ARG;
+        if (q.side_fwd == 1 && r > SIDE_MAX_R) return LORA_ERR_UNSUPPORTED;
+        if (q.side_bwd == 1 && r > SIDE_MAX_R_BWD) return LORA_ERR_UNSUPPORTED;
+        if (q.g_group > 0 && q.g_group * r > SIDE_RED_BYTES / (128 * 4)) return LORA_ERR_UNSUPPORTED;
+    }
+    std::lock_guard<std::mutex> lk(g_plan_mu);
+    for (size_t i = 0; i < g_overrides.size(); ++i)
+        if (g_overrides[i].M == M && g_overrides[i].d_in == d_in && g_overrides[i].d_out == d_out &&
+            g_overrides[i].r == r) {
+            if (plan)
+                g_overrides[i].p = *plan;
+            else
+                g_overrides.erase(g_overrides.begin() + static_cast<std::ptrdiff_t>(i));
+            return LORA_OK;
+        }
+    if (!plan) return LORA_OK;
+    if (g_overrides.size() >= MAX_OVERRIDES) return LORA_ERR_UNSUPPORTED;
+    g_overrides.push_back({M, d_in, d_out, r, *plan});
+    return LORA_OK;
+}
+
+lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, lora_plan_t *plan) {
+    if (!plan || op < LORA_OP_FWD || op > LORA_OP_BWD_FP8) return LORA_ERR_INVALID_ARG;
+    const int wf = op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
+    if (check_shapes(M, d_in, d_out, r, 1.0f, wf) != LORA_OK) return LORA_ERR_INVALID_ARG;
+    Plan pl;
+    make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
+    std::memset(plan, 0, sizeof(*plan));
+    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8);
+    plan->side_fwd = pl.side ? 1 : 2;
+    plan->side_bwd = bwd ? (pl.side_bwd ? 1 : 2) : 0;
+    plan->xa_cluster = pl.side ? pl.sx.C : 0;
+    plan->g_cluster = pl.side_bwd ? pl.sg.C : 0;
+    plan->g_group = pl.side_bwd ? pl.sg.group : 0;
+    plan->da_cluster = pl.side_bwd ? pl.sd.C : 0;
+    plan->fwd_tail = pl.fwd_tail ? 1 : 2;
+    plan->dx_overlap = bwd ? (pl.dx_overlap ? 1 : 2) : 0;
+    const bool sk_bwd = bwd && !pl.side_bwd;
+    plan->splitk[0] = pl.side ? 0 : pl.s_xa.splits;
+    plan->splitk[1] = sk_bwd ? pl.s_g.splits : 0;
+    plan->splitk[2] = sk_bwd ? pl.s_db.splits : 0;
+    plan->splitk[3] = sk_bwd ? pl.s_da.splits : 0;
+    return LORA_OK;
 }
 
 lora_status_t lora_linear_check(void *workspace, void *stream) {

@@ -251,6 +251,51 @@ def lora_linear_bwd_fp8(dY, x, W8, W8scale, A, B, xa_save, dX, dA, dB, alpha, ws
     _check(st, "lora_linear_bwd_fp8")
 
 
+class lora_plan_t(ctypes.Structure):
+    """The plan of one layer shape (include/lora_linear.h); 0 = the library's choice."""
+    _fields_ = [("side_fwd", ctypes.c_int32), ("side_bwd", ctypes.c_int32), ("xa_cluster", ctypes.c_int32),
+                ("g_cluster", ctypes.c_int32), ("g_group", ctypes.c_int32), ("da_cluster", ctypes.c_int32),
+                ("fwd_tail", ctypes.c_int32), ("dx_overlap", ctypes.c_int32), ("splitk", ctypes.c_int32 * 4)]
+
+    FIELDS = ("side_fwd", "side_bwd", "xa_cluster", "g_cluster", "g_group", "da_cluster", "fwd_tail", "dx_overlap")
+
+    def as_dict(self) -> dict:
+        d = {k: int(getattr(self, k)) for k in self.FIELDS}
+        d["splitk"] = [int(v) for v in self.splitk]
+        return d
+
+    @classmethod
+    def from_dict(cls, d: dict) -> "lora_plan_t":
+        p = cls()
+        for k in cls.FIELDS:
+            setattr(p, k, int(d.get(k, 0)))
+        for i, v in enumerate(d.get("splitk", [0, 0, 0, 0])):
+            p.splitk[i] = int(v)
+        return p
+
+
+def lora_linear_set_plan(M: int, d_in: int, d_out: int, r: int, plan):
+    """Install a plan (a lora_plan_t or a dict of its fields) for this shape; None removes it."""
+    fn = load_library().lora_linear_set_plan
+    fn.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    if plan is None:
+        _check(fn(M, d_in, d_out, r, None), "lora_linear_set_plan")
+        return
+    p = plan if isinstance(plan, lora_plan_t) else lora_plan_t.from_dict(plan)
+    _check(fn(M, d_in, d_out, r, ctypes.byref(p)), "lora_linear_set_plan")
+
+
+def lora_linear_get_plan(op: int, M: int, d_in: int, d_out: int, r: int) -> dict:
+    """The plan `op` uses for this shape, as a dict of lora_plan_t's fields."""
+    fn = load_library().lora_linear_get_plan
+    fn.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    p = lora_plan_t()
+    _check(fn(op, M, d_in, d_out, r, ctypes.byref(p)), "lora_linear_get_plan")
+    return p.as_dict()
+
+
 def lora_linear_check(ws, stream=None):
     ptr = None if ws is None else _ws(ws)[0]  # no workspace: only wait for the stream
     _check(load_library().lora_linear_check(ptr, _stream(stream)), "lora_linear_check")
