@@ -112,10 +112,11 @@ typedef struct {
     int32_t xa_cluster; /* side s.xa: CTAs per cluster, 1, 2 or 4 (they split d_in) */
     int32_t g_cluster;  /* side s.g + dB: CTAs per cluster, 1, 2 or 4 (they split d_out) */
     int32_t g_group;    /* side s.g + dB: 128-token blocks per round, 1..6, with g_group * r <= 64 */
-    int32_t da_cluster; /* side dA: CTAs per cluster, 1 or 2 (they split the tokens) */
+    int32_t da_cluster; /* side dA: CTAs per cluster, 1, 2 or 4 (they split the tokens) */
     int32_t fwd_tail;   /* forward main GEMM: 1 a partial last wave is cut along N, 2 it is not */
     int32_t dx_overlap; /* backward: 1 dA (and dB) start beside the dX GEMM's last wave, whose tiles
-                           stay whole; 2 they follow the dX GEMM, whose last wave is cut along N */
+                           stay whole (the library's choice); 2 they follow the dX GEMM, whose
+                           last wave is cut along N where it can be */
     int32_t splitk[4];  /* split-K kernels: K splits (1 .. 64) of s.xa, s.g, dB and dA */
 } lora_plan_t;
 

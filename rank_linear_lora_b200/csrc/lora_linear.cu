@@ -454,13 +454,13 @@ struct SidePlan {
     int C = 1, clusters = 0, group = 1, rounds = 0, per_cta = 0, n_out = 0, n_red = 0;
 };
 
-constexpr int SIDE_XA_STAGES = 8;
-constexpr int SIDE_GDB_STAGES = 3;
-constexpr int SIDE_DA_STAGES = 4;
+constexpr int SIDE_XA_STAGES = 8;   // 24 KB stages: 128 KB of x in flight
+constexpr int SIDE_GDB_STAGES = 4;  // 48 KB stages: 128 KB of dY in flight
+constexpr int SIDE_DA_STAGES = 5;   // 40 KB stages: 160 KB of x in flight
 
 // Cluster sizes of the side kernels.  A cluster's CTAs (one per SM: each holds ~225 KB
 // of shared memory) must fit in one GPC together; clusters of 8 did not all fit at once
-// on B200 and ran in two waves, clusters of 4 did.  dA, which starts on the SMs the dX
+// on B200 and ran in two waves, clusters of 4 did.  dA, when it starts on the SMs the dX
 // GEMM's CTA pairs leave as they finish, takes pairs.
 constexpr int SIDE_MAX_C = 4;
 constexpr int SIDE_MAX_C_DA = 2;
@@ -531,7 +531,7 @@ SidePlan side_plan_gdb(int64_t M, int64_t d_out, int r, int sms, int force_c = 0
 // round of `group` token blocks: r / (64 * group) of the dY stream's bytes, with group
 // at most 64 / r (the landing area).  It is taken up to r = 32 (at most a quarter of the
 // stream); wider ranks run the backward's side products on the split-K kernels.
-constexpr int SIDE_MAX_R_BWD = 32;
+constexpr int SIDE_MAX_R_BWD = SIDE_MAX_R_NARROW;
 
 struct Plan {
     size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0;
@@ -542,7 +542,9 @@ struct Plan {
     bool side_bwd = false;      // s.g + dB and dA on the side kernels (r <= 32)
     SidePlan sx, sg, sd;        // s.xa, s.g + dB partials, dA + dB
     bool fwd_tail = true;       // forward main GEMM: cut a partial last wave along N
-    bool dx_overlap = true;     // dA (and dB) beside the dX GEMM's last wave
+    int dx_mode = 0;            // 0: dA beside the dX GEMM's last wave unless that wave can be cut
+                                // along N (then dA follows); 1: always beside; 2: always after
+    int da_force_c = 0;         // dA's cluster size if the plan fixes it
 };
 
 // ------------------------------------------------------------------ plan overrides
@@ -586,7 +588,8 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     pl->side = ov.side_fwd ? ov.side_fwd == 1 : (r <= SIDE_MAX_R && side_enabled());
     pl->side_bwd = bwd && (ov.side_bwd ? ov.side_bwd == 1 : (r <= SIDE_MAX_R_BWD && side_enabled()));
     pl->fwd_tail = ov.fwd_tail != 2;
-    pl->dx_overlap = ov.dx_overlap != 2;
+    pl->dx_mode = ov.dx_overlap;
+    pl->da_force_c = ov.da_cluster;
     // split-K counters and partials (every s.xa when not on the side kernels; the
     // backward's s.g, dB and dA when not on the side kernels)
     const bool sk_xa = !pl->side, sk_bwd = bwd && !pl->side_bwd;
@@ -625,6 +628,19 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     }
     pl->total = off;
     return true;
+}
+
+// The backward's dA placement: beside the dX GEMM's last wave (true) or after it.  The
+// library's choice is beside: cutting the dX GEMM's last wave along N saves half a tile,
+// but dA after it then pays a whole launch, ramp and reduction on the critical path
+// (measured at the attention projection on one B200: 250 us per fwd+bwd against 234-242
+// us with dA hidden in the whole last wave).
+bool dx_overlaps(const Plan &pl, int64_t M, int64_t d_in, int pair_clusters, bool coded) {
+    (void)M;
+    (void)d_in;
+    (void)pair_clusters;
+    (void)coded;
+    return pl.dx_mode != 2;
 }
 
 // ------------------------------------------------------------------ validation
@@ -812,6 +828,14 @@ lora_status_t side_xa(const Ctx &c, const uint16_t *x, const uint16_t *A, uint16
     return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
 }
 
+// MN-major narrow operand [rows][r] of the s.g + dB and dA kernels: box {nb, 128} with
+// the swizzle whose span is nb bf16 (32 bytes for nb = 16, 64 bytes for nb = 32).
+bool tmap_narrow(CUtensorMap *m, const void *base, int r, int64_t rows, int nb) {
+    return lora_host::tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, r, rows, nb, 128,
+                              nb == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+int narrow_n(int r) { return r <= 16 ? 16 : 32; }
+
 // One pass over dY: s.g = bf16(s . dY.B) -> ws g [M, r], and dB's partials over each
 // round's tokens -> ws [rounds][d_out][r].  B [d_out, r] and s.xa [M, r] are read MN-major.
 lora_status_t side_gdb(const Ctx &c, const uint16_t *dY, const uint16_t *B, const uint16_t *sxa, int64_t M,
@@ -819,9 +843,10 @@ lora_status_t side_gdb(const Ctx &c, const uint16_t *dY, const uint16_t *B, cons
     const SidePlan &sp = c.plan.sg;
     SideArgs a = side_args(c);
     side_fill(a, sp, r);
+    a.nb = narrow_n(r);
     if (!tmap_bf16(&a.tmX, dY, d_out, M, 64, 128)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmS0, B, r, d_out, 64, 128)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmS1, sxa, r, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_narrow(&a.tmS0, B, r, d_out, a.nb)) return LORA_ERR_CUDA;
+    if (!tmap_narrow(&a.tmS1, sxa, r, M, a.nb)) return LORA_ERR_CUDA;
     a.rows_valid = static_cast<int>(M);
     a.scale = s;
     a.out_bf16 = reinterpret_cast<uint16_t *>(c.ws + c.plan.g);
@@ -836,13 +861,14 @@ lora_status_t side_gdb(const Ctx &c, const uint16_t *dY, const uint16_t *B, cons
 // launched right after the dX GEMM, whose outputs it does not read, so it starts on the
 // SMs that GEMM's last wave leaves idle; `grid_cap` bounds its CTAs.
 lora_status_t side_da(const Ctx &c, const uint16_t *x, const uint16_t *sg, float *dA, float *dB, int64_t M,
-                      int64_t d_in, int64_t d_out, int r, bool defer, int grid_cap) {
-    const SidePlan &sp = c.plan.sd;
+                      int64_t d_in, int64_t d_out, int r, bool defer, int grid_cap, int max_c) {
+    const SidePlan sp = side_plan(c.plan.sd.n_out, c.plan.sd.n_red, PLAN_SMS, max_c, c.plan.da_force_c);
     SideArgs a = side_args(c);
     side_fill(a, sp, r);
     a.defer_dep_wait = defer ? 1 : 0;
+    a.nb = narrow_n(r);
     if (!tmap_bf16(&a.tmX, x, d_in, M, 64, 128)) return LORA_ERR_CUDA;
-    if (!tmap_bf16(&a.tmS0, sg, r, M, 64, 128)) return LORA_ERR_CUDA;
+    if (!tmap_narrow(&a.tmS0, sg, r, M, a.nb)) return LORA_ERR_CUDA;
     a.rows_valid = static_cast<int>(d_in);
     a.out_f32 = dA;
     a.db_part = reinterpret_cast<float *>(c.ws + c.plan.part_db);
@@ -1046,7 +1072,8 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
     // dependent launch), they start on the SMs its last wave leaves idle and wait for
     // it only before they exit.  The dX tail is then left whole (no narrow tiles) so
     // those SMs free up early.
-    const bool overlap = dX != nullptr && pdl_enabled() && c.plan.dx_overlap;
+    const int dx_pairs = dX ? std::min(pair_clusters(c.info, true, wt.wf), PLAN_SMS / 2) : 0;
+    const bool overlap = dX != nullptr && pdl_enabled() && dx_overlaps(c.plan, M, d_in, dx_pairs, wt.coded());
     int idle = 0;
     if (dX) {
         // W [d_out, d_in] (or its codes) and A [r, d_in] are read MN-major (d_in contiguous).
@@ -1054,10 +1081,13 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
         LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
     }
     if (c.plan.side_bwd) {
-        // On the idle SMs alone when there are enough of them to be worth a cluster grid;
-        // otherwise every SM, the rest of the CTAs starting as the dX CTAs exit.
+        // dA reads nothing the dX GEMM writes, so it waits for that GEMM only before it
+        // exits and its CTAs take SMs as they free up.  Beside a whole last wave: pairs on
+        // that wave's idle SMs when there are enough of them to be worth a cluster grid;
+        // otherwise (and after a last wave cut along N) every SM, in clusters of up to 4.
+        const bool defer = dX != nullptr && pdl_enabled();
         const int cap = (overlap && idle >= 32) ? idle : PLAN_SMS;
-        LORA_TRY(side_da(c, x, sg, dA, dB, M, d_in, d_out, r, overlap, cap));
+        LORA_TRY(side_da(c, x, sg, dA, dB, M, d_in, d_out, r, defer, cap, overlap ? SIDE_MAX_C_DA : SIDE_MAX_C));
         return LORA_OK;
     }
     // Grid: the idle SMs when they can take all the dB / dA split tiles within about
@@ -1162,7 +1192,7 @@ lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r
             return false;
         };
         if (!in(q.side_fwd, {0, 1, 2}) || !in(q.side_bwd, {0, 1, 2}) || !in(q.xa_cluster, {0, 1, 2, 4}) ||
-            !in(q.g_cluster, {0, 1, 2, 4}) || q.g_group < 0 || q.g_group > 6 || !in(q.da_cluster, {0, 1, 2}) ||
+            !in(q.g_cluster, {0, 1, 2, 4}) || q.g_group < 0 || q.g_group > 6 || !in(q.da_cluster, {0, 1, 2, 4}) ||
             !in(q.fwd_tail, {0, 1, 2}) || !in(q.dx_overlap, {0, 1, 2}))
             return LORA_ERR_INVALID_ARG;
         for (int i = 0; i < 4; ++i)
@@ -1200,9 +1230,13 @@ lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_ou
     plan->xa_cluster = pl.side ? pl.sx.C : 0;
     plan->g_cluster = pl.side_bwd ? pl.sg.C : 0;
     plan->g_group = pl.side_bwd ? pl.sg.group : 0;
-    plan->da_cluster = pl.side_bwd ? pl.sd.C : 0;
+    const bool coded = wf != WF_BF16;
+    const bool overlap = dx_overlaps(pl, M, d_in, PLAN_SMS / 2, coded);
+    plan->da_cluster = pl.side_bwd ? side_plan(pl.sd.n_out, pl.sd.n_red, PLAN_SMS,
+                                               overlap ? SIDE_MAX_C_DA : SIDE_MAX_C, pl.da_force_c).C
+                                   : 0;
     plan->fwd_tail = pl.fwd_tail ? 1 : 2;
-    plan->dx_overlap = bwd ? (pl.dx_overlap ? 1 : 2) : 0;
+    plan->dx_overlap = bwd ? (overlap ? 1 : 2) : 0;
     const bool sk_bwd = bwd && !pl.side_bwd;
     plan->splitk[0] = pl.side ? 0 : pl.s_xa.splits;
     plan->splitk[1] = sk_bwd ? pl.s_g.splits : 0;

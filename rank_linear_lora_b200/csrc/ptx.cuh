@@ -238,14 +238,27 @@ __device__ __forceinline__ void tc_commit_pair_mc(uint32_t bar, uint16_t cta_mas
 //                 LBO unused.
 //   MN-major tile: K rows of 64 bf16 (128 B) per 64-wide MN chunk; 8-row atoms
 //                 1024 B apart along K (SBO); MN chunks LBO bytes apart.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// Swizzle modes of the descriptor's layout field: 128-, 64- and 32-byte swizzle (the
+// span of one row of an 8-row swizzle atom; TMA's SWIZZLE_128B / _64B / _32B).
+constexpr uint32_t SDESC_SW128 = 2, SDESC_SW64 = 4, SDESC_SW32 = 6;
+
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint32_t layout) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
     d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
     d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
     d |= 1ull << 46;
-    d |= 2ull << 61;
+    d |= static_cast<uint64_t>(layout) << 61;
     return d;
+}
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return sdesc(saddr, lbo_bytes, sbo_bytes, SDESC_SW128);
+}
+// MN-major tile of N = 16 (32-byte swizzle) or N = 32 (64-byte swizzle) columns: rows of
+// N bf16 along K, 8-row atoms N * 16 bytes apart (SBO); one atom along N (LBO unused).
+// A K step of 16 rows advances the start by two atoms.
+__device__ __forceinline__ uint64_t sdesc_mn_narrow(uint32_t saddr, int n) {
+    return sdesc(saddr, 16, static_cast<uint32_t>(n) * 16u, n == 16 ? SDESC_SW32 : SDESC_SW64);
 }
 
 // Instruction descriptor of kind::f16: D fp32, A and B bf16, optional MN-major

@@ -40,13 +40,16 @@ enum SideMode { SIDE_XA = 0, SIDE_GDB = 1, SIDE_DA = 2 };
 constexpr int SIDE_THREADS = 192;
 constexpr int SIDE_MAX_R = 64;   // widest rank the side kernels take (MN-major operands are 64 wide)
 constexpr int SIDE_RED_BYTES = 128 * SIDE_MAX_R * 4;  // reduction landing area: group * 128 * r fp32 at most
+constexpr int SIDE_MAX_R_NARROW = 32;  // s.g + dB and dA: r <= 32, their narrow operands N = 16 or 32
 
 struct SideArgs {
     CUtensorMap tmX;   // the streamed operand: x (XA, DA) or dY (GDB); bf16, box {64, 128}, 128B swizzle
-    CUtensorMap tmS0;  // XA: A [r, d_in] box {64, nr}; GDB: B [d_out, r] box {64, 128}; DA: s.g [M, r] box {64, 128}
-    CUtensorMap tmS1;  // GDB: s.xa [M, r] box {64, 128}
+    CUtensorMap tmS0;  // XA: A [r, d_in] box {64, nr}, 128B swizzle; GDB: B [d_out, r], DA: s.g [M, r],
+                       // box {nb, 128} with the 32B (nb = 16) or 64B (nb = 32) swizzle
+    CUtensorMap tmS1;  // GDB: s.xa [M, r], as tmS0
     int r;             // rank (multiple of 8, <= SIDE_MAX_R)
     int nr;            // XA: MMA N = r rounded up to 16
+    int nb;            // GDB, DA: MMA N of the narrow operands (B, s.xa, s.g): 16 (r <= 16) or 32
     int n_out;         // 128-row output blocks: ceil(M/128) (XA, GDB) or ceil(d_in/128) (DA)
     int rows_valid;    // output rows: M (XA, GDB) or d_in (DA)
     int n_red;         // reduction blocks: ceil(d_in/64) (XA), ceil(d_out/128) (GDB), ceil(M/128) (DA)
@@ -71,24 +74,24 @@ struct SideCfg {
     // 128B-swizzled chunks of 128 rows each (32 KB)
     static constexpr int X_BYTES = (MODE == SIDE_XA) ? 128 * 64 * 2 : 2 * 128 * 64 * 2;
     // small operands: XA the A tile [nr <= 64 rows x 64] K-major; GDB the B tile [128
-    // K rows x 64] and the s.xa tile [128 K rows x 64], both MN-major; DA the s.g tile
-    static constexpr int S0_BYTES = (MODE == SIDE_XA) ? 64 * 64 * 2 : 128 * 64 * 2;
-    static constexpr int S1_BYTES = (MODE == SIDE_GDB) ? 128 * 64 * 2 : 0;
+    // K rows x nb] and the s.xa tile [128 K rows x nb], both MN-major; DA the s.g tile
+    static constexpr int S0_BYTES = (MODE == SIDE_XA) ? 64 * 64 * 2 : 128 * SIDE_MAX_R_NARROW * 2;
+    static constexpr int S1_BYTES = (MODE == SIDE_GDB) ? 128 * SIDE_MAX_R_NARROW * 2 : 0;
     static constexpr int STAGE_BYTES = X_BYTES + S0_BYTES + S1_BYTES;
     // the cluster reduction's landing area: C slots of each owned row, group * 128 * r
-    // fp32 in all (at most 128 x 64 for one output block)
-    static constexpr int RED_BYTES = SIDE_RED_BYTES;
+    // fp32 in all (XA: one block of r <= 64; GDB: group * r <= 64; DA: one block of r <= 32)
+    static constexpr int RED_BYTES = (MODE == SIDE_DA) ? 128 * SIDE_MAX_R_NARROW * 4 : SIDE_RED_BYTES;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + RED_BYTES + BAR_BYTES;
     static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
     static_assert(STAGE_BYTES % 1024 == 0, "stage tiles stay 1024-byte aligned");
 };
 
-// TMEM columns a side kernel allocates: XA and DA one 64-column accumulator; GDB
-// `group` g accumulators and two dB accumulators, 64 columns each.
-__host__ __device__ constexpr int side_tmem_cols(int mode, int group) {
-    const int need = mode == SIDE_GDB ? (group + 2) * 64 : 64;
-    return need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+// TMEM columns a side kernel allocates: XA one accumulator of nr <= 64 columns, DA one
+// of nb; GDB `group` g accumulators and two dB accumulators of nb columns each.
+__host__ __device__ constexpr int side_tmem_cols(int mode, int group, int nb) {
+    const int need = mode == SIDE_GDB ? (group + 2) * nb : mode == SIDE_DA ? nb : 64;
+    return need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 }
 
 __device__ __forceinline__ uint32_t cluster_nctarank() {
@@ -138,7 +141,8 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
     const int q = static_cast<int>(cluster_ctarank());
     const int cl = static_cast<int>(blockIdx.x) / C;
     const int n_clusters = static_cast<int>(gridDim.x) / C;
-    const int tmem_cols = side_tmem_cols(MODE, p.group);
+    const int tmem_cols = side_tmem_cols(MODE, p.group, p.nb);
+    const int nb = p.nb;
     unsigned long long *trace = p.trace ? p.trace + static_cast<size_t>(blockIdx.x) * TRACE_WORDS : nullptr;
     if (trace && threadIdx.x == 0) {
         uint32_t smid;
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                         } else if (MODE == SIDE_GDB) {
                             // dY [128 tokens of block o][128 columns of block kb] as two chunks,
                             // B rows of block kb, s.xa rows of block o
-                            mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                            mbar_arrive_expect_tx(fb, Cfg::X_BYTES + 2 * 128 * nb * 2);
                             tma_load_2d(xs, &p.tmX, fb, kb * 128, o * 128);
                             tma_load_2d(xs + 16384, &p.tmX, fb, kb * 128 + 64, o * 128);
                             tma_load_2d(s0, &p.tmS0, fb, 0, kb * 128);
@@ -255,7 +259,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                         } else {
                             // x [128 tokens of block kb][128 columns of d_in block o] as two
                             // chunks, s.g rows of token block kb
-                            mbar_arrive_expect_tx(fb, Cfg::STAGE_BYTES);
+                            mbar_arrive_expect_tx(fb, Cfg::X_BYTES + 128 * nb * 2);
                             tma_load_2d(xs, &p.tmX, fb, o * 128, kb * 128);
                             tma_load_2d(xs + 16384, &p.tmX, fb, o * 128 + 64, kb * 128);
                             tma_load_2d(s0, &p.tmS0, fb, 0, kb * 128);
@@ -287,7 +291,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                             break;
                         }
                         tc_fence_after();
-                        db_tmem = tmem_base + static_cast<uint32_t>((p.group + b) * 64);
+                        db_tmem = tmem_base + static_cast<uint32_t>((p.group + b) * nb);
                     }
                     for (int i = 0; i < o_n; ++i) {
                         const uint32_t fb = smem_u32(&full_bar[m_stage]);
@@ -307,26 +311,28 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                                 tc_mma_bf16(tmem_base, ad + (kk * 32 >> 4), bd + (kk * 32 >> 4), idesc,
                                             (kb > kb_lo || kk > 0) ? 1u : 0u);
                         } else if (MODE == SIDE_GDB) {
-                            // g acc of block i [128 tokens x 64] += dY tile (K-major, K = 128 columns) . B
-                            constexpr uint32_t idesc_g = idesc_bf16(128, 64, false, true);
-                            const uint32_t g_tmem = tmem_base + static_cast<uint32_t>(i * 64);
-                            const uint64_t bd = sdesc_sw128(s0, 64 * 128, 1024);
+                            // g acc of block i [128 tokens x nb] += dY tile (K-major, K = 128 columns) . B
+                            const uint32_t idesc_g = idesc_bf16(128, nb, false, true);
+                            const uint32_t g_tmem = tmem_base + static_cast<uint32_t>(i * nb);
+                            const uint64_t bd = sdesc_mn_narrow(s0, nb);
+                            const uint32_t bstep = static_cast<uint32_t>(nb) * 32u >> 4;  // 16 K rows
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint64_t ad = sdesc_sw128(xs + (kk >> 2) * 16384, 16, 1024) + ((kk & 3) * 32 >> 4);
-                                tc_mma_bf16(g_tmem, ad, bd + (kk * 2048 >> 4), idesc_g, (kb > kb_lo || kk > 0) ? 1u : 0u);
+                                tc_mma_bf16(g_tmem, ad, bd + kk * bstep, idesc_g, (kb > kb_lo || kk > 0) ? 1u : 0u);
                             }
-                            // dB acc [128 columns x 64] += dY tile^T (MN-major, K = 128 tokens) . s.xa
-                            constexpr uint32_t idesc_b = idesc_bf16(128, 64, true, true);
-                            const uint64_t ad2 = sdesc_sw128(xs, 16384, 1024), bd2 = sdesc_sw128(s1, 64 * 128, 1024);
+                            // dB acc [128 columns x nb] += dY tile^T (MN-major, K = 128 tokens) . s.xa
+                            const uint32_t idesc_b = idesc_bf16(128, nb, true, true);
+                            const uint64_t ad2 = sdesc_sw128(xs, 16384, 1024), bd2 = sdesc_mn_narrow(s1, nb);
                             for (int kk = 0; kk < 8; ++kk)
-                                tc_mma_bf16(db_tmem, ad2 + (kk * 2048 >> 4), bd2 + (kk * 2048 >> 4), idesc_b,
+                                tc_mma_bf16(db_tmem, ad2 + (kk * 2048 >> 4), bd2 + kk * bstep, idesc_b,
                                             (i > 0 || kk > 0) ? 1u : 0u);
                         } else {
-                            // dA^T acc [128 columns of d_in x 64] += x tile^T (MN-major, K = 128 tokens) . s.g
-                            constexpr uint32_t idesc_a = idesc_bf16(128, 64, true, true);
-                            const uint64_t ad = sdesc_sw128(xs, 16384, 1024), bd = sdesc_sw128(s0, 64 * 128, 1024);
+                            // dA^T acc [128 columns of d_in x nb] += x tile^T (MN-major, K = 128 tokens) . s.g
+                            const uint32_t idesc_a = idesc_bf16(128, nb, true, true);
+                            const uint64_t ad = sdesc_sw128(xs, 16384, 1024), bd = sdesc_mn_narrow(s0, nb);
+                            const uint32_t bstep = static_cast<uint32_t>(nb) * 32u >> 4;  // 16 K rows
                             for (int kk = 0; kk < 8; ++kk)
-                                tc_mma_bf16(tmem_base, ad + (kk * 2048 >> 4), bd + (kk * 2048 >> 4), idesc_a,
+                                tc_mma_bf16(tmem_base, ad + (kk * 2048 >> 4), bd + kk * bstep, idesc_a,
                                             (kb > kb_lo || kk > 0) ? 1u : 0u);
                         }
                         tc_commit(smem_u32(&empty_bar[m_stage]));
@@ -370,7 +376,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                     float *dst = p.db_part + (static_cast<int64_t>(t) * p.d_out + n) * r;
                     for (int c0 = 0; c0 < r; c0 += 8) {
                         uint32_t v[8];
-                        tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>((p.group + b) * 64 + c0), v);
+                        tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>((p.group + b) * nb + c0), v);
                         tc_wait_ld();
                         if (n < p.d_out) {
                             float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
@@ -406,7 +412,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
                     if (acc_ok && has_work) {
                         uint32_t v[8];
-                        tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>(i * 64 + c0), v);
+                        tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>(i * (MODE == SIDE_XA ? 64 : nb) + c0), v);
                         tc_wait_ld();
                         a = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
                                         __uint_as_float(v[3]));

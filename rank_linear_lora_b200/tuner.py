@@ -12,7 +12,8 @@ sums differs, so a tuned plan meets the same bounds against the oracle.
 The search is coordinate descent from the library's own plan: each field in turn takes
 each of its admissible values with the others held, and the best value stays.  A
 candidate is timed as the median of `rounds` CUDA-event measurements of `reps`
-back-to-back forward + backward calls on the current stream.
+back-to-back forward + backward calls on the current stream, the calls rotating through
+sets of x and dY larger than L2 together, so the streamed operands come from DRAM.
 """
 from __future__ import annotations
 
@@ -34,7 +35,7 @@ def field_options(r: int) -> dict:
         "side_bwd": [1, 2] if r <= SIDE_MAX_R_BWD else [2],
         "g_cluster": [1, 2, 4],
         "g_group": [a for a in range(1, 7) if a * r <= 64],
-        "da_cluster": [1, 2],
+        "da_cluster": [1, 2, 4],
         "fwd_tail": [1, 2],
         "dx_overlap": [1, 2],
     }
@@ -84,8 +85,16 @@ def _op_pair(wf: str):
             "fp8": (L.OP_FWD_FP8, L.OP_BWD_FP8)}[wf]
 
 
+# Bytes of the per-call streamed inputs (x and dY) the timed calls rotate through: more
+# than twice the B200's 126 MB L2, so each call reads them from DRAM as in training
+# (otherwise the HBM-bound side products look as fast as they would from L2).
+ROTATE_BYTES = 256 << 20
+MAX_SETS = 8
+
+
 class _Layer:
-    """Device buffers of one layer shape (random values: only timing is measured)."""
+    """Device buffers of one layer shape (random values: only timing is measured), with
+    several sets of x and dY that successive calls rotate through."""
 
     def __init__(self, M, d_in, d_out, r, wf, alpha, device):
         import torch
@@ -95,7 +104,11 @@ class _Layer:
             return (torch.randn(*shape, generator=g) * scale).to(torch.bfloat16).to(device)
 
         self.shape, self.wf, self.alpha, self.device = (M, d_in, d_out, r), wf, alpha, device
-        self.x, self.dY = bf(M, d_in), bf(M, d_out)
+        per_set = M * (d_in + d_out) * 2
+        n_sets = max(1, min(MAX_SETS, -(-ROTATE_BYTES // per_set)))
+        self.sets = [(bf(M, d_in), bf(M, d_out)) for _ in range(n_sets)]
+        self.turn = 0
+        self.x, self.dY = self.sets[0]
         self.A, self.B = bf(r, d_in, scale=d_in ** -0.5), bf(d_out, r, scale=0.02)
         if wf == "q4":
             self.Wq = torch.randint(1, 16, (d_out, d_in // 2), generator=g, dtype=torch.uint8).to(device)
@@ -119,6 +132,8 @@ class _Layer:
         self.wsb = L.workspace(bop, *self.shape, device=self.device)
 
     def step(self):
+        self.x, self.dY = self.sets[self.turn % len(self.sets)]
+        self.turn += 1
         a = self.alpha
         if self.wf == "q4":
             L.lora_linear_fwd_q4(self.x, self.Wq, self.Ws, self.A, self.B, self.h, self.xa, a, self.wsf)

@@ -22,6 +22,7 @@ def clean():
 def test_set_get_clear_and_workspace_follows():
     default = L.lora_linear_get_plan(L.OP_BWD, *SHAPE)
     assert default["side_fwd"] == 1 and default["side_bwd"] == 1 and default["dx_overlap"] == 1
+    assert default["da_cluster"] == 2  # pairs, beside the dX GEMM's CTA pairs
     n0 = L.lora_linear_workspace_size(L.OP_BWD, *SHAPE)
     L.lora_linear_set_plan(*SHAPE, dict(side_bwd=2, splitk=[0, 8, 16, 16]))
     p = L.lora_linear_get_plan(L.OP_BWD, *SHAPE)
@@ -39,7 +40,7 @@ def test_set_get_clear_and_workspace_follows():
 
 @pytest.mark.parametrize("bad,status", [
     (dict(side_fwd=3), 1), (dict(xa_cluster=3), 1), (dict(xa_cluster=8), 1), (dict(g_group=7), 1),
-    (dict(g_group=-1), 1), (dict(da_cluster=4), 1), (dict(fwd_tail=3), 1), (dict(splitk=[65, 0, 0, 0]), 1),
+    (dict(g_group=-1), 1), (dict(da_cluster=8), 1), (dict(fwd_tail=3), 1), (dict(splitk=[65, 0, 0, 0]), 1),
     (dict(splitk=[0, -1, 0, 0]), 1)])
 def test_rejects_out_of_range_fields(bad, status):
     with pytest.raises(L.LoraError) as e:
