@@ -80,8 +80,16 @@ static double e4m3_to_f64(uint8_t c) {
  * int4 storage restored on the fly).  wfmt 2: 8-bit FP8 E4M3 codes [d_out, d_in], one
  * per byte, with a bf16 scale per row: w'[n, k] = e4m3(q[n, k]) * scale[n] (page
  * "ms-swift高效微调组合：LoRA+UnSloth提速实践", section 3.2: weights stored in FP8,
- * computed in BF16).
+ * computed in BF16).  wfmt 3: 4-bit codebook code (the BNB-style 4-bit format of page
+ * "ms-swift框架下UnSloth与Liger-Kernel优化实战", section UnSloth：让LoRA真正“低秩”起来),
+ * codes and scales laid out as wfmt 1, w'[n, k] = codebook[q[n, k]] * scale[n, k / 64]
+ * with the 16 codebook values set by oracle_set_codebook (NF4: the NormalFloat values).
  */
+static double g_codebook[16];
+
+void oracle_set_codebook(const double *cb) {
+    for (int i = 0; i < 16; ++i) g_codebook[i] = cb[i];
+}
 typedef struct {
     int wfmt;
     const uint16_t *w;
@@ -107,7 +115,10 @@ static void w_row(const wsrc_t *W, int64_t n, double *row) {
     for (int64_t k = 0; k < W->d_in; ++k) {
         uint8_t byte = p[k / 2];
         int code = (k % 2 == 0) ? (byte & 0x0F) : (byte >> 4);
-        row[k] = (double)(code - 8) * bf16_to_f64(sc[k / Q4_BLOCK]) / 7.0;
+        if (W->wfmt == 3)
+            row[k] = g_codebook[code] * bf16_to_f64(sc[k / Q4_BLOCK]);
+        else
+            row[k] = (double)(code - 8) * bf16_to_f64(sc[k / Q4_BLOCK]) / 7.0;
     }
 }
 

@@ -43,6 +43,7 @@ def _load():
         lib = ctypes.CDLL(_LIB)
         P, I64, D, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_int
         lib.oracle_threads.restype = I
+        lib.oracle_set_codebook.argtypes = [P]
         lib.oracle_set_threads.argtypes = [I]
         lib.oracle_weight.argtypes = [I, P, P, P, I64, I64, P]
         lib.oracle_xa.argtypes = [P, P, I64, I64, I64, P]
@@ -71,16 +72,22 @@ def set_threads(n: int) -> None:
     _load().oracle_set_threads(int(n))
 
 
-def _wargs(W=None, Wq=None, Wscale=None, W8=None, W8scale=None):
+def _wargs(W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None):
     if W is not None:
         return 0, _u16(W), None, None
     if W8 is not None:
         return 2, None, np.ascontiguousarray(W8, dtype=np.uint8), _u16(W8scale)
+    if codebook is not None:
+        cb = np.ascontiguousarray(codebook, dtype=np.float64)
+        if cb.shape != (16,):
+            raise ValueError("codebook: 16 values")
+        _load().oracle_set_codebook(cb.ctypes.data_as(ctypes.c_void_p))
+        return 3, None, np.ascontiguousarray(Wq, dtype=np.uint8), _u16(Wscale)
     return 1, None, np.ascontiguousarray(Wq, dtype=np.uint8), _u16(Wscale)
 
 
-def weight(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None) -> np.ndarray:
-    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
+def weight(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None) -> np.ndarray:
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale, codebook)
     out = np.empty((d_out, d_in), dtype=np.float64)
     _load().oracle_weight(fmt, _p(w), _p(q), _p(sc), d_out, d_in, _p(out))
     return out
@@ -96,13 +103,14 @@ def xa(x, A) -> np.ndarray:
     return out
 
 
-def h(x, B, xa_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None) -> np.ndarray:
+def h(x, B, xa_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None,
+      rows=None) -> np.ndarray:
     """Step 2: h = x . W^T + s * xa . B^T for all rows, or only ``rows``."""
     x, B = _u16(x), _u16(B)
     M, d_in = x.shape
     d_out, r = B.shape
     xa_ = np.ascontiguousarray(xa_, dtype=np.float64)
-    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale, codebook)
     rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = M if rr is None else len(rr)
     out = np.empty((n, d_out), dtype=np.float64)
@@ -121,13 +129,14 @@ def g(dY, B) -> np.ndarray:
     return out
 
 
-def dx(dY, A, g_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None) -> np.ndarray:
+def dx(dY, A, g_, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None,
+       rows=None) -> np.ndarray:
     """Step 4: dX = dY . W + s * g . A for all rows, or only ``rows``."""
     dY, A = _u16(dY), _u16(A)
     M, d_out = dY.shape
     r, d_in = A.shape
     g_ = np.ascontiguousarray(g_, dtype=np.float64)
-    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale)
+    fmt, w, q, sc = _wargs(W, Wq, Wscale, W8, W8scale, codebook)
     rr = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
     n = M if rr is None else len(rr)
     out = np.empty((n, d_in), dtype=np.float64)
@@ -158,19 +167,20 @@ def da(x, g_, s) -> np.ndarray:
     return out
 
 
-def forward(x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None):
+def forward(x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None, rows=None):
     """Steps 1-2.  Returns (h, xa)."""
     xa_ = xa(x, A)
-    return h(x, B, xa_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, rows=rows), xa_
+    return h(x, B, xa_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, codebook=codebook, rows=rows), xa_
 
 
-def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=None, xa_=None):
+def backward(dY, x, A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None, rows=None,
+             xa_=None):
     """Steps 1, 3-6.  Returns dict with dX (all rows or ``rows``), dA, dB, g, xa."""
     if xa_ is None:
         xa_ = xa(x, A)
     g_ = g(dY, B)
     return {
-        "dX": dx(dY, A, g_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, rows=rows),
+        "dX": dx(dY, A, g_, s, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, codebook=codebook, rows=rows),
         "dA": da(x, g_, s),
         "dB": db(dY, xa_, s),
         "g": g_,
@@ -190,7 +200,7 @@ def _f64(bits) -> np.ndarray:
     return (_u16(bits).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
-def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=2048):
+def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, rows=2048, codebook=None):
     """(n0, fp64 rows n0 .. n0+k) of the dequantised weight, block by block."""
     for n0 in range(0, d_out, rows):
         n1 = min(d_out, n0 + rows)
@@ -199,11 +209,12 @@ def _weight_blocks(d_out, d_in, W=None, Wq=None, Wscale=None, W8=None, W8scale=N
         elif W8 is not None:
             yield n0, weight(n1 - n0, d_in, W8=np.ascontiguousarray(W8)[n0:n1], W8scale=_u16(W8scale)[n0:n1])
         else:
-            yield n0, weight(n1 - n0, d_in, Wq=np.ascontiguousarray(Wq)[n0:n1], Wscale=_u16(Wscale)[n0:n1])
+            yield n0, weight(n1 - n0, d_in, Wq=np.ascontiguousarray(Wq)[n0:n1], Wscale=_u16(Wscale)[n0:n1],
+                             codebook=codebook)
 
 
-def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, xa_=None,
-                  block_rows=2048):
+def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None,
+                  xa_=None, block_rows=2048):
     """Step 2 projected: (h . v [M], u^T . h [d_out]) for v [d_out], u [M], with
     h . v = x . (W^T v) + s * xa . (B^T v) and u^T . h = W (x^T u) + s * B (xa^T u)."""
     M, d_in = np.shape(x)
@@ -213,7 +224,7 @@ def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8
     wt_v = np.zeros(d_in)
     xt_u = xf.T @ u
     col = np.empty(d_out)
-    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows):
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows, codebook=codebook):
         wt_v += Wb.T @ v[n0:n0 + len(Wb)]
         col[n0:n0 + len(Wb)] = Wb @ xt_u
     row = xf @ wt_v + s * (xa_ @ (Bf.T @ v))
@@ -221,8 +232,8 @@ def h_projections(x, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8
     return row, col
 
 
-def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, g_=None,
-                   block_rows=2048):
+def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None,
+                   g_=None, block_rows=2048):
     """Step 4 projected: (dX . v [M], u^T . dX [d_in]) for v [d_in], u [M], with
     dX . v = dY . (W v) + s * g . (A v) and u^T . dX = (dY^T u)^T W + s * (g^T u)^T A."""
     M, d_out = np.shape(dY)
@@ -232,7 +243,7 @@ def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, 
     w_v = np.empty(d_out)
     dyt_u = dYf.T @ u
     col = np.zeros(d_in)
-    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows):
+    for n0, Wb in _weight_blocks(d_out, d_in, W, Wq, Wscale, W8, W8scale, rows=block_rows, codebook=codebook):
         w_v[n0:n0 + len(Wb)] = Wb @ v
         col += dyt_u[n0:n0 + len(Wb)] @ Wb
     row = dYf @ w_v + s * (g_ @ (Af @ v))
@@ -240,12 +251,13 @@ def dx_projections(dY, A, B, s, v, u, *, W=None, Wq=None, Wscale=None, W8=None, 
     return row, col
 
 
-def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None) -> np.ndarray:
+def merged_weight(A, B, s, *, W=None, Wq=None, Wscale=None, W8=None, W8scale=None, codebook=None) -> np.ndarray:
     """The merged weight of step 2, W + s * B . A, in fp64 [d_out, d_in]: the weight for
     which h = x . (W + s B A)^T (the adapter folded in for deployment).  The 4-bit weight
     is decoded by the same rule as steps 2 and 4."""
     d_out, d_in = np.shape(B)[0], np.shape(A)[1]
-    return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale) + s * (_f64(B) @ _f64(A))
+    return weight(d_out, d_in, W=W, Wq=Wq, Wscale=Wscale, W8=W8, W8scale=W8scale, codebook=codebook) + s * (
+        _f64(B) @ _f64(A))
 
 
 # ------------------------------------------------------------------ whole tensors at full size

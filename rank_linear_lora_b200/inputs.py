@@ -156,6 +156,60 @@ def unpack_q4_codes(packed: np.ndarray) -> np.ndarray:
     return q
 
 
+def nf4_codebook() -> np.ndarray:
+    """The 16 values of the 4-bit NormalFloat data type (QLoRA; the format of BNB-style
+    4-bit weights), in increasing order, fp64.
+
+    Construction: codes split the standard normal into equal-probability bins on each
+    side of an exact zero, each side scaled so its extreme value is 1.  The positive
+    side takes the quantiles Phi^-1(p) at 8 evenly spaced probabilities p from 1 - delta
+    down to 1/2 (1/2 excluded), the negative side -Phi^-1(p) at 7 such probabilities,
+    and zero joins them: 7 negative values, 0, 8 positive values.  delta, the tail
+    probability beyond the outermost value, is the midpoint of 1/(2*15) and 1/(2*16)
+    (half a bin of the 15- and 16-bin grids), which keeps the extreme quantiles finite.
+    """
+    from scipy.special import ndtri
+    delta = 0.5 * (1.0 / 30.0 + 1.0 / 32.0)
+    pos = ndtri(np.linspace(1.0 - delta, 0.5, 9)[:-1])
+    neg = -ndtri(np.linspace(1.0 - delta, 0.5, 8)[:-1])
+    return np.sort(np.concatenate([neg / np.abs(neg).max(), [0.0], pos / pos.max()]))
+
+
+def quantise_codebook(w32: np.ndarray, codebook: np.ndarray):
+    """4-bit codebook code of a frozen weight [d_out, d_in] (fp32 draws).
+
+    Per block of 64 consecutive d_in elements: absmax = max |w| (fp32), stored as
+    bf16(absmax) (nearest-even); each weight's code is the index of the codebook value
+    nearest to w / stored scale (fp64; ties to the lower index); a block with absmax 0
+    gets the code of the value nearest 0.  Packing as quantise_q4 (low nibble = even
+    index).  Returns (packed uint8 [d_out, d_in/2], scale bf16 bits [d_out, d_in/64]).
+    """
+    d_out, d_in = w32.shape
+    assert d_in % Q4_BLOCK == 0
+    cb = np.asarray(codebook, dtype=np.float64)
+    assert cb.shape == (16,) and np.all(np.diff(cb) > 0)
+    mids = 0.5 * (cb[1:] + cb[:-1])  # decision boundaries; value == boundary -> lower index
+    out_q = np.empty((d_out, d_in // 2), dtype=np.uint8)
+    out_s = np.empty((d_out, d_in // Q4_BLOCK), dtype=np.uint16)
+    rows = max(1, (1 << 22) // d_in)
+
+    def work(r0):
+        r1 = min(d_out, r0 + rows)
+        wb = w32[r0:r1].reshape(r1 - r0, d_in // Q4_BLOCK, Q4_BLOCK)
+        amax = np.abs(wb).max(axis=2).astype(np.float32)
+        sbits = f32_to_bf16_bits(amax)
+        sc = bf16_bits_to_f32(sbits).astype(np.float64)
+        safe = np.where(sc > 0, sc, 1.0)
+        t = np.where(sc[:, :, None] > 0, wb.astype(np.float64) / safe[:, :, None], 0.0)
+        q = np.searchsorted(mids, t, side="left").astype(np.uint8).reshape(r1 - r0, d_in)
+        out_q[r0:r1] = (q[:, 0::2] & 0x0F) | (q[:, 1::2] << 4)
+        out_s[r0:r1] = sbits
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+        list(ex.map(work, range(0, d_out, rows)))
+    return out_q, out_s
+
+
 E4M3_MAX = 448.0
 
 
@@ -237,6 +291,7 @@ class LayerSpec:
     layer: int = 0
     proj: int = 1
     fp8: bool = False
+    nf4: bool = False   # frozen weight as 4-bit NormalFloat codes (codebook input)
 
     @property
     def s(self) -> float:
@@ -306,6 +361,7 @@ class LayerInputs:
     Wscale: np.ndarray | None  # bf16 bits [d_out, d_in/64] (q4 only)
     W8: np.ndarray | None = None       # uint8 E4M3 codes [d_out, d_in] (fp8 only)
     W8scale: np.ndarray | None = None  # bf16 bits [d_out] (fp8 only)
+    codebook: np.ndarray | None = None  # fp64 [16] (nf4 only; Wq, Wscale hold its codes)
 
 
 def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) -> LayerInputs:
@@ -332,4 +388,8 @@ def make_inputs(spec: LayerSpec, *, zero_A: bool = False, zero_B: bool = False) 
     if spec.fp8:
         W8, W8s = quantise_fp8(w32)
         return LayerInputs(spec, x, A, B, dY, None, None, None, W8, W8s)
+    if spec.nf4:
+        cb = nf4_codebook()
+        Wq, Ws = quantise_codebook(w32, cb)
+        return LayerInputs(spec, x, A, B, dY, None, Wq, Ws, codebook=cb)
     return LayerInputs(spec, x, A, B, dY, f32_to_bf16_bits(w32), None, None)

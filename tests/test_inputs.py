@@ -76,3 +76,46 @@ def test_e4m3_encoder_exact_values_and_ties():
     assert list(inputs.e4m3_encode(np.array([1.0625, 1.1875, -1.0625, 448.0]))) == [0x38, 0x3A, 0xB8, 0x7E]
     with pytest.raises(ValueError):
         inputs.e4m3_encode(np.array([449.0]))
+
+
+def test_nf4_codebook_construction():
+    """16 increasing values with an exact zero at code 7 and +-1 at the ends; each side
+    holds standard-normal quantiles at evenly spaced probabilities (the NormalFloat
+    construction), and the published values of the format come out."""
+    from scipy.special import ndtr
+    cb = inputs.nf4_codebook()
+    assert cb.shape == (16,) and np.all(np.diff(cb) > 0)
+    assert cb[0] == -1.0 and cb[7] == 0.0 and cb[15] == 1.0
+    delta = 0.5 * (1 / 30 + 1 / 32)
+    from scipy.special import ndtri
+    top = ndtri(1 - delta)
+    p_pos = ndtr(cb[8:] * top)          # 8 probabilities, 1/2 excluded, evenly spaced up to 1 - delta
+    p_neg = ndtr(-cb[:7] * top)         # 7 probabilities on the negative side
+    np.testing.assert_allclose(np.diff(p_pos), (0.5 - delta) / 8, rtol=1e-12)
+    np.testing.assert_allclose(np.diff(p_neg[::-1]), (0.5 - delta) / 7, rtol=1e-12)
+    # values of the NormalFloat-4 table as printed with 7 digits
+    np.testing.assert_allclose(cb[[1, 6, 8, 14]], [-0.6961928, -0.0910500, 0.0795803, 0.7229568], atol=2e-7)
+
+
+def test_codebook_quantiser_picks_the_nearest_value():
+    cb = inputs.nf4_codebook()
+    rng = np.random.default_rng(5)
+    w = rng.standard_normal((6, 192)).astype(np.float32)
+    w[0, :4] = [np.abs(w[0, :64]).max(), -np.abs(w[0, :64]).max(), 0.0, 0.0]
+    w[1, 64:128] = 0.0                   # a block of zeros: scale 0, code of 0
+    packed, scales = inputs.quantise_codebook(w, cb)
+    q = inputs.unpack_q4_codes(packed)
+    sc = inputs.bf16_bits_to_f32(scales).astype(np.float64)
+    assert sc[1, 1] == 0.0 and np.all(q[1, 64:128] == 7)
+    for n in range(6):
+        for k in range(192):
+            s = sc[n, k // 64]
+            if s == 0:
+                continue
+            t = float(w[n, k]) / s
+            best = int(np.argmin(np.abs(cb - t)))
+            assert q[n, k] == best or abs(abs(cb[q[n, k]] - t) - abs(cb[best] - t)) < 1e-15, (n, k)
+    amax = np.abs(w[0, :64]).max()
+    assert q[0, 2] == 7 and q[0, 3] == 7
+    if inputs.bf16_bits_to_f32(scales)[0, 0] <= amax:  # rounding of the scale may put w/scale a hair above 1
+        assert q[0, 0] == 15 and q[0, 1] == 0

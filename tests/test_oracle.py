@@ -423,3 +423,36 @@ def test_dense_steps_match_the_loops(fmt):
                                    rtol=0, atol=1e-13 * np.abs(h).max())
         np.testing.assert_allclose(oracle.dx_dense(inp.dY[r0:r1], inp.A, bwd["g"][r0:r1], spec.s, Wf),
                                    bwd["dX"][r0:r1], rtol=0, atol=1e-13 * np.abs(bwd["dX"]).max())
+
+
+def test_codebook_format_with_the_linear_codebook_is_the_4bit_format():
+    """Weight format 3 (codebook[q] * scale) with codebook (i - 8) / 7 decodes exactly as
+    format 1 ((q - 8) * scale / 7) through other code: every output agrees."""
+    spec = inputs.LayerSpec("cb", 40, 192, 72, 16, alpha=32.0, q4=True, seed=0xCB)
+    inp = inputs.make_inputs(spec)
+    lin = (np.arange(16) - 8) / 7.0
+    w1 = oracle.weight(72, 192, Wq=inp.Wq, Wscale=inp.Wscale)
+    w3 = oracle.weight(72, 192, Wq=inp.Wq, Wscale=inp.Wscale, codebook=lin)
+    np.testing.assert_allclose(w3, w1, rtol=0, atol=1e-15 * np.abs(w1).max())
+    h1, xa1 = oracle.forward(inp.x, inp.A, inp.B, spec.s, Wq=inp.Wq, Wscale=inp.Wscale)
+    h3, _ = oracle.forward(inp.x, inp.A, inp.B, spec.s, Wq=inp.Wq, Wscale=inp.Wscale, codebook=lin)
+    np.testing.assert_allclose(h3, h1, rtol=0, atol=1e-13 * np.abs(h1).max())
+    b1 = oracle.backward(inp.dY, inp.x, inp.A, inp.B, spec.s, Wq=inp.Wq, Wscale=inp.Wscale, xa_=xa1)
+    b3 = oracle.backward(inp.dY, inp.x, inp.A, inp.B, spec.s, Wq=inp.Wq, Wscale=inp.Wscale, codebook=lin, xa_=xa1)
+    np.testing.assert_allclose(b3["dX"], b1["dX"], rtol=0, atol=1e-13 * np.abs(b1["dX"]).max())
+
+
+def test_nf4_forward_reads_decoded_columns():
+    """With x = e_k the forward returns column k of the decoded weight: codebook[q] *
+    scale of the code's 64-block, for every code value the NF4 weight uses."""
+    spec = inputs.LayerSpec("nf4", 192, 192, 40, 8, alpha=16.0, nf4=True, seed=0x4F)
+    inp = inputs.make_inputs(spec)
+    x = np.zeros((192, 192), dtype=np.uint16)
+    x[np.arange(192), np.arange(192)] = 0x3F80  # bf16 1.0
+    zeroB = np.zeros_like(inp.B)
+    h, _ = oracle.forward(x, inp.A, zeroB, spec.s, Wq=inp.Wq, Wscale=inp.Wscale, codebook=inp.codebook)
+    q = inputs.unpack_q4_codes(inp.Wq)
+    sc = inputs.bf16_bits_to_f32(inp.Wscale).astype(np.float64)
+    want = inp.codebook[q] * np.repeat(sc, 64, axis=1)
+    np.testing.assert_array_equal(h, want.T)
+    assert len(np.unique(q)) == 16

@@ -2,7 +2,7 @@
 
 Each case copies the oracle into a temporary tree, plants one plausible mistake in
 oracle.c (a dropped term or scale, a wrong sign, a transposed operand, an index
-error, a wrong offset or bit order in a weight code), and runs the pins of
+error, a wrong offset, bit order, codebook entry or scale in a weight code), and runs the pins of
 test_oracle.py against that copy in a subprocess: at least one pin must fail (pytest
 exit status 1, a failed test, not a crash or a collection error).  An unchanged copy
 run the same way must pass.  Every planted mistake keeps its indices inside the
@@ -28,10 +28,15 @@ MUTANTS = {  # name: (text of oracle.c, replacement)
     "da_transposed": ("dA[j * d_in + k] = s * acc[(k - k0) * r + j];", "dA[k * r + j] = s * acc[(k - k0) * r + j];"),
     "q4_offset": ("(double)(code - 8)", "(double)(code - 7)"),
     "q4_nibble_order": ("(k % 2 == 0) ? (byte & 0x0F) : (byte >> 4)", "(k % 2 == 1) ? (byte & 0x0F) : (byte >> 4)"),
-    "q4_scale_block": ("sc[k / Q4_BLOCK]", "sc[k / Q4_BLOCK / 2]"),
+    "q4_scale_block": ("(double)(code - 8) * bf16_to_f64(sc[k / Q4_BLOCK])",
+                       "(double)(code - 8) * bf16_to_f64(sc[k / Q4_BLOCK / 2])"),
     "fp8_exponent_bias": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "fp8_subnormal_step": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
     "fp8_row_scale": ("bf16_to_f64(W->scale[n])", "bf16_to_f64(W->scale[0])"),
+    "codebook_reversed": ("row[k] = g_codebook[code] * bf16_to_f64(sc[k / Q4_BLOCK]);",
+                          "row[k] = g_codebook[15 - code] * bf16_to_f64(sc[k / Q4_BLOCK]);"),
+    "codebook_without_scale": ("row[k] = g_codebook[code] * bf16_to_f64(sc[k / Q4_BLOCK]);",
+                               "row[k] = g_codebook[code];"),
 }
 
 
