@@ -50,6 +50,8 @@ def parse():
     p.add_argument("--layer", type=int, default=0, help="layer of a multi-layer workload")
     p.add_argument("--fp8", action="store_true",
                    help="store the workload's frozen weight as FP8 (E4M3 codes, one bf16 scale per row)")
+    p.add_argument("--nf4", action="store_true",
+                   help="store the workload's frozen weight as 4-bit NF4 codes (codebook weight, d_in % 64 == 0)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--backend", choices=["nccl", "gloo"], default="nccl",
@@ -79,7 +81,8 @@ def algorithmic_bytes(spec) -> float:
     columns per row); A, xa and dA hold every projection's ranks."""
     M, di, do, r = spec.M, spec.d_in, spec.d_out, spec.r
     rb = r // spec.proj
-    w = do * di // 2 + do * (di // 64) * 2 if spec.q4 else do * di + do * 2 if spec.fp8 else do * di * 2
+    w = (do * di // 2 + do * (di // 64) * 2 if (spec.q4 or spec.nf4) else do * di + do * 2 if spec.fp8
+         else do * di * 2)
     fwd = M * di * 2 + w + r * di * 2 + do * rb * 2 + M * do * 2 + M * r * 2
     bwd = M * do * 2 + M * di * 2 + w + r * di * 2 + do * rb * 2 + M * r * 2 + M * di * 2 + r * di * 4 + do * rb * 4
     return float(fwd + bwd)
@@ -87,7 +90,7 @@ def algorithmic_bytes(spec) -> float:
 
 # The sources the layer's kernels and their launches are built from: lora_linear.cu and
 # every header it includes (the merge and the workspace-free forward are other files).
-LAYER_SOURCES = ("lora_linear.cu", "tc_gemm.cuh", "tc_gemm2.cuh", "ptx.cuh", "tmap.h")
+LAYER_SOURCES = ("lora_linear.cu", "side.cuh", "tc_gemm.cuh", "tc_gemm2.cuh", "ptx.cuh", "tmap.h")
 
 
 def kernel_source_hash() -> str:
@@ -196,7 +199,7 @@ class ClockSampler:
 def config_dict(spec, workload_name: str, world: int) -> dict:
     """The workload as both arms name it (identical keys and values)."""
     return {"workload": workload_name, "M": spec.M, "d_in": spec.d_in, "d_out": spec.d_out, "r": spec.r,
-            "alpha": spec.alpha, "q4": spec.q4, "fp8": spec.fp8, "projections": spec.proj,
+            "alpha": spec.alpha, "q4": spec.q4, "fp8": spec.fp8, "nf4": spec.nf4, "projections": spec.proj,
             "tokens_per_step": spec.M * world,
             "l2": f"{N_SETS} rotating input sets (> L2); no flush inside the timed region",
             "parallelism": f"dp{world}"}
@@ -334,7 +337,7 @@ def _oracle_step(oracle, inp, spec, start, tokens):
     rows = [(start + i) % M for i in range(tokens)]
     x, dY = inp.x[rows], inp.dY[rows]
     wkw = (dict(Wq=inp.Wq, Wscale=inp.Wscale) if spec.q4 else dict(W8=inp.W8, W8scale=inp.W8scale) if spec.fp8
-           else dict(W=inp.W))
+           else dict(Wq=inp.Wq, Wscale=inp.Wscale, codebook=inp.codebook) if spec.nf4 else dict(W=inp.W))
     h, xa = oracle.forward(x, inp.A, inp.B, spec.s, **wkw)
     oracle.backward(dY, x, inp.A, inp.B, spec.s, xa_=xa, **wkw)
 
@@ -402,6 +405,9 @@ def main():
     if args.fp8:
         spec = spec.with_(q4=False, fp8=True)
         workload_name += " with the FP8 weight"
+    if args.nf4:
+        spec = spec.with_(q4=False, nf4=True)
+        workload_name += " with the NF4 weight"
     if args.shape:
         M_, di_, do_ = (int(v) for v in args.shape.split(","))
         spec = spec.with_(M=M_, d_in=di_, d_out=do_)
@@ -444,9 +450,10 @@ def main():
         if k == 0:
             host_inputs = inp
         s = {"x": d16(inp.x), "A": d16(inp.A), "B": d16(inp.B), "dY": d16(inp.dY)}
-        if spec.q4:
+        if spec.q4 or spec.nf4:
             s["Wq"] = torch.from_numpy(inp.Wq).to(dev)
             s["Wscale"] = d16(inp.Wscale)
+            s["cb"] = inp.codebook
         elif spec.fp8:
             s["W8"] = torch.from_numpy(inp.W8).to(dev)
             s["W8scale"] = d16(inp.W8scale)
@@ -458,7 +465,7 @@ def main():
         s["grad"] = PackedGrads(r, di, do, device=dev)  # fp32 [dA | dB], the one all-reduced buffer
         s["dA"], s["dB"] = s["grad"].dA, s["grad"].dB
         fop, bop = ((L.OP_FWD_Q4, L.OP_BWD_Q4) if spec.q4 else (L.OP_FWD_FP8, L.OP_BWD_FP8) if spec.fp8
-                    else (L.OP_FWD, L.OP_BWD))
+                    else (L.OP_FWD_NF4, L.OP_BWD_NF4) if spec.nf4 else (L.OP_FWD, L.OP_BWD))
         s["wsf"] = L.workspace(fop, M, di, do, r, device=dev)
         s["wsb"] = L.workspace(bop, M, di, do, r, device=dev)
         sets.append(s)
@@ -471,6 +478,11 @@ def main():
         elif spec.fp8:
             L.lora_linear_fwd_fp8(s["x"], s["W8"], s["W8scale"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
             L.lora_linear_bwd_fp8(s["dY"], s["x"], s["W8"], s["W8scale"], s["A"], s["B"], s["xa"], s["dX"],
+                                  s["dA"], s["dB"], alpha, s["wsb"])
+        elif spec.nf4:
+            L.lora_linear_fwd_nf4(s["x"], s["Wq"], s["Wscale"], s["cb"], s["A"], s["B"], s["h"], s["xa"], alpha,
+                                  s["wsf"])
+            L.lora_linear_bwd_nf4(s["dY"], s["x"], s["Wq"], s["Wscale"], s["cb"], s["A"], s["B"], s["xa"], s["dX"],
                                   s["dA"], s["dB"], alpha, s["wsb"])
         else:
             L.lora_linear_fwd(s["x"], s["W"], s["A"], s["B"], s["h"], s["xa"], alpha, s["wsf"])
@@ -572,6 +584,9 @@ def main():
             elif spec.fp8:
                 L.lora_linear_fwd_fp8(st["x"], st["W8"], st["W8scale"], st["A"], st["B"], st["h"], st["xa"], alpha,
                                       st["wsf"])
+            elif spec.nf4:
+                L.lora_linear_fwd_nf4(st["x"], st["Wq"], st["Wscale"], st["cb"], st["A"], st["B"], st["h"], st["xa"],
+                                      alpha, st["wsf"])
             else:
                 L.lora_linear_fwd(st["x"], st["W"], st["A"], st["B"], st["h"], st["xa"], alpha, st["wsf"])
 
@@ -582,6 +597,9 @@ def main():
             elif spec.fp8:
                 L.lora_linear_bwd_fp8(st["dY"], st["x"], st["W8"], st["W8scale"], st["A"], st["B"], st["xa"],
                                       st["dX"], st["dA"], st["dB"], alpha, st["wsb"])
+            elif spec.nf4:
+                L.lora_linear_bwd_nf4(st["dY"], st["x"], st["Wq"], st["Wscale"], st["cb"], st["A"], st["B"],
+                                      st["xa"], st["dX"], st["dA"], st["dB"], alpha, st["wsb"])
             else:
                 L.lora_linear_bwd(st["dY"], st["x"], st["W"], st["A"], st["B"], st["xa"], st["dX"], st["dA"],
                                   st["dB"], alpha, st["wsb"])
@@ -605,7 +623,7 @@ def main():
     # Context, not the reference arm: the unfused composition of the same layer in PyTorch
     # with autograd (x@W.T + s*(x@A.T)@B.T, cuBLAS bf16), same inputs, same GPU.
     context = None
-    if world == 1 and not spec.q4 and not spec.fp8:
+    if world == 1 and not spec.q4 and not spec.fp8 and not spec.nf4:
         st = sets[0]
         xg = st["x"].detach().clone().requires_grad_(True)
         Ag = st["A"].detach().clone().requires_grad_(True)
@@ -639,7 +657,7 @@ def main():
     # median of 20.  Before each launch L2 is flushed by reading 256 MB (clean lines: a
     # write would leave ~126 MB of dirty lines for the merge to write back).
     merge = None
-    if rank == 0 and not spec.fp8:
+    if rank == 0 and not spec.fp8 and not spec.nf4:
         s0 = sets[0]
         w_out = torch.empty(do, di, dtype=torch.bfloat16, device=dev)
         flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)

@@ -38,7 +38,7 @@
  *     1 <= M <= 2^30; d_in and d_out multiples of 8 in 8 .. 2^24, with
  *     ceil(M/128) * ceil(max(d_in, d_out)/128) <= 2^31 - 1 (32-bit tile counts: only
  *     an output of more than 2^45 elements reaches it); 1 <= r <= 256 with r % 8 == 0; alpha finite;
- *     for *_q4 also d_in % 64 == 0; for *_fp8 d_in % 16 == 0.
+ *     for *_q4 and *_nf4 also d_in % 64 == 0; for *_fp8 d_in % 16 == 0.
  *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
  *     aligned, be zero-filled before its first use, and must not be used by two calls
  *     that may run at the same time.  Every call that completes leaves the workspace's
@@ -48,8 +48,8 @@
  *     for its predecessor in the stream before touching global memory, so stream
  *     order is preserved; only launch latency and set-up overlap.
  *   - The device must be compute capability 10.0 (B200); otherwise
- *     LORA_ERR_UNSUPPORTED is returned and nothing runs.  The *_q4 and *_fp8 entry
- *     points also need two-SM clusters (CTA pairs); without them they return
+ *     LORA_ERR_UNSUPPORTED is returned and nothing runs.  The *_q4, *_fp8 and *_nf4
+ *     entry points also need two-SM clusters (CTA pairs); without them they return
  *     LORA_ERR_UNSUPPORTED.
  *   - Device-side waits are bounded.  A wait that runs out sets an error word in the
  *     workspace and the kernels return early; lora_linear_check() reports it.
@@ -91,7 +91,9 @@ typedef enum {
     LORA_OP_FWD_Q4 = 2,
     LORA_OP_BWD_Q4 = 3,
     LORA_OP_FWD_FP8 = 4,
-    LORA_OP_BWD_FP8 = 5
+    LORA_OP_BWD_FP8 = 5,
+    LORA_OP_FWD_NF4 = 6,
+    LORA_OP_BWD_NF4 = 7
 } lora_op_t;
 
 /*
@@ -217,6 +219,33 @@ LORA_API lora_status_t lora_linear_bwd_fp8(const uint16_t *dY, const uint16_t *x
                                            const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB,
                                            int64_t M, int64_t d_in, int64_t d_out, int r, float alpha,
                                            void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Forward with a 4-bit codebook weight, the BNB-style 4-bit format (page
+ * "ms-swift框架下UnSloth与Liger-Kernel优化实战", section UnSloth：让LoRA真正“低秩”起来:
+ * BNB 4-bit weights restored on the fly): each weight is a 4-bit index into a table of
+ * 16 values, scaled by a bf16 absmax per 64 weights along d_in,
+ *     w'[n, k] = codebook[q[n, k]] * Wscale[n, k / 64].
+ * NF4 is the codebook of the 4-bit NormalFloat type (16 quantiles of a standard normal
+ * scaled to [-1, 1], with an exact zero); any 16 finite values work.  Codes and scales
+ * are laid out as in lora_linear_fwd_q4 (Wq [d_out, d_in/2], low nibble = even index;
+ * Wscale [d_out, d_in/64]); `codebook` points to 16 floats in HOST memory, read during
+ * the call.  The codes are decoded in shared memory inside the GEMMs: each table value
+ * codebook[i] * scale is formed in fp32 and rounded once to bf16.  d_in % 64 == 0;
+ * workspace of LORA_OP_FWD_NF4; a non-finite codebook value gives LORA_ERR_INVALID_ARG. */
+LORA_API lora_status_t lora_linear_fwd_nf4(const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale,
+                                           const float *codebook, const uint16_t *A, const uint16_t *B,
+                                           uint16_t *h, uint16_t *xa_save, int64_t M, int64_t d_in,
+                                           int64_t d_out, int r, float alpha, void *workspace,
+                                           size_t workspace_bytes, void *stream);
+
+/* Backward with the 4-bit codebook weight (same passage and layout); as lora_linear_bwd
+ * with W replaced by (Wq, Wscale, codebook); workspace of LORA_OP_BWD_NF4. */
+LORA_API lora_status_t lora_linear_bwd_nf4(const uint16_t *dY, const uint16_t *x, const uint8_t *Wq,
+                                           const uint16_t *Wscale, const float *codebook, const uint16_t *A,
+                                           const uint16_t *B, const uint16_t *xa_save, uint16_t *dX, float *dA,
+                                           float *dB, int64_t M, int64_t d_in, int64_t d_out, int r,
+                                           float alpha, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * Forward without a workspace, for callers that cannot allocate device memory: a

@@ -197,7 +197,7 @@ constexpr int PAIR_STAGES_FP8 = 4;  // the FP8 code rings take twice the 4-bit o
 
 template <int WF>
 constexpr int pair_stages() {
-    return WF == WF_Q4 ? PAIR_STAGES_Q4 : WF == WF_FP8 ? PAIR_STAGES_FP8 : PAIR_STAGES;
+    return (WF == WF_Q4 || WF == WF_CB) ? PAIR_STAGES_Q4 : WF == WF_FP8 ? PAIR_STAGES_FP8 : PAIR_STAGES;
 }
 
 template <bool B_MN, int WF>
@@ -362,8 +362,8 @@ int probe_pair_clusters(const DevInfo *dev) {
 
 // Clusters of two CTAs of the pair kernel that can be resident at once (0 if none).
 int pair_clusters(DevInfo *dev, bool b_mn, int wf) {
-    static int cached[64][6] = {};
-    static bool probed[64][6] = {};
+    static int cached[64][8] = {};
+    static bool probed[64][8] = {};
     int d = 0;
     cudaGetDevice(&d);
     std::lock_guard<std::mutex> lk(g_mu);
@@ -377,7 +377,9 @@ int pair_clusters(DevInfo *dev, bool b_mn, int wf) {
             case 2: cached[d][v] = probe_pair_clusters<false, WF_Q4>(dev); break;
             case 3: cached[d][v] = probe_pair_clusters<true, WF_Q4>(dev); break;
             case 4: cached[d][v] = probe_pair_clusters<false, WF_FP8>(dev); break;
-            default: cached[d][v] = probe_pair_clusters<true, WF_FP8>(dev); break;
+            case 5: cached[d][v] = probe_pair_clusters<true, WF_FP8>(dev); break;
+            case 6: cached[d][v] = probe_pair_clusters<false, WF_CB>(dev); break;
+            default: cached[d][v] = probe_pair_clusters<true, WF_CB>(dev); break;
         }
     }
     return cached[d][v];
@@ -392,7 +394,7 @@ enum {
     AB_T64 = 9, AB_T128, AB_T256,
     AB_PAIR_K = 12, AB_PAIR_MN = 13, AB_PAIR_K_Q4 = 14, AB_PAIR_MN_Q4 = 15,
     AB_SIDE_XA = 16, AB_SIDE_GDB = 17, AB_SIDE_DA = 18,
-    AB_PAIR_K_FP8 = 19, AB_PAIR_MN_FP8 = 20,
+    AB_PAIR_K_FP8 = 19, AB_PAIR_MN_FP8 = 20, AB_PAIR_K_CB = 21, AB_PAIR_MN_CB = 22,
 };
 
 int bn_class_kmajor(int r) { return r <= 16 ? 16 : r <= 64 ? 64 : r <= 128 ? 128 : 256; }
@@ -529,9 +531,12 @@ SidePlan side_plan_gdb(int64_t M, int64_t d_out, int r, int sms, int force_c = 0
 
 // The one-pass backward (s.g with dB's partials, then dA) writes one fp32 dB partial per
 // round of `group` token blocks: r / (64 * group) of the dY stream's bytes, with group
-// at most 64 / r (the landing area).  It is taken up to r = 32 (at most a quarter of the
-// stream); wider ranks run the backward's side products on the split-K kernels.
+// at most 64 / r (the landing area), and dA reads them back.  The library takes it up to
+// r = 16 (at most an eighth of the stream; at r = 32 the stacked gate + up layer wrote
+// 90 MB of partials and ran 41 us slower per step than on the split-K kernels); a plan
+// can ask for it up to r = 32, the widest its narrow operands take.
 constexpr int SIDE_MAX_R_BWD = SIDE_MAX_R_NARROW;
+constexpr int SIDE_DEFAULT_R_BWD = 16;
 
 struct Plan {
     size_t err = 0, ctr = 0, xa = 0, g = 0, part_xa = 0, part_g = 0, part_db = 0, part_da = 0;
@@ -577,7 +582,7 @@ Split forced_split(int64_t kb, int splits) {
 }
 
 bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, Plan *pl) {
-    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8);
+    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8 || op == LORA_OP_BWD_NF4);
     const int64_t mt_tok = cdiv(M, BM), mt_in = cdiv(d_in, BM), mt_out = cdiv(d_out, BM);
     lora_plan_t ov;
     std::memset(&ov, 0, sizeof(ov));
@@ -586,7 +591,7 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     pl->err = off;
     off += 256;
     pl->side = ov.side_fwd ? ov.side_fwd == 1 : (r <= SIDE_MAX_R && side_enabled());
-    pl->side_bwd = bwd && (ov.side_bwd ? ov.side_bwd == 1 : (r <= SIDE_MAX_R_BWD && side_enabled()));
+    pl->side_bwd = bwd && (ov.side_bwd ? ov.side_bwd == 1 : (r <= SIDE_DEFAULT_R_BWD && side_enabled()));
     pl->fwd_tail = ov.fwd_tail != 2;
     pl->dx_mode = ov.dx_overlap;
     pl->da_force_c = ov.da_cluster;
@@ -656,7 +661,7 @@ lora_status_t check_shapes(int64_t M, int64_t d_in, int64_t d_out, int r, float 
     if (((M + 127) / 128) * ((std::max(d_in, d_out) + 127) / 128) > INT32_MAX) return LORA_ERR_INVALID_ARG;
     if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
     if (!std::isfinite(alpha)) return LORA_ERR_INVALID_ARG;
-    if (wf == WF_Q4 && d_in % 64) return LORA_ERR_INVALID_ARG;   // one scale per 64 codes
+    if ((wf == WF_Q4 || wf == WF_CB) && d_in % 64) return LORA_ERR_INVALID_ARG;  // one scale per 64 codes
     if (wf == WF_FP8 && d_in % 16) return LORA_ERR_INVALID_ARG;  // code rows of whole 16-byte units
     return LORA_OK;
 }
@@ -891,6 +896,7 @@ struct MainOperands {
     const uint16_t *Wscale = nullptr;  // its bf16 scales: [d_out, d_in / 64] (4-bit) or [d_out] (FP8)
     int64_t q_rows = 0, q_cols = 0;    // W shape [d_out, d_in]
     int wf = WF_BF16;
+    const float *codebook = nullptr;   // 4-bit codebook weight: its 16 values (host)
 };
 
 // `idle_sms` (optional) receives how many SMs the last wave leaves without work.
@@ -908,7 +914,9 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
     if (q4 && pair_C == 0) return LORA_ERR_UNSUPPORTED;  // decoded weights run on CTA pairs only
     if (q4) {
         a.wscale = o.Wscale;
-        a.scale_ld = o.wf == WF_Q4 ? static_cast<int>(o.q_cols / 64) : 1;
+        a.scale_ld = o.wf == WF_FP8 ? 1 : static_cast<int>(o.q_cols / 64);
+        if (o.wf == WF_CB)
+            for (int i = 0; i < 16; ++i) a.cb[i] = o.codebook[i];
         a.scale_rows = static_cast<int>(o.q_rows);
         // codes [d_out][d_in / 2] (4-bit) or [d_out][d_in] (FP8) bytes; each dequant warp
         // fetches DQ_QROWS rows x the bytes of 64 codes at a time
@@ -949,6 +957,9 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         else if (o.wf == WF_FP8)
             e = b_mn ? launch_pair<true, WF_FP8>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_FP8, kind)
                      : launch_pair<false, WF_FP8>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_FP8, kind);
+        else if (o.wf == WF_CB)
+            e = b_mn ? launch_pair<true, WF_CB>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN_CB, kind)
+                     : launch_pair<false, WF_CB>(a, 2 * clusters, c.st, c.info, AB_PAIR_K_CB, kind);
         else
             e = b_mn ? launch_pair<true, WF_BF16>(a, 2 * clusters, c.st, c.info, AB_PAIR_MN, kind)
                      : launch_pair<false, WF_BF16>(a, 2 * clusters, c.st, c.info, AB_PAIR_K, kind);
@@ -1009,11 +1020,16 @@ struct Weight {
     const uint8_t *Wq = nullptr;       // 4-bit or FP8 codes
     const uint16_t *Wscale = nullptr;
     int wf = WF_BF16;
+    const float *codebook = nullptr;   // WF_CB: 16 values (host memory)
     bool coded() const { return wf != WF_BF16; }
-    bool present() const { return coded() ? (Wq && Wscale) : W != nullptr; }
+    bool present() const { return coded() ? (Wq && Wscale && (wf != WF_CB || codebook)) : W != nullptr; }
     bool aligned() const { return coded() ? (aligned16(Wq) && aligned16(Wscale)) : aligned16(W); }
-    int op_fwd() const { return wf == WF_Q4 ? LORA_OP_FWD_Q4 : wf == WF_FP8 ? LORA_OP_FWD_FP8 : LORA_OP_FWD; }
-    int op_bwd() const { return wf == WF_Q4 ? LORA_OP_BWD_Q4 : wf == WF_FP8 ? LORA_OP_BWD_FP8 : LORA_OP_BWD; }
+    int op_fwd() const {
+        return wf == WF_Q4 ? LORA_OP_FWD_Q4 : wf == WF_FP8 ? LORA_OP_FWD_FP8 : wf == WF_CB ? LORA_OP_FWD_NF4 : LORA_OP_FWD;
+    }
+    int op_bwd() const {
+        return wf == WF_Q4 ? LORA_OP_BWD_Q4 : wf == WF_FP8 ? LORA_OP_BWD_FP8 : wf == WF_CB ? LORA_OP_BWD_NF4 : LORA_OP_BWD;
+    }
 };
 
 MainOperands main_operands(const Weight &wt, const void *A0, const void *A1, const void *B1, void *C,
@@ -1023,6 +1039,7 @@ MainOperands main_operands(const Weight &wt, const void *A0, const void *A1, con
         o.Wq = wt.Wq;
         o.Wscale = wt.Wscale;
         o.wf = wt.wf;
+        o.codebook = wt.codebook;
         o.q_rows = d_out;
         o.q_cols = d_in;
     }
@@ -1034,6 +1051,9 @@ lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, c
                        size_t ws_bytes, void *stream) {
     LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.wf));
     if (!x || !wt.present() || !A || !B || !h) return LORA_ERR_INVALID_ARG;
+    if (wt.wf == WF_CB)
+        for (int i = 0; i < 16; ++i)
+            if (!std::isfinite(wt.codebook[i])) return LORA_ERR_INVALID_ARG;
     if (!aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(h) ||
         (xa_save && !aligned16(xa_save)))
         return LORA_ERR_MISALIGNED;
@@ -1051,6 +1071,9 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
                        int64_t d_in, int64_t d_out, int r, float alpha, void *ws, size_t ws_bytes, void *stream) {
     LORA_TRY(check_shapes(M, d_in, d_out, r, alpha, wt.wf));
     if (!dY || !x || !wt.present() || !A || !B || !dA || !dB) return LORA_ERR_INVALID_ARG;
+    if (wt.wf == WF_CB)
+        for (int i = 0; i < 16; ++i)
+            if (!std::isfinite(wt.codebook[i])) return LORA_ERR_INVALID_ARG;
     if (!aligned16(dY) || !aligned16(x) || !wt.aligned() || !aligned16(A) || !aligned16(B) || !aligned16(dA) ||
         !aligned16(dB) || (xa_save && !aligned16(xa_save)) || (dX && !aligned16(dX)))
         return LORA_ERR_MISALIGNED;
@@ -1106,8 +1129,8 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
 extern "C" {
 
 size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r) {
-    if (op < LORA_OP_FWD || op > LORA_OP_BWD_FP8) return 0;
-    const int wf = op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
+    if (op < LORA_OP_FWD || op > LORA_OP_BWD_NF4) return 0;
+    const int wf = op >= LORA_OP_FWD_NF4 ? WF_CB : op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
     if (check_shapes(M, d_in, d_out, r, 1.0f, wf) != LORA_OK) return 0;
     Plan pl;
     make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
@@ -1218,13 +1241,13 @@ lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r
 }
 
 lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, lora_plan_t *plan) {
-    if (!plan || op < LORA_OP_FWD || op > LORA_OP_BWD_FP8) return LORA_ERR_INVALID_ARG;
-    const int wf = op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
+    if (!plan || op < LORA_OP_FWD || op > LORA_OP_BWD_NF4) return LORA_ERR_INVALID_ARG;
+    const int wf = op >= LORA_OP_FWD_NF4 ? WF_CB : op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
     if (check_shapes(M, d_in, d_out, r, 1.0f, wf) != LORA_OK) return LORA_ERR_INVALID_ARG;
     Plan pl;
     make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
     std::memset(plan, 0, sizeof(*plan));
-    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8);
+    const bool bwd = (op == LORA_OP_BWD || op == LORA_OP_BWD_Q4 || op == LORA_OP_BWD_FP8 || op == LORA_OP_BWD_NF4);
     plan->side_fwd = pl.side ? 1 : 2;
     plan->side_bwd = bwd ? (pl.side_bwd ? 1 : 2) : 0;
     plan->xa_cluster = pl.side ? pl.sx.C : 0;
@@ -1243,6 +1266,34 @@ lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_ou
     plan->splitk[2] = sk_bwd ? pl.s_db.splits : 0;
     plan->splitk[3] = sk_bwd ? pl.s_da.splits : 0;
     return LORA_OK;
+}
+
+lora_status_t lora_linear_fwd_nf4(const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale, const float *codebook,
+                                  const uint16_t *A, const uint16_t *B, uint16_t *h, uint16_t *xa_save, int64_t M,
+                                  int64_t d_in, int64_t d_out, int r, float alpha, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    Weight wt;
+    wt.Wq = Wq;
+    wt.Wscale = Wscale;
+    wt.codebook = codebook;
+    wt.wf = WF_CB;
+    if (!Wq || !Wscale || !codebook) return LORA_ERR_INVALID_ARG;
+    return fwd_impl(x, wt, A, B, h, xa_save, M, d_in, d_out, r, alpha, workspace, workspace_bytes, stream);
+}
+
+lora_status_t lora_linear_bwd_nf4(const uint16_t *dY, const uint16_t *x, const uint8_t *Wq, const uint16_t *Wscale,
+                                  const float *codebook, const uint16_t *A, const uint16_t *B,
+                                  const uint16_t *xa_save, uint16_t *dX, float *dA, float *dB, int64_t M,
+                                  int64_t d_in, int64_t d_out, int r, float alpha, void *workspace,
+                                  size_t workspace_bytes, void *stream) {
+    Weight wt;
+    wt.Wq = Wq;
+    wt.Wscale = Wscale;
+    wt.codebook = codebook;
+    wt.wf = WF_CB;
+    if (!Wq || !Wscale || !codebook) return LORA_ERR_INVALID_ARG;
+    return bwd_impl(dY, x, wt, A, B, xa_save, dX, dA, dB, M, d_in, d_out, r, alpha, workspace, workspace_bytes,
+                    stream);
 }
 
 lora_status_t lora_linear_check(void *workspace, void *stream) {

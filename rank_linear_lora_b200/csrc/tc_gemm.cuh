@@ -101,6 +101,7 @@ struct GemmArgs {
     const uint16_t *wscale;
     int scale_ld;
     int scale_rows;
+    float cb[16];            // 4-bit codebook weight: the 16 values of the code
     int *err;                // device error word
     unsigned long long *trace;  // optional per-CTA timestamps (TRACE_WORDS each), or null
     // 1: this kernel reads nothing its stream predecessor writes, so it starts its work

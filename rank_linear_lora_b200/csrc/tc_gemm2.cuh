@@ -44,8 +44,9 @@ constexpr int DQ_GROUPS = DQ_WARPS / DQ_GROUP_WARPS;       // groups that take K
 constexpr int DQ_QDEPTH = 1;         // packed-code slots per dequant warp (own K blocks in flight)
 constexpr int DQ_QROWS = 32 * DQ_RUNS;                     // runs fetched per warp and K block
 
-// Frozen-weight formats of the pair GEMM.
-enum WeightFmt { WF_BF16 = 0, WF_Q4 = 1, WF_FP8 = 2 };
+// Frozen-weight formats of the pair GEMM: bf16, the linear 4-bit code, FP8 E4M3, and a
+// 4-bit code decoded through a 16-value codebook (e.g. NF4).
+enum WeightFmt { WF_BF16 = 0, WF_Q4 = 1, WF_FP8 = 2, WF_CB = 3 };
 // Bytes of codes per run of 64 weights: two 4-bit codes per byte, or one E4M3 code per byte.
 __host__ __device__ constexpr int dq_run_bytes(int wf) { return wf == WF_FP8 ? 64 : 32; }
 // One packed-code slot of a dequant warp: DQ_QROWS runs.
@@ -142,6 +143,56 @@ __device__ __forceinline__ uint4 fp8_decode8(uint32_t w0, uint32_t w1, float sc)
     r.y = fp8_pair(w0 >> 16, sc);
     r.z = fp8_pair(w1 & 0xFFFFu, sc);
     r.w = fp8_pair(w1 >> 16, sc);
+    return r;
+}
+
+// 4-bit codebook decode.  The 16 values of a run's table, codebook[i] * scale rounded
+// once to bf16, are held as byte tables: lo[t] / hi[t] hold the low / high bytes of
+// entries 4t .. 4t+3.  A prmt picks 4 bytes from 8 by 3-bit selectors, so entries 0-7
+// and 8-15 are looked up separately and bit 3 of each code chooses between them.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+struct CbTable {
+    uint32_t lo[4], hi[4];
+};
+__device__ __forceinline__ CbTable cb_table(const float (&cb)[16], float sc) {
+    CbTable t;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {  // entries 4q .. 4q+3
+        uint32_t w0, w1;           // bf16x2 (entry 4q+1 : 4q), (4q+3 : 4q+2)
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w0) : "f"(cb[4 * q + 1] * sc), "f"(cb[4 * q] * sc));
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w1) : "f"(cb[4 * q + 3] * sc), "f"(cb[4 * q + 2] * sc));
+        t.lo[q] = prmt(w0, w1, 0x6420);
+        t.hi[q] = prmt(w0, w1, 0x7531);
+    }
+    return t;
+}
+// Codes c0..c3 in the low nibbles of the bytes of v -> the low (L) and high (H) bytes of
+// their four bf16 table values, byte i for code i.
+__device__ __forceinline__ void cb_look4(const CbTable &t, uint32_t v, uint32_t &L, uint32_t &H) {
+    const uint32_t x = v & 0x07070707u;
+    const uint32_t sel = prmt(x | (x >> 4), 0u, 0x4420);  // nibble i = c_i & 7
+    const uint32_t m = prmt(v << 4, 0u, 0xBA98);          // byte i = 0xFF where c_i >= 8
+    const uint32_t l0 = prmt(t.lo[0], t.lo[1], sel), l1 = prmt(t.lo[2], t.lo[3], sel);
+    const uint32_t h0 = prmt(t.hi[0], t.hi[1], sel), h1 = prmt(t.hi[2], t.hi[3], sel);
+    L = (l0 & ~m) | (l1 & m);
+    H = (h0 & ~m) | (h1 & m);
+}
+// One 32-bit word of 4-bit codes (element i in bits 4i..4i+3) to 8 bf16 table values.
+__device__ __forceinline__ uint4 cb_decode8(const CbTable &t, uint32_t word) {
+    uint32_t Le, He, Lo, Ho;
+    cb_look4(t, word & 0x0F0F0F0Fu, Le, He);          // elements 0, 2, 4, 6
+    cb_look4(t, (word >> 4) & 0x0F0F0F0Fu, Lo, Ho);   // elements 1, 3, 5, 7
+    const uint32_t ev01 = prmt(Le, He, 0x5140), od01 = prmt(Lo, Ho, 0x5140);  // {e0, e2}, {e1, e3}
+    const uint32_t ev23 = prmt(Le, He, 0x7362), od23 = prmt(Lo, Ho, 0x7362);  // {e4, e6}, {e5, e7}
+    uint4 r;
+    r.x = prmt(ev01, od01, 0x5410);
+    r.y = prmt(ev01, od01, 0x7632);
+    r.z = prmt(ev23, od23, 0x5410);
+    r.w = prmt(ev23, od23, 0x7632);
     return r;
 }
 
@@ -547,6 +598,13 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                         *reinterpret_cast<uint4 *>(row + (((2 * h) ^ (rn & 7)) * 16)) = fp8_decode8(v.x, v.y, sc_f);
                         *reinterpret_cast<uint4 *>(row + (((2 * h + 1) ^ (rn & 7)) * 16)) = fp8_decode8(v.z, v.w, sc_f);
                     }
+                } else if constexpr (WF == WF_CB) {
+                    const CbTable tb = cb_table(p.cb, __uint_as_float(sc[i] << 16));
+                    const uint4 v0 = src[0], v1 = src[1];
+                    const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = cb_decode8(tb, wds[c]);
                 } else {
                     const uint4 v0 = src[0], v1 = src[1];
                     const float s7 = __uint_as_float(sc[i] << 16) / 7.0f;

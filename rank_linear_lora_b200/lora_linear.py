@@ -21,7 +21,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "lora_linear.h")
 LORA_OK = 0
 STATUS = {0: "LORA_OK", 1: "LORA_ERR_INVALID_ARG", 2: "LORA_ERR_MISALIGNED", 3: "LORA_ERR_UNSUPPORTED",
           4: "LORA_ERR_WORKSPACE", 5: "LORA_ERR_CUDA", 6: "LORA_ERR_TIMEOUT"}
-OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4, OP_FWD_FP8, OP_BWD_FP8 = 0, 1, 2, 3, 4, 5
+OP_FWD, OP_BWD, OP_FWD_Q4, OP_BWD_Q4, OP_FWD_FP8, OP_BWD_FP8, OP_FWD_NF4, OP_BWD_NF4 = 0, 1, 2, 3, 4, 5, 6, 7
 KERNEL_KINDS = ["xa", "fwd_main", "g", "dx_main", "dadb"]
 
 
@@ -50,9 +50,11 @@ def load_library():
     lib.lora_linear_fwd_q4.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     lib.lora_linear_bwd_q4.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     lib.lora_linear_fwd_fp8.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_fwd_nf4.argtypes = [P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
+    lib.lora_linear_bwd_nf4.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     lib.lora_linear_bwd_fp8.argtypes = [P, P, P, P, P, P, P, P, P, P, I64, I64, I64, I, F, P, SZ, P]
     for f in ("lora_linear_fwd", "lora_linear_bwd", "lora_linear_fwd_q4", "lora_linear_bwd_q4", "lora_linear_fwd_fp8",
-              "lora_linear_bwd_fp8"):
+              "lora_linear_bwd_fp8", "lora_linear_fwd_nf4", "lora_linear_bwd_nf4"):
         getattr(lib, f).restype = I
     lib.lora_linear_check.argtypes = [P, P]
     lib.lora_linear_check.restype = I
@@ -294,6 +296,55 @@ def lora_linear_get_plan(op: int, M: int, d_in: int, d_out: int, r: int) -> dict
     p = lora_plan_t()
     _check(fn(op, M, d_in, d_out, r, ctypes.byref(p)), "lora_linear_get_plan")
     return p.as_dict()
+
+
+def _codebook(codebook):
+    """16 host float32 values (any sequence; a CUDA tensor is copied to the host)."""
+    import numpy as np
+    cb = codebook.detach().cpu().numpy() if isinstance(codebook, torch.Tensor) else codebook
+    cb = np.ascontiguousarray(np.asarray(cb, dtype=np.float32).reshape(-1))
+    if cb.shape != (16,):
+        raise ValueError("codebook: expected 16 values")
+    return cb, cb.ctypes.data_as(ctypes.c_void_p)
+
+
+def lora_linear_fwd_nf4(x, Wq, Wscale, codebook, A, B, h, xa_save, alpha, ws, stream=None):
+    """Forward with a 4-bit codebook weight (e.g. NF4): w' = codebook[q] * Wscale[n, k/64]."""
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = Wq.shape[0]
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r)), (h, "h", (M, d_out))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    keep, cbp = _codebook(codebook)
+    st = load_library().lora_linear_fwd_nf4(_ptr(x), _ptr(Wq), _ptr(Wscale), cbp, _ptr(A), _ptr(B), _ptr(h),
+                                            _ptr(xa_save), M, d_in, d_out, r, float(alpha), *_ws(ws),
+                                            _stream(stream))
+    del keep
+    _check(st, "lora_linear_fwd_nf4")
+
+
+def lora_linear_bwd_nf4(dY, x, Wq, Wscale, codebook, A, B, xa_save, dX, dA, dB, alpha, ws, stream=None):
+    M, d_in = x.shape
+    r = A.shape[0]
+    d_out = Wq.shape[0]
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((dY, "dY", (M, d_out)), (x, "x", (M, d_in)), (A, "A", (r, d_in)), (B, "B", (d_out, r))):
+        _bf16(t, n, s)
+    if xa_save is not None:
+        _bf16(xa_save, "xa_save", (M, r))
+    if dX is not None:
+        _bf16(dX, "dX", (M, d_in))
+    _f32(dA, "dA", (r, d_in))
+    _f32(dB, "dB", (d_out, r))
+    keep, cbp = _codebook(codebook)
+    st = load_library().lora_linear_bwd_nf4(_ptr(dY), _ptr(x), _ptr(Wq), _ptr(Wscale), cbp, _ptr(A), _ptr(B),
+                                            _ptr(xa_save), _ptr(dX), _ptr(dA), _ptr(dB), M, d_in, d_out, r,
+                                            float(alpha), *_ws(ws), _stream(stream))
+    del keep
+    _check(st, "lora_linear_bwd_nf4")
 
 
 def lora_linear_check(ws, stream=None):

@@ -41,8 +41,9 @@ class DeviceLayer:
         self.x, self.A, self.B, self.dY = (dev_bf16(a) for a in (inp.x, inp.A, inp.B, inp.dY))
         self.q4 = sp.q4
         self.fp8 = getattr(sp, "fp8", False)
+        self.nf4 = getattr(sp, "nf4", False)
         self.W = None
-        if sp.q4:
+        if sp.q4 or self.nf4:
             self.Wq, self.Wscale = dev_u8(inp.Wq), dev_bf16(inp.Wscale)
         elif self.fp8:
             self.W8, self.W8scale = dev_u8(inp.W8), dev_bf16(inp.W8scale)
@@ -55,7 +56,7 @@ class DeviceLayer:
         self.dA = torch.empty(r, di, dtype=torch.float32, device="cuda")
         self.dB = torch.empty(do, r, dtype=torch.float32, device="cuda")
         fop, bop = ((L.OP_FWD_Q4, L.OP_BWD_Q4) if sp.q4 else (L.OP_FWD_FP8, L.OP_BWD_FP8) if self.fp8
-                    else (L.OP_FWD, L.OP_BWD))
+                    else (L.OP_FWD_NF4, L.OP_BWD_NF4) if self.nf4 else (L.OP_FWD, L.OP_BWD))
         self.ws_f = L.workspace(fop, M, di, do, r)
         self.ws_b = L.workspace(bop, M, di, do, r)
 
@@ -66,6 +67,9 @@ class DeviceLayer:
         elif self.fp8:
             L.lora_linear_fwd_fp8(self.x, self.W8, self.W8scale, self.A, self.B, self.h, xa, self.spec.alpha,
                                   self.ws_f)
+        elif self.nf4:
+            L.lora_linear_fwd_nf4(self.x, self.Wq, self.Wscale, self.inp.codebook, self.A, self.B, self.h, xa,
+                                  self.spec.alpha, self.ws_f)
         else:
             L.lora_linear_fwd(self.x, self.W, self.A, self.B, self.h, xa, self.spec.alpha, self.ws_f)
 
@@ -78,6 +82,9 @@ class DeviceLayer:
         elif self.fp8:
             L.lora_linear_bwd_fp8(self.dY, self.x, self.W8, self.W8scale, self.A, self.B, xa, dX, self.dA, self.dB,
                                   self.spec.alpha, self.ws_b)
+        elif self.nf4:
+            L.lora_linear_bwd_nf4(self.dY, self.x, self.Wq, self.Wscale, self.inp.codebook, self.A, self.B, xa, dX,
+                                  self.dA, self.dB, self.spec.alpha, self.ws_b)
         else:
             L.lora_linear_bwd(self.dY, self.x, self.W, self.A, self.B, xa, dX, self.dA, self.dB, self.spec.alpha,
                               self.ws_b)
@@ -103,14 +110,21 @@ def shared_input_projections(M, d_in, d_outs, r, alpha, q4, seed) -> list:
     return layers
 
 
-def oracle_ref(inp: inputs.LayerInputs, rows=None) -> dict:
+def weight_kwargs(inp: inputs.LayerInputs) -> dict:
+    """The oracle's keyword arguments for a layer's frozen weight, in its format."""
     sp = inp.spec
     if sp.q4:
-        wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale)
-    elif sp.fp8:
-        wkw = dict(W8=inp.W8, W8scale=inp.W8scale)
-    else:
-        wkw = dict(W=inp.W)
+        return dict(Wq=inp.Wq, Wscale=inp.Wscale)
+    if getattr(sp, "fp8", False):
+        return dict(W8=inp.W8, W8scale=inp.W8scale)
+    if getattr(sp, "nf4", False):
+        return dict(Wq=inp.Wq, Wscale=inp.Wscale, codebook=inp.codebook)
+    return dict(W=inp.W)
+
+
+def oracle_ref(inp: inputs.LayerInputs, rows=None) -> dict:
+    sp = inp.spec
+    wkw = weight_kwargs(inp)
     h, xa = oracle.forward(inp.x, inp.A, inp.B, sp.s, rows=rows, **wkw)
     bw = oracle.backward(inp.dY, inp.x, inp.A, inp.B, sp.s, rows=rows, xa_=xa, **wkw)
     return {"h": h, "xa": xa, "dX": bw["dX"], "dA": bw["dA"], "dB": bw["dB"], "g": bw["g"]}
@@ -160,8 +174,7 @@ def check_projections(dl: "DeviceLayer", inp: inputs.LayerInputs, ref: dict, see
     sp = inp.spec
     rng = np.random.default_rng(0xC0DE + seed)
     M, di, do = sp.M, sp.d_in, sp.d_out
-    wkw = (dict(Wq=inp.Wq, Wscale=inp.Wscale) if sp.q4 else dict(W8=inp.W8, W8scale=inp.W8scale)
-           if getattr(sp, "fp8", False) else dict(W=inp.W))
+    wkw = weight_kwargs(inp)
     u = rng.choice([-1.0, 1.0], M)
     v_h = rng.choice([-1.0, 1.0], do)
     v_x = rng.choice([-1.0, 1.0], di)
@@ -231,12 +244,7 @@ def compare_every_element(dl: "DeviceLayer", inp: inputs.LayerInputs, block_rows
     primitive), a block of rows at a time.  Returns the worst error / bound per output
     and the oracle's wall time."""
     sp = inp.spec
-    if sp.q4:
-        wkw = dict(Wq=inp.Wq, Wscale=inp.Wscale)
-    elif getattr(sp, "fp8", False):
-        wkw = dict(W8=inp.W8, W8scale=inp.W8scale)
-    else:
-        wkw = dict(W=inp.W)
+    wkw = weight_kwargs(inp)
     if torch.cuda.is_available():
         torch.cuda.synchronize()
     t_oracle = 0.0

@@ -42,7 +42,7 @@ def test_workspace_sizes(lib):
     assert L.lora_linear_workspace_size(L.OP_FWD, 64, 256, 256, 12) == 0
     assert L.lora_linear_workspace_size(L.OP_FWD, 64, 256, 256, 264) == 0
     assert L.lora_linear_workspace_size(L.OP_FWD_Q4, 64, 96, 256, 8) == 0
-    assert L.lora_linear_workspace_size(7, 64, 256, 256, 8) == 0
+    assert L.lora_linear_workspace_size(8, 64, 256, 256, 8) == 0
 
 
 def _fwd(lib, x=0x1000, W=0x2000, A=0x3000, B_=0x4000, h=0x5000, xa=None, M=64, di=256, do=256, r=8,
@@ -124,7 +124,7 @@ def test_fp8_validation_before_any_device_work(lib):
             op - 4, 4096, 4096, 4096, 8)  # the workspace does not depend on the weight's format
     assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1040, 256, 8) > 0      # d_in % 16 == 0 suffices
     assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1032, 256, 8) == 0     # d_in % 16 != 0
-    assert L.lora_linear_workspace_size(6, 64, 256, 256, 8) == 0
+    assert L.lora_linear_workspace_size(8, 64, 256, 256, 8) == 0
     P = ctypes.c_void_p
     fn = lib.lora_linear_fwd_fp8
 
@@ -139,3 +139,30 @@ def test_fp8_validation_before_any_device_work(lib):
     st = lib.lora_linear_bwd_fp8(P(0x1000), P(0x1000), P(0x2000), P(0x2800), P(0x3000), P(0x4000), None, None,
                                  None, P(0x7000), 64, 256, 256, 8, 16.0, P(0x10000), 1 << 30, None)
     assert st == 1  # dA is required
+
+
+def test_nf4_validation_before_any_device_work(lib):
+    """The 4-bit codebook entry points: workspace sizes, and argument checks (codes,
+    scales and a host codebook of finite values required, d_in % 64 == 0) before any
+    launch."""
+    import numpy as np
+    assert {"lora_linear_fwd_nf4", "lora_linear_bwd_nf4"} <= set(L.declared_functions())
+    for op in (L.OP_FWD_NF4, L.OP_BWD_NF4):
+        assert L.lora_linear_workspace_size(op, 4096, 8192, 28672, 16) == L.lora_linear_workspace_size(
+            op - 4, 4096, 8192, 28672, 16)
+    assert L.lora_linear_workspace_size(L.OP_FWD_NF4, 64, 96, 256, 8) == 0  # d_in % 64 != 0
+    P = ctypes.c_void_p
+    cb = np.linspace(-1, 1, 16).astype(np.float32)
+    bad = cb.copy()
+    bad[5] = np.nan
+    fn = lib.lora_linear_fwd_nf4
+
+    def fwd(codebook=cb, Wq=0x2000, di=256):
+        cbp = None if codebook is None else codebook.ctypes.data_as(P)
+        return fn(P(0x1000), P(Wq), P(0x2800), cbp, P(0x3000), P(0x4000), P(0x5000), None, 64, di, 256, 8, 16.0,
+                  P(0x10000), 1 << 30, None)
+    assert fwd(codebook=None) == 1
+    assert fwd(codebook=bad) == 1
+    assert fwd(Wq=None) == 1
+    assert fwd(di=288) == 1        # not a multiple of 64
+    assert fwd(Wq=0x2004) == 2

@@ -382,3 +382,55 @@ def test_fp8_full_size_every_element(idx):
     res = compare_every_element(dl, inp)
     print(f"{spec.name} fp8: {res['elements']} elements, oracle {res['oracle_s']:.1f} s; worst error / bound "
           + ", ".join(f"{k} {v:.3f}" for k, v in res["worst"].items()))
+
+
+# 4-bit codebook weight (NF4 codebook): codes decoded through the 16-value table in
+# shared memory inside both main GEMMs; every element against the oracle's format 3.
+NF4_SHAPES = [
+    (200, 320, 200, 16),     # ragged M and d_out
+    (520, 512, 768, 24),     # rank tail r % 16 != 0
+    (1100, 640, 4000, 16),   # forward: several work items per CTA pair
+    (1100, 4096, 1000, 16),  # dX: K = d_out ragged
+]
+
+
+@pytest.mark.parametrize("shape", NF4_SHAPES, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_nf4_every_element(shape):
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("nf4", M, di, do, r, alpha=2.0 * r, nf4=True, seed=0x4F4 + M)
+    inp, dl = _run_full(spec)
+    compare_every_element(dl, inp)
+
+
+def test_nf4_weight_dominated_every_code():
+    """B = 0: h and dX are the decoded weight's products alone, and the weight uses all
+    16 codes, so a wrong table entry, byte order or half-table choice shows."""
+    spec = inputs.LayerSpec("nf4w", 256, 192, 320, 8, alpha=16.0, nf4=True, seed=0x4F5)
+    inp, dl = _run_full(spec, zero_B=True)
+    assert len(np.unique(inputs.unpack_q4_codes(inp.Wq))) == 16
+    compare_every_element(dl, inp)
+
+
+def test_nf4_full_size_every_element():
+    """The up projection's size (M=4096, 8192 -> 28672, r=16) with the NF4 weight."""
+    spec = inputs.workload(4).layers[0].with_(q4=False, nf4=True)
+    inp, dl = _run_full(spec)
+    res = compare_every_element(dl, inp)
+    print(f"{spec.name} nf4: {res['elements']} elements, oracle {res['oracle_s']:.1f} s; worst error / bound "
+          + ", ".join(f"{k} {v:.3f}" for k, v in res["worst"].items()))
+
+
+@pytest.mark.parametrize("shape", [(1024, 512, 3000, 32), (520, 640, 768, 24), (2048, 2048, 2048, 32)],
+                         ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_one_pass_backward_at_ranks_above_the_default(shape):
+    """s.g + dB in one pass over dY, and dA, at r = 24 and 32 (64-byte swizzled narrow
+    operands, N = 32), which a plan selects (the library's own choice is split-K there)."""
+    M, di, do, r = shape
+    L.lora_linear_set_plan(M, di, do, r, dict(side_bwd=1))
+    try:
+        assert L.lora_linear_get_plan(L.OP_BWD, M, di, do, r)["side_bwd"] == 1
+        spec = inputs.LayerSpec("onepass", M, di, do, r, alpha=2.0 * r, seed=0x1BA + M)
+        inp, dl = _run_full(spec)
+        compare_every_element(dl, inp)
+    finally:
+        L.lora_linear_set_plan(M, di, do, r, None)
