@@ -6,14 +6,13 @@
 // "UnSloth加速库集成：编译级优化带来的性能飞跃", section 为什么标准LoRA会慢？).  The
 // 4-bit variant starts from the decoded code, w = (q - 8) * scale / 7.
 //
-// The work is one read of W and one write of W' (HBM-bound); the rank-r update costs r
-// FMAs per element.  One CTA of 256 threads owns a 32-row x 256-column tile: it stages
-// its 32 rows of B and the 256-column panel of A in shared memory, 64 ranks at a time,
-// and each thread accumulates a 4-row x 8-column micro-tile in fp32 (bf16 products are
-// exact in fp32), adds the weight in fp32 and rounds once to bf16.  Every global access
-// is a 16-byte vector of 8 consecutive columns; a warp covers 256 columns of one row
-// (coalesced).  W' may be W itself (in place): a CTA reads each element of its tile
-// before it writes it, and tiles are disjoint.
+// The work is one read of W and one write of W' (HBM-bound).  Up to r = 64 the rank-r
+// update runs on the tensor cores (k_merge_tc: a tcgen05 contraction over the ranks into
+// TMEM, the weight added in the epilogue, TMA in and out); wider ranks take k_merge, a
+// CUDA-core kernel whose threads accumulate 4-row x 8-column micro-tiles in fp32.  Both
+// add the weight in fp32 and round once to bf16 (bf16 products are exact in fp32).  W'
+// may be W itself (in place): a tile is read before it is written, and tiles are
+// disjoint.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -147,166 +146,282 @@ __global__ void __launch_bounds__(THREADS) k_merge(const uint16_t *W, const uint
     }
 }
 
-// ---------------------------------------------------------------- TMA-fed ring (r <= 64)
-// The simple kernel above keeps only ~48 KB in flight per SM (three resident CTAs, a
-// 16 KB tile each), which at the loaded DRAM latency holds it near 2.5 TB/s.  Here one
-// persistent CTA per SM runs a ring of stages: a producer thread TMA-loads each tile's
-// weight (bf16 16 KB, or 4 KB of codes), its A panel (r x 256) and its 32 rows of B
-// into a free stage, ~100 KB ahead of its eight consumer warps (two CTAs per SM), which compute from
-// shared memory exactly as the simple kernel does and store W'.  All waits are bounded
-// (2 s); a timeout sets g_merge_err, read by lora_linear_merge_check.
-constexpr int CONSUMERS = 8;
-constexpr int THREADS_TMA = 32 * (CONSUMERS + 1);
-constexpr int MAX_STAGES = 8;
-constexpr int RING_SMEM = 110 * 1024;  // per CTA; two CTAs (16 consumer warps) per SM
+// ---------------------------------------------------------------- tensor cores (r <= 64)
+// The kernel above spends ~14 instructions per element on the rank-r update (shared-memory
+// operand loads, widening, r FMAs) and is issue-bound at less than half the HBM bandwidth.
+// Here the update s * B . A of a 128-row x 128-column tile is one to four tcgen05 MMAs
+// (M = 128, N = 128, K = 16 ranks each) into an fp32 TMEM accumulator, and the epilogue
+// only adds the weight: tcgen05.ld of 32 columns, the weight from the TMA-staged tile in
+// shared memory, one fp32 FMA and one rounding per element, the result written over the
+// staged tile (bf16 weight) or into a staging tile (4-bit weight), then TMA-stored.
+// Roles as in the layer's kernels: warp 0 the TMA producer, warp 1 TMEM and the
+// single-thread MMA issue, warps 2..5 the epilogue (one accumulator row each thread);
+// three stages of operands, two TMEM accumulators.  Persistent, one CTA per SM, tiles in
+// row-major order.  128 columns rather than 256: a 4096 x 4096 weight is 1024 tiles, 6.9
+// per SM, where 256-column tiles would leave 14% of the SMs' time on a partial last wave.
+// Every wait is bounded (2 s); a timeout sets g_merge_err (lora_linear_merge_check).
+constexpr int TC_M = 128, TC_N = 128, TC_STAGES = 3, TC_ACC = 2, TC_THREADS = 192;
+constexpr int TC_CHUNKS = TC_N / 64;              // 64-column chunks (one 128B-swizzle box each)
+constexpr int TC_W_BYTES = TC_M * TC_N * 2;       // bf16 weight tile, or an output staging tile
+constexpr int TC_Q_BYTES = TC_M * TC_N / 2;       // 4-bit codes of the tile
+constexpr int TC_B_BYTES = TC_M * 64 * 2;         // B rows [128 x 64 ranks], K-major, 128B swizzle
+constexpr int TC_A_BYTES = TC_CHUNKS * 64 * 128;  // A panel: 64-column chunks x 64 ranks, MN-major
 
 __device__ int g_merge_err;
 
 struct MergeArgs {
-    CUtensorMap tmW;  // bf16 W [d_out][d_in] box {256, 32}, or codes uint8 [d_out][d_in/2] box {128, 32}
-    CUtensorMap tmA;  // bf16 A [r][d_in], box {256, r}
-    CUtensorMap tmB;  // bf16 B [d_out][r], box {r, 32}
-    const uint16_t *Wscale;
-    uint16_t *Wout;
+    CUtensorMap tmW;    // bf16 W [d_out][d_in] box {64, 128}, 128B swizzle; or codes uint8 [d_out][d_in/2] box {64, 128}
+    CUtensorMap tmOut;  // bf16 W' [d_out][d_in] box {64, 128}, 128B swizzle
+    CUtensorMap tmA;    // bf16 A [r][d_in] box {64, kr}, 128B swizzle (the MMA's MN-major B operand)
+    CUtensorMap tmB;    // bf16 B [d_out][r] box {64, 128}, 128B swizzle (the MMA's K-major A operand)
+    const uint16_t *Wscale;  // 4-bit weight: bf16 [d_out][d_in/64]
     int64_t d_in, d_out, col_tiles, tiles;
-    int r, stages;
-    uint32_t w_bytes, a_bytes, stage_bytes;
+    int kr;             // r rounded up to 16 (the MMAs' K); ranks past r are zero-filled by TMA
     float s;
     int *err;
 };
 
 template <bool Q4>
-__global__ void __launch_bounds__(THREADS_TMA, 2) k_merge_ring(const __grid_constant__ MergeArgs p) {
+struct MergeCfg {
+    static constexpr int WSTAGE = Q4 ? TC_Q_BYTES : TC_W_BYTES;
+    static constexpr int STAGE_BYTES = WSTAGE + TC_B_BYTES + TC_A_BYTES;
+    static constexpr int STAGING = Q4 ? 2 * TC_W_BYTES : 0;  // 4-bit weight: output tiles staged apart
+    static constexpr int SMEM_BYTES = 1024 + TC_STAGES * STAGE_BYTES + STAGING + 256;
+    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled boxes");
+    static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
+};
+
+template <bool Q4>
+__global__ void __launch_bounds__(TC_THREADS, 1) k_merge_tc(const __grid_constant__ MergeArgs p) {
+    using Cfg = MergeCfg<Q4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full_bar = reinterpret_cast<uint64_t *>(smem + p.stages * p.stage_bytes);  // [stages]
-    uint64_t *empty_bar = full_bar + MAX_STAGES;                                        // [stages]
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty_bar + MAX_STAGES);
+    uint8_t *staging = smem + TC_STAGES * Cfg::STAGE_BYTES;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(staging + Cfg::STAGING);
+    uint64_t *full_bar = bars;                      // [stages] the tile's operands landed
+    uint64_t *empty_bar = bars + TC_STAGES;         // [stages] the stage (and its store) is done with
+    uint64_t *tfull_bar = bars + 2 * TC_STAGES;     // [acc] accumulator ready
+    uint64_t *tempty_bar = tfull_bar + TC_ACC;      // [acc] accumulator drained
+    uint64_t *drain_bar = tempty_bar + TC_ACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
     if (threadIdx.x == 0) {
-        for (int st = 0; st < p.stages; ++st) {
-            lora::mbar_init(lora::smem_u32(&full_bar[st]), 1);
-            lora::mbar_init(lora::smem_u32(&empty_bar[st]), CONSUMERS);
+        for (int b = 0; b < TC_STAGES; ++b) {
+            lora::mbar_init(lora::smem_u32(&full_bar[b]), 1);
+            lora::mbar_init(lora::smem_u32(&empty_bar[b]), 1);
         }
+        for (int b = 0; b < TC_ACC; ++b) {
+            lora::mbar_init(lora::smem_u32(&tfull_bar[b]), 1);
+            lora::mbar_init(lora::smem_u32(&tempty_bar[b]), 4);
+        }
+        lora::mbar_init(lora::smem_u32(drain_bar), 1);
         *abort_flag = 0;
         lora::fence_mbar_init();
     }
+    if (warp == 0 && lane == 0) {
+        lora::tma_prefetch_desc(&p.tmW);
+        lora::tma_prefetch_desc(&p.tmOut);
+        lora::tma_prefetch_desc(&p.tmA);
+        lora::tma_prefetch_desc(&p.tmB);
+    }
+    if (warp == 1) {
+        lora::tmem_alloc(lora::smem_u32(tmem_slot), TC_ACC * TC_N);
+        lora::tmem_relinquish();
+    }
+    lora::tc_fence_before();
     __syncthreads();
+    lora::tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == CONSUMERS) {
-        // ---------------------------------------------------------------- producer
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            lora::tma_prefetch_desc(&p.tmW);
-            lora::tma_prefetch_desc(&p.tmA);
-            lora::tma_prefetch_desc(&p.tmB);
+            uint32_t issued = 0, issued_phase = 0;
             int k = 0;
             for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
-                const int st = k % p.stages;
-                const uint32_t ph = static_cast<uint32_t>(k / p.stages) & 1u;
+                const int st = k % TC_STAGES;
+                const uint32_t ph = static_cast<uint32_t>(k / TC_STAGES) & 1u;
                 if (!lora::wait_bounded(lora::smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag, p.err,
                                         lora::DERR_WAIT_EMPTY))
                     break;
-                const int row0 = static_cast<int>((t / p.col_tiles) * MT);
-                const int col0 = static_cast<int>((t % p.col_tiles) * NT);
-                uint8_t *base = smem + st * p.stage_bytes;
+                const int row0 = static_cast<int>((t / p.col_tiles) * TC_M);
+                const int col0 = static_cast<int>((t % p.col_tiles) * TC_N);
+                uint8_t *base = smem + st * Cfg::STAGE_BYTES;
                 const uint32_t fb = lora::smem_u32(&full_bar[st]);
-                lora::mbar_arrive_expect_tx(fb, p.stage_bytes);
-                lora::tma_load_2d(lora::smem_u32(base), &p.tmW, fb, Q4 ? col0 / 2 : col0, row0);
-                lora::tma_load_2d(lora::smem_u32(base + p.w_bytes), &p.tmA, fb, col0, 0);
-                lora::tma_load_2d(lora::smem_u32(base + p.w_bytes + p.a_bytes), &p.tmB, fb, 0, row0);
+                lora::mbar_arrive_expect_tx(
+                    fb, Cfg::WSTAGE + TC_B_BYTES + static_cast<uint32_t>(TC_CHUNKS * 128 * p.kr));
+                if (Q4) {
+                    lora::tma_load_2d(lora::smem_u32(base), &p.tmW, fb, col0 / 2, row0);
+                } else {
+                    for (int j = 0; j < TC_CHUNKS; ++j)
+                        lora::tma_load_2d(lora::smem_u32(base + j * 16384), &p.tmW, fb, col0 + 64 * j, row0);
+                }
+                lora::tma_load_2d(lora::smem_u32(base + Cfg::WSTAGE), &p.tmB, fb, 0, row0);
+                for (int j = 0; j < TC_CHUNKS; ++j)
+                    lora::tma_load_2d(lora::smem_u32(base + Cfg::WSTAGE + TC_B_BYTES + j * 8192), &p.tmA, fb,
+                                      col0 + 64 * j, 0);
+                issued |= 1u << st;
+                issued_phase = (issued_phase & ~(1u << st)) | (ph << st);
             }
             // copies still in flight (only after a failed wait) land before the CTA exits
-            for (int j = k > p.stages ? k - p.stages : 0; j < k; ++j) {
-                volatile int never = 0;
-                lora::wait_bounded(lora::smem_u32(&full_bar[j % p.stages]),
-                                   static_cast<uint32_t>(j / p.stages) & 1u, &never, p.err, lora::DERR_WAIT_DRAIN);
-            }
+            for (int st = 0; st < TC_STAGES; ++st)
+                if (issued & (1u << st)) {
+                    volatile int never = 0;
+                    lora::wait_bounded(lora::smem_u32(&full_bar[st]), (issued_phase >> st) & 1u, &never, p.err,
+                                       lora::DERR_WAIT_DRAIN);
+                }
         }
-        return;
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // acc [128 rows x 128 columns] = B rows (K-major) . A panel (MN-major), K = kr ranks
+            constexpr uint32_t idesc = lora::idesc_bf16(TC_M, TC_N, false, true);
+            int k = 0;
+            for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
+                const int st = k % TC_STAGES, buf = k % TC_ACC;
+                if (!lora::wait_bounded(lora::smem_u32(&tempty_bar[buf]), (static_cast<uint32_t>(k / TC_ACC) & 1u) ^ 1u,
+                                        abort_flag, p.err, lora::DERR_WAIT_TMEM_EMPTY))
+                    break;
+                if (!lora::wait_bounded(lora::smem_u32(&full_bar[st]), static_cast<uint32_t>(k / TC_STAGES) & 1u,
+                                        abort_flag, p.err, lora::DERR_WAIT_FULL))
+                    break;
+                lora::tc_fence_after();
+                const uint32_t bsm = lora::smem_u32(smem + st * Cfg::STAGE_BYTES + Cfg::WSTAGE);
+                // K-major 128B swizzle: 8-row groups 1024 bytes apart, a K step of 16 = 32 bytes
+                const uint64_t ad = lora::sdesc_sw128(bsm, 16, 1024);
+                // MN-major 128B swizzle: 64-column chunks 8192 bytes apart (LBO), 8-rank
+                // groups 1024 bytes apart (SBO), a K step of 16 ranks = 2048 bytes
+                const uint64_t bd = lora::sdesc_sw128(bsm + TC_B_BYTES, 8192, 1024);
+                for (int kk = 0; kk < p.kr / 16; ++kk)
+                    lora::tc_mma_bf16(tmem_base + static_cast<uint32_t>(buf * TC_N), ad + (kk * 32 >> 4),
+                                      bd + (kk * 2048 >> 4), idesc, kk > 0 ? 1u : 0u);
+                lora::tc_commit(lora::smem_u32(&tfull_bar[buf]));
+            }
+            lora::tc_commit(lora::smem_u32(drain_bar));
+            volatile int never = 0;
+            lora::wait_bounded(lora::smem_u32(drain_bar), 0, &never, p.err, lora::DERR_WAIT_DRAIN);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp & 3;  // warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
+        const int lr = q * 32 + lane;  // accumulator row = tile row
+        const int et = threadIdx.x - 64;
+        int k = 0, prev_st = -1;
+        for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
+            const int st = k % TC_STAGES, buf = k % TC_ACC;
+            const uint32_t sph = static_cast<uint32_t>(k / TC_STAGES) & 1u;
+            if (et == 0)
+                epi_ok[0] = lora::wait_bounded(lora::smem_u32(&tfull_bar[buf]), static_cast<uint32_t>(k / TC_ACC) & 1u,
+                                               abort_flag, p.err, lora::DERR_WAIT_TMEM_FULL)
+                                ? 1
+                                : 0;
+            lora::named_bar_sync(1, 128);
+            const bool ok = epi_ok[0] != 0;
+            lora::named_bar_sync(1, 128);
+            if (!ok) break;
+            // the stage's operands landed before the MMA ran, so this returns at once; it
+            // makes the weight tile's TMA writes visible to this thread
+            lora::wait_bounded(lora::smem_u32(&full_bar[st]), sph, abort_flag, p.err, lora::DERR_WAIT_FULL);
+            lora::tc_fence_after();
+            const int64_t row = (t / p.col_tiles) * TC_M + lr;
+            const int64_t col0 = (t % p.col_tiles) * TC_N;
+            uint8_t *wst = smem + st * Cfg::STAGE_BYTES;
+            uint8_t *out = Q4 ? staging + (k & 1) * TC_W_BYTES : wst;  // 64-column chunks, 128B swizzle
+            const uint32_t t_row =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * TC_N);
+#pragma unroll 1
+            for (int c = 0; c < TC_CHUNKS; ++c) {
+                uint32_t v0[32], v1[32];
+                lora::tmem_ld_32x32b_x32(t_row + c * 64, v0);
+                lora::tmem_ld_32x32b_x32(t_row + c * 64 + 32, v1);
+                lora::tc_wait_ld();
+                if (c == TC_CHUNKS - 1) {
+                    lora::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) lora::mbar_arrive(lora::smem_u32(&tempty_bar[buf]));
+                }
+                float w[64];
+                if (Q4) {
+                    // 64 codes of this row (32 bytes, low nibble = even column) and their scale
+                    const uint4 *qp = reinterpret_cast<const uint4 *>(wst + lr * (TC_N / 2) + c * 32);
+                    const uint4 q0 = qp[0], q1 = qp[1];
+                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                    const int64_t gcol = col0 + c * 64;
+                    const float s7 = (row < p.d_out && gcol < p.d_in)
+                                         ? bf16_to_f32(p.Wscale[row * (p.d_in / 64) + gcol / 64]) / 7.0f
+                                         : 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float d8[8];
+                        decode8_f32(words[j], s7, d8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[j * 8 + e] = d8[e];
+                    }
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint4 wv =
+                            *reinterpret_cast<const uint4 *>(wst + c * 16384 + lr * 128 + ((ch ^ (lr & 7)) * 16));
+                        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            w[ch * 8 + 2 * e] = __uint_as_float(ww[e] << 16);
+                            w[ch * 8 + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = ch * 8 + 2 * e;
+                        const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
+                        const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
+                        __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(p.s, a0, w[col]), fmaf(p.s, a1, w[col + 1]));
+                        o[e] = *reinterpret_cast<uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(out + c * 16384 + lr * 128 + ((ch ^ (lr & 7)) * 16)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
+            }
+            lora::fence_proxy_async_smem();
+            lora::named_bar_sync(1, 128);
+            if (et == 0) {
+                for (int c = 0; c < TC_CHUNKS; ++c)
+                    if (col0 + 64 * c < p.d_in)  // a chunk wholly past d_in has nothing to store
+                        lora::tma_store_2d(&p.tmOut, lora::smem_u32(out + c * 16384),
+                                           static_cast<int32_t>(col0 + 64 * c),
+                                           static_cast<int32_t>((t / p.col_tiles) * TC_M));
+                lora::bulk_commit_group();
+                if (Q4) {
+                    // the codes are in registers already; the other staging tile's store
+                    // has read it before the next tile writes there
+                    lora::mbar_arrive(lora::smem_u32(&empty_bar[st]));
+                    lora::bulk_wait_group_read<1>();
+                } else {
+                    // the stage holds this tile's output until its store has read it: free
+                    // the previous tile's stage once that store (one group back) has
+                    lora::bulk_wait_group_read<1>();
+                    if (prev_st >= 0) lora::mbar_arrive(lora::smem_u32(&empty_bar[prev_st]));
+                }
+            }
+            lora::named_bar_sync(1, 128);
+            prev_st = st;
+        }
+        if (et == 0) lora::bulk_wait_group<0>();
     }
 
-    // -------------------------------------------------------------------- consumers
-    const int r = p.r;
-    int k = 0;
-    // scale words of the next tile (4-bit), fetched one tile ahead
-    auto scales_of = [&](int64_t t, uint16_t (&sc)[4]) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sc[i] = 0;
-        if (!Q4 || t >= p.tiles) return;
-        const int64_t row = (t / p.col_tiles) * MT + warp * 4, col = (t % p.col_tiles) * NT + lane * 8;
-        if (col >= p.d_in) return;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (row + i < p.d_out) sc[i] = p.Wscale[(row + i) * (p.d_in / 64) + col / 64];
-    };
-    uint16_t sc_next[4];
-    scales_of(blockIdx.x, sc_next);
-    for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
-        uint16_t sc[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) sc[i] = sc_next[i];
-        scales_of(t + gridDim.x, sc_next);
-        const int st = k % p.stages;
-        const uint32_t ph = static_cast<uint32_t>(k / p.stages) & 1u;
-        if (!__all_sync(0xffffffffu, lora::wait_bounded(lora::smem_u32(&full_bar[st]), ph, abort_flag, p.err,
-                                                        lora::DERR_WAIT_FULL)))
-            break;
-        const uint8_t *base = smem + st * p.stage_bytes;
-        const uint16_t *sA = reinterpret_cast<const uint16_t *>(base + p.w_bytes);            // [r][256]
-        const uint16_t *sB = reinterpret_cast<const uint16_t *>(base + p.w_bytes + p.a_bytes);  // [32][r]
-        float acc[4][8];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-#pragma unroll 4
-        for (int jj = 0; jj < r; ++jj) {
-            const uint4 av = *reinterpret_cast<const uint4 *>(sA + jj * NT + lane * 8);
-            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-            float a[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                a[2 * q] = __uint_as_float(aw[q] << 16);
-                a[2 * q + 1] = __uint_as_float(aw[q] & 0xFFFF0000u);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float b = bf16_to_f32(sB[(warp * 4 + i) * r + jj]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(b, a[e], acc[i][e]);
-            }
-        }
-        const int64_t row0 = (t / p.col_tiles) * MT, col = (t % p.col_tiles) * NT + lane * 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int lr = warp * 4 + i;
-            const int64_t row = row0 + lr;
-            float w[8];
-            if (Q4) {
-                decode8_f32(*reinterpret_cast<const uint32_t *>(base + lr * (NT / 2) + lane * 4),
-                            bf16_to_f32(sc[i]) / 7.0f, w);
-            } else {
-                const uint4 wv = *reinterpret_cast<const uint4 *>(base + (lr * NT + lane * 8) * 2);
-                const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    w[2 * q] = __uint_as_float(ww[q] << 16);
-                    w[2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
-                }
-            }
-            if (row < p.d_out && col < p.d_in) {
-                uint32_t out[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(p.s, acc[i][2 * q], w[2 * q]),
-                                                              fmaf(p.s, acc[i][2 * q + 1], w[2 * q + 1]));
-                    out[q] = *reinterpret_cast<uint32_t *>(&b2);
-                }
-                *reinterpret_cast<uint4 *>(p.Wout + row * p.d_in + col) = make_uint4(out[0], out[1], out[2], out[3]);
-            }
-        }
-        __syncwarp();  // every lane is done with this stage
-        if (lane == 0) lora::mbar_arrive(lora::smem_u32(&empty_bar[st]));
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    lora::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        lora::tc_fence_after();
+        lora::tmem_dealloc(tmem_base, TC_ACC * TC_N);
     }
 }
 
@@ -328,13 +443,6 @@ lora_status_t merge_checks(const void *w0, const void *scale, const void *A, con
 }
 
 // ------------------------------------------------------------------ host
-// Row-major 2D tensor [rows][cols] of `esize`-byte elements, box {box_cols, box_rows},
-// no swizzle (threads read the tiles), zero fill outside.
-bool tmap_plain(CUtensorMap *m, CUtensorMapDataType type, int esize, const void *base, uint64_t cols, uint64_t rows,
-                uint32_t box_cols, uint32_t box_rows) {
-    return lora_host::tmap_2d(m, type, esize, base, cols, rows, box_cols, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 std::mutex g_err_mu;
 int *g_err_addr[64] = {};
 
@@ -360,38 +468,41 @@ lora_status_t merge_launch(bool q4, const uint16_t *W, const uint8_t *Wq, const 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t col_tiles = (d_in + NT - 1) / NT, tiles = ((d_out + MT - 1) / MT) * col_tiles;
 
-    MergeArgs a;
-    std::memset(&a, 0, sizeof(a));
-    a.w_bytes = q4 ? MT * NT / 2 : MT * NT * 2;
-    a.a_bytes = static_cast<uint32_t>(r) * NT * 2;
-    a.stage_bytes = a.w_bytes + a.a_bytes + static_cast<uint32_t>(MT * r * 2);
-    a.stages = static_cast<int>(std::min<int64_t>(MAX_STAGES, RING_SMEM / a.stage_bytes));
-    if (r <= 64 && a.stages >= 2) {
+    if (r <= 64) {
         int *err = merge_err_word(dev);
         if (!err) return LORA_ERR_CUDA;
-        const bool maps = (q4 ? tmap_plain(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, d_in / 2, d_out, NT / 2, MT)
-                              : tmap_plain(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d_in, d_out, NT, MT)) &&
-                          tmap_plain(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d_in, r, NT, r) &&
-                          tmap_plain(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, d_out, r, MT);
+        MergeArgs a;
+        std::memset(&a, 0, sizeof(a));
+        a.kr = (r + 15) / 16 * 16;
+        const bool maps =
+            (q4 ? lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, d_in / 2, d_out, TC_N / 2, TC_M,
+                                     CU_TENSOR_MAP_SWIZZLE_NONE)
+                : lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d_in, d_out, 64, TC_M,
+                                     CU_TENSOR_MAP_SWIZZLE_128B)) &&
+            lora_host::tmap_2d(&a.tmOut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Wout, d_in, d_out, 64, TC_M,
+                               CU_TENSOR_MAP_SWIZZLE_128B) &&
+            lora_host::tmap_2d(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d_in, r, 64, a.kr,
+                               CU_TENSOR_MAP_SWIZZLE_128B) &&
+            lora_host::tmap_2d(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, d_out, 64, TC_M,
+                               CU_TENSOR_MAP_SWIZZLE_128B);
         if (!maps) return LORA_ERR_CUDA;
+        const int64_t tc_col_tiles = (d_in + TC_N - 1) / TC_N;
         a.Wscale = Wscale;
-        a.Wout = Wout;
         a.d_in = d_in;
         a.d_out = d_out;
-        a.col_tiles = col_tiles;
-        a.tiles = tiles;
-        a.r = r;
+        a.col_tiles = tc_col_tiles;
+        a.tiles = ((d_out + TC_M - 1) / TC_M) * tc_col_tiles;
         a.s = s;
         a.err = err;
-        const int smem = 1024 + a.stages * static_cast<int>(a.stage_bytes) + 2 * MAX_STAGES * 8 + 16;
-        auto kern = q4 ? k_merge_ring<true> : k_merge_ring<false>;
+        auto kern = q4 ? k_merge_tc<true> : k_merge_tc<false>;
+        const int smem = q4 ? MergeCfg<true>::SMEM_BYTES : MergeCfg<false>::SMEM_BYTES;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
             return LORA_ERR_CUDA;
-        const unsigned grid = static_cast<unsigned>(std::min<int64_t>(tiles, 2 * sms));
-        kern<<<grid, THREADS_TMA, smem, st>>>(a);
+        const unsigned grid = static_cast<unsigned>(std::min<int64_t>(a.tiles, sms));
+        kern<<<grid, TC_THREADS, smem, st>>>(a);
         return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
     }
-    // r > 64: the A panel does not fit a multi-stage ring; one tile per CTA
+    // r > 64: the CUDA-core kernel, one tile per CTA
     const dim3 grid(static_cast<unsigned>(tiles));
     if (q4)
         k_merge<true><<<grid, THREADS, 0, st>>>(nullptr, Wq, Wscale, A, B, Wout, d_in, d_out, r, s);

@@ -61,11 +61,21 @@ def _ref(inp, spec, r0=0, r1=None):
 
 
 SHAPES = [  # d_out, d_in, r, q4
-    (200, 320, 8, False),
-    (333, 520, 24, False),    # ragged rows and a ragged last 256-column tile
+    # r <= 64: tensor-core kernel, 128 x 128 tiles
+    (200, 320, 8, False),     # ragged last tile: its second 64-column chunk lies past d_in
+    (333, 520, 24, False),    # ragged rows; K = 32 with ranks 24..31 zero-filled
+    (129, 136, 16, False),    # one row and 8 columns into the last tiles
+    (1, 64, 8, False),        # one row, one chunk
+    (1000, 4104, 40, False),  # 264 tiles: two per CTA on most SMs
+    (1200, 6000, 64, False),  # 470 tiles: the three stages and two accumulators wrap
+    (256, 384, 48, False),
+    (64, 1024, 56, False),
+    (200, 320, 16, True),
+    (300, 1216, 64, True),    # 4-bit: a last tile half past d_in
+    (520, 4160, 32, True),
+    # r > 64: CUDA-core kernel
     (64, 264, 72, False),     # r crosses the 64-rank staging chunk
     (40, 512, 256, False),
-    (200, 320, 16, True),
     (96, 512, 72, True),
 ]
 
