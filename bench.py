@@ -657,7 +657,7 @@ def main():
     # median of 20.  Before each launch L2 is flushed by reading 256 MB (clean lines: a
     # write would leave ~126 MB of dirty lines for the merge to write back).
     merge = None
-    if rank == 0 and not spec.fp8 and not spec.nf4:
+    if rank == 0:
         s0 = sets[0]
         w_out = torch.empty(do, di, dtype=torch.bfloat16, device=dev)
         flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
@@ -665,6 +665,10 @@ def main():
         def merge_once():
             if spec.q4:
                 L.lora_linear_merge_q4(s0["Wq"], s0["Wscale"], s0["A"], s0["B"], w_out, alpha)
+            elif spec.nf4:
+                L.lora_linear_merge_nf4(s0["Wq"], s0["Wscale"], s0["cb"], s0["A"], s0["B"], w_out, alpha)
+            elif spec.fp8:
+                L.lora_linear_merge_fp8(s0["W8"], s0["W8scale"], s0["A"], s0["B"], w_out, alpha)
             else:
                 L.lora_linear_merge(s0["W"], s0["A"], s0["B"], w_out, alpha)
 
@@ -682,12 +686,14 @@ def main():
             times.append(m0.elapsed_time(m1))
         del flush
         t_merge = sorted(times)[len(times) // 2]
-        w_bytes = (do * di // 2 + do * (di // 64) * 2) if spec.q4 else do * di * 2
+        w_bytes = (do * di // 2 + do * (di // 64) * 2 if (spec.q4 or spec.nf4)
+                   else do * di + do * 2 if spec.fp8 else do * di * 2)
         m_bytes = w_bytes + r * di * 2 + do * r * 2 + do * di * 2
         ach = m_bytes / (t_merge * 1e-3) / 1e9
         merge = {"us": t_merge * 1e3, "bytes": m_bytes, "achieved_gbs": ach, "peak_gbs": peaks["hbm_gbs"],
                  "frac": ach / peaks["hbm_gbs"], "bound": "hbm",
-                 "what": "W' = W + s.B.A (4-bit W decoded)" if spec.q4 else "W' = W + s.B.A"}
+                 "what": "W' = W + s.B.A" + (" (4-bit W decoded)" if spec.q4 else " (NF4 W decoded)" if spec.nf4
+                                             else " (FP8 W decoded)" if spec.fp8 else "")}
 
     # end to end through the C ABI with host buffers: every step copies its inputs in from
     # pinned host memory and its outputs back out (W stays resident: frozen model state).

@@ -310,10 +310,10 @@ LORA_API const char *lora_status_string(lora_status_t status);
  *   W, W_out  bf16 [d_out, d_in] row-major; W_out may equal W (in place) but must not
  *             otherwise overlap it.
  *   A [r, d_in], B [d_out, r]  bf16 row-major.  Every pointer 16-byte aligned.
- * Per element: w + s * sum_j B[n, j] * A[j, k] in fp32 (the bf16 products are exact,
- * summed in j order), rounded once to bf16.  For r <= 64 a persistent TMA-fed kernel
- * streams the tiles (bounded waits; see lora_linear_merge_check); larger r uses one CTA
- * per tile.  Requires 8 <= d_in <= 2^24 with
+ * Per element: w + s * sum_j B[n, j] * A[j, k], the sum formed on the tensor cores in
+ * fp32 (the bf16 products are exact), the weight added in fp32, rounded once to bf16.
+ * A persistent TMA-fed kernel streams 128 x 128 tiles (bounded waits; see
+ * lora_linear_merge_check).  Requires 8 <= d_in <= 2^24 with
  * d_in % 8 == 0, 1 <= d_out <= 2^24, 1 <= r <= 256, r % 8 == 0, finite alpha; otherwise
  * LORA_ERR_INVALID_ARG / LORA_ERR_MISALIGNED before any launch.  Stream-ordered,
  * allocates nothing, needs no workspace.
@@ -329,6 +329,23 @@ LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uint16_t *A, c
 LORA_API lora_status_t lora_linear_merge_q4(const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
                                             const uint16_t *B, uint16_t *W_out, int64_t d_in, int64_t d_out, int r,
                                             float alpha, void *stream);
+
+/* The same from the FP8 (E4M3) weight (codes W8 [d_out, d_in] uint8, one bf16 scale per
+ * row W8scale [d_out], layout as lora_linear_fwd_fp8; d_in % 16 == 0):
+ *     W_out = e4m3(q) * scale + s * B . A
+ * with the decoded weight exact in fp32, rounded once to bf16 with the update. */
+LORA_API lora_status_t lora_linear_merge_fp8(const uint8_t *W8, const uint16_t *W8scale, const uint16_t *A,
+                                             const uint16_t *B, uint16_t *W_out, int64_t d_in, int64_t d_out, int r,
+                                             float alpha, void *stream);
+
+/* The same from the 4-bit codebook weight (Wq, Wscale and `codebook`, 16 floats in HOST
+ * memory read during the call, as lora_linear_fwd_nf4; d_in % 64 == 0):
+ *     W_out = codebook[q] * scale + s * B . A
+ * with codebook[q] * scale formed in fp32; a non-finite codebook value gives
+ * LORA_ERR_INVALID_ARG. */
+LORA_API lora_status_t lora_linear_merge_nf4(const uint8_t *Wq, const uint16_t *Wscale, const float *codebook,
+                                             const uint16_t *A, const uint16_t *B, uint16_t *W_out, int64_t d_in,
+                                             int64_t d_out, int r, float alpha, void *stream);
 
 /* Waits for `stream`, then reads and clears the merge kernels' device error word
  * (their pipeline waits are bounded like the layer's).  LORA_OK, LORA_ERR_TIMEOUT, or

@@ -3,224 +3,196 @@
 // (page "ms-swift框架下UnSloth与Liger-Kernel优化实战", section 设计权衡与最佳实践, item 4:
 // before inference the model is exported in the standard format, the adapter merged
 // into the weight; the merged weight follows from h = W x + B (A x) of page
-// "UnSloth加速库集成：编译级优化带来的性能飞跃", section 为什么标准LoRA会慢？).  The
-// 4-bit variant starts from the decoded code, w = (q - 8) * scale / 7.
+// "UnSloth加速库集成：编译级优化带来的性能飞跃", section 为什么标准LoRA会慢？).  A stored
+// weight in one of the layer's coded formats is decoded first: the 4-bit code
+// (q - 8) * scale / 7, the FP8 (E4M3) code e4m3(q) * row scale, or the 4-bit codebook
+// (NF4) codebook[q] * scale.
 //
-// The work is one read of W and one write of W' (HBM-bound).  Up to r = 64 the rank-r
-// update runs on the tensor cores (k_merge_tc: a tcgen05 contraction over the ranks into
-// TMEM, the weight added in the epilogue, TMA in and out); wider ranks take k_merge, a
-// CUDA-core kernel whose threads accumulate 4-row x 8-column micro-tiles in fp32.  Both
-// add the weight in fp32 and round once to bf16 (bf16 products are exact in fp32).  W'
-// may be W itself (in place): a tile is read before it is written, and tiles are
-// disjoint.
+// The work is one read of W and one write of W' (HBM-bound).  The rank-r update of a
+// 128-row x 128-column tile is a tcgen05 contraction over the ranks (M = 128, N = 128,
+// K = 16 per instruction) into an fp32 TMEM accumulator; the epilogue adds the decoded
+// weight in fp32 and rounds once to bf16 (bf16 products are exact in fp32).  W' may be
+// W itself (in place): a tile is read before it is written, and tiles are disjoint.
+//
+// Roles: warp 0 the TMA producer, warp 1 TMEM and the single-thread MMA issue, warps
+// 2..9 the epilogue (warp w drains TMEM lane quarter w % 4, the first or second 64
+// columns of the tile).  Two rings in shared memory: weight tiles (deep, since the
+// stream that sets the rate needs ~100 KB of reads in flight per SM) and rank chunks
+// (up to 64 ranks of B's 128 rows and of A's 128 columns each; narrow swizzles for
+// r <= 32 so they take little room).  A bf16 weight tile is overwritten by its result
+// and TMA-stored from there; a coded tile is decoded into one of two bf16 staging
+// tiles.  Persistent, one CTA per SM, tiles in row-major order.  Every wait is bounded
+// (2 s); a timeout sets g_merge_err, which lora_linear_merge_check reads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
 
 #include "../../include/lora_linear.h"
-#include "tc_gemm.cuh"  // bounded mbarrier waits, TMA and mbarrier wrappers
+#include "tc_gemm.cuh"  // bounded mbarrier waits, TMA, mbarrier and tcgen05 wrappers
 #include "tmap.h"
 
 namespace {
 
-constexpr int MT = 32;        // rows per CTA tile
-constexpr int NT = 256;       // columns per CTA tile
-constexpr int RCH = 64;       // ranks staged per pass
-constexpr int THREADS = 256;  // 8 warps; warp w owns rows 4w .. 4w+3, lane owns 8 columns
+enum MergeFmt { MF_BF16 = 0, MF_Q4 = 1, MF_FP8 = 2, MF_CB = 3 };
 
-__device__ __forceinline__ float bf16_to_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
-
-// Decoded 4-bit weight, 8 consecutive columns from one 32-bit word of codes (low nibble
-// = even column), in fp32: (q - 8) * (scale / 7), the rule of the main GEMMs' decode.
-__device__ __forceinline__ void decode8_f32(uint32_t word, float s7, float (&w)[8]) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) w[e] = static_cast<float>(static_cast<int>((word >> (4 * e)) & 0xFu) - 8) * s7;
-}
-
-template <bool Q4>
-__global__ void __launch_bounds__(THREADS) k_merge(const uint16_t *W, const uint8_t *Wq,  // may alias Wout
-                                                   const uint16_t *__restrict__ Wscale, const uint16_t *__restrict__ A,
-                                                   const uint16_t *__restrict__ B, uint16_t *Wout, int64_t d_in,
-                                                   int64_t d_out, int r, float s) {
-    __shared__ __align__(16) uint16_t sA[RCH][NT];  // A[j0 + jj][col0 + c]
-    __shared__ __align__(16) uint16_t sB[MT][RCH];  // B[row0 + i][j0 + jj]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // Tiles in row-major order (column tile fastest), so the CTAs resident at one time
-    // read whole rows of W together rather than one 512-byte piece of many rows.
-    const int64_t col_tiles = (d_in + NT - 1) / NT;
-    const int64_t row0 = (static_cast<int64_t>(blockIdx.x) / col_tiles) * MT;
-    const int64_t col0 = (static_cast<int64_t>(blockIdx.x) % col_tiles) * NT;
-    const int64_t col = col0 + lane * 8;  // this thread's 8 columns
-    const bool col_ok = col < d_in;       // d_in % 8 == 0, so a group is all in or all out
-
-    // This thread's weight (4 rows x 8 columns) is loaded first, so its DRAM latency
-    // overlaps the staging and the FMAs below; every load precedes every store, which
-    // keeps W' = W (in place) correct.
-    uint4 wv[4];     // bf16 weight
-    uint32_t qw[4];  // 4-bit weight: one word of codes per row
-    uint16_t sc[4];  //               and its group scale
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t row = row0 + warp * 4 + i;
-        wv[i] = make_uint4(0, 0, 0, 0);
-        qw[i] = 0;
-        sc[i] = 0;
-        if (col_ok && row < d_out) {
-            if (Q4) {
-                qw[i] = *reinterpret_cast<const uint32_t *>(Wq + row * (d_in / 2) + col / 2);
-                sc[i] = Wscale[row * (d_in / 64) + col / 64];
-            } else {
-                wv[i] = *reinterpret_cast<const uint4 *>(W + row * d_in + col);
-            }
-        }
-    }
-
-    float acc[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-
-    for (int j0 = 0; j0 < r; j0 += RCH) {
-        const int rc = min(RCH, r - j0);
-        __syncthreads();  // the previous chunk's readers are done
-        // A panel: rc rows x 256 columns, 16 bytes per load (zero past d_in)
-        for (int v = threadIdx.x; v < rc * (NT / 8); v += THREADS) {
-            const int jj = v / (NT / 8), c8 = (v % (NT / 8)) * 8;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (col0 + c8 < d_in) val = *reinterpret_cast<const uint4 *>(A + (j0 + jj) * d_in + col0 + c8);
-            *reinterpret_cast<uint4 *>(&sA[jj][c8]) = val;
-        }
-        // B rows: 32 rows x rc ranks (zero past d_out)
-        for (int v = threadIdx.x; v < MT * rc; v += THREADS) {
-            const int i = v / rc, jj = v % rc;
-            sB[i][jj] = (row0 + i < d_out) ? B[(row0 + i) * r + j0 + jj] : uint16_t(0);
-        }
-        __syncthreads();
-        for (int jj = 0; jj < rc; ++jj) {
-            const uint4 av = *reinterpret_cast<const uint4 *>(&sA[jj][lane * 8]);
-            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-            float a[8];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                a[2 * q] = __uint_as_float(aw[q] << 16);
-                a[2 * q + 1] = __uint_as_float(aw[q] & 0xFFFF0000u);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float b = bf16_to_f32(sB[warp * 4 + i][jj]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[i][e] = fmaf(b, a[e], acc[i][e]);
-            }
-        }
-    }
-    if (!col_ok) return;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int64_t row = row0 + warp * 4 + i;
-        if (row >= d_out) break;
-        float w[8];
-        if (Q4) {
-            decode8_f32(qw[i], bf16_to_f32(sc[i]) / 7.0f, w);
-        } else {
-            const uint32_t ww[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                w[2 * q] = __uint_as_float(ww[q] << 16);
-                w[2 * q + 1] = __uint_as_float(ww[q] & 0xFFFF0000u);
-            }
-        }
-        uint32_t out[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(s, acc[i][2 * q], w[2 * q]),
-                                                      fmaf(s, acc[i][2 * q + 1], w[2 * q + 1]));
-            out[q] = *reinterpret_cast<uint32_t *>(&b2);
-        }
-        *reinterpret_cast<uint4 *>(Wout + row * d_in + col) = make_uint4(out[0], out[1], out[2], out[3]);
-    }
-}
-
-// ---------------------------------------------------------------- tensor cores (r <= 64)
-// The kernel above spends ~14 instructions per element on the rank-r update (shared-memory
-// operand loads, widening, r FMAs) and is issue-bound at less than half the HBM bandwidth.
-// Here the update s * B . A of a 128-row x 128-column tile is one to four tcgen05 MMAs
-// (M = 128, N = 128, K = 16 ranks each) into an fp32 TMEM accumulator, and the epilogue
-// only adds the weight: tcgen05.ld of 32 columns, the weight from the TMA-staged tile in
-// shared memory, one fp32 FMA and one rounding per element, the result written over the
-// staged tile (bf16 weight) or into a staging tile (4-bit weight), then TMA-stored.
-// Roles as in the layer's kernels: warp 0 the TMA producer, warp 1 TMEM and the
-// single-thread MMA issue, warps 2..5 the epilogue (one accumulator row each thread);
-// three stages of operands, two TMEM accumulators.  Persistent, one CTA per SM, tiles in
-// row-major order.  128 columns rather than 256: a 4096 x 4096 weight is 1024 tiles, 6.9
-// per SM, where 256-column tiles would leave 14% of the SMs' time on a partial last wave.
-// Every wait is bounded (2 s); a timeout sets g_merge_err (lora_linear_merge_check).
-constexpr int TC_M = 128, TC_N = 128, TC_STAGES = 3, TC_ACC = 2, TC_THREADS = 192;
-constexpr int TC_CHUNKS = TC_N / 64;              // 64-column chunks (one 128B-swizzle box each)
-constexpr int TC_W_BYTES = TC_M * TC_N * 2;       // bf16 weight tile, or an output staging tile
-constexpr int TC_Q_BYTES = TC_M * TC_N / 2;       // 4-bit codes of the tile
-constexpr int TC_B_BYTES = TC_M * 64 * 2;         // B rows [128 x 64 ranks], K-major, 128B swizzle
-constexpr int TC_A_BYTES = TC_CHUNKS * 64 * 128;  // A panel: 64-column chunks x 64 ranks, MN-major
+constexpr int TM = 128, TN = 128;         // tile rows, columns
+constexpr int EPI_WARPS = 8, THREADS = 64 + 32 * EPI_WARPS;
+constexpr int MAX_WS = 8, MAX_OS = 4;     // ring depths (barrier arrays)
+constexpr int ACC = 2;                    // TMEM accumulators of TN columns
+constexpr int OUT_BYTES = TM * TN * 2;    // one bf16 tile (two 64-column boxes, 128B swizzle)
+constexpr int SMEM_LIMIT = 232448;        // 227 KB per CTA
+constexpr int SMEM_RESERVED = 1024 + 512; // alignment slack; barriers, codebook, TMEM slot (~310 B)
 
 __device__ int g_merge_err;
 
+// Bytes of one stored weight tile in each format.
+__host__ __device__ constexpr int w_tile_bytes(int wf) {
+    return wf == MF_BF16 ? OUT_BYTES : wf == MF_FP8 ? TM * TN : TM * TN / 2;
+}
+
 struct MergeArgs {
-    CUtensorMap tmW;    // bf16 W [d_out][d_in] box {64, 128}, 128B swizzle; or codes uint8 [d_out][d_in/2] box {64, 128}
-    CUtensorMap tmOut;  // bf16 W' [d_out][d_in] box {64, 128}, 128B swizzle
-    CUtensorMap tmA;    // bf16 A [r][d_in] box {64, kr}, 128B swizzle (the MMA's MN-major B operand)
-    CUtensorMap tmB;    // bf16 B [d_out][r] box {64, 128}, 128B swizzle (the MMA's K-major A operand)
-    const uint16_t *Wscale;  // 4-bit weight: bf16 [d_out][d_in/64]
+    CUtensorMap tmW;    // bf16 W: box {64, 128}, 128B swizzle; FP8 codes: {128 B, 128}, 128B swizzle;
+                        // 4-bit codes [d_out][d_in/2]: {64 B, 128}, 64B swizzle
+    CUtensorMap tmOut;  // bf16 W' box {64, 128}, 128B swizzle
+    CUtensorMap tmA;    // bf16 A [r][d_in] box {64, cr}, 128B swizzle (the MMA's MN-major B operand)
+    CUtensorMap tmB;    // bf16 B [d_out][r] box {nb, 128}, swizzle span nb * 2 bytes (K-major A operand)
+    const uint16_t *Wscale;  // bf16: 4-bit formats [d_out][d_in/64]; FP8 [d_out]
+    float cb[16];            // codebook format: the 16 values
     int64_t d_in, d_out, col_tiles, tiles;
-    int kr;             // r rounded up to 16 (the MMAs' K); ranks past r are zero-filled by TMA
+    int n_chunks;       // rank chunks per tile
+    int cr;             // ranks per chunk (a multiple of 16, <= 64)
+    int kr_last;        // MMA K of the last chunk (ranks past r are zero-filled by TMA)
+    int nb;             // B box width: 16, 32 or 64 ranks
+    int n_ws, n_os;     // ring depths
+    int w_stage, o_stage, b_bytes;  // bytes
     float s;
     int *err;
 };
 
-template <bool Q4>
-struct MergeCfg {
-    static constexpr int WSTAGE = Q4 ? TC_Q_BYTES : TC_W_BYTES;
-    static constexpr int STAGE_BYTES = WSTAGE + TC_B_BYTES + TC_A_BYTES;
-    static constexpr int STAGING = Q4 ? 2 * TC_W_BYTES : 0;  // 4-bit weight: output tiles staged apart
-    static constexpr int SMEM_BYTES = 1024 + TC_STAGES * STAGE_BYTES + STAGING + 256;
-    static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1024-byte alignment of the swizzled boxes");
-    static_assert(SMEM_BYTES <= 232448, "at most 227 KB of shared memory per CTA");
-};
+__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
-template <bool Q4>
-__global__ void __launch_bounds__(TC_THREADS, 1) k_merge_tc(const __grid_constant__ MergeArgs p) {
-    using Cfg = MergeCfg<Q4>;
+// Two E4M3 codes (element 0 in the low byte) to fp32, exactly (E4M3 -> f16 -> f32).
+__device__ __forceinline__ void e4m3x2_f32(uint32_t two, float &lo, float &hi) {
+    asm("{\n\t.reg .b16 c, hl, hh;\n\t.reg .b32 h;\n\t"
+        "cvt.u16.u32 c, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h, c;\n\t"
+        "mov.b32 {hl, hh}, h;\n\t"
+        "cvt.f32.f16 %0, hl;\n\t"
+        "cvt.f32.f16 %1, hh;\n\t}"
+        : "=f"(lo), "=f"(hi)
+        : "r"(two));
+}
+
+// The decoded weight of this thread's row over one 64-column half c of the tile, in
+// fp32.  wst: the weight tile in shared memory, in its format's TMA layout.
+template <int WF>
+__device__ __forceinline__ void load_w64(const MergeArgs &p, const uint8_t *wst, const float *cbs, int lr, int c,
+                                         int64_t row, int64_t gcol, float (&w)[64]) {
+    if (WF == MF_BF16) {
+        // box c: 128 rows of 128 bytes, 16-byte piece j of row lr at (j ^ (lr & 7)) * 16
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(wst + c * 16384 + lr * 128 + ((j ^ (lr & 7)) << 4));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w[8 * j + 2 * e] = __uint_as_float(u[e] << 16);
+                w[8 * j + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
+            }
+        }
+    } else if (WF == MF_FP8) {
+        // 128 rows of 128 code bytes (128B swizzle); this half is pieces 4c .. 4c+3
+        const float sc = row < p.d_out ? bf16f(p.Wscale[row]) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(wst + lr * 128 + (((4 * c + j) ^ (lr & 7)) << 4));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float f0, f1, f2, f3;
+                e4m3x2_f32(u[e] & 0xFFFFu, f0, f1);
+                e4m3x2_f32(u[e] >> 16, f2, f3);
+                w[16 * j + 4 * e] = f0 * sc;
+                w[16 * j + 4 * e + 1] = f1 * sc;
+                w[16 * j + 4 * e + 2] = f2 * sc;
+                w[16 * j + 4 * e + 3] = f3 * sc;
+            }
+        }
+    } else {
+        // 128 rows of 64 code bytes (64B swizzle: piece j of row lr at (j ^ ((lr >> 1) & 3)) * 16);
+        // this half is pieces 2c, 2c+1; low nibble = even column; one scale per 64 columns
+        const float sc = (row < p.d_out && gcol < p.d_in) ? bf16f(p.Wscale[row * (p.d_in / 64) + gcol / 64]) : 0.f;
+        const float s7 = sc / 7.0f;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const uint4 v =
+                *reinterpret_cast<const uint4 *>(wst + lr * 64 + (((2 * c + j) ^ ((lr >> 1) & 3)) << 4));
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t lo = u[e] & 0x0F0F0F0Fu, hi = (u[e] >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int k = 32 * j + 8 * e + 2 * b;
+                    if (WF == MF_Q4) {
+                        // 2^23 + q exactly, then q - 8 exactly, then one rounding: (q - 8) * (scale / 7)
+                        const float fl = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + b));
+                        const float fh = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + b));
+                        w[k] = (fl - 8388616.0f) * s7;
+                        w[k + 1] = (fh - 8388616.0f) * s7;
+                    } else {
+                        w[k] = cbs[(lo >> (8 * b)) & 0xFu] * sc;
+                        w[k + 1] = cbs[(hi >> (8 * b)) & 0xFu] * sc;
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int WF>
+__global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__ MergeArgs p) {
+    constexpr bool kInPlace = WF == MF_BF16;  // the result overwrites the staged weight tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *staging = smem + TC_STAGES * Cfg::STAGE_BYTES;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(staging + Cfg::STAGING);
-    uint64_t *full_bar = bars;                      // [stages] the tile's operands landed
-    uint64_t *empty_bar = bars + TC_STAGES;         // [stages] the stage (and its store) is done with
-    uint64_t *tfull_bar = bars + 2 * TC_STAGES;     // [acc] accumulator ready
-    uint64_t *tempty_bar = tfull_bar + TC_ACC;      // [acc] accumulator drained
-    uint64_t *drain_bar = tempty_bar + TC_ACC;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    uint8_t *wring = smem;                          // n_ws weight tiles
+    uint8_t *oring = wring + p.n_ws * p.w_stage;    // n_os rank chunks: [B rows | A panel]
+    uint8_t *staging = oring + p.n_os * p.o_stage;  // coded formats: 2 bf16 output tiles
+    uint64_t *bars = reinterpret_cast<uint64_t *>(staging + (kInPlace ? 0 : 2 * OUT_BYTES));
+    uint64_t *wfull = bars, *wempty = bars + MAX_WS;
+    uint64_t *ofull = bars + 2 * MAX_WS, *oempty = ofull + MAX_OS;
+    uint64_t *tfull = oempty + MAX_OS, *tempty = tfull + ACC;
+    uint64_t *drain = tempty + ACC;
+    float *cbs = reinterpret_cast<float *>(drain + 1);  // [16]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cbs + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int b = 0; b < TC_STAGES; ++b) {
-            lora::mbar_init(lora::smem_u32(&full_bar[b]), 1);
-            lora::mbar_init(lora::smem_u32(&empty_bar[b]), 1);
+        for (int b = 0; b < MAX_WS; ++b) {
+            lora::mbar_init(lora::smem_u32(&wfull[b]), 1);
+            lora::mbar_init(lora::smem_u32(&wempty[b]), 1);
         }
-        for (int b = 0; b < TC_ACC; ++b) {
-            lora::mbar_init(lora::smem_u32(&tfull_bar[b]), 1);
-            lora::mbar_init(lora::smem_u32(&tempty_bar[b]), 4);
+        for (int b = 0; b < MAX_OS; ++b) {
+            lora::mbar_init(lora::smem_u32(&ofull[b]), 1);
+            lora::mbar_init(lora::smem_u32(&oempty[b]), 1);
         }
-        lora::mbar_init(lora::smem_u32(drain_bar), 1);
+        for (int b = 0; b < ACC; ++b) {
+            lora::mbar_init(lora::smem_u32(&tfull[b]), 1);
+            lora::mbar_init(lora::smem_u32(&tempty[b]), EPI_WARPS);
+        }
+        lora::mbar_init(lora::smem_u32(drain), 1);
         *abort_flag = 0;
         lora::fence_mbar_init();
     }
+    if (threadIdx.x < 16) cbs[threadIdx.x] = p.cb[threadIdx.x];
     if (warp == 0 && lane == 0) {
         lora::tma_prefetch_desc(&p.tmW);
         lora::tma_prefetch_desc(&p.tmOut);
@@ -228,189 +200,193 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_merge_tc(const __grid_constan
         lora::tma_prefetch_desc(&p.tmB);
     }
     if (warp == 1) {
-        lora::tmem_alloc(lora::smem_u32(tmem_slot), TC_ACC * TC_N);
+        lora::tmem_alloc(lora::smem_u32(tmem_slot), ACC * TN);
         lora::tmem_relinquish();
     }
     lora::tc_fence_before();
     __syncthreads();
     lora::tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    const uint32_t a_box_bytes = static_cast<uint32_t>(p.cr) * 128u;  // one 64-column box of A
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            uint32_t issued = 0, issued_phase = 0;
-            int k = 0;
-            for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
-                const int st = k % TC_STAGES;
-                const uint32_t ph = static_cast<uint32_t>(k / TC_STAGES) & 1u;
-                if (!lora::wait_bounded(lora::smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag, p.err,
+            uint32_t w_issued = 0, w_ph = 0, o_issued = 0, o_ph = 0;
+            int k = 0, oc = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++k) {
+                const int row0 = static_cast<int>((t / p.col_tiles) * TM);
+                const int col0 = static_cast<int>((t % p.col_tiles) * TN);
+                const int ws = k % p.n_ws;
+                const uint32_t wph = static_cast<uint32_t>(k / p.n_ws) & 1u;
+                if (!lora::wait_bounded(lora::smem_u32(&wempty[ws]), wph ^ 1u, abort_flag, p.err,
                                         lora::DERR_WAIT_EMPTY))
                     break;
-                const int row0 = static_cast<int>((t / p.col_tiles) * TC_M);
-                const int col0 = static_cast<int>((t % p.col_tiles) * TC_N);
-                uint8_t *base = smem + st * Cfg::STAGE_BYTES;
-                const uint32_t fb = lora::smem_u32(&full_bar[st]);
-                lora::mbar_arrive_expect_tx(
-                    fb, Cfg::WSTAGE + TC_B_BYTES + static_cast<uint32_t>(TC_CHUNKS * 128 * p.kr));
-                if (Q4) {
-                    lora::tma_load_2d(lora::smem_u32(base), &p.tmW, fb, col0 / 2, row0);
+                uint8_t *wdst = wring + ws * p.w_stage;
+                const uint32_t wb = lora::smem_u32(&wfull[ws]);
+                lora::mbar_arrive_expect_tx(wb, static_cast<uint32_t>(p.w_stage));
+                if (WF == MF_BF16) {
+                    lora::tma_load_2d(lora::smem_u32(wdst), &p.tmW, wb, col0, row0);
+                    lora::tma_load_2d(lora::smem_u32(wdst + 16384), &p.tmW, wb, col0 + 64, row0);
+                } else if (WF == MF_FP8) {
+                    lora::tma_load_2d(lora::smem_u32(wdst), &p.tmW, wb, col0, row0);
                 } else {
-                    for (int j = 0; j < TC_CHUNKS; ++j)
-                        lora::tma_load_2d(lora::smem_u32(base + j * 16384), &p.tmW, fb, col0 + 64 * j, row0);
+                    lora::tma_load_2d(lora::smem_u32(wdst), &p.tmW, wb, col0 / 2, row0);
                 }
-                lora::tma_load_2d(lora::smem_u32(base + Cfg::WSTAGE), &p.tmB, fb, 0, row0);
-                for (int j = 0; j < TC_CHUNKS; ++j)
-                    lora::tma_load_2d(lora::smem_u32(base + Cfg::WSTAGE + TC_B_BYTES + j * 8192), &p.tmA, fb,
-                                      col0 + 64 * j, 0);
-                issued |= 1u << st;
-                issued_phase = (issued_phase & ~(1u << st)) | (ph << st);
+                w_issued |= 1u << ws;
+                w_ph = (w_ph & ~(1u << ws)) | (wph << ws);
+                for (int ch = 0; ch < p.n_chunks; ++ch, ++oc) {
+                    const int os = oc % p.n_os;
+                    const uint32_t oph = static_cast<uint32_t>(oc / p.n_os) & 1u;
+                    if (!lora::wait_bounded(lora::smem_u32(&oempty[os]), oph ^ 1u, abort_flag, p.err,
+                                            lora::DERR_WAIT_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *odst = oring + os * p.o_stage;
+                    const uint32_t ob = lora::smem_u32(&ofull[os]);
+                    lora::mbar_arrive_expect_tx(ob, static_cast<uint32_t>(p.b_bytes) + 2u * a_box_bytes);
+                    lora::tma_load_2d(lora::smem_u32(odst), &p.tmB, ob, 64 * ch, row0);
+                    lora::tma_load_2d(lora::smem_u32(odst + p.b_bytes), &p.tmA, ob, col0, 64 * ch);
+                    lora::tma_load_2d(lora::smem_u32(odst + p.b_bytes + a_box_bytes), &p.tmA, ob, col0 + 64,
+                                      64 * ch);
+                    o_issued |= 1u << os;
+                    o_ph = (o_ph & ~(1u << os)) | (oph << os);
+                }
             }
             // copies still in flight (only after a failed wait) land before the CTA exits
-            for (int st = 0; st < TC_STAGES; ++st)
-                if (issued & (1u << st)) {
-                    volatile int never = 0;
-                    lora::wait_bounded(lora::smem_u32(&full_bar[st]), (issued_phase >> st) & 1u, &never, p.err,
+            volatile int never = 0;
+            for (int b = 0; b < p.n_ws; ++b)
+                if (w_issued & (1u << b))
+                    lora::wait_bounded(lora::smem_u32(&wfull[b]), (w_ph >> b) & 1u, &never, p.err,
                                        lora::DERR_WAIT_DRAIN);
-                }
+            for (int b = 0; b < p.n_os; ++b)
+                if (o_issued & (1u << b))
+                    lora::wait_bounded(lora::smem_u32(&ofull[b]), (o_ph >> b) & 1u, &never, p.err,
+                                       lora::DERR_WAIT_DRAIN);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            // acc [128 rows x 128 columns] = B rows (K-major) . A panel (MN-major), K = kr ranks
-            constexpr uint32_t idesc = lora::idesc_bf16(TC_M, TC_N, false, true);
-            int k = 0;
-            for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
-                const int st = k % TC_STAGES, buf = k % TC_ACC;
-                if (!lora::wait_bounded(lora::smem_u32(&tempty_bar[buf]), (static_cast<uint32_t>(k / TC_ACC) & 1u) ^ 1u,
+            // acc [128 rows x 128 columns] += B rows (K-major) . A panel (MN-major), chunk by chunk
+            constexpr uint32_t idesc = lora::idesc_bf16(TM, TN, false, true);
+            const uint32_t b_layout =
+                p.nb == 16 ? lora::SDESC_SW32 : (p.nb == 32 ? lora::SDESC_SW64 : lora::SDESC_SW128);
+            int k = 0, oc = 0;
+            bool ok = true;
+            for (int64_t t = blockIdx.x; ok && t < p.tiles; t += gridDim.x, ++k) {
+                const int buf = k % ACC;
+                if (!lora::wait_bounded(lora::smem_u32(&tempty[buf]), (static_cast<uint32_t>(k / ACC) & 1u) ^ 1u,
                                         abort_flag, p.err, lora::DERR_WAIT_TMEM_EMPTY))
                     break;
-                if (!lora::wait_bounded(lora::smem_u32(&full_bar[st]), static_cast<uint32_t>(k / TC_STAGES) & 1u,
-                                        abort_flag, p.err, lora::DERR_WAIT_FULL))
-                    break;
                 lora::tc_fence_after();
-                const uint32_t bsm = lora::smem_u32(smem + st * Cfg::STAGE_BYTES + Cfg::WSTAGE);
-                // K-major 128B swizzle: 8-row groups 1024 bytes apart, a K step of 16 = 32 bytes
-                const uint64_t ad = lora::sdesc_sw128(bsm, 16, 1024);
-                // MN-major 128B swizzle: 64-column chunks 8192 bytes apart (LBO), 8-rank
-                // groups 1024 bytes apart (SBO), a K step of 16 ranks = 2048 bytes
-                const uint64_t bd = lora::sdesc_sw128(bsm + TC_B_BYTES, 8192, 1024);
-                for (int kk = 0; kk < p.kr / 16; ++kk)
-                    lora::tc_mma_bf16(tmem_base + static_cast<uint32_t>(buf * TC_N), ad + (kk * 32 >> 4),
-                                      bd + (kk * 2048 >> 4), idesc, kk > 0 ? 1u : 0u);
-                lora::tc_commit(lora::smem_u32(&tfull_bar[buf]));
+                for (int ch = 0; ch < p.n_chunks; ++ch, ++oc) {
+                    const int os = oc % p.n_os;
+                    if (!lora::wait_bounded(lora::smem_u32(&ofull[os]), static_cast<uint32_t>(oc / p.n_os) & 1u,
+                                            abort_flag, p.err, lora::DERR_WAIT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    lora::tc_fence_after();
+                    const uint32_t bsm = lora::smem_u32(oring + os * p.o_stage);
+                    // B rows: rows of nb ranks, 8-row swizzle atoms nb * 16 bytes apart; a K
+                    // step of 16 ranks is 32 bytes along the row
+                    const uint64_t ad = lora::sdesc(bsm, 16, static_cast<uint32_t>(p.nb) * 16u, b_layout);
+                    // A panel: two 64-column boxes (LBO apart), 8-rank atoms 1024 bytes apart;
+                    // a K step of 16 ranks is 2048 bytes
+                    const uint64_t bd = lora::sdesc_sw128(bsm + p.b_bytes, a_box_bytes, 1024);
+                    const int ksteps = (ch == p.n_chunks - 1 ? p.kr_last : p.cr) / 16;
+                    for (int kk = 0; kk < ksteps; ++kk)
+                        lora::tc_mma_bf16(tmem_base + static_cast<uint32_t>(buf * TN), ad + (kk * 32 >> 4),
+                                          bd + (kk * 2048 >> 4), idesc, (ch > 0 || kk > 0) ? 1u : 0u);
+                    lora::tc_commit(lora::smem_u32(&oempty[os]));
+                }
+                if (!ok) break;
+                lora::tc_commit(lora::smem_u32(&tfull[buf]));
             }
-            lora::tc_commit(lora::smem_u32(drain_bar));
+            lora::tc_commit(lora::smem_u32(drain));
             volatile int never = 0;
-            lora::wait_bounded(lora::smem_u32(drain_bar), 0, &never, p.err, lora::DERR_WAIT_DRAIN);
+            lora::wait_bounded(lora::smem_u32(drain), 0, &never, p.err, lora::DERR_WAIT_DRAIN);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;  // warps 2..5 -> TMEM lane quarters 2, 3, 0, 1
-        const int lr = q * 32 + lane;  // accumulator row = tile row
+        const int q = warp & 3;         // TMEM lane quarter (warps 2..9 -> 2, 3, 0, 1, 2, 3, 0, 1)
+        const int c = (warp - 2) >> 2;  // this warp's 64 columns of the tile
+        const int lr = q * 32 + lane;   // accumulator row = tile row
         const int et = threadIdx.x - 64;
-        int k = 0, prev_st = -1;
+        int k = 0, prev_ws = -1;
         for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
-            const int st = k % TC_STAGES, buf = k % TC_ACC;
-            const uint32_t sph = static_cast<uint32_t>(k / TC_STAGES) & 1u;
+            const int buf = k % ACC, ws = k % p.n_ws;
+            const uint32_t wph = static_cast<uint32_t>(k / p.n_ws) & 1u;
             if (et == 0)
-                epi_ok[0] = lora::wait_bounded(lora::smem_u32(&tfull_bar[buf]), static_cast<uint32_t>(k / TC_ACC) & 1u,
-                                               abort_flag, p.err, lora::DERR_WAIT_TMEM_FULL)
+                epi_ok[0] = (lora::wait_bounded(lora::smem_u32(&tfull[buf]), static_cast<uint32_t>(k / ACC) & 1u,
+                                                abort_flag, p.err, lora::DERR_WAIT_TMEM_FULL) &&
+                             lora::wait_bounded(lora::smem_u32(&wfull[ws]), wph, abort_flag, p.err,
+                                                lora::DERR_WAIT_FULL))
                                 ? 1
                                 : 0;
-            lora::named_bar_sync(1, 128);
+            lora::named_bar_sync(1, 32 * EPI_WARPS);
             const bool ok = epi_ok[0] != 0;
-            lora::named_bar_sync(1, 128);
+            lora::named_bar_sync(1, 32 * EPI_WARPS);
             if (!ok) break;
-            // the stage's operands landed before the MMA ran, so this returns at once; it
-            // makes the weight tile's TMA writes visible to this thread
-            lora::wait_bounded(lora::smem_u32(&full_bar[st]), sph, abort_flag, p.err, lora::DERR_WAIT_FULL);
+            // the weight tile has landed (seen above); this wait makes its TMA writes
+            // visible to this thread and returns at once
+            lora::wait_bounded(lora::smem_u32(&wfull[ws]), wph, abort_flag, p.err, lora::DERR_WAIT_FULL);
             lora::tc_fence_after();
-            const int64_t row = (t / p.col_tiles) * TC_M + lr;
-            const int64_t col0 = (t % p.col_tiles) * TC_N;
-            uint8_t *wst = smem + st * Cfg::STAGE_BYTES;
-            uint8_t *out = Q4 ? staging + (k & 1) * TC_W_BYTES : wst;  // 64-column chunks, 128B swizzle
-            const uint32_t t_row =
-                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * TC_N);
-#pragma unroll 1
-            for (int c = 0; c < TC_CHUNKS; ++c) {
-                uint32_t v0[32], v1[32];
-                lora::tmem_ld_32x32b_x32(t_row + c * 64, v0);
-                lora::tmem_ld_32x32b_x32(t_row + c * 64 + 32, v1);
-                lora::tc_wait_ld();
-                if (c == TC_CHUNKS - 1) {
-                    lora::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) lora::mbar_arrive(lora::smem_u32(&tempty_bar[buf]));
+            const int64_t row0 = (t / p.col_tiles) * TM;
+            const int64_t col0 = (t % p.col_tiles) * TN;
+            const uint8_t *wst = wring + ws * p.w_stage;
+            uint8_t *out = kInPlace ? wring + ws * p.w_stage : staging + (k & 1) * OUT_BYTES;
+
+            uint32_t v0[32], v1[32];
+            const uint32_t t_addr =
+                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * TN + c * 64);
+            lora::tmem_ld_32x32b_x32(t_addr, v0);
+            lora::tmem_ld_32x32b_x32(t_addr + 32, v1);
+            float w[64];
+            load_w64<WF>(p, wst, cbs, lr, c, row0 + lr, col0 + 64 * c, w);
+            lora::tc_wait_ld();
+            lora::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) lora::mbar_arrive(lora::smem_u32(&tempty[buf]));
+            // (in place, a thread overwrites exactly the 64 weights of its row it has just read)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                uint32_t o[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 8 * j + 2 * e;
+                    const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
+                    const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
+                    __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(p.s, a0, w[col]), fmaf(p.s, a1, w[col + 1]));
+                    o[e] = *reinterpret_cast<uint32_t *>(&b2);
                 }
-                float w[64];
-                if (Q4) {
-                    // 64 codes of this row (32 bytes, low nibble = even column) and their scale
-                    const uint4 *qp = reinterpret_cast<const uint4 *>(wst + lr * (TC_N / 2) + c * 32);
-                    const uint4 q0 = qp[0], q1 = qp[1];
-                    const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                    const int64_t gcol = col0 + c * 64;
-                    const float s7 = (row < p.d_out && gcol < p.d_in)
-                                         ? bf16_to_f32(p.Wscale[row * (p.d_in / 64) + gcol / 64]) / 7.0f
-                                         : 0.f;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        float d8[8];
-                        decode8_f32(words[j], s7, d8);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) w[j * 8 + e] = d8[e];
-                    }
-                } else {
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint4 wv =
-                            *reinterpret_cast<const uint4 *>(wst + c * 16384 + lr * 128 + ((ch ^ (lr & 7)) * 16));
-                        const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            w[ch * 8 + 2 * e] = __uint_as_float(ww[e] << 16);
-                            w[ch * 8 + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    uint32_t o[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int col = ch * 8 + 2 * e;
-                        const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
-                        const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(p.s, a0, w[col]), fmaf(p.s, a1, w[col + 1]));
-                        o[e] = *reinterpret_cast<uint32_t *>(&b2);
-                    }
-                    *reinterpret_cast<uint4 *>(out + c * 16384 + lr * 128 + ((ch ^ (lr & 7)) * 16)) =
-                        make_uint4(o[0], o[1], o[2], o[3]);
-                }
+                *reinterpret_cast<uint4 *>(out + c * 16384 + lr * 128 + ((j ^ (lr & 7)) << 4)) =
+                    make_uint4(o[0], o[1], o[2], o[3]);
             }
             lora::fence_proxy_async_smem();
-            lora::named_bar_sync(1, 128);
+            lora::named_bar_sync(1, 32 * EPI_WARPS);
             if (et == 0) {
-                for (int c = 0; c < TC_CHUNKS; ++c)
-                    if (col0 + 64 * c < p.d_in)  // a chunk wholly past d_in has nothing to store
-                        lora::tma_store_2d(&p.tmOut, lora::smem_u32(out + c * 16384),
-                                           static_cast<int32_t>(col0 + 64 * c),
-                                           static_cast<int32_t>((t / p.col_tiles) * TC_M));
+                for (int cc = 0; cc < 2; ++cc)
+                    if (col0 + 64 * cc < p.d_in)  // a box wholly past d_in has nothing to store
+                        lora::tma_store_2d(&p.tmOut, lora::smem_u32(out + cc * 16384),
+                                           static_cast<int32_t>(col0 + 64 * cc), static_cast<int32_t>(row0));
                 lora::bulk_commit_group();
-                if (Q4) {
-                    // the codes are in registers already; the other staging tile's store
-                    // has read it before the next tile writes there
-                    lora::mbar_arrive(lora::smem_u32(&empty_bar[st]));
-                    lora::bulk_wait_group_read<1>();
-                } else {
-                    // the stage holds this tile's output until its store has read it: free
+                if (kInPlace) {
+                    // this tile's stage holds its output until the store has read it: free
                     // the previous tile's stage once that store (one group back) has
                     lora::bulk_wait_group_read<1>();
-                    if (prev_st >= 0) lora::mbar_arrive(lora::smem_u32(&empty_bar[prev_st]));
+                    if (prev_ws >= 0) lora::mbar_arrive(lora::smem_u32(&wempty[prev_ws]));
+                } else {
+                    // the codes are decoded already; the other staging tile's store must have
+                    // read it before the next tile is written there
+                    lora::mbar_arrive(lora::smem_u32(&wempty[ws]));
+                    lora::bulk_wait_group_read<1>();
                 }
             }
-            lora::named_bar_sync(1, 128);
-            prev_st = st;
+            lora::named_bar_sync(1, 32 * EPI_WARPS);
+            prev_ws = ws;
         }
         if (et == 0) lora::bulk_wait_group<0>();
     }
@@ -421,23 +397,36 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k_merge_tc(const __grid_constan
     __syncthreads();
     if (warp == 1) {
         lora::tc_fence_after();
-        lora::tmem_dealloc(tmem_base, TC_ACC * TC_N);
+        lora::tmem_dealloc(tmem_base, ACC * TN);
     }
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Every pointer 16-byte aligned, as for the layer: the ring kernel reads W (or the codes),
-// A and B by TMA and the other kernel reads W and A in 16-byte vectors.
-lora_status_t merge_checks(const void *w0, const void *scale, const void *A, const void *B, const void *Wout,
-                           int64_t d_in, int64_t d_out, int r, float alpha, bool q4) {
-    if (!w0 || !A || !B || !Wout || (q4 && !scale)) return LORA_ERR_INVALID_ARG;
-    if (d_in < 8 || d_out < 1 || d_in % 8 || (q4 && d_in % 64)) return LORA_ERR_INVALID_ARG;
+// The weight as the caller stores it.
+struct MergeWeight {
+    int wf = MF_BF16;
+    const void *w = nullptr;          // bf16 W, or the codes
+    const uint16_t *scale = nullptr;  // coded formats
+    const float *codebook = nullptr;  // MF_CB: 16 values (host)
+};
+
+// Every pointer 16-byte aligned (TMA), sizes within the tensor maps' ranges.
+lora_status_t merge_checks(const MergeWeight &mw, const void *A, const void *B, const void *Wout, int64_t d_in,
+                           int64_t d_out, int r, float alpha) {
+    const bool coded = mw.wf != MF_BF16;
+    if (!mw.w || !A || !B || !Wout || (coded && !mw.scale) || (mw.wf == MF_CB && !mw.codebook))
+        return LORA_ERR_INVALID_ARG;
+    if (d_in < 8 || d_out < 1 || d_in % 8) return LORA_ERR_INVALID_ARG;
+    if ((mw.wf == MF_Q4 || mw.wf == MF_CB) && d_in % 64) return LORA_ERR_INVALID_ARG;
+    if (mw.wf == MF_FP8 && d_in % 16) return LORA_ERR_INVALID_ARG;
     if (d_in > (int64_t(1) << 24) || d_out > (int64_t(1) << 24)) return LORA_ERR_INVALID_ARG;
-    if (((d_out + MT - 1) / MT) * ((d_in + NT - 1) / NT) > 0x7FFFFFFF) return LORA_ERR_INVALID_ARG;
     if (r < 1 || r > 256 || r % 8) return LORA_ERR_INVALID_ARG;
     if (!(alpha == alpha) || alpha > 3.4e38f || alpha < -3.4e38f) return LORA_ERR_INVALID_ARG;
-    if (!aligned16(w0) || !aligned16(A) || !aligned16(B) || !aligned16(Wout) || (q4 && !aligned16(scale)))
+    if (mw.wf == MF_CB)
+        for (int i = 0; i < 16; ++i)
+            if (!std::isfinite(mw.codebook[i])) return LORA_ERR_INVALID_ARG;
+    if (!aligned16(mw.w) || !aligned16(A) || !aligned16(B) || !aligned16(Wout) || (coded && !aligned16(mw.scale)))
         return LORA_ERR_MISALIGNED;
     return LORA_OK;
 }
@@ -456,59 +445,95 @@ int *merge_err_word(int dev) {
     return g_err_addr[dev];
 }
 
-lora_status_t merge_launch(bool q4, const uint16_t *W, const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
-                           const uint16_t *B, uint16_t *Wout, int64_t d_in, int64_t d_out, int r, float alpha,
-                           void *stream) {
+// Ring depths: the rank-chunk ring gets about 64 KB (2 to 4 chunks), the weight ring
+// the rest, up to 8 tiles.
+void merge_rings(int wf, int o_stage, int &n_ws, int &n_os) {
+    n_os = std::max(2, std::min(MAX_OS, 65536 / o_stage));
+    const int staging = wf == MF_BF16 ? 0 : 2 * OUT_BYTES;
+    const int avail = SMEM_LIMIT - SMEM_RESERVED - staging - n_os * o_stage;
+    n_ws = std::min(MAX_WS, avail / w_tile_bytes(wf));
+}
+
+template <int WF>
+cudaError_t merge_kernel_launch(const MergeArgs &a, int grid, cudaStream_t st) {
+    const int smem = SMEM_RESERVED + a.n_ws * a.w_stage + a.n_os * a.o_stage + (WF == MF_BF16 ? 0 : 2 * OUT_BYTES);
+    const cudaError_t e = cudaFuncSetAttribute(k_merge_tc<WF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_merge_tc<WF><<<grid, THREADS, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+lora_status_t merge_launch(const MergeWeight &mw, const uint16_t *A, const uint16_t *B, uint16_t *Wout, int64_t d_in,
+                           int64_t d_out, int r, float alpha, void *stream) {
     int dev = 0, major = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return LORA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return LORA_ERR_CUDA;
     if (major != 10) return LORA_ERR_UNSUPPORTED;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return LORA_ERR_CUDA;
-    const float s = alpha / static_cast<float>(r);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int64_t col_tiles = (d_in + NT - 1) / NT, tiles = ((d_out + MT - 1) / MT) * col_tiles;
+    int *err = merge_err_word(dev);
+    if (!err) return LORA_ERR_CUDA;
 
-    if (r <= 64) {
-        int *err = merge_err_word(dev);
-        if (!err) return LORA_ERR_CUDA;
-        MergeArgs a;
-        std::memset(&a, 0, sizeof(a));
-        a.kr = (r + 15) / 16 * 16;
-        const bool maps =
-            (q4 ? lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, d_in / 2, d_out, TC_N / 2, TC_M,
-                                     CU_TENSOR_MAP_SWIZZLE_NONE)
-                : lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, d_in, d_out, 64, TC_M,
-                                     CU_TENSOR_MAP_SWIZZLE_128B)) &&
-            lora_host::tmap_2d(&a.tmOut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Wout, d_in, d_out, 64, TC_M,
-                               CU_TENSOR_MAP_SWIZZLE_128B) &&
-            lora_host::tmap_2d(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d_in, r, 64, a.kr,
-                               CU_TENSOR_MAP_SWIZZLE_128B) &&
-            lora_host::tmap_2d(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, d_out, 64, TC_M,
-                               CU_TENSOR_MAP_SWIZZLE_128B);
-        if (!maps) return LORA_ERR_CUDA;
-        const int64_t tc_col_tiles = (d_in + TC_N - 1) / TC_N;
-        a.Wscale = Wscale;
-        a.d_in = d_in;
-        a.d_out = d_out;
-        a.col_tiles = tc_col_tiles;
-        a.tiles = ((d_out + TC_M - 1) / TC_M) * tc_col_tiles;
-        a.s = s;
-        a.err = err;
-        auto kern = q4 ? k_merge_tc<true> : k_merge_tc<false>;
-        const int smem = q4 ? MergeCfg<true>::SMEM_BYTES : MergeCfg<false>::SMEM_BYTES;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-            return LORA_ERR_CUDA;
-        const unsigned grid = static_cast<unsigned>(std::min<int64_t>(a.tiles, sms));
-        kern<<<grid, TC_THREADS, smem, st>>>(a);
-        return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    MergeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int kr = (r + 15) / 16 * 16;
+    a.n_chunks = (kr + 63) / 64;
+    a.cr = std::min(kr, 64);
+    a.kr_last = kr - 64 * (a.n_chunks - 1);
+    a.nb = kr <= 16 ? 16 : (kr <= 32 ? 32 : 64);
+    a.b_bytes = TM * a.nb * 2;
+    a.o_stage = a.b_bytes + 2 * a.cr * 128;
+    a.w_stage = w_tile_bytes(mw.wf);
+    merge_rings(mw.wf, a.o_stage, a.n_ws, a.n_os);
+    const CUtensorMapSwizzle b_swz = a.nb == 16   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                     : a.nb == 32 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                  : CU_TENSOR_MAP_SWIZZLE_128B;
+    bool maps = true;
+    switch (mw.wf) {
+        case MF_BF16:
+            maps = lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, mw.w, d_in, d_out, 64, TM,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+            break;
+        case MF_FP8:
+            maps = lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, mw.w, d_in, d_out, TN, TM,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+            break;
+        default:
+            maps = lora_host::tmap_2d(&a.tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, mw.w, d_in / 2, d_out, TN / 2, TM,
+                                      CU_TENSOR_MAP_SWIZZLE_64B);
     }
-    // r > 64: the CUDA-core kernel, one tile per CTA
-    const dim3 grid(static_cast<unsigned>(tiles));
-    if (q4)
-        k_merge<true><<<grid, THREADS, 0, st>>>(nullptr, Wq, Wscale, A, B, Wout, d_in, d_out, r, s);
-    else
-        k_merge<false><<<grid, THREADS, 0, st>>>(W, nullptr, nullptr, A, B, Wout, d_in, d_out, r, s);
-    return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+    maps = maps &&
+           lora_host::tmap_2d(&a.tmOut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Wout, d_in, d_out, 64, TM,
+                              CU_TENSOR_MAP_SWIZZLE_128B) &&
+           lora_host::tmap_2d(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d_in, r, 64, a.cr,
+                              CU_TENSOR_MAP_SWIZZLE_128B) &&
+           lora_host::tmap_2d(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, B, r, d_out, a.nb, TM, b_swz);
+    if (!maps) return LORA_ERR_CUDA;
+    a.Wscale = mw.scale;
+    if (mw.wf == MF_CB)
+        for (int i = 0; i < 16; ++i) a.cb[i] = mw.codebook[i];
+    a.d_in = d_in;
+    a.d_out = d_out;
+    a.col_tiles = (d_in + TN - 1) / TN;
+    a.tiles = ((d_out + TM - 1) / TM) * a.col_tiles;
+    a.s = alpha / static_cast<float>(r);
+    a.err = err;
+    const int grid = static_cast<int>(std::min<int64_t>(a.tiles, sms));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaSuccess;
+    switch (mw.wf) {
+        case MF_BF16: e = merge_kernel_launch<MF_BF16>(a, grid, st); break;
+        case MF_Q4: e = merge_kernel_launch<MF_Q4>(a, grid, st); break;
+        case MF_FP8: e = merge_kernel_launch<MF_FP8>(a, grid, st); break;
+        default: e = merge_kernel_launch<MF_CB>(a, grid, st);
+    }
+    return e == cudaSuccess ? LORA_OK : LORA_ERR_CUDA;
+}
+
+lora_status_t merge(const MergeWeight &mw, const uint16_t *A, const uint16_t *B, uint16_t *W_out, int64_t d_in,
+                    int64_t d_out, int r, float alpha, void *stream) {
+    const lora_status_t st = merge_checks(mw, A, B, W_out, d_in, d_out, r, alpha);
+    if (st != LORA_OK) return st;
+    return merge_launch(mw, A, B, W_out, d_in, d_out, r, alpha, stream);
 }
 
 }  // namespace
@@ -516,17 +541,41 @@ lora_status_t merge_launch(bool q4, const uint16_t *W, const uint8_t *Wq, const 
 extern "C" LORA_API lora_status_t lora_linear_merge(const uint16_t *W, const uint16_t *A, const uint16_t *B,
                                                     uint16_t *W_out, int64_t d_in, int64_t d_out, int r, float alpha,
                                                     void *stream) {
-    const lora_status_t st = merge_checks(W, nullptr, A, B, W_out, d_in, d_out, r, alpha, false);
-    if (st != LORA_OK) return st;
-    return merge_launch(false, W, nullptr, nullptr, A, B, W_out, d_in, d_out, r, alpha, stream);
+    MergeWeight mw;
+    mw.w = W;
+    return merge(mw, A, B, W_out, d_in, d_out, r, alpha, stream);
 }
 
 extern "C" LORA_API lora_status_t lora_linear_merge_q4(const uint8_t *Wq, const uint16_t *Wscale, const uint16_t *A,
                                                        const uint16_t *B, uint16_t *W_out, int64_t d_in, int64_t d_out,
                                                        int r, float alpha, void *stream) {
-    const lora_status_t st = merge_checks(Wq, Wscale, A, B, W_out, d_in, d_out, r, alpha, true);
-    if (st != LORA_OK) return st;
-    return merge_launch(true, nullptr, Wq, Wscale, A, B, W_out, d_in, d_out, r, alpha, stream);
+    MergeWeight mw;
+    mw.wf = MF_Q4;
+    mw.w = Wq;
+    mw.scale = Wscale;
+    return merge(mw, A, B, W_out, d_in, d_out, r, alpha, stream);
+}
+
+extern "C" LORA_API lora_status_t lora_linear_merge_fp8(const uint8_t *W8, const uint16_t *W8scale, const uint16_t *A,
+                                                        const uint16_t *B, uint16_t *W_out, int64_t d_in,
+                                                        int64_t d_out, int r, float alpha, void *stream) {
+    MergeWeight mw;
+    mw.wf = MF_FP8;
+    mw.w = W8;
+    mw.scale = W8scale;
+    return merge(mw, A, B, W_out, d_in, d_out, r, alpha, stream);
+}
+
+extern "C" LORA_API lora_status_t lora_linear_merge_nf4(const uint8_t *Wq, const uint16_t *Wscale,
+                                                        const float *codebook, const uint16_t *A, const uint16_t *B,
+                                                        uint16_t *W_out, int64_t d_in, int64_t d_out, int r,
+                                                        float alpha, void *stream) {
+    MergeWeight mw;
+    mw.wf = MF_CB;
+    mw.w = Wq;
+    mw.scale = Wscale;
+    mw.codebook = codebook;
+    return merge(mw, A, B, W_out, d_in, d_out, r, alpha, stream);
 }
 
 extern "C" LORA_API lora_status_t lora_linear_merge_check(void *stream) {

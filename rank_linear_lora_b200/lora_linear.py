@@ -381,6 +381,39 @@ def lora_linear_merge_q4(Wq, Wscale, A, B, W_out, alpha, stream=None):
            "lora_linear_merge_q4")
 
 
+def lora_linear_merge_fp8(W8, W8scale, A, B, W_out, alpha, stream=None):
+    """W_out = e4m3(W8) * W8scale[row] + (alpha / r) * B . A in bf16."""
+    d_out, d_in = W8.shape
+    r = A.shape[0]
+    _fp8(W8, W8scale, d_out, d_in)
+    for t, n, s in ((A, "A", (r, d_in)), (B, "B", (d_out, r)), (W_out, "W_out", (d_out, d_in))):
+        _bf16(t, n, s)
+    fn = load_library().lora_linear_merge_fp8
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, P, I64, I64, I, F, P]
+    fn.restype = I
+    _check(fn(_ptr(W8), _ptr(W8scale), _ptr(A), _ptr(B), _ptr(W_out), d_in, d_out, r, float(alpha),
+              _stream(stream)), "lora_linear_merge_fp8")
+
+
+def lora_linear_merge_nf4(Wq, Wscale, codebook, A, B, W_out, alpha, stream=None):
+    """W_out = codebook[Wq] * Wscale[n, k/64] + (alpha / r) * B . A in bf16."""
+    d_out = Wq.shape[0]
+    r, d_in = A.shape
+    _q4(Wq, Wscale, d_out, d_in)
+    for t, n, s in ((A, "A", (r, d_in)), (B, "B", (d_out, r)), (W_out, "W_out", (d_out, d_in))):
+        _bf16(t, n, s)
+    keep, cbp = _codebook(codebook)
+    fn = load_library().lora_linear_merge_nf4
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    fn.argtypes = [P, P, P, P, P, P, I64, I64, I, F, P]
+    fn.restype = I
+    st = fn(_ptr(Wq), _ptr(Wscale), cbp, _ptr(A), _ptr(B), _ptr(W_out), d_in, d_out, r, float(alpha),
+            _stream(stream))
+    del keep
+    _check(st, "lora_linear_merge_nf4")
+
+
 def lora_linear_merge_check(stream=None):
     fn = load_library().lora_linear_merge_check
     fn.argtypes = [ctypes.c_void_p]

@@ -115,6 +115,39 @@ def test_merge_argument_checks(lib):
     assert q(sc=0x5002) == 2 and q(Wq=0x1008) == 2
 
 
+def test_merge_fp8_and_nf4_argument_checks(lib):
+    """The FP8 and codebook merges: scales (and the codebook) required and finite, the
+    formats' d_in rules, alignment, all before any launch."""
+    import numpy as np
+    assert {"lora_linear_merge_fp8", "lora_linear_merge_nf4"} <= set(L.declared_functions())
+    P, I64, I, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+    m8 = lib.lora_linear_merge_fp8
+    m8.argtypes = [P, P, P, P, P, I64, I64, I, F, P]
+    m8.restype = I
+    mn = lib.lora_linear_merge_nf4
+    mn.argtypes = [P, P, P, P, P, P, I64, I64, I, F, P]
+    mn.restype = I
+    good = np.linspace(-1.0, 1.0, 16).astype(np.float32)
+    bad_cb = good.copy()
+    bad_cb[3] = np.nan
+
+    def f(W8=0x1000, sc=0x5000, A=0x2000, B_=0x3000, out=0x4000, di=256, do=64, r=8, alpha=16.0):
+        return m8(P(W8), P(sc), P(A), P(B_), P(out), di, do, r, alpha, None)
+
+    def n(Wq=0x1000, sc=0x5000, cb=good, A=0x2000, B_=0x3000, out=0x4000, di=256, do=64, r=8, alpha=16.0):
+        cbp = None if cb is None else cb.ctypes.data_as(P)
+        return mn(P(Wq), P(sc), cbp, P(A), P(B_), P(out), di, do, r, alpha, None)
+
+    assert f(sc=None) == 1 and f(W8=None) == 1
+    assert f(di=264) == 1                             # FP8 weight: d_in % 16 == 0
+    assert f(r=72, alpha=float("nan")) == 1
+    assert f(sc=0x5008) == 2 and f(W8=0x1004) == 2
+    assert n(cb=None) == 1 and n(sc=None) == 1
+    assert n(cb=bad_cb) == 1                          # a non-finite codebook value
+    assert n(di=320 + 32) == 1                        # codebook weight: d_in % 64 == 0
+    assert n(Wq=0x1008) == 2 and n(out=0x4004) == 2
+
+
 def test_fp8_validation_before_any_device_work(lib):
     """The FP8 entry points: workspace sizes for their ops, and argument checks (codes
     and scales required, 16-byte aligned, d_in % 16 == 0) before any launch."""
