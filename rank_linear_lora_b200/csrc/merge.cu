@@ -15,14 +15,18 @@
 // W itself (in place): a tile is read before it is written, and tiles are disjoint.
 //
 // Roles: warp 0 the TMA producer, warp 1 TMEM and the single-thread MMA issue, warps
-// 2..9 the epilogue (warp w drains TMEM lane quarter w % 4, the first or second 64
-// columns of the tile).  Two rings in shared memory: weight tiles (deep, since the
-// stream that sets the rate needs ~100 KB of reads in flight per SM) and rank chunks
-// (up to 64 ranks of B's 128 rows and of A's 128 columns each; narrow swizzles for
-// r <= 32 so they take little room).  A bf16 weight tile is overwritten by its result
-// and TMA-stored from there; a coded tile is decoded into one of two bf16 staging
-// tiles.  Persistent, one CTA per SM, tiles in row-major order.  Every wait is bounded
-// (2 s); a timeout sets g_merge_err, which lora_linear_merge_check reads.
+// 2..9 the epilogue in two groups of four that take alternate tiles (four TMEM
+// accumulators, so both groups and the MMA stay busy).  Each epilogue warp drains its
+// TMEM lane quarter (32 rows of the tile), adds the weight and TMA-stores its own 32-row
+// boxes: no barrier spans warps, so the per-tile latency of one warp (TMEM load,
+// shared-memory reads, arithmetic, store) overlaps the others'.  Two rings in shared
+// memory: weight tiles (deep, since the stream needs ~100 KB of reads in flight per SM)
+// and rank chunks (up to 64 ranks of B's 128 rows and of A's 128 columns each; narrow
+// swizzles for r <= 32 so they take little room).  A bf16 weight tile is overwritten by
+// its result and stored from there; a coded tile is decoded into its group's bf16
+// staging tile.  The coded formats' scales are loaded one tile ahead.  Persistent, one
+// CTA per SM, tiles in row-major order.  Every wait is bounded (2 s); a timeout sets
+// g_merge_err, which lora_linear_merge_check reads.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,6 +34,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -44,7 +49,7 @@ enum MergeFmt { MF_BF16 = 0, MF_Q4 = 1, MF_FP8 = 2, MF_CB = 3 };
 constexpr int TM = 128, TN = 128;         // tile rows, columns
 constexpr int EPI_WARPS = 8, THREADS = 64 + 32 * EPI_WARPS;
 constexpr int MAX_WS = 8, MAX_OS = 4;     // ring depths (barrier arrays)
-constexpr int ACC = 2;                    // TMEM accumulators of TN columns
+constexpr int ACC = 4;                    // TMEM accumulators of TN columns (all 512 columns)
 constexpr int OUT_BYTES = TM * TN * 2;    // one bf16 tile (two 64-column boxes, 128B swizzle)
 constexpr int SMEM_LIMIT = 232448;        // 227 KB per CTA
 constexpr int SMEM_RESERVED = 1024 + 512; // alignment slack; barriers, codebook, TMEM slot (~310 B)
@@ -59,7 +64,7 @@ __host__ __device__ constexpr int w_tile_bytes(int wf) {
 struct MergeArgs {
     CUtensorMap tmW;    // bf16 W: box {64, 128}, 128B swizzle; FP8 codes: {128 B, 128}, 128B swizzle;
                         // 4-bit codes [d_out][d_in/2]: {64 B, 128}, 64B swizzle
-    CUtensorMap tmOut;  // bf16 W' box {64, 128}, 128B swizzle
+    CUtensorMap tmOut;  // bf16 W' box {64, 32} (one warp's rows), 128B swizzle
     CUtensorMap tmA;    // bf16 A [r][d_in] box {64, cr}, 128B swizzle (the MMA's MN-major B operand)
     CUtensorMap tmB;    // bf16 B [d_out][r] box {nb, 128}, swizzle span nb * 2 bytes (K-major A operand)
     const uint16_t *Wscale;  // bf16: 4-bit formats [d_out][d_in/64]; FP8 [d_out]
@@ -89,11 +94,37 @@ __device__ __forceinline__ void e4m3x2_f32(uint32_t two, float &lo, float &hi) {
         : "r"(two));
 }
 
+// Packed fp32 pairs (Blackwell's f32x2 arithmetic: two fp32 lanes per instruction, each
+// rounded as its scalar form).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+// bf16x2 of (s * acc + w) for two adjacent columns: one fp32 FMA each, one rounding to bf16.
+__device__ __forceinline__ uint32_t fma_bf16x2(uint32_t acc_lo, uint32_t acc_hi, uint64_t s2, uint64_t w2) {
+    uint32_t out;
+    asm("{\n\t.reg .b64 a, d;\n\t.reg .b32 e, o;\n\t"
+        "mov.b64 a, {%1, %2};\n\t"
+        "fma.rn.f32x2 d, a, %3, %4;\n\t"
+        "mov.b64 {e, o}, d;\n\t"
+        "cvt.rn.bf16x2.f32 %0, o, e;\n\t}"
+        : "=r"(out)
+        : "r"(acc_lo), "r"(acc_hi), "l"(s2), "l"(w2));
+    return out;
+}
+
 // The decoded weight of this thread's row over one 64-column half c of the tile, in
-// fp32.  wst: the weight tile in shared memory, in its format's TMA layout.
+// fp32, as 32 packed pairs (columns 2i, 2i + 1).  wst: the weight tile in shared
+// memory, in its format's TMA layout; sc: the scale that applies (coded formats).
 template <int WF>
-__device__ __forceinline__ void load_w64(const MergeArgs &p, const uint8_t *wst, const float *cbs, int lr, int c,
-                                         int64_t row, int64_t gcol, float (&w)[64]) {
+__device__ __forceinline__ void load_w64(const uint8_t *wst, const float *cbs, int lr, int c, float sc,
+                                         uint64_t (&w)[32]) {
     if (WF == MF_BF16) {
         // box c: 128 rows of 128 bytes, 16-byte piece j of row lr at (j ^ (lr & 7)) * 16
 #pragma unroll
@@ -101,14 +132,13 @@ __device__ __forceinline__ void load_w64(const MergeArgs &p, const uint8_t *wst,
             const uint4 v = *reinterpret_cast<const uint4 *>(wst + c * 16384 + lr * 128 + ((j ^ (lr & 7)) << 4));
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                w[8 * j + 2 * e] = __uint_as_float(u[e] << 16);
-                w[8 * j + 2 * e + 1] = __uint_as_float(u[e] & 0xFFFF0000u);
-            }
+            for (int e = 0; e < 4; ++e)
+                w[4 * j + e] = pack2(__uint_as_float(u[e] << 16), __uint_as_float(u[e] & 0xFFFF0000u));
         }
     } else if (WF == MF_FP8) {
-        // 128 rows of 128 code bytes (128B swizzle); this half is pieces 4c .. 4c+3
-        const float sc = row < p.d_out ? bf16f(p.Wscale[row]) : 0.f;
+        // 128 rows of 128 code bytes (128B swizzle); this half is pieces 4c .. 4c+3; sc: the
+        // row's scale; e4m3(q) * sc is exact in fp32
+        const uint64_t sc2 = pack2(sc, sc);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const uint4 v = *reinterpret_cast<const uint4 *>(wst + lr * 128 + (((4 * c + j) ^ (lr & 7)) << 4));
@@ -118,17 +148,16 @@ __device__ __forceinline__ void load_w64(const MergeArgs &p, const uint8_t *wst,
                 float f0, f1, f2, f3;
                 e4m3x2_f32(u[e] & 0xFFFFu, f0, f1);
                 e4m3x2_f32(u[e] >> 16, f2, f3);
-                w[16 * j + 4 * e] = f0 * sc;
-                w[16 * j + 4 * e + 1] = f1 * sc;
-                w[16 * j + 4 * e + 2] = f2 * sc;
-                w[16 * j + 4 * e + 3] = f3 * sc;
+                w[8 * j + 2 * e] = mul2(pack2(f0, f1), sc2);
+                w[8 * j + 2 * e + 1] = mul2(pack2(f2, f3), sc2);
             }
         }
     } else {
         // 128 rows of 64 code bytes (64B swizzle: piece j of row lr at (j ^ ((lr >> 1) & 3)) * 16);
-        // this half is pieces 2c, 2c+1; low nibble = even column; one scale per 64 columns
-        const float sc = (row < p.d_out && gcol < p.d_in) ? bf16f(p.Wscale[row * (p.d_in / 64) + gcol / 64]) : 0.f;
-        const float s7 = sc / 7.0f;
+        // this half is pieces 2c, 2c+1; a byte holds columns 2i (low nibble) and 2i + 1;
+        // sc: the half's 64-column scale
+        const uint64_t s2 = WF == MF_Q4 ? pack2(sc / 7.0f, sc / 7.0f) : pack2(sc, sc);
+        constexpr uint64_t kMinus2p23p8x2 = 0xCB000008CB000008ull;  // -(2^23 + 8) in both halves
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const uint4 v =
@@ -139,17 +168,17 @@ __device__ __forceinline__ void load_w64(const MergeArgs &p, const uint8_t *wst,
                 const uint32_t lo = u[e] & 0x0F0F0F0Fu, hi = (u[e] >> 4) & 0x0F0F0F0Fu;
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
-                    const int k = 32 * j + 8 * e + 2 * b;
+                    uint64_t f;
                     if (WF == MF_Q4) {
-                        // 2^23 + q exactly, then q - 8 exactly, then one rounding: (q - 8) * (scale / 7)
-                        const float fl = __uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + b));
-                        const float fh = __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + b));
-                        w[k] = (fl - 8388616.0f) * s7;
-                        w[k + 1] = (fh - 8388616.0f) * s7;
+                        // 2^23 + q exactly (the code under the exponent of 2^23), then q - 8
+                        // exactly, then one rounding: (q - 8) * (scale / 7)
+                        uint64_t t = pack2(__uint_as_float(__byte_perm(lo, 0x4B000000u, 0x7650 + b)),
+                                           __uint_as_float(__byte_perm(hi, 0x4B000000u, 0x7650 + b)));
+                        asm("add.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(t), "l"(kMinus2p23p8x2));
                     } else {
-                        w[k] = cbs[(lo >> (8 * b)) & 0xFu] * sc;
-                        w[k + 1] = cbs[(hi >> (8 * b)) & 0xFu] * sc;
+                        f = pack2(cbs[(lo >> (8 * b)) & 0xFu], cbs[(hi >> (8 * b)) & 0xFu]);
                     }
+                    w[16 * j + 4 * e + b] = mul2(f, s2);
                 }
             }
         }
@@ -163,7 +192,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *wring = smem;                          // n_ws weight tiles
     uint8_t *oring = wring + p.n_ws * p.w_stage;    // n_os rank chunks: [B rows | A panel]
-    uint8_t *staging = oring + p.n_os * p.o_stage;  // coded formats: 2 bf16 output tiles
+    uint8_t *staging = oring + p.n_os * p.o_stage;  // coded formats: one bf16 output tile per group
     uint64_t *bars = reinterpret_cast<uint64_t *>(staging + (kInPlace ? 0 : 2 * OUT_BYTES));
     uint64_t *wfull = bars, *wempty = bars + MAX_WS;
     uint64_t *ofull = bars + 2 * MAX_WS, *oempty = ofull + MAX_OS;
@@ -172,13 +201,12 @@ __global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__
     float *cbs = reinterpret_cast<float *>(drain + 1);  // [16]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cbs + 16);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < MAX_WS; ++b) {
             lora::mbar_init(lora::smem_u32(&wfull[b]), 1);
-            lora::mbar_init(lora::smem_u32(&wempty[b]), 1);
+            lora::mbar_init(lora::smem_u32(&wempty[b]), 4);  // the 4 warps of the tile's group
         }
         for (int b = 0; b < MAX_OS; ++b) {
             lora::mbar_init(lora::smem_u32(&ofull[b]), 1);
@@ -186,7 +214,7 @@ __global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__
         }
         for (int b = 0; b < ACC; ++b) {
             lora::mbar_init(lora::smem_u32(&tfull[b]), 1);
-            lora::mbar_init(lora::smem_u32(&tempty[b]), EPI_WARPS);
+            lora::mbar_init(lora::smem_u32(&tempty[b]), 4);
         }
         lora::mbar_init(lora::smem_u32(drain), 1);
         *abort_flag = 0;
@@ -206,6 +234,10 @@ __global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__
     lora::tc_fence_before();
     __syncthreads();
     lora::tc_fence_after();
+    // set-up above overlaps the previous kernel's tail (programmatic dependent launch);
+    // nothing below touches global memory before that kernel has completed
+    lora::grid_dep_wait();
+    lora::grid_dep_launch_dependents();
     const uint32_t tmem_base = *tmem_slot;
     const uint32_t a_box_bytes = static_cast<uint32_t>(p.cr) * 128u;  // one 64-column box of A
 
@@ -311,84 +343,105 @@ __global__ void __launch_bounds__(THREADS, 1) k_merge_tc(const __grid_constant__
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp & 3;         // TMEM lane quarter (warps 2..9 -> 2, 3, 0, 1, 2, 3, 0, 1)
-        const int c = (warp - 2) >> 2;  // this warp's 64 columns of the tile
-        const int lr = q * 32 + lane;   // accumulator row = tile row
-        const int et = threadIdx.x - 64;
-        int k = 0, prev_ws = -1;
-        for (int64_t t = blockIdx.x; t < p.tiles; t += gridDim.x, ++k) {
+        // Every warp works on its own: warp group g = (warp - 2) / 4 takes the CTA's tiles
+        // k = g, g + 2, ...; within a tile, warp w drains TMEM lane quarter w % 4 (32 rows,
+        // all 128 columns) and stores its own 32-row boxes, so no barrier spans warps.
+        const int q = warp & 3;          // TMEM lane quarter (warps 2..9 -> 2, 3, 0, 1, 2, 3, 0, 1)
+        const int g = (warp - 2) >> 2;   // warp group
+        const int lr = q * 32 + lane;    // accumulator row = tile row
+        const uint64_t s2 = pack2(p.s, p.s);
+        uint8_t *const stage_out = staging + g * OUT_BYTES;  // coded formats: this group's output tile
+        // scales of tile t for this thread's row: FP8 one per row; 4-bit one per 64 columns
+        auto load_scales = [&](int64_t t, float &s0, float &s1) {
+            s0 = s1 = 0.f;
+            if (WF == MF_BF16 || t >= p.tiles) return;
+            const int64_t row = (t / p.col_tiles) * TM + lr, col0 = (t % p.col_tiles) * TN;
+            if (row >= p.d_out) return;
+            if (WF == MF_FP8) {
+                s0 = s1 = bf16f(p.Wscale[row]);
+            } else {
+                const uint16_t *sr = p.Wscale + row * (p.d_in / 64) + col0 / 64;
+                s0 = bf16f(sr[0]);
+                if (col0 + 64 < p.d_in) s1 = bf16f(sr[1]);
+            }
+        };
+        float sc0, sc1;
+        load_scales(blockIdx.x + static_cast<int64_t>(g) * gridDim.x, sc0, sc1);
+        for (int k = g;; k += 2) {
+            const int64_t t = blockIdx.x + static_cast<int64_t>(k) * gridDim.x;
+            if (t >= p.tiles) break;
             const int buf = k % ACC, ws = k % p.n_ws;
             const uint32_t wph = static_cast<uint32_t>(k / p.n_ws) & 1u;
-            if (et == 0)
-                epi_ok[0] = (lora::wait_bounded(lora::smem_u32(&tfull[buf]), static_cast<uint32_t>(k / ACC) & 1u,
-                                                abort_flag, p.err, lora::DERR_WAIT_TMEM_FULL) &&
-                             lora::wait_bounded(lora::smem_u32(&wfull[ws]), wph, abort_flag, p.err,
-                                                lora::DERR_WAIT_FULL))
-                                ? 1
-                                : 0;
-            lora::named_bar_sync(1, 32 * EPI_WARPS);
-            const bool ok = epi_ok[0] != 0;
-            lora::named_bar_sync(1, 32 * EPI_WARPS);
-            if (!ok) break;
-            // the weight tile has landed (seen above); this wait makes its TMA writes
-            // visible to this thread and returns at once
-            lora::wait_bounded(lora::smem_u32(&wfull[ws]), wph, abort_flag, p.err, lora::DERR_WAIT_FULL);
+            // the next tile's scales load while this one is processed (DRAM latency off the path)
+            float nx0, nx1;
+            load_scales(t + 2 * static_cast<int64_t>(gridDim.x), nx0, nx1);
+            const bool ok = lora::wait_bounded(lora::smem_u32(&tfull[buf]), static_cast<uint32_t>(k / ACC) & 1u,
+                                               abort_flag, p.err, lora::DERR_WAIT_TMEM_FULL) &&
+                            lora::wait_bounded(lora::smem_u32(&wfull[ws]), wph, abort_flag, p.err,
+                                               lora::DERR_WAIT_FULL);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;  // the warp leaves together
             lora::tc_fence_after();
             const int64_t row0 = (t / p.col_tiles) * TM;
             const int64_t col0 = (t % p.col_tiles) * TN;
             const uint8_t *wst = wring + ws * p.w_stage;
-            uint8_t *out = kInPlace ? wring + ws * p.w_stage : staging + (k & 1) * OUT_BYTES;
-
-            uint32_t v0[32], v1[32];
-            const uint32_t t_addr =
-                tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * TN + c * 64);
-            lora::tmem_ld_32x32b_x32(t_addr, v0);
-            lora::tmem_ld_32x32b_x32(t_addr + 32, v1);
-            float w[64];
-            load_w64<WF>(p, wst, cbs, lr, c, row0 + lr, col0 + 64 * c, w);
-            lora::tc_wait_ld();
-            lora::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) lora::mbar_arrive(lora::smem_u32(&tempty[buf]));
-            // (in place, a thread overwrites exactly the 64 weights of its row it has just read)
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint32_t o[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 8 * j + 2 * e;
-                    const float a0 = __uint_as_float(col < 32 ? v0[col] : v1[col - 32]);
-                    const float a1 = __uint_as_float(col + 1 < 32 ? v0[col + 1] : v1[col + 1 - 32]);
-                    __nv_bfloat162 b2 = __floats2bfloat162_rn(fmaf(p.s, a0, w[col]), fmaf(p.s, a1, w[col + 1]));
-                    o[e] = *reinterpret_cast<uint32_t *>(&b2);
+            uint8_t *out = kInPlace ? wring + ws * p.w_stage : stage_out;
+            if (!kInPlace) {
+                // this warp's rows of the group's output tile: its previous store has read them
+                if (lane == 0) lora::bulk_wait_group_read<0>();
+                __syncwarp();
+            }
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * TN);
+#pragma unroll 1
+            for (int c = 0; c < 2; ++c) {
+                uint32_t v0[32], v1[32];
+                lora::tmem_ld_32x32b_x32(t_row + c * 64, v0);
+                lora::tmem_ld_32x32b_x32(t_row + c * 64 + 32, v1);
+                uint64_t w[32];
+                load_w64<WF>(wst, cbs, lr, c, c == 0 ? sc0 : sc1, w);
+                lora::tc_wait_ld();
+                if (c == 1) {
+                    lora::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) lora::mbar_arrive(lora::smem_u32(&tempty[buf]));
                 }
-                *reinterpret_cast<uint4 *>(out + c * 16384 + lr * 128 + ((j ^ (lr & 7)) << 4)) =
-                    make_uint4(o[0], o[1], o[2], o[3]);
+                // (in place, a thread overwrites exactly the 64 weights of its row it has just read)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t o[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int col = 8 * j + 2 * e;  // even: the pair never straddles v0 / v1
+                        o[e] = col < 32 ? fma_bf16x2(v0[col], v0[col + 1], s2, w[4 * j + e])
+                                        : fma_bf16x2(v1[col - 32], v1[col - 31], s2, w[4 * j + e]);
+                    }
+                    *reinterpret_cast<uint4 *>(out + c * 16384 + lr * 128 + ((j ^ (lr & 7)) << 4)) =
+                        make_uint4(o[0], o[1], o[2], o[3]);
+                }
             }
             lora::fence_proxy_async_smem();
-            lora::named_bar_sync(1, 32 * EPI_WARPS);
-            if (et == 0) {
-                for (int cc = 0; cc < 2; ++cc)
-                    if (col0 + 64 * cc < p.d_in)  // a box wholly past d_in has nothing to store
-                        lora::tma_store_2d(&p.tmOut, lora::smem_u32(out + cc * 16384),
-                                           static_cast<int32_t>(col0 + 64 * cc), static_cast<int32_t>(row0));
+            __syncwarp();
+            if (lane == 0) {
+                if (!kInPlace) lora::mbar_arrive(lora::smem_u32(&wempty[ws]));  // the codes are decoded
+                // this warp's 32 rows: two boxes of 64 columns (the 128B swizzle repeats every
+                // 8 rows, so a 32-row box at row 32q of the tile has the tile's layout)
+                if (row0 + 32 * q < p.d_out)
+                    for (int cc = 0; cc < 2; ++cc)
+                        if (col0 + 64 * cc < p.d_in)  // a box wholly past the weight has nothing to store
+                            lora::tma_store_2d(&p.tmOut, lora::smem_u32(out + cc * 16384 + q * 32 * 128),
+                                               static_cast<int32_t>(col0 + 64 * cc),
+                                               static_cast<int32_t>(row0 + 32 * q));
                 lora::bulk_commit_group();
                 if (kInPlace) {
-                    // this tile's stage holds its output until the store has read it: free
-                    // the previous tile's stage once that store (one group back) has
-                    lora::bulk_wait_group_read<1>();
-                    if (prev_ws >= 0) lora::mbar_arrive(lora::smem_u32(&wempty[prev_ws]));
-                } else {
-                    // the codes are decoded already; the other staging tile's store must have
-                    // read it before the next tile is written there
+                    // the stage holds the output until the store has read it
+                    lora::bulk_wait_group_read<0>();
                     lora::mbar_arrive(lora::smem_u32(&wempty[ws]));
-                    lora::bulk_wait_group_read<1>();
                 }
             }
-            lora::named_bar_sync(1, 32 * EPI_WARPS);
-            prev_ws = ws;
+            __syncwarp();
+            sc0 = nx0;
+            sc1 = nx1;
         }
-        if (et == 0) lora::bulk_wait_group<0>();
+        if (lane == 0) lora::bulk_wait_group<0>();
     }
 
     // ---------------------------------------------------------------- teardown
@@ -454,13 +507,32 @@ void merge_rings(int wf, int o_stage, int &n_ws, int &n_os) {
     n_ws = std::min(MAX_WS, avail / w_tile_bytes(wf));
 }
 
+// Programmatic dependent launch, as for the layer's kernels (LORA_LINEAR_PDL=0 turns it
+// off, for measurement): merges of a model's layers run back to back, and each one's
+// launch and set-up overlap the previous one's last tiles.
+bool merge_pdl_enabled() {
+    const char *v = std::getenv("LORA_LINEAR_PDL");
+    return !(v && v[0] == '0');
+}
+
 template <int WF>
 cudaError_t merge_kernel_launch(const MergeArgs &a, int grid, cudaStream_t st) {
     const int smem = SMEM_RESERVED + a.n_ws * a.w_stage + a.n_os * a.o_stage + (WF == MF_BF16 ? 0 : 2 * OUT_BYTES);
-    const cudaError_t e = cudaFuncSetAttribute(k_merge_tc<WF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(k_merge_tc<WF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_merge_tc<WF><<<grid, THREADS, smem, st>>>(a);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = merge_pdl_enabled() ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, k_merge_tc<WF>, a);
+    return e == cudaSuccess ? cudaGetLastError() : e;
 }
 
 lora_status_t merge_launch(const MergeWeight &mw, const uint16_t *A, const uint16_t *B, uint16_t *Wout, int64_t d_in,
@@ -502,7 +574,7 @@ lora_status_t merge_launch(const MergeWeight &mw, const uint16_t *A, const uint1
                                       CU_TENSOR_MAP_SWIZZLE_64B);
     }
     maps = maps &&
-           lora_host::tmap_2d(&a.tmOut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Wout, d_in, d_out, 64, TM,
+           lora_host::tmap_2d(&a.tmOut, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Wout, d_in, d_out, 64, 32,
                               CU_TENSOR_MAP_SWIZZLE_128B) &&
            lora_host::tmap_2d(&a.tmA, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A, d_in, r, 64, a.cr,
                               CU_TENSOR_MAP_SWIZZLE_128B) &&
