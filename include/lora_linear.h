@@ -39,7 +39,9 @@
  *     ceil(M/128) * ceil(max(d_in, d_out)/128) <= 2^31 - 1 (32-bit tile counts: only
  *     an output of more than 2^45 elements reaches it); 1 <= r <= 256 with r % 8 == 0; alpha finite;
  *     for *_q4 and *_nf4 also d_in % 64 == 0; for *_fp8 d_in % 16 == 0.
- *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes, be 256-byte
+ *   - The workspace must hold lora_linear_workspace_size(op, ...) bytes (the bf16
+ *     forward also runs in less, down to the size without its K-split hand-over buffer,
+ *     cutting its last wave along N instead: see lora_plan_t.fwd_tail), be 256-byte
  *     aligned, be zero-filled before its first use, and must not be used by two calls
  *     that may run at the same time.  Every call that completes leaves the workspace's
  *     arrival counters at zero again, so a workspace is zeroed once, not per call
@@ -115,7 +117,11 @@ typedef struct {
     int32_t g_cluster;  /* side s.g + dB: CTAs per cluster, 1, 2 or 4 (they split d_out) */
     int32_t g_group;    /* side s.g + dB: 128-token blocks per round, 1..6, with g_group * r <= 64 */
     int32_t da_cluster; /* side dA: CTAs per cluster, 1, 2 or 4 (they split the tokens) */
-    int32_t fwd_tail;   /* forward main GEMM: 1 a partial last wave is cut along N, 2 it is not */
+    int32_t fwd_tail;   /* forward main GEMM: 1 a partial last wave is cut along N, 2 it is not,
+                           3 (bf16 weight; the library's choice there) each of its tiles is cut
+                           along K into two halves on two CTA pairs, the first handing its fp32
+                           accumulator to the second through the workspace (a workspace below
+                           lora_linear_workspace_size's figure but at least the rest cuts along N) */
     int32_t dx_overlap; /* backward: 1 dA (and dB) start beside the dX GEMM's last wave, whose tiles
                            stay whole (the library's choice); 2 they follow the dX GEMM, whose
                            last wave is cut along N where it can be */

@@ -424,6 +424,7 @@ Split choose_split(int64_t mt, int64_t kb, int sms) {
 }
 
 constexpr int PLAN_SMS = 148;  // SMs a launch uses at most (sizes splits and the workspace)
+constexpr int KSPLIT_MIN_KB = 32;  // K blocks of 64 below which the forward's tail is not cut along K
 
 // Main-GEMM schedule: whole 128 x 256 tiles in waves over G CTAs; a partial last
 // wave of R tiles is cut along N into 2 or 4 narrower tiles (one per CTA) when they
@@ -546,7 +547,11 @@ struct Plan {
     bool side = false;          // s.xa on the side kernels (r <= 64)
     bool side_bwd = false;      // s.g + dB and dA on the side kernels (r <= 32)
     SidePlan sx, sg, sd;        // s.xa, s.g + dB partials, dA + dB
-    bool fwd_tail = true;       // forward main GEMM: cut a partial last wave along N
+    bool fwd_tail = true;       // forward main GEMM: cut a partial last wave (along N, or along K below)
+    bool fwd_ksplit = false;    // bf16 forward: cut it along K instead, tiles handed over in fp32
+    size_t ks_part = 0, ks_flag = 0;  // K-split hand-over buffers (the end of the workspace)
+    int ks_tiles = 0;           // tail tiles they hold
+    size_t total_min = 0;       // the workspace without them (the forward then cuts along N)
     int dx_mode = 0;            // 0: dA beside the dX GEMM's last wave unless that wave can be cut
                                 // along N (then dA follows); 1: always beside; 2: always after
     int da_force_c = 0;         // dA's cluster size if the plan fixes it
@@ -593,6 +598,7 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
     pl->side = ov.side_fwd ? ov.side_fwd == 1 : (r <= SIDE_MAX_R && side_enabled());
     pl->side_bwd = bwd && (ov.side_bwd ? ov.side_bwd == 1 : (r <= SIDE_DEFAULT_R_BWD && side_enabled()));
     pl->fwd_tail = ov.fwd_tail != 2;
+    pl->fwd_ksplit = op == LORA_OP_FWD && (ov.fwd_tail == 0 || ov.fwd_tail == 3);
     pl->dx_mode = ov.dx_overlap;
     pl->da_force_c = ov.da_cluster;
     // split-K counters and partials (every s.xa when not on the side kernels; the
@@ -629,6 +635,23 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
             off = align256(off + static_cast<size_t>(pl->s_db.splits) * mt_out * BM * r * 4);
             pl->part_da = off;
             off = align256(off + static_cast<size_t>(pl->s_da.splits) * mt_in * BM * r * 4);
+        }
+    }
+    pl->total_min = off;
+    if (pl->fwd_ksplit) {
+        // the last wave of the CTA-pair forward GEMM (256 x 256 tiles on PLAN_SMS / 2 clusters):
+        // K-split when it holds at most half as many tiles as there are clusters
+        // and its K (d_in + r) is at least KSPLIT_MIN_KB blocks: half a tile must outweigh the
+        // hand-over (~2 us)
+        const int64_t C = PLAN_SMS / 2, T = cdiv(M, 256) * cdiv(d_out, 256), R = T % C;
+        if (T >= C && R > 0 && 2 * R <= C && cdiv(d_in, BK) + cdiv(r, BK) >= KSPLIT_MIN_KB) {
+            pl->ks_tiles = static_cast<int>(R);
+            pl->ks_flag = off;
+            off = align256(off + static_cast<size_t>(R) * 4 * sizeof(int));
+            pl->ks_part = off;
+            off = align256(off + static_cast<size_t>(R) * 256 * 256 * 4);
+        } else {
+            pl->fwd_ksplit = false;
         }
     }
     pl->total = off;
@@ -681,7 +704,8 @@ lora_status_t prepare(int op, int64_t M, int64_t d_in, int64_t d_out, int r, voi
     make_plan(op, M, d_in, d_out, r, PLAN_SMS, &c->plan);
     if (!ws) return LORA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return LORA_ERR_MISALIGNED;
-    if (ws_bytes < c->plan.total) return LORA_ERR_WORKSPACE;
+    if (ws_bytes < c->plan.total_min) return LORA_ERR_WORKSPACE;
+    if (ws_bytes < c->plan.total) c->plan.fwd_ksplit = false;  // no room for the K-split hand-over
     c->ws = static_cast<uint8_t *>(ws);
     c->st = static_cast<cudaStream_t>(stream);
     return LORA_OK;
@@ -900,8 +924,10 @@ struct MainOperands {
 };
 
 // `idle_sms` (optional) receives how many SMs the last wave leaves without work.
+// `ksplit`: cut a partial last wave along K (bf16 weight, workspace permitting) rather
+// than along N.
 lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t N, int64_t K0, int r, bool b_mn,
-                        int kind, bool allow_tail_split, int *idle_sms = nullptr) {
+                        int kind, bool allow_tail_split, int *idle_sms = nullptr, bool ksplit = false) {
     GemmArgs a = base_args(c);
     a.kb0 = static_cast<int>(cdiv(K0, BK));
     a.kb1 = static_cast<int>(cdiv(r, BK));
@@ -932,11 +958,17 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
         a.num_tiles = static_cast<int>(T);
         a.group_m = std::min(a.m_tiles, 8);
         const int64_t W = T / pair_C, R = T % pair_C;
-        const bool split = allow_tail_split && W >= 1 && R > 0 && 2 * R <= pair_C;
-        a.dp_tiles = static_cast<int>(split ? W * pair_C : T);
-        a.dp_waves = static_cast<int>(split ? W : cdiv(T, pair_C));
-        a.tail_tiles = static_cast<int>(split ? R : 0);
+        const bool kcut = ksplit && !q4 && W >= 1 && R > 0 && 2 * R <= pair_C && R <= c.plan.ks_tiles;
+        const bool split = !kcut && allow_tail_split && W >= 1 && R > 0 && 2 * R <= pair_C;
+        a.dp_tiles = static_cast<int>(split || kcut ? W * pair_C : T);
+        a.dp_waves = static_cast<int>(split || kcut ? W : cdiv(T, pair_C));
+        a.tail_tiles = static_cast<int>(split || kcut ? R : 0);
         a.tail_split = split ? 2 : 1;
+        if (kcut) {
+            a.tail_ksplit = 1;
+            a.ks_part = reinterpret_cast<float *>(c.ws + c.plan.ks_part);
+            a.ks_flag = reinterpret_cast<int *>(c.ws + c.plan.ks_flag);
+        }
         if (b_mn) {
             if (!q4 && !tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
             if (!tmap_bf16(&a.tmB1, o.B1, N, r, 64, 64)) return LORA_ERR_CUDA;
@@ -948,7 +980,7 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
                 if (!tmap_bf16(&a.tmB1n, o.B1, r, N, 64, CTA_BN / 2)) return LORA_ERR_CUDA;
             }
         }
-        const int clusters = split ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
+        const int clusters = split || kcut ? pair_C : static_cast<int>(std::min<int64_t>(T, pair_C));
         if (idle_sms) *idle_sms = (!split && R > 0 && W >= 1) ? c.info->sms - static_cast<int>(2 * R) : 0;
         cudaError_t e;
         if (o.wf == WF_Q4)
@@ -1063,7 +1095,7 @@ lora_status_t fwd_impl(const uint16_t *x, const Weight &wt, const uint16_t *A, c
     uint16_t *sxa = xa_save ? xa_save : reinterpret_cast<uint16_t *>(c.ws + c.plan.xa);
     LORA_TRY(c.plan.side ? side_xa(c, x, A, sxa, M, d_in, r, s) : step_xa(c, x, A, sxa, M, d_in, r, s));
     const MainOperands o = main_operands(wt, x, sxa, B, h, d_out, d_in);
-    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, c.plan.fwd_tail);
+    return step_main(c, o, M, d_out, d_in, r, false, LORA_K_FWD_MAIN, c.plan.fwd_tail, nullptr, c.plan.fwd_ksplit);
 }
 
 lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, const uint16_t *A,
@@ -1127,6 +1159,17 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
 
 // ====================================================================== C ABI
 extern "C" {
+
+// The smallest workspace the operation runs in (the bf16 forward without its K-split
+// hand-over buffer); 0 for invalid arguments.  Used by the workspace-free forward.
+size_t lora_workspace_min(int op, int64_t M, int64_t d_in, int64_t d_out, int r) {
+    if (op < LORA_OP_FWD || op > LORA_OP_BWD_NF4) return 0;
+    const int wf = op >= LORA_OP_FWD_NF4 ? WF_CB : op >= LORA_OP_FWD_FP8 ? WF_FP8 : op >= LORA_OP_FWD_Q4 ? WF_Q4 : WF_BF16;
+    if (check_shapes(M, d_in, d_out, r, 1.0f, wf) != LORA_OK) return 0;
+    Plan pl;
+    make_plan(op, M, d_in, d_out, r, PLAN_SMS, &pl);
+    return pl.total_min;
+}
 
 size_t lora_linear_workspace_size(int op, int64_t M, int64_t d_in, int64_t d_out, int r) {
     if (op < LORA_OP_FWD || op > LORA_OP_BWD_NF4) return 0;
@@ -1216,7 +1259,7 @@ lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r
         };
         if (!in(q.side_fwd, {0, 1, 2}) || !in(q.side_bwd, {0, 1, 2}) || !in(q.xa_cluster, {0, 1, 2, 4}) ||
             !in(q.g_cluster, {0, 1, 2, 4}) || q.g_group < 0 || q.g_group > 6 || !in(q.da_cluster, {0, 1, 2, 4}) ||
-            !in(q.fwd_tail, {0, 1, 2}) || !in(q.dx_overlap, {0, 1, 2}))
+            !in(q.fwd_tail, {0, 1, 2, 3}) || !in(q.dx_overlap, {0, 1, 2}))
             return LORA_ERR_INVALID_ARG;
         for (int i = 0; i < 4; ++i)
             if (q.splitk[i] < 0 || q.splitk[i] > 64) return LORA_ERR_INVALID_ARG;
@@ -1258,7 +1301,9 @@ lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_ou
     plan->da_cluster = pl.side_bwd ? side_plan(pl.sd.n_out, pl.sd.n_red, PLAN_SMS,
                                                overlap ? SIDE_MAX_C_DA : SIDE_MAX_C, pl.da_force_c).C
                                    : 0;
-    plan->fwd_tail = pl.fwd_tail ? 1 : 2;
+    Plan fp;  // the forward of the same weight format (a backward plan reports the forward's tail)
+    make_plan(op & ~1, M, d_in, d_out, r, PLAN_SMS, &fp);
+    plan->fwd_tail = !fp.fwd_tail ? 2 : fp.fwd_ksplit ? 3 : 1;
     plan->dx_overlap = bwd ? (overlap ? 1 : 2) : 0;
     const bool sk_bwd = bwd && !pl.side_bwd;
     plan->splitk[0] = pl.side ? 0 : pl.s_xa.splits;

@@ -87,11 +87,16 @@ lora_status_t scratch_address(cudaStream_t stream, void **out) {
 
 }  // namespace
 
+// In lora_linear.cu (same library, not exported).
+extern "C" size_t lora_workspace_min(int op, int64_t M, int64_t d_in, int64_t d_out, int r);
+
 extern "C" LORA_API lora_status_t lora_linear_fwd_noalloc(const uint16_t *x, const uint16_t *W,
                                                           const uint16_t *A, const uint16_t *B, uint16_t *h,
                                                           uint16_t *xa_save, int64_t M, int64_t d_in,
                                                           int64_t d_out, int r, float alpha, void *stream) {
-    const size_t need = lora_linear_workspace_size(LORA_OP_FWD, M, d_in, d_out, r);
+    // the forward's smallest workspace: without room for the K-split hand-over buffer it
+    // cuts a partial last wave along N, computing the same function
+    const size_t need = lora_workspace_min(LORA_OP_FWD, M, d_in, d_out, r);
     if (need == 0) return LORA_ERR_INVALID_ARG;
     if (need > kNoallocScratchBytes) return LORA_ERR_WORKSPACE;  // problem too large for the fixed scratch
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -87,10 +87,14 @@ struct SideCfg {
     static_assert(STAGE_BYTES % 1024 == 0, "stage tiles stay 1024-byte aligned");
 };
 
+// dB accumulators of the s.g + dB kernel: the epilogue drains one per 128-column block
+// while the MMA fills the others, so its drain latency stays off the stream.
+constexpr int SIDE_NDB = 4;
+
 // TMEM columns a side kernel allocates: XA one accumulator of nr <= 64 columns, DA one
-// of nb; GDB `group` g accumulators and two dB accumulators of nb columns each.
+// of nb; GDB `group` g accumulators and SIDE_NDB dB accumulators of nb columns each.
 __host__ __device__ constexpr int side_tmem_cols(int mode, int group, int nb) {
-    const int need = mode == SIDE_GDB ? (group + 2) * nb : mode == SIDE_DA ? nb : 64;
+    const int need = mode == SIDE_GDB ? (group + SIDE_NDB) * nb : mode == SIDE_DA ? nb : 64;
     return need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
 }
 
@@ -128,10 +132,10 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
     uint64_t *full_bar = bars;                 // [STAGES]
     uint64_t *empty_bar = bars + STAGES;       // [STAGES]
     uint64_t *acc_bar = bars + 2 * STAGES;     // [1] the round's accumulators are complete
-    uint64_t *dbf_bar = bars + 2 * STAGES + 1; // [2] GDB: a dB accumulator is complete
-    uint64_t *dbe_bar = bars + 2 * STAGES + 3; // [2] GDB: a dB accumulator has been drained
-    uint64_t *drain_bar = bars + 2 * STAGES + 5;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 6);
+    uint64_t *dbf_bar = bars + 2 * STAGES + 1;             // [SIDE_NDB] GDB: a dB accumulator is complete
+    uint64_t *dbe_bar = dbf_bar + SIDE_NDB;                // [SIDE_NDB] GDB: a dB accumulator has been drained
+    uint64_t *drain_bar = dbe_bar + SIDE_NDB;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *epi_ok = reinterpret_cast<volatile int *>(tmem_slot + 2);
 
@@ -157,7 +161,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
             mbar_init(smem_u32(&empty_bar[s]), 1);
         }
         mbar_init(smem_u32(acc_bar), 1);
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < SIDE_NDB; ++b) {
             mbar_init(smem_u32(&dbf_bar[b]), 1);
             mbar_init(smem_u32(&dbe_bar[b]), 4);
         }
@@ -284,8 +288,8 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                     uint32_t db_tmem = 0;
                     if (MODE == SIDE_GDB) {
                         // the dB accumulator of this column block: free once drained
-                        const int b = db_use & 1;
-                        if (!wait_bounded(smem_u32(&dbe_bar[b]), ((db_use >> 1) & 1) ^ 1u, abort_flag, p.err,
+                        const int b = db_use % SIDE_NDB;
+                        if (!wait_bounded(smem_u32(&dbe_bar[b]), ((db_use / SIDE_NDB) & 1) ^ 1u, abort_flag, p.err,
                                           DERR_WAIT_TMEM_EMPTY)) {
                             ok = false;
                             break;
@@ -342,7 +346,7 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
                         }
                     }
                     if (MODE == SIDE_GDB && ok) {
-                        tc_commit(smem_u32(&dbf_bar[db_use & 1]));
+                        tc_commit(smem_u32(&dbf_bar[db_use % SIDE_NDB]));
                         ++db_use;
                     }
                 }
@@ -360,35 +364,37 @@ __global__ void __launch_bounds__(SIDE_THREADS, 1) k_side(const __grid_constant_
             const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(qd * 32) << 16);
             if (MODE == SIDE_GDB && has_work) {
                 // dB partial of each column block of this CTA, for this round's tokens
+                // Each warp drains its own 32 rows on its own (its lanes wait, the warp votes),
+                // with one TMEM load of all nb columns: no barrier spans warps, so the drain's
+                // latency overlaps the MMAs into the other dB accumulators.
                 for (int kb = kb_lo; kb < kb_hi; ++kb) {
-                    const int b = db_use & 1;
-                    if (et == 0)
-                        epi_ok[0] = (!*abort_flag && wait_bounded(smem_u32(&dbf_bar[b]), (db_use >> 1) & 1u,
-                                                                  abort_flag, p.err, DERR_WAIT_TMEM_FULL))
-                                        ? 1
-                                        : 0;
-                    named_bar_sync(1, 128);
-                    const bool okk = epi_ok[0] != 0;
-                    named_bar_sync(1, 128);  // everyone has read epi_ok before it is reused
-                    if (!okk) break;
+                    const int b = db_use % SIDE_NDB;
+                    const bool okk = !*abort_flag && wait_bounded(smem_u32(&dbf_bar[b]), (db_use / SIDE_NDB) & 1u,
+                                                                  abort_flag, p.err, DERR_WAIT_TMEM_FULL);
+                    if (!__all_sync(0xFFFFFFFFu, okk)) break;
                     tc_fence_after();
                     const int n = kb * 128 + row;
                     float *dst = p.db_part + (static_cast<int64_t>(t) * p.d_out + n) * r;
-                    for (int c0 = 0; c0 < r; c0 += 8) {
-                        uint32_t v[8];
-                        tmem_ld_32x32b_x8(lane_base + static_cast<uint32_t>((p.group + b) * nb + c0), v);
-                        tc_wait_ld();
-                        if (n < p.d_out) {
-                            float4 *d4 = reinterpret_cast<float4 *>(dst + c0);
-                            d4[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]),
-                                                __uint_as_float(v[3]));
-                            d4[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]),
-                                                __uint_as_float(v[7]));
-                        }
+                    uint32_t v[32];
+                    const uint32_t taddr = lane_base + static_cast<uint32_t>((p.group + b) * nb);
+                    if (nb == 16) {
+                        uint32_t (&v16)[16] = *reinterpret_cast<uint32_t(*)[16]>(v);
+                        tmem_ld_32x32b_x16(taddr, v16);
+                    } else {
+                        tmem_ld_32x32b_x32(taddr, v);
                     }
+                    tc_wait_ld();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&dbe_bar[b]));
+                    if (n < p.d_out) {
+#pragma unroll
+                        for (int c0 = 0; c0 < 32; c0 += 4)  // constant indices keep v in registers
+                            if (c0 < r)
+                                *reinterpret_cast<float4 *>(dst + c0) =
+                                    make_float4(__uint_as_float(v[c0]), __uint_as_float(v[c0 + 1]),
+                                                __uint_as_float(v[c0 + 2]), __uint_as_float(v[c0 + 3]));
+                    }
                     ++db_use;
                 }
             }

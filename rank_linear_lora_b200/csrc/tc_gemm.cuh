@@ -58,6 +58,7 @@ enum DevErr {
     DERR_WAIT_TMEM_EMPTY = 0x103,
     DERR_WAIT_TMEM_FULL = 0x104,
     DERR_WAIT_DRAIN = 0x105,
+    DERR_WAIT_PARTIAL = 0x106,  // a K-split tail tile's first half never published its partial
 };
 
 // One skinny split-K problem: output [rows_valid, n_valid] over K = kb0 * 64.
@@ -108,7 +109,23 @@ struct GemmArgs {
     // without waiting and waits for the predecessor only before it exits; its own
     // completion then still implies the predecessor's (stream order is kept).
     int defer_dep_wait;
+    // CTA-pair GEMM, bf16 weight: 1 cuts each last-wave tile along K into two items on
+    // two clusters; the first hands its fp32 accumulator over through ks_part and raises
+    // its flag in ks_flag (zero on entry, cleared by the reader), the second adds it.
+    int tail_ksplit;
+    float *ks_part;          // [tail tile][CTA rank][chunk (4)][16-byte column group (16)][row (128)] float4
+    int *ks_flag;            // [tail tile][CTA rank]
 };
+
+// Release / acquire of a global int at GPU scope (the K-split tail's hand-over).
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 // Trace record of one CTA (globaltimer ns unless noted).
 enum TraceField {
@@ -175,6 +192,25 @@ __device__ __forceinline__ bool wait_count_bounded(uint32_t addr, uint32_t targe
     for (uint32_t i = 1;; ++i) {
         __nanosleep(32);
         if (ld_acquire_shared(addr) >= target) return true;
+        if ((i & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                atomicCAS(err, 0, code);
+                return false;
+            }
+        }
+    }
+}
+
+// Bounded wait until a global flag is nonzero (acquire at GPU scope); false on timeout
+// (recording `code`) or abort, as wait_bounded.
+__device__ __forceinline__ bool wait_flag_bounded(const int *flag, volatile int *abort_flag, int *err, int code) {
+    if (ld_acquire_gpu(flag) != 0) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(flag) != 0) return true;
         if ((i & 31u) == 0) {
             if (*abort_flag) return false;
             if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {

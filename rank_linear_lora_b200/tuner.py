@@ -36,7 +36,7 @@ def field_options(r: int) -> dict:
         "g_cluster": [1, 2, 4],
         "g_group": [a for a in range(1, 7) if a * r <= 64],
         "da_cluster": [1, 2, 4],
-        "fwd_tail": [1, 2],
+        "fwd_tail": [1, 2, 3],
         "dx_overlap": [1, 2],
     }
     return opts

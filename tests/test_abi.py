@@ -34,8 +34,13 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     for op in (L.OP_FWD, L.OP_BWD, L.OP_FWD_Q4, L.OP_BWD_Q4):
         assert L.lora_linear_workspace_size(op, 4096, 8192, 28672, 16) > 0
+    # the bf16 forward holds the K-split hand-over buffer when its last wave is cut along K
+    # (34 tail tiles of 256 x 256 fp32 at 4096 x 4096 x 4096); the 4-bit forward does not
+    assert L.lora_linear_workspace_size(L.OP_FWD, 4096, 4096, 4096, 8) >= 34 * 256 * 256 * 4
     assert L.lora_linear_workspace_size(L.OP_BWD, 4096, 4096, 4096, 8) > L.lora_linear_workspace_size(
-        L.OP_FWD, 4096, 4096, 4096, 8)
+        L.OP_FWD_Q4, 4096, 4096, 4096, 8)
+    assert L.lora_linear_get_plan(L.OP_FWD, 4096, 4096, 4096, 8)["fwd_tail"] == 3
+    assert L.lora_linear_get_plan(L.OP_FWD_Q4, 4096, 4096, 4096, 8)["fwd_tail"] == 1
     # invalid sizes -> 0
     assert L.lora_linear_workspace_size(L.OP_FWD, 0, 256, 256, 8) == 0
     assert L.lora_linear_workspace_size(L.OP_FWD, 64, 250, 256, 8) == 0
@@ -154,7 +159,7 @@ def test_fp8_validation_before_any_device_work(lib):
     assert {"lora_linear_fwd_fp8", "lora_linear_bwd_fp8"} <= set(L.declared_functions())
     for op in (L.OP_FWD_FP8, L.OP_BWD_FP8):
         assert L.lora_linear_workspace_size(op, 4096, 4096, 4096, 8) == L.lora_linear_workspace_size(
-            op - 4, 4096, 4096, 4096, 8)  # the workspace does not depend on the weight's format
+            op - 2, 4096, 4096, 4096, 8)  # the coded weights' workspaces do not depend on the format
     assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1040, 256, 8) > 0      # d_in % 16 == 0 suffices
     assert L.lora_linear_workspace_size(L.OP_FWD_FP8, 64, 1032, 256, 8) == 0     # d_in % 16 != 0
     assert L.lora_linear_workspace_size(8, 64, 256, 256, 8) == 0

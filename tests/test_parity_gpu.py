@@ -190,6 +190,53 @@ def test_tail_wave_split(shape):
     compare_all(dl.results(), oracle_ref(inp), spec.s)
 
 
+# Forward shapes whose CTA-pair GEMM (256 x 256 tiles on 74 pairs) leaves a last wave of
+# at most 37 tiles: each is cut along K into two items on two pairs (the library's
+# choice for the bf16 weight), the first handing its fp32 accumulator to the second.
+KSPLIT = [
+    (1280, 4096, 4096, 8),    # 80 tiles: 6 tail tiles, 32 + 33 K blocks
+    (1200, 2040, 4000, 24),   # ragged M, K and N; the rank-r block in the second half
+    (1280, 2048, 4096, 136),  # three rank-r blocks, all in the second half
+    (2304, 3072, 2816, 16),   # 99 tiles: 25 tail tiles on 50 pairs
+]
+
+
+def _check_forward(dl, ref, s):
+    got = dl.results()
+    assert_close("h", got["h"], ref["h"], TOL_HX, RMS_HX)
+    assert_close("xa_save", got["xa"], s * ref["xa"], (2 ** -8, 1e-6), RMS_HX)
+
+
+@pytest.mark.parametrize("shape", KSPLIT, ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_forward_last_wave_cut_along_k(shape):
+    """Every element against the oracle with the K-split tail and with the N-split one
+    (plan override), and the K-split result the same bit for bit on a second call."""
+    M, di, do, r = shape
+    assert L.lora_linear_get_plan(L.OP_FWD, M, di, do, r)["fwd_tail"] == 3
+    assert L.lora_linear_get_plan(L.OP_FWD, M, 1024, do, r)["fwd_tail"] == 1  # short K: cut along N
+    spec = inputs.LayerSpec("ksplit", M, di, do, r, alpha=2.0 * r, seed=0x4B + M + di)
+    inp = inputs.make_inputs(spec)
+    ref = oracle_ref(inp)
+    dl = DeviceLayer(inp)
+    dl.forward()
+    dl.check()
+    h1 = dl.h.clone()
+    _check_forward(dl, ref, spec.s)
+    dl.forward()
+    dl.check()
+    assert torch.equal(h1.view(torch.int16), dl.h.view(torch.int16)), "K-split tail not deterministic"
+    plan = L.lora_linear_get_plan(L.OP_FWD, M, di, do, r)
+    plan["fwd_tail"] = 1
+    try:
+        L.lora_linear_set_plan(M, di, do, r, plan)
+        dn = DeviceLayer(inp)
+        dn.forward()
+        dn.check()
+        _check_forward(dn, ref, spec.s)
+    finally:
+        L.lora_linear_set_plan(M, di, do, r, None)
+
+
 @pytest.mark.parametrize("shape", [TAIL_WAVE[0], TAIL_WAVE[1], TAIL_WAVE[2]], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
 def test_single_sm_main_gemm(shape, monkeypatch):
     """The single-SM main-GEMM kernel (chosen when CTA pairs are unavailable) on the

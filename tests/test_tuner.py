@@ -40,7 +40,7 @@ def test_set_get_clear_and_workspace_follows():
 
 @pytest.mark.parametrize("bad,status", [
     (dict(side_fwd=3), 1), (dict(xa_cluster=3), 1), (dict(xa_cluster=8), 1), (dict(g_group=7), 1),
-    (dict(g_group=-1), 1), (dict(da_cluster=8), 1), (dict(fwd_tail=3), 1), (dict(splitk=[65, 0, 0, 0]), 1),
+    (dict(g_group=-1), 1), (dict(da_cluster=8), 1), (dict(fwd_tail=4), 1), (dict(splitk=[65, 0, 0, 0]), 1),
     (dict(splitk=[0, -1, 0, 0]), 1)])
 def test_rejects_out_of_range_fields(bad, status):
     with pytest.raises(L.LoraError) as e:

@@ -40,10 +40,19 @@ def test_fwd_noalloc_matches_fwd_on_two_calls(shape):
     x, W, A, B = (dev_bf16(a) for a in (inp.x, inp.W, inp.A, inp.B))
     h_ref = torch.empty(M, d_out, dtype=torch.bfloat16, device="cuda")
     xa_ref = torch.empty(M, r, dtype=torch.bfloat16, device="cuda")
-    ws = L.workspace(L.OP_FWD, M, d_in, d_out, r)
+    # The ordinary forward on a workspace of the scratch's 4 MiB: the same plan as the
+    # workspace-free call (the full workspace may add the K-split hand-over buffer, whose
+    # last-wave tiles sum in another order).
+    ws = torch.zeros(4 << 20, dtype=torch.uint8, device="cuda")
     L.lora_linear_fwd(x, W, A, B, h_ref, xa_ref, spec.alpha, ws)
     L.lora_linear_check(ws)
     _oracle_check(inp, h_ref, xa_ref)
+    # and on the full workspace (K-split tail where the shape has one), against the oracle
+    h_full = torch.empty_like(h_ref)
+    ws_full = L.workspace(L.OP_FWD, M, d_in, d_out, r)
+    L.lora_linear_fwd(x, W, A, B, h_full, None, spec.alpha, ws_full)
+    L.lora_linear_check(ws_full)
+    _oracle_check(inp, h_full, xa_ref)
     for call in range(2):
         h = torch.full((M, d_out), float("nan"), dtype=torch.bfloat16, device="cuda")
         xa = torch.full((M, r), float("nan"), dtype=torch.bfloat16, device="cuda")
