@@ -124,7 +124,8 @@ typedef struct {
                            lora_linear_workspace_size's figure but at least the rest cuts along N) */
     int32_t dx_overlap; /* backward: 1 dA (and dB) start beside the dX GEMM's last wave, whose tiles
                            stay whole (the library's choice); 2 they follow the dX GEMM, whose
-                           last wave is cut along N where it can be */
+                           last wave is cut along N where it can be; 3 (bf16 weight) they follow
+                           it, its last wave cut along K as fwd_tail 3 describes */
     int32_t splitk[4];  /* split-K kernels: K splits (1 .. 64) of s.xa, s.g, dB and dA */
 } lora_plan_t;
 

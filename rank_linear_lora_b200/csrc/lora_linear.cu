@@ -549,6 +549,7 @@ struct Plan {
     SidePlan sx, sg, sd;        // s.xa, s.g + dB partials, dA + dB
     bool fwd_tail = true;       // forward main GEMM: cut a partial last wave (along N, or along K below)
     bool fwd_ksplit = false;    // bf16 forward: cut it along K instead, tiles handed over in fp32
+    bool dx_ksplit = false;     // bf16 backward: the dX GEMM's last wave cut along K, dA + dB after it
     size_t ks_part = 0, ks_flag = 0;  // K-split hand-over buffers (the end of the workspace)
     int ks_tiles = 0;           // tail tiles they hold
     size_t total_min = 0;       // the workspace without them (the forward then cuts along N)
@@ -638,20 +639,22 @@ bool make_plan(int op, int64_t M, int64_t d_in, int64_t d_out, int r, int sms, P
         }
     }
     pl->total_min = off;
-    if (pl->fwd_ksplit) {
-        // the last wave of the CTA-pair forward GEMM (256 x 256 tiles on PLAN_SMS / 2 clusters):
-        // K-split when it holds at most half as many tiles as there are clusters
-        // and its K (d_in + r) is at least KSPLIT_MIN_KB blocks: half a tile must outweigh the
-        // hand-over (~2 us)
-        const int64_t C = PLAN_SMS / 2, T = cdiv(M, 256) * cdiv(d_out, 256), R = T % C;
-        if (T >= C && R > 0 && 2 * R <= C && cdiv(d_in, BK) + cdiv(r, BK) >= KSPLIT_MIN_KB) {
+    pl->dx_ksplit = op == LORA_OP_BWD && ov.dx_overlap == 3;
+    if (pl->fwd_ksplit || pl->dx_ksplit) {
+        // the last wave of the CTA-pair GEMM (256 x 256 tiles on PLAN_SMS / 2 clusters; the
+        // forward's N = d_out, K = d_in, dX's N = d_in, K = d_out): K-split when it holds at
+        // most half as many tiles as there are clusters and K + r is at least KSPLIT_MIN_KB
+        // blocks (half a tile must outweigh the hand-over)
+        const int64_t N = pl->fwd_ksplit ? d_out : d_in, K = pl->fwd_ksplit ? d_in : d_out;
+        const int64_t C = PLAN_SMS / 2, T = cdiv(M, 256) * cdiv(N, 256), R = T % C;
+        if (T >= C && R > 0 && 2 * R <= C && cdiv(K, BK) + cdiv(r, BK) >= KSPLIT_MIN_KB) {
             pl->ks_tiles = static_cast<int>(R);
             pl->ks_flag = off;
             off = align256(off + static_cast<size_t>(R) * 4 * sizeof(int));
             pl->ks_part = off;
             off = align256(off + static_cast<size_t>(R) * 256 * 256 * 4);
         } else {
-            pl->fwd_ksplit = false;
+            pl->fwd_ksplit = pl->dx_ksplit = false;
         }
     }
     pl->total = off;
@@ -668,7 +671,7 @@ bool dx_overlaps(const Plan &pl, int64_t M, int64_t d_in, int pair_clusters, boo
     (void)d_in;
     (void)pair_clusters;
     (void)coded;
-    return pl.dx_mode != 2;
+    return pl.dx_mode != 2 && !pl.dx_ksplit;
 }
 
 // ------------------------------------------------------------------ validation
@@ -705,7 +708,7 @@ lora_status_t prepare(int op, int64_t M, int64_t d_in, int64_t d_out, int r, voi
     if (!ws) return LORA_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(ws) & 255u) return LORA_ERR_MISALIGNED;
     if (ws_bytes < c->plan.total_min) return LORA_ERR_WORKSPACE;
-    if (ws_bytes < c->plan.total) c->plan.fwd_ksplit = false;  // no room for the K-split hand-over
+    if (ws_bytes < c->plan.total) c->plan.fwd_ksplit = c->plan.dx_ksplit = false;  // no room for the hand-over
     c->ws = static_cast<uint8_t *>(ws);
     c->st = static_cast<cudaStream_t>(stream);
     return LORA_OK;
@@ -1133,7 +1136,7 @@ lora_status_t bwd_impl(const uint16_t *dY, const uint16_t *x, const Weight &wt, 
     if (dX) {
         // W [d_out, d_in] (or its codes) and A [r, d_in] are read MN-major (d_in contiguous).
         const MainOperands o = main_operands(wt, dY, sg, A, dX, d_out, d_in);
-        LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle));
+        LORA_TRY(step_main(c, o, M, d_in, d_out, r, true, LORA_K_DX_MAIN, !overlap, &idle, c.plan.dx_ksplit));
     }
     if (c.plan.side_bwd) {
         // dA reads nothing the dX GEMM writes, so it waits for that GEMM only before it
@@ -1259,7 +1262,7 @@ lora_status_t lora_linear_set_plan(int64_t M, int64_t d_in, int64_t d_out, int r
         };
         if (!in(q.side_fwd, {0, 1, 2}) || !in(q.side_bwd, {0, 1, 2}) || !in(q.xa_cluster, {0, 1, 2, 4}) ||
             !in(q.g_cluster, {0, 1, 2, 4}) || q.g_group < 0 || q.g_group > 6 || !in(q.da_cluster, {0, 1, 2, 4}) ||
-            !in(q.fwd_tail, {0, 1, 2, 3}) || !in(q.dx_overlap, {0, 1, 2}))
+            !in(q.fwd_tail, {0, 1, 2, 3}) || !in(q.dx_overlap, {0, 1, 2, 3}))
             return LORA_ERR_INVALID_ARG;
         for (int i = 0; i < 4; ++i)
             if (q.splitk[i] < 0 || q.splitk[i] > 64) return LORA_ERR_INVALID_ARG;
@@ -1304,7 +1307,7 @@ lora_status_t lora_linear_get_plan(int op, int64_t M, int64_t d_in, int64_t d_ou
     Plan fp;  // the forward of the same weight format (a backward plan reports the forward's tail)
     make_plan(op & ~1, M, d_in, d_out, r, PLAN_SMS, &fp);
     plan->fwd_tail = !fp.fwd_tail ? 2 : fp.fwd_ksplit ? 3 : 1;
-    plan->dx_overlap = bwd ? (overlap ? 1 : 2) : 0;
+    plan->dx_overlap = bwd ? (pl.dx_ksplit ? 3 : overlap ? 1 : 2) : 0;
     const bool sk_bwd = bwd && !pl.side_bwd;
     plan->splitk[0] = pl.side ? 0 : pl.s_xa.splits;
     plan->splitk[1] = sk_bwd ? pl.s_g.splits : 0;

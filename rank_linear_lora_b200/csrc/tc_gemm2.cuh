@@ -203,18 +203,18 @@ __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, in
     w.piece = 0;
     w.nsplit = 1;
     if (p.tail_ksplit) {
-        // Last-wave tile tt cut along K: its first half is the FIRST item of cluster 2tt (so
-        // the hand-over of its fp32 partial overlaps that cluster's later tiles), its second
-        // half (the rank-r tail with it) the LAST item of cluster 2tt + 1, which adds the
-        // partial.  Both clusters then run W + 1/2 tiles.
+        // Last-wave tile tt cut along K into two halves, the FIRST items of clusters 2tt and
+        // 2tt + 1: the first half hands its fp32 partial over, the second (with the rank-r
+        // tail) adds it; both hand-overs overlap the clusters' later tiles, and every
+        // cluster ends after its whole tiles (W + 1/2 tiles on clusters 0 .. 2R-1).
         const int tt = cluster >> 1;
-        const bool in_tail = tt < p.tail_tiles;
-        const int kb_all = p.kb0 + p.kb1, kb_mid = kb_all / 2;
-        if (in_tail && (cluster & 1) == 0) {
+        if (tt < p.tail_tiles) {
             if (i == 0) {
+                const int kb_all = p.kb0 + p.kb1, kb_mid = kb_all / 2;
                 raster(p, p.dp_tiles + tt, w.m, w.n);
-                w.kb_hi = kb_mid;
-                w.piece = 1;
+                w.kb_lo = (cluster & 1) ? kb_mid : 0;
+                w.kb_hi = (cluster & 1) ? kb_all : kb_mid;
+                w.piece = 1 + (cluster & 1);
                 w.job = tt;
                 w.col0 = w.n * PAIR_BN;
                 return true;
@@ -225,14 +225,6 @@ __device__ __forceinline__ bool get_pair_item(const GemmArgs &p, int cluster, in
             const int t = cluster + i * n_clusters;
             if (t >= p.dp_tiles) return false;
             raster(p, t, w.m, w.n);
-            w.col0 = w.n * PAIR_BN;
-            return true;
-        }
-        if (in_tail && (cluster & 1) == 1 && i == p.dp_waves) {
-            raster(p, p.dp_tiles + tt, w.m, w.n);
-            w.kb_lo = kb_mid;
-            w.piece = 2;
-            w.job = tt;
             w.col0 = w.n * PAIR_BN;
             return true;
         }
@@ -283,7 +275,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
     // dequant groups run ahead of the MMA by different amounts, so a parity wait on the
     // stage's empty barrier could match a later phase than the one meant.
     uint32_t *bfree = tmem_slot + 5;
-    uint64_t *ks_bar = reinterpret_cast<uint64_t *>(tmem_slot + 6);  // K-split tail: the partial landed
+    volatile int *ks_ok = reinterpret_cast<volatile int *>(tmem_slot + 6);  // K-split tail: the partial is there
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -309,7 +301,6 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
             mbar_init(smem_u32(&tempty_bar[b]), 8);
         }
         mbar_init(smem_u32(drain_bar), 1);
-        mbar_init(smem_u32(ks_bar), 1);
         if (DQ) {
             for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * DQ_GROUP_WARPS);
             for (int q = 0; q < DQ_WARPS * DQ_QDEPTH; ++q) mbar_init(smem_u32(&qfull_bar[q]), 1);
@@ -712,15 +703,14 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
             if (!epi_ok[it & 1]) break;
             tc_fence_after();
             if (!DQ && w.piece > 0) {
-                // Last-wave tile cut along K.  The first half (piece 1, its cluster's first item)
-                // hands this CTA's 128 rows of its fp32 accumulator to the workspace straight from
-                // registers while the cluster's next tiles run, then raises its flag; the second
-                // half (piece 2, another cluster's last item) copies them into its idle pipeline
-                // buffers (one bulk copy), adds them to its own accumulator and stores the tile.
-                // Hand-over layout, 128 KB per CTA: float4 [chunk (4)][16-byte column group (16)]
-                // [row (128)], so a warp's accesses are 512 contiguous bytes.
+                // Last-wave tile cut along K (both halves are their clusters' first items; the
+                // MMAs of the next tile run in the other TMEM accumulator meanwhile).  The first
+                // half (piece 1) hands this CTA's 128 rows of its fp32 accumulator to the
+                // workspace from registers and raises its flag; the second (piece 2) reads them,
+                // adds them to its own accumulator and stores the tile.  Hand-over layout,
+                // 128 KB per CTA: float4 [chunk (4)][16-byte column group (16)][row (128)], so a
+                // warp's accesses are 512 contiguous bytes.
                 constexpr uint32_t KS_BYTES = 4 * 16 * 128 * 16;
-                static_assert(DQ || STAGES * Cfg::STAGE_BYTES >= KS_BYTES, "the hand-over fits the pipeline buffers");
                 const int slot = w.job * 2 + static_cast<int>(rank);
                 float4 *part = reinterpret_cast<float4 *>(p.ks_part) + static_cast<size_t>(slot) * (KS_BYTES / 16);
                 const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
@@ -751,30 +741,24 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     if (trace && epi_tid == 0 && it < 8) trace[TR_TILE_DONE0 + it] = globaltimer_ns();
                     continue;
                 }
-                // piece 2: the partial (published long before; the wait is bounded), copied in.
-                // (The result goes to the other epi_ok slot: this one may still be read by a
-                // thread behind the barrier after the accumulator wait; the other was last
-                // read before it.)
+                // piece 2: the first half's partial, once its flag is up (both halves are their
+                // clusters' first items, so this wait overlaps this cluster's next tile; bounded).
+                // Its own flag slot: the epilogue's epi_ok slots are reused by the next items.
                 if (epi_tid == 0) {
-                    bool ok = wait_flag_bounded(p.ks_flag + slot, abort_flag, p.err, DERR_WAIT_PARTIAL);
-                    if (ok) {
-                        p.ks_flag[slot] = 0;  // zero again for the next call
-                        fence_proxy_async_global();
-                        mbar_arrive_expect_tx(smem_u32(ks_bar), KS_BYTES);
-                        bulk_load(smem_u32(smem), part, KS_BYTES, smem_u32(ks_bar));
-                        ok = wait_bounded(smem_u32(ks_bar), 0, abort_flag, p.err, DERR_WAIT_PARTIAL);
-                    }
-                    epi_ok[(it + 1) & 1] = ok ? 1 : 0;
+                    const bool ok = wait_flag_bounded(p.ks_flag + slot, abort_flag, p.err, DERR_WAIT_PARTIAL);
+                    if (ok) p.ks_flag[slot] = 0;  // zero again for the next call
+                    *ks_ok = ok ? 1 : 0;
                 }
                 named_bar_sync(1, 128);
-                if (!epi_ok[(it + 1) & 1]) break;
-                wait_bounded(smem_u32(ks_bar), 0, abort_flag, p.err, DERR_WAIT_PARTIAL);  // seen: returns at once
-                const float4 *recv = reinterpret_cast<const float4 *>(smem) + q * 32 + lane;
+                if (!*ks_ok) break;
                 uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
                 const int out_row = w.m * PAIR_BM + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
                     uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                    float4 o[16];
+#pragma unroll
+                    for (int g = 0; g < 16; ++g) o[g] = __ldcg(part + (ch * 16 + g) * 128 + q * 32 + lane);
                     uint32_t v0[32], v1[32];
                     tmem_ld_32x32b_x32(t_row + ch * 64, v0);
                     tmem_ld_32x32b_x32(t_row + ch * 64 + 32, v1);
@@ -787,12 +771,11 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     // own accumulator + the first half's (two terms: the order does not change the sum)
 #pragma unroll
                     for (int g = 0; g < 16; ++g) {
-                        const float4 o = recv[(ch * 16 + g) * 128];
                         uint32_t *dst = g < 8 ? &v0[4 * g] : &v1[4 * (g - 8)];
-                        dst[0] = __float_as_uint(__uint_as_float(dst[0]) + o.x);
-                        dst[1] = __float_as_uint(__uint_as_float(dst[1]) + o.y);
-                        dst[2] = __float_as_uint(__uint_as_float(dst[2]) + o.z);
-                        dst[3] = __float_as_uint(__uint_as_float(dst[3]) + o.w);
+                        dst[0] = __float_as_uint(__uint_as_float(dst[0]) + o[g].x);
+                        dst[1] = __float_as_uint(__uint_as_float(dst[1]) + o[g].y);
+                        dst[2] = __float_as_uint(__uint_as_float(dst[2]) + o[g].z);
+                        dst[3] = __float_as_uint(__uint_as_float(dst[3]) + o[g].w);
                     }
                     if (lane == 0) bulk_wait_group_read<1>();
                     __syncwarp();

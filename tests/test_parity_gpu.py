@@ -237,6 +237,31 @@ def test_forward_last_wave_cut_along_k(shape):
         L.lora_linear_set_plan(M, di, do, r, None)
 
 
+@pytest.mark.parametrize("shape", [(1280, 4096, 4096, 8), (1200, 4000, 2040, 24)], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_dx_last_wave_cut_along_k(shape):
+    """The backward with the dX GEMM's last wave cut along K (plan dx_overlap 3; dA and
+    dB after it): every output against the oracle, dX the same bit for bit twice."""
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("dxksplit", M, di, do, r, alpha=2.0 * r, seed=0xD5 + M + do)
+    inp = inputs.make_inputs(spec)
+    plan = L.lora_linear_get_plan(L.OP_BWD, M, di, do, r)
+    plan["dx_overlap"] = 3
+    try:
+        L.lora_linear_set_plan(M, di, do, r, plan)
+        assert L.lora_linear_get_plan(L.OP_BWD, M, di, do, r)["dx_overlap"] == 3
+        dl = DeviceLayer(inp)
+        dl.forward()
+        dl.backward()
+        dl.check()
+        dx1 = dl.dX.clone()
+        compare_all(dl.results(), oracle_ref(inp), spec.s)
+        dl.backward()
+        dl.check()
+        assert torch.equal(dx1.view(torch.int16), dl.dX.view(torch.int16)), "K-split dX not deterministic"
+    finally:
+        L.lora_linear_set_plan(M, di, do, r, None)
+
+
 @pytest.mark.parametrize("shape", [TAIL_WAVE[0], TAIL_WAVE[1], TAIL_WAVE[2]], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
 def test_single_sm_main_gemm(shape, monkeypatch):
     """The single-SM main-GEMM kernel (chosen when CTA pairs are unavailable) on the
