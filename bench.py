@@ -511,7 +511,9 @@ def main():
         if timing_hooks:
             L.lora_linear_timing_read()
             L.lora_linear_timing_enable(True)
-        torch.cuda._sleep(int(5e6 + 2e5 * n_steps))  # let the host enqueue every step ahead
+        # let the host enqueue every step ahead of the GPU (with the timing hooks an event
+        # pair per launch costs the host more than a step takes on the GPU)
+        torch.cuda._sleep(int(5e6 + (1.5e6 if timing_hooks else 2e5) * n_steps))
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         n0 = L.lora_linear_launch_count()

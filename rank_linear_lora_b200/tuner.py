@@ -37,7 +37,7 @@ def field_options(r: int) -> dict:
         "g_group": [a for a in range(1, 7) if a * r <= 64],
         "da_cluster": [1, 2, 4],
         "fwd_tail": [1, 2, 3],
-        "dx_overlap": [1, 2],
+        "dx_overlap": [1, 2, 3],
     }
     return opts
 
@@ -82,7 +82,7 @@ def coordinate_descent(start: dict, r: int, cost) -> tuple:
 
 def _op_pair(wf: str):
     return {"bf16": (L.OP_FWD, L.OP_BWD), "q4": (L.OP_FWD_Q4, L.OP_BWD_Q4),
-            "fp8": (L.OP_FWD_FP8, L.OP_BWD_FP8)}[wf]
+            "fp8": (L.OP_FWD_FP8, L.OP_BWD_FP8), "nf4": (L.OP_FWD_NF4, L.OP_BWD_NF4)}[wf]
 
 
 # Bytes of the per-call streamed inputs (x and dY) the timed calls rotate through: more
@@ -110,9 +110,12 @@ class _Layer:
         self.turn = 0
         self.x, self.dY = self.sets[0]
         self.A, self.B = bf(r, d_in, scale=d_in ** -0.5), bf(d_out, r, scale=0.02)
-        if wf == "q4":
+        if wf in ("q4", "nf4"):
             self.Wq = torch.randint(1, 16, (d_out, d_in // 2), generator=g, dtype=torch.uint8).to(device)
             self.Ws = bf(d_out, d_in // 64, scale=0.01).abs()
+            if wf == "nf4":
+                from .inputs import nf4_codebook
+                self.codebook = nf4_codebook()
         elif wf == "fp8":
             self.W8 = torch.randint(0, 0x7E, (d_out, d_in), generator=g, dtype=torch.uint8).to(device)
             self.W8s = bf(d_out, scale=1e-3).abs()
@@ -139,6 +142,11 @@ class _Layer:
             L.lora_linear_fwd_q4(self.x, self.Wq, self.Ws, self.A, self.B, self.h, self.xa, a, self.wsf)
             L.lora_linear_bwd_q4(self.dY, self.x, self.Wq, self.Ws, self.A, self.B, self.xa, self.dX, self.dA,
                                  self.dB, a, self.wsb)
+        elif self.wf == "nf4":
+            cb = self.codebook
+            L.lora_linear_fwd_nf4(self.x, self.Wq, self.Ws, cb, self.A, self.B, self.h, self.xa, a, self.wsf)
+            L.lora_linear_bwd_nf4(self.dY, self.x, self.Wq, self.Ws, cb, self.A, self.B, self.xa, self.dX, self.dA,
+                                  self.dB, a, self.wsb)
         elif self.wf == "fp8":
             L.lora_linear_fwd_fp8(self.x, self.W8, self.W8s, self.A, self.B, self.h, self.xa, a, self.wsf)
             L.lora_linear_bwd_fp8(self.dY, self.x, self.W8, self.W8s, self.A, self.B, self.xa, self.dX, self.dA,
@@ -194,6 +202,10 @@ def tune(M: int, d_in: int, d_out: int, r: int, wf: str = "bf16", alpha: float =
     if best_us is None or (t_default is not None and t_default <= best_us):
         best, best_us = start, t_default
     L.lora_linear_set_plan(M, d_in, d_out, r, best)
+    # what runs: a field value that does not apply to this shape (a K-split tail where the
+    # last wave is not cut, say) reads back as the library's fallback
+    effective = L.lora_linear_get_plan(bop, M, d_in, d_out, r)
+    best = {k: effective[k] for k in L.lora_plan_t.FIELDS}
     return {"plan": best, "us": best_us, "default_plan": default, "default_us": t_default,
             "tried": [{"plan": p, "us": c} for p, c in tried]}
 
