@@ -973,7 +973,14 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
             a.ks_flag = reinterpret_cast<int *>(c.ws + c.plan.ks_flag);
         }
         if (b_mn) {
-            if (!q4 && !tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
+            // bf16 weight: the 3D column-chunk map when N is a multiple of 64 (one copy per
+            // CTA and K block; two 2D copies cost ~7% of the dX GEMM at 4096 x 4096)
+            a.b3d = !q4 && N % 64 == 0 ? 1 : 0;
+            if (a.b3d) {
+                if (!lora_host::tmap_mn_chunks(&a.tmB0, o.B0, N, K0)) return LORA_ERR_CUDA;
+            } else if (!q4 && !tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) {
+                return LORA_ERR_CUDA;
+            }
             if (!tmap_bf16(&a.tmB1, o.B1, N, r, 64, 64)) return LORA_ERR_CUDA;
         } else {
             if (!q4 && !tmap_bf16(&a.tmB0, o.B0, K0, N, 64, CTA_BN)) return LORA_ERR_CUDA;

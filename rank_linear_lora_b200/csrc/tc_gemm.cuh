@@ -115,6 +115,9 @@ struct GemmArgs {
     int tail_ksplit;
     float *ks_part;          // [tail tile][CTA rank][chunk (4)][16-byte column group (16)][row (128)] float4
     int *ks_flag;            // [tail tile][CTA rank]
+    // CTA-pair GEMM, MN-major bf16 weight: 1 when tmB0 is the 3D column-chunk map, so a
+    // CTA's 128 weight columns of a K block come in one copy instead of two.
+    int b3d;
 };
 
 // Release / acquire of a global int at GPU scope (the K-split tail's hand-over).

@@ -376,9 +376,15 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     tma_load_2d_pair(a_dst, seg1 ? &p.tmA1 : &p.tmA0, fb_leader, k0, a_row);
                     if (!b_tma) {
                     } else if (B_MN) {
-                        const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
-                        for (int j = 0; j < bn_cta / 64; ++j)
-                            tma_load_2d_pair(b_dst + j * 64 * 128, tb, fb_leader, b_row + 64 * j, k0);
+                        // the weight's 128 columns in one 3D copy (two 64-column chunks), else
+                        // one 2D copy per 64-column chunk
+                        if (p.b3d && !seg1 && bn_cta == 128) {
+                            tma_load_3d_pair(b_dst, &p.tmB0, fb_leader, 0, k0, b_row / 64);
+                        } else {
+                            const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
+                            for (int j = 0; j < bn_cta / 64; ++j)
+                                tma_load_2d_pair(b_dst + j * 64 * 128, tb, fb_leader, b_row + 64 * j, k0);
+                        }
                     } else {
                         const CUtensorMap *tb = w.nsplit == 1 ? (seg1 ? &p.tmB1 : &p.tmB0)
                                                               : (seg1 ? &p.tmB1n : &p.tmB0n);

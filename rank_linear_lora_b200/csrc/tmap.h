@@ -1,5 +1,5 @@
-// tmap.h -- host helper shared by the library's translation units: 2D TMA tensor maps
-// of row-major tensors, through the driver's cuTensorMapEncodeTiled (looked up once via
+// tmap.h -- host helper shared by the library's translation units: TMA tensor maps of
+// row-major tensors (2D, and the 3D column-chunk view of an MN-major operand), through the driver's cuTensorMapEncodeTiled (looked up once via
 // the runtime's driver entry point, so the library needs no link to libcuda).
 #pragma once
 
@@ -40,6 +40,22 @@ inline bool tmap_2d(CUtensorMap *m, CUtensorMapDataType type, int esize, const v
     cuuint32_t estr[2] = {1, 1};
     return fn(m, type, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// MN-major bf16 operand [K rows][N cols] (N a multiple of 64) as the 3D tensor
+// {64 columns, K rows, N/64 column chunks}: one box {64, 64, 2} brings two 64-column chunks
+// of 64 K rows, chunk after chunk in shared memory (the layout of two 2D boxes {64, 64}),
+// in one copy instead of two.  False if the map cannot be made.
+inline bool tmap_mn_chunks(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn || cols % 64 != 0) return false;
+    cuuint64_t dims[3] = {64, rows, cols / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, 64, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace lora_host
