@@ -196,6 +196,38 @@ class ClockSampler:
                 "samples": len(self.samples)}
 
 
+def device_spans(step, st, max_ctas: int = 512) -> dict:
+    """{kernel kind: us from its first CTA's entry to its last CTA's exit} over one step
+    whose launches are kept apart (no programmatic overlap), from the library's per-CTA
+    device trace (a kind launched more than once in the step keeps its last launch)."""
+    import torch
+    from rank_linear_lora_b200 import lora_linear as L
+    kinds = L.KERNEL_KINDS
+    buf = torch.zeros(len(kinds) * max_ctas * L.TRACE_WORDS, dtype=torch.int64, device="cuda")
+    torch.cuda.synchronize()
+    # with the timing hooks on, the event between launches keeps each kernel from starting
+    # early beside its predecessor, so its CTAs do not enter before their work can begin
+    L.lora_linear_timing_read()
+    L.lora_linear_timing_enable(True)
+    L.lora_linear_trace_enable(buf)
+    try:
+        torch.cuda._sleep(int(2e6))  # the host enqueues the whole step ahead of the GPU
+        step(st)
+        torch.cuda.synchronize()
+    finally:
+        L.lora_linear_trace_enable(None)
+        L.lora_linear_timing_enable(False)
+        L.lora_linear_timing_read()
+    tr = buf.cpu().numpy().reshape(len(kinds), max_ctas, L.TRACE_WORDS)
+    entry, exit_ = L.TRACE_FIELDS.index("entry"), L.TRACE_FIELDS.index("exit")
+    out = {}
+    for i, k in enumerate(kinds):
+        rows = tr[i][tr[i][:, entry] > 0]
+        if len(rows):
+            out[k] = float(rows[:, exit_].max() - rows[:, entry].min()) / 1e3
+    return out
+
+
 def config_dict(spec, workload_name: str, world: int) -> dict:
     """The workload as both arms name it (identical keys and values)."""
     return {"workload": workload_name, "M": spec.M, "d_in": spec.d_in, "d_out": spec.d_out, "r": spec.r,
@@ -573,6 +605,12 @@ def main():
     step_roof = {"t_roof_us": t_roof * 1e6, "t_meas_us": ms_per_step * 1e3, "frac": t_roof / (ms_per_step * 1e-3),
                  "definition": f"max(FLOP / bf16 {peak_kind} peak, algorithmic bytes / HBM peak) over the measured step time"}
     kernels = {k: {"us_per_launch": (v[0] / v[1] * 1e3) if v[1] else None, "launches": v[1]} for k, v in rec.items()}
+    # Each kernel's own device span in one traced step (the library's per-CTA trace:
+    # globaltimer at the first CTA's entry and at the last CTA's exit).  The event pair of
+    # the timing pass also brackets the launch, which adds 6-8 us to every kernel here.
+    for k, span in device_spans(step, sets[0]).items():
+        if k in kernels:
+            kernels[k]["span_us"] = span
 
     # Forward and backward separately: events around each call over 50 steps (the event
     # between them breaks the programmatic-launch overlap of the two, so the parts sum to
