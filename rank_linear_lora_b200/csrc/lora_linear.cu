@@ -977,7 +977,9 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
             // CTA and K block; two 2D copies cost ~7% of the dX GEMM at 4096 x 4096)
             a.b3d = !q4 && N % 64 == 0 ? 1 : 0;
             if (a.b3d) {
+                // 3D map for whole tiles, 2D map for the 64-column halves of split tail tiles
                 if (!lora_host::tmap_mn_chunks(&a.tmB0, o.B0, N, K0)) return LORA_ERR_CUDA;
+                if (!tmap_bf16(&a.tmB0n, o.B0, N, K0, 64, 64)) return LORA_ERR_CUDA;
             } else if (!q4 && !tmap_bf16(&a.tmB0, o.B0, N, K0, 64, 64)) {
                 return LORA_ERR_CUDA;
             }

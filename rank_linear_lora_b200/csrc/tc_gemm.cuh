@@ -82,7 +82,7 @@ struct GemmArgs {
     CUtensorMap tmA0, tmB0;  // segment 0
     CUtensorMap tmA1, tmB1;  // segment 1 (rank-r tail), used when kb1 > 0
     CUtensorMap tmC;         // EPI_STORE output (bf16, box 64 x 32, 128B swizzle)
-    CUtensorMap tmB0n, tmB1n;  // K-major B with box rows BN / tail_split (narrow tail tiles)
+    CUtensorMap tmB0n, tmB1n;  // K-major B with box rows BN / tail_split (narrow tail tiles); see b3d
     CUtensorMap tmQ;           // 4-bit frozen weight: packed codes (uint8), no swizzle
     int m_tiles, n_tiles;
     int kb0, kb1;            // 64-wide K blocks per segment
@@ -116,7 +116,8 @@ struct GemmArgs {
     float *ks_part;          // [tail tile][CTA rank][chunk (4)][16-byte column group (16)][row (128)] float4
     int *ks_flag;            // [tail tile][CTA rank]
     // CTA-pair GEMM, MN-major bf16 weight: 1 when tmB0 is the 3D column-chunk map, so a
-    // CTA's 128 weight columns of a K block come in one copy instead of two.
+    // CTA's 128 weight columns of a K block come in one copy instead of two; tmB0n is
+    // then the weight's 2D map {64, 64}, for the 64-column halves of split tail tiles.
     int b3d;
 };
 

@@ -377,11 +377,12 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     if (!b_tma) {
                     } else if (B_MN) {
                         // the weight's 128 columns in one 3D copy (two 64-column chunks), else
-                        // one 2D copy per 64-column chunk
+                        // one 2D copy per 64-column chunk (with the 3D map in tmB0, the
+                        // weight's 2D map is tmB0n: a 2D copy must name a 2D map)
                         if (p.b3d && !seg1 && bn_cta == 128) {
                             tma_load_3d_pair(b_dst, &p.tmB0, fb_leader, 0, k0, b_row / 64);
                         } else {
-                            const CUtensorMap *tb = seg1 ? &p.tmB1 : &p.tmB0;
+                            const CUtensorMap *tb = seg1 ? &p.tmB1 : p.b3d ? &p.tmB0n : &p.tmB0;
                             for (int j = 0; j < bn_cta / 64; ++j)
                                 tma_load_2d_pair(b_dst + j * 64 * 128, tb, fb_leader, b_row + 64 * j, k0);
                         }

@@ -262,6 +262,30 @@ def test_dx_last_wave_cut_along_k(shape):
         L.lora_linear_set_plan(M, di, do, r, None)
 
 
+@pytest.mark.parametrize("shape", [(1280, 4096, 4096, 8), (1280, 4032, 2040, 16), (1200, 4000, 2040, 24)],
+                         ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_dx_last_wave_cut_along_n(shape):
+    """The backward with the dX GEMM's last wave cut along N (plan dx_overlap 2): its
+    tail tiles stage 64 weight columns per CTA by 2D copies while whole tiles take the
+    3D column-chunk copy (d_in a multiple of 64; the last shape only 2D copies).  Every
+    output against the oracle."""
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("dxnsplit", M, di, do, r, alpha=2.0 * r, seed=0xD6 + M + di)
+    inp = inputs.make_inputs(spec)
+    plan = L.lora_linear_get_plan(L.OP_BWD, M, di, do, r)
+    plan["dx_overlap"] = 2
+    try:
+        L.lora_linear_set_plan(M, di, do, r, plan)
+        assert L.lora_linear_get_plan(L.OP_BWD, M, di, do, r)["dx_overlap"] == 2
+        dl = DeviceLayer(inp)
+        dl.forward()
+        dl.backward()
+        dl.check()
+        compare_all(dl.results(), oracle_ref(inp), spec.s)
+    finally:
+        L.lora_linear_set_plan(M, di, do, r, None)
+
+
 @pytest.mark.parametrize("shape", [TAIL_WAVE[0], TAIL_WAVE[1], TAIL_WAVE[2]], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
 def test_single_sm_main_gemm(shape, monkeypatch):
     """The single-SM main-GEMM kernel (chosen when CTA pairs are unavailable) on the
