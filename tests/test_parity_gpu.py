@@ -297,9 +297,14 @@ def test_single_sm_main_gemm(shape, monkeypatch):
     compare_all(dl.results(), oracle_ref(inp), spec.s)
 
 
-def test_without_programmatic_launch(monkeypatch):
+@pytest.mark.parametrize("shape", [(520, 640, 768, 16), (1280, 4096, 4096, 8)], ids=lambda s: "M%d_in%d_out%d_r%d" % s)
+def test_without_programmatic_launch(shape, monkeypatch):
+    """Every launch without programmatic dependent launch.  The second shape has a
+    partial last wave: dA + dB then run after the dX GEMM, whose tail tiles are cut
+    along N (2D weight copies beside the 3D ones of whole tiles)."""
     monkeypatch.setenv("LORA_LINEAR_PDL", "0")
-    spec = inputs.LayerSpec("nopdl", 520, 640, 768, 16, alpha=32.0, seed=0x99)
+    M, di, do, r = shape
+    spec = inputs.LayerSpec("nopdl", M, di, do, r, alpha=2.0 * r, seed=0x99 + M)
     inp, dl = _run_full(spec)
     compare_all(dl.results(), oracle_ref(inp), spec.s)
 
