@@ -119,30 +119,37 @@ __device__ __forceinline__ uint4 q4_decode8(uint32_t word, uint64_t s7x2) {
 }
 
 // Eight E4M3 codes (two 32-bit words, element i in byte i) to eight bf16 values
-// e4m3(q) * scale: each code pair converts exactly to f16x2, each half widens exactly to
-// fp32, the fp32 product with the bf16 scale is exact (4 + 8 significant bits), and the
-// conversion to bf16x2 is the one rounding.
-__device__ __forceinline__ uint32_t fp8_pair(uint32_t two_codes, float sc) {
-    uint32_t out;
-    asm("{\n\t.reg .b16 c;\n\t.reg .b32 h;\n\t.reg .b16 hl, hh;\n\t.reg .f32 fl, fh;\n\t"
-        "cvt.u16.u32 c, %1;\n\t"
-        "cvt.rn.f16x2.e4m3x2 h, c;\n\t"
-        "mov.b32 {hl, hh}, h;\n\t"
-        "cvt.f32.f16 fl, hl;\n\t"
-        "cvt.f32.f16 fh, hh;\n\t"
-        "mul.rn.f32 fl, fl, %2;\n\t"
-        "mul.rn.f32 fh, fh, %2;\n\t"
-        "cvt.rn.bf16x2.f32 %0, fh, fl;\n\t}"
-        : "=r"(out)
-        : "r"(two_codes), "f"(sc));
-    return out;
+// e4m3(q) * scale, four codes at a time: each code pair converts exactly to f16x2, each
+// half widens exactly to fp32, the packed fp32 product with the bf16 scale is exact
+// (4 + 8 significant bits), and the conversion to bf16x2 is the one rounding (NaN codes
+// stay NaN).  `scx2` is the fp32 scale in both halves.
+__device__ __forceinline__ void fp8_quad(uint32_t w, uint64_t scx2, uint32_t &p01, uint32_t &p23) {
+    asm("{\n\t.reg .b16 c0, c1, a0, a1, a2, a3;\n\t.reg .b32 h0, h1;\n\t.reg .f32 f0, f1, f2, f3;\n\t"
+        ".reg .b64 v0, v1;\n\t"
+        "mov.b32 {c0, c1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h0, c0;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h1, c1;\n\t"
+        "mov.b32 {a0, a1}, h0;\n\t"
+        "mov.b32 {a2, a3}, h1;\n\t"
+        "cvt.f32.f16 f0, a0;\n\t"
+        "cvt.f32.f16 f1, a1;\n\t"
+        "cvt.f32.f16 f2, a2;\n\t"
+        "cvt.f32.f16 f3, a3;\n\t"
+        "mov.b64 v0, {f0, f1};\n\t"
+        "mov.b64 v1, {f2, f3};\n\t"
+        "mul.rn.f32x2 v0, v0, %3;\n\t"
+        "mul.rn.f32x2 v1, v1, %3;\n\t"
+        "mov.b64 {f0, f1}, v0;\n\t"
+        "mov.b64 {f2, f3}, v1;\n\t"
+        "cvt.rn.bf16x2.f32 %0, f1, f0;\n\t"
+        "cvt.rn.bf16x2.f32 %1, f3, f2;\n\t}"
+        : "=r"(p01), "=r"(p23)
+        : "r"(w), "l"(scx2));
 }
-__device__ __forceinline__ uint4 fp8_decode8(uint32_t w0, uint32_t w1, float sc) {
+__device__ __forceinline__ uint4 fp8_decode8(uint32_t w0, uint32_t w1, uint64_t scx2) {
     uint4 r;
-    r.x = fp8_pair(w0 & 0xFFFFu, sc);
-    r.y = fp8_pair(w0 >> 16, sc);
-    r.z = fp8_pair(w1 & 0xFFFFu, sc);
-    r.w = fp8_pair(w1 >> 16, sc);
+    fp8_quad(w0, scx2, r.x, r.y);
+    fp8_quad(w1, scx2, r.z, r.w);
     return r;
 }
 
@@ -627,12 +634,12 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
                 if constexpr (WF == WF_FP8) {
                     // 64 codes: 16-byte chunk c of the bf16 row holds codes 8c .. 8c+7
-                    const float sc_f = __uint_as_float(sc[i] << 16);
+                    const uint64_t scx2 = (static_cast<uint64_t>(sc[i] << 16) << 32) | (sc[i] << 16);
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const uint4 v = src[h];
-                        *reinterpret_cast<uint4 *>(row + (((2 * h) ^ (rn & 7)) * 16)) = fp8_decode8(v.x, v.y, sc_f);
-                        *reinterpret_cast<uint4 *>(row + (((2 * h + 1) ^ (rn & 7)) * 16)) = fp8_decode8(v.z, v.w, sc_f);
+                        *reinterpret_cast<uint4 *>(row + (((2 * h) ^ (rn & 7)) * 16)) = fp8_decode8(v.x, v.y, scx2);
+                        *reinterpret_cast<uint4 *>(row + (((2 * h + 1) ^ (rn & 7)) * 16)) = fp8_decode8(v.z, v.w, scx2);
                     }
                 } else if constexpr (WF == WF_CB) {
                     const CbTable tb = cb_table(p.cb, __uint_as_float(sc[i] << 16));
