@@ -193,7 +193,7 @@ cudaError_t launch_gemm(const GemmArgs &args, int grid, cudaStream_t st, DevInfo
 
 constexpr int PAIR_STAGES = 6;
 constexpr int PAIR_STAGES_Q4 = 5;
-constexpr int PAIR_STAGES_FP8 = 4;  // the FP8 code rings take twice the 4-bit ones' shared memory
+constexpr int PAIR_STAGES_FP8 = 5;  // with one run per thread, the FP8 code slots take what the 4-bit ones do
 
 template <int WF>
 constexpr int pair_stages() {
@@ -948,9 +948,9 @@ lora_status_t step_main(const Ctx &c, const MainOperands &o, int64_t M, int64_t 
             for (int i = 0; i < 16; ++i) a.cb[i] = o.codebook[i];
         a.scale_rows = static_cast<int>(o.q_rows);
         // codes [d_out][d_in / 2] (4-bit) or [d_out][d_in] (FP8) bytes; each dequant warp
-        // fetches DQ_QROWS rows x the bytes of 64 codes at a time
+        // fetches dq_qrows rows x the bytes of 64 codes at a time
         const int rb = dq_run_bytes(o.wf);
-        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols * rb / 64, o.q_rows, rb, DQ_QROWS)) return LORA_ERR_CUDA;
+        if (!tmap_u8(&a.tmQ, o.Wq, o.q_cols * rb / 64, o.q_rows, rb, dq_qrows(o.wf))) return LORA_ERR_CUDA;
         allow_tail_split = false;
     }
     if (pair_C > 0) {

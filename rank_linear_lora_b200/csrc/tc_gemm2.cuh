@@ -37,20 +37,23 @@ namespace lora {
 constexpr int PAIR_BM = 256;      // output rows per pair tile (128 per CTA)
 constexpr int PAIR_BN = 256;      // output columns per pair tile
 constexpr int CTA_BN = PAIR_BN / 2;  // B rows (N) staged per CTA
-constexpr int DQ_WARPS = 12;         // 4-bit weight: dequant warps per CTA (3 idle warps besides)
-constexpr int DQ_RUNS = 2;           // 32-byte runs of codes (64 elements each) per thread per K block
-constexpr int DQ_GROUP_WARPS = 4 / DQ_RUNS;               // warps decoding one 128-run B tile
-constexpr int DQ_GROUPS = DQ_WARPS / DQ_GROUP_WARPS;       // groups that take K blocks in turn
+constexpr int DQ_WARPS = 12;         // coded weight: dequant warps per CTA (3 idle warps besides)
 constexpr int DQ_QDEPTH = 1;         // packed-code slots per dequant warp (own K blocks in flight)
-constexpr int DQ_QROWS = 32 * DQ_RUNS;                     // runs fetched per warp and K block
 
 // Frozen-weight formats of the pair GEMM: bf16, the linear 4-bit code, FP8 E4M3, and a
 // 4-bit code decoded through a 16-value codebook (e.g. NF4).
 enum WeightFmt { WF_BF16 = 0, WF_Q4 = 1, WF_FP8 = 2, WF_CB = 3 };
 // Bytes of codes per run of 64 weights: two 4-bit codes per byte, or one E4M3 code per byte.
 __host__ __device__ constexpr int dq_run_bytes(int wf) { return wf == WF_FP8 ? 64 : 32; }
-// One packed-code slot of a dequant warp: DQ_QROWS runs.
-__host__ __device__ constexpr int dq_qslot(int wf) { return DQ_QROWS * dq_run_bytes(wf); }
+// Runs of 64 codes a thread decodes per K block: two for the 4-bit codes (the per-block
+// fixed cost, the codebook table included, paid once per two runs); one for FP8, whose
+// halved code slots leave room for a fifth pipeline stage.
+__host__ __device__ constexpr int dq_runs(int wf) { return wf == WF_FP8 ? 1 : 2; }
+__host__ __device__ constexpr int dq_group_warps(int wf) { return 4 / dq_runs(wf); }  // warps per 128-run B tile
+__host__ __device__ constexpr int dq_groups(int wf) { return DQ_WARPS / dq_group_warps(wf); }  // take K blocks in turn
+__host__ __device__ constexpr int dq_qrows(int wf) { return 32 * dq_runs(wf); }  // runs fetched per warp and K block
+// One packed-code slot of a dequant warp: dq_qrows runs.
+__host__ __device__ constexpr int dq_qslot(int wf) { return dq_qrows(wf) * dq_run_bytes(wf); }
 
 // A warp's scheduler (SM sub-partition) is its id mod 4.  The single-thread MMA issuer
 // (warp 1) must issue each tcgen05.mma as soon as the tensor core takes the previous one
@@ -77,7 +80,8 @@ struct PairCfg {
     static constexpr int B_BYTES = CTA_BN * BK * 2;   // 16 KB: this CTA's 128 rows of B
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int Q_BYTES = DQ ? DQ_WARPS * DQ_QDEPTH * dq_qslot(WF) : 0;  // per-warp packed-code rings
-    static constexpr int EPI_BYTES = 4 * 2 * 32 * 128;
+    static constexpr int EPI_BUFS = 2;  // output staging per epilogue warp: 32 rows x 64 columns, double-buffered
+    static constexpr int EPI_BYTES = 4 * EPI_BUFS * 32 * 128;
     static constexpr int TMEM_COLS = 2 * PAIR_BN;     // two 256-column accumulators
     static constexpr int BAR_BYTES = DQ ? 1024 : 512;
     static constexpr int THREADS = DQ ? NUM_THREADS + 32 * dq_warp_span(DQ_WARPS) : NUM_THREADS;  // + dequant warps
@@ -309,7 +313,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
         }
         mbar_init(smem_u32(drain_bar), 1);
         if (DQ) {
-            for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * DQ_GROUP_WARPS);
+            for (int s = 0; s < STAGES; ++s) mbar_init(smem_u32(&bready_bar[s]), 2 * dq_group_warps(WF));
             for (int q = 0; q < DQ_WARPS * DQ_QDEPTH; ++q) mbar_init(smem_u32(&qfull_bar[q]), 1);
         }
         *abort_flag = 0;
@@ -530,6 +534,8 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
         // per-block cost outside the decode (waits, scale fetch, addressing, the
         // cluster-scope release) is paid once per DQ_RUNS runs, and one block takes a
         // group microseconds end to end, so DQ_GROUPS blocks are in flight at once.
+        constexpr int DQ_RUNS = dq_runs(WF), DQ_GROUP_WARPS = dq_group_warps(WF), DQ_GROUPS = dq_groups(WF),
+                      DQ_QROWS = dq_qrows(WF);
         static_assert(DQ_RUNS == 1 || DQ_RUNS == 2, "a warp's runs stay inside one 64-run chunk");
         const int dw = dq_index(warp);                       // dequant warp 0 .. DQ_WARPS-1
         const int grp = dw / DQ_GROUP_WARPS, wg = dw % DQ_GROUP_WARPS;
@@ -765,11 +771,11 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                 }
                 named_bar_sync(1, 128);
                 if (!*ks_ok) break;
-                uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
+                uint8_t *stage_base = sEpi + (q * Cfg::EPI_BUFS) * (32 * 128);
                 const int out_row = w.m * PAIR_BM + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
                 for (int ch = 0; ch < 4; ++ch) {
-                    uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                    uint8_t *sbuf = stage_base + (ch % Cfg::EPI_BUFS) * (32 * 128);
                     float4 o[16];
 #pragma unroll
                     for (int g = 0; g < 16; ++g) o[g] = __ldcg(part + (ch * 16 + g) * 128 + q * 32 + lane);
@@ -791,7 +797,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                         dst[2] = __float_as_uint(__uint_as_float(dst[2]) + o[g].z);
                         dst[3] = __float_as_uint(__uint_as_float(dst[3]) + o[g].w);
                     }
-                    if (lane == 0) bulk_wait_group_read<1>();
+                    if (lane == 0) bulk_wait_group_read<Cfg::EPI_BUFS - 1>();
                     __syncwarp();
                     stage_row64(sbuf, lane, v0, v1);
                     fence_proxy_async_smem();
@@ -806,15 +812,15 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
             }
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                                    static_cast<uint32_t>(buf * PAIR_BN);
-            uint8_t *stage_base = sEpi + (q * 2) * (32 * 128);
+            uint8_t *stage_base = sEpi + (q * Cfg::EPI_BUFS) * (32 * 128);
             const int nch = (PAIR_BN / 64) / w.nsplit;
             const int out_row = w.m * PAIR_BM + static_cast<int>(rank) * 128 + q * 32;
 #pragma unroll 1
             for (int ch = 0; ch < nch; ++ch) {
-                uint8_t *sbuf = stage_base + (ch & 1) * (32 * 128);
+                uint8_t *sbuf = stage_base + (ch % Cfg::EPI_BUFS) * (32 * 128);
                 if (DQ) {
                     // 32 columns at a time: the dequant warps leave fewer registers per thread
-                    if (lane == 0) bulk_wait_group_read<1>();
+                    if (lane == 0) bulk_wait_group_read<Cfg::EPI_BUFS - 1>();
                     __syncwarp();
 #pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
@@ -838,7 +844,7 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
                     }
-                    if (lane == 0) bulk_wait_group_read<1>();
+                    if (lane == 0) bulk_wait_group_read<Cfg::EPI_BUFS - 1>();
                     __syncwarp();
                     stage_row64(sbuf, lane, v0, v1);
                 }
