@@ -69,3 +69,35 @@ def test_gpus_2_spawns_two_ranks_and_prints_one_line():
     assert out["n_gpus"] == 2 and out["world_size"] == 2 and out["dry_run"] is True
     assert out["reduced_grads_match_whole_batch"] is True
     assert out["config"]["parallelism"] == "dp2"
+
+
+def test_traffic_figures_follow_the_kernel_sources(tmp_path, monkeypatch):
+    """A stored ncu traffic figure is reported only while the layer's kernel sources are
+    the ones it was measured on: a comment or blank-space edit keeps it, a code edit
+    voids it (the line then carries null)."""
+    import shutil
+    sys.path.insert(0, ROOT)
+    import bench
+    d = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    wl = next(iter(d["workloads"]))
+    csrc = tmp_path / "rank_linear_lora_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in bench.LAYER_SOURCES:
+        shutil.copy(os.path.join(ROOT, "rank_linear_lora_b200", "csrc", f), csrc / f)
+    (tmp_path / "profiles").mkdir()
+    d["kernel_source_hash"] = "0" * 16
+    json.dump(d, open(tmp_path / "profiles" / "traffic.json", "w"))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    assert len(h0) == 16 and int(h0, 16) >= 0
+    assert bench.stored_traffic("dx_main", wl) is None  # figure of other sources
+    d["kernel_source_hash"] = h0
+    json.dump(d, open(tmp_path / "profiles" / "traffic.json", "w"))
+    want = d["workloads"][wl]["kernels"]["dx_main"]["dram_bytes_per_launch"]
+    assert bench.stored_traffic("dx_main", wl) == want
+    ptx = csrc / "ptx.cuh"
+    text = ptx.read_text()
+    ptx.write_text("// an added comment\n\n" + text.replace("\n", "\n  ", 3))
+    assert bench.kernel_source_hash() == h0 and bench.stored_traffic("dx_main", wl) == want
+    ptx.write_text(text + "\nstatic int an_added_symbol;\n")
+    assert bench.kernel_source_hash() != h0 and bench.stored_traffic("dx_main", wl) is None
