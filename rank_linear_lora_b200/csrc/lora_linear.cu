@@ -88,12 +88,14 @@ bool tmap_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, u
                               CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// Row-major 2D uint8 tensor [rows][cols_bytes], box {box_bytes, box_rows}, no swizzle
-// (the packed 4-bit codes, read by threads rather than by the tensor cores).
+// Row-major 2D uint8 tensor [rows][cols_bytes], box {box_bytes, box_rows} of 32- or 64-byte
+// rows (the packed codes, read by threads rather than by the tensor cores), with the
+// swizzle of the row's width: it moves each row's 16-byte chunks so that the 32 lanes of
+// a warp, each reading one row, spread over all the shared-memory banks.
 bool tmap_u8(CUtensorMap *m, const void *base, uint64_t cols_bytes, uint64_t rows, uint32_t box_bytes,
              uint32_t box_rows) {
-    return lora_host::tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, cols_bytes, rows, box_bytes, box_rows,
-                              CU_TENSOR_MAP_SWIZZLE_NONE);
+    const CUtensorMapSwizzle swz = box_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    return lora_host::tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, cols_bytes, rows, box_bytes, box_rows, swz);
 }
 
 // ------------------------------------------------------------------ timing hooks

@@ -634,8 +634,12 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
             for (int i = 0; i < DQ_RUNS; ++i) {
                 const int run = r0 + lane + 32 * i;
                 const int rn = B_MN ? (run & 63) : run, jc = B_MN ? (run >> 6) : 0;
-                const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * QSLOT +
-                                                                   (lane + 32 * i) * dq_run_bytes(WF));
+                // the slot holds the runs in rows of RB bytes, swizzled by the TMA: chunk t
+                // of row lr sits at t ^ ((lr >> 1) & 3) (64-byte rows) or t ^ ((lr >> 2) & 1)
+                // (32-byte rows), the slot being 1024-byte-aligned
+                const int lr = lane + 32 * i;
+                const uint4 *src = reinterpret_cast<const uint4 *>(qring + slot * QSLOT + lr * dq_run_bytes(WF));
+                const int sw = dq_run_bytes(WF) == 64 ? ((lr >> 1) & 3) : ((lr >> 2) & 1);
                 uint8_t *row =
                     sB + stage * Cfg::B_BYTES + (B_MN ? jc * 64 * 128 : 0) + (rn >> 3) * 1024 + (rn & 7) * 128;
                 if constexpr (WF == WF_FP8) {
@@ -643,19 +647,19 @@ __global__ void __launch_bounds__(PairCfg<B_MN, WF, STAGES>::THREADS, 1)
                     const uint64_t scx2 = (static_cast<uint64_t>(sc[i] << 16) << 32) | (sc[i] << 16);
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        const uint4 v = src[h];
+                        const uint4 v = src[h ^ sw];
                         *reinterpret_cast<uint4 *>(row + (((2 * h) ^ (rn & 7)) * 16)) = fp8_decode8(v.x, v.y, scx2);
                         *reinterpret_cast<uint4 *>(row + (((2 * h + 1) ^ (rn & 7)) * 16)) = fp8_decode8(v.z, v.w, scx2);
                     }
                 } else if constexpr (WF == WF_CB) {
                     const CbTable tb = cb_table(p.cb, __uint_as_float(sc[i] << 16));
-                    const uint4 v0 = src[0], v1 = src[1];
+                    const uint4 v0 = src[sw], v1 = src[1 ^ sw];
                     const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
                     for (int c = 0; c < 8; ++c)
                         *reinterpret_cast<uint4 *>(row + ((c ^ (rn & 7)) * 16)) = cb_decode8(tb, wds[c]);
                 } else {
-                    const uint4 v0 = src[0], v1 = src[1];
+                    const uint4 v0 = src[sw], v1 = src[1 ^ sw];
                     const float s7 = __uint_as_float(sc[i] << 16) / 7.0f;
                     const uint64_t s7x2 = (static_cast<uint64_t>(__float_as_uint(s7)) << 32) | __float_as_uint(s7);
                     const uint32_t wds[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
